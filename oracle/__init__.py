@@ -1,0 +1,307 @@
+"""CPU oracle for the MoE routing-and-dispatch layer.
+
+TEST INFRASTRUCTURE ONLY. Only tests/, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import it. It
+imports nothing from the CUDA package and the CUDA package imports nothing
+from it; they share only the seeded input generators.
+
+The arithmetic lives in ``moe_oracle.c`` (plain C, double accumulation,
+single thread); this module marshals numpy arrays and composes the steps in
+the order of the pages' statement of the problem ("Expert choice routing",
+aicassindra.com, section "The math: a gating matrix and top-k over tokens"):
+scores -> top-k -> gather -> per-expert FFN -> gate scale -> scatter_add.
+
+Parity status: every function here is pinned by ``tests/test_oracle_*.py``
+against closed forms, brute force, library special cases or the pages'
+worked numbers, except the synthetic routing statistics (experts-per-token
+histogram shape, overflow rates, MaxVio trajectory), which the pages measure
+on trained models: those are reported, "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import numpy as np
+
+from .build import build as _build
+
+SOFTMAX, SIGMOID = 0, 1
+RELU, GELU, SWIGLU = 0, 1, 2
+W_RAW, W_NORMALIZED = 0, 1
+STORE_F32, STORE_BF16 = 0, 1
+
+_LIB = None
+
+_i32p = np.ctypeslib.ndpointer(dtype=np.int32, flags="C_CONTIGUOUS")
+_u8p = np.ctypeslib.ndpointer(dtype=np.uint8, flags="C_CONTIGUOUS")
+_f32p = np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS")
+_f64p = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
+
+
+def _opt(ptype):
+    """ndpointer that also accepts None (NULL)."""
+
+    class _Opt(ptype):
+        @classmethod
+        def from_param(cls, obj):
+            if obj is None:
+                return None
+            return ptype.from_param(obj)
+
+    return _Opt
+
+
+def lib() -> ctypes.CDLL:
+    global _LIB
+    if _LIB is None:
+        path = _build()
+        L = ctypes.CDLL(path)
+        c_int, c_float, c_double = ctypes.c_int, ctypes.c_float, ctypes.c_double
+        L.orc_round_bf16.argtypes = [c_double]
+        L.orc_round_bf16.restype = c_float
+        L.orc_round_bf16_n.argtypes = [ctypes.c_longlong, _f64p, _f32p]
+        L.orc_round_bf16_n.restype = None
+        L.orc_router.argtypes = [c_int, c_int, c_int, _f32p, _f32p, _opt(_f32p), c_int,
+                                 _f32p, _f32p, _f64p]
+        L.orc_select_ec.argtypes = [c_int, c_int, c_int, _f32p, _i32p, _f32p]
+        L.orc_select_tc.argtypes = [c_int, c_int, c_int, _f32p, _opt(_f32p), c_int, c_int,
+                                    c_int, c_int, _i32p, _f32p]
+        L.orc_capacity.argtypes = [c_int, c_int, c_int, _i32p, c_int, _u8p, _i32p, _i32p,
+                                   _i32p]
+        L.orc_expert_ffn.argtypes = [c_int, c_int, c_int, c_int, c_int, _f32p, _f32p,
+                                     _opt(_f32p), _f32p, _f32p]
+        L.orc_combine.argtypes = [c_int, c_int, c_int, _i32p, _f32p, _f32p, c_int, _f32p]
+        L.orc_aux.argtypes = [c_int, c_int, c_int, _i32p, _f32p, _f64p, c_double, c_double,
+                              ctypes.POINTER(c_double), ctypes.POINTER(c_double),
+                              ctypes.POINTER(c_double)]
+        L.orc_bias_update.argtypes = [c_int, c_int, c_int, _i32p, c_float, _f32p]
+        L.orc_ec_histogram.argtypes = [c_int, c_int, c_int, _i32p, _i32p]
+        for name in ("orc_router", "orc_select_ec", "orc_select_tc", "orc_capacity",
+                     "orc_expert_ffn", "orc_combine", "orc_aux", "orc_bias_update",
+                     "orc_ec_histogram"):
+            getattr(L, name).restype = None
+        _LIB = L
+    return _LIB
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _i32(a):
+    return np.ascontiguousarray(a, dtype=np.int32)
+
+
+# --------------------------------------------------------------------------
+# single steps
+# --------------------------------------------------------------------------
+
+def round_bf16(a) -> np.ndarray:
+    """Round each value to the nearest bf16 (ties to even); float32 result."""
+    flat = np.ascontiguousarray(np.asarray(a, dtype=np.float64).ravel())
+    out = np.empty(flat.shape, np.float32)
+    lib().orc_round_bf16_n(flat.size, flat, out)
+    return out.reshape(np.shape(a))
+
+
+def router(X, Wg, logit_bias=None, score=SOFTMAX):
+    """logits = X.W_g (+ logit bias), S = softmax/sigmoid(logits), lse per row."""
+    X = _f32(X)
+    Wg = _f32(Wg)
+    n, d = X.shape
+    d2, E = Wg.shape
+    assert d == d2
+    logits = np.empty((n, E), np.float32)
+    S = np.empty((n, E), np.float32)
+    lse = np.empty((n,), np.float64)
+    lib().orc_router(n, d, E, X, Wg, None if logit_bias is None else _f32(logit_bias),
+                     score, logits, S, lse)
+    return logits, S, lse
+
+
+def ec_quota(n: int, E: int, c: float) -> int:
+    """Expert-choice tokens per expert, k = n c / E ("Token choice vs expert
+    choice routing in MoE", section "Who picks whom"); floor when inexact."""
+    return int(math.floor(n * c / E + 1e-9))
+
+
+def capacity_of(n: int, E: int, cf: float) -> int:
+    """Per-expert buffer = tokens per batch / experts x capacity factor
+    ("MoE routing strategies explained", section "2. Top-1 switch routing
+    with a capacity factor"); floor when inexact."""
+    return int(math.floor(n / E * cf + 1e-9))
+
+
+def select_ec(S, k: int):
+    S = _f32(S)
+    n, E = S.shape
+    assert 1 <= k <= n
+    I = np.empty((E, k), np.int32)
+    G = np.empty((E, k), np.float32)
+    lib().orc_select_ec(n, E, k, S, I, G)
+    return I, G
+
+
+def select_tc(S, K: int, sel_bias=None, n_groups: int = 1, topk_groups: int = 1,
+              group_topn: int = 1, weights: int = W_RAW):
+    S = _f32(S)
+    n, E = S.shape
+    if n_groups > 1:
+        assert E % n_groups == 0 and 1 <= topk_groups <= n_groups
+        assert 1 <= group_topn <= E // n_groups <= 1024
+        assert K <= topk_groups * (E // n_groups)
+    assert 1 <= K <= E
+    idx = np.empty((n, K), np.int32)
+    w = np.empty((n, K), np.float32)
+    lib().orc_select_tc(n, E, K, S, None if sel_bias is None else _f32(sel_bias),
+                        n_groups, topk_groups, group_topn, weights, idx, w)
+    return idx, w
+
+
+def apply_capacity(idx, E: int, cap: int):
+    """Returns drop [n,K] u8, load [E], kept [E], pos [n,K] (-1 when dropped)."""
+    idx = _i32(idx)
+    n, K = idx.shape
+    drop = np.empty((n, K), np.uint8)
+    load = np.empty((E,), np.int32)
+    kept = np.empty((E,), np.int32)
+    pos = np.empty((n, K), np.int32)
+    lib().orc_capacity(n, E, K, idx, int(cap), drop, load, kept, pos)
+    return drop, load, kept, pos
+
+
+def expert_ffn(X, W1, W3, W2, act: int, store: int):
+    X = _f32(X)
+    m, d = X.shape
+    h = W1.shape[0]
+    Y = np.empty((m, d), np.float32)
+    if m:
+        lib().orc_expert_ffn(m, d, h, act, store, X, _f32(W1),
+                             None if W3 is None else _f32(W3), _f32(W2), Y)
+    return Y
+
+
+def combine(n: int, pair_token, pair_gate, Y, store: int):
+    Y = _f32(Y)
+    P = len(pair_token)
+    d = Y.shape[1]
+    out = np.empty((n, d), np.float32)
+    lib().orc_combine(n, d, P, _i32(pair_token), _f32(pair_gate), Y, store, out)
+    return out
+
+
+def aux(load, S, lse, K: int, lb_coef: float = 0.01, z_coef: float = 0.001):
+    S = _f32(S)
+    n, E = S.shape
+    lb, z, mv = ctypes.c_double(), ctypes.c_double(), ctypes.c_double()
+    lib().orc_aux(n, E, K, _i32(load), S, np.ascontiguousarray(lse, np.float64),
+                  lb_coef, z_coef, ctypes.byref(lb), ctypes.byref(z), ctypes.byref(mv))
+    return lb.value, z.value, mv.value
+
+
+def bias_update(load, n: int, K: int, rate: float, bias):
+    b = np.array(bias, dtype=np.float32, copy=True)
+    lib().orc_bias_update(n, len(b), K, _i32(load), rate, b)
+    return b
+
+
+def ec_histogram(I, n: int):
+    I = _i32(I)
+    E, k = I.shape
+    hist = np.empty((E + 1,), np.int32)
+    lib().orc_ec_histogram(n, E, k, I, hist)
+    return hist
+
+
+# --------------------------------------------------------------------------
+# the whole layer
+# --------------------------------------------------------------------------
+
+def route(spec: dict, S, lse=None, sel_bias=None):
+    """Selection + capacity + aux from a score matrix, per ``spec``:
+
+    mode 'ec' | 'tc'; k (EC tokens per expert) or K (TC experts per token);
+    capacity (-1 dropless); n_groups/topk_groups/group_topn; weights.
+    Returns a dict of the routing tensors."""
+    S = _f32(S)
+    n, E = S.shape
+    r = {"S": S}
+    if spec["mode"] == "ec":
+        I, G = select_ec(S, spec["k"])
+        r.update(I=I, G=G, hist=ec_histogram(I, n),
+                 load=np.full((E,), spec["k"], np.int32))
+        r["kept"] = r["load"].copy()
+    else:
+        K = spec["K"]
+        idx, w = select_tc(S, K, sel_bias, spec.get("n_groups", 1), spec.get("topk_groups", 1),
+                           spec.get("group_topn", 1), spec.get("weights", W_RAW))
+        drop, load, kept, pos = apply_capacity(idx, E, spec.get("capacity", -1))
+        r.update(idx=idx, w=w, drop=drop, load=load, kept=kept, pos=pos)
+        if lse is not None:
+            r["lb"], r["z"], r["maxvio"] = aux(load, S, lse, K, spec.get("lb_coef", 0.01),
+                                               spec.get("z_coef", 0.001))
+    return r
+
+
+def token_pairs(spec: dict, routing: dict, n: int, tokens=None):
+    """The (token, expert, gate) pairs whose FFN output reaches `tokens`
+    (all tokens when None), ordered by token then expert."""
+    want = None if tokens is None else set(int(t) for t in tokens)
+    pairs = []
+    if spec["mode"] == "ec":
+        I, G = routing["I"], routing["G"]
+        E, k = I.shape
+        for e in range(E):
+            for j in range(k):
+                t = int(I[e, j])
+                if want is None or t in want:
+                    pairs.append((t, e, float(G[e, j])))
+    else:
+        idx, w, drop = routing["idx"], routing["w"], routing["drop"]
+        nK = idx.shape[1]
+        rows = range(n) if want is None else sorted(want)
+        for t in rows:
+            for j in range(nK):
+                if not drop[t, j]:
+                    pairs.append((t, int(idx[t, j]), float(w[t, j])))
+    pairs.sort(key=lambda p: (p[0], p[1]))
+    return pairs
+
+
+def layer_forward(spec: dict, X, routing: dict, expert_weights, shared_weights=None,
+                  tokens=None):
+    """out rows for `tokens` (all when None) of the MoE layer given a routing.
+
+    expert_weights(e) -> (W1 [h,d], W3 [h,d] or None, W2 [d,h]) as float32;
+    shared_weights(s) -> same for always-on shared expert s (weight 1,
+    "MoE routing strategies explained", section "3. Shared plus routed
+    experts"). The residual is not added: the layer returns scatter_add only.
+    """
+    X = _f32(X)
+    n, d = X.shape
+    store, act = spec["store"], spec["act"]
+    pairs = token_pairs(spec, routing, n, tokens)
+    rows = list(range(n)) if tokens is None else [int(t) for t in tokens]
+    pos_of = {t: i for i, t in enumerate(rows)}
+    Ys, ptok, pgate = [], [], []
+    by_e = {}
+    for t, e, g in pairs:
+        by_e.setdefault(e, []).append((t, g))
+    for e in sorted(by_e):
+        W1, W3, W2 = expert_weights(e)
+        ts = [t for t, _ in by_e[e]]
+        Y = expert_ffn(X[ts], W1, W3, W2, act, store)
+        Ys.append(Y)
+        ptok += [pos_of[t] for t in ts]
+        pgate += [g for _, g in by_e[e]]
+    for s in range(spec.get("n_shared", 0)):
+        W1, W3, W2 = shared_weights(s)
+        Ys.append(expert_ffn(X[rows], W1, W3, W2, act, store))
+        ptok += list(range(len(rows)))
+        pgate += [1.0] * len(rows)
+    Yall = np.concatenate(Ys, 0) if Ys else np.zeros((0, d), np.float32)
+    order = np.argsort(np.asarray(ptok, np.int64), kind="stable")
+    return combine(len(rows), np.asarray(ptok, np.int32)[order],
+                   np.asarray(pgate, np.float32)[order], Yall[order], store)
