@@ -1,0 +1,505 @@
+// C-ABI entry points of libmoe: host-side validation, derived sizes,
+// workspace layout and the launch sequence of each call. Nothing here
+// allocates, frees or synchronises (except moe_read_error).
+#include <math.h>
+#include <string.h>
+
+#include "device_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+static bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+moe_status derive(const moe_config* c, Derived* d) {
+  if (!c || !d) return MOE_ERR_INVALID_ARG;
+  if (c->n < 1 || c->d < 1 || c->h < 1 || c->E < 1) return MOE_ERR_INVALID_ARG;
+  if (c->E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+  if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (c->mode != MOE_EXPERT_CHOICE && c->mode != MOE_TOKEN_CHOICE) return MOE_ERR_INVALID_ARG;
+  if (c->score != MOE_SCORE_SOFTMAX && c->score != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (c->act != MOE_ACT_RELU && c->act != MOE_ACT_GELU && c->act != MOE_ACT_SWIGLU)
+    return MOE_ERR_INVALID_ARG;
+  if (c->weights != MOE_W_RAW && c->weights != MOE_W_NORMALIZED) return MOE_ERR_INVALID_ARG;
+  if (c->n_shared < 0 || c->n_shared > MOE_MAX_SHARED) return MOE_ERR_INVALID_ARG;
+  if (c->dtype == MOE_BF16) {
+    if (c->d % 64 || c->h % 64) return MOE_ERR_UNSUPPORTED;
+    if (c->n_shared > 0 && c->n < 128) return MOE_ERR_UNSUPPORTED;
+  } else {
+    if (c->d % 8 || c->h % 8) return MOE_ERR_UNSUPPORTED;
+  }
+  const int E = c->E, n = c->n;
+  d->n_pad = (int)round_up(n, kRowAlign);
+  if (c->mode == MOE_EXPERT_CHOICE) {
+    int k = c->k;
+    if (k == 0) {
+      if (!(c->capacity_factor > 0.0f)) return MOE_ERR_INVALID_ARG;
+      k = (int)floor((double)n * (double)c->capacity_factor / (double)E + 1e-9);
+    }
+    if (k < 1 || k > n) return MOE_ERR_INVALID_ARG;
+    if (n > MOE_EC_MAX_TOKENS) return MOE_ERR_UNSUPPORTED;
+    d->k = k;
+    d->cap = k;
+    d->slots = E;
+    d->kpad = (int)round_up(k, kRowAlign);
+    d->rows_routed = (long long)E * d->kpad;
+  } else {
+    const int K = c->k;
+    if (K < 1 || K > E || K > MOE_MAX_TOPK) return MOE_ERR_INVALID_ARG;
+    int cap;
+    if (c->capacity < 0) {
+      cap = -1;
+    } else if (c->capacity == 0) {
+      if (!(c->capacity_factor > 0.0f)) return MOE_ERR_INVALID_ARG;
+      cap = (int)floor((double)n / (double)E * (double)c->capacity_factor + 1e-9);
+      if (cap < 1) return MOE_ERR_INVALID_ARG;
+    } else {
+      cap = c->capacity;
+    }
+    if (c->n_groups > 1) {
+      const int G = c->n_groups;
+      if (E % G) return MOE_ERR_INVALID_ARG;
+      const int gs = E / G;
+      const int et = router_tile_et(E);
+      const int V = et >= 32 ? et / 32 : 1;
+      if (gs % V || !is_pow2(gs / V) || gs / V > 32) return MOE_ERR_UNSUPPORTED;
+      if (c->topk_groups < 1 || c->topk_groups > G) return MOE_ERR_INVALID_ARG;
+      if (c->group_topn < 1 || c->group_topn > gs) return MOE_ERR_INVALID_ARG;
+      if (K > c->topk_groups * gs) return MOE_ERR_INVALID_ARG;
+    }
+    d->k = K;
+    d->cap = cap;
+    d->slots = K;
+    d->kpad = 0;
+    long long a = (long long)n * K;
+    long long bound = round_up(a + (long long)E * (kRowAlign - 1), kRowAlign);
+    bound = bound / kRowAlign * kRowAlign;
+    if (cap >= 0) {
+      long long capb = (long long)E * round_up(cap, kRowAlign);
+      if (capb < bound) bound = capb;
+    }
+    // floor to a multiple of 128 of (a + 127 E) is also a valid bound
+    long long fl = (a + (long long)E * (kRowAlign - 1)) / kRowAlign * kRowAlign;
+    if (fl < bound) bound = fl;
+    if (bound < kRowAlign) bound = kRowAlign;
+    d->rows_routed = bound;
+  }
+  d->shared_base = d->rows_routed;
+  d->rows = d->rows_routed + (long long)c->n_shared * d->n_pad;
+  if (d->rows > (1LL << 30)) return MOE_ERR_UNSUPPORTED;
+  d->router_blocks = ceil_div(n, 32);  // covers every router tile height (>= 32 rows)
+  d->tok_blocks = ceil_div(n, kTokBlock);
+  return MOE_OK;
+}
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+WsLayout ws_layout(const moe_config* c, const Derived& d) {
+  WsLayout w{};
+  size_t off = 0;
+  w.err = off;
+  off += MOE_WS_ERROR_BYTES;
+  w.colsum = off;
+  off = align_up(off + (size_t)d.router_blocks * c->E * 4, 256);
+  w.lse2 = off;
+  off = align_up(off + (size_t)d.router_blocks * 8, 256);
+  w.blk_hist = off;
+  off = align_up(off + (size_t)d.tok_blocks * c->E * 4, 256);
+  w.blk_base = off;
+  off = align_up(off + (size_t)d.tok_blocks * c->E * 4, 256);
+  w.ec_row = off;
+  if (c->mode == MOE_EXPERT_CHOICE) off = align_up(off + (size_t)c->n * c->E * 4, 256);
+  w.ec_gate = off;
+  if (c->mode == MOE_EXPERT_CHOICE) off = align_up(off + (size_t)c->n * c->E * 4, 256);
+  w.route_end = align_up(off, 1024);
+  const size_t elt = c->dtype == MOE_BF16 ? 2 : 4;
+  off = w.route_end;
+  w.xperm = off;
+  off = align_up(off + (size_t)d.rows * c->d * elt, 1024);
+  w.hbuf = off;
+  off = align_up(off + (size_t)d.rows * c->h * elt, 1024);
+  w.yperm = off;
+  off = align_up(off + (size_t)d.rows * c->d * elt, 1024);
+  w.layer_end = off;
+  return w;
+}
+
+static moe_status check_route_out(const moe_config* c, const moe_route_out* o) {
+  if (!o) return MOE_ERR_INVALID_ARG;
+  if (!o->idx || !o->gate || !o->load || !o->counts || !o->offsets || !o->row_token ||
+      !o->tok_row || !o->tok_gate || !o->scores || !o->aux)
+    return MOE_ERR_INVALID_ARG;
+  if (c->mode == MOE_TOKEN_CHOICE && !o->drop) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+static moe_status check_ws(void* ws, size_t have, size_t need) {
+  if (!ws) return MOE_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) & 255) return MOE_ERR_WORKSPACE;
+  if (have < need) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+template <typename T>
+static T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+#define MOE_CU(x)                          \
+  do {                                     \
+    if ((x) != cudaSuccess) return MOE_ERR_CUDA; \
+  } while (0)
+
+// selection bookkeeping after the scores (and, for TC, idx/gate) exist
+static moe_status finish_route(const moe_config* c, const Derived& dv, const WsLayout& w,
+                               moe_route_out* o, void* ws, const float* S, int colsum_blocks,
+                               bool have_lse, cudaStream_t s) {
+  int* err = at<int>(ws, w.err);
+  if (c->mode == MOE_EXPERT_CHOICE) {
+    SelectEcArgs a{};
+    a.S = S;
+    a.n = c->n;
+    a.E = c->E;
+    a.k = dv.k;
+    a.kpad = dv.kpad;
+    a.idx = o->idx;
+    a.gate = o->gate;
+    a.ec_row = at<int32_t>(ws, w.ec_row);
+    a.ec_gate = at<float>(ws, w.ec_gate);
+    a.row_token = o->row_token;
+    a.load = o->load;
+    a.counts = o->counts;
+    a.offsets = o->offsets;
+    a.err = err;
+    MOE_CU(launch_select_ec(a, s));
+    EcFinishArgs f{};
+    f.ec_row = a.ec_row;
+    f.ec_gate = a.ec_gate;
+    f.n = c->n;
+    f.E = c->E;
+    f.tok_row = o->tok_row;
+    f.tok_gate = o->tok_gate;
+    f.hist = o->ec_hist;
+    f.aux = o->aux;
+    f.lse2 = have_lse ? at<double>(ws, w.lse2) : nullptr;
+    f.lse_blocks = colsum_blocks;
+    f.z_coef = c->z_coef;
+    MOE_CU(launch_ec_finish(f, s));
+    return MOE_OK;
+  }
+  TcAssignArgs a{};
+  a.idx = o->idx;
+  a.gate = o->gate;
+  a.n = c->n;
+  a.E = c->E;
+  a.K = dv.k;
+  a.cap = dv.cap;
+  a.tok_blocks = dv.tok_blocks;
+  a.blk_hist = at<int32_t>(ws, w.blk_hist);
+  a.blk_base = at<int32_t>(ws, w.blk_base);
+  a.load = o->load;
+  a.counts = o->counts;
+  a.offsets = o->offsets;
+  a.row_token = o->row_token;
+  a.tok_row = o->tok_row;
+  a.tok_gate = o->tok_gate;
+  a.drop = o->drop;
+  a.aux = o->aux;
+  a.colsum = at<float>(ws, w.colsum);
+  a.colsum_blocks = colsum_blocks;
+  a.lse2 = have_lse ? at<double>(ws, w.lse2) : nullptr;
+  a.lse_blocks = colsum_blocks;
+  a.lb_coef = c->lb_coef;
+  a.z_coef = c->z_coef;
+  MOE_CU(launch_tc_assign(a, s));
+  return MOE_OK;
+}
+
+static moe_status route_impl(const moe_config* c, const Derived& dv, const WsLayout& w,
+                             const void* X, const float* Wg, const float* logit_bias,
+                             const float* sel_bias, moe_route_out* o, void* ws,
+                             cudaStream_t s) {
+  RouterArgs r{};
+  r.X = X;
+  r.Wg = Wg;
+  r.logit_bias = logit_bias;
+  r.sel_bias = c->mode == MOE_TOKEN_CHOICE ? sel_bias : nullptr;
+  r.n = c->n;
+  r.d = c->d;
+  r.E = c->E;
+  r.x_bf16 = c->dtype == MOE_BF16;
+  r.score = c->score;
+  r.K = c->mode == MOE_TOKEN_CHOICE ? dv.k : 0;
+  r.n_groups = c->n_groups > 1 ? c->n_groups : 1;
+  r.topk_groups = c->topk_groups;
+  r.group_topn = c->group_topn;
+  r.weights = c->weights;
+  r.idx = o->idx;
+  r.gate = o->gate;
+  r.logits = o->logits;
+  r.scores = o->scores;
+  r.lse = o->lse;
+  r.colsum = at<float>(ws, w.colsum);
+  r.lse2 = at<double>(ws, w.lse2);
+  MOE_CU(launch_router(r, s));
+  return finish_route(c, dv, w, o, ws, o->scores, ceil_div(c->n, router_block_rows(c->E)),
+                      true, s);
+}
+
+static moe_status ffn_impl(const moe_config* c, const Derived& dv, const void* X,
+                           const void* X_perm, const int32_t* offsets, const void* W1,
+                           const void* W3, const void* W2, const void* sW1, const void* sW3,
+                           const void* sW2, void* H, void* Y, int* err, cudaStream_t s) {
+  if (!X_perm || !offsets || !W1 || !W2 || !H || !Y) return MOE_ERR_INVALID_ARG;
+  if (c->act == MOE_ACT_SWIGLU && !W3) return MOE_ERR_INVALID_ARG;
+  if (c->n_shared > 0) {
+    if (!X || !sW1 || !sW2) return MOE_ERR_INVALID_ARG;
+    if (c->act == MOE_ACT_SWIGLU && !sW3) return MOE_ERR_INVALID_ARG;
+  }
+  FfnArgs f{};
+  f.X = X;
+  f.X_perm = X_perm;
+  f.offsets = offsets;
+  f.W1 = W1;
+  f.W3 = W3;
+  f.W2 = W2;
+  f.sW1 = sW1;
+  f.sW3 = sW3;
+  f.sW2 = sW2;
+  f.H = H;
+  f.Y = Y;
+  f.n = c->n;
+  f.d = c->d;
+  f.h = c->h;
+  f.E = c->E;
+  f.act = c->act;
+  f.n_shared = c->n_shared;
+  f.n_pad = dv.n_pad;
+  f.rows_routed = dv.rows_routed;
+  f.shared_base = dv.shared_base;
+  f.rows = dv.rows;
+  f.err = err;
+  return c->dtype == MOE_BF16 ? run_ffn_bf16(f, s) : run_ffn_f32(f, s);
+}
+
+static moe_status dispatch_impl(const moe_config* c, const Derived& dv, const void* X,
+                                const moe_route_out* o, void* X_perm, cudaStream_t s) {
+  GatherArgs g{};
+  g.X = X;
+  g.row_token = o->row_token;
+  g.offsets = o->offsets;
+  g.E = c->E;
+  g.d = c->d;
+  g.elt_bytes = c->dtype == MOE_BF16 ? 2 : 4;
+  g.max_rows = dv.rows_routed;
+  g.X_perm = X_perm;
+  MOE_CU(launch_gather(g, s));
+  return MOE_OK;
+}
+
+static moe_status combine_impl(const moe_config* c, const Derived& dv, const void* Y,
+                               const moe_route_out* o, void* out, cudaStream_t s) {
+  CombineArgs a{};
+  a.Y = Y;
+  a.tok_row = o->tok_row;
+  a.tok_gate = o->tok_gate;
+  a.n = c->n;
+  a.d = c->d;
+  a.slots = dv.slots;
+  a.bf16 = c->dtype == MOE_BF16;
+  a.n_shared = c->n_shared;
+  a.n_pad = dv.n_pad;
+  a.shared_base = dv.shared_base;
+  a.max_rows = dv.rows_routed;
+  a.out = out;
+  MOE_CU(launch_combine(a, s));
+  return MOE_OK;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape or option";
+    case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_TIMEOUT: return "a bounded device wait gave up";
+  }
+  return "unknown status";
+}
+
+moe_status moe_validate(const moe_config* cfg) {
+  Derived d;
+  return derive(cfg, &d);
+}
+
+moe_status moe_sizes(const moe_config* cfg, int* k_eff, int* capacity_eff, int* slots,
+                     int* rows, int* shared_row_base) {
+  Derived d;
+  moe_status st = derive(cfg, &d);
+  if (st != MOE_OK) return st;
+  if (k_eff) *k_eff = d.k;
+  if (capacity_eff) *capacity_eff = cfg->mode == MOE_TOKEN_CHOICE ? d.cap : d.k;
+  if (slots) *slots = d.slots;
+  if (rows) *rows = (int)d.rows;
+  if (shared_row_base) *shared_row_base = (int)d.shared_base;
+  return MOE_OK;
+}
+
+moe_status moe_workspace_size(const moe_config* cfg, size_t* route_bytes,
+                              size_t* layer_bytes) {
+  Derived d;
+  moe_status st = derive(cfg, &d);
+  if (st != MOE_OK) return st;
+  const WsLayout w = ws_layout(cfg, d);
+  if (route_bytes) *route_bytes = w.route_end;
+  if (layer_bytes) *layer_bytes = w.layer_end;
+  return MOE_OK;
+}
+
+moe_status moe_route(const moe_config* cfg, const void* X, const float* Wg,
+                     const float* logit_bias, const float* sel_bias, moe_route_out* out,
+                     void* ws, size_t ws_bytes, moe_stream_t stream) {
+  Derived d;
+  moe_status st = derive(cfg, &d);
+  if (st != MOE_OK) return st;
+  if (!X || !Wg) return MOE_ERR_INVALID_ARG;
+  if ((st = check_route_out(cfg, out)) != MOE_OK) return st;
+  const WsLayout w = ws_layout(cfg, d);
+  if ((st = check_ws(ws, ws_bytes, w.route_end)) != MOE_OK) return st;
+  return route_impl(cfg, d, w, X, Wg, logit_bias, sel_bias, out, ws, (cudaStream_t)stream);
+}
+
+moe_status moe_route_from_scores(const moe_config* cfg, const float* S, const float* sel_bias,
+                                 moe_route_out* out, void* ws, size_t ws_bytes,
+                                 moe_stream_t stream) {
+  Derived d;
+  moe_status st = derive(cfg, &d);
+  if (st != MOE_OK) return st;
+  if (!S) return MOE_ERR_INVALID_ARG;
+  if ((st = check_route_out(cfg, out)) != MOE_OK) return st;
+  const WsLayout w = ws_layout(cfg, d);
+  if ((st = check_ws(ws, ws_bytes, w.route_end)) != MOE_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cfg->mode == MOE_TOKEN_CHOICE) {
+    SelectTcArgs a{};
+    a.S = S;
+    a.sel_bias = sel_bias;
+    a.n = cfg->n;
+    a.E = cfg->E;
+    a.K = d.k;
+    a.n_groups = cfg->n_groups > 1 ? cfg->n_groups : 1;
+    a.topk_groups = cfg->topk_groups;
+    a.group_topn = cfg->group_topn;
+    a.weights = cfg->weights;
+    a.idx = out->idx;
+    a.gate = out->gate;
+    a.scores_copy = out->scores != S ? out->scores : nullptr;
+    a.colsum = at<float>(ws, w.colsum);
+    MOE_CU(launch_select_tc(a, s));
+    return finish_route(cfg, d, w, out, ws, S, ceil_div(cfg->n, select_tc_block_rows()), false,
+                        s);
+  }
+  if (out->scores != S)
+    MOE_CU(cudaMemcpyAsync(out->scores, S, (size_t)cfg->n * cfg->E * sizeof(float),
+                           cudaMemcpyDeviceToDevice, s));
+  return finish_route(cfg, d, w, out, ws, S, 0, false, s);
+}
+
+moe_status moe_dispatch(const moe_config* cfg, const void* X, const moe_route_out* route,
+                        void* X_perm, moe_stream_t stream) {
+  Derived d;
+  moe_status st = derive(cfg, &d);
+  if (st != MOE_OK) return st;
+  if (!X || !X_perm || !route || !route->row_token || !route->offsets)
+    return MOE_ERR_INVALID_ARG;
+  return dispatch_impl(cfg, d, X, route, X_perm, (cudaStream_t)stream);
+}
+
+moe_status moe_expert_ffn(const moe_config* cfg, const void* X, const void* X_perm,
+                          const int32_t* offsets, const void* W1, const void* W3,
+                          const void* W2, const void* sW1, const void* sW3, const void* sW2,
+                          void* H, void* Y_perm, void* ws, size_t ws_bytes,
+                          moe_stream_t stream) {
+  Derived d;
+  moe_status st = derive(cfg, &d);
+  if (st != MOE_OK) return st;
+  if ((st = check_ws(ws, ws_bytes, MOE_WS_ERROR_BYTES)) != MOE_OK) return st;
+  return ffn_impl(cfg, d, X, X_perm, offsets, W1, W3, W2, sW1, sW3, sW2, H, Y_perm,
+                  at<int>(ws, 0), (cudaStream_t)stream);
+}
+
+moe_status moe_combine(const moe_config* cfg, const void* Y_perm, const moe_route_out* route,
+                       void* out, moe_stream_t stream) {
+  Derived d;
+  moe_status st = derive(cfg, &d);
+  if (st != MOE_OK) return st;
+  if (!Y_perm || !out || !route || !route->tok_row || !route->tok_gate)
+    return MOE_ERR_INVALID_ARG;
+  return combine_impl(cfg, d, Y_perm, route, out, (cudaStream_t)stream);
+}
+
+moe_status moe_layer_forward(const moe_config* cfg, const void* X, const float* Wg,
+                             const float* logit_bias, const float* sel_bias, const void* W1,
+                             const void* W3, const void* W2, const void* sW1, const void* sW3,
+                             const void* sW2, void* out, moe_route_out* route, void* ws,
+                             size_t ws_bytes, moe_stream_t stream) {
+  Derived d;
+  moe_status st = derive(cfg, &d);
+  if (st != MOE_OK) return st;
+  if (!X || !Wg || !out || !W1 || !W2) return MOE_ERR_INVALID_ARG;
+  if ((st = check_route_out(cfg, route)) != MOE_OK) return st;
+  const WsLayout w = ws_layout(cfg, d);
+  if ((st = check_ws(ws, ws_bytes, w.layer_end)) != MOE_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  void* xp = at<void>(ws, w.xperm);
+  void* hb = at<void>(ws, w.hbuf);
+  void* yp = at<void>(ws, w.yperm);
+  if ((st = route_impl(cfg, d, w, X, Wg, logit_bias, sel_bias, route, ws, s)) != MOE_OK)
+    return st;
+  if ((st = dispatch_impl(cfg, d, X, route, xp, s)) != MOE_OK) return st;
+  if ((st = ffn_impl(cfg, d, X, xp, route->offsets, W1, W3, W2, sW1, sW3, sW2, hb, yp,
+                     at<int>(ws, w.err), s)) != MOE_OK)
+    return st;
+  return combine_impl(cfg, d, yp, route, out, s);
+}
+
+moe_status moe_bias_update(const moe_config* cfg, const int32_t* load, float rate, float* bias,
+                           moe_stream_t stream) {
+  Derived d;
+  moe_status st = derive(cfg, &d);
+  if (st != MOE_OK) return st;
+  if (cfg->mode != MOE_TOKEN_CHOICE) return MOE_ERR_INVALID_ARG;
+  if (!load || !bias) return MOE_ERR_INVALID_ARG;
+  MOE_CU(launch_bias_update(cfg->n, cfg->E, d.k, load, rate, bias, (cudaStream_t)stream));
+  return MOE_OK;
+}
+
+moe_status moe_workspace_init(void* ws, moe_stream_t stream) {
+  if (!ws) return MOE_ERR_WORKSPACE;
+  MOE_CU(cudaMemsetAsync(ws, 0, MOE_WS_ERROR_BYTES, (cudaStream_t)stream));
+  return MOE_OK;
+}
+
+moe_status moe_read_error(void* ws, moe_stream_t stream, int* detail) {
+  if (!ws) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  int code = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpy(&code, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpy(ws, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (detail) *detail = code;
+  if (code == 0) return MOE_OK;
+  return (code & 0xF00) == kErrGemmTimeout ? MOE_ERR_TIMEOUT : MOE_ERR_CUDA;
+}
+
+}  // extern "C"

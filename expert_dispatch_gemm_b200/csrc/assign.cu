@@ -1,0 +1,405 @@
+// Selection bookkeeping: expert-choice top-k over the token axis, token-choice
+// capacity (arrival positions, drop mask, counts, offsets), the per-token
+// slot lists used by the combine, and the aux values.
+//
+// "Expert choice routing" (aicassindra.com), "The math: a gating matrix and
+// top-k over tokens": G, I = TopK(S^T, k), I and G are [E,k]; "Token choice
+// vs expert choice routing in MoE" (fanout.sh), "Dropped tokens flow in
+// opposite directions": assignments that arrive after an expert's buffer is
+// full skip it; "MoE routing strategies explained" (ncijnetwork.com), "2.
+// Top-1 switch routing with a capacity factor".
+#include "device_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+// fp32 -> uint32 whose unsigned order is the float order (-0 folded to +0).
+__device__ __forceinline__ uint32_t ordered_key(float f) {
+  f = f + 0.0f;  // -0 + 0 = +0 under round-to-nearest
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// ---------------------------------------------------------------------------
+// Expert choice: one CTA per expert. Radix-select the k-th largest key of the
+// column, take every key above it plus the lowest-index ties, then sort the
+// k picks by (score desc, token asc) with a bitonic sort of composite keys.
+// ---------------------------------------------------------------------------
+constexpr int kEcThreads = 1024;
+
+__global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
+  extern __shared__ __align__(16) unsigned char ec_smem[];
+  const int n = a.n, E = a.E, k = a.k, e = blockIdx.x;
+  int kp = 1;
+  while (kp < k) kp <<= 1;
+  uint64_t* sbuf = reinterpret_cast<uint64_t*>(ec_smem);           // [kp]
+  uint32_t* key = reinterpret_cast<uint32_t*>(sbuf + kp);          // [n]
+  __shared__ int hist[256];
+  __shared__ int warp_tot[32];
+  __shared__ uint32_t s_prefix, s_mask;
+  __shared__ int s_need, s_cnt;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  for (int t = tid; t < n; t += kEcThreads) {
+    key[t] = ordered_key(a.S[(size_t)t * E + e]);
+    a.ec_row[(size_t)t * E + e] = -1;
+    a.ec_gate[(size_t)t * E + e] = 0.0f;
+  }
+  if (tid == 0) {
+    s_prefix = 0u;
+    s_mask = 0u;
+    s_need = k;
+    s_cnt = 0;
+  }
+  __syncthreads();
+
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int i = tid; i < 256; i += kEcThreads) hist[i] = 0;
+    __syncthreads();
+    const uint32_t prefix = s_prefix, mask = s_mask;
+    for (int t = tid; t < n; t += kEcThreads) {
+      const uint32_t u = key[t];
+      if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // lane l holds digits 255-8l down to 248-8l (descending)
+      int cnt[8], local = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        cnt[i] = hist[255 - 8 * lane - i];
+        local += cnt[i];
+      }
+      int incl = local;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const int excl = incl - local;
+      const int need = s_need;
+      const bool here = excl < need && need <= incl;
+      const unsigned who = __ballot_sync(0xffffffffu, here);
+      if (here && lane == __ffs(who) - 1) {
+        int above = excl;
+        int digit = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (above + cnt[i] >= need) {
+            digit = 255 - 8 * lane - i;
+            break;
+          }
+          above += cnt[i];
+        }
+        s_need = need - above;
+        s_prefix = prefix | ((uint32_t)digit << shift);
+        s_mask = mask | (255u << shift);
+      }
+    }
+    __syncthreads();
+  }
+  const uint32_t T = s_prefix;
+  const int need_eq = s_need;  // ties at T to take, lowest token first
+
+  // ordered count of ties: thread tid owns tokens [tid*C, tid*C + C)
+  const int C = (n + kEcThreads - 1) / kEcThreads;
+  const int t0 = tid * C, t1 = min(n, t0 + C);
+  int my_eq = 0;
+  for (int t = t0; t < t1; ++t) my_eq += (key[t] == T);
+  int incl = my_eq;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  int wbase = 0;
+  for (int w = 0; w < warp; ++w) wbase += warp_tot[w];
+  int rank = wbase + incl - my_eq;
+  for (int t = t0; t < t1; ++t) {
+    const uint32_t u = key[t];
+    bool sel = u > T;
+    if (u == T) {
+      sel = rank < need_eq;
+      ++rank;
+    }
+    if (sel) {
+      const int slot = atomicAdd(&s_cnt, 1);
+      sbuf[slot] = ((uint64_t)u << 32) | (uint64_t)(0xffffffffu - (uint32_t)t);
+    }
+  }
+  __syncthreads();
+  for (int i = k + tid; i < kp; i += kEcThreads) sbuf[i] = 0ull;
+  __syncthreads();
+  // bitonic sort, descending
+  for (int size = 2; size <= kp; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = tid; i < kp / 2; i += kEcThreads) {
+        const int lo = 2 * i - (i & (stride - 1));
+        const int hi = lo + stride;
+        const bool desc = ((lo & size) == 0);
+        const uint64_t x = sbuf[lo], y = sbuf[hi];
+        if ((x < y) == desc) {
+          sbuf[lo] = y;
+          sbuf[hi] = x;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  if (s_cnt != k && tid == 0) report_error(a.err, kErrBadIndex | 1);
+  for (int j = tid; j < a.kpad; j += kEcThreads) {
+    const size_t row = (size_t)e * a.kpad + j;
+    if (j < k) {
+      const int t = (int)(0xffffffffu - (uint32_t)(sbuf[j] & 0xffffffffull));
+      const float g = a.S[(size_t)t * E + e];
+      a.idx[(size_t)e * k + j] = t;
+      a.gate[(size_t)e * k + j] = g;
+      a.row_token[row] = t;
+      a.ec_row[(size_t)t * E + e] = (int)row;
+      a.ec_gate[(size_t)t * E + e] = g;
+    } else {
+      a.row_token[row] = -1;
+    }
+  }
+  if (tid == 0) {
+    a.load[e] = k;
+    a.counts[e] = k;
+    a.offsets[e] = e * a.kpad;
+    if (e == E - 1) a.offsets[E] = E * a.kpad;
+  }
+}
+
+cudaError_t launch_select_ec(const SelectEcArgs& a, cudaStream_t s) {
+  int kp = 1;
+  while (kp < a.k) kp <<= 1;
+  const size_t bytes = (size_t)kp * 8 + (size_t)a.n * 4;
+  cudaError_t err = cudaFuncSetAttribute(select_ec_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)bytes);
+  if (err != cudaSuccess) return err;
+  select_ec_kernel<<<a.E, kEcThreads, bytes, s>>>(a);
+  return cudaGetLastError();
+}
+
+// Expert choice: compact each token's picks (expert order) into its slot
+// list, the experts-per-token histogram and the aux values. Warp per token.
+__global__ void __launch_bounds__(256) ec_finish_kernel(EcFinishArgs a) {
+  __shared__ int hist_s[MOE_MAX_EXPERTS + 1];
+  __shared__ int none_s;
+  const int E = a.E, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i <= E; i += blockDim.x) hist_s[i] = 0;
+  if (threadIdx.x == 0) none_s = 0;
+  __syncthreads();
+  const int t = blockIdx.x * 8 + warp;
+  if (t < a.n) {
+    int base = 0;
+    for (int c = 0; c < E; c += 32) {
+      const int e = c + lane;
+      int r = -1;
+      float g = 0.0f;
+      if (e < E) {
+        r = a.ec_row[(size_t)t * E + e];
+        g = a.ec_gate[(size_t)t * E + e];
+      }
+      const unsigned m = __ballot_sync(0xffffffffu, r >= 0);
+      if (r >= 0) {
+        const int p = base + __popc(m & ((1u << lane) - 1u));
+        a.tok_row[(size_t)t * E + p] = r;
+        a.tok_gate[(size_t)t * E + p] = g;
+      }
+      base += __popc(m);
+    }
+    for (int p = base + lane; p < E; p += 32) {
+      a.tok_row[(size_t)t * E + p] = -1;
+      a.tok_gate[(size_t)t * E + p] = 0.0f;
+    }
+    if (lane == 0) {
+      atomicAdd(&hist_s[base], 1);
+      if (base == 0) atomicAdd(&none_s, 1);
+    }
+  }
+  __syncthreads();
+  if (a.hist)
+    for (int i = threadIdx.x; i <= E; i += blockDim.x)
+      if (hist_s[i]) atomicAdd(&a.hist[i], hist_s[i]);
+  if (threadIdx.x == 0 && none_s) atomicAdd(&a.aux[MOE_AUX_TOKENS_NO_EXPERT], (float)none_s);
+}
+
+// zero the accumulators the EC finish kernel adds into and set fixed aux
+__global__ void ec_aux_init_kernel(EcFinishArgs a) {
+  for (int i = threadIdx.x; i <= a.E; i += blockDim.x)
+    if (a.hist) a.hist[i] = 0;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < MOE_AUX_LEN; ++i) a.aux[i] = 0.0f;
+    if (a.lse2) {
+      double s = 0.0;
+      for (int b = 0; b < a.lse_blocks; ++b) s += a.lse2[b];
+      a.aux[MOE_AUX_Z] = (float)((double)a.z_coef * s / (double)a.n);
+    }
+  }
+}
+
+cudaError_t launch_ec_finish(const EcFinishArgs& a, cudaStream_t s) {
+  ec_aux_init_kernel<<<1, 256, 0, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  ec_finish_kernel<<<ceil_div(a.n, 8), 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Token choice: per-block expert histograms, a scan over blocks (counts,
+// offsets, aux), then arrival positions, drops and slot lists.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kTokBlock) tc_hist_kernel(TcAssignArgs a) {
+  __shared__ int hist[MOE_MAX_EXPERTS];
+  for (int i = threadIdx.x; i < a.E; i += kTokBlock) hist[i] = 0;
+  __syncthreads();
+  const int t = blockIdx.x * kTokBlock + threadIdx.x;
+  if (t < a.n)
+    for (int j = 0; j < a.K; ++j) {
+      const int e = a.idx[(size_t)t * a.K + j];
+      if ((unsigned)e < (unsigned)a.E) atomicAdd(&hist[e], 1);
+    }
+  __syncthreads();
+  for (int i = threadIdx.x; i < a.E; i += kTokBlock)
+    a.blk_hist[(size_t)blockIdx.x * a.E + i] = hist[i];
+}
+
+__global__ void __launch_bounds__(1024) tc_scan_kernel(TcAssignArgs a) {
+  __shared__ int seg[MOE_MAX_EXPERTS];
+  __shared__ int off[MOE_MAX_EXPERTS + 1];
+  __shared__ double fp[MOE_MAX_EXPERTS];
+  const int E = a.E, tid = threadIdx.x;
+  for (int e = tid; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int b = 0; b < a.tok_blocks; ++b) {
+      a.blk_base[(size_t)b * E + e] = run;
+      run += a.blk_hist[(size_t)b * E + e];
+    }
+    const int kept = a.cap < 0 ? run : min(run, a.cap);
+    a.load[e] = run;
+    a.counts[e] = kept;
+    seg[e] = (kept + kRowAlign - 1) / kRowAlign * kRowAlign;
+    double col = 0.0;
+    for (int b = 0; b < a.colsum_blocks; ++b) col += (double)a.colsum[(size_t)b * E + e];
+    fp[e] = ((double)run / ((double)a.n * a.K)) * (col / (double)a.n);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    double lbs = 0.0;
+    int mx = 0;
+    long long dropped = 0;
+    for (int e = 0; e < E; ++e) {
+      off[e] = run;
+      run += seg[e];
+      lbs += fp[e];
+      mx = max(mx, a.load[e]);
+      dropped += a.load[e] - a.counts[e];
+    }
+    off[E] = run;
+    a.aux[MOE_AUX_LB] = (float)((double)a.lb_coef * E * lbs);
+    double z = 0.0;
+    if (a.lse2) {
+      for (int b = 0; b < a.lse_blocks; ++b) z += a.lse2[b];
+      z = (double)a.z_coef * z / (double)a.n;
+    }
+    a.aux[MOE_AUX_Z] = (float)z;
+    a.aux[MOE_AUX_MAXVIO] = (float)((double)mx / ((double)a.n * a.K / E) - 1.0);
+    a.aux[MOE_AUX_DROPPED] = (float)dropped;
+    a.aux[MOE_AUX_TOKENS_SOME_DROPPED] = 0.0f;
+    a.aux[MOE_AUX_TOKENS_ALL_DROPPED] = 0.0f;
+    a.aux[MOE_AUX_TOKENS_NO_EXPERT] = 0.0f;
+    a.aux[MOE_AUX_RESERVED] = 0.0f;
+  }
+  __syncthreads();
+  for (int e = tid; e <= E; e += blockDim.x) a.offsets[e] = off[e];
+  // padding rows of each segment
+  for (int e = 0; e < E; ++e) {
+    const int lo = off[e] + a.counts[e], hi = off[e + 1];
+    for (int r = lo + tid; r < hi; r += blockDim.x) a.row_token[r] = -1;
+  }
+}
+
+__global__ void __launch_bounds__(kTokBlock) tc_scatter_kernel(TcAssignArgs a) {
+  extern __shared__ __align__(16) unsigned char sc_smem[];
+  const int E = a.E, K = a.K;
+  uint32_t* mask = reinterpret_cast<uint32_t*>(sc_smem);      // [32][E]
+  int* wbase = reinterpret_cast<int*>(mask + 32 * E);         // [32][E]
+  __shared__ int some_s, all_s;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < 32 * E; i += kTokBlock) mask[i] = 0u;
+  if (tid == 0) {
+    some_s = 0;
+    all_s = 0;
+  }
+  __syncthreads();
+  const int t = blockIdx.x * kTokBlock + tid;
+  const bool live = t < a.n;
+  if (live)
+    for (int j = 0; j < K; ++j) {
+      const int e = a.idx[(size_t)t * K + j];
+      if ((unsigned)e < (unsigned)E) atomicOr(&mask[warp * E + e], 1u << lane);
+    }
+  __syncthreads();
+  for (int e = tid; e < E; e += kTokBlock) {
+    int run = 0;
+    for (int w = 0; w < 32; ++w) {
+      wbase[w * E + e] = run;
+      run += __popc(mask[w * E + e]);
+    }
+  }
+  __syncthreads();
+  if (live) {
+    int kept = 0;
+    for (int j = 0; j < K; ++j) {
+      const size_t aj = (size_t)t * K + j;
+      const int e = a.idx[aj];
+      bool keep = false;
+      int row = -1;
+      if ((unsigned)e < (unsigned)E) {
+        const int pos = a.blk_base[(size_t)blockIdx.x * E + e] + wbase[warp * E + e] +
+                        __popc(mask[warp * E + e] & ((1u << lane) - 1u));
+        keep = a.cap < 0 || pos < a.cap;
+        if (keep) {
+          row = a.offsets[e] + pos;
+          a.row_token[row] = t;
+          a.tok_row[(size_t)t * K + kept] = row;
+          a.tok_gate[(size_t)t * K + kept] = a.gate[aj];
+          ++kept;
+        }
+      }
+      a.drop[aj] = keep ? 0 : 1;
+    }
+    for (int j = kept; j < K; ++j) {
+      a.tok_row[(size_t)t * K + j] = -1;
+      a.tok_gate[(size_t)t * K + j] = 0.0f;
+    }
+    if (kept < K) atomicAdd(&some_s, 1);
+    if (kept == 0) atomicAdd(&all_s, 1);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    if (some_s) atomicAdd(&a.aux[MOE_AUX_TOKENS_SOME_DROPPED], (float)some_s);
+    if (all_s) atomicAdd(&a.aux[MOE_AUX_TOKENS_ALL_DROPPED], (float)all_s);
+  }
+}
+
+cudaError_t launch_tc_assign(const TcAssignArgs& a, cudaStream_t s) {
+  tc_hist_kernel<<<a.tok_blocks, kTokBlock, 0, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  tc_scan_kernel<<<1, 1024, 0, s>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t bytes = (size_t)64 * a.E * 4;
+  e = cudaFuncSetAttribute(tc_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)bytes);
+  if (e != cudaSuccess) return e;
+  tc_scatter_kernel<<<a.tok_blocks, kTokBlock, bytes, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

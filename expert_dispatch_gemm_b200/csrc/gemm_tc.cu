@@ -1,0 +1,490 @@
+// Grouped expert FFN on the 5th-generation tensor cores (tcgen05 + TMEM).
+//
+// "Expert choice routing" (aicassindra.com), "The math: a gating matrix and
+// top-k over tokens": the gathered per-expert batches are dense matrices
+// "ideal for batched matmuls"; each expert's FFN is one up projection (with
+// the activation, or SwiGLU's two projections fused) and one down projection.
+//
+// One persistent CTA per SM, warp-specialised:
+//   warp 0      TMA producer: A tile 128x64 and B tile 256x64 (bf16, 128-byte
+//               swizzle) per stage into a 4-deep shared-memory ring;
+//   warp 1      allocates 512 TMEM columns and issues tcgen05.mma
+//               (M=128, N=256, K=16) from one thread; commits free the smem
+//               stage and, per tile, hand the accumulator to the epilogue;
+//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, activation, bf16,
+//               16-byte stores of each thread's row.
+// Two TMEM accumulators (2 x 256 columns) let the epilogue of one tile
+// overlap the main loop of the next. Tiles are (128-row block of one
+// expert's segment, 256-column block); rows of a block never straddle two
+// experts because segments start on 128-row boundaries. The B tile of a
+// SwiGLU up projection holds 128 rows of W1 followed by the same 128 rows of
+// W3, so one N=256 MMA produces both halves of the gate.
+// Every mbarrier wait is bounded; on a timeout the CTA records an error,
+// stops issuing, waits (bounded) for its own copies and MMAs, frees TMEM and
+// returns.
+#include <cuda.h>
+#include <math.h>
+
+#include <mutex>
+
+#include "device_common.cuh"
+#include "moe_internal.h"
+#include "sm100.cuh"
+
+namespace moe {
+
+constexpr int kBM = 128, kBN = 256, kBK = 64, kStages = 4;
+constexpr int kABytes = kBM * kBK * 2;       // 16 KB
+constexpr int kBBytes = kBN * kBK * 2;       // 32 KB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kTmemCols = 512;
+constexpr int kGemmThreads = 192;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+enum { ACT_NONE = 0, ACT_RELU = 1, ACT_GELU = 2, ACT_SWIGLU = 3 };
+
+struct TcGemmParams {
+  const int32_t* offsets;
+  int E;
+  int K;                    // reduction length (multiple of 64)
+  int n_out;                // output columns
+  int nt_tiles;             // column blocks
+  int b_rows_per_expert;    // rows of B per expert
+  int shared_tiles_per;     // 128-row blocks per shared expert
+  int n_shared;
+  int max_routed_tiles;     // host bound on offsets[E] / 128
+  long long a1_row_base;    // shared experts' A rows: base + s*stride + block*128
+  long long a1_row_stride;
+  long long out_shared_base;
+  long long n_pad;
+  __nv_bfloat16* out;       // [rows, n_out]
+  int* err;
+};
+
+struct SharedState {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  volatile int abort_flag;
+  int offs[MOE_MAX_EXPERTS + 1];
+};
+
+__device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, SharedState* st,
+                                             int* err, int code) {
+  if (sm100::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (sm100::mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (st->abort_flag) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        st->abort_flag = 1;
+        report_error(err, code);
+        return false;
+      }
+    }
+  }
+}
+
+struct TileCoord {
+  int a_sel, a_row, b_sel, b_row;
+  long long out_row;
+  int col0;
+};
+
+template <int ACT>
+__device__ __forceinline__ TileCoord decode_tile(int tile, const TcGemmParams& p,
+                                                 const int* offs, int Tr) {
+  constexpr int BNO = ACT == ACT_SWIGLU ? kBN / 2 : kBN;
+  TileCoord c;
+  const int mt = tile / p.nt_tiles, nt = tile % p.nt_tiles;
+  if (mt < Tr) {
+    const int row = mt * kBM;
+    int lo = 0, hi = p.E - 1;  // largest e with offs[e] <= row
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (offs[mid] <= row) lo = mid; else hi = mid - 1;
+    }
+    c.a_sel = 0;
+    c.a_row = row;
+    c.b_sel = 0;
+    c.b_row = lo * p.b_rows_per_expert;
+    c.out_row = row;
+  } else {
+    const int q = mt - Tr;
+    const int s = q / p.shared_tiles_per, lm = q % p.shared_tiles_per;
+    c.a_sel = 1;
+    c.a_row = (int)(p.a1_row_base + s * p.a1_row_stride + (long long)lm * kBM);
+    c.b_sel = 1;
+    c.b_row = s * p.b_rows_per_expert;
+    c.out_row = p.out_shared_base + s * p.n_pad + (long long)lm * kBM;
+  }
+  c.col0 = nt * BNO;
+  c.b_row += c.col0;
+  return c;
+}
+
+template <int ACT>
+__device__ __forceinline__ float act_fn(float v) {
+  if (ACT == ACT_RELU) return fmaxf(v, 0.0f);
+  if (ACT == ACT_GELU) return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));
+  return v;
+}
+
+template <int ACT>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    tc_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,
+                           const __grid_constant__ CUtensorMap tmA1,
+                           const __grid_constant__ CUtensorMap tmB0,
+                           const __grid_constant__ CUtensorMap tmB0g,
+                           const __grid_constant__ CUtensorMap tmB1,
+                           const __grid_constant__ CUtensorMap tmB1g, const TcGemmParams p) {
+  constexpr bool SWIGLU = ACT == ACT_SWIGLU;
+  extern __shared__ __align__(1024) unsigned char gsm[];
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(gsm) + 1023) & ~uintptr_t(1023));
+  unsigned char* sA = base;                            // [kStages][16 KB]
+  unsigned char* sB = base + kStages * kABytes;        // [kStages][32 KB]
+  SharedState* st = reinterpret_cast<SharedState*>(base + kStages * kStageBytes);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i <= p.E; i += kGemmThreads) st->offs[i] = p.offsets[i];
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      sm100::mbar_init(&st->full[s], 1);
+      sm100::mbar_init(&st->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      sm100::mbar_init(&st->tfull[a], 1);
+      sm100::mbar_init(&st->tempty[a], 128);
+    }
+    sm100::mbar_init(&st->drain, 1);
+    st->abort_flag = 0;
+    sm100::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    sm100::tma_prefetch_desc(&tmA0);
+    sm100::tma_prefetch_desc(&tmB0);
+    if (SWIGLU) sm100::tma_prefetch_desc(&tmB0g);
+  }
+  if (warp == 1) {
+    sm100::tmem_alloc(&st->tmem_base, kTmemCols);
+    sm100::tmem_relinquish();
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem = st->tmem_base;
+
+  const int Tr = min(max(st->offs[p.E], 0) / kBM, p.max_routed_tiles);
+  const int total = (Tr + p.n_shared * p.shared_tiles_per) * p.nt_tiles;
+  const int KB = p.K / kBK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        const TileCoord c = decode_tile<ACT>(tile, p, st->offs, Tr);
+        const CUtensorMap* ma = c.a_sel ? &tmA1 : &tmA0;
+        const CUtensorMap* mb = c.b_sel ? &tmB1 : &tmB0;
+        const CUtensorMap* mbg = c.b_sel ? &tmB1g : &tmB0g;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!bounded_wait(&st->empty[stage], phase ^ 1u, st, p.err, kErrGemmTimeout | 0x01)) {
+            ok = false;
+            break;
+          }
+          sm100::mbar_arrive_expect_tx(&st->full[stage], kStageBytes);
+          unsigned char* a_dst = sA + stage * kABytes;
+          unsigned char* b_dst = sB + stage * kBBytes;
+          sm100::tma_load_2d(a_dst, ma, &st->full[stage], kb * kBK, c.a_row);
+          if (SWIGLU) {
+            sm100::tma_load_2d(b_dst, mb, &st->full[stage], kb * kBK, c.b_row);
+            sm100::tma_load_2d(b_dst + kBBytes / 2, mbg, &st->full[stage], kb * kBK, c.b_row);
+          } else {
+            sm100::tma_load_2d(b_dst, mb, &st->full[stage], kb * kBK, c.b_row);
+          }
+          ++issued;
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // wait (bounded) for the copies still in flight into our stages
+        int s = stage;
+        uint32_t ph = phase;
+        const int pending = issued < kStages ? issued : kStages;
+        for (int i = 0; i < pending; ++i) {
+          if (--s < 0) {
+            s = kStages - 1;
+            ph ^= 1u;
+          }
+          const uint64_t t0 = global_timer_ns();
+          while (!sm100::mbar_try_wait(&st->full[s], ph) &&
+                 global_timer_ns() - t0 < kWaitLimitNs) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = sm100::idesc_bf16_f32(kBM, kBN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++local) {
+        const int acc = local & 1;
+        const uint32_t acc_phase = (uint32_t)(local >> 1) & 1u;
+        if (!bounded_wait(&st->tempty[acc], acc_phase ^ 1u, st, p.err, kErrGemmTimeout | 0x12)) {
+          ok = false;
+          break;
+        }
+        sm100::tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(acc * kBN);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!bounded_wait(&st->full[stage], phase, st, p.err, kErrGemmTimeout | 0x13)) {
+            ok = false;
+            break;
+          }
+          sm100::tc_fence_after();
+          const uint64_t adesc = sm100::sw128_kmajor_desc(sm100::smem_addr(sA + stage * kABytes));
+          const uint64_t bdesc = sm100::sw128_kmajor_desc(sm100::smem_addr(sB + stage * kBBytes));
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            // +32 bytes along K inside the swizzled 128-byte row = +2 in the
+            // address field
+            sm100::umma_f16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0);
+          }
+          sm100::umma_commit(&st->empty[stage]);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        sm100::umma_commit(&st->tfull[acc]);
+      }
+      // wait (bounded) until every MMA this thread issued has completed
+      sm100::umma_commit(&st->drain);
+      const uint64_t t0 = global_timer_ns();
+      while (!sm100::mbar_try_wait(&st->drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+      }
+    }
+  } else {
+    // epilogue warps 2..5: TMEM lane quadrant = warp % 4
+    const int q = warp & 3;
+    const int row_in_tile = q * 32 + lane;
+    constexpr int BNO = SWIGLU ? kBN / 2 : kBN;
+    int local = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+      const int acc = local & 1;
+      const uint32_t acc_phase = (uint32_t)(local >> 1) & 1u;
+      if (!bounded_wait(&st->tfull[acc], acc_phase, st, p.err, kErrGemmTimeout | 0x24)) break;
+      sm100::tc_fence_after();
+      const TileCoord c = decode_tile<ACT>(tile, p, st->offs, Tr);
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN);
+      __nv_bfloat16* orow = p.out + (size_t)(c.out_row + row_in_tile) * p.n_out;
+#pragma unroll 1
+      for (int cc = 0; cc < BNO; cc += 32) {
+        if (c.col0 + cc >= p.n_out) break;
+        uint32_t v[32];
+        sm100::tmem_ld_32x32b_x32(tbase + cc, v);
+        float f[32];
+        if (SWIGLU) {
+          uint32_t g[32];
+          sm100::tmem_ld_32x32b_x32(tbase + BNO + cc, g);
+          sm100::tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float a = __uint_as_float(v[i]);
+            const float b = __uint_as_float(g[i]);
+            f[i] = a * __frcp_rn(1.0f + __expf(-a)) * b;
+          }
+        } else {
+          sm100::tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) f[i] = act_fn<ACT>(__uint_as_float(v[i]));
+        }
+        uint4* dst = reinterpret_cast<uint4*>(orow + c.col0 + cc);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint4 o;
+          o.x = pack_bf16x2(f[8 * j + 0], f[8 * j + 1]);
+          o.y = pack_bf16x2(f[8 * j + 2], f[8 * j + 3]);
+          o.z = pack_bf16x2(f[8 * j + 4], f[8 * j + 5]);
+          o.w = pack_bf16x2(f[8 * j + 6], f[8 * j + 7]);
+          dst[j] = o;
+        }
+      }
+      sm100::tc_fence_before();
+      sm100::mbar_arrive(&st->tempty[acc]);
+    }
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    sm100::tc_fence_after();
+    sm100::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 row-major [rows, cols] map with a box of 64 columns x box_rows rows
+// and 128-byte swizzle. Out-of-range elements load as zero.
+static bool make_map(CUtensorMap* m, const void* ptr, long long rows, long long cols,
+                     int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows < box_rows || cols < kBK) return false;
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || ((cols * 2) & 15)) return false;
+  const cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t gstride[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
+  const cuuint32_t estride[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), gdim, gstride,
+            box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static size_t gemm_smem_bytes() {
+  return (size_t)kStages * kStageBytes + sizeof(SharedState) + 1024;
+}
+
+template <int ACT>
+static cudaError_t launch_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0,
+                             const CUtensorMap& b0g, const CUtensorMap& b1,
+                             const CUtensorMap& b1g, const TcGemmParams& p, int grid,
+                             cudaStream_t s) {
+  auto kern = tc_grouped_gemm_kernel<ACT>;
+  const size_t bytes = gemm_smem_bytes();
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kGemmThreads, bytes, s>>>(a0, a1, b0, b0g, b1, b1g, p);
+  return cudaGetLastError();
+}
+
+static int num_sms() {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+moe_status run_ffn_bf16(const FfnArgs& f, cudaStream_t s) {
+  const bool swiglu = f.act == MOE_ACT_SWIGLU;
+  const long long rows = f.rows;
+  const int sh_tiles = f.n_pad / kBM;
+  // ---- up projection: H = act(X_perm W1^T) or silu(X_perm W1^T) * (X_perm W3^T)
+  CUtensorMap a0, a1, b0, b0g, b1, b1g;
+  const int up_box = swiglu ? kBN / 2 : kBN;
+  if (!make_map(&a0, f.X_perm, rows, f.d, kBM)) return MOE_ERR_UNSUPPORTED;
+  if (f.n_shared > 0) {
+    if (!make_map(&a1, f.X, f.n, f.d, kBM)) return MOE_ERR_UNSUPPORTED;
+  } else {
+    a1 = a0;
+  }
+  if (!make_map(&b0, f.W1, (long long)f.E * f.h, f.d, up_box)) return MOE_ERR_UNSUPPORTED;
+  if (swiglu) {
+    if (!make_map(&b0g, f.W3, (long long)f.E * f.h, f.d, up_box)) return MOE_ERR_UNSUPPORTED;
+  } else {
+    b0g = b0;
+  }
+  if (f.n_shared > 0) {
+    if (!make_map(&b1, f.sW1, (long long)f.n_shared * f.h, f.d, up_box))
+      return MOE_ERR_UNSUPPORTED;
+    if (swiglu) {
+      if (!make_map(&b1g, f.sW3, (long long)f.n_shared * f.h, f.d, up_box))
+        return MOE_ERR_UNSUPPORTED;
+    } else {
+      b1g = b1;
+    }
+  } else {
+    b1 = b0;
+    b1g = b0g;
+  }
+  TcGemmParams p{};
+  p.offsets = f.offsets;
+  p.E = f.E;
+  p.K = f.d;
+  p.n_out = f.h;
+  p.nt_tiles = ceil_div(f.h, up_box);
+  p.b_rows_per_expert = f.h;
+  p.shared_tiles_per = sh_tiles;
+  p.n_shared = f.n_shared;
+  p.max_routed_tiles = (int)(f.rows_routed / kBM);
+  p.a1_row_base = 0;
+  p.a1_row_stride = 0;
+  p.out_shared_base = f.shared_base;
+  p.n_pad = f.n_pad;
+  p.out = static_cast<__nv_bfloat16*>(f.H);
+  p.err = f.err;
+  const int sms = num_sms();
+  long long tiles_up = (rows / kBM) * p.nt_tiles;
+  int grid = (int)(tiles_up < sms ? tiles_up : sms);
+  if (grid < 1) grid = 1;
+  cudaError_t e;
+  switch (f.act) {
+    case MOE_ACT_RELU: e = launch_tc<ACT_RELU>(a0, a1, b0, b0g, b1, b1g, p, grid, s); break;
+    case MOE_ACT_GELU: e = launch_tc<ACT_GELU>(a0, a1, b0, b0g, b1, b1g, p, grid, s); break;
+    default: e = launch_tc<ACT_SWIGLU>(a0, a1, b0, b0g, b1, b1g, p, grid, s); break;
+  }
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+
+  // ---- down projection: Y = H W2^T
+  CUtensorMap da0, db0, db1;
+  if (!make_map(&da0, f.H, rows, f.h, kBM)) return MOE_ERR_UNSUPPORTED;
+  if (!make_map(&db0, f.W2, (long long)f.E * f.d, f.h, kBN)) return MOE_ERR_UNSUPPORTED;
+  if (f.n_shared > 0) {
+    if (!make_map(&db1, f.sW2, (long long)f.n_shared * f.d, f.h, kBN))
+      return MOE_ERR_UNSUPPORTED;
+  } else {
+    db1 = db0;
+  }
+  TcGemmParams q = p;
+  q.K = f.h;
+  q.n_out = f.d;
+  q.nt_tiles = ceil_div(f.d, kBN);
+  q.b_rows_per_expert = f.d;
+  q.a1_row_base = f.shared_base;
+  q.a1_row_stride = f.n_pad;
+  q.out = static_cast<__nv_bfloat16*>(f.Y);
+  long long tiles_dn = (rows / kBM) * q.nt_tiles;
+  grid = (int)(tiles_dn < sms ? tiles_dn : sms);
+  if (grid < 1) grid = 1;
+  e = launch_tc<ACT_NONE>(da0, da0, db0, db0, db1, db1, q, grid, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+}  // namespace moe

@@ -1,0 +1,172 @@
+// Internal host-side declarations shared by the libmoe translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+constexpr int kTokBlock = 1024;   // tokens per block in the capacity scan
+constexpr int kRowAlign = MOE_ROW_ALIGN;
+
+inline int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+inline long long round_up(long long a, long long b) { return (a + b - 1) / b * b; }
+
+// Router tile: rows per CTA for a padded expert count ET.
+int router_tile_et(int E);
+int router_block_rows(int E);
+
+struct Derived {
+  int k;            // EC tokens per expert / TC experts per token
+  int cap;          // TC rows per expert, -1 dropless (EC: k)
+  int slots;        // columns of tok_row
+  int kpad;         // EC: k rounded up to the row alignment
+  long long rows_routed;  // upper bound on offsets[E]
+  long long rows;         // rows of X_perm / H / Y_perm
+  long long shared_base;  // first shared-expert row
+  int n_pad;              // roundup(n, 128)
+  int router_blocks;      // CTAs of the router / score-selection pass
+  int tok_blocks;         // token blocks of the capacity scan
+};
+
+// Workspace regions (byte offsets from the workspace base).
+struct WsLayout {
+  size_t err;        // 256 B error words
+  size_t colsum;     // [router_blocks, E] f32 partial column sums of S
+  size_t lse2;       // [router_blocks] f64 partial sums of lse^2
+  size_t blk_hist;   // [tok_blocks, E] i32
+  size_t blk_base;   // [tok_blocks, E] i32
+  size_t ec_row;     // [n, E] i32 (expert choice, dense)
+  size_t ec_gate;    // [n, E] f32 (expert choice, dense)
+  size_t route_end;
+  size_t xperm, hbuf, yperm;  // layer only
+  size_t layer_end;
+};
+
+moe_status derive(const moe_config* c, Derived* d);
+WsLayout ws_layout(const moe_config* c, const Derived& d);
+
+// ----- launchers (return the launch error; nothing is synchronised) -----
+struct RouterArgs {
+  const void* X;
+  const float* Wg;
+  const float* logit_bias;
+  const float* sel_bias;
+  int n, d, E, x_bf16, score;
+  // token choice selection (fused), or K = 0 for expert choice
+  int K, n_groups, topk_groups, group_topn, weights;
+  int32_t* idx;
+  float* gate;
+  float* logits;     // optional
+  float* scores;
+  float* lse;        // optional
+  float* colsum;     // [blocks, E]
+  double* lse2;      // [blocks]
+};
+cudaError_t launch_router(const RouterArgs& a, cudaStream_t s);
+
+struct SelectTcArgs {
+  const float* S;
+  const float* sel_bias;
+  int n, E, K, n_groups, topk_groups, group_topn, weights;
+  int32_t* idx;
+  float* gate;
+  float* scores_copy;  // optional copy of S
+  float* colsum;       // [blocks, E]
+};
+cudaError_t launch_select_tc(const SelectTcArgs& a, cudaStream_t s);
+int select_tc_block_rows();
+
+struct SelectEcArgs {
+  const float* S;
+  int n, E, k, kpad;
+  int32_t* idx;
+  float* gate;
+  int32_t* ec_row;    // [n, E] dense: dispatched row or -1
+  float* ec_gate;     // [n, E]
+  int32_t* row_token; // [E * kpad]
+  int32_t* load;
+  int32_t* counts;
+  int32_t* offsets;
+  int* err;
+};
+cudaError_t launch_select_ec(const SelectEcArgs& a, cudaStream_t s);
+
+struct EcFinishArgs {
+  const int32_t* ec_row;
+  const float* ec_gate;
+  int n, E;
+  int32_t* tok_row;
+  float* tok_gate;
+  int32_t* hist;        // optional [E+1]
+  float* aux;
+  const double* lse2;   // [lse_blocks] or NULL
+  int lse_blocks;
+  float z_coef;
+};
+cudaError_t launch_ec_finish(const EcFinishArgs& a, cudaStream_t s);
+
+struct TcAssignArgs {
+  const int32_t* idx;
+  const float* gate;
+  int n, E, K, cap, tok_blocks;
+  int32_t* blk_hist;
+  int32_t* blk_base;
+  int32_t* load;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* row_token;
+  int32_t* tok_row;
+  float* tok_gate;
+  uint8_t* drop;
+  float* aux;
+  const float* colsum;
+  int colsum_blocks;
+  const double* lse2;   // or NULL
+  int lse_blocks;
+  float lb_coef, z_coef;
+};
+cudaError_t launch_tc_assign(const TcAssignArgs& a, cudaStream_t s);
+
+struct GatherArgs {
+  const void* X;
+  const int32_t* row_token;
+  const int32_t* offsets;  // offsets[E] = rows in use
+  int E, d, elt_bytes;
+  long long max_rows;
+  void* X_perm;
+};
+cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s);
+
+struct CombineArgs {
+  const void* Y;
+  const int32_t* tok_row;
+  const float* tok_gate;
+  int n, d, slots, bf16, n_shared, n_pad;
+  long long shared_base;
+  long long max_rows;   // routed rows bound; larger slot entries are ignored
+  void* out;
+};
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
+
+struct FfnArgs {
+  const void* X;        // [n, d] (shared experts read it)
+  const void* X_perm;   // [rows, d]
+  const int32_t* offsets;
+  const void *W1, *W3, *W2, *sW1, *sW3, *sW2;
+  void* H;              // [rows, h]
+  void* Y;              // [rows, d]
+  int n, d, h, E, act, n_shared, n_pad;
+  long long rows_routed, shared_base, rows;
+  int* err;
+};
+moe_status run_ffn_bf16(const FfnArgs& a, cudaStream_t s);
+moe_status run_ffn_f32(const FfnArgs& a, cudaStream_t s);
+
+cudaError_t launch_bias_update(int n, int E, int K, const int32_t* load, float rate,
+                               float* bias, cudaStream_t s);
+
+}  // namespace moe

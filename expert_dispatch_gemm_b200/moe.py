@@ -1,0 +1,300 @@
+"""Thin Python binding of libmoe (include/moe.h) over torch device tensors.
+
+Argument marshalling only: every step of the layer runs in libmoe's CUDA
+kernels. torch allocates the device memory and supplies the stream. The
+library must have been built (``python -m expert_dispatch_gemm_b200.build``);
+if ``libmoe.so`` is missing every call raises, there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+from .workloads import Workload
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe.so")
+
+# enums and limits of include/moe.h
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, \
+    MOE_ERR_TIMEOUT = range(6)
+MOE_EXPERT_CHOICE, MOE_TOKEN_CHOICE = 0, 1
+MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID = 0, 1
+MOE_W_RAW, MOE_W_NORMALIZED = 0, 1
+MOE_ACT_RELU, MOE_ACT_GELU, MOE_ACT_SWIGLU = 0, 1, 2
+MOE_F32, MOE_BF16 = 0, 1
+MOE_ROW_ALIGN = 128
+MOE_AUX_LEN = 8
+AUX_NAMES = ["lb_loss", "z_loss", "maxvio", "dropped_assignments", "tokens_some_dropped",
+             "tokens_all_dropped", "tokens_no_expert", "reserved"]
+
+# every entry point include/moe.h declares
+API_SYMBOLS = ["moe_status_string", "moe_validate", "moe_sizes", "moe_workspace_size",
+               "moe_route", "moe_route_from_scores", "moe_dispatch", "moe_expert_ffn",
+               "moe_combine", "moe_layer_forward", "moe_bias_update", "moe_workspace_init",
+               "moe_read_error"]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+class MoeConfig(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_int), ("d", ctypes.c_int), ("E", ctypes.c_int),
+                ("h", ctypes.c_int), ("mode", ctypes.c_int), ("score", ctypes.c_int),
+                ("k", ctypes.c_int), ("capacity_factor", ctypes.c_float),
+                ("capacity", ctypes.c_int), ("n_groups", ctypes.c_int),
+                ("topk_groups", ctypes.c_int), ("group_topn", ctypes.c_int),
+                ("weights", ctypes.c_int), ("act", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("n_shared", ctypes.c_int), ("lb_coef", ctypes.c_float),
+                ("z_coef", ctypes.c_float)]
+
+
+class MoeRouteOut(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_void_p) for name in
+                ("idx", "gate", "load", "counts", "offsets", "row_token", "tok_row",
+                 "tok_gate", "drop", "scores", "logits", "lse", "aux", "ec_hist")]
+
+
+_LIB = None
+
+
+def lib() -> ctypes.CDLL:
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m expert_dispatch_gemm_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.c_void_p
+        cfgp = ctypes.POINTER(MoeConfig)
+        outp = ctypes.POINTER(MoeRouteOut)
+        L.moe_status_string.argtypes = [ctypes.c_int]
+        L.moe_status_string.restype = ctypes.c_char_p
+        L.moe_validate.argtypes = [cfgp]
+        ip = ctypes.POINTER(ctypes.c_int)
+        L.moe_sizes.argtypes = [cfgp, ip, ip, ip, ip, ip]
+        L.moe_workspace_size.argtypes = [cfgp, ctypes.POINTER(ctypes.c_size_t),
+                                         ctypes.POINTER(ctypes.c_size_t)]
+        L.moe_route.argtypes = [cfgp, P, P, P, P, outp, P, ctypes.c_size_t, P]
+        L.moe_route_from_scores.argtypes = [cfgp, P, P, outp, P, ctypes.c_size_t, P]
+        L.moe_dispatch.argtypes = [cfgp, P, outp, P, P]
+        L.moe_expert_ffn.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P,
+                                     ctypes.c_size_t, P]
+        L.moe_combine.argtypes = [cfgp, P, outp, P, P]
+        L.moe_layer_forward.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, outp, P,
+                                        ctypes.c_size_t, P]
+        L.moe_bias_update.argtypes = [cfgp, P, ctypes.c_float, P, P]
+        L.moe_workspace_init.argtypes = [P, P]
+        L.moe_read_error.argtypes = [P, P, ip]
+        for s in API_SYMBOLS[1:]:
+            getattr(L, s).restype = ctypes.c_int
+        _LIB = L
+    return _LIB
+
+
+def status_string(status: int) -> str:
+    return lib().moe_status_string(status).decode()
+
+
+def _check(status: int, what: str):
+    if status != MOE_OK:
+        raise MoeError(status, what)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+# ---------------------------------------------------------------------------
+# configs
+# ---------------------------------------------------------------------------
+
+def config(w: Workload, **override) -> MoeConfig:
+    """The C config of a workload (k / capacity derived by the library)."""
+    ec = w.mode == "ec"
+    c = MoeConfig(
+        n=w.n, d=w.d, E=w.E, h=w.h,
+        mode=MOE_EXPERT_CHOICE if ec else MOE_TOKEN_CHOICE,
+        score=MOE_SCORE_SIGMOID if w.score == "sigmoid" else MOE_SCORE_SOFTMAX,
+        k=0 if ec else w.K,
+        capacity_factor=w.c if ec else w.capacity_factor,
+        capacity=0 if (not ec and w.capacity_factor > 0) else -1,
+        n_groups=w.n_groups, topk_groups=w.topk_groups, group_topn=w.group_topn,
+        weights=MOE_W_NORMALIZED if w.weights == "normalized" else MOE_W_RAW,
+        act={"relu": MOE_ACT_RELU, "gelu": MOE_ACT_GELU, "swiglu": MOE_ACT_SWIGLU}[w.act],
+        dtype=MOE_F32 if w.dtype == "f32" else MOE_BF16,
+        n_shared=w.n_shared, lb_coef=w.lb_coef, z_coef=w.z_coef)
+    for k, v in override.items():
+        setattr(c, k, v)
+    return c
+
+
+@dataclass
+class Sizes:
+    k: int
+    capacity: int
+    slots: int
+    rows: int
+    shared_row_base: int
+    route_ws: int
+    layer_ws: int
+
+
+def sizes(cfg: MoeConfig) -> Sizes:
+    L = lib()
+    k, cap, slots, rows, sb = (ctypes.c_int() for _ in range(5))
+    _check(L.moe_sizes(ctypes.byref(cfg), ctypes.byref(k), ctypes.byref(cap),
+                       ctypes.byref(slots), ctypes.byref(rows), ctypes.byref(sb)), "moe_sizes")
+    r, l = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(L.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(r), ctypes.byref(l)),
+           "moe_workspace_size")
+    return Sizes(k.value, cap.value, slots.value, rows.value, sb.value, r.value, l.value)
+
+
+def validate(cfg: MoeConfig) -> int:
+    return lib().moe_validate(ctypes.byref(cfg))
+
+
+# ---------------------------------------------------------------------------
+# buffers (torch allocates; the library only fills them)
+# ---------------------------------------------------------------------------
+
+class RouteBuffers:
+    """Device tensors of one moe_route_out."""
+
+    def __init__(self, cfg: MoeConfig, device, logits: bool = True):
+        sz = sizes(cfg)
+        n, E = cfg.n, cfg.E
+        ec = cfg.mode == MOE_EXPERT_CHOICE
+        i32, f32 = torch.int32, torch.float32
+        shape = (E, sz.k) if ec else (n, sz.k)
+        self.idx = torch.empty(shape, dtype=i32, device=device)
+        self.gate = torch.empty(shape, dtype=f32, device=device)
+        self.load = torch.empty(E, dtype=i32, device=device)
+        self.counts = torch.empty(E, dtype=i32, device=device)
+        self.offsets = torch.empty(E + 1, dtype=i32, device=device)
+        self.row_token = torch.empty(max(sz.rows, 1), dtype=i32, device=device)
+        self.tok_row = torch.empty((n, sz.slots), dtype=i32, device=device)
+        self.tok_gate = torch.empty((n, sz.slots), dtype=f32, device=device)
+        self.drop = None if ec else torch.empty((n, sz.k), dtype=torch.uint8, device=device)
+        self.scores = torch.empty((n, E), dtype=f32, device=device)
+        self.logits = torch.empty((n, E), dtype=f32, device=device) if logits else None
+        self.lse = torch.empty(n, dtype=f32, device=device) if logits else None
+        self.aux = torch.empty(MOE_AUX_LEN, dtype=f32, device=device)
+        self.ec_hist = torch.empty(E + 1, dtype=i32, device=device) if ec else None
+        self.sizes = sz
+        self.c = MoeRouteOut(*[None if t is None else t.data_ptr() for t in (
+            self.idx, self.gate, self.load, self.counts, self.offsets, self.row_token,
+            self.tok_row, self.tok_gate, self.drop, self.scores, self.logits, self.lse,
+            self.aux, self.ec_hist)])
+
+    def aux_dict(self) -> dict:
+        return dict(zip(AUX_NAMES, self.aux.tolist()))
+
+
+def workspace(cfg: MoeConfig, device, layer: bool = True, stream=None) -> torch.Tensor:
+    """A zero-initialised, 256-byte aligned workspace (torch caching allocator)."""
+    sz = sizes(cfg)
+    nbytes = sz.layer_ws if layer else sz.route_ws
+    ws = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+    off = (-ws.data_ptr()) % 256
+    ws = ws[off:off + nbytes]
+    _check(lib().moe_workspace_init(_ptr(ws), _stream(stream)), "moe_workspace_init")
+    return ws
+
+
+# ---------------------------------------------------------------------------
+# entry points (same names as the C ABI)
+# ---------------------------------------------------------------------------
+
+def moe_route(cfg, X, Wg, logit_bias, sel_bias, route: RouteBuffers, ws, stream=None):
+    _check(lib().moe_route(ctypes.byref(cfg), _ptr(X), _ptr(Wg), _ptr(logit_bias),
+                           _ptr(sel_bias), ctypes.byref(route.c), _ptr(ws), ws.numel(),
+                           _stream(stream)), "moe_route")
+
+
+def moe_route_from_scores(cfg, S, sel_bias, route: RouteBuffers, ws, stream=None):
+    _check(lib().moe_route_from_scores(ctypes.byref(cfg), _ptr(S), _ptr(sel_bias),
+                                       ctypes.byref(route.c), _ptr(ws), ws.numel(),
+                                       _stream(stream)), "moe_route_from_scores")
+
+
+def moe_dispatch(cfg, X, route: RouteBuffers, X_perm, stream=None):
+    _check(lib().moe_dispatch(ctypes.byref(cfg), _ptr(X), ctypes.byref(route.c),
+                              _ptr(X_perm), _stream(stream)), "moe_dispatch")
+
+
+def moe_expert_ffn(cfg, X, X_perm, offsets, W1, W3, W2, sW1, sW3, sW2, H, Y_perm, ws,
+                   stream=None):
+    _check(lib().moe_expert_ffn(ctypes.byref(cfg), _ptr(X), _ptr(X_perm), _ptr(offsets),
+                                _ptr(W1), _ptr(W3), _ptr(W2), _ptr(sW1), _ptr(sW3), _ptr(sW2),
+                                _ptr(H), _ptr(Y_perm), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_expert_ffn")
+
+
+def moe_combine(cfg, Y_perm, route: RouteBuffers, out, stream=None):
+    _check(lib().moe_combine(ctypes.byref(cfg), _ptr(Y_perm), ctypes.byref(route.c),
+                             _ptr(out), _stream(stream)), "moe_combine")
+
+
+def moe_layer_forward(cfg, X, Wg, logit_bias, sel_bias, W1, W3, W2, sW1, sW3, sW2, out,
+                      route: RouteBuffers, ws, stream=None):
+    _check(lib().moe_layer_forward(ctypes.byref(cfg), _ptr(X), _ptr(Wg), _ptr(logit_bias),
+                                   _ptr(sel_bias), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(sW1),
+                                   _ptr(sW3), _ptr(sW2), _ptr(out), ctypes.byref(route.c),
+                                   _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_layer_forward")
+
+
+def moe_bias_update(cfg, load, rate: float, bias, stream=None):
+    _check(lib().moe_bias_update(ctypes.byref(cfg), _ptr(load), ctypes.c_float(rate),
+                                 _ptr(bias), _stream(stream)), "moe_bias_update")
+
+
+def moe_read_error(ws, stream=None):
+    detail = ctypes.c_int()
+    st = lib().moe_read_error(_ptr(ws), _stream(stream), ctypes.byref(detail))
+    return st, detail.value
+
+
+# ---------------------------------------------------------------------------
+# a whole layer with its buffers
+# ---------------------------------------------------------------------------
+
+class Layer:
+    """Inputs, weights, buffers and workspace of one workload on one device."""
+
+    def __init__(self, w: Workload, inputs: dict, device, **cfg_override):
+        self.w = w
+        self.cfg = config(w, **cfg_override)
+        self.device = device
+        self.inp = inputs
+        self.route = RouteBuffers(self.cfg, device)
+        self.ws = workspace(self.cfg, device, layer=True)
+        self.out = torch.empty((w.n, w.d), dtype=w.torch_dtype, device=device)
+        self.sizes = self.route.sizes
+
+    def forward(self, X=None, stream=None):
+        i = self.inp
+        moe_layer_forward(self.cfg, i["X"] if X is None else X, i["Wg"], i.get("logit_bias"),
+                          i.get("sel_bias"), i["W1"], i.get("W3"), i["W2"], i.get("sW1"),
+                          i.get("sW3"), i.get("sW2"), self.out, self.route, self.ws, stream)
+        return self.out

@@ -1,0 +1,268 @@
+/*
+ * libmoe: the forward hot path of a mixture-of-experts layer on one B200
+ * (sm_100a): route -> dispatch -> grouped expert FFN -> gate-scaled combine.
+ *
+ * Source pages of the operations (cited by title and section):
+ *   [TC-vs-EC]  "Token choice vs expert choice routing in MoE" (fanout.sh)
+ *   [EC-math]   "Expert choice routing" (aicassindra.com, transformer math)
+ *   [TC-card]   "MoE token-choice routing" (zenaique.com flashcard)
+ *   [Strat]     "How MoE routing strategies make large language models
+ *                efficient" (ehga.org)
+ *   [Guide]     "MoE routing strategies explained: top-k, expert choice,
+ *                sigmoid gating and dynamic routing (2026 guide)"
+ *                (ncijnetwork.com)
+ *
+ * Conventions shared by every entry point
+ *   - Every tensor argument is a DEVICE pointer to contiguous row-major
+ *     memory owned by the caller. The library never allocates or frees
+ *     memory, never synchronises the stream (except moe_read_error), and
+ *     never keeps a pointer after a call returns.
+ *   - All work is enqueued on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) in launch order; outputs are valid once the stream
+ *     reaches them.
+ *   - Arguments are validated on the host before any launch; on a non-OK
+ *     status nothing was enqueued. MOE_ERR_CUDA means a launch failed (the
+ *     stream may hold the launches enqueued before it).
+ *   - Device-side waits are bounded (about 4 s); a wait that gives up writes
+ *     an error code into the first 256 bytes of the workspace, and the
+ *     kernel returns. moe_read_error() reports it as MOE_ERR_TIMEOUT.
+ *   - Indices are int32, gates fp32. Activations X, expert weights, the
+ *     dispatched rows, the hidden activations and the expert outputs are
+ *     all of the config's dtype (fp32 or bf16); the router weight W_g, the
+ *     logits and the scores are always fp32.
+ *
+ * Dispatched-row layout ("dense per-expert batches", [EC-math] "The math:
+ * a gating matrix and top-k over tokens")
+ *   Expert e's rows form one contiguous segment of X_perm / H / Y_perm
+ *   starting at offsets[e]; every segment starts on a multiple of
+ *   MOE_ROW_ALIGN rows, so one 128-row GEMM tile never spans two experts.
+ *   The padding rows between segments are never read for results and are
+ *   left unwritten. Within a segment the rows are in token order (token
+ *   choice) or in the expert's selection order (expert choice). Shared
+ *   experts, when present, own n_pad = roundup(n, 128) rows each after the
+ *   routed rows, starting at row moe_shared_row_base().
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(MOE_BUILD)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ROW_ALIGN 128
+#define MOE_AUX_LEN 8
+#define MOE_MAX_EXPERTS 256
+#define MOE_MAX_TOPK 32
+#define MOE_MAX_SHARED 4
+#define MOE_EC_MAX_TOKENS 16384
+#define MOE_WS_ERROR_BYTES 256
+
+/* a cudaStream_t */
+typedef struct CUstream_st* moe_stream_t;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* a null required pointer, a bad size or mode */
+  MOE_ERR_UNSUPPORTED = 2, /* a valid shape this build has no kernel for */
+  MOE_ERR_WORKSPACE = 3,   /* workspace null or smaller than required */
+  MOE_ERR_CUDA = 4,        /* a CUDA call or launch failed */
+  MOE_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up */
+} moe_status;
+
+/* [EC-math] "The routing problem: who picks whom": the same score matrix,
+ * top-k along the expert axis (token choice) or the token axis (expert
+ * choice). */
+typedef enum { MOE_EXPERT_CHOICE = 0, MOE_TOKEN_CHOICE = 1 } moe_mode;
+
+/* softmax over experts ([EC-math] "The transposed selection") or an
+ * element-wise sigmoid ([Guide] "4. Sigmoid gating with aux-loss-free
+ * bias"). */
+typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score;
+
+/* Token-choice mixing weights: RAW = the score of the selected expert;
+ * NORMALIZED = the selected raw scores divided by their sum. For softmax
+ * scores NORMALIZED equals a softmax over the kept logits ([Guide] "1.
+ * Softmax top-k token choice"); for sigmoid scores it is [Guide] "4." */
+typedef enum { MOE_W_RAW = 0, MOE_W_NORMALIZED = 1 } moe_weights;
+
+/* expert FFN: Y = act(X W1^T) W2^T, or SwiGLU Y = (silu(X W1^T) * X W3^T) W2^T;
+ * GELU is the exact erf form. */
+typedef enum { MOE_ACT_RELU = 0, MOE_ACT_GELU = 1, MOE_ACT_SWIGLU = 2 } moe_act;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+typedef struct {
+  int n;  /* tokens in the routing group (the whole batch) */
+  int d;  /* model dim; multiple of 64 (bf16) or of 8 (fp32) */
+  int E;  /* routed experts, 1..MOE_MAX_EXPERTS */
+  int h;  /* expert hidden dim; multiple of 64 (bf16) or of 8 (fp32) */
+  moe_mode mode;
+  moe_score score;
+  /* token choice: experts per token (1..min(E, MOE_MAX_TOPK)).
+   * expert choice: tokens per expert; 0 derives k = floor(n c / E) with
+   * c = capacity_factor ([TC-vs-EC] "Who picks whom"). */
+  int k;
+  float capacity_factor;
+  /* token choice only: -1 = dropless; 0 = floor(n / E * capacity_factor)
+   * ([Guide] "2. Top-1 switch routing with a capacity factor"); > 0 =
+   * explicit rows per expert. Assignments past the buffer are dropped in
+   * token order ([TC-vs-EC] "Dropped tokens flow in opposite directions"). */
+  int capacity;
+  /* group-limited token choice ([Guide] "5. Group-limited and node-limited
+   * routing"): n_groups contiguous expert groups; a group's score is the
+   * fp32 sum of its group_topn largest selection keys; the topk_groups best
+   * groups are kept. n_groups <= 1 disables it. */
+  int n_groups, topk_groups, group_topn;
+  moe_weights weights;
+  moe_act act;
+  moe_dtype dtype;
+  /* always-on shared experts added with weight 1 ([Guide] "3. Shared plus
+   * routed experts"); 0..MOE_MAX_SHARED, same hidden size h. */
+  int n_shared;
+  /* aux-loss coefficients ([TC-vs-EC] "What each direction guarantees") */
+  float lb_coef, z_coef;
+} moe_config;
+
+/* aux[] slots (fp32) */
+enum {
+  MOE_AUX_LB = 0,          /* lb_coef * E * sum_e (load_e / (n K)) * mean_t S[t,e] (token choice) */
+  MOE_AUX_Z = 1,           /* z_coef * mean_t logsumexp(logits_t)^2 (moe_route only) */
+  MOE_AUX_MAXVIO = 2,      /* max_e load_e / (n K / E) - 1 (token choice) */
+  MOE_AUX_DROPPED = 3,     /* assignments dropped by the capacity */
+  MOE_AUX_TOKENS_SOME_DROPPED = 4,
+  MOE_AUX_TOKENS_ALL_DROPPED = 5,
+  MOE_AUX_TOKENS_NO_EXPERT = 6, /* expert choice: tokens no expert picked */
+  MOE_AUX_RESERVED = 7
+};
+
+/* Routing results. Every pointer is a caller-owned device buffer.
+ * slots = K (token choice) or E (expert choice); rows = moe_rows(). */
+typedef struct {
+  int32_t* idx;       /* required. TC: [n,K] expert ids in (key desc, id asc)
+                         order; EC: [E,k] token ids in (score desc, token asc)
+                         order ([EC-math] "The math": I = TopK(S^T, k)) */
+  float* gate;        /* required. same shape as idx: mixing weight (TC) or
+                         gate G = S[token, e] (EC) */
+  int32_t* load;      /* required. [E] selections per expert before capacity */
+  int32_t* counts;    /* required. [E] rows kept per expert */
+  int32_t* offsets;   /* required. [E+1] first dispatched row of each expert;
+                         offsets[E] = routed rows in use (padded) */
+  int32_t* row_token; /* required. [rows] source token of each dispatched row,
+                         -1 on padding rows (entries past offsets[E] unused) */
+  int32_t* tok_row;   /* required. [n, slots] dispatched rows feeding each
+                         token: the kept ones first (TC: selection order; EC:
+                         expert order), then -1 */
+  float* tok_gate;    /* required. [n, slots] the matching gates, 0 past the end */
+  uint8_t* drop;      /* TC required, EC ignored. [n,K] 1 = dropped by capacity */
+  float* scores;      /* required. [n,E] S = softmax or sigmoid of the logits */
+  float* logits;      /* optional. [n,E] logits (moe_route only) */
+  float* lse;         /* optional. [n] logsumexp of each logits row (moe_route only) */
+  float* aux;         /* required. [MOE_AUX_LEN], see the enum above */
+  int32_t* ec_hist;   /* optional (EC). [E+1] tokens picked by exactly j experts */
+} moe_route_out;
+
+/* Human-readable name of a status. Never NULL. */
+MOE_API const char* moe_status_string(moe_status s);
+
+/* Checks a config; MOE_OK if every entry point accepts it. */
+MOE_API moe_status moe_validate(const moe_config* cfg);
+
+/* Derived sizes: k_eff (EC tokens per expert or TC experts per token),
+ * capacity_eff (TC rows per expert, -1 dropless), slots (columns of
+ * tok_row), rows (rows of X_perm / H / Y_perm, shared rows included),
+ * shared_row_base (first shared-expert row). Any output pointer may be NULL. */
+MOE_API moe_status moe_sizes(const moe_config* cfg, int* k_eff, int* capacity_eff, int* slots,
+                     int* rows, int* shared_row_base);
+
+/* Workspace bytes for moe_route / moe_route_from_scores / moe_expert_ffn
+ * (route_bytes) and for moe_layer_forward (layer_bytes, which also holds
+ * X_perm, H and Y_perm). Any output pointer may be NULL. The workspace needs
+ * 256-byte alignment; only its first MOE_WS_ERROR_BYTES (the error word)
+ * must be zeroed once, by moe_workspace_init, before the first call. */
+MOE_API moe_status moe_workspace_size(const moe_config* cfg, size_t* route_bytes,
+                              size_t* layer_bytes);
+
+/* Router + selection + capacity + aux.
+ * X [n,d] (cfg dtype), Wg [d,E] fp32, logit_bias [E] fp32 or NULL (added to
+ * the logits: it moves both selection and weights), sel_bias [E] fp32 or
+ * NULL (token choice only: added to the scores for selection only, [Guide]
+ * "4. Sigmoid gating with aux-loss-free bias").
+ * [EC-math] "The transposed selection": S = softmax(X W_g); [TC-card]
+ * "Token-choice: the token picks experts": z_t = W h_t. */
+MOE_API moe_status moe_route(const moe_config* cfg, const void* X, const float* Wg,
+                     const float* logit_bias, const float* sel_bias, moe_route_out* out,
+                     void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Selection + capacity + aux from a caller-supplied score matrix S [n,E]
+ * fp32 (scores written to out->scores are copied from S). Given identical S,
+ * idx, load, counts, offsets, row_token, tok_row and drop are bit-identical
+ * to moe_route's. aux Z is 0 (no logits). */
+MOE_API moe_status moe_route_from_scores(const moe_config* cfg, const float* S,
+                                 const float* sel_bias, moe_route_out* out, void* ws,
+                                 size_t ws_bytes, moe_stream_t stream);
+
+/* Gather ([EC-math] "The math": X_in[e] = P[e] X with P = onehot(I), done as
+ * an index gather): X_perm[r] = X[row_token[r]] for every routed row
+ * r < offsets[E] with row_token[r] >= 0. X [n,d], X_perm [rows,d]. */
+MOE_API moe_status moe_dispatch(const moe_config* cfg, const void* X, const moe_route_out* route,
+                        void* X_perm, moe_stream_t stream);
+
+/* Grouped expert FFN over the dispatched layout ([EC-math] "The math":
+ * Expert_e(X_in[e]) on dense per-expert batches). Routed expert e reads rows
+ * [offsets[e], offsets[e+1]) of X_perm; shared expert s reads all n rows of
+ * X. W1, W3 [E,h,d]; W2 [E,d,h]; sW1, sW3 [n_shared,h,d]; sW2
+ * [n_shared,d,h]; W3 / sW3 only for SwiGLU (else NULL); shared pointers only
+ * when n_shared > 0. H [rows,h] receives the hidden activations, Y_perm
+ * [rows,d] the expert outputs (gate not applied). bf16 runs on the tcgen05
+ * tensor cores with fp32 accumulation; fp32 runs on FFMA. */
+MOE_API moe_status moe_expert_ffn(const moe_config* cfg, const void* X, const void* X_perm,
+                          const int32_t* offsets, const void* W1, const void* W3,
+                          const void* W2, const void* sW1, const void* sW3,
+                          const void* sW2, void* H, void* Y_perm, void* ws,
+                          size_t ws_bytes, moe_stream_t stream);
+
+/* Gate-scaled combine ([EC-math] "The math": Y[e] = G[e] * Expert_e(.),
+ * out = scatter_add(Y, I)), computed owner-side: out[t] = sum over t's
+ * tok_row entries of tok_gate * Y_perm[row] (+ each shared expert's row with
+ * weight 1), accumulated in fp32 in list order, stored in the cfg dtype. A
+ * token with no entry gets 0 (it passes on the residual, which the caller
+ * adds). out [n,d]. */
+MOE_API moe_status moe_combine(const moe_config* cfg, const void* Y_perm, const moe_route_out* route,
+                       void* out, moe_stream_t stream);
+
+/* The whole layer: moe_route, moe_dispatch, moe_expert_ffn, moe_combine on
+ * one stream, with X_perm / H / Y_perm inside the workspace (layer_bytes). */
+MOE_API moe_status moe_layer_forward(const moe_config* cfg, const void* X, const float* Wg,
+                             const float* logit_bias, const float* sel_bias,
+                             const void* W1, const void* W3, const void* W2,
+                             const void* sW1, const void* sW3, const void* sW2, void* out,
+                             moe_route_out* route, void* ws, size_t ws_bytes,
+                             moe_stream_t stream);
+
+/* Selection-bias update after a step ([Guide] "4. Sigmoid gating with
+ * aux-loss-free bias"): bias[e] -= rate * sign(load[e] - n K / E), in fp32;
+ * load [E] int32 (from moe_route_out.load), bias [E] fp32 updated in place. */
+MOE_API moe_status moe_bias_update(const moe_config* cfg, const int32_t* load, float rate,
+                           float* bias, moe_stream_t stream);
+
+/* Zeroes the error word at the start of `ws` (enqueued on `stream`). */
+MOE_API moe_status moe_workspace_init(void* ws, moe_stream_t stream);
+
+/* Synchronises `stream`, then reads and clears the error word at the start
+ * of `ws`: MOE_OK, MOE_ERR_TIMEOUT (a bounded wait gave up) or MOE_ERR_CUDA.
+ * If detail != NULL it receives the raw device code (0 = none). */
+MOE_API moe_status moe_read_error(void* ws, moe_stream_t stream, int* detail);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H */

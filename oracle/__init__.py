@@ -219,6 +219,26 @@ def ec_histogram(I, n: int):
 # the whole layer
 # --------------------------------------------------------------------------
 
+def spec_of(w) -> dict:
+    """Oracle spec of a workload description (any object with the fields
+    mode, n, E, c, K, capacity_factor, n_groups, topk_groups, group_topn,
+    weights, act, dtype, n_shared, score, lb_coef, z_coef). The quota and
+    the capacity are derived here, from the pages' formulas."""
+    if w.mode == "ec":
+        spec = dict(mode="ec", k=ec_quota(w.n, w.E, w.c))
+    else:
+        cap = capacity_of(w.n, w.E, w.capacity_factor) if w.capacity_factor > 0 else -1
+        spec = dict(mode="tc", K=w.K, capacity=cap, n_groups=w.n_groups,
+                    topk_groups=w.topk_groups, group_topn=w.group_topn,
+                    weights=W_NORMALIZED if w.weights == "normalized" else W_RAW)
+    spec.update(act={"relu": RELU, "gelu": GELU, "swiglu": SWIGLU}[w.act],
+                store=STORE_F32 if w.dtype == "f32" else STORE_BF16,
+                n_shared=w.n_shared,
+                score=SIGMOID if w.score == "sigmoid" else SOFTMAX,
+                lb_coef=w.lb_coef, z_coef=w.z_coef)
+    return spec
+
+
 def route(spec: dict, S, lse=None, sel_bias=None):
     """Selection + capacity + aux from a score matrix, per ``spec``:
 

@@ -52,13 +52,20 @@ static float round_store(double v, int store) {
 void orc_router(int n, int d, int E, const float* X, const float* Wg,
                 const float* logit_bias, int score, float* logits, float* S,
                 double* lse) {
+  double* acc = (double*)malloc(sizeof(double) * (size_t)E);
   for (int t = 0; t < n; ++t) {
+    /* each logit is the plain sum over i = 0..d-1 in increasing order; the
+     * expert index runs innermost only so that W_g is read row by row */
+    for (int e = 0; e < E; ++e) acc[e] = 0.0;
+    for (int i = 0; i < d; ++i) {
+      const double x = (double)X[(size_t)t * d + i];
+      const float* w = Wg + (size_t)i * E;
+      for (int e = 0; e < E; ++e) acc[e] += x * (double)w[e];
+    }
     for (int e = 0; e < E; ++e) {
-      double acc = 0.0;
-      for (int i = 0; i < d; ++i)
-        acc += (double)X[(size_t)t * d + i] * (double)Wg[(size_t)i * E + e];
-      if (logit_bias) acc += (double)logit_bias[e];
-      logits[(size_t)t * E + e] = (float)acc;
+      double v = acc[e];
+      if (logit_bias) v += (double)logit_bias[e];
+      logits[(size_t)t * E + e] = (float)v;
     }
     const float* L = logits + (size_t)t * E;
     double m = L[0];
@@ -76,6 +83,7 @@ void orc_router(int n, int d, int E, const float* X, const float* Wg,
       S[(size_t)t * E + e] = (float)s;
     }
   }
+  free(acc);
 }
 
 /* ------------------------------------------------------------------ */

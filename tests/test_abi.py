@@ -1,0 +1,179 @@
+"""Host-side checks of the C-ABI library (no GPU needed).
+
+The library loads, exports every entry point include/moe.h declares, its
+structs have the layout the header gives, and argument validation rejects
+bad configs, missing pointers and short workspaces before any launch.
+"""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+from expert_dispatch_gemm_b200 import build as build_mod
+from expert_dispatch_gemm_b200 import moe
+from expert_dispatch_gemm_b200 import workloads as wl
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build_mod.build()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^MOE_API\s+[^(]*?\b(moe_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported():
+    syms = declared_symbols()
+    assert len(syms) == 13
+    assert sorted(moe.API_SYMBOLS) == syms
+    L = ctypes.CDLL(moe.LIB_PATH)
+    for s in syms:
+        assert hasattr(L, s), s
+    out = subprocess.run(["nm", "-D", "--defined-only", moe.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = sorted(m for m in re.findall(r" T (moe_\w+)", out))
+    assert exported == syms  # nothing else leaks out of the library
+
+
+def test_struct_layout_matches_header():
+    src = r"""
+    #include <stdio.h>
+    #include <stddef.h>
+    #include "moe.h"
+    int main(void) {
+      printf("%zu %zu %zu %zu %zu\n", sizeof(moe_config), offsetof(moe_config, capacity_factor),
+             offsetof(moe_config, z_coef), sizeof(moe_route_out),
+             offsetof(moe_route_out, ec_hist));
+      return 0;
+    }
+    """
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "t.c")
+        exe = os.path.join(d, "t")
+        open(c, "w").write(src)
+        subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), c, "-o", exe])
+        vals = [int(x) for x in subprocess.check_output([exe]).split()]
+    assert vals == [ctypes.sizeof(moe.MoeConfig), moe.MoeConfig.capacity_factor.offset,
+                    moe.MoeConfig.z_coef.offset, ctypes.sizeof(moe.MoeRouteOut),
+                    moe.MoeRouteOut.ec_hist.offset]
+
+
+def test_status_strings():
+    for s in range(6):
+        assert moe.status_string(s)
+    assert moe.status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("w", wl.FULL + wl.SMALL, ids=lambda w: w.name)
+def test_derived_sizes_match_the_pages(w):
+    cfg = moe.config(w)
+    assert moe.validate(cfg) == moe.MOE_OK
+    sz = moe.sizes(cfg)
+    spec = oracle.spec_of(w)
+    if w.mode == "ec":
+        assert sz.k == spec["k"]
+        assert sz.slots == w.E
+        assert sz.rows == w.E * ((sz.k + 127) // 128 * 128) + w.n_shared * ((w.n + 127) // 128 * 128)
+    else:
+        assert sz.k == w.K
+        assert sz.capacity == spec["capacity"]
+        assert sz.slots == w.K
+    assert sz.route_ws > 0 and sz.layer_ws > sz.route_ws
+    assert sz.rows % 128 == 0
+
+
+def test_worked_quotas_through_the_library():
+    # 4,096 tokens, 64 experts, c = 2 -> 128 per expert; 1024, 8, 2 -> 256
+    for n, E, k in [(4096, 64, 128), (1024, 8, 256)]:
+        cfg = moe.config(wl.EC_BF16.replace(n=n, E=E))
+        assert moe.sizes(cfg).k == k
+    cfg = moe.config(wl.TC_TOP2_CAP)
+    assert moe.sizes(cfg).capacity == 1280
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("n", 0, moe.MOE_ERR_INVALID_ARG),
+    ("E", 0, moe.MOE_ERR_INVALID_ARG),
+    ("E", 257, moe.MOE_ERR_UNSUPPORTED),
+    ("d", 100, moe.MOE_ERR_UNSUPPORTED),       # bf16 needs d % 64 == 0
+    ("h", 96, moe.MOE_ERR_UNSUPPORTED),
+    ("k", 0, moe.MOE_ERR_INVALID_ARG),         # token choice needs K >= 1
+    ("k", 65, moe.MOE_ERR_INVALID_ARG),        # K > E
+    ("mode", 7, moe.MOE_ERR_INVALID_ARG),
+    ("act", 9, moe.MOE_ERR_INVALID_ARG),
+    ("n_groups", 3, moe.MOE_ERR_INVALID_ARG),  # 64 % 3 != 0
+    ("n_shared", 5, moe.MOE_ERR_INVALID_ARG),
+])
+def test_invalid_configs_rejected(field, value, status):
+    base = wl.TC_DROPLESS if field != "n_groups" else wl.TC_DROPLESS.replace(
+        n_groups=2, topk_groups=1, group_topn=2)
+    cfg = moe.config(base)
+    setattr(cfg, field, value)
+    assert moe.validate(cfg) == status
+
+
+def test_expert_choice_limits():
+    cfg = moe.config(wl.EC_BF16.replace(n=20000))
+    assert moe.validate(cfg) == moe.MOE_ERR_UNSUPPORTED  # one column must fit on chip
+    cfg = moe.config(wl.EC_BF16)
+    cfg.k = 5000  # more tokens per expert than tokens
+    assert moe.validate(cfg) == moe.MOE_ERR_INVALID_ARG
+
+
+def _fake(n):
+    """Non-null, 256-aligned fake device addresses: never dereferenced,
+    because validation fails before any launch."""
+    return ctypes.c_void_p(0x10000000 + 256 * n)
+
+
+def test_null_pointers_and_short_workspace_fail_before_launch():
+    L = moe.lib()
+    cfg = moe.config(wl.SMALL[2])
+    sz = moe.sizes(cfg)
+    out = moe.MoeRouteOut(*[0x20000000 + 4096 * i for i in range(14)])
+    # X missing
+    st = L.moe_route(ctypes.byref(cfg), None, _fake(1), None, None, ctypes.byref(out),
+                     _fake(2), sz.route_ws, None)
+    assert st == moe.MOE_ERR_INVALID_ARG
+    # required output missing (drop is required for token choice)
+    bad = moe.MoeRouteOut(*[0x20000000 + 4096 * i for i in range(14)])
+    bad.drop = None
+    st = L.moe_route(ctypes.byref(cfg), _fake(0), _fake(1), None, None, ctypes.byref(bad),
+                     _fake(2), sz.route_ws, None)
+    assert st == moe.MOE_ERR_INVALID_ARG
+    # workspace too small / misaligned / missing
+    st = L.moe_route(ctypes.byref(cfg), _fake(0), _fake(1), None, None, ctypes.byref(out),
+                     _fake(2), sz.route_ws - 1, None)
+    assert st == moe.MOE_ERR_WORKSPACE
+    st = L.moe_route(ctypes.byref(cfg), _fake(0), _fake(1), None, None, ctypes.byref(out),
+                     ctypes.c_void_p(0x10000010), sz.route_ws, None)
+    assert st == moe.MOE_ERR_WORKSPACE
+    st = L.moe_layer_forward(ctypes.byref(cfg), _fake(0), _fake(1), None, None, _fake(3),
+                             _fake(4), _fake(5), None, None, None, _fake(6), ctypes.byref(out),
+                             _fake(2), sz.route_ws, None)
+    assert st == moe.MOE_ERR_WORKSPACE  # the layer needs the larger workspace
+    # SwiGLU without W3
+    st = L.moe_expert_ffn(ctypes.byref(cfg), _fake(0), _fake(1), _fake(2), _fake(3), None,
+                          _fake(5), None, None, None, _fake(6), _fake(7), _fake(8), 4096, None)
+    assert st == moe.MOE_ERR_INVALID_ARG
+    # bias update is a token-choice operation
+    ec = moe.config(wl.EC_FP32)
+    st = L.moe_bias_update(ctypes.byref(ec), _fake(0), ctypes.c_float(0.001), _fake(1), None)
+    assert st == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_read_error(None, None, None) == moe.MOE_ERR_WORKSPACE
+
+
+def test_binding_refuses_to_run_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(moe, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(moe, "_LIB", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        moe.lib()

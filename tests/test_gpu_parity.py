@@ -1,0 +1,269 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.
+
+  * identical score matrices -> routing bit-exact (indices, counts, offsets,
+    dispatched-row order, drop masks, slot lists);
+  * end to end from X -> logits/scores within fp32 rounding, selections equal
+    except where the oracle's boundary gap is below 1e-5, layer outputs within
+    max-abs 1e-4 (fp32) or relative error 2e-2 (bf16);
+  * full-size workloads in the benchmark's launch configuration, checked on
+    sampled tokens the oracle computes one by one;
+  * edge cases: ties, a single expert, all experts, k = n, capacity 1, one
+    token, ragged tails.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from expert_dispatch_gemm_b200 import moe
+from expert_dispatch_gemm_b200 import workloads as wl
+from tests.gpu_common import (check_routing_exact, compare_out, expert_weights_from,
+                              explained_routing_diff, host, weights_rtol)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(autouse=True)
+def _cleanup():
+    yield
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def _sel_bias(w, seed, scale=0.05):
+    if w.score != "sigmoid":
+        return None
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(w.E, generator=g) * scale).float()
+
+
+def _ws_ok(ws):
+    st, detail = moe.moe_read_error(ws)
+    assert st == moe.MOE_OK, f"device error word {detail:#x}"
+
+
+# --------------------------------------------------------------------------
+# identical scores -> bit-exact routing
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("kind", ["random", "ties"])
+@pytest.mark.parametrize("w", wl.SMALL + wl.FULL, ids=lambda w: w.name)
+def test_route_from_scores_bit_exact(w, kind):
+    S = (wl.tie_heavy_scores(w.n, w.E, 5, seed=11) if kind == "ties"
+         else wl.random_scores(w.n, w.E, seed=12))
+    bias = _sel_bias(w, 13)
+    cfg = moe.config(w)
+    rb = moe.RouteBuffers(cfg, DEV, logits=False)
+    ws = moe.workspace(cfg, DEV, layer=False)
+    moe.moe_route_from_scores(cfg, S.to(DEV), None if bias is None else bias.to(DEV), rb, ws)
+    torch.cuda.synchronize()
+    spec = oracle.spec_of(w)
+    Sn = S.numpy()
+    bn = None if bias is None else bias.numpy()
+    r = oracle.route(spec, Sn, None, bn)
+    check_routing_exact(spec, r, rb, w.n, w.E, weights_rtol(spec))
+    np.testing.assert_array_equal(host(rb.scores), Sn)
+    aux = rb.aux.cpu().numpy()
+    if spec["mode"] == "tc":
+        lb, _, mv = oracle.aux(r["load"], Sn, np.zeros(w.n), spec["K"], w.lb_coef, w.z_coef)
+        np.testing.assert_allclose(aux[moe.AUX_NAMES.index("lb_loss")], lb, rtol=1e-5)
+        np.testing.assert_allclose(aux[2], mv, rtol=1e-6, atol=1e-7)
+        assert aux[3] == int((r["load"] - r["kept"]).sum())
+        assert aux[4] == int((r["drop"].sum(1) > 0).sum())
+        assert aux[5] == int((r["drop"].sum(1) == spec["K"]).sum())
+    else:
+        assert aux[6] == r["hist"][0]
+    _ws_ok(ws)
+
+
+# --------------------------------------------------------------------------
+# end to end from X (small sizes)
+# --------------------------------------------------------------------------
+
+def _oracle_from_x(w, inp):
+    spec = oracle.spec_of(w)
+    lb = inp.get("logit_bias")
+    logits, S, lse = oracle.router(host(inp["X"]), host(inp["Wg"]), host(lb), spec["score"])
+    sb = inp.get("sel_bias")
+    r = oracle.route(spec, S, lse, host(sb))
+    return spec, logits, S, lse, r
+
+
+@pytest.mark.parametrize("w", wl.SMALL, ids=lambda w: w.name)
+def test_route_from_x(w):
+    inp = wl.make_inputs(w, DEV, experts=False)
+    cfg = moe.config(w)
+    rb = moe.RouteBuffers(cfg, DEV)
+    ws = moe.workspace(cfg, DEV, layer=False)
+    moe.moe_route(cfg, inp["X"], inp["Wg"], inp["logit_bias"], inp["sel_bias"], rb, ws)
+    torch.cuda.synchronize()
+    spec, logits, S, lse, r = _oracle_from_x(w, inp)
+    np.testing.assert_allclose(host(rb.logits), logits, rtol=1e-5, atol=2e-5)
+    np.testing.assert_allclose(host(rb.scores), S, rtol=2e-5, atol=1e-7)
+    np.testing.assert_allclose(host(rb.lse), lse, rtol=1e-5, atol=2e-5)
+    bad = explained_routing_diff(spec, r, rb, S, host(inp.get("sel_bias")))
+    if not bad:
+        check_routing_exact(spec, r, rb, w.n, w.E, weights_rtol=5e-5)
+    aux = rb.aux.cpu().numpy()
+    z = w.z_coef * float(np.mean(lse ** 2))
+    np.testing.assert_allclose(aux[1], z, rtol=1e-4)
+    if spec["mode"] == "tc":
+        np.testing.assert_allclose(aux[0], r["lb"], rtol=1e-4)
+    _ws_ok(ws)
+
+
+@pytest.mark.parametrize("w", wl.SMALL, ids=lambda w: w.name)
+def test_layer_small(w):
+    inp = wl.make_inputs(w, DEV)
+    layer = moe.Layer(w, inp, DEV)
+    out = layer.forward()
+    torch.cuda.synchronize()
+    spec, logits, S, lse, r = _oracle_from_x(w, inp)
+    bad = explained_routing_diff(spec, r, layer.route, S, host(inp.get("sel_bias")))
+    ref = oracle.layer_forward(spec, host(inp["X"]), r, expert_weights_from(inp),
+                               expert_weights_from(inp, "s") if w.n_shared else None)
+    keep = np.array([t not in bad for t in range(w.n)])
+    assert keep.mean() > 0.99
+    compare_out(spec["store"], host(out)[keep], ref[keep], w.name)
+    _ws_ok(layer.ws)
+
+
+def test_stepwise_calls_equal_layer_forward():
+    w = wl.SMALL[3]
+    inp = wl.make_inputs(w, DEV)
+    layer = moe.Layer(w, inp, DEV)
+    ref = layer.forward().clone()
+    cfg = layer.cfg
+    sz = moe.sizes(cfg)
+    rb = moe.RouteBuffers(cfg, DEV)
+    ws = moe.workspace(cfg, DEV, layer=False)
+    dt = w.torch_dtype
+    X_perm = torch.empty((sz.rows, w.d), dtype=dt, device=DEV)
+    H = torch.empty((sz.rows, w.h), dtype=dt, device=DEV)
+    Y = torch.empty((sz.rows, w.d), dtype=dt, device=DEV)
+    out = torch.empty((w.n, w.d), dtype=dt, device=DEV)
+    moe.moe_route(cfg, inp["X"], inp["Wg"], None, None, rb, ws)
+    moe.moe_dispatch(cfg, inp["X"], rb, X_perm)
+    moe.moe_expert_ffn(cfg, inp["X"], X_perm, rb.offsets, inp["W1"], inp["W3"], inp["W2"],
+                       None, None, None, H, Y, ws)
+    moe.moe_combine(cfg, Y, rb, out)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    used = int(rb.offsets[-1])
+    rt = rb.row_token[:used]
+    real = rt >= 0
+    # the gather is an exact copy of the source rows
+    assert torch.equal(X_perm[:used][real], inp["X"][rt[real].long()])
+    _ws_ok(ws)
+
+
+# --------------------------------------------------------------------------
+# selection-bias steps ("4. Sigmoid gating with aux-loss-free bias")
+# --------------------------------------------------------------------------
+
+def test_bias_steps_bit_exact_on_identical_scores():
+    w = wl.SMALL[4]
+    cfg = moe.config(w)
+    spec = oracle.spec_of(w)
+    rb = moe.RouteBuffers(cfg, DEV, logits=False)
+    ws = moe.workspace(cfg, DEV, layer=False)
+    bias_g = torch.zeros(w.E, dtype=torch.float32, device=DEV)
+    bias_o = np.zeros(w.E, np.float32)
+    for step in range(6):
+        S = wl.random_scores(w.n, w.E, seed=100 + step) * 0.02 + 0.5  # narrow, bias matters
+        moe.moe_route_from_scores(cfg, S.to(DEV), bias_g, rb, ws)
+        r = oracle.route(spec, S.numpy(), None, bias_o)
+        moe.moe_bias_update(cfg, rb.load, w.bias_rate, bias_g)
+        bias_o = oracle.bias_update(r["load"], w.n, w.K, w.bias_rate, bias_o)
+        torch.cuda.synchronize()
+        check_routing_exact(spec, r, rb, w.n, w.E, weights_rtol(spec))
+        np.testing.assert_array_equal(bias_g.cpu().numpy(), bias_o)
+    assert np.abs(bias_o).max() > 0
+    _ws_ok(ws)
+
+
+# --------------------------------------------------------------------------
+# full-size workloads, sampled tokens
+# --------------------------------------------------------------------------
+
+def _sample_tokens(w, r, S, spec, count, seed):
+    rng = np.random.default_rng(seed)
+    picks = set(rng.choice(w.n, size=min(count, w.n), replace=False).tolist())
+    if spec["mode"] == "tc" and spec.get("capacity", -1) >= 0:
+        dropped = np.nonzero(r["drop"].any(1))[0]
+        picks |= set(dropped[:2].tolist())
+        picks |= set(np.nonzero(r["drop"].all(1))[0][:1].tolist())
+    if spec["mode"] == "ec":
+        per_token = np.bincount(r["I"].ravel(), minlength=w.n)
+        picks |= set(np.nonzero(per_token == 0)[0][:2].tolist())   # no expert at all
+        picks |= set(np.argsort(-per_token, kind="stable")[:1].tolist())  # most experts
+    return sorted(picks)
+
+
+@pytest.mark.parametrize("w", wl.FULL, ids=lambda w: w.name)
+def test_full_size_sampled(w):
+    inp = wl.make_inputs(w, DEV)
+    layer = moe.Layer(w, inp, DEV)
+    out = layer.forward()
+    torch.cuda.synchronize()
+    spec, logits, S, lse, r = _oracle_from_x(w, inp)
+    np.testing.assert_allclose(host(layer.route.logits), logits, rtol=1e-5, atol=5e-5)
+    bad = explained_routing_diff(spec, r, layer.route, S, host(inp.get("sel_bias")))
+    assert len(bad) <= max(4, w.n // 1000)
+    tokens = [t for t in _sample_tokens(w, r, S, spec, 8, seed=5) if t not in bad]
+    ref = oracle.layer_forward(spec, host(inp["X"]), r, expert_weights_from(inp),
+                               expert_weights_from(inp, "s") if w.n_shared else None,
+                               tokens=tokens)
+    got = host(out[torch.as_tensor(tokens, device=DEV)])
+    compare_out(spec["store"], got, ref, w.name)
+    if spec["mode"] == "tc" and spec.get("capacity", -1) >= 0:
+        dropped_all = [i for i, t in enumerate(tokens) if r["drop"][t].all()]
+        assert all((got[i] == 0).all() for i in dropped_all)  # residual only
+    _ws_ok(layer.ws)
+
+
+# --------------------------------------------------------------------------
+# edge cases
+# --------------------------------------------------------------------------
+
+EDGE = [
+    wl.TC_DROPLESS.replace(name="tc-all-experts-k8of8", n=200, d=128, E=8, K=8, h=128),
+    wl.TC_DROPLESS.replace(name="tc-single-expert", n=130, d=64, E=1, K=1, h=64),
+    wl.TC_DROPLESS.replace(name="tc-one-token", n=1, d=128, E=16, K=2, h=192),
+    wl.TC_TOP2_CAP.replace(name="tc-capacity-1", n=64, d=64, E=8, h=64,
+                           capacity_factor=0.125, logit_skew_var=0.0),
+    wl.EC_BF16.replace(name="ec-k-equals-n", n=256, d=128, E=4, h=128, c=4.0),
+    wl.EC_BF16.replace(name="ec-k1", n=300, d=64, E=16, h=64, c=0.06),
+    wl.EC_FP32.replace(name="ec-fp32-ragged", n=200, d=40, E=5, h=24, c=1.5),
+    wl.TC_SIGMOID_GROUPED.replace(name="tc-grouped-keep-all", n=260, d=128, E=32, h=64,
+                                  topk_groups=8, bias_steps=0),
+    wl.TC_SIGMOID_GROUPED.replace(name="tc-grouped-f32-relu", n=150, d=64, E=64, h=32,
+                                  dtype="f32", act="relu", n_shared=2, bias_steps=0),
+]
+
+
+@pytest.mark.parametrize("w", EDGE, ids=lambda w: w.name)
+def test_edge_cases(w):
+    test_layer_small(w)
+
+
+def test_capacity_one_all_equal_scores():
+    w = EDGE[3]
+    cfg = moe.config(w)
+    assert moe.sizes(cfg).capacity == 1
+    S = torch.full((w.n, w.E), 0.125)
+    rb = moe.RouteBuffers(cfg, DEV, logits=False)
+    ws = moe.workspace(cfg, DEV, layer=False)
+    moe.moe_route_from_scores(cfg, S.to(DEV), None, rb, ws)
+    torch.cuda.synchronize()
+    # ties -> experts 0 and 1 for every token; only token 0 fits
+    assert (rb.idx.cpu()[:, 0] == 0).all() and (rb.idx.cpu()[:, 1] == 1).all()
+    assert rb.counts.cpu().tolist() == [1, 1, 0, 0, 0, 0, 0, 0]
+    drop = rb.drop.cpu()
+    assert drop[0].sum() == 0 and (drop[1:] == 1).all()
+    spec = oracle.spec_of(w)
+    check_routing_exact(spec, oracle.route(spec, S.numpy()), rb, w.n, w.E, weights_rtol(spec))
