@@ -1,0 +1,427 @@
+"""Benchmark of the MoE routing-and-dispatch layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl reference]
+
+One step = one pass of the whole hot path over one batch: moe_route
+(router GEMM + scores + top-k + capacity scan) -> moe_dispatch (gather) ->
+moe_expert_ffn (tcgen05 grouped GEMM, up + down) -> moe_combine. Inputs and
+weights are resident in HBM before timing; L2 (126 MB) is flushed by writing
+a 256 MB buffer between timed steps, outside the timed events. Each stage is
+timed with CUDA events on the launching stream.
+
+Default workload: the expert-choice layer of the pages' worked example
+(4,096 tokens, d 1024, 64 experts, c = 2, GELU FFN 1024 -> 4096 -> 1024, bf16).
+
+Multi-GPU: the layer does not shard in this build ("replicas only"): each
+rank runs an independent replica, no collective touches the data path, and
+the timed region is the max over ranks.
+
+--impl reference times the CPU oracle as it stands (single thread) on the
+same workload, one bounded sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from expert_dispatch_gemm_b200 import workloads as wl  # noqa: E402
+
+METRIC = "MoE-layer fwd tokens/s on 1 B200; route/dispatch HBM GB/s; expert-GEMM TC util %"
+DEFAULT = wl.EC_BF16
+L2_FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p["hbm_gbs"], p["bf16_tflops"], p.get("bf16_tflops_sustained"), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work per stage (each input read once, each output written once)
+# ---------------------------------------------------------------------------
+
+def algorithmic(w: wl.Workload, k_eff: int, rows_gathered: int, expert_rows):
+    """bytes per stage and FLOPs of the grouped GEMM."""
+    xb = 4 if w.dtype == "f32" else 2
+    n, d, E, h = w.n, w.d, w.E, w.h
+    slots = E * k_eff if w.mode == "ec" else n * k_eff
+    route = n * d * xb + d * E * 4 + slots * 8
+    if w.mode == "ec":
+        route += 2 * n * E * 4  # the score matrix is written and read back (one global pass)
+    A = rows_gathered
+    dispatch = n * d * xb + A * d * xb
+    nproj = 3 if w.act == "swiglu" else 2
+    active = int(sum(1 for m in expert_rows if m > 0))
+    weights = (active + w.n_shared) * nproj * h * d * xb
+    rows_all = A + w.n_shared * n
+    ffn_bytes = weights + rows_all * d * xb + 2 * rows_all * h * xb + rows_all * d * xb
+    flops = 2.0 * rows_all * d * h * nproj
+    combine = A * d * xb + w.n_shared * n * d * xb + n * d * xb
+    return dict(route=route, dispatch=dispatch, ffn=ffn_bytes, combine=combine), flops
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def traffic_for(kernel_src: str, workload: str):
+    """DRAM bytes per launch of the grouped GEMM from the committed ncu summary,
+    or None when the device code changed since that capture (the hash covers
+    the source up to its host-side section) or the workload was not captured."""
+    path = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        dev_code = open(kernel_src, "rb").read().split(b"// host side")[0]
+        if rec.get("kernel_sha") != hashlib.sha256(dev_code).hexdigest()[:16]:
+            return None
+        return rec.get("bytes_per_launch", {}).get(workload)
+    except Exception:
+        return None
+
+
+def run_gpu(args, w: wl.Workload):
+    import torch.distributed as dist
+
+    from expert_dispatch_gemm_b200 import moe
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    inp = wl.make_inputs(w, dev)
+    cfg = moe.config(w)
+    sz = moe.sizes(cfg)
+    rb = moe.RouteBuffers(cfg, dev)
+    ws = moe.workspace(cfg, dev, layer=False)
+    dt = w.torch_dtype
+    X_perm = torch.empty((sz.rows, w.d), dtype=dt, device=dev)
+    H = torch.empty((sz.rows, w.h), dtype=dt, device=dev)
+    Y = torch.empty((sz.rows, w.d), dtype=dt, device=dev)
+    out = torch.empty((w.n, w.d), dtype=dt, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sb = inp["sel_bias"]
+
+    def step(ev=None, X=None):
+        X = inp["X"] if X is None else X
+        if ev: ev[0].record(stream)
+        moe.moe_route(cfg, X, inp["Wg"], inp["logit_bias"], sb, rb, ws, stream)
+        if ev: ev[1].record(stream)
+        moe.moe_dispatch(cfg, X, rb, X_perm, stream)
+        if ev: ev[2].record(stream)
+        moe.moe_expert_ffn(cfg, X, X_perm, rb.offsets, inp["W1"], inp["W3"], inp["W2"],
+                           inp.get("sW1"), inp.get("sW3"), inp.get("sW2"), H, Y, ws, stream)
+        if ev: ev[3].record(stream)
+        moe.moe_combine(cfg, Y, rb, out, stream)
+        if ev: ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    st, detail = moe.moe_read_error(ws)
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"device error after warm-up: {detail:#x}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        t_wall0 = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()  # outside the timed events: L2 starts cold every step
+            step(evs[i])
+        torch.cuda.synchronize(dev)
+        t_wall = time.perf_counter() - t_wall0
+    if world > 1:
+        dist.barrier()
+    stage_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)]
+                         for i in range(args.steps)])
+    step_ms = stage_ms.sum(1)
+    total_ms = float(step_ms.sum())
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    st, detail = moe.moe_read_error(ws)
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"device error in the timed region: {detail:#x}")
+
+    # ---- end to end: pinned host input -> layer -> host output, every step
+    Xh = inp["X"].cpu().pin_memory()
+    outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    Xd = torch.empty_like(inp["X"])
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    for i in range(max(1, args.warmup)):
+        Xd.copy_(Xh, non_blocking=True)
+        step(X=Xd)
+        outh.copy_(out, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_ev[i][0].record(stream)
+        Xd.copy_(Xh, non_blocking=True)
+        step(X=Xd)
+        outh.copy_(out, non_blocking=True)
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = float(np.sum([a.elapsed_time(b) for a, b in e2e_ev]))
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    # ---- algorithmic work and rooflines
+    counts = rb.counts.cpu().numpy()
+    rows_gathered = int(counts.sum())
+    k_eff = sz.k
+    bytes_, flops = algorithmic(w, k_eff, rows_gathered, counts)
+    hbm, tc_burst, tc_sust, src = peaks()
+    med = np.median(stage_ms, 0)
+    names = ["route", "dispatch", "ffn", "combine"]
+    stages = {}
+    for j, nm in enumerate(names):
+        gbs = bytes_[nm] / (med[j] * 1e-3) / 1e9
+        stages[nm] = {"ms": round(float(med[j]), 4), "GB/s": round(gbs, 1),
+                      "hbm_frac": round(gbs / hbm, 3)}
+    ffn_tflops = flops / (med[2] * 1e-3) / 1e12
+    stages["ffn"]["TFLOP/s"] = round(ffn_tflops, 1)
+    stages["ffn"]["tc_frac"] = round(ffn_tflops / tc_burst, 3)
+    # dominant kernel: the grouped GEMM (2 launches per step: up and down)
+    t_hbm = bytes_["ffn"] / (hbm * 1e9)
+    t_tc = flops / (tc_burst * 1e12)
+    per_launch_ms = float(med[2]) / 2.0
+    kernel_src = os.path.join(ROOT, "expert_dispatch_gemm_b200", "csrc", "gemm_tc.cu")
+    traffic = traffic_for(kernel_src, w.name) if w.dtype == "bf16" else None
+    if t_hbm >= t_tc:
+        ach = bytes_["ffn"] / 2 / (per_launch_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(ach / hbm, 3)}
+    else:
+        ach = flops / 2 / (per_launch_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": tc_burst,
+                "unit": "TFLOP/s", "frac": round(ach / tc_burst, 3)}
+    roof.update({"traffic": traffic, "kernel": "tc_grouped_gemm_kernel (up + down, avg)",
+                 "peak_source": src,
+                 "algorithmic_per_launch": bytes_["ffn"] / 2 if roof["bound"] == "hbm"
+                 else flops / 2})
+
+    tokens = w.n * world
+    value = tokens * args.steps / (total_ms * 1e-3)
+    e2e_value = tokens * args.steps / (e2e_ms * 1e-3)
+    launches_per_step = (4 if w.mode == "ec" else 4) + 1 + (2 if w.dtype == "bf16" else 2) + 1
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded N(0,1) activations, random-init weights)",
+        "config": {"workload": w.name, "tokens": w.n, "d_model": w.d, "experts": w.E,
+                   "hidden": w.h, "routing": ("expert-choice c=%g" % w.c if w.mode == "ec"
+                                              else "token-choice top-%d" % w.K),
+                   "parallelism": f"replicas{world}" if world > 1 else "single-gpu",
+                   "l2": "flushed between timed steps (256 MB write, outside the events)"},
+        "roofline": roof,
+        "stages": stages,
+        "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(Xh.numel() * Xh.element_size()),
+                "d2h_bytes_per_step": int(outh.numel() * outh.element_size())},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+        "wall_s_timed": round(t_wall, 4),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w, inp, budget_s=args.cpu_budget)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline leg and reference arm)
+# ---------------------------------------------------------------------------
+
+def _oracle_layer_sample(w, X, Wg, lb, sb, weights, sample_tokens):
+    """Routing of the whole batch, FFN + combine for `sample_tokens`."""
+    import oracle
+    spec = oracle.spec_of(w)
+    t0 = time.perf_counter()
+    _, S, lse = oracle.router(X, Wg, lb, spec["score"])
+    r = oracle.route(spec, S, lse, sb)
+    t_route = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.layer_forward(spec, X, r, weights, None, tokens=sample_tokens)
+    t_ffn = time.perf_counter() - t0
+    return t_route, t_ffn
+
+
+def _host_inputs(w, inp=None):
+    if inp is None:
+        inp = wl.make_inputs(w, "cuda" if torch.cuda.is_available() else "cpu")
+
+    def h(t):
+        return None if t is None else t.detach().float().cpu().numpy()
+    X, Wg, lb, sb = h(inp["X"]), h(inp["Wg"]), h(inp.get("logit_bias")), h(inp.get("sel_bias"))
+    W1, W3, W2 = inp["W1"], inp.get("W3"), inp["W2"]
+
+    def weights(e):
+        return h(W1[e]), None if W3 is None else h(W3[e]), h(W2[e])
+    return X, Wg, lb, sb, weights
+
+
+def cpu_baseline(w, inp=None, budget_s=20.0, sample=None):
+    X, Wg, lb, sb, weights = _host_inputs(w, inp)
+    rng = np.random.default_rng(0)
+    if sample is None:
+        # size the FFN sample from a short probe so the whole leg takes ~budget_s
+        probe = sorted(rng.choice(w.n, size=min(8, w.n), replace=False).tolist())
+        t_route, t_ffn = _oracle_layer_sample(w, X, Wg, lb, sb, weights, probe)
+        per_tok = t_ffn / len(probe)
+        sample = int(max(8, min(w.n, (budget_s - t_route) / max(per_tok, 1e-6))))
+    toks = sorted(rng.choice(w.n, size=min(sample, w.n), replace=False).tolist())
+    t_route, t_ffn = _oracle_layer_sample(w, X, Wg, lb, sb, weights, toks)
+    est = t_route + t_ffn / len(toks) * w.n
+    return {"value": round(w.n / est, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": (f"routing of all {w.n} tokens ({t_route:.2f} s) + expert FFN and "
+                       f"combine of {len(toks)} seeded tokens ({t_ffn:.2f} s), extrapolated "
+                       f"to {w.n} tokens; single-threaded C oracle, fp64")}
+
+
+def run_reference(args, w):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    X, Wg, lb, sb, weights = _host_inputs(w)
+    rng = np.random.default_rng(1)
+    sample = args.ref_sample
+    times = []
+    for i in range(args.warmup + args.steps):
+        toks = sorted(rng.choice(w.n, size=min(sample, w.n), replace=False).tolist())
+        t_route, t_ffn = _oracle_layer_sample(w, X, Wg, lb, sb, weights, toks)
+        if i >= args.warmup:
+            times.append(t_route + t_ffn / len(toks) * w.n)
+    est = float(np.mean(times))
+    value = w.n / est
+    res = {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(est * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+           "config": {"workload": w.name, "tokens": w.n, "d_model": w.d, "experts": w.E,
+                      "hidden": w.h},
+           "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": 1,
+                            "kind": "oracle",
+                            "sample": (f"per step: routing of all {w.n} tokens + expert FFN "
+                                       f"and combine of {sample} seeded tokens, extrapolated "
+                                       f"to {w.n}; single-threaded C oracle")},
+           "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT.name, choices=sorted(wl.BY_NAME))
+    ap.add_argument("--impl", default="libmoe", choices=["libmoe", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--ref-sample", type=int, default=48)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = wl.BY_NAME[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    main()

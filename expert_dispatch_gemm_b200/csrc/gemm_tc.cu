@@ -360,11 +360,12 @@ static EncodeTiledFn encode_fn() {
 }
 
 // 2-D bf16 row-major [rows, cols] map with a box of 64 columns x box_rows rows
-// and 128-byte swizzle. Out-of-range elements load as zero.
+// and 128-byte swizzle. Out-of-range elements (including a box taller than
+// the whole tensor) load as zero.
 static bool make_map(CUtensorMap* m, const void* ptr, long long rows, long long cols,
                      int box_rows) {
   EncodeTiledFn fn = encode_fn();
-  if (!fn || rows < box_rows || cols < kBK) return false;
+  if (!fn || rows < 1 || cols < kBK) return false;
   if ((reinterpret_cast<uintptr_t>(ptr) & 15) || ((cols * 2) & 15)) return false;
   const cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   const cuuint64_t gstride[1] = {(cuuint64_t)cols * 2};
