@@ -20,7 +20,7 @@ LIB = os.path.join(PKG, "libmoe.so")
 INCLUDE = os.path.join(ROOT, "include")
 
 SOURCES = ["api.cu", "router.cu", "assign.cu", "dispatch_combine.cu", "ffn_f32.cu",
-           "gemm_tc.cu"]
+           "gemm_tc.cu", "route_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -35,7 +35,8 @@ AUX_NAMES = ["lb_loss", "z_loss", "maxvio", "dropped_assignments", "tokens_some_
 API_SYMBOLS = ["moe_status_string", "moe_validate", "moe_sizes", "moe_workspace_size",
                "moe_route", "moe_route_from_scores", "moe_dispatch", "moe_expert_ffn",
                "moe_combine", "moe_layer_forward", "moe_bias_update", "moe_workspace_init",
-               "moe_read_error"]
+               "moe_read_error", "moe_route_noalloc"]
+MOE_ROUTE_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
 class MoeError(RuntimeError):
@@ -92,6 +93,7 @@ def lib() -> ctypes.CDLL:
         L.moe_bias_update.argtypes = [cfgp, P, ctypes.c_float, P, P]
         L.moe_workspace_init.argtypes = [P, P]
         L.moe_read_error.argtypes = [P, P, ip]
+        L.moe_route_noalloc.argtypes = [cfgp, P, P, P, P, outp, P]
         for s in API_SYMBOLS[1:]:
             getattr(L, s).restype = ctypes.c_int
         _LIB = L
@@ -267,6 +269,14 @@ def moe_layer_forward(cfg, X, Wg, logit_bias, sel_bias, W1, W3, W2, sW1, sW3, sW
 def moe_bias_update(cfg, load, rate: float, bias, stream=None):
     _check(lib().moe_bias_update(ctypes.byref(cfg), _ptr(load), ctypes.c_float(rate),
                                  _ptr(bias), _stream(stream)), "moe_bias_update")
+
+
+def moe_route_noalloc(cfg, X, Wg, logit_bias, sel_bias, route: RouteBuffers, stream=None):
+    """moe_route with the library's built-in scratch instead of a workspace,
+    for callers that cannot allocate device memory (see include/moe.h)."""
+    _check(lib().moe_route_noalloc(ctypes.byref(cfg), _ptr(X), _ptr(Wg), _ptr(logit_bias),
+                                   _ptr(sel_bias), ctypes.byref(route.c), _stream(stream)),
+           "moe_route_noalloc")
 
 
 def moe_read_error(ws, stream=None):

@@ -254,6 +254,25 @@ MOE_API moe_status moe_layer_forward(const moe_config* cfg, const void* X, const
 MOE_API moe_status moe_bias_update(const moe_config* cfg, const int32_t* load, float rate,
                            float* bias, moe_stream_t stream);
 
+/* moe_route without a workspace, for callers that cannot allocate device
+ * memory when they route (an application whose device memory budget is fixed
+ * at start-up, or a plugin inside a framework that owns all device
+ * allocations). The pages have no counterpart: this is a memory-management
+ * variant of moe_route, with identical arguments minus the workspace and
+ * identical results. Its scratch is a library-owned static device array of
+ * MOE_ROUTE_NOALLOC_SCRATCH_BYTES, held on every GPU that loads the library
+ * until the process exits; configs needing more routing scratch than that
+ * (moe_workspace_size's route_bytes) return MOE_ERR_WORKSPACE before
+ * anything is enqueued. It calls no cudaMalloc, cudaFree or other allocating
+ * routine. The first call on a device looks up the array's device address
+ * and zeroes its error word (a synchronous cudaMemset); make that first call
+ * before any stream capture. Every call shares the one array, so calls that
+ * overlap on the GPU (on different streams or threads) race. */
+#define MOE_ROUTE_NOALLOC_SCRATCH_BYTES (4u << 20)
+MOE_API moe_status moe_route_noalloc(const moe_config* cfg, const void* X, const float* Wg,
+                                     const float* logit_bias, const float* sel_bias,
+                                     moe_route_out* out, moe_stream_t stream);
+
 /* Zeroes the error word at the start of `ws` (enqueued on `stream`). */
 MOE_API moe_status moe_workspace_init(void* ws, moe_stream_t stream);
 
