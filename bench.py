@@ -290,7 +290,9 @@ def run_gpu(args, w: wl.Workload):
     tokens = w.n * world
     value = tokens * args.steps / (total_ms * 1e-3)
     e2e_value = tokens * args.steps / (e2e_ms * 1e-3)
-    launches_per_step = (4 if w.mode == "ec" else 4) + 1 + (2 if w.dtype == "bf16" else 2) + 1
+    # route: router + select_ec + ec_finish (EC) or router + hist + scan + scatter (TC);
+    # dispatch: gather; expert FFN: up + down; combine
+    launches_per_step = (3 if w.mode == "ec" else 4) + 1 + 2 + 1
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,

@@ -87,7 +87,8 @@ moe_status derive(const moe_config* c, Derived* d) {
   d->shared_base = d->rows_routed;
   d->rows = d->rows_routed + (long long)c->n_shared * d->n_pad;
   if (d->rows > (1LL << 30)) return MOE_ERR_UNSUPPORTED;
-  d->router_blocks = ceil_div(n, 32);  // covers every router tile height (>= 32 rows)
+  // covers every router tile height and the score-only selection blocks
+  d->router_blocks = ceil_div(n, kRouterMinBlockRows);
   d->tok_blocks = ceil_div(n, kTokBlock);
   return MOE_OK;
 }
@@ -171,6 +172,11 @@ static moe_status finish_route(const moe_config* c, const Derived& dv, const WsL
     a.counts = o->counts;
     a.offsets = o->offsets;
     a.err = err;
+    a.hist = o->ec_hist;
+    a.aux = o->aux;
+    a.lse2 = have_lse ? at<double>(ws, w.lse2) : nullptr;
+    a.lse_blocks = colsum_blocks;
+    a.z_coef = c->z_coef;
     MOE_CU(launch_select_ec(a, s));
     EcFinishArgs f{};
     f.ec_row = a.ec_row;
@@ -242,8 +248,8 @@ static moe_status route_impl(const moe_config* c, const Derived& dv, const WsLay
   r.colsum = at<float>(ws, w.colsum);
   r.lse2 = at<double>(ws, w.lse2);
   MOE_CU(launch_router(r, s));
-  return finish_route(c, dv, w, o, ws, o->scores, ceil_div(c->n, router_block_rows(c->E)),
-                      true, s);
+  return finish_route(c, dv, w, o, ws, o->scores,
+                      ceil_div(c->n, router_block_rows(c->E, c->n)), true, s);
 }
 
 static moe_status ffn_impl(const moe_config* c, const Derived& dv, const void* X,
@@ -279,6 +285,10 @@ static moe_status ffn_impl(const moe_config* c, const Derived& dv, const void* X
   f.shared_base = dv.shared_base;
   f.rows = dv.rows;
   f.err = err;
+  // CTA pairs compute two 128-row blocks of one expert per tile: worth it when
+  // experts own several blocks (token choice, or expert choice with k > 128);
+  // with one block per expert half of a pair's MMA work would be padding
+  f.pair = c->mode == MOE_TOKEN_CHOICE || dv.kpad >= 2 * kRowAlign;
   return c->dtype == MOE_BF16 ? run_ffn_bf16(f, s) : run_ffn_f32(f, s);
 }
 

@@ -58,9 +58,15 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
     for (int i = tid; i < 256; i += kEcThreads) hist[i] = 0;
     __syncthreads();
     const uint32_t prefix = s_prefix, mask = s_mask;
-    for (int t = tid; t < n; t += kEcThreads) {
-      const uint32_t u = key[t];
-      if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1);
+    // keys share their leading digits, so aggregate per warp: one shared
+    // atomic per distinct digit instead of one per key
+    for (int t0 = 0; t0 < n; t0 += kEcThreads) {
+      const int t = t0 + tid;
+      const uint32_t u = t < n ? key[t] : 0u;
+      const bool cand = t < n && (u & mask) == prefix;
+      const int digit = cand ? (int)((u >> shift) & 255u) : 256 + lane;  // unique when idle
+      const unsigned peers = __match_any_sync(0xffffffffu, digit);
+      if (cand && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
     }
     __syncthreads();
     if (warp == 0) {
@@ -168,6 +174,19 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
     a.offsets[e] = e * a.kpad;
     if (e == E - 1) a.offsets[E] = E * a.kpad;
   }
+  if (e == 0) {
+    // zero what the finish kernel accumulates into, and the fixed aux slots
+    if (a.hist)
+      for (int i = tid; i <= E; i += kEcThreads) a.hist[i] = 0;
+    if (tid < MOE_AUX_LEN && tid != MOE_AUX_Z) a.aux[tid] = 0.0f;
+    if (warp == 1) {
+      double s = 0.0;
+      if (a.lse2)
+        for (int b = lane; b < a.lse_blocks; b += 32) s += a.lse2[b];
+      for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0) a.aux[MOE_AUX_Z] = (float)((double)a.z_coef * s / (double)n);
+    }
+  }
 }
 
 cudaError_t launch_select_ec(const SelectEcArgs& a, cudaStream_t s) {
@@ -226,24 +245,8 @@ __global__ void __launch_bounds__(256) ec_finish_kernel(EcFinishArgs a) {
   if (threadIdx.x == 0 && none_s) atomicAdd(&a.aux[MOE_AUX_TOKENS_NO_EXPERT], (float)none_s);
 }
 
-// zero the accumulators the EC finish kernel adds into and set fixed aux
-__global__ void ec_aux_init_kernel(EcFinishArgs a) {
-  for (int i = threadIdx.x; i <= a.E; i += blockDim.x)
-    if (a.hist) a.hist[i] = 0;
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < MOE_AUX_LEN; ++i) a.aux[i] = 0.0f;
-    if (a.lse2) {
-      double s = 0.0;
-      for (int b = 0; b < a.lse_blocks; ++b) s += a.lse2[b];
-      a.aux[MOE_AUX_Z] = (float)((double)a.z_coef * s / (double)a.n);
-    }
-  }
-}
-
+// (select_ec_kernel's block 0 has zeroed hist and the aux slots)
 cudaError_t launch_ec_finish(const EcFinishArgs& a, cudaStream_t s) {
-  ec_aux_init_kernel<<<1, 256, 0, s>>>(a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
   ec_finish_kernel<<<ceil_div(a.n, 8), 256, 0, s>>>(a);
   return cudaGetLastError();
 }

@@ -337,6 +337,326 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// CTA-pair variant (cta_group::2). A cluster of two CTAs on one TPC computes a
+// 256 x 256 tile: each CTA loads 128 rows of A and one half (128 rows) of the
+// 256-row B tile into its own shared memory, the pair leader issues
+// tcgen05.mma.cta_group::2 (M=256, N=256, K=16), and each CTA's TMEM receives
+// its own 128 rows. Per CTA that is 32 KB of operands per 64-deep k-block
+// instead of 48 KB, and the ring holds six stages instead of four. Both CTAs'
+// TMA loads complete on the leader's stage barrier; MMA commits arrive on
+// both CTAs' barriers (multicast commit); both epilogues release the
+// accumulator on the leader's barrier. A pair tile takes two consecutive
+// 128-row blocks of one expert's segment; when the expert has an odd number
+// of blocks the second CTA recomputes the first block and stores nothing.
+// For SwiGLU the leader's B half is 128 rows of W1 and the peer's the same
+// rows of W3, so TMEM columns 0..127 / 128..255 hold the two projections.
+// ---------------------------------------------------------------------------
+constexpr int kPStages = 6;
+constexpr int kPABytes = kBM * kBK * 2;           // 16 KB: this CTA's 128 rows of A
+constexpr int kPBBytes = (kBN / 2) * kBK * 2;     // 16 KB: this CTA's half of B
+constexpr int kPStageBytes = kPABytes + kPBBytes; // 32 KB
+
+struct PairState {
+  uint64_t full[kPStages];   // leader: both CTAs' bytes of a stage have landed
+  uint64_t empty[kPStages];  // each CTA: its copy of a stage may be refilled
+  uint64_t tfull[2];         // each CTA: accumulator ready to read
+  uint64_t tempty[2];        // leader: both epilogues are done with an accumulator
+  uint64_t drain;
+  uint32_t tmem_base;
+  volatile int abort_flag;
+  int offs[MOE_MAX_EXPERTS + 1];
+  int pprefix[MOE_MAX_EXPERTS + 1];  // pair tiles of the experts before e
+};
+
+template <bool CLUSTER_ACQUIRE>
+__device__ __forceinline__ bool bounded_wait_pair(uint64_t* bar, uint32_t parity, PairState* st,
+                                                  int* err, int code) {
+  auto probe = [&]() {
+    return CLUSTER_ACQUIRE ? sm100::mbar_try_wait_cluster(bar, parity)
+                           : sm100::mbar_try_wait(bar, parity);
+  };
+  if (probe()) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (probe()) return true;
+    if ((it & 63u) == 0) {
+      if (st->abort_flag) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        st->abort_flag = 1;
+        report_error(err, code);
+        return false;
+      }
+    }
+  }
+}
+
+struct PairCoord {
+  int a_sel, a_row, b_sel, b_row;
+  long long out_row;
+  int col0;
+  bool valid;
+};
+
+template <int ACT>
+__device__ __forceinline__ PairCoord decode_pair(int tile, const TcGemmParams& p,
+                                                 const int* offs, const int* pprefix, int Pr,
+                                                 uint32_t rank) {
+  constexpr int BNO = ACT == ACT_SWIGLU ? kBN / 2 : kBN;
+  PairCoord c;
+  const int pt = tile / p.nt_tiles, nt = tile % p.nt_tiles;
+  int b_base;
+  if (pt < Pr) {
+    int lo = 0, hi = p.E - 1;  // largest e with pprefix[e] <= pt
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pprefix[mid] <= pt) lo = mid; else hi = mid - 1;
+    }
+    const int j = pt - pprefix[lo];
+    const int cnt = (offs[lo + 1] - offs[lo]) / kBM;
+    int mloc = 2 * j + (int)rank;
+    c.valid = mloc < cnt;
+    if (!c.valid) mloc = 2 * j;
+    const int row = offs[lo] + mloc * kBM;
+    c.a_sel = 0;
+    c.a_row = row;
+    c.out_row = row;
+    c.b_sel = 0;
+    b_base = lo * p.b_rows_per_expert;
+  } else {
+    const int spp = (p.shared_tiles_per + 1) / 2;
+    const int q = pt - Pr;
+    const int s = q / spp, jj = q % spp;
+    int lm = 2 * jj + (int)rank;
+    c.valid = lm < p.shared_tiles_per;
+    if (!c.valid) lm = 2 * jj;
+    c.a_sel = 1;
+    c.a_row = (int)(p.a1_row_base + s * p.a1_row_stride + (long long)lm * kBM);
+    c.out_row = p.out_shared_base + s * p.n_pad + (long long)lm * kBM;
+    c.b_sel = 1;
+    b_base = s * p.b_rows_per_expert;
+  }
+  c.col0 = nt * BNO;
+  c.b_row = b_base + c.col0 + (ACT == ACT_SWIGLU ? 0 : (int)rank * (kBN / 2));
+  return c;
+}
+
+template <int ACT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    tc_grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0,
+                                const __grid_constant__ CUtensorMap tmA1,
+                                const __grid_constant__ CUtensorMap tmB0,
+                                const __grid_constant__ CUtensorMap tmB0g,
+                                const __grid_constant__ CUtensorMap tmB1,
+                                const __grid_constant__ CUtensorMap tmB1g,
+                                const TcGemmParams p) {
+  constexpr bool SWIGLU = ACT == ACT_SWIGLU;
+  extern __shared__ __align__(1024) unsigned char gsm[];
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(gsm) + 1023) & ~uintptr_t(1023));
+  PairState* st = reinterpret_cast<PairState*>(base + kPStages * kPStageBytes);
+  auto sA = [&](int s) { return base + s * kPStageBytes; };
+  auto sB = [&](int s) { return base + s * kPStageBytes + kPABytes; };
+
+  const uint32_t rank = sm100::cluster_ctarank();
+  const bool leader = rank == 0;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i <= p.E; i += kGemmThreads) st->offs[i] = p.offsets[i];
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int e = 0; e < p.E; ++e) {
+      st->pprefix[e] = run;
+      const int cnt = max(st->offs[e + 1] - st->offs[e], 0) / kBM;
+      run += (cnt + 1) / 2;
+    }
+    st->pprefix[p.E] = run;
+    for (int s = 0; s < kPStages; ++s) {
+      sm100::mbar_init(&st->full[s], 1);
+      sm100::mbar_init(&st->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      sm100::mbar_init(&st->tfull[a], 1);
+      sm100::mbar_init(&st->tempty[a], 256);
+    }
+    sm100::mbar_init(&st->drain, 1);
+    st->abort_flag = 0;
+    sm100::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    sm100::tma_prefetch_desc(&tmA0);
+    sm100::tma_prefetch_desc(&tmB0);
+    if (SWIGLU) sm100::tma_prefetch_desc(&tmB0g);
+  }
+  if (warp == 1) {
+    sm100::tmem_alloc_pair(&st->tmem_base, kTmemCols);
+    sm100::tmem_relinquish_pair();
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::cluster_sync();  // both CTAs' barriers exist before any remote arrive
+  sm100::tc_fence_after();
+  const uint32_t tmem = st->tmem_base;
+
+  const int Pr = min(st->pprefix[p.E], p.max_routed_tiles);
+  const int spp = (p.shared_tiles_per + 1) / 2;
+  const int total = (Pr + p.n_shared * spp) * p.nt_tiles;
+  const int KB = p.K / kBK;
+  const int pair_id = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int tile = pair_id; ok && tile < total; tile += num_pairs) {
+        const PairCoord c = decode_pair<ACT>(tile, p, st->offs, st->pprefix, Pr, rank);
+        const CUtensorMap* ma = c.a_sel ? &tmA1 : &tmA0;
+        const CUtensorMap* mb;
+        if (SWIGLU)
+          mb = leader ? (c.b_sel ? &tmB1 : &tmB0) : (c.b_sel ? &tmB1g : &tmB0g);
+        else
+          mb = c.b_sel ? &tmB1 : &tmB0;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!bounded_wait_pair<false>(&st->empty[stage], phase ^ 1u, st, p.err,
+                                        kErrGemmTimeout | 0x41)) {
+            ok = false;
+            break;
+          }
+          const uint32_t full_leader = sm100::mapa_shared(sm100::smem_addr(&st->full[stage]), 0);
+          if (leader) sm100::mbar_arrive_expect_tx(&st->full[stage], 2 * kPStageBytes);
+          sm100::tma_load_2d_pair(sA(stage), ma, full_leader, kb * kBK, c.a_row);
+          sm100::tma_load_2d_pair(sB(stage), mb, full_leader, kb * kBK, c.b_row);
+          ++issued;
+          if (++stage == kPStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok && leader) {
+        // wait (bounded) until the copies of the outstanding stages have landed
+        int s = stage;
+        uint32_t ph = phase;
+        const int pending = issued < kPStages ? issued : kPStages;
+        for (int i = 0; i < pending; ++i) {
+          if (--s < 0) {
+            s = kPStages - 1;
+            ph ^= 1u;
+          }
+          const uint64_t t0 = global_timer_ns();
+          while (!sm100::mbar_try_wait(&st->full[s], ph) &&
+                 global_timer_ns() - t0 < kWaitLimitNs) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = sm100::idesc_bf16_f32(2 * kBM, kBN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int tile = pair_id; ok && tile < total; tile += num_pairs, ++local) {
+        const int acc = local & 1;
+        const uint32_t acc_phase = (uint32_t)(local >> 1) & 1u;
+        if (!bounded_wait_pair<true>(&st->tempty[acc], acc_phase ^ 1u, st, p.err,
+                                     kErrGemmTimeout | 0x52)) {
+          ok = false;
+          break;
+        }
+        sm100::tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(acc * kBN);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!bounded_wait_pair<false>(&st->full[stage], phase, st, p.err,
+                                        kErrGemmTimeout | 0x53)) {
+            ok = false;
+            break;
+          }
+          sm100::tc_fence_after();
+          const uint64_t adesc = sm100::sw128_kmajor_desc(sm100::smem_addr(sA(stage)));
+          const uint64_t bdesc = sm100::sw128_kmajor_desc(sm100::smem_addr(sB(stage)));
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k)
+            sm100::umma_f16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0);
+          sm100::umma_commit_pair_mc(&st->empty[stage], 0x3);
+          if (++stage == kPStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        sm100::umma_commit_pair_mc(&st->tfull[acc], 0x3);
+      }
+      sm100::umma_commit_pair_mc(&st->drain, 0x1);
+      const uint64_t t0 = global_timer_ns();
+      while (!sm100::mbar_try_wait(&st->drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    const int row_in_tile = q * 32 + lane;
+    constexpr int BNO = SWIGLU ? kBN / 2 : kBN;
+    int local = 0;
+    for (int tile = pair_id; tile < total; tile += num_pairs, ++local) {
+      const int acc = local & 1;
+      const uint32_t acc_phase = (uint32_t)(local >> 1) & 1u;
+      if (!bounded_wait_pair<true>(&st->tfull[acc], acc_phase, st, p.err,
+                                   kErrGemmTimeout | 0x64))
+        break;
+      sm100::tc_fence_after();
+      const PairCoord c = decode_pair<ACT>(tile, p, st->offs, st->pprefix, Pr, rank);
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN);
+      __nv_bfloat16* orow = p.out + (size_t)(c.out_row + row_in_tile) * p.n_out;
+      if (c.valid) {
+#pragma unroll 1
+        for (int cc = 0; cc < BNO; cc += 32) {
+          if (c.col0 + cc >= p.n_out) break;
+          uint32_t v[32];
+          sm100::tmem_ld_32x32b_x32(tbase + cc, v);
+          float f[32];
+          if (SWIGLU) {
+            uint32_t g[32];
+            sm100::tmem_ld_32x32b_x32(tbase + BNO + cc, g);
+            sm100::tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float a = __uint_as_float(v[i]);
+              const float b = __uint_as_float(g[i]);
+              f[i] = a * __frcp_rn(1.0f + __expf(-a)) * b;
+            }
+          } else {
+            sm100::tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) f[i] = act_fn<ACT>(__uint_as_float(v[i]));
+          }
+          uint4* dst = reinterpret_cast<uint4*>(orow + c.col0 + cc);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint4 o;
+            o.x = pack_bf16x2(f[8 * j + 0], f[8 * j + 1]);
+            o.y = pack_bf16x2(f[8 * j + 2], f[8 * j + 3]);
+            o.z = pack_bf16x2(f[8 * j + 4], f[8 * j + 5]);
+            o.w = pack_bf16x2(f[8 * j + 6], f[8 * j + 7]);
+            dst[j] = o;
+          }
+        }
+      }
+      sm100::tc_fence_before();
+      sm100::mbar_arrive_cluster(sm100::mapa_shared(sm100::smem_addr(&st->tempty[acc]), 0));
+    }
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::cluster_sync();  // no CTA leaves while its peer may still signal it
+  if (warp == 1) {
+    sm100::tc_fence_after();
+    sm100::tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -377,21 +697,33 @@ static bool make_map(CUtensorMap* m, const void* ptr, long long rows, long long 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-static size_t gemm_smem_bytes() {
-  return (size_t)kStages * kStageBytes + sizeof(SharedState) + 1024;
+static size_t gemm_smem_bytes(bool pair) {
+  return pair ? (size_t)kPStages * kPStageBytes + sizeof(PairState) + 1024
+              : (size_t)kStages * kStageBytes + sizeof(SharedState) + 1024;
 }
 
+struct Maps {
+  CUtensorMap a0, a1, b0, b0g, b1, b1g;
+};
+
+// grid: CTAs for the single-CTA kernel, CTA pairs for the pair kernel
 template <int ACT>
-static cudaError_t launch_tc(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0,
-                             const CUtensorMap& b0g, const CUtensorMap& b1,
-                             const CUtensorMap& b1g, const TcGemmParams& p, int grid,
-                             cudaStream_t s) {
-  auto kern = tc_grouped_gemm_kernel<ACT>;
-  const size_t bytes = gemm_smem_bytes();
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-  if (e != cudaSuccess) return e;
-  kern<<<grid, kGemmThreads, bytes, s>>>(a0, a1, b0, b0g, b1, b1g, p);
+static cudaError_t launch_gemm(const Maps& m, const TcGemmParams& p, bool pair, int grid,
+                               cudaStream_t s) {
+  const size_t bytes = gemm_smem_bytes(pair);
+  if (pair) {
+    auto kern = tc_grouped_gemm_pair_kernel<ACT>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return e;
+    kern<<<2 * grid, kGemmThreads, bytes, s>>>(m.a0, m.a1, m.b0, m.b0g, m.b1, m.b1g, p);
+  } else {
+    auto kern = tc_grouped_gemm_kernel<ACT>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kGemmThreads, bytes, s>>>(m.a0, m.a1, m.b0, m.b0g, m.b1, m.b1g, p);
+  }
   return cudaGetLastError();
 }
 
@@ -402,44 +734,69 @@ static int num_sms() {
   return sms;
 }
 
+// Persistent grid: one CTA (or CTA pair) per SM (pair of SMs), never more
+// than there are tiles.
+static int persistent_grid(const TcGemmParams& p, bool pair) {
+  const int sms = num_sms();
+  long long units;
+  int slots;
+  if (pair) {
+    const long long spp = (p.shared_tiles_per + 1) / 2;
+    units = ((long long)p.max_routed_tiles + p.n_shared * spp) * p.nt_tiles;
+    slots = sms / 2;
+  } else {
+    units = ((long long)p.max_routed_tiles + (long long)p.n_shared * p.shared_tiles_per) *
+            p.nt_tiles;
+    slots = sms;
+  }
+  long long g = units < slots ? units : slots;
+  return g < 1 ? 1 : (int)g;
+}
+
 moe_status run_ffn_bf16(const FfnArgs& f, cudaStream_t s) {
   const bool swiglu = f.act == MOE_ACT_SWIGLU;
+  const bool pair = f.pair;
   const long long rows = f.rows;
   const int sh_tiles = f.n_pad / kBM;
   // ---- up projection: H = act(X_perm W1^T) or silu(X_perm W1^T) * (X_perm W3^T)
-  CUtensorMap a0, a1, b0, b0g, b1, b1g;
-  const int up_box = swiglu ? kBN / 2 : kBN;
-  if (!make_map(&a0, f.X_perm, rows, f.d, kBM)) return MOE_ERR_UNSUPPORTED;
+  // B box rows: a pair CTA loads half of the 256-row B tile; a single CTA
+  // loads all of it (SwiGLU: 128 rows of W1 plus 128 of W3)
+  const int b_box_up = (pair || swiglu) ? kBN / 2 : kBN;
+  const int b_box_dn = pair ? kBN / 2 : kBN;
+  const int out_cols_up = swiglu ? kBN / 2 : kBN;
+  Maps m;
+  if (!make_map(&m.a0, f.X_perm, rows, f.d, kBM)) return MOE_ERR_UNSUPPORTED;
   if (f.n_shared > 0) {
-    if (!make_map(&a1, f.X, f.n, f.d, kBM)) return MOE_ERR_UNSUPPORTED;
+    if (!make_map(&m.a1, f.X, f.n, f.d, kBM)) return MOE_ERR_UNSUPPORTED;
   } else {
-    a1 = a0;
+    m.a1 = m.a0;
   }
-  if (!make_map(&b0, f.W1, (long long)f.E * f.h, f.d, up_box)) return MOE_ERR_UNSUPPORTED;
+  if (!make_map(&m.b0, f.W1, (long long)f.E * f.h, f.d, b_box_up)) return MOE_ERR_UNSUPPORTED;
   if (swiglu) {
-    if (!make_map(&b0g, f.W3, (long long)f.E * f.h, f.d, up_box)) return MOE_ERR_UNSUPPORTED;
+    if (!make_map(&m.b0g, f.W3, (long long)f.E * f.h, f.d, b_box_up))
+      return MOE_ERR_UNSUPPORTED;
   } else {
-    b0g = b0;
+    m.b0g = m.b0;
   }
   if (f.n_shared > 0) {
-    if (!make_map(&b1, f.sW1, (long long)f.n_shared * f.h, f.d, up_box))
+    if (!make_map(&m.b1, f.sW1, (long long)f.n_shared * f.h, f.d, b_box_up))
       return MOE_ERR_UNSUPPORTED;
     if (swiglu) {
-      if (!make_map(&b1g, f.sW3, (long long)f.n_shared * f.h, f.d, up_box))
+      if (!make_map(&m.b1g, f.sW3, (long long)f.n_shared * f.h, f.d, b_box_up))
         return MOE_ERR_UNSUPPORTED;
     } else {
-      b1g = b1;
+      m.b1g = m.b1;
     }
   } else {
-    b1 = b0;
-    b1g = b0g;
+    m.b1 = m.b0;
+    m.b1g = m.b0g;
   }
   TcGemmParams p{};
   p.offsets = f.offsets;
   p.E = f.E;
   p.K = f.d;
   p.n_out = f.h;
-  p.nt_tiles = ceil_div(f.h, up_box);
+  p.nt_tiles = ceil_div(f.h, out_cols_up);
   p.b_rows_per_expert = f.h;
   p.shared_tiles_per = sh_tiles;
   p.n_shared = f.n_shared;
@@ -450,28 +807,28 @@ moe_status run_ffn_bf16(const FfnArgs& f, cudaStream_t s) {
   p.n_pad = f.n_pad;
   p.out = static_cast<__nv_bfloat16*>(f.H);
   p.err = f.err;
-  const int sms = num_sms();
-  long long tiles_up = (rows / kBM) * p.nt_tiles;
-  int grid = (int)(tiles_up < sms ? tiles_up : sms);
-  if (grid < 1) grid = 1;
   cudaError_t e;
+  const int grid_up = persistent_grid(p, pair);
   switch (f.act) {
-    case MOE_ACT_RELU: e = launch_tc<ACT_RELU>(a0, a1, b0, b0g, b1, b1g, p, grid, s); break;
-    case MOE_ACT_GELU: e = launch_tc<ACT_GELU>(a0, a1, b0, b0g, b1, b1g, p, grid, s); break;
-    default: e = launch_tc<ACT_SWIGLU>(a0, a1, b0, b0g, b1, b1g, p, grid, s); break;
+    case MOE_ACT_RELU: e = launch_gemm<ACT_RELU>(m, p, pair, grid_up, s); break;
+    case MOE_ACT_GELU: e = launch_gemm<ACT_GELU>(m, p, pair, grid_up, s); break;
+    default: e = launch_gemm<ACT_SWIGLU>(m, p, pair, grid_up, s); break;
   }
   if (e != cudaSuccess) return MOE_ERR_CUDA;
 
   // ---- down projection: Y = H W2^T
-  CUtensorMap da0, db0, db1;
-  if (!make_map(&da0, f.H, rows, f.h, kBM)) return MOE_ERR_UNSUPPORTED;
-  if (!make_map(&db0, f.W2, (long long)f.E * f.d, f.h, kBN)) return MOE_ERR_UNSUPPORTED;
+  Maps dm;
+  if (!make_map(&dm.a0, f.H, rows, f.h, kBM)) return MOE_ERR_UNSUPPORTED;
+  dm.a1 = dm.a0;
+  if (!make_map(&dm.b0, f.W2, (long long)f.E * f.d, f.h, b_box_dn)) return MOE_ERR_UNSUPPORTED;
+  dm.b0g = dm.b0;
   if (f.n_shared > 0) {
-    if (!make_map(&db1, f.sW2, (long long)f.n_shared * f.d, f.h, kBN))
+    if (!make_map(&dm.b1, f.sW2, (long long)f.n_shared * f.d, f.h, b_box_dn))
       return MOE_ERR_UNSUPPORTED;
   } else {
-    db1 = db0;
+    dm.b1 = dm.b0;
   }
+  dm.b1g = dm.b1;
   TcGemmParams q = p;
   q.K = f.h;
   q.n_out = f.d;
@@ -480,10 +837,7 @@ moe_status run_ffn_bf16(const FfnArgs& f, cudaStream_t s) {
   q.a1_row_base = f.shared_base;
   q.a1_row_stride = f.n_pad;
   q.out = static_cast<__nv_bfloat16*>(f.Y);
-  long long tiles_dn = (rows / kBM) * q.nt_tiles;
-  grid = (int)(tiles_dn < sms ? tiles_dn : sms);
-  if (grid < 1) grid = 1;
-  e = launch_tc<ACT_NONE>(da0, da0, db0, db0, db1, db1, q, grid, s);
+  e = launch_gemm<ACT_NONE>(dm, q, pair, persistent_grid(q, pair), s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }

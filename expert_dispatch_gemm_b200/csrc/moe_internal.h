@@ -15,9 +15,10 @@ constexpr int kRowAlign = MOE_ROW_ALIGN;
 inline int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 inline long long round_up(long long a, long long b) { return (a + b - 1) / b * b; }
 
-// Router tile: rows per CTA for a padded expert count ET.
+// Router tile: padded expert count, and rows per CTA for (E, n) (>= 16).
 int router_tile_et(int E);
-int router_block_rows(int E);
+int router_block_rows(int E, int n);
+constexpr int kRouterMinBlockRows = 16;
 
 struct Derived {
   int k;            // EC tokens per expert / TC experts per token
@@ -92,6 +93,12 @@ struct SelectEcArgs {
   int32_t* counts;
   int32_t* offsets;
   int* err;
+  // block 0 also resets the accumulators the finish kernel adds into
+  int32_t* hist;        // optional [E+1]
+  float* aux;
+  const double* lse2;   // [lse_blocks] or NULL
+  int lse_blocks;
+  float z_coef;
 };
 cudaError_t launch_select_ec(const SelectEcArgs& a, cudaStream_t s);
 
@@ -162,6 +169,7 @@ struct FfnArgs {
   int n, d, h, E, act, n_shared, n_pad;
   long long rows_routed, shared_base, rows;
   int* err;
+  bool pair;  // bf16: CTA-pair (cta_group::2) kernel instead of the single-CTA one
 };
 moe_status run_ffn_bf16(const FfnArgs& a, cudaStream_t s);
 moe_status run_ffn_f32(const FfnArgs& a, cudaStream_t s);

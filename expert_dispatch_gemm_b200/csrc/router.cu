@@ -12,6 +12,14 @@
 // The router contraction stays on CUDA cores in fp32: its scores decide
 // integer selections, and the expert FFN is the only step that runs on the
 // tensor cores.
+//
+// Main loop: one CTA owns BM rows and all E columns (so the epilogue sees
+// whole rows). X and W_g chunks of BK along d stream through a 4-deep
+// cp.async ring; each X chunk is converted once to fp32 into a transposed
+// tile. Each thread holds TM x TN accumulators; a lane's TN columns are two
+// groups of 4 that sit 4*LY columns apart, so every 8-lane phase of a 128-bit
+// shared load reads one contiguous 128 bytes (no bank conflicts). WK > 1
+// splits each chunk's k range across warp groups, summed in a fixed order.
 #include <math.h>
 
 #include "device_common.cuh"
@@ -19,54 +27,88 @@
 
 namespace moe {
 
-// Per-thread TM x TN outputs; LX x LY lanes per warp; WX x WY x WK warps
-// (WK splits each K chunk; partial sums are reduced in a fixed order).
-template <int ET>
-struct RouterTile;
-template <>
-struct RouterTile<8> {
-  static constexpr int TM = 1, TN = 8, LX = 32, LY = 1, WX = 1, WY = 1, WK = 8;
+template <int ET_, int TM_, int TN_, int LX_, int WX_, int WY_, int WK_, int BK_, int ST_>
+struct RCfg {
+  static constexpr int ET = ET_, TM = TM_, TN = TN_, LX = LX_, LY = 32 / LX_, WX = WX_,
+                       WY = WY_, WK = WK_, BK = BK_, ST = ST_, BM = WX_ * LX_ * TM_;
+  static_assert(WY * LY * TN == ET, "columns");
+  static_assert(WX * WY * WK == 8, "8 warps");
+  static_assert(TN == 4 || TN == 8, "TN");
+  static_assert(BK % WK == 0 && ST >= 2, "pipeline");
 };
-template <>
-struct RouterTile<32> {
-  static constexpr int TM = 2, TN = 4, LX = 4, LY = 8, WX = 4, WY = 1, WK = 2;
-};
-template <>
-struct RouterTile<64> {
-  static constexpr int TM = 2, TN = 8, LX = 4, LY = 8, WX = 8, WY = 1, WK = 1;
-};
-template <>
-struct RouterTile<128> {
-  static constexpr int TM = 2, TN = 8, LX = 4, LY = 8, WX = 4, WY = 2, WK = 1;
-};
-template <>
-struct RouterTile<256> {
-  static constexpr int TM = 4, TN = 8, LX = 4, LY = 8, WX = 2, WY = 4, WK = 1;
-};
+// 4 x 8 register tiles wherever E allows (half the shared-memory bytes per FMA
+// of 2 x 8); the "s" variants trade rows per CTA for an in-CTA K split when the
+// batch is too small to give every SM a CTA. E = 8 is bound by reading X, so
+// its chunks are long (BK 128) to keep ~48 KB in flight per CTA.
+//                   ET   TM TN LX WX WY WK  BK  ST
+using R8 = RCfg<8, 1, 8, 32, 1, 1, 8, 128, 4>;
+using R32 = RCfg<32, 2, 4, 4, 4, 1, 2, 64, 4>;
+using R64 = RCfg<64, 4, 8, 4, 4, 1, 2, 32, 4>;
+using R64s = RCfg<64, 4, 8, 4, 1, 1, 8, 32, 4>;
+using R128 = RCfg<128, 4, 8, 4, 2, 2, 2, 32, 4>;
+using R256 = RCfg<256, 4, 8, 4, 2, 4, 1, 32, 3>;
+using R256s = RCfg<256, 2, 8, 4, 2, 4, 1, 32, 3>;
 
-constexpr int kRouterBK = 32;
 constexpr int kSelectRowsPerWarp = 4;
 
 int router_tile_et(int E) {
   return E <= 8 ? 8 : E <= 32 ? 32 : E <= 64 ? 64 : E <= 128 ? 128 : 256;
 }
 
-template <int ET>
-constexpr int router_bm() {
-  return RouterTile<ET>::WX * RouterTile<ET>::LX * RouterTile<ET>::TM;
+static int num_sms_cached() {
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      sms = 148;
+  }
+  return sms;
 }
 
-int router_block_rows(int E) {
-  switch (router_tile_et(E)) {
-    case 8: return router_bm<8>();
-    case 32: return router_bm<32>();
-    case 64: return router_bm<64>();
-    case 128: return router_bm<128>();
-    default: return router_bm<256>();
+// Which tile variant a (E, n) uses: the small-row variant when the big tile
+// would leave SMs without a CTA.
+static int router_variant(int E, int n) {
+  const int et = router_tile_et(E);
+  const int sms = num_sms_cached();
+  if (et == 64) return (n + R64::BM - 1) / R64::BM >= sms ? 64 : 65;
+  if (et == 256) return (n + R256::BM - 1) / R256::BM >= sms ? 256 : 257;
+  return et;
+}
+
+int router_block_rows(int E, int n) {
+  switch (router_variant(E, n)) {
+    case 8: return R8::BM;
+    case 32: return R32::BM;
+    case 64: return R64::BM;
+    case 65: return R64s::BM;
+    case 128: return R128::BM;
+    case 256: return R256::BM;
+    default: return R256s::BM;
   }
 }
 
 int select_tc_block_rows() { return 8 * kSelectRowsPerWarp; }
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+  const int n = valid ? 16 : 0;  // 0 source bytes = zero fill
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(n)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src, bool valid) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+  const int n = valid ? 4 : 0;
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(d), "l"(src), "r"(n)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 // ---------------------------------------------------------------------------
 // Token-choice selection of one row by one warp. Lane l holds experts
@@ -157,175 +199,169 @@ __device__ __forceinline__ void tc_select_row(const float (&key)[V], const float
 // ---------------------------------------------------------------------------
 // Router GEMM + epilogue
 // ---------------------------------------------------------------------------
-template <int ET, bool XBF16>
+template <class C, bool XBF16>
+struct RouterSmem {
+  static constexpr int XB = XBF16 ? 2 : 4;
+  static constexpr int AST = C::BM + 4;  // transposed fp32 A tile row stride
+  static constexpr size_t xs_bytes = (size_t)C::ST * C::BM * C::BK * XB;
+  static constexpr size_t ws_bytes = (size_t)C::ST * C::BK * C::ET * 4;
+  static constexpr size_t as_bytes = (size_t)C::BK * AST * 4;
+  static constexpr size_t main_bytes = xs_bytes + ws_bytes + as_bytes;
+  static constexpr size_t epi_bytes =
+      ((size_t)C::WK * C::BM * (C::ET + 1) + 8 * C::ET) * 4 + 8 * 8;
+  static constexpr size_t bytes = (main_bytes > epi_bytes ? main_bytes : epi_bytes) + 128;
+};
+
+template <class C, bool XBF16>
 __global__ void __launch_bounds__(256) router_kernel(RouterArgs a) {
-  using T = RouterTile<ET>;
-  constexpr int BM = router_bm<ET>();
-  constexpr int BK = kRouterBK;
-  constexpr int AST = BM + 4;  // As row stride (floats)
+  using SM = RouterSmem<C, XBF16>;
+  constexpr int ET = C::ET, BM = C::BM, BK = C::BK, TM = C::TM, TN = C::TN;
+  constexpr int XB = SM::XB, AST = SM::AST;
   constexpr int V = ET >= 32 ? ET / 32 : 1;
-  extern __shared__ __align__(16) float smem[];
-  float* As = smem;                 // [2][BK][AST]
-  float* Bs = As + 2 * BK * AST;    // [2][BK][ET]
+  extern __shared__ __align__(16) unsigned char rsm[];
+  unsigned char* Xs = rsm;                                        // [S][BM][BK] raw
+  float* Ws = reinterpret_cast<float*>(rsm + SM::xs_bytes);       // [S][BK][ET]
+  float* As = reinterpret_cast<float*>(rsm + SM::xs_bytes + SM::ws_bytes);  // [BK][AST]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int lx = lane / T::LY, ly = lane % T::LY;
-  const int wk = warp / (T::WX * T::WY);
-  const int wrem = warp % (T::WX * T::WY);
-  const int wx = wrem / T::WY, wy = wrem % T::WY;
-  const int row0 = (wx * T::LX + lx) * T::TM;
-  const int col0 = (wy * T::LY + ly) * T::TN;
+  const int lx = lane / C::LY, ly = lane % C::LY;
+  const int wk = warp / (C::WX * C::WY);
+  const int wrem = warp % (C::WX * C::WY);
+  const int wx = wrem / C::WY, wy = wrem % C::WY;
+  const int row0 = (wx * C::LX + lx) * TM;
+  const int colb = wy * C::LY * TN + ly * 4;  // first column of group 0; group g adds g*4*LY
   const int m0 = blockIdx.x * BM;
   const int n = a.n, d = a.d, E = a.E;
-
-  constexpr int XV = XBF16 ? 8 : 4;             // elements per 16-byte vector
-  constexpr int XVEC = BM * BK / XV;
-  constexpr int XPT = (XVEC + 255) / 256;
-  constexpr int WPT = (BK * ET + 255) / 256;        // scalar Wg loads per thread
-  constexpr int WV4 = (BK * ET / 4 + 255) / 256;    // float4 Wg loads per thread
-  constexpr int WREG = WPT > 4 * WV4 ? WPT : 4 * WV4;
   const bool w_vec = (E % 4 == 0);
 
-  float acc[T::TM][T::TN];
+  float acc[TM][TN];
 #pragma unroll
-  for (int i = 0; i < T::TM; ++i)
+  for (int i = 0; i < TM; ++i)
 #pragma unroll
-    for (int j = 0; j < T::TN; ++j) acc[i][j] = 0.0f;
+    for (int j = 0; j < TN; ++j) acc[i][j] = 0.0f;
 
-  uint4 xr[XPT];
-  float wr[WREG];
-
-  auto load_regs = [&](int kb) {
-#pragma unroll
-    for (int i = 0; i < XPT; ++i) {
-      const int v = tid + i * 256;
-      xr[i] = make_uint4(0, 0, 0, 0);
-      if (v < XVEC) {
-        const int r = v / (BK / XV), kv = v % (BK / XV);
-        const int row = m0 + r, k = kb + kv * XV;
-        if (row < n && k < d) {
-          const char* base = reinterpret_cast<const char*>(a.X);
-          const size_t off = ((size_t)row * d + k) * (XBF16 ? 2 : 4);
-          xr[i] = __ldg(reinterpret_cast<const uint4*>(base + off));
-        }
-      }
+  // stage loader: X chunk [BM][BK] and W_g chunk [BK][ET] of chunk `c`
+  auto issue = [&](int c) {
+    const int st = c % C::ST;
+    const int k0 = c * BK;
+    constexpr int XCH = BM * BK * XB / 16;          // 16-byte pieces of the X chunk
+    constexpr int XPR = BK * XB / 16;               // pieces per row
+    unsigned char* xs = Xs + (size_t)st * BM * BK * XB;
+    for (int q = tid; q < XCH; q += 256) {
+      const int r = q / XPR, p = q % XPR;
+      const int row = m0 + r, k = k0 + p * (16 / XB);
+      const bool ok = row < n && k < d;
+      const char* src = static_cast<const char*>(a.X) +
+                        ((size_t)(ok ? row : 0) * d + (ok ? k : 0)) * XB;
+      cp_async16(xs + (size_t)r * BK * XB + p * 16, src, ok);
     }
+    float* ws = Ws + (size_t)st * BK * ET;
     if (w_vec) {
-#pragma unroll
-      for (int i = 0; i < WV4; ++i) {
-        const int v = tid + i * 256;  // float4 index in the [BK][ET] tile
-        if (v < BK * ET / 4) {
-          const int kk = v / (ET / 4), c = (v % (ET / 4)) * 4;
-          const int k = kb + kk;
-          float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (k < d && c < E) f = __ldg(reinterpret_cast<const float4*>(a.Wg + (size_t)k * E + c));
-          wr[4 * i + 0] = f.x;
-          wr[4 * i + 1] = f.y;
-          wr[4 * i + 2] = f.z;
-          wr[4 * i + 3] = f.w;
-        }
+      constexpr int WCH = BK * ET / 4;
+      for (int q = tid; q < WCH; q += 256) {
+        const int kk = q / (ET / 4), c4 = (q % (ET / 4)) * 4;
+        const int k = k0 + kk;
+        const bool ok = k < d && c4 < E;
+        cp_async16(ws + kk * ET + c4, a.Wg + (ok ? (size_t)k * E + c4 : 0), ok);
       }
     } else {
-#pragma unroll
-      for (int i = 0; i < WPT; ++i) {
-        const int v = tid + i * 256;
-        wr[i] = 0.0f;
-        if (v < BK * ET) {
-          const int kk = v / ET, c = v % ET;
-          const int k = kb + kk;
-          if (k < d && c < E) wr[i] = __ldg(a.Wg + (size_t)k * E + c);
-        }
-      }
-    }
-  };
-
-  auto store_smem = [&](int buf) {
-    float* as = As + buf * BK * AST;
-    float* bs = Bs + buf * BK * ET;
-#pragma unroll
-    for (int i = 0; i < XPT; ++i) {
-      const int v = tid + i * 256;
-      if (v < XVEC) {
-        const int r = v / (BK / XV), kv = v % (BK / XV);
-        if (XBF16) {
-          const uint32_t w4[4] = {xr[i].x, xr[i].y, xr[i].z, xr[i].w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            as[(kv * XV + 2 * j) * AST + r] = __uint_as_float(w4[j] << 16);
-            as[(kv * XV + 2 * j + 1) * AST + r] = __uint_as_float(w4[j] & 0xffff0000u);
-          }
-        } else {
-          as[(kv * XV + 0) * AST + r] = __uint_as_float(xr[i].x);
-          as[(kv * XV + 1) * AST + r] = __uint_as_float(xr[i].y);
-          as[(kv * XV + 2) * AST + r] = __uint_as_float(xr[i].z);
-          as[(kv * XV + 3) * AST + r] = __uint_as_float(xr[i].w);
-        }
-      }
-    }
-    if (w_vec) {
-#pragma unroll
-      for (int i = 0; i < WV4; ++i) {
-        const int v = tid + i * 256;
-        if (v < BK * ET / 4) {
-          *reinterpret_cast<float4*>(bs + v * 4) =
-              make_float4(wr[4 * i], wr[4 * i + 1], wr[4 * i + 2], wr[4 * i + 3]);
-        }
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < WPT; ++i) {
-        const int v = tid + i * 256;
-        if (v < BK * ET) bs[v] = wr[i];
+      constexpr int WCH = BK * ET;
+      for (int q = tid; q < WCH; q += 256) {
+        const int kk = q / ET, cc = q % ET;
+        const int k = k0 + kk;
+        const bool ok = k < d && cc < E;
+        cp_async4(ws + kk * ET + cc, a.Wg + (ok ? (size_t)k * E + cc : 0), ok);
       }
     }
   };
 
   const int nchunks = (d + BK - 1) / BK;
-  load_regs(0);
-  store_smem(0);
-  __syncthreads();
-  for (int c = 0; c < nchunks; ++c) {
-    if (c + 1 < nchunks) load_regs((c + 1) * BK);
-    const float* as = As + (c & 1) * BK * AST;
-    const float* bs = Bs + (c & 1) * BK * ET;
-#pragma unroll
-    for (int q = 0; q < BK / T::WK; ++q) {
-      const int kk = wk * (BK / T::WK) + q;
-      float av[T::TM], bv[T::TN];
-#pragma unroll
-      for (int i = 0; i < T::TM; ++i) av[i] = as[kk * AST + row0 + i];
-#pragma unroll
-      for (int j = 0; j < T::TN; ++j) bv[j] = bs[kk * ET + col0 + j];
-#pragma unroll
-      for (int i = 0; i < T::TM; ++i)
-#pragma unroll
-        for (int j = 0; j < T::TN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-    }
-    if (c + 1 < nchunks) store_smem((c + 1) & 1);
-    __syncthreads();
+#pragma unroll 1
+  for (int c = 0; c < C::ST - 1; ++c) {
+    if (c < nchunks) issue(c);
+    cp_async_commit();
   }
+#pragma unroll 1
+  for (int c = 0; c < nchunks; ++c) {
+    cp_async_wait<C::ST - 2>();
+    __syncthreads();
+    {  // convert the X chunk to fp32, transposed: As[kk][r]
+      const int st = c % C::ST;
+      const unsigned char* xs = Xs + (size_t)st * BM * BK * XB;
+      constexpr int EPP = 16 / XB;                 // elements per 16-byte piece
+      constexpr int PCS = BM * BK / EPP;
+      for (int q = tid; q < PCS; q += 256) {
+        const int r = q % BM, p = q / BM;
+        const uint4 v = *reinterpret_cast<const uint4*>(xs + (size_t)r * BK * XB + p * 16);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+        if (XBF16) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            As[(p * 8 + 2 * j) * AST + r] = __uint_as_float(w4[j] << 16);
+            As[(p * 8 + 2 * j + 1) * AST + r] = __uint_as_float(w4[j] & 0xffff0000u);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) As[(p * 4 + j) * AST + r] = __uint_as_float(w4[j]);
+        }
+      }
+    }
+    __syncthreads();
+    if (c + C::ST - 1 < nchunks) issue(c + C::ST - 1);
+    cp_async_commit();
+    const float* ws = Ws + (size_t)(c % C::ST) * BK * ET;
+#pragma unroll
+    for (int q = 0; q < BK / C::WK; ++q) {
+      const int kk = wk * (BK / C::WK) + q;
+      float av[TM], bv[TN];
+      if (TM == 4) {
+        const float4 t = *reinterpret_cast<const float4*>(As + kk * AST + row0);
+        av[0] = t.x; av[1] = t.y; av[2 % TM] = t.z; av[3 % TM] = t.w;
+      } else if (TM == 2) {
+        const float2 t = *reinterpret_cast<const float2*>(As + kk * AST + row0);
+        av[0] = t.x; av[1 % TM] = t.y;
+      } else {
+        av[0] = As[kk * AST + row0];
+      }
+#pragma unroll
+      for (int g = 0; g < TN / 4; ++g) {
+        const float4 t = *reinterpret_cast<const float4*>(ws + kk * ET + colb + g * 4 * C::LY);
+        bv[4 * g + 0] = t.x;
+        bv[4 * g + 1] = t.y;
+        bv[4 * g + 2] = t.z;
+        bv[4 * g + 3] = t.w;
+      }
+#pragma unroll
+      for (int i = 0; i < TM; ++i)
+#pragma unroll
+        for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+  }
+  cp_async_wait<0>();
+  __syncthreads();
 
   // ---- epilogue: logits tile in shared memory ----
   constexpr int LST = ET + 1;
-  float* Ls = smem;  // [WK][BM][LST]
+  float* Ls = reinterpret_cast<float*>(rsm);  // [WK][BM][LST]
 #pragma unroll
-  for (int i = 0; i < T::TM; ++i)
+  for (int i = 0; i < TM; ++i)
 #pragma unroll
-    for (int j = 0; j < T::TN; ++j) Ls[(wk * BM + row0 + i) * LST + col0 + j] = acc[i][j];
+    for (int j = 0; j < TN; ++j)
+      Ls[(wk * BM + row0 + i) * LST + colb + (j / 4) * 4 * C::LY + (j % 4)] = acc[i][j];
   __syncthreads();
-  if (T::WK > 1) {
+  if (C::WK > 1) {
     for (int q = tid; q < BM * ET; q += 256) {
       const int r = q / ET, cc = q % ET;
       float s = Ls[r * LST + cc];
 #pragma unroll
-      for (int w = 1; w < T::WK; ++w) s += Ls[(w * BM + r) * LST + cc];
+      for (int w = 1; w < C::WK; ++w) s += Ls[(w * BM + r) * LST + cc];
       Ls[r * LST + cc] = s;
     }
     __syncthreads();
   }
 
-  float* colsum_w = smem + T::WK * BM * LST;              // [8][ET]
-  double* lse2_w = reinterpret_cast<double*>(colsum_w + 8 * ET);  // [8]
+  float* colsum_w = Ls + C::WK * BM * LST;                          // [8][ET]
+  double* lse2_w = reinterpret_cast<double*>(colsum_w + 8 * ET);     // [8]
   float csum[V];
 #pragma unroll
   for (int v = 0; v < V; ++v) csum[v] = 0.0f;
@@ -384,52 +420,46 @@ __global__ void __launch_bounds__(256) router_kernel(RouterArgs a) {
   if (lane == 0) lse2_w[warp] = my_lse2;
   __syncthreads();
   for (int cc = tid; cc < E; cc += 256) {
-    float s = 0.0f;
-    for (int w = 0; w < 8; ++w) s += colsum_w[w * ET + cc];
-    a.colsum[(size_t)blockIdx.x * E + cc] = s;
+    float sum = 0.0f;
+    for (int w = 0; w < 8; ++w) sum += colsum_w[w * ET + cc];
+    a.colsum[(size_t)blockIdx.x * E + cc] = sum;
   }
   if (tid == 0) {
-    double s = 0.0;
-    for (int w = 0; w < 8; ++w) s += lse2_w[w];
-    a.lse2[blockIdx.x] = s;
+    double sum = 0.0;
+    for (int w = 0; w < 8; ++w) sum += lse2_w[w];
+    a.lse2[blockIdx.x] = sum;
   }
 }
 
-template <int ET, bool XBF16>
+template <class C, bool XBF16>
 static cudaError_t launch_router_t(const RouterArgs& a, cudaStream_t s) {
-  using T = RouterTile<ET>;
-  constexpr int BM = router_bm<ET>();
-  const size_t main_f = 2 * kRouterBK * (BM + 4) + 2 * kRouterBK * ET;
-  const size_t epi_f = (size_t)T::WK * BM * (ET + 1) + 8 * ET + 2 * 8;
-  const size_t bytes = (main_f > epi_f ? main_f : epi_f) * sizeof(float) + 64;
-  auto kern = router_kernel<ET, XBF16>;
+  const size_t bytes = RouterSmem<C, XBF16>::bytes;
+  auto kern = router_kernel<C, XBF16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)bytes);
   if (e != cudaSuccess) return e;
-  const int grid = ceil_div(a.n, BM);
+  const int grid = ceil_div(a.n, C::BM);
   kern<<<grid, 256, bytes, s>>>(a);
   return cudaGetLastError();
 }
 
-cudaError_t launch_router(const RouterArgs& a, cudaStream_t s) {
-  const int et = router_tile_et(a.E);
-  if (a.x_bf16) {
-    switch (et) {
-      case 8: return launch_router_t<8, true>(a, s);
-      case 32: return launch_router_t<32, true>(a, s);
-      case 64: return launch_router_t<64, true>(a, s);
-      case 128: return launch_router_t<128, true>(a, s);
-      default: return launch_router_t<256, true>(a, s);
-    }
-  }
-  switch (et) {
-    case 8: return launch_router_t<8, false>(a, s);
-    case 32: return launch_router_t<32, false>(a, s);
-    case 64: return launch_router_t<64, false>(a, s);
-    case 128: return launch_router_t<128, false>(a, s);
-    default: return launch_router_t<256, false>(a, s);
+template <bool XBF16>
+static cudaError_t launch_router_dt(const RouterArgs& a, cudaStream_t s) {
+  switch (router_variant(a.E, a.n)) {
+    case 8: return launch_router_t<R8, XBF16>(a, s);
+    case 32: return launch_router_t<R32, XBF16>(a, s);
+    case 64: return launch_router_t<R64, XBF16>(a, s);
+    case 65: return launch_router_t<R64s, XBF16>(a, s);
+    case 128: return launch_router_t<R128, XBF16>(a, s);
+    case 256: return launch_router_t<R256, XBF16>(a, s);
+    default: return launch_router_t<R256s, XBF16>(a, s);
   }
 }
+
+cudaError_t launch_router(const RouterArgs& a, cudaStream_t s) {
+  return a.x_bf16 ? launch_router_dt<true>(a, s) : launch_router_dt<false>(a, s);
+}
+
 
 // ---------------------------------------------------------------------------
 // Token-choice selection from a given score matrix (one warp per row).
