@@ -3,9 +3,10 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl reference]
 
-One step = one pass of the whole hot path over one batch: moe_route
-(router GEMM + scores + top-k + capacity scan) -> moe_dispatch (gather) ->
-moe_expert_ffn (tcgen05 grouped GEMM, up + down) -> moe_combine. Inputs and
+One step = one pass of the whole hot path over one batch, the calls
+moe_layer_forward makes: moe_route (router GEMM + scores + top-k + capacity
+scan) -> moe_dispatch (gather) -> moe_expert_ffn (tcgen05 grouped GEMM, up +
+down) -> moe_combine. Inputs and
 weights are resident in HBM before timing; L2 (126 MB) is flushed by writing
 a 256 MB buffer between timed steps, outside the timed events. Each stage is
 timed with CUDA events on the launching stream.
@@ -51,6 +52,25 @@ def peaks():
         return p["hbm_gbs"], p["bf16_tflops"], p.get("bf16_tflops_sustained"), "measured"
     except Exception:
         return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# multi-rank plumbing (replicas only: no collective touches the data path)
+# ---------------------------------------------------------------------------
+
+def max_over_ranks(value_ms: float, device=None) -> float:
+    """The slowest rank's time: every rank calls this in the same order."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value_ms)
+    t = torch.tensor([float(value_ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: int, world: int, steps: int, total_ms: float) -> float:
+    """Units all ranks processed per second over the max-over-ranks time."""
+    return units_per_rank * world * steps / (total_ms * 1e-3)
 
 
 # ---------------------------------------------------------------------------
@@ -182,6 +202,8 @@ def run_gpu(args, w: wl.Workload):
     sb = inp["sel_bias"]
 
     def step(ev=None, X=None):
+        """One pass of the layer, the calls moe_layer_forward makes:
+        route -> dispatch gather -> grouped expert FFN -> combine."""
         X = inp["X"] if X is None else X
         if ev: ev[0].record(stream)
         moe.moe_route(cfg, X, inp["Wg"], inp["logit_bias"], sb, rb, ws, stream)
@@ -219,10 +241,7 @@ def run_gpu(args, w: wl.Workload):
                          for i in range(args.steps)])
     step_ms = stage_ms.sum(1)
     total_ms = float(step_ms.sum())
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev)
     st, detail = moe.moe_read_error(ws)
     if st != moe.MOE_OK:
         raise RuntimeError(f"device error in the timed region: {detail:#x}")
@@ -247,10 +266,8 @@ def run_gpu(args, w: wl.Workload):
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = float(np.sum([a.elapsed_time(b) for a, b in e2e_ev]))
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dev)
+
 
     # ---- algorithmic work and rooflines
     counts = rb.counts.cpu().numpy()
@@ -287,9 +304,8 @@ def run_gpu(args, w: wl.Workload):
                  "algorithmic_per_launch": bytes_["ffn"] / 2 if roof["bound"] == "hbm"
                  else flops / 2})
 
-    tokens = w.n * world
-    value = tokens * args.steps / (total_ms * 1e-3)
-    e2e_value = tokens * args.steps / (e2e_ms * 1e-3)
+    value = whole_job_rate(w.n, world, args.steps, total_ms)
+    e2e_value = whole_job_rate(w.n, world, args.steps, e2e_ms)
     # route: router + select_ec + ec_finish (EC) or router + hist + scan + scatter (TC);
     # dispatch: gather; expert FFN: up + down; combine
     launches_per_step = (3 if w.mode == "ec" else 4) + 1 + 2 + 1

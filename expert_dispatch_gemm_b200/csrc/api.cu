@@ -252,11 +252,15 @@ static moe_status route_impl(const moe_config* c, const Derived& dv, const WsLay
                       ceil_div(c->n, router_block_rows(c->E, c->n)), true, s);
 }
 
+// X_perm == NULL: the routed rows are read from X through row_token (the
+// dispatch gather fused into the first projection's A loads)
 static moe_status ffn_impl(const moe_config* c, const Derived& dv, const void* X,
-                           const void* X_perm, const int32_t* offsets, const void* W1,
-                           const void* W3, const void* W2, const void* sW1, const void* sW3,
-                           const void* sW2, void* H, void* Y, int* err, cudaStream_t s) {
-  if (!X_perm || !offsets || !W1 || !W2 || !H || !Y) return MOE_ERR_INVALID_ARG;
+                           const void* X_perm, const int32_t* row_token, const int32_t* offsets,
+                           const void* W1, const void* W3, const void* W2, const void* sW1,
+                           const void* sW3, const void* sW2, void* H, void* Y, int* err,
+                           cudaStream_t s) {
+  if (!offsets || !W1 || !W2 || !H || !Y) return MOE_ERR_INVALID_ARG;
+  if (!X_perm && (!X || !row_token)) return MOE_ERR_INVALID_ARG;
   if (c->act == MOE_ACT_SWIGLU && !W3) return MOE_ERR_INVALID_ARG;
   if (c->n_shared > 0) {
     if (!X || !sW1 || !sW2) return MOE_ERR_INVALID_ARG;
@@ -265,6 +269,7 @@ static moe_status ffn_impl(const moe_config* c, const Derived& dv, const void* X
   FfnArgs f{};
   f.X = X;
   f.X_perm = X_perm;
+  f.row_token = row_token;
   f.offsets = offsets;
   f.W1 = W1;
   f.W3 = W3;
@@ -441,7 +446,8 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* X, const void* X_pe
   moe_status st = derive(cfg, &d);
   if (st != MOE_OK) return st;
   if ((st = check_ws(ws, ws_bytes, MOE_WS_ERROR_BYTES)) != MOE_OK) return st;
-  return ffn_impl(cfg, d, X, X_perm, offsets, W1, W3, W2, sW1, sW3, sW2, H, Y_perm,
+  if (!X_perm) return MOE_ERR_INVALID_ARG;
+  return ffn_impl(cfg, d, X, X_perm, nullptr, offsets, W1, W3, W2, sW1, sW3, sW2, H, Y_perm,
                   at<int>(ws, 0), (cudaStream_t)stream);
 }
 
@@ -473,11 +479,28 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* X, const float* 
   void* yp = at<void>(ws, w.yperm);
   if ((st = route_impl(cfg, d, w, X, Wg, logit_bias, sel_bias, route, ws, s)) != MOE_OK)
     return st;
+  // the gather stays a separate pass: fused into the GEMM's A loads it costs
+  // 32 four-row TMA gathers per 64-deep k-block, which the TMA unit issues
+  // far slower than the two box loads the unfused GEMM needs
   if ((st = dispatch_impl(cfg, d, X, route, xp, s)) != MOE_OK) return st;
-  if ((st = ffn_impl(cfg, d, X, xp, route->offsets, W1, W3, W2, sW1, sW3, sW2, hb, yp,
+  if ((st = ffn_impl(cfg, d, X, xp, nullptr, route->offsets, W1, W3, W2, sW1, sW3, sW2, hb, yp,
                      at<int>(ws, w.err), s)) != MOE_OK)
     return st;
   return combine_impl(cfg, d, yp, route, out, s);
+}
+
+moe_status moe_expert_ffn_gathered(const moe_config* cfg, const void* X,
+                                   const moe_route_out* route, const void* W1, const void* W3,
+                                   const void* W2, const void* sW1, const void* sW3,
+                                   const void* sW2, void* H, void* Y_perm, void* ws,
+                                   size_t ws_bytes, moe_stream_t stream) {
+  Derived d;
+  moe_status st = derive(cfg, &d);
+  if (st != MOE_OK) return st;
+  if (!X || !route || !route->row_token || !route->offsets) return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(ws, ws_bytes, MOE_WS_ERROR_BYTES)) != MOE_OK) return st;
+  return ffn_impl(cfg, d, X, nullptr, route->row_token, route->offsets, W1, W3, W2, sW1, sW3,
+                  sW2, H, Y_perm, at<int>(ws, 0), (cudaStream_t)stream);
 }
 
 moe_status moe_bias_update(const moe_config* cfg, const int32_t* load, float rate, float* bias,

@@ -22,34 +22,62 @@ __device__ __forceinline__ uint32_t ordered_key(float f) {
 
 // ---------------------------------------------------------------------------
 // Expert choice: one CTA per expert. Radix-select the k-th largest key of the
-// column, take every key above it plus the lowest-index ties, then sort the
-// k picks by (score desc, token asc) with a bitonic sort of composite keys.
+// column, take every key above it plus the lowest-index ties (ordered block
+// scans, no atomics), then order the k picks by (score desc, token asc): by
+// counting ranks for k <= kEcRankMax, by a bitonic sort of 64-bit composite
+// keys beyond that. The dense slot map is [E, n] so each CTA clears and
+// fills its own contiguous row.
 // ---------------------------------------------------------------------------
 constexpr int kEcThreads = 1024;
+constexpr int kEcRankMax = 1024;
+
+// exclusive prefix sum over the CTA (threads in order); returns the total
+__device__ __forceinline__ int block_exclusive_scan(int v, int* excl, int* warp_tot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  __syncthreads();  // warp_tot may still be read from a previous scan
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  int wbase = 0, total = 0;
+  const int nw = blockDim.x >> 5;
+  for (int w = 0; w < nw; ++w) {
+    const int x = warp_tot[w];
+    if (w < warp) wbase += x;
+    total += x;
+  }
+  *excl = wbase + incl - v;
+  return total;
+}
 
 __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
   extern __shared__ __align__(16) unsigned char ec_smem[];
   const int n = a.n, E = a.E, k = a.k, e = blockIdx.x;
+  const bool by_rank = k <= kEcRankMax;
   int kp = 1;
   while (kp < k) kp <<= 1;
-  uint64_t* sbuf = reinterpret_cast<uint64_t*>(ec_smem);           // [kp]
-  uint32_t* key = reinterpret_cast<uint32_t*>(sbuf + kp);          // [n]
+  const int nbuf = by_rank ? k : kp;
+  uint64_t* sbuf = reinterpret_cast<uint64_t*>(ec_smem);                    // [nbuf]
+  uint64_t* sorted = by_rank ? sbuf + k : sbuf;                              // [k]
+  uint32_t* key = reinterpret_cast<uint32_t*>(sbuf + (by_rank ? 2 * k : kp));  // [n]
   __shared__ int hist[256];
   __shared__ int warp_tot[32];
   __shared__ uint32_t s_prefix, s_mask;
-  __shared__ int s_need, s_cnt;
+  __shared__ int s_need;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int32_t* my_rows = a.ec_row + (size_t)e * n;
 
   for (int t = tid; t < n; t += kEcThreads) {
     key[t] = ordered_key(a.S[(size_t)t * E + e]);
-    a.ec_row[(size_t)t * E + e] = -1;
-    a.ec_gate[(size_t)t * E + e] = 0.0f;
+    my_rows[t] = -1;
   }
   if (tid == 0) {
     s_prefix = 0u;
     s_mask = 0u;
     s_need = k;
-    s_cnt = 0;
   }
   __syncthreads();
 
@@ -107,63 +135,74 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
   const uint32_t T = s_prefix;
   const int need_eq = s_need;  // ties at T to take, lowest token first
 
-  // ordered count of ties: thread tid owns tokens [tid*C, tid*C + C)
+  // thread tid owns tokens [tid*C, tid*C + C): the ties' ranks in token order,
+  // then every pick's slot in token order
   const int C = (n + kEcThreads - 1) / kEcThreads;
   const int t0 = tid * C, t1 = min(n, t0 + C);
   int my_eq = 0;
   for (int t = t0; t < t1; ++t) my_eq += (key[t] == T);
-  int incl = my_eq;
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) warp_tot[warp] = incl;
-  __syncthreads();
-  int wbase = 0;
-  for (int w = 0; w < warp; ++w) wbase += warp_tot[w];
-  int rank = wbase + incl - my_eq;
-  for (int t = t0; t < t1; ++t) {
-    const uint32_t u = key[t];
-    bool sel = u > T;
-    if (u == T) {
-      sel = rank < need_eq;
-      ++rank;
-    }
-    if (sel) {
-      const int slot = atomicAdd(&s_cnt, 1);
-      sbuf[slot] = ((uint64_t)u << 32) | (uint64_t)(0xffffffffu - (uint32_t)t);
+  int eq_base;
+  block_exclusive_scan(my_eq, &eq_base, warp_tot);
+  int my_sel = 0;
+  {
+    int rank = eq_base;
+    for (int t = t0; t < t1; ++t) {
+      const uint32_t u = key[t];
+      if (u > T) ++my_sel;
+      else if (u == T) my_sel += (rank++ < need_eq);
     }
   }
+  int slot;
+  const int total = block_exclusive_scan(my_sel, &slot, warp_tot);
+  {
+    int rank = eq_base;
+    for (int t = t0; t < t1; ++t) {
+      const uint32_t u = key[t];
+      bool sel = u > T;
+      if (u == T) sel = rank++ < need_eq;
+      if (sel) sbuf[slot++] = ((uint64_t)u << 32) | (uint64_t)(0xffffffffu - (uint32_t)t);
+    }
+  }
+  if (total != k && tid == 0) report_error(a.err, kErrBadIndex | 1);
   __syncthreads();
-  for (int i = k + tid; i < kp; i += kEcThreads) sbuf[i] = 0ull;
-  __syncthreads();
-  // bitonic sort, descending
-  for (int size = 2; size <= kp; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = tid; i < kp / 2; i += kEcThreads) {
-        const int lo = 2 * i - (i & (stride - 1));
-        const int hi = lo + stride;
-        const bool desc = ((lo & size) == 0);
-        const uint64_t x = sbuf[lo], y = sbuf[hi];
-        if ((x < y) == desc) {
-          sbuf[lo] = y;
-          sbuf[hi] = x;
+  if (by_rank) {
+    // composite keys are distinct: a pick's place is how many picks beat it
+    for (int j = tid; j < k; j += kEcThreads) {
+      const uint64_t c = sbuf[j];
+      int r = 0;
+      for (int i = 0; i < k; ++i) r += sbuf[i] > c;
+      sorted[r] = c;
+    }
+  } else {
+    for (int i = k + tid; i < kp; i += kEcThreads) sbuf[i] = 0ull;
+    __syncthreads();
+    for (int size = 2; size <= kp; size <<= 1) {
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        for (int i = tid; i < kp / 2; i += kEcThreads) {
+          const int lo = 2 * i - (i & (stride - 1));
+          const int hi = lo + stride;
+          const bool desc = ((lo & size) == 0);
+          const uint64_t x = sbuf[lo], y = sbuf[hi];
+          if ((x < y) == desc) {
+            sbuf[lo] = y;
+            sbuf[hi] = x;
+          }
         }
+        __syncthreads();
       }
-      __syncthreads();
     }
   }
-  if (s_cnt != k && tid == 0) report_error(a.err, kErrBadIndex | 1);
+  __syncthreads();
   for (int j = tid; j < a.kpad; j += kEcThreads) {
     const size_t row = (size_t)e * a.kpad + j;
     if (j < k) {
-      const int t = (int)(0xffffffffu - (uint32_t)(sbuf[j] & 0xffffffffull));
+      const int t = (int)(0xffffffffu - (uint32_t)(sorted[j] & 0xffffffffull));
       const float g = a.S[(size_t)t * E + e];
       a.idx[(size_t)e * k + j] = t;
       a.gate[(size_t)e * k + j] = g;
       a.row_token[row] = t;
-      a.ec_row[(size_t)t * E + e] = (int)row;
-      a.ec_gate[(size_t)t * E + e] = g;
+      my_rows[t] = (int)row;
+      a.ec_gate[(size_t)e * n + t] = g;
     } else {
       a.row_token[row] = -1;
     }
@@ -189,10 +228,15 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
   }
 }
 
-cudaError_t launch_select_ec(const SelectEcArgs& a, cudaStream_t s) {
+static size_t select_ec_smem(int n, int k) {
   int kp = 1;
-  while (kp < a.k) kp <<= 1;
-  const size_t bytes = (size_t)kp * 8 + (size_t)a.n * 4;
+  while (kp < k) kp <<= 1;
+  const size_t buf = k <= kEcRankMax ? (size_t)2 * k * 8 : (size_t)kp * 8;
+  return buf + (size_t)n * 4;
+}
+
+cudaError_t launch_select_ec(const SelectEcArgs& a, cudaStream_t s) {
+  const size_t bytes = select_ec_smem(a.n, a.k);
   cudaError_t err = cudaFuncSetAttribute(select_ec_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)bytes);
@@ -201,31 +245,33 @@ cudaError_t launch_select_ec(const SelectEcArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-// Expert choice: compact each token's picks (expert order) into its slot
-// list, the experts-per-token histogram and the aux values. Warp per token.
+// Expert choice: each token's picks (expert order) compacted into its slot
+// list, the experts-per-token histogram and the aux count of tokens no expert
+// picked. A CTA transposes a [E, 32-token] tile of the slot map through
+// shared memory (coalesced reads), then one warp per token compacts it.
 __global__ void __launch_bounds__(256) ec_finish_kernel(EcFinishArgs a) {
+  __shared__ int rows_s[MOE_MAX_EXPERTS][33];
   __shared__ int hist_s[MOE_MAX_EXPERTS + 1];
   __shared__ int none_s;
-  const int E = a.E, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int E = a.E, n = a.n, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t0 = blockIdx.x * 32;
   for (int i = threadIdx.x; i <= E; i += blockDim.x) hist_s[i] = 0;
   if (threadIdx.x == 0) none_s = 0;
+  for (int e = warp; e < E; e += 8)
+    rows_s[e][lane] = t0 + lane < n ? a.ec_row[(size_t)e * n + t0 + lane] : -1;
   __syncthreads();
-  const int t = blockIdx.x * 8 + warp;
-  if (t < a.n) {
+  for (int tt = warp; tt < 32; tt += 8) {
+    const int t = t0 + tt;
+    if (t >= n) break;
     int base = 0;
     for (int c = 0; c < E; c += 32) {
       const int e = c + lane;
-      int r = -1;
-      float g = 0.0f;
-      if (e < E) {
-        r = a.ec_row[(size_t)t * E + e];
-        g = a.ec_gate[(size_t)t * E + e];
-      }
+      const int r = e < E ? rows_s[e][tt] : -1;
       const unsigned m = __ballot_sync(0xffffffffu, r >= 0);
       if (r >= 0) {
         const int p = base + __popc(m & ((1u << lane) - 1u));
         a.tok_row[(size_t)t * E + p] = r;
-        a.tok_gate[(size_t)t * E + p] = g;
+        a.tok_gate[(size_t)t * E + p] = a.ec_gate[(size_t)e * n + t];
       }
       base += __popc(m);
     }
@@ -247,7 +293,7 @@ __global__ void __launch_bounds__(256) ec_finish_kernel(EcFinishArgs a) {
 
 // (select_ec_kernel's block 0 has zeroed hist and the aux slots)
 cudaError_t launch_ec_finish(const EcFinishArgs& a, cudaStream_t s) {
-  ec_finish_kernel<<<ceil_div(a.n, 8), 256, 0, s>>>(a);
+  ec_finish_kernel<<<ceil_div(a.n, 32), 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 
@@ -274,7 +320,19 @@ __global__ void __launch_bounds__(1024) tc_scan_kernel(TcAssignArgs a) {
   __shared__ int seg[MOE_MAX_EXPERTS];
   __shared__ int off[MOE_MAX_EXPERTS + 1];
   __shared__ double fp[MOE_MAX_EXPERTS];
+  __shared__ double part[1024];  // [slice][expert] partial column sums of S
   const int E = a.E, tid = threadIdx.x;
+  // column sums of S for the balance loss: thread (slice, e) adds the router
+  // blocks b = slice, slice + S, ... in order; the slices are then added in
+  // order, so the result does not depend on scheduling
+  const int S = max(1, (int)blockDim.x / E);
+  if (tid < S * E) {
+    const int e = tid % E, slice = tid / E;
+    double col = 0.0;
+    for (int b = slice; b < a.colsum_blocks; b += S) col += (double)a.colsum[(size_t)b * E + e];
+    part[tid] = col;
+  }
+  __syncthreads();
   for (int e = tid; e < E; e += blockDim.x) {
     int run = 0;
     for (int b = 0; b < a.tok_blocks; ++b) {
@@ -286,7 +344,7 @@ __global__ void __launch_bounds__(1024) tc_scan_kernel(TcAssignArgs a) {
     a.counts[e] = kept;
     seg[e] = (kept + kRowAlign - 1) / kRowAlign * kRowAlign;
     double col = 0.0;
-    for (int b = 0; b < a.colsum_blocks; ++b) col += (double)a.colsum[(size_t)b * E + e];
+    for (int sl = 0; sl < S; ++sl) col += part[sl * E + e];
     fp[e] = ((double)run / ((double)a.n * a.K)) * (col / (double)a.n);
   }
   __syncthreads();

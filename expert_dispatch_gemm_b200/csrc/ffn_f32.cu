@@ -14,7 +14,9 @@ namespace moe {
 constexpr int kFBM = 64, kFBN = 64, kFBK = 16;
 
 struct F32GemmArgs {
-  const float* A;        // routed A rows [rows, K]
+  const float* A;        // routed A rows [rows, K], or NULL: gather X rows via row_token
+  const float* Xg;       // X [n, K] for the gathered routed rows
+  const int32_t* row_token;
   const float* A_shared; // shared A rows [n, K] (X for the up projection, else A)
   long long a_shared_base;  // row of shared expert 0 in A_shared, stride a_shared_stride
   long long a_shared_stride;
@@ -50,11 +52,13 @@ __global__ void __launch_bounds__(256) ffn_f32_kernel(F32GemmArgs a) {
   const float* B3 = nullptr;
   long long out_row0;
   int a_rows_valid;  // rows of this tile backed by real A rows
+  bool gathered = false;
   if (m0 < a.rows_routed) {
     const int used = a.offsets[a.E];
     if (m0 >= used) return;
     const int e = find_expert(a.offsets, a.E, (int)m0);
-    A = a.A + m0 * a.K;
+    gathered = a.A == nullptr;
+    A = gathered ? a.Xg : a.A + m0 * a.K;
     B = a.B + (size_t)e * a.N * a.K;
     if (SWIGLU) B3 = a.B3 + (size_t)e * a.N * a.K;
     out_row0 = m0;
@@ -77,7 +81,16 @@ __global__ void __launch_bounds__(256) ffn_f32_kernel(F32GemmArgs a) {
       const int q = tid + i * 256;  // 0..1023 over a 64 x 16 tile
       const int r = q / kFBK, kk = q % kFBK;
       const int k = k0 + kk;
-      As[kk][r] = (r < a_rows_valid && k < a.K) ? A[(size_t)r * a.K + k] : 0.0f;
+      float av = 0.0f;
+      if (r < a_rows_valid && k < a.K) {
+        if (gathered) {
+          const int t = a.row_token[m0 + r];
+          if (t >= 0) av = A[(size_t)t * a.K + k];
+        } else {
+          av = A[(size_t)r * a.K + k];
+        }
+      }
+      As[kk][r] = av;
       const int c = n0 + r;
       Bs[kk][r] = (c < a.N && k < a.K) ? B[(size_t)c * a.K + k] : 0.0f;
       if (SWIGLU) B3s[kk][r] = (c < a.N && k < a.K) ? B3[(size_t)c * a.K + k] : 0.0f;
@@ -137,6 +150,8 @@ moe_status run_ffn_f32(const FfnArgs& f, cudaStream_t s) {
   const long long total_rows = f.rows_routed + (long long)f.n_shared * f.n_pad;
   F32GemmArgs up{};
   up.A = static_cast<const float*>(f.X_perm);
+  up.Xg = static_cast<const float*>(f.X);
+  up.row_token = f.row_token;
   up.A_shared = static_cast<const float*>(f.X);
   up.a_shared_base = 0;
   up.a_shared_stride = 0;

@@ -59,6 +59,7 @@ struct TcGemmParams {
   long long n_pad;
   __nv_bfloat16* out;       // [rows, n_out]
   int* err;
+  const int32_t* row_token;  // source token of each dispatched row (gathered A)
 };
 
 struct SharedState {
@@ -134,14 +135,15 @@ __device__ __forceinline__ float act_fn(float v) {
   return v;
 }
 
-template <int ACT>
+template <int ACT, bool GATHER>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,
                            const __grid_constant__ CUtensorMap tmA1,
                            const __grid_constant__ CUtensorMap tmB0,
                            const __grid_constant__ CUtensorMap tmB0g,
                            const __grid_constant__ CUtensorMap tmB1,
-                           const __grid_constant__ CUtensorMap tmB1g, const TcGemmParams p) {
+                           const __grid_constant__ CUtensorMap tmB1g,
+                           const __grid_constant__ CUtensorMap tmXg, const TcGemmParams p) {
   constexpr bool SWIGLU = ACT == ACT_SWIGLU;
   extern __shared__ __align__(1024) unsigned char gsm[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
@@ -184,38 +186,56 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int KB = p.K / kBK;
 
   if (warp == 0) {
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int issued = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-        const TileCoord c = decode_tile<ACT>(tile, p, st->offs, Tr);
-        const CUtensorMap* ma = c.a_sel ? &tmA1 : &tmA0;
-        const CUtensorMap* mb = c.b_sel ? &tmB1 : &tmB0;
-        const CUtensorMap* mbg = c.b_sel ? &tmB1g : &tmB0g;
-        for (int kb = 0; kb < KB; ++kb) {
-          if (!bounded_wait(&st->empty[stage], phase ^ 1u, st, p.err, kErrGemmTimeout | 0x01)) {
-            ok = false;
-            break;
-          }
+    // the whole warp walks the schedule; lane 0 waits and issues the 2-D
+    // loads, and with GATHER every lane issues one 4-row gather of A
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+      const TileCoord c = decode_tile<ACT>(tile, p, st->offs, Tr);
+      const CUtensorMap* ma = c.a_sel ? &tmA1 : &tmA0;
+      const CUtensorMap* mb = c.b_sel ? &tmB1 : &tmB0;
+      const CUtensorMap* mbg = c.b_sel ? &tmB1g : &tmB0g;
+      // routed rows straight from X: lane l brings rows 4l..4l+3 of the block;
+      // padding rows read token 0 and their outputs are never used
+      const bool gather = GATHER && c.a_sel == 0;
+      int tok[4] = {0, 0, 0, 0};
+      if (gather) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tok[j] = max(p.row_token[c.a_row + 4 * lane + j], 0);
+      }
+      for (int kb = 0; kb < KB; ++kb) {
+        int okw = 1;
+        if (lane == 0)
+          okw = bounded_wait(&st->empty[stage], phase ^ 1u, st, p.err, kErrGemmTimeout | 0x01);
+        if (!__shfl_sync(0xffffffffu, okw, 0)) {
+          ok = false;
+          break;
+        }
+        unsigned char* a_dst = sA + stage * kABytes;
+        unsigned char* b_dst = sB + stage * kBBytes;
+        if (lane == 0) {
           sm100::mbar_arrive_expect_tx(&st->full[stage], kStageBytes);
-          unsigned char* a_dst = sA + stage * kABytes;
-          unsigned char* b_dst = sB + stage * kBBytes;
-          sm100::tma_load_2d(a_dst, ma, &st->full[stage], kb * kBK, c.a_row);
+          if (!gather) sm100::tma_load_2d(a_dst, ma, &st->full[stage], kb * kBK, c.a_row);
           if (SWIGLU) {
             sm100::tma_load_2d(b_dst, mb, &st->full[stage], kb * kBK, c.b_row);
             sm100::tma_load_2d(b_dst + kBBytes / 2, mbg, &st->full[stage], kb * kBK, c.b_row);
           } else {
             sm100::tma_load_2d(b_dst, mb, &st->full[stage], kb * kBK, c.b_row);
           }
-          ++issued;
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
+        }
+        if (gather)
+          sm100::tma_gather4(a_dst + lane * 4 * (kBK * 2), &tmXg, &st->full[stage], kb * kBK,
+                             tok[0], tok[1], tok[2], tok[3]);
+        ++issued;
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
+    }
+    if (lane == 0) {
       if (!ok) {
         // wait (bounded) for the copies still in flight into our stages
         int s = stage;
@@ -440,7 +460,7 @@ __device__ __forceinline__ PairCoord decode_pair(int tile, const TcGemmParams& p
   return c;
 }
 
-template <int ACT>
+template <int ACT, bool GATHER>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     tc_grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0,
                                 const __grid_constant__ CUtensorMap tmA1,
@@ -448,6 +468,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                                 const __grid_constant__ CUtensorMap tmB0g,
                                 const __grid_constant__ CUtensorMap tmB1,
                                 const __grid_constant__ CUtensorMap tmB1g,
+                                const __grid_constant__ CUtensorMap tmXg,
                                 const TcGemmParams p) {
   constexpr bool SWIGLU = ACT == ACT_SWIGLU;
   extern __shared__ __align__(1024) unsigned char gsm[];
@@ -504,36 +525,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const int pair_id = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
 
   if (warp == 0) {
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int issued = 0;
-      bool ok = true;
-      for (int tile = pair_id; ok && tile < total; tile += num_pairs) {
-        const PairCoord c = decode_pair<ACT>(tile, p, st->offs, st->pprefix, Pr, rank);
-        const CUtensorMap* ma = c.a_sel ? &tmA1 : &tmA0;
-        const CUtensorMap* mb;
-        if (SWIGLU)
-          mb = leader ? (c.b_sel ? &tmB1 : &tmB0) : (c.b_sel ? &tmB1g : &tmB0g);
-        else
-          mb = c.b_sel ? &tmB1 : &tmB0;
-        for (int kb = 0; kb < KB; ++kb) {
-          if (!bounded_wait_pair<false>(&st->empty[stage], phase ^ 1u, st, p.err,
-                                        kErrGemmTimeout | 0x41)) {
-            ok = false;
-            break;
-          }
-          const uint32_t full_leader = sm100::mapa_shared(sm100::smem_addr(&st->full[stage]), 0);
+    // the whole warp walks the schedule; lane 0 waits and issues the 2-D
+    // loads, and with GATHER every lane issues one 4-row gather of A
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued = 0;
+    bool ok = true;
+    for (int tile = pair_id; ok && tile < total; tile += num_pairs) {
+      const PairCoord c = decode_pair<ACT>(tile, p, st->offs, st->pprefix, Pr, rank);
+      const CUtensorMap* ma = c.a_sel ? &tmA1 : &tmA0;
+      const CUtensorMap* mb;
+      if (SWIGLU)
+        mb = leader ? (c.b_sel ? &tmB1 : &tmB0) : (c.b_sel ? &tmB1g : &tmB0g);
+      else
+        mb = c.b_sel ? &tmB1 : &tmB0;
+      // routed rows straight from X: lane l brings rows 4l..4l+3 of the block;
+      // padding rows read token 0 and their outputs are never used
+      const bool gather = GATHER && c.a_sel == 0;
+      int tok[4] = {0, 0, 0, 0};
+      if (gather) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tok[j] = max(p.row_token[c.a_row + 4 * lane + j], 0);
+      }
+      for (int kb = 0; kb < KB; ++kb) {
+        int okw = 1;
+        if (lane == 0)
+          okw = bounded_wait_pair<false>(&st->empty[stage], phase ^ 1u, st, p.err,
+                                         kErrGemmTimeout | 0x41);
+        if (!__shfl_sync(0xffffffffu, okw, 0)) {
+          ok = false;
+          break;
+        }
+        const uint32_t full_leader = sm100::mapa_shared(sm100::smem_addr(&st->full[stage]), 0);
+        if (lane == 0) {
           if (leader) sm100::mbar_arrive_expect_tx(&st->full[stage], 2 * kPStageBytes);
-          sm100::tma_load_2d_pair(sA(stage), ma, full_leader, kb * kBK, c.a_row);
+          if (!gather) sm100::tma_load_2d_pair(sA(stage), ma, full_leader, kb * kBK, c.a_row);
           sm100::tma_load_2d_pair(sB(stage), mb, full_leader, kb * kBK, c.b_row);
-          ++issued;
-          if (++stage == kPStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
+        }
+        if (gather)
+          sm100::tma_gather4_pair(sA(stage) + lane * 4 * (kBK * 2), &tmXg, full_leader,
+                                  kb * kBK, tok[0], tok[1], tok[2], tok[3]);
+        ++issued;
+        if (++stage == kPStages) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
+    }
+    if (lane == 0) {
       if (!ok && leader) {
         // wait (bounded) until the copies of the outstanding stages have landed
         int s = stage;
@@ -703,28 +742,29 @@ static size_t gemm_smem_bytes(bool pair) {
 }
 
 struct Maps {
-  CUtensorMap a0, a1, b0, b0g, b1, b1g;
+  CUtensorMap a0, a1, b0, b0g, b1, b1g, xg;  // xg: X with a one-row box (gathered A)
 };
+
+template <class K>
+static cudaError_t launch_one(K kern, const Maps& m, const TcGemmParams& p, int ctas,
+                             size_t bytes, cudaStream_t s) {
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  kern<<<ctas, kGemmThreads, bytes, s>>>(m.a0, m.a1, m.b0, m.b0g, m.b1, m.b1g, m.xg, p);
+  return cudaGetLastError();
+}
 
 // grid: CTAs for the single-CTA kernel, CTA pairs for the pair kernel
 template <int ACT>
-static cudaError_t launch_gemm(const Maps& m, const TcGemmParams& p, bool pair, int grid,
-                               cudaStream_t s) {
+static cudaError_t launch_gemm(const Maps& m, const TcGemmParams& p, bool pair, bool gather,
+                               int grid, cudaStream_t s) {
   const size_t bytes = gemm_smem_bytes(pair);
-  if (pair) {
-    auto kern = tc_grouped_gemm_pair_kernel<ACT>;
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-    if (e != cudaSuccess) return e;
-    kern<<<2 * grid, kGemmThreads, bytes, s>>>(m.a0, m.a1, m.b0, m.b0g, m.b1, m.b1g, p);
-  } else {
-    auto kern = tc_grouped_gemm_kernel<ACT>;
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-    if (e != cudaSuccess) return e;
-    kern<<<grid, kGemmThreads, bytes, s>>>(m.a0, m.a1, m.b0, m.b0g, m.b1, m.b1g, p);
-  }
-  return cudaGetLastError();
+  if (pair)
+    return gather ? launch_one(tc_grouped_gemm_pair_kernel<ACT, true>, m, p, 2 * grid, bytes, s)
+                  : launch_one(tc_grouped_gemm_pair_kernel<ACT, false>, m, p, 2 * grid, bytes, s);
+  return gather ? launch_one(tc_grouped_gemm_kernel<ACT, true>, m, p, grid, bytes, s)
+                : launch_one(tc_grouped_gemm_kernel<ACT, false>, m, p, grid, bytes, s);
 }
 
 static int num_sms() {
@@ -765,7 +805,15 @@ moe_status run_ffn_bf16(const FfnArgs& f, cudaStream_t s) {
   const int b_box_dn = pair ? kBN / 2 : kBN;
   const int out_cols_up = swiglu ? kBN / 2 : kBN;
   Maps m;
-  if (!make_map(&m.a0, f.X_perm, rows, f.d, kBM)) return MOE_ERR_UNSUPPORTED;
+  const bool gather = f.X_perm == nullptr;  // A rows read from X through row_token
+  if (gather) {
+    // a box one row high: what a 4-row gather needs
+    if (!make_map(&m.xg, f.X, f.n, f.d, 1)) return MOE_ERR_UNSUPPORTED;
+    m.a0 = m.xg;  // unused for routed tiles when gathering
+  } else {
+    if (!make_map(&m.a0, f.X_perm, rows, f.d, kBM)) return MOE_ERR_UNSUPPORTED;
+    m.xg = m.a0;
+  }
   if (f.n_shared > 0) {
     if (!make_map(&m.a1, f.X, f.n, f.d, kBM)) return MOE_ERR_UNSUPPORTED;
   } else {
@@ -807,12 +855,13 @@ moe_status run_ffn_bf16(const FfnArgs& f, cudaStream_t s) {
   p.n_pad = f.n_pad;
   p.out = static_cast<__nv_bfloat16*>(f.H);
   p.err = f.err;
+  p.row_token = f.row_token;
   cudaError_t e;
   const int grid_up = persistent_grid(p, pair);
   switch (f.act) {
-    case MOE_ACT_RELU: e = launch_gemm<ACT_RELU>(m, p, pair, grid_up, s); break;
-    case MOE_ACT_GELU: e = launch_gemm<ACT_GELU>(m, p, pair, grid_up, s); break;
-    default: e = launch_gemm<ACT_SWIGLU>(m, p, pair, grid_up, s); break;
+    case MOE_ACT_RELU: e = launch_gemm<ACT_RELU>(m, p, pair, gather, grid_up, s); break;
+    case MOE_ACT_GELU: e = launch_gemm<ACT_GELU>(m, p, pair, gather, grid_up, s); break;
+    default: e = launch_gemm<ACT_SWIGLU>(m, p, pair, gather, grid_up, s); break;
   }
   if (e != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -829,6 +878,7 @@ moe_status run_ffn_bf16(const FfnArgs& f, cudaStream_t s) {
     dm.b1 = dm.b0;
   }
   dm.b1g = dm.b1;
+  dm.xg = dm.a0;
   TcGemmParams q = p;
   q.K = f.h;
   q.n_out = f.d;
@@ -837,7 +887,7 @@ moe_status run_ffn_bf16(const FfnArgs& f, cudaStream_t s) {
   q.a1_row_base = f.shared_base;
   q.a1_row_stride = f.n_pad;
   q.out = static_cast<__nv_bfloat16*>(f.Y);
-  e = launch_gemm<ACT_NONE>(dm, q, pair, persistent_grid(q, pair), s);
+  e = launch_gemm<ACT_NONE>(dm, q, pair, false, persistent_grid(q, pair), s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }

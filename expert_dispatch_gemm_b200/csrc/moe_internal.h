@@ -161,7 +161,8 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 
 struct FfnArgs {
   const void* X;        // [n, d] (shared experts read it)
-  const void* X_perm;   // [rows, d]
+  const void* X_perm;   // [rows, d], or NULL: routed rows are read from X via row_token
+  const int32_t* row_token;  // [rows] (needed when X_perm is NULL)
   const int32_t* offsets;
   const void *W1, *W3, *W2, *sW1, *sW3, *sW2;
   void* H;              // [rows, h]

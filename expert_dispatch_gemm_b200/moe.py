@@ -35,7 +35,7 @@ AUX_NAMES = ["lb_loss", "z_loss", "maxvio", "dropped_assignments", "tokens_some_
 API_SYMBOLS = ["moe_status_string", "moe_validate", "moe_sizes", "moe_workspace_size",
                "moe_route", "moe_route_from_scores", "moe_dispatch", "moe_expert_ffn",
                "moe_combine", "moe_layer_forward", "moe_bias_update", "moe_workspace_init",
-               "moe_read_error", "moe_route_noalloc"]
+               "moe_read_error", "moe_route_noalloc", "moe_expert_ffn_gathered"]
 MOE_ROUTE_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -94,6 +94,8 @@ def lib() -> ctypes.CDLL:
         L.moe_workspace_init.argtypes = [P, P]
         L.moe_read_error.argtypes = [P, P, ip]
         L.moe_route_noalloc.argtypes = [cfgp, P, P, P, P, outp, P]
+        L.moe_expert_ffn_gathered.argtypes = [cfgp, P, outp, P, P, P, P, P, P, P, P, P,
+                                              ctypes.c_size_t, P]
         for s in API_SYMBOLS[1:]:
             getattr(L, s).restype = ctypes.c_int
         _LIB = L
@@ -250,6 +252,14 @@ def moe_expert_ffn(cfg, X, X_perm, offsets, W1, W3, W2, sW1, sW3, sW2, H, Y_perm
                                 _ptr(W1), _ptr(W3), _ptr(W2), _ptr(sW1), _ptr(sW3), _ptr(sW2),
                                 _ptr(H), _ptr(Y_perm), _ptr(ws), ws.numel(), _stream(stream)),
            "moe_expert_ffn")
+
+
+def moe_expert_ffn_gathered(cfg, X, route: RouteBuffers, W1, W3, W2, sW1, sW3, sW2, H, Y_perm,
+                            ws, stream=None):
+    _check(lib().moe_expert_ffn_gathered(ctypes.byref(cfg), _ptr(X), ctypes.byref(route.c),
+                                         _ptr(W1), _ptr(W3), _ptr(W2), _ptr(sW1), _ptr(sW3),
+                                         _ptr(sW2), _ptr(H), _ptr(Y_perm), _ptr(ws), ws.numel(),
+                                         _stream(stream)), "moe_expert_ffn_gathered")
 
 
 def moe_combine(cfg, Y_perm, route: RouteBuffers, out, stream=None):

@@ -230,6 +230,23 @@ MOE_API moe_status moe_expert_ffn(const moe_config* cfg, const void* X, const vo
                           const void* sW2, void* H, void* Y_perm, void* ws,
                           size_t ws_bytes, moe_stream_t stream);
 
+/* moe_dispatch + moe_expert_ffn without X_perm: the first projection reads
+ * each routed row of X directly (row r of expert e's segment is
+ * X[route->row_token[r]]; padding rows read token 0 and are never used), so
+ * the gathered copy never goes through HBM ([EC-math] "The math": X_in[e] =
+ * P[e] X feeds Expert_e). Same weights, H, Y_perm and workspace as
+ * moe_expert_ffn; results are identical to dispatch followed by
+ * moe_expert_ffn. bf16 gathers with TMA tile::gather4 loads, 32 per 64-deep
+ * k-block of a 128-row tile: it saves X_perm's memory and HBM round trip but
+ * runs the first projection about 2x slower than the unfused pair on B200,
+ * so moe_layer_forward does not use it. */
+MOE_API moe_status moe_expert_ffn_gathered(const moe_config* cfg, const void* X,
+                                           const moe_route_out* route, const void* W1,
+                                           const void* W3, const void* W2, const void* sW1,
+                                           const void* sW3, const void* sW2, void* H,
+                                           void* Y_perm, void* ws, size_t ws_bytes,
+                                           moe_stream_t stream);
+
 /* Gate-scaled combine ([EC-math] "The math": Y[e] = G[e] * Expert_e(.),
  * out = scatter_add(Y, I)), computed owner-side: out[t] = sum over t's
  * tok_row entries of tok_gate * Y_perm[row] (+ each shared expert's row with
@@ -239,8 +256,8 @@ MOE_API moe_status moe_expert_ffn(const moe_config* cfg, const void* X, const vo
 MOE_API moe_status moe_combine(const moe_config* cfg, const void* Y_perm, const moe_route_out* route,
                        void* out, moe_stream_t stream);
 
-/* The whole layer: moe_route, moe_dispatch, moe_expert_ffn, moe_combine on
- * one stream, with X_perm / H / Y_perm inside the workspace (layer_bytes). */
+/* The whole layer on one stream: moe_route, moe_dispatch, moe_expert_ffn,
+ * moe_combine, with X_perm, H and Y_perm inside the workspace (layer_bytes). */
 MOE_API moe_status moe_layer_forward(const moe_config* cfg, const void* X, const float* Wg,
                              const float* logit_bias, const float* sel_bias,
                              const void* W1, const void* W3, const void* W2,

@@ -161,6 +161,42 @@ def test_stepwise_calls_equal_layer_forward():
     _ws_ok(ws)
 
 
+def _gathered_vs_unfused(w):
+    """moe_expert_ffn_gathered (rows read from X through row_token) against
+    moe_dispatch + moe_expert_ffn: same rows in, same arithmetic, so H and Y
+    must agree bit for bit on every real (non-padding) row."""
+    inp = wl.make_inputs(w, DEV)
+    cfg = moe.config(w)
+    sz = moe.sizes(cfg)
+    rb = moe.RouteBuffers(cfg, DEV)
+    ws = moe.workspace(cfg, DEV, layer=False)
+    dt = w.torch_dtype
+    X_perm = torch.empty((sz.rows, w.d), dtype=dt, device=DEV)
+    H1, H2 = (torch.empty((sz.rows, w.h), dtype=dt, device=DEV) for _ in range(2))
+    Y1, Y2 = (torch.empty((sz.rows, w.d), dtype=dt, device=DEV) for _ in range(2))
+    moe.moe_route(cfg, inp["X"], inp["Wg"], inp["logit_bias"], inp["sel_bias"], rb, ws)
+    moe.moe_dispatch(cfg, inp["X"], rb, X_perm)
+    args = (inp["W1"], inp.get("W3"), inp["W2"], inp.get("sW1"), inp.get("sW3"), inp.get("sW2"))
+    moe.moe_expert_ffn(cfg, inp["X"], X_perm, rb.offsets, *args, H1, Y1, ws)
+    moe.moe_expert_ffn_gathered(cfg, inp["X"], rb, *args, H2, Y2, ws)
+    torch.cuda.synchronize()
+    used = int(rb.offsets[-1])
+    real = torch.nonzero(rb.row_token[:used] >= 0).flatten()
+    if w.n_shared:
+        for s in range(w.n_shared):
+            base = sz.shared_row_base + s * ((w.n + 127) // 128 * 128)
+            real = torch.cat([real, torch.arange(base, base + w.n, device=DEV)])
+    assert real.numel() > 0
+    assert torch.equal(H1[real], H2[real])
+    assert torch.equal(Y1[real], Y2[real])
+    _ws_ok(ws)
+
+
+@pytest.mark.parametrize("w", wl.SMALL, ids=lambda w: w.name)
+def test_gathered_ffn_equals_dispatch_then_ffn(w):
+    _gathered_vs_unfused(w)
+
+
 # --------------------------------------------------------------------------
 # selection-bias steps ("4. Sigmoid gating with aux-loss-free bias")
 # --------------------------------------------------------------------------
@@ -249,6 +285,7 @@ EDGE = [
 @pytest.mark.parametrize("w", EDGE, ids=lambda w: w.name)
 def test_edge_cases(w):
     test_layer_small(w)
+    _gathered_vs_unfused(w)
 
 
 def test_capacity_one_all_equal_scores():
