@@ -53,10 +53,21 @@ def _opt(ptype):
     return _Opt
 
 
+_LIB_PATH_OVERRIDE = None
+
+
+def use_library(path):
+    """Load the oracle from another build of moe_oracle.c (the mutation tests
+    point this at a deliberately broken copy); None restores the default."""
+    global _LIB, _LIB_PATH_OVERRIDE
+    _LIB_PATH_OVERRIDE = path
+    _LIB = None
+
+
 def lib() -> ctypes.CDLL:
     global _LIB
     if _LIB is None:
-        path = _build()
+        path = _LIB_PATH_OVERRIDE or _build()
         L = ctypes.CDLL(path)
         c_int, c_float, c_double = ctypes.c_int, ctypes.c_float, ctypes.c_double
         L.orc_round_bf16.argtypes = [c_double]
