@@ -201,10 +201,11 @@ def run_gpu(args, w: wl.Workload):
     stream = torch.cuda.current_stream(dev)
     sb = inp["sel_bias"]
 
-    def step(ev=None, X=None):
+    def step(ev=None, X=None, out_buf=None):
         """One pass of the layer, the calls moe_layer_forward makes:
         route -> dispatch gather -> grouped expert FFN -> combine."""
         X = inp["X"] if X is None else X
+        o = out if out_buf is None else out_buf
         if ev: ev[0].record(stream)
         moe.moe_route(cfg, X, inp["Wg"], inp["logit_bias"], sb, rb, ws, stream)
         if ev: ev[1].record(stream)
@@ -213,7 +214,7 @@ def run_gpu(args, w: wl.Workload):
         moe.moe_expert_ffn(cfg, X, X_perm, rb.offsets, inp["W1"], inp["W3"], inp["W2"],
                            inp.get("sW1"), inp.get("sW3"), inp.get("sW2"), H, Y, ws, stream)
         if ev: ev[3].record(stream)
-        moe.moe_combine(cfg, Y, rb, out, stream)
+        moe.moe_combine(cfg, Y, rb, o, stream)
         if ev: ev[4].record(stream)
 
     for _ in range(args.warmup):
@@ -246,26 +247,48 @@ def run_gpu(args, w: wl.Workload):
     if st != moe.MOE_OK:
         raise RuntimeError(f"device error in the timed region: {detail:#x}")
 
-    # ---- end to end: pinned host input -> layer -> host output, every step
+    # ---- end to end: every step copies its input X from pinned host memory
+    # and its output back to pinned host memory, through the same public
+    # calls. The copies run on their own streams, double-buffered, so step
+    # i+1's input upload and step i-1's download overlap step i's compute.
     Xh = inp["X"].cpu().pin_memory()
-    outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    Xd = torch.empty_like(inp["X"])
-    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
-    for i in range(max(1, args.warmup)):
-        Xd.copy_(Xh, non_blocking=True)
-        step(X=Xd)
-        outh.copy_(out, non_blocking=True)
+    outh = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    Xd = [torch.empty_like(inp["X"]) for _ in range(2)]
+    outd = [torch.empty_like(out) for _ in range(2)]
+    up_s, down_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]     # upload of buffer b done
+    ev_used = [torch.cuda.Event() for _ in range(2)]   # compute done with buffer b
+    ev_out = [torch.cuda.Event() for _ in range(2)]    # download of buffer b done
+
+    def e2e_run(nsteps):
+        for i in range(nsteps):
+            b = i & 1
+            if i >= 2:
+                up_s.wait_event(ev_used[b])
+            with torch.cuda.stream(up_s):
+                Xd[b].copy_(Xh, non_blocking=True)
+            ev_in[b].record(up_s)
+            stream.wait_event(ev_in[b])
+            if i >= 2:
+                stream.wait_event(ev_out[b])
+            step(X=Xd[b], out_buf=outd[b])
+            ev_used[b].record(stream)
+            down_s.wait_event(ev_used[b])
+            with torch.cuda.stream(down_s):
+                outh[b].copy_(outd[b], non_blocking=True)
+            ev_out[b].record(down_s)
+
+    e2e_run(max(2, args.warmup))
     torch.cuda.synchronize(dev)
-    for i in range(args.steps):
-        flush.zero_()
-        e2e_ev[i][0].record(stream)
-        Xd.copy_(Xh, non_blocking=True)
-        step(X=Xd)
-        outh.copy_(out, non_blocking=True)
-        e2e_ev[i][1].record(stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    up_s.wait_event(e0)
+    e2e_run(args.steps)
+    stream.wait_event(ev_out[0])
+    stream.wait_event(ev_out[1])
+    e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = float(np.sum([a.elapsed_time(b) for a, b in e2e_ev]))
+    e2e_ms = e0.elapsed_time(e1)
     e2e_ms = max_over_ranks(e2e_ms, dev)
 
 
@@ -282,12 +305,20 @@ def run_gpu(args, w: wl.Workload):
         gbs = bytes_[nm] / (med[j] * 1e-3) / 1e9
         stages[nm] = {"ms": round(float(med[j]), 4), "GB/s": round(gbs, 1),
                       "hbm_frac": round(gbs / hbm, 3)}
+    # The burst tensor peak fits a GEMM that runs alone at full clock; when the
+    # power cap held the clocks down during the timed steps, the GEMM ran as
+    # part of a long power-capped loop and the sustained peak is the fair one.
+    clocks = clk.summary()
+    capped = "sw_power_cap" in clocks.get("reasons", [])
+    use_sust = bool(capped and tc_sust)
+    tc_peak = tc_sust if use_sust else tc_burst
+    tc_peak_kind = "sustained (sw_power_cap active)" if use_sust else "burst"
     ffn_tflops = flops / (med[2] * 1e-3) / 1e12
     stages["ffn"]["TFLOP/s"] = round(ffn_tflops, 1)
-    stages["ffn"]["tc_frac"] = round(ffn_tflops / tc_burst, 3)
+    stages["ffn"]["tc_frac"] = round(ffn_tflops / tc_peak, 3)
     # dominant kernel: the grouped GEMM (2 launches per step: up and down)
     t_hbm = bytes_["ffn"] / (hbm * 1e9)
-    t_tc = flops / (tc_burst * 1e12)
+    t_tc = flops / (tc_peak * 1e12)
     per_launch_ms = float(med[2]) / 2.0
     kernel_src = os.path.join(ROOT, "expert_dispatch_gemm_b200", "csrc", "gemm_tc.cu")
     traffic = traffic_for(kernel_src, w.name) if w.dtype == "bf16" else None
@@ -297,8 +328,9 @@ def run_gpu(args, w: wl.Workload):
                 "frac": round(ach / hbm, 3)}
     else:
         ach = flops / 2 / (per_launch_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": tc_burst,
-                "unit": "TFLOP/s", "frac": round(ach / tc_burst, 3)}
+        roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": tc_peak,
+                "unit": "TFLOP/s", "frac": round(ach / tc_peak, 3),
+                "peak_kind": tc_peak_kind}
     roof.update({"traffic": traffic, "kernel": "tc_grouped_gemm_kernel (up + down, avg)",
                  "peak_source": src,
                  "algorithmic_per_launch": bytes_["ffn"] / 2 if roof["bound"] == "hbm"
@@ -325,9 +357,11 @@ def run_gpu(args, w: wl.Workload):
         "stages": stages,
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(Xh.numel() * Xh.element_size()),
-                "d2h_bytes_per_step": int(outh.numel() * outh.element_size())},
+                "d2h_bytes_per_step": int(outh[0].numel() * outh[0].element_size()),
+                "note": "pinned host X -> device -> layer -> host out every step; copies "
+                        "double-buffered on their own streams; no L2 flush"},
         "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk.summary(),
+        "clocks": clocks,
         "wall_s_timed": round(t_wall, 4),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -30,8 +30,10 @@ __device__ __forceinline__ uint32_t ordered_key(float f) {
 // ---------------------------------------------------------------------------
 constexpr int kEcThreads = 1024;
 constexpr int kEcRankMax = 1024;
+constexpr int kEcMaxPerThread = MOE_EC_MAX_TOKENS / kEcThreads;  // 16 keys in registers
 
-// exclusive prefix sum over the CTA (threads in order); returns the total
+// exclusive prefix sum over the CTA (threads in order); returns the total.
+// The 32 warp totals are scanned with shuffles by every warp.
 __device__ __forceinline__ int block_exclusive_scan(int v, int* excl, int* warp_tot) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int incl = v;
@@ -42,13 +44,15 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* excl, int* warp_
   __syncthreads();  // warp_tot may still be read from a previous scan
   if (lane == 31) warp_tot[warp] = incl;
   __syncthreads();
-  int wbase = 0, total = 0;
   const int nw = blockDim.x >> 5;
-  for (int w = 0; w < nw; ++w) {
-    const int x = warp_tot[w];
-    if (w < warp) wbase += x;
-    total += x;
+  const int wt = lane < nw ? warp_tot[lane] : 0;
+  int winc = wt;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, winc, o);
+    if (lane >= o) winc += y;
   }
+  const int wbase = __shfl_sync(0xffffffffu, winc - wt, warp);
+  const int total = __shfl_sync(0xffffffffu, winc, 31);
   *excl = wbase + incl - v;
   return total;
 }
@@ -59,10 +63,9 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
   const bool by_rank = k <= kEcRankMax;
   int kp = 1;
   while (kp < k) kp <<= 1;
-  const int nbuf = by_rank ? k : kp;
-  uint64_t* sbuf = reinterpret_cast<uint64_t*>(ec_smem);                    // [nbuf]
-  uint64_t* sorted = by_rank ? sbuf + k : sbuf;                              // [k]
-  uint32_t* key = reinterpret_cast<uint32_t*>(sbuf + (by_rank ? 2 * k : kp));  // [n]
+  uint64_t* sbuf = reinterpret_cast<uint64_t*>(ec_smem);    // [k] picks, or [kp] to sort
+  uint64_t* sorted = by_rank ? sbuf + k : sbuf;              // [k]
+  int* whist = reinterpret_cast<int*>(sbuf + (by_rank ? 2 * k : kp));  // [32 warps][256]
   __shared__ int hist[256];
   __shared__ int warp_tot[32];
   __shared__ uint32_t s_prefix, s_mask;
@@ -70,10 +73,16 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int32_t* my_rows = a.ec_row + (size_t)e * n;
 
-  for (int t = tid; t < n; t += kEcThreads) {
-    key[t] = ordered_key(a.S[(size_t)t * E + e]);
-    my_rows[t] = -1;
+  // thread tid owns tokens [tid*C, tid*C + C), keys kept in registers
+  const int C = (n + kEcThreads - 1) / kEcThreads;
+  const int t0 = tid * C;
+  uint32_t kreg[kEcMaxPerThread];
+#pragma unroll
+  for (int i = 0; i < kEcMaxPerThread; ++i) {
+    const int t = t0 + i;
+    kreg[i] = (i < C && t < n) ? ordered_key(a.S[(size_t)t * E + e]) : 0u;
   }
+  for (int t = tid; t < n; t += kEcThreads) my_rows[t] = -1;
   if (tid == 0) {
     s_prefix = 0u;
     s_mask = 0u;
@@ -81,20 +90,23 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
   }
   __syncthreads();
 
+  int* myhist = whist + warp * 256;
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
-    for (int i = tid; i < 256; i += kEcThreads) hist[i] = 0;
-    __syncthreads();
+    for (int i = lane; i < 256; i += 32) myhist[i] = 0;
     const uint32_t prefix = s_prefix, mask = s_mask;
-    // keys share their leading digits, so aggregate per warp: one shared
-    // atomic per distinct digit instead of one per key
-    for (int t0 = 0; t0 < n; t0 += kEcThreads) {
-      const int t = t0 + tid;
-      const uint32_t u = t < n ? key[t] : 0u;
-      const bool cand = t < n && (u & mask) == prefix;
-      const int digit = cand ? (int)((u >> shift) & 255u) : 256 + lane;  // unique when idle
-      const unsigned peers = __match_any_sync(0xffffffffu, digit);
-      if (cand && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < kEcMaxPerThread; ++i) {
+      const int t = t0 + i;
+      if (i < C && t < n && (kreg[i] & mask) == prefix)
+        atomicAdd(&myhist[(kreg[i] >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    for (int b = tid; b < 256; b += kEcThreads) {
+      int c = 0;
+      for (int w = 0; w < kEcThreads / 32; ++w) c += whist[w * 256 + b];
+      hist[b] = c;
     }
     __syncthreads();
     if (warp == 0) {
@@ -135,32 +147,35 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
   const uint32_t T = s_prefix;
   const int need_eq = s_need;  // ties at T to take, lowest token first
 
-  // thread tid owns tokens [tid*C, tid*C + C): the ties' ranks in token order,
-  // then every pick's slot in token order
-  const int C = (n + kEcThreads - 1) / kEcThreads;
-  const int t0 = tid * C, t1 = min(n, t0 + C);
+  // the ties' ranks in token order, then every pick's slot in token order
   int my_eq = 0;
-  for (int t = t0; t < t1; ++t) my_eq += (key[t] == T);
+#pragma unroll
+  for (int i = 0; i < kEcMaxPerThread; ++i)
+    my_eq += (i < C && t0 + i < n && kreg[i] == T);
   int eq_base;
   block_exclusive_scan(my_eq, &eq_base, warp_tot);
   int my_sel = 0;
   {
     int rank = eq_base;
-    for (int t = t0; t < t1; ++t) {
-      const uint32_t u = key[t];
-      if (u > T) ++my_sel;
-      else if (u == T) my_sel += (rank++ < need_eq);
+#pragma unroll
+    for (int i = 0; i < kEcMaxPerThread; ++i) {
+      if (!(i < C && t0 + i < n)) continue;
+      if (kreg[i] > T) ++my_sel;
+      else if (kreg[i] == T) my_sel += (rank++ < need_eq);
     }
   }
   int slot;
   const int total = block_exclusive_scan(my_sel, &slot, warp_tot);
   {
     int rank = eq_base;
-    for (int t = t0; t < t1; ++t) {
-      const uint32_t u = key[t];
+#pragma unroll
+    for (int i = 0; i < kEcMaxPerThread; ++i) {
+      if (!(i < C && t0 + i < n)) continue;
+      const uint32_t u = kreg[i];
       bool sel = u > T;
       if (u == T) sel = rank++ < need_eq;
-      if (sel) sbuf[slot++] = ((uint64_t)u << 32) | (uint64_t)(0xffffffffu - (uint32_t)t);
+      if (sel)
+        sbuf[slot++] = ((uint64_t)u << 32) | (uint64_t)(0xffffffffu - (uint32_t)(t0 + i));
     }
   }
   if (total != k && tid == 0) report_error(a.err, kErrBadIndex | 1);
@@ -170,6 +185,7 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
     for (int j = tid; j < k; j += kEcThreads) {
       const uint64_t c = sbuf[j];
       int r = 0;
+#pragma unroll 8
       for (int i = 0; i < k; ++i) r += sbuf[i] > c;
       sorted[r] = c;
     }
@@ -229,10 +245,11 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
 }
 
 static size_t select_ec_smem(int n, int k) {
+  (void)n;
   int kp = 1;
   while (kp < k) kp <<= 1;
   const size_t buf = k <= kEcRankMax ? (size_t)2 * k * 8 : (size_t)kp * 8;
-  return buf + (size_t)n * 4;
+  return buf + (size_t)(kEcThreads / 32) * 256 * 4;
 }
 
 cudaError_t launch_select_ec(const SelectEcArgs& a, cudaStream_t s) {
@@ -250,15 +267,21 @@ cudaError_t launch_select_ec(const SelectEcArgs& a, cudaStream_t s) {
 // picked. A CTA transposes a [E, 32-token] tile of the slot map through
 // shared memory (coalesced reads), then one warp per token compacts it.
 __global__ void __launch_bounds__(256) ec_finish_kernel(EcFinishArgs a) {
-  __shared__ int rows_s[MOE_MAX_EXPERTS][33];
+  extern __shared__ __align__(16) unsigned char fin_smem[];
+  int* rows_s = reinterpret_cast<int*>(fin_smem);              // [E][33]
+  float* gates_s = reinterpret_cast<float*>(rows_s + a.E * 33);  // [E][33]
   __shared__ int hist_s[MOE_MAX_EXPERTS + 1];
   __shared__ int none_s;
   const int E = a.E, n = a.n, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int t0 = blockIdx.x * 32;
   for (int i = threadIdx.x; i <= E; i += blockDim.x) hist_s[i] = 0;
   if (threadIdx.x == 0) none_s = 0;
-  for (int e = warp; e < E; e += 8)
-    rows_s[e][lane] = t0 + lane < n ? a.ec_row[(size_t)e * n + t0 + lane] : -1;
+  for (int e = warp; e < E; e += 8) {
+    const bool in = t0 + lane < n;
+    const int r = in ? a.ec_row[(size_t)e * n + t0 + lane] : -1;
+    rows_s[e * 33 + lane] = r;
+    gates_s[e * 33 + lane] = r >= 0 ? a.ec_gate[(size_t)e * n + t0 + lane] : 0.0f;
+  }
   __syncthreads();
   for (int tt = warp; tt < 32; tt += 8) {
     const int t = t0 + tt;
@@ -266,12 +289,12 @@ __global__ void __launch_bounds__(256) ec_finish_kernel(EcFinishArgs a) {
     int base = 0;
     for (int c = 0; c < E; c += 32) {
       const int e = c + lane;
-      const int r = e < E ? rows_s[e][tt] : -1;
+      const int r = e < E ? rows_s[e * 33 + tt] : -1;
       const unsigned m = __ballot_sync(0xffffffffu, r >= 0);
       if (r >= 0) {
         const int p = base + __popc(m & ((1u << lane) - 1u));
         a.tok_row[(size_t)t * E + p] = r;
-        a.tok_gate[(size_t)t * E + p] = a.ec_gate[(size_t)e * n + t];
+        a.tok_gate[(size_t)t * E + p] = gates_s[e * 33 + tt];
       }
       base += __popc(m);
     }
@@ -293,7 +316,11 @@ __global__ void __launch_bounds__(256) ec_finish_kernel(EcFinishArgs a) {
 
 // (select_ec_kernel's block 0 has zeroed hist and the aux slots)
 cudaError_t launch_ec_finish(const EcFinishArgs& a, cudaStream_t s) {
-  ec_finish_kernel<<<ceil_div(a.n, 32), 256, 0, s>>>(a);
+  const size_t bytes = (size_t)a.E * 33 * 8;
+  cudaError_t e = cudaFuncSetAttribute(ec_finish_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  ec_finish_kernel<<<ceil_div(a.n, 32), 256, bytes, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -71,6 +71,7 @@ struct SharedState {
   uint32_t tmem_base;
   volatile int abort_flag;
   int offs[MOE_MAX_EXPERTS + 1];
+  int tprefix[MOE_MAX_EXPERTS + 1];  // tiles of the experts before e
 };
 
 __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, SharedState* st,
@@ -96,27 +97,38 @@ struct TileCoord {
   int col0;
 };
 
+// Tile schedule: expert by expert; inside an expert column block by column
+// block, and the expert's 128-row blocks innermost, so CTAs that run at the
+// same time share one weight tile (read from HBM once) instead of each
+// streaming a different one. Shared experts follow the routed ones.
 template <int ACT>
 __device__ __forceinline__ TileCoord decode_tile(int tile, const TcGemmParams& p,
-                                                 const int* offs, int Tr) {
+                                                 const int* offs, const int* tprefix,
+                                                 int routed_tiles) {
   constexpr int BNO = ACT == ACT_SWIGLU ? kBN / 2 : kBN;
   TileCoord c;
-  const int mt = tile / p.nt_tiles, nt = tile % p.nt_tiles;
-  if (mt < Tr) {
-    const int row = mt * kBM;
-    int lo = 0, hi = p.E - 1;  // largest e with offs[e] <= row
+  int nt;
+  if (tile < routed_tiles) {
+    int lo = 0, hi = p.E - 1;  // largest e with tprefix[e] <= tile
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (offs[mid] <= row) lo = mid; else hi = mid - 1;
+      if (tprefix[mid] <= tile) lo = mid; else hi = mid - 1;
     }
+    const int local = tile - tprefix[lo];
+    const int blocks = max((offs[lo + 1] - offs[lo]) / kBM, 1);
+    nt = local / blocks;
+    const int row = offs[lo] + (local % blocks) * kBM;
     c.a_sel = 0;
     c.a_row = row;
     c.b_sel = 0;
     c.b_row = lo * p.b_rows_per_expert;
     c.out_row = row;
   } else {
-    const int q = mt - Tr;
-    const int s = q / p.shared_tiles_per, lm = q % p.shared_tiles_per;
+    const int per = p.shared_tiles_per * p.nt_tiles;
+    const int q = tile - routed_tiles;
+    const int s = q / per, local = q % per;
+    nt = local / p.shared_tiles_per;
+    const int lm = local % p.shared_tiles_per;
     c.a_sel = 1;
     c.a_row = (int)(p.a1_row_base + s * p.a1_row_stride + (long long)lm * kBM);
     c.b_sel = 1;
@@ -154,7 +166,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int i = tid; i <= p.E; i += kGemmThreads) st->offs[i] = p.offsets[i];
+  __syncthreads();
   if (tid == 0) {
+    int run = 0;
+    for (int e = 0; e < p.E; ++e) {
+      st->tprefix[e] = run;
+      run += max(st->offs[e + 1] - st->offs[e], 0) / kBM * p.nt_tiles;
+    }
+    st->tprefix[p.E] = run;
     for (int s = 0; s < kStages; ++s) {
       sm100::mbar_init(&st->full[s], 1);
       sm100::mbar_init(&st->empty[s], 1);
@@ -181,8 +200,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   sm100::tc_fence_after();
   const uint32_t tmem = st->tmem_base;
 
-  const int Tr = min(max(st->offs[p.E], 0) / kBM, p.max_routed_tiles);
-  const int total = (Tr + p.n_shared * p.shared_tiles_per) * p.nt_tiles;
+  const int routed = min(st->tprefix[p.E], p.max_routed_tiles * p.nt_tiles);
+  const int total = routed + p.n_shared * p.shared_tiles_per * p.nt_tiles;
   const int KB = p.K / kBK;
 
   if (warp == 0) {
@@ -193,7 +212,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int issued = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-      const TileCoord c = decode_tile<ACT>(tile, p, st->offs, Tr);
+      const TileCoord c = decode_tile<ACT>(tile, p, st->offs, st->tprefix, routed);
       const CUtensorMap* ma = c.a_sel ? &tmA1 : &tmA0;
       const CUtensorMap* mb = c.b_sel ? &tmB1 : &tmB0;
       const CUtensorMap* mbg = c.b_sel ? &tmB1g : &tmB0g;
@@ -309,7 +328,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t acc_phase = (uint32_t)(local >> 1) & 1u;
       if (!bounded_wait(&st->tfull[acc], acc_phase, st, p.err, kErrGemmTimeout | 0x24)) break;
       sm100::tc_fence_after();
-      const TileCoord c = decode_tile<ACT>(tile, p, st->offs, Tr);
+      const TileCoord c = decode_tile<ACT>(tile, p, st->offs, st->tprefix, routed);
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN);
       __nv_bfloat16* orow = p.out + (size_t)(c.out_row + row_in_tile) * p.n_out;
 #pragma unroll 1
@@ -385,7 +404,7 @@ struct PairState {
   uint32_t tmem_base;
   volatile int abort_flag;
   int offs[MOE_MAX_EXPERTS + 1];
-  int pprefix[MOE_MAX_EXPERTS + 1];  // pair tiles of the experts before e
+  int tprefix[MOE_MAX_EXPERTS + 1];  // pair tiles of the experts before e
 };
 
 template <bool CLUSTER_ACQUIRE>
@@ -417,22 +436,25 @@ struct PairCoord {
   bool valid;
 };
 
+// Same schedule as decode_tile, over pairs of 128-row blocks.
 template <int ACT>
 __device__ __forceinline__ PairCoord decode_pair(int tile, const TcGemmParams& p,
-                                                 const int* offs, const int* pprefix, int Pr,
-                                                 uint32_t rank) {
+                                                 const int* offs, const int* tprefix,
+                                                 int routed_tiles, uint32_t rank) {
   constexpr int BNO = ACT == ACT_SWIGLU ? kBN / 2 : kBN;
   PairCoord c;
-  const int pt = tile / p.nt_tiles, nt = tile % p.nt_tiles;
-  int b_base;
-  if (pt < Pr) {
-    int lo = 0, hi = p.E - 1;  // largest e with pprefix[e] <= pt
+  int b_base, nt;
+  if (tile < routed_tiles) {
+    int lo = 0, hi = p.E - 1;  // largest e with tprefix[e] <= tile
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (pprefix[mid] <= pt) lo = mid; else hi = mid - 1;
+      if (tprefix[mid] <= tile) lo = mid; else hi = mid - 1;
     }
-    const int j = pt - pprefix[lo];
     const int cnt = (offs[lo + 1] - offs[lo]) / kBM;
+    const int pairs = max((cnt + 1) / 2, 1);
+    const int local = tile - tprefix[lo];
+    nt = local / pairs;
+    const int j = local % pairs;
     int mloc = 2 * j + (int)rank;
     c.valid = mloc < cnt;
     if (!c.valid) mloc = 2 * j;
@@ -444,8 +466,11 @@ __device__ __forceinline__ PairCoord decode_pair(int tile, const TcGemmParams& p
     b_base = lo * p.b_rows_per_expert;
   } else {
     const int spp = (p.shared_tiles_per + 1) / 2;
-    const int q = pt - Pr;
-    const int s = q / spp, jj = q % spp;
+    const int per = spp * p.nt_tiles;
+    const int q = tile - routed_tiles;
+    const int s = q / per, local = q % per;
+    nt = local / spp;
+    const int jj = local % spp;
     int lm = 2 * jj + (int)rank;
     c.valid = lm < p.shared_tiles_per;
     if (!c.valid) lm = 2 * jj;
@@ -486,11 +511,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   if (tid == 0) {
     int run = 0;
     for (int e = 0; e < p.E; ++e) {
-      st->pprefix[e] = run;
+      st->tprefix[e] = run;
       const int cnt = max(st->offs[e + 1] - st->offs[e], 0) / kBM;
-      run += (cnt + 1) / 2;
+      run += (cnt + 1) / 2 * p.nt_tiles;
     }
-    st->pprefix[p.E] = run;
+    st->tprefix[p.E] = run;
     for (int s = 0; s < kPStages; ++s) {
       sm100::mbar_init(&st->full[s], 1);
       sm100::mbar_init(&st->empty[s], 1);
@@ -518,9 +543,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   sm100::tc_fence_after();
   const uint32_t tmem = st->tmem_base;
 
-  const int Pr = min(st->pprefix[p.E], p.max_routed_tiles);
+  const int routed = min(st->tprefix[p.E], p.max_routed_tiles * p.nt_tiles);
   const int spp = (p.shared_tiles_per + 1) / 2;
-  const int total = (Pr + p.n_shared * spp) * p.nt_tiles;
+  const int total = routed + p.n_shared * spp * p.nt_tiles;
   const int KB = p.K / kBK;
   const int pair_id = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
 
@@ -532,7 +557,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     int issued = 0;
     bool ok = true;
     for (int tile = pair_id; ok && tile < total; tile += num_pairs) {
-      const PairCoord c = decode_pair<ACT>(tile, p, st->offs, st->pprefix, Pr, rank);
+      const PairCoord c = decode_pair<ACT>(tile, p, st->offs, st->tprefix, routed, rank);
       const CUtensorMap* ma = c.a_sel ? &tmA1 : &tmA0;
       const CUtensorMap* mb;
       if (SWIGLU)
@@ -645,7 +670,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                                    kErrGemmTimeout | 0x64))
         break;
       sm100::tc_fence_after();
-      const PairCoord c = decode_pair<ACT>(tile, p, st->offs, st->pprefix, Pr, rank);
+      const PairCoord c = decode_pair<ACT>(tile, p, st->offs, st->tprefix, routed, rank);
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN);
       __nv_bfloat16* orow = p.out + (size_t)(c.out_row + row_in_tile) * p.n_out;
       if (c.valid) {
