@@ -157,6 +157,32 @@ class ClockSampler:
 # GPU arm
 # ---------------------------------------------------------------------------
 
+def ffma_peak_tflops(dev) -> float:
+    """FP32 FFMA throughput of this device, measured with the probe kernel in
+    libmoe_probe.so (the router's roof; not among the measured HBM / tensor
+    peaks). Median of 5 timed launches after 2 warm-ups."""
+    import ctypes
+    lib = ctypes.CDLL(os.path.join(ROOT, "expert_dispatch_gemm_b200", "libmoe_probe.so"))
+    lib.moe_probe_ffma.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    blocks, iters = sms * 8, 2048
+    out = torch.empty(blocks, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    times = []
+    for i in range(7):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        rc = lib.moe_probe_ffma(blocks, iters, out.data_ptr(), ctypes.c_void_p(stream.cuda_stream))
+        e1.record(stream)
+        if rc != 0:
+            raise RuntimeError(f"FFMA probe launch failed: {rc}")
+        torch.cuda.synchronize(dev)
+        if i >= 2:
+            times.append(e0.elapsed_time(e1))
+    flops = 2.0 * blocks * 256 * iters * 16
+    return flops / (float(np.median(times)) * 1e-3) / 1e12
+
+
 def traffic_for(kernel_src: str, workload: str):
     """DRAM bytes per launch of the grouped GEMM from the committed ncu summary,
     or None when the device code changed since that capture (the hash covers
@@ -225,7 +251,7 @@ def run_gpu(args, w: wl.Workload):
     if st != moe.MOE_OK:
         raise RuntimeError(f"device error after warm-up: {detail:#x}")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -233,16 +259,26 @@ def run_gpu(args, w: wl.Workload):
         t_wall0 = time.perf_counter()
         for i in range(args.steps):
             flush.zero_()  # outside the timed events: L2 starts cold every step
-            step(evs[i])
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
         torch.cuda.synchronize(dev)
         t_wall = time.perf_counter() - t_wall0
     if world > 1:
         dist.barrier()
-    stage_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)]
-                         for i in range(args.steps)])
-    step_ms = stage_ms.sum(1)
+    step_ms = np.array([evs[i][0].elapsed_time(evs[i][1]) for i in range(args.steps)])
     total_ms = float(step_ms.sum())
     total_ms = max_over_ranks(total_ms, dev)
+    # per-stage breakdown: a second pass with an event between the stages
+    # (those events keep a stage's kernels from overlapping the previous
+    # stage's tail, so the stages add up to a little more than a step)
+    sevs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        step(sevs[i])
+    torch.cuda.synchronize(dev)
+    stage_ms = np.array([[sevs[i][j].elapsed_time(sevs[i][j + 1]) for j in range(4)]
+                         for i in range(args.steps)])
     st, detail = moe.moe_read_error(ws)
     if st != moe.MOE_OK:
         raise RuntimeError(f"device error in the timed region: {detail:#x}")
@@ -313,6 +349,14 @@ def run_gpu(args, w: wl.Workload):
     use_sust = bool(capped and tc_sust)
     tc_peak = tc_sust if use_sust else tc_burst
     tc_peak_kind = "sustained (sw_power_cap active)" if use_sust else "burst"
+    # the router contraction runs on FP32 FFMA: its roof is that pipe, taken
+    # here over the whole route stage (router + selection kernels)
+    ffma_peak = ffma_peak_tflops(dev)
+    router_flops = 2.0 * w.n * w.d * w.E
+    route_tflops = router_flops / (med[0] * 1e-3) / 1e12
+    stages["route"].update({"router_FLOP": router_flops, "FFMA_TFLOP/s": round(route_tflops, 2),
+                            "ffma_peak_TFLOP/s": round(ffma_peak, 1),
+                            "ffma_frac": round(route_tflops / ffma_peak, 3)})
     ffn_tflops = flops / (med[2] * 1e-3) / 1e12
     stages["ffn"]["TFLOP/s"] = round(ffn_tflops, 1)
     stages["ffn"]["tc_frac"] = round(ffn_tflops / tc_peak, 3)
@@ -355,6 +399,8 @@ def run_gpu(args, w: wl.Workload):
                    "l2": "flushed between timed steps (256 MB write, outside the events)"},
         "roofline": roof,
         "stages": stages,
+        "stages_note": "medians of a second pass with an event between stages; value and "
+                       "ms_per_step come from whole-step events",
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(Xh.numel() * Xh.element_size()),
                 "d2h_bytes_per_step": int(outh[0].numel() * outh[0].element_size()),

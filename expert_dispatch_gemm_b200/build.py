@@ -3,7 +3,9 @@
     python -m expert_dispatch_gemm_b200.build [--force] [--verbose-ptxas]
 
 Objects go to expert_dispatch_gemm_b200/_build/, the shared library to
-expert_dispatch_gemm_b200/libmoe.so. No GPU is needed to build.
+expert_dispatch_gemm_b200/libmoe.so. The FP32 FFMA throughput probe that the
+benchmark uses for the router's roof goes to libmoe_probe.so. No GPU is
+needed to build.
 """
 from __future__ import annotations
 
@@ -21,6 +23,8 @@ INCLUDE = os.path.join(ROOT, "include")
 
 SOURCES = ["api.cu", "router.cu", "assign.cu", "dispatch_combine.cu", "ffn_f32.cu",
            "gemm_tc.cu", "route_noalloc.cu"]
+PROBE_SOURCES = ["probe.cu"]
+PROBE_LIB = os.path.join(PKG, "libmoe_probe.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -42,10 +46,16 @@ def _flags(extra=()):
 
 
 def build(force: bool = False, ptxas_verbose: bool = False) -> str:
+    lib = _build_lib(SOURCES, LIB, force, ptxas_verbose)
+    _build_lib(PROBE_SOURCES, PROBE_LIB, force, ptxas_verbose)
+    return lib
+
+
+def _build_lib(sources, out_lib, force, ptxas_verbose) -> str:
     os.makedirs(BUILD, exist_ok=True)
     hdr_t = max(os.path.getmtime(h) for h in _headers())
     jobs = []
-    for src in SOURCES:
+    for src in sources:
         s = os.path.join(CSRC, src)
         o = os.path.join(BUILD, src.replace(".cu", ".o"))
         if force or ptxas_verbose or not os.path.exists(o) or \
@@ -61,13 +71,13 @@ def build(force: bool = False, ptxas_verbose: bool = False) -> str:
                 sys.stderr.write(r.stdout + r.stderr)
             if r.returncode != 0:
                 raise RuntimeError("nvcc failed: " + " ".join(cmd))
-    objs = [os.path.join(BUILD, s.replace(".cu", ".o")) for s in SOURCES]
-    if force or jobs or not os.path.exists(LIB) or \
-            os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
-        cmd = [nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", LIB + ".tmp", *objs]
+    objs = [os.path.join(BUILD, s.replace(".cu", ".o")) for s in sources]
+    if force or jobs or not os.path.exists(out_lib) or \
+            os.path.getmtime(out_lib) < max(os.path.getmtime(o) for o in objs):
+        cmd = [nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", out_lib + ".tmp", *objs]
         subprocess.check_call(cmd)
-        os.replace(LIB + ".tmp", LIB)
-    return LIB
+        os.replace(out_lib + ".tmp", out_lib)
+    return out_lib
 
 
 if __name__ == "__main__":

@@ -297,17 +297,27 @@ static moe_status ffn_impl(const moe_config* c, const Derived& dv, const void* X
   return c->dtype == MOE_BF16 ? run_ffn_bf16(f, s) : run_ffn_f32(f, s);
 }
 
+// err: the workspace error word, or NULL (standalone moe_dispatch)
 static moe_status dispatch_impl(const moe_config* c, const Derived& dv, const void* X,
-                                const moe_route_out* o, void* X_perm, cudaStream_t s) {
+                                const moe_route_out* o, void* X_perm, int* err,
+                                cudaStream_t s) {
+  if ((reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(X_perm)) & 15)
+    return MOE_ERR_INVALID_ARG;
   GatherArgs g{};
   g.X = X;
+  g.tok_row = o->tok_row;
   g.row_token = o->row_token;
   g.offsets = o->offsets;
   g.E = c->E;
-  g.d = c->d;
-  g.elt_bytes = c->dtype == MOE_BF16 ? 2 : 4;
+  g.n = c->n;
+  g.fanout = c->mode == MOE_TOKEN_CHOICE
+                 ? dv.k
+                 : (int)(((long long)dv.k * c->E + c->n - 1) / c->n);
+  g.slots = dv.slots;
+  g.row_bytes = c->d * (c->dtype == MOE_BF16 ? 2 : 4);
   g.max_rows = dv.rows_routed;
   g.X_perm = X_perm;
+  g.err = err;
   MOE_CU(launch_gather(g, s));
   return MOE_OK;
 }
@@ -432,9 +442,9 @@ moe_status moe_dispatch(const moe_config* cfg, const void* X, const moe_route_ou
   Derived d;
   moe_status st = derive(cfg, &d);
   if (st != MOE_OK) return st;
-  if (!X || !X_perm || !route || !route->row_token || !route->offsets)
+  if (!X || !X_perm || !route || !route->tok_row || !route->row_token || !route->offsets)
     return MOE_ERR_INVALID_ARG;
-  return dispatch_impl(cfg, d, X, route, X_perm, (cudaStream_t)stream);
+  return dispatch_impl(cfg, d, X, route, X_perm, nullptr, (cudaStream_t)stream);
 }
 
 moe_status moe_expert_ffn(const moe_config* cfg, const void* X, const void* X_perm,
@@ -482,7 +492,7 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* X, const float* 
   // the gather stays a separate pass: fused into the GEMM's A loads it costs
   // 32 four-row TMA gathers per 64-deep k-block, which the TMA unit issues
   // far slower than the two box loads the unfused GEMM needs
-  if ((st = dispatch_impl(cfg, d, X, route, xp, s)) != MOE_OK) return st;
+  if ((st = dispatch_impl(cfg, d, X, route, xp, at<int>(ws, w.err), s)) != MOE_OK) return st;
   if ((st = ffn_impl(cfg, d, X, xp, nullptr, route->offsets, W1, W3, W2, sW1, sW3, sW2, hb, yp,
                      at<int>(ws, w.err), s)) != MOE_OK)
     return st;
@@ -530,6 +540,7 @@ moe_status moe_read_error(void* ws, moe_stream_t stream, int* detail) {
   const int zero = 0;
   if (cudaMemcpy(ws, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
     return MOE_ERR_CUDA;
+  if (code == 0) code = take_dispatch_error();
   if (detail) *detail = code;
   if (code == 0) return MOE_OK;
   return (code & 0xF00) == kErrGemmTimeout ? MOE_ERR_TIMEOUT : MOE_ERR_CUDA;

@@ -58,6 +58,8 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* excl, int* warp_
 }
 
 __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(16) unsigned char ec_smem[];
   const int n = a.n, E = a.E, k = a.k, e = blockIdx.x;
   const bool by_rank = k <= kEcRankMax;
@@ -258,8 +260,7 @@ cudaError_t launch_select_ec(const SelectEcArgs& a, cudaStream_t s) {
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)bytes);
   if (err != cudaSuccess) return err;
-  select_ec_kernel<<<a.E, kEcThreads, bytes, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(select_ec_kernel, a.E, kEcThreads, bytes, s, a);
 }
 
 // Expert choice: each token's picks (expert order) compacted into its slot
@@ -267,6 +268,8 @@ cudaError_t launch_select_ec(const SelectEcArgs& a, cudaStream_t s) {
 // picked. A CTA transposes a [E, 32-token] tile of the slot map through
 // shared memory (coalesced reads), then one warp per token compacts it.
 __global__ void __launch_bounds__(256) ec_finish_kernel(EcFinishArgs a) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(16) unsigned char fin_smem[];
   int* rows_s = reinterpret_cast<int*>(fin_smem);              // [E][33]
   float* gates_s = reinterpret_cast<float*>(rows_s + a.E * 33);  // [E][33]
@@ -320,8 +323,7 @@ cudaError_t launch_ec_finish(const EcFinishArgs& a, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(ec_finish_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
-  ec_finish_kernel<<<ceil_div(a.n, 32), 256, bytes, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(ec_finish_kernel, ceil_div(a.n, 32), 256, bytes, s, a);
 }
 
 // ---------------------------------------------------------------------------
@@ -329,6 +331,8 @@ cudaError_t launch_ec_finish(const EcFinishArgs& a, cudaStream_t s) {
 // offsets, aux), then arrival positions, drops and slot lists.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kTokBlock) tc_hist_kernel(TcAssignArgs a) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int hist[MOE_MAX_EXPERTS];
   for (int i = threadIdx.x; i < a.E; i += kTokBlock) hist[i] = 0;
   __syncthreads();
@@ -344,6 +348,8 @@ __global__ void __launch_bounds__(kTokBlock) tc_hist_kernel(TcAssignArgs a) {
 }
 
 __global__ void __launch_bounds__(1024) tc_scan_kernel(TcAssignArgs a) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int seg[MOE_MAX_EXPERTS];
   __shared__ int off[MOE_MAX_EXPERTS + 1];
   __shared__ double fp[MOE_MAX_EXPERTS];
@@ -412,6 +418,8 @@ __global__ void __launch_bounds__(1024) tc_scan_kernel(TcAssignArgs a) {
 }
 
 __global__ void __launch_bounds__(kTokBlock) tc_scatter_kernel(TcAssignArgs a) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(16) unsigned char sc_smem[];
   const int E = a.E, K = a.K;
   uint32_t* mask = reinterpret_cast<uint32_t*>(sc_smem);      // [32][E]
@@ -476,18 +484,15 @@ __global__ void __launch_bounds__(kTokBlock) tc_scatter_kernel(TcAssignArgs a) {
 }
 
 cudaError_t launch_tc_assign(const TcAssignArgs& a, cudaStream_t s) {
-  tc_hist_kernel<<<a.tok_blocks, kTokBlock, 0, s>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(tc_hist_kernel, a.tok_blocks, kTokBlock, 0, s, a);
   if (e != cudaSuccess) return e;
-  tc_scan_kernel<<<1, 1024, 0, s>>>(a);
-  e = cudaGetLastError();
+  e = launch_pdl(tc_scan_kernel, 1, 1024, 0, s, a);
   if (e != cudaSuccess) return e;
   const size_t bytes = (size_t)64 * a.E * 4;
   e = cudaFuncSetAttribute(tc_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)bytes);
   if (e != cudaSuccess) return e;
-  tc_scatter_kernel<<<a.tok_blocks, kTokBlock, bytes, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(tc_scatter_kernel, a.tok_blocks, kTokBlock, bytes, s, a);
 }
 
 }  // namespace moe

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace moe {
 
 // Device error codes written to the workspace error word.
@@ -13,6 +15,34 @@ enum : int {
   kErrGemmTimeout = 0x100,   // | role << 4 | which barrier
   kErrBadIndex = 0x200,
 };
+
+// Programmatic dependent launch. Every kernel of the library is launched
+// with programmatic stream serialisation (launch_pdl): it may start while the
+// previous kernel in the stream is finishing, so it calls pdl_wait() before
+// it touches anything that kernel wrote (the wait returns once the previous
+// grid has completed and its writes are visible; every kernel waits, so the
+// order is transitive). pdl_trigger() lets the next kernel's CTAs be
+// scheduled early, as this kernel's CTAs leave their SMs.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 __device__ __forceinline__ void report_error(int* err, int code) {
   if (err) atomicCAS(err, 0, code);

@@ -8,42 +8,194 @@
 // and the result does not depend on scheduling.
 #include "device_common.cuh"
 #include "moe_internal.h"
+#include "sm100.cuh"
 
 namespace moe {
 
-// One warp per dispatched row, 16-byte vectors, four in flight per lane.
-__global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
-  const int rows = min((long long)a.offsets[a.E], a.max_rows);
+// ---------------------------------------------------------------------------
+// Dispatch gather, token by token, with TMA row staging. Each warp runs its
+// own ring of row buffers in shared memory. Lane 0 brings a token's row (or
+// one segment of a long row) in with one bulk copy that completes on the
+// slot's mbarrier; then each lane that holds one of the token's dispatched
+// rows (tok_row: kept entries first, then -1) writes the staged bytes there
+// with a bulk copy out of shared memory. X is read from HBM once, every
+// dispatched row is written once, and the copy engine moves all the bytes.
+// Loads run ring - 1 units ahead of the stores. The slot wait is bounded: on
+// a timeout the warp records an error, waits (bounded) for its own loads
+// still in flight, and stops.
+// ---------------------------------------------------------------------------
+constexpr int kGatherSeg = 16384;   // largest staged unit, bytes
+constexpr int kGatherMaxRing = 8;
+constexpr int kGatherMaxWarps = 8;
+constexpr size_t kGatherSmemBudget = 200 * 1024;
+constexpr uint64_t kGatherWaitNs = 2000000000ull;  // 2 s
+constexpr int kGatherRowRegs = MOE_MAX_EXPERTS / 32;
+// average rows per token from which the staged kernel is used (measured on
+// B200: it wins at 8 rows per token, loses at 2)
+constexpr int kGatherStagedFanout = 4;
+
+__device__ int g_dispatch_error;  // timeouts of standalone dispatch calls
+
+__global__ void gather_kernel(GatherArgs a, int seg, int nseg, int ring, int slot_stride) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ __align__(128) unsigned char gsm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  unsigned char* buf = gsm + (size_t)warp * ring * slot_stride;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(gsm + (size_t)warps * ring * slot_stride) +
+                  warp * kGatherMaxRing;
+  int* err = a.err ? a.err : &g_dispatch_error;
+  if (lane == 0) {
+    for (int i = 0; i < ring; ++i) sm100::mbar_init(&bar[i], 1);
+    sm100::fence_mbar_init();
+  }
+  __syncwarp();
+  const int row_bytes = a.row_bytes;
+  const long long units = (long long)a.n * nseg;
+  const long long first = (long long)blockIdx.x * warps + warp;
+  const long long stride = (long long)gridDim.x * warps;
+  const unsigned char* X = static_cast<const unsigned char*>(a.X);
+  unsigned char* XP = static_cast<unsigned char*>(a.X_perm);
+  auto unit_bytes = [&](int sg) { return (uint32_t)min(seg, row_bytes - sg * seg); };
+  auto issue = [&](long long i) {  // lane 0: stage unit i of this warp
+    const long long u = first + i * stride;
+    if (u >= units) return;
+    const int t = (int)(u / nseg), sg = (int)(u % nseg);
+    const int slot = (int)(i % ring);
+    const uint32_t b = unit_bytes(sg);
+    sm100::mbar_arrive_expect_tx(&bar[slot], b);
+    sm100::bulk_load_smem(buf + (size_t)slot * slot_stride,
+                          X + (size_t)t * row_bytes + (size_t)sg * seg, b, &bar[slot]);
+  };
+  if (lane == 0)
+    for (int i = 0; i < ring - 1; ++i) issue(i);
+  long long i = 0;
+  bool ok = true;
+  for (; first + i * stride < units; ++i) {
+    const long long u = first + i * stride;
+    const int t = (int)(u / nseg), sg = (int)(u % nseg);
+    const int slot = (int)(i % ring);
+    const uint32_t parity = (uint32_t)((i / ring) & 1);
+    int rr[kGatherRowRegs];
+#pragma unroll
+    for (int c = 0; c < kGatherRowRegs; ++c) {
+      const int j = c * 32 + lane;
+      rr[c] = j < a.slots ? a.tok_row[(size_t)t * a.slots + j] : -1;
+    }
+    // refill the slot unit i - 1 used: its stores finished reading it
+    if (lane == 0) issue(i + ring - 1);
+    int okw = 1;
+    if (lane == 0) {
+      if (!sm100::mbar_try_wait(&bar[slot], parity)) {
+        const uint64_t t0 = global_timer_ns();
+        while (!sm100::mbar_try_wait(&bar[slot], parity)) {
+          if (global_timer_ns() - t0 > kGatherWaitNs) {
+            report_error(err, kErrGemmTimeout | 0x50);
+            okw = 0;
+            break;
+          }
+        }
+      }
+    }
+    if (!__shfl_sync(0xffffffffu, okw, 0)) {
+      ok = false;
+      break;
+    }
+    sm100::fence_proxy_async_smem();
+    const unsigned char* src = buf + (size_t)slot * slot_stride;
+    const uint32_t b = unit_bytes(sg);
+#pragma unroll
+    for (int c = 0; c < kGatherRowRegs; ++c) {
+      const int r = rr[c];
+      if (r >= 0 && r < a.max_rows)
+        sm100::bulk_store_global(XP + (size_t)r * row_bytes + (size_t)sg * seg, src, b);
+    }
+    sm100::bulk_commit_group();
+    sm100::bulk_wait_read_all();
+    __syncwarp();
+  }
+  if (!ok && lane == 0) {
+    // wait (bounded) for the loads this warp still has in flight
+    for (long long q = i; q < i + ring - 1 + 1 && first + q * stride < units; ++q) {
+      const uint64_t t0 = global_timer_ns();
+      while (!sm100::mbar_try_wait(&bar[q % ring], (uint32_t)((q / ring) & 1)) &&
+             global_timer_ns() - t0 < kGatherWaitNs) {
+      }
+    }
+  }
+  sm100::bulk_wait_all();
+}
+
+// Low fan-out (a token feeds one or two rows on average): one warp per
+// dispatched row, 16-byte vectors, four in flight per lane. A token's row is
+// then read about once anyway, and every row gets its own warp at once,
+// where the staged kernel would serialise a few round trips per warp.
+__global__ void __launch_bounds__(256) gather_rows_kernel(GatherArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  const long long rows = min((long long)a.offsets[a.E], a.max_rows);
   const int lane = threadIdx.x & 31;
-  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int nw = (gridDim.x * blockDim.x) >> 5;
-  const int nvec = a.d * a.elt_bytes / 16;
+  const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  const int nvec = a.row_bytes / 16;
   const uint4* src = reinterpret_cast<const uint4*>(a.X);
   uint4* dst = reinterpret_cast<uint4*>(a.X_perm);
-  for (int r = gw; r < rows; r += nw) {
+  for (long long r = gw; r < rows; r += nw) {
     const int t = a.row_token[r];
-    if (t < 0) continue;
-    const uint4* s = src + (size_t)t * nvec;
+    if (t < 0 || t >= a.n) continue;
+    const uint4* sp = src + (size_t)t * nvec;
     uint4* o = dst + (size_t)r * nvec;
     int v = lane;
     for (; v + 96 < nvec; v += 128) {
-      const uint4 x0 = __ldg(s + v), x1 = __ldg(s + v + 32), x2 = __ldg(s + v + 64),
-                  x3 = __ldg(s + v + 96);
+      const uint4 x0 = __ldg(sp + v), x1 = __ldg(sp + v + 32), x2 = __ldg(sp + v + 64),
+                  x3 = __ldg(sp + v + 96);
       o[v] = x0;
       o[v + 32] = x1;
       o[v + 64] = x2;
       o[v + 96] = x3;
     }
-    for (; v < nvec; v += 32) o[v] = __ldg(s + v);
+    for (; v < nvec; v += 32) o[v] = __ldg(sp + v);
   }
 }
 
+int take_dispatch_error() {
+  int code = 0;
+  if (cudaMemcpyFromSymbol(&code, g_dispatch_error, sizeof(int)) != cudaSuccess) return 0;
+  if (code) {
+    const int zero = 0;
+    cudaMemcpyToSymbol(g_dispatch_error, &zero, sizeof(int));
+  }
+  return code;
+}
+
 cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s) {
-  int dev = 0, sms = 148;
+  if (a.row_bytes <= 0 || a.row_bytes % 16 || a.n < 1) return cudaErrorInvalidValue;
+  if (a.fanout < kGatherStagedFanout) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return launch_pdl(gather_rows_kernel, sms * 8, 256, 0, s, a);
+  }
+  const int nseg = (a.row_bytes + kGatherSeg - 1) / kGatherSeg;
+  const int seg = ((a.row_bytes + nseg - 1) / nseg + 15) / 16 * 16;
+  if ((long long)(nseg - 1) * seg >= a.row_bytes) return cudaErrorInvalidValue;
+  const int slot_stride = (seg + 127) / 128 * 128;
+  int ring = (int)(kGatherSmemBudget / ((size_t)kGatherMaxWarps * slot_stride));
+  ring = ring < 2 ? 2 : ring > kGatherMaxRing ? kGatherMaxRing : ring;
+  int warps = (int)(kGatherSmemBudget / ((size_t)ring * slot_stride));
+  warps = warps < 1 ? 1 : warps > kGatherMaxWarps ? kGatherMaxWarps : warps;
+  const size_t smem = (size_t)warps * ring * slot_stride + (size_t)warps * kGatherMaxRing * 8;
+  int dev = 0, sms = 148, max_smem = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  gather_kernel<<<sms * 8, 256, 0, s>>>(a);
-  return cudaGetLastError();
+  cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+  cudaError_t e = cudaFuncSetAttribute(gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  int per_sm = (int)(max_smem / (smem + 1024));
+  per_sm = per_sm < 1 ? 1 : per_sm > 4 ? 4 : per_sm;
+  return launch_pdl(gather_kernel, sms * per_sm, warps * 32, smem, s, a, seg, nseg, ring, slot_stride);
 }
 
 // One CTA per token; each thread owns 16-byte chunks of the output row and
@@ -51,6 +203,8 @@ cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s) {
 // experts with weight 1.
 template <bool BF16>
 __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int rows_s[MOE_MAX_EXPERTS];
   __shared__ float gates_s[MOE_MAX_EXPERTS];
   __shared__ int cnt_s;
@@ -110,10 +264,8 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
   if (a.bf16)
-    combine_kernel<true><<<a.n, 128, 0, s>>>(a);
-  else
-    combine_kernel<false><<<a.n, 128, 0, s>>>(a);
-  return cudaGetLastError();
+    return launch_pdl(combine_kernel<true>, a.n, 128, 0, s, a);
+  return launch_pdl(combine_kernel<false>, a.n, 128, 0, s, a);
 }
 
 // "MoE routing strategies explained", "4. Sigmoid gating with aux-loss-free
@@ -121,6 +273,8 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
 // idle ones. The sign is taken exactly in integers: load*E vs n*K.
 __global__ void bias_update_kernel(int n, int E, int K, const int32_t* load, float rate,
                                    float* bias) {
+  pdl_wait();
+  pdl_trigger();
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= E) return;
   const long long diff = (long long)load[e] * E - (long long)n * K;
@@ -132,8 +286,7 @@ __global__ void bias_update_kernel(int n, int E, int K, const int32_t* load, flo
 
 cudaError_t launch_bias_update(int n, int E, int K, const int32_t* load, float rate,
                                float* bias, cudaStream_t s) {
-  bias_update_kernel<<<ceil_div(E, 256), 256, 0, s>>>(n, E, K, load, rate, bias);
-  return cudaGetLastError();
+  return launch_pdl(bias_update_kernel, ceil_div(E, 256), 256, 0, s, n, E, K, load, rate, bias);
 }
 
 }  // namespace moe

@@ -42,6 +42,8 @@ __device__ __forceinline__ int find_expert(const int32_t* offsets, int E, int ro
 
 template <bool SWIGLU>
 __global__ void __launch_bounds__(256) ffn_f32_kernel(F32GemmArgs a) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float As[kFBK][kFBM + 4];
   __shared__ float Bs[kFBK][kFBN + 4];
   __shared__ float B3s[SWIGLU ? kFBK : 1][kFBN + 4];
@@ -140,10 +142,8 @@ static cudaError_t launch_f32_gemm(const F32GemmArgs& a, long long total_rows,
                                    cudaStream_t s) {
   dim3 grid(ceil_div(a.N, kFBN), (unsigned)(total_rows / kFBM));
   if (a.act == 3)
-    ffn_f32_kernel<true><<<grid, 256, 0, s>>>(a);
-  else
-    ffn_f32_kernel<false><<<grid, 256, 0, s>>>(a);
-  return cudaGetLastError();
+    return launch_pdl(ffn_f32_kernel<true>, grid, 256, 0, s, a);
+  return launch_pdl(ffn_f32_kernel<false>, grid, 256, 0, s, a);
 }
 
 moe_status run_ffn_f32(const FfnArgs& f, cudaStream_t s) {

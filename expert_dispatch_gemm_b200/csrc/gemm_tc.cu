@@ -165,15 +165,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   SharedState* st = reinterpret_cast<SharedState*>(base + kStages * kStageBytes);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int i = tid; i <= p.E; i += kGemmThreads) st->offs[i] = p.offsets[i];
-  __syncthreads();
   if (tid == 0) {
-    int run = 0;
-    for (int e = 0; e < p.E; ++e) {
-      st->tprefix[e] = run;
-      run += max(st->offs[e + 1] - st->offs[e], 0) / kBM * p.nt_tiles;
-    }
-    st->tprefix[p.E] = run;
     for (int s = 0; s < kStages; ++s) {
       sm100::mbar_init(&st->full[s], 1);
       sm100::mbar_init(&st->empty[s], 1);
@@ -194,6 +186,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) {
     sm100::tmem_alloc(&st->tmem_base, kTmemCols);
     sm100::tmem_relinquish();
+  }
+  // the set-up above overlaps the previous kernel's tail; from here on the
+  // routing offsets (and, for the second projection, H) are read
+  pdl_wait();
+  pdl_trigger();
+  for (int i = tid; i <= p.E; i += kGemmThreads) st->offs[i] = p.offsets[i];
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int e = 0; e < p.E; ++e) {
+      st->tprefix[e] = run;
+      run += max(st->offs[e + 1] - st->offs[e], 0) / kBM * p.nt_tiles;
+    }
+    st->tprefix[p.E] = run;
   }
   sm100::tc_fence_before();
   __syncthreads();
@@ -506,16 +512,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const uint32_t rank = sm100::cluster_ctarank();
   const bool leader = rank == 0;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int i = tid; i <= p.E; i += kGemmThreads) st->offs[i] = p.offsets[i];
-  __syncthreads();
   if (tid == 0) {
-    int run = 0;
-    for (int e = 0; e < p.E; ++e) {
-      st->tprefix[e] = run;
-      const int cnt = max(st->offs[e + 1] - st->offs[e], 0) / kBM;
-      run += (cnt + 1) / 2 * p.nt_tiles;
-    }
-    st->tprefix[p.E] = run;
     for (int s = 0; s < kPStages; ++s) {
       sm100::mbar_init(&st->full[s], 1);
       sm100::mbar_init(&st->empty[s], 1);
@@ -536,6 +533,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) {
     sm100::tmem_alloc_pair(&st->tmem_base, kTmemCols);
     sm100::tmem_relinquish_pair();
+  }
+  // the set-up above overlaps the previous kernel's tail; from here on the
+  // routing offsets (and, for the second projection, H) are read
+  pdl_wait();
+  pdl_trigger();
+  for (int i = tid; i <= p.E; i += kGemmThreads) st->offs[i] = p.offsets[i];
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int e = 0; e < p.E; ++e) {
+      st->tprefix[e] = run;
+      const int cnt = max(st->offs[e + 1] - st->offs[e], 0) / kBM;
+      run += (cnt + 1) / 2 * p.nt_tiles;
+    }
+    st->tprefix[p.E] = run;
   }
   sm100::tc_fence_before();
   __syncthreads();
@@ -776,8 +788,7 @@ static cudaError_t launch_one(K kern, const Maps& m, const TcGemmParams& p, int 
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
-  kern<<<ctas, kGemmThreads, bytes, s>>>(m.a0, m.a1, m.b0, m.b0g, m.b1, m.b1g, m.xg, p);
-  return cudaGetLastError();
+  return launch_pdl(kern, ctas, kGemmThreads, bytes, s, m.a0, m.a1, m.b0, m.b0g, m.b1, m.b1g, m.xg, p);
 }
 
 // grid: CTAs for the single-CTA kernel, CTA pairs for the pair kernel

@@ -140,13 +140,19 @@ cudaError_t launch_tc_assign(const TcAssignArgs& a, cudaStream_t s);
 
 struct GatherArgs {
   const void* X;
-  const int32_t* row_token;
-  const int32_t* offsets;  // offsets[E] = rows in use
-  int E, d, elt_bytes;
+  const int32_t* tok_row;    // [n, slots]: the token's dispatched rows, then -1
+  const int32_t* row_token;  // [rows]: source token of each row, -1 padding
+  const int32_t* offsets;    // [E+1]: offsets[E] = rows in use
+  int E, n, slots;
+  int fanout;                // expected rows per token (K, or EC capacity factor)
+  int row_bytes;           // d * element size (a multiple of 16)
   long long max_rows;
   void* X_perm;
+  int* err;                // device error word, or NULL for the module's own
 };
 cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s);
+// Reads and clears the error word of dispatch calls made without a workspace.
+int take_dispatch_error();
 
 struct CombineArgs {
   const void* Y;

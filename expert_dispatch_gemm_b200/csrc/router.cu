@@ -34,19 +34,21 @@ struct RCfg {
   static_assert(WY * LY * TN == ET, "columns");
   static_assert(WX * WY * WK == 8, "8 warps");
   static_assert(TN == 4 || TN == 8, "TN");
+  static_assert(TM == 1 || TM == 2 || TM % 4 == 0, "TM");
   static_assert(BK % WK == 0 && ST >= 2, "pipeline");
 };
-// 4 x 8 register tiles wherever E allows (half the shared-memory bytes per FMA
-// of 2 x 8); the "s" variants trade rows per CTA for an in-CTA K split when the
-// batch is too small to give every SM a CTA. E = 8 is bound by reading X, so
-// its chunks are long (BK 128) to keep ~48 KB in flight per CTA.
+// 4 x 8 (E = 64, 128) or 8 x 8 (E = 256) register tiles: the larger the tile
+// the fewer shared-memory fragment loads per FMA. The "s" variants trade rows
+// per CTA for an in-CTA K split when the batch is too small to give every SM
+// a CTA. E = 8 is bound by reading X, so its chunks are long (BK 128) to keep
+// ~48 KB in flight per CTA.
 //                   ET   TM TN LX WX WY WK  BK  ST
 using R8 = RCfg<8, 1, 8, 32, 1, 1, 8, 128, 4>;
 using R32 = RCfg<32, 2, 4, 4, 4, 1, 2, 64, 4>;
 using R64 = RCfg<64, 4, 8, 4, 4, 1, 2, 32, 4>;
-using R64s = RCfg<64, 4, 8, 4, 1, 1, 8, 32, 4>;
+using R64s = RCfg<64, 4, 8, 4, 1, 1, 8, 64, 4>;
 using R128 = RCfg<128, 4, 8, 4, 2, 2, 2, 32, 4>;
-using R256 = RCfg<256, 4, 8, 4, 2, 4, 1, 32, 3>;
+using R256 = RCfg<256, 8, 8, 4, 1, 4, 2, 32, 3>;
 using R256s = RCfg<256, 2, 8, 4, 2, 4, 1, 32, 3>;
 
 constexpr int kSelectRowsPerWarp = 4;
@@ -197,6 +199,91 @@ __device__ __forceinline__ void tc_select_row(const float (&key)[V], const float
 }
 
 // ---------------------------------------------------------------------------
+// Row epilogue shared by both router main loops. Ls holds the CTA's logits
+// tile [BM][ET + 1] without the logit bias; 8 warps take one row at a time.
+// Adds the bias, applies the score function, writes logits / scores / lse,
+// selects the token-choice experts, and leaves this CTA's partial column sums
+// of S and its sum of lse^2 in colsum / lse2 at index blockIdx.x.
+// colsum_w [8][ET] floats and lse2_w [8] doubles are shared-memory scratch.
+// ---------------------------------------------------------------------------
+template <int ET>
+__device__ __forceinline__ void router_rows_epilogue(const RouterArgs& a, const float* Ls,
+                                                     float* colsum_w, double* lse2_w, int BM,
+                                                     int m0) {
+  constexpr int LST = ET + 1;
+  constexpr int V = ET >= 32 ? ET / 32 : 1;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int n = a.n, E = a.E;
+  float csum[V];
+#pragma unroll
+  for (int v = 0; v < V; ++v) csum[v] = 0.0f;
+  double my_lse2 = 0.0;
+
+  for (int r = warp; r < BM; r += 8) {
+    const int t = m0 + r;
+    if (t >= n) break;
+    float l[V], s[V], key[V];
+    bool ok[V];
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+      const int cc = lane * V + v;
+      ok[v] = cc < E;
+      l[v] = ok[v] ? Ls[r * LST + cc] + (a.logit_bias ? a.logit_bias[cc] : 0.0f) : -INFINITY;
+    }
+    float m = -INFINITY;
+#pragma unroll
+    for (int v = 0; v < V; ++v) m = fmaxf(m, l[v]);
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float ex[V], z = 0.0f;
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+      ex[v] = ok[v] ? expf(l[v] - m) : 0.0f;
+      z += ex[v];
+    }
+    for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    const float lse = m + logf(z);
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+      if (a.score == MOE_SCORE_SIGMOID)
+        s[v] = ok[v] ? 1.0f / (1.0f + expf(-l[v])) : 0.0f;
+      else
+        s[v] = ex[v] / z;
+      csum[v] += ok[v] ? s[v] : 0.0f;
+      const int cc = lane * V + v;
+      if (ok[v]) {
+        a.scores[(size_t)t * E + cc] = s[v];
+        if (a.logits) a.logits[(size_t)t * E + cc] = l[v];
+      }
+      key[v] = ok[v] ? (a.sel_bias ? s[v] + a.sel_bias[cc] : s[v]) : 0.0f;
+    }
+    if (lane == 0) {
+      if (a.lse) a.lse[t] = lse;
+      my_lse2 += (double)lse * (double)lse;
+    }
+    if (a.K > 0)
+      tc_select_row<V>(key, s, ok, lane, E, a.K, a.n_groups, a.topk_groups, a.group_topn,
+                       a.weights, a.idx + (size_t)t * a.K, a.gate + (size_t)t * a.K);
+  }
+#pragma unroll
+  for (int v = 0; v < V; ++v) {
+    const int cc = lane * V + v;
+    if (cc < ET) colsum_w[warp * ET + cc] = csum[v];
+  }
+  if (lane == 0) lse2_w[warp] = my_lse2;
+  __syncthreads();
+  for (int cc = tid; cc < E; cc += 256) {
+    float sum = 0.0f;
+    for (int w = 0; w < 8; ++w) sum += colsum_w[w * ET + cc];
+    a.colsum[(size_t)blockIdx.x * E + cc] = sum;
+  }
+  if (tid == 0) {
+    double sum = 0.0;
+    for (int w = 0; w < 8; ++w) sum += lse2_w[w];
+    a.lse2[blockIdx.x] = sum;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Router GEMM + epilogue
 // ---------------------------------------------------------------------------
 template <class C, bool XBF16>
@@ -214,6 +301,8 @@ struct RouterSmem {
 
 template <class C, bool XBF16>
 __global__ void __launch_bounds__(256) router_kernel(RouterArgs a) {
+  pdl_wait();
+  pdl_trigger();
   using SM = RouterSmem<C, XBF16>;
   constexpr int ET = C::ET, BM = C::BM, BK = C::BK, TM = C::TM, TN = C::TN;
   constexpr int XB = SM::XB, AST = SM::AST;
@@ -314,9 +403,15 @@ __global__ void __launch_bounds__(256) router_kernel(RouterArgs a) {
     for (int q = 0; q < BK / C::WK; ++q) {
       const int kk = wk * (BK / C::WK) + q;
       float av[TM], bv[TN];
-      if (TM == 4) {
-        const float4 t = *reinterpret_cast<const float4*>(As + kk * AST + row0);
-        av[0] = t.x; av[1] = t.y; av[2 % TM] = t.z; av[3 % TM] = t.w;
+      if (TM % 4 == 0) {
+#pragma unroll
+        for (int i4 = 0; i4 < TM / 4; ++i4) {
+          const float4 t = *reinterpret_cast<const float4*>(As + kk * AST + row0 + 4 * i4);
+          av[(4 * i4 + 0) % TM] = t.x;
+          av[(4 * i4 + 1) % TM] = t.y;
+          av[(4 * i4 + 2) % TM] = t.z;
+          av[(4 * i4 + 3) % TM] = t.w;
+        }
       } else if (TM == 2) {
         const float2 t = *reinterpret_cast<const float2*>(As + kk * AST + row0);
         av[0] = t.x; av[1 % TM] = t.y;
@@ -362,73 +457,7 @@ __global__ void __launch_bounds__(256) router_kernel(RouterArgs a) {
 
   float* colsum_w = Ls + C::WK * BM * LST;                          // [8][ET]
   double* lse2_w = reinterpret_cast<double*>(colsum_w + 8 * ET);     // [8]
-  float csum[V];
-#pragma unroll
-  for (int v = 0; v < V; ++v) csum[v] = 0.0f;
-  double my_lse2 = 0.0;
-
-  for (int r = warp; r < BM; r += 8) {
-    const int t = m0 + r;
-    if (t >= n) break;
-    float l[V], s[V], key[V];
-    bool ok[V];
-#pragma unroll
-    for (int v = 0; v < V; ++v) {
-      const int cc = lane * V + v;
-      ok[v] = cc < E;
-      l[v] = ok[v] ? Ls[r * LST + cc] + (a.logit_bias ? a.logit_bias[cc] : 0.0f) : -INFINITY;
-    }
-    float m = -INFINITY;
-#pragma unroll
-    for (int v = 0; v < V; ++v) m = fmaxf(m, l[v]);
-    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float ex[V], z = 0.0f;
-#pragma unroll
-    for (int v = 0; v < V; ++v) {
-      ex[v] = ok[v] ? expf(l[v] - m) : 0.0f;
-      z += ex[v];
-    }
-    for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-    const float lse = m + logf(z);
-#pragma unroll
-    for (int v = 0; v < V; ++v) {
-      if (a.score == MOE_SCORE_SIGMOID)
-        s[v] = ok[v] ? 1.0f / (1.0f + expf(-l[v])) : 0.0f;
-      else
-        s[v] = ex[v] / z;
-      csum[v] += ok[v] ? s[v] : 0.0f;
-      const int cc = lane * V + v;
-      if (ok[v]) {
-        a.scores[(size_t)t * E + cc] = s[v];
-        if (a.logits) a.logits[(size_t)t * E + cc] = l[v];
-      }
-      key[v] = ok[v] ? (a.sel_bias ? s[v] + a.sel_bias[cc] : s[v]) : 0.0f;
-    }
-    if (lane == 0) {
-      if (a.lse) a.lse[t] = lse;
-      my_lse2 += (double)lse * (double)lse;
-    }
-    if (a.K > 0)
-      tc_select_row<V>(key, s, ok, lane, E, a.K, a.n_groups, a.topk_groups, a.group_topn,
-                       a.weights, a.idx + (size_t)t * a.K, a.gate + (size_t)t * a.K);
-  }
-#pragma unroll
-  for (int v = 0; v < V; ++v) {
-    const int cc = lane * V + v;
-    if (cc < ET) colsum_w[warp * ET + cc] = csum[v];
-  }
-  if (lane == 0) lse2_w[warp] = my_lse2;
-  __syncthreads();
-  for (int cc = tid; cc < E; cc += 256) {
-    float sum = 0.0f;
-    for (int w = 0; w < 8; ++w) sum += colsum_w[w * ET + cc];
-    a.colsum[(size_t)blockIdx.x * E + cc] = sum;
-  }
-  if (tid == 0) {
-    double sum = 0.0;
-    for (int w = 0; w < 8; ++w) sum += lse2_w[w];
-    a.lse2[blockIdx.x] = sum;
-  }
+  router_rows_epilogue<ET>(a, Ls, colsum_w, lse2_w, BM, m0);
 }
 
 template <class C, bool XBF16>
@@ -439,8 +468,7 @@ static cudaError_t launch_router_t(const RouterArgs& a, cudaStream_t s) {
                                        (int)bytes);
   if (e != cudaSuccess) return e;
   const int grid = ceil_div(a.n, C::BM);
-  kern<<<grid, 256, bytes, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, 256, bytes, s, a);
 }
 
 template <bool XBF16>
@@ -468,6 +496,8 @@ cudaError_t launch_router(const RouterArgs& a, cudaStream_t s) {
 // ---------------------------------------------------------------------------
 template <int V>
 __global__ void __launch_bounds__(256) select_tc_kernel(SelectTcArgs a) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float colsum_w[8][V * 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int rows_per_block = 8 * kSelectRowsPerWarp;
@@ -507,12 +537,11 @@ cudaError_t launch_select_tc(const SelectTcArgs& a, cudaStream_t s) {
   const int et = router_tile_et(a.E);
   switch (et) {
     case 8:
-    case 32: select_tc_kernel<1><<<grid, 256, 0, s>>>(a); break;
-    case 64: select_tc_kernel<2><<<grid, 256, 0, s>>>(a); break;
-    case 128: select_tc_kernel<4><<<grid, 256, 0, s>>>(a); break;
-    default: select_tc_kernel<8><<<grid, 256, 0, s>>>(a); break;
+    case 32: return launch_pdl(select_tc_kernel<1>, grid, 256, 0, s, a);
+    case 64: return launch_pdl(select_tc_kernel<2>, grid, 256, 0, s, a);
+    case 128: return launch_pdl(select_tc_kernel<4>, grid, 256, 0, s, a);
+    default: return launch_pdl(select_tc_kernel<8>, grid, 256, 0, s, a);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace moe

@@ -211,8 +211,15 @@ MOE_API moe_status moe_route_from_scores(const moe_config* cfg, const float* S,
                                  size_t ws_bytes, moe_stream_t stream);
 
 /* Gather ([EC-math] "The math": X_in[e] = P[e] X with P = onehot(I), done as
- * an index gather): X_perm[r] = X[row_token[r]] for every routed row
- * r < offsets[E] with row_token[r] >= 0. X [n,d], X_perm [rows,d]. */
+ * an index gather): X_perm[r] = X[t] for every token t and every row r >= 0
+ * of its list route->tok_row[t, :] (the same rows as those with
+ * row_token[r] == t). X [n,d], X_perm [rows,d], both 16-byte aligned (else
+ * MOE_ERR_INVALID_ARG). Rows not in any list are left untouched. Uses
+ * route->tok_row, row_token and offsets. When a token feeds 4 or more rows
+ * (token choice with K >= 4), each token's row is read once and written to
+ * all of its rows by TMA bulk copies staged in shared memory; the staging
+ * wait is bounded, and a timeout is reported by the next moe_read_error on
+ * this device. Otherwise each row is copied by one warp with 16-byte loads. */
 MOE_API moe_status moe_dispatch(const moe_config* cfg, const void* X, const moe_route_out* route,
                         void* X_perm, moe_stream_t stream);
 
@@ -294,8 +301,10 @@ MOE_API moe_status moe_route_noalloc(const moe_config* cfg, const void* X, const
 MOE_API moe_status moe_workspace_init(void* ws, moe_stream_t stream);
 
 /* Synchronises `stream`, then reads and clears the error word at the start
- * of `ws`: MOE_OK, MOE_ERR_TIMEOUT (a bounded wait gave up) or MOE_ERR_CUDA.
- * If detail != NULL it receives the raw device code (0 = none). */
+ * of `ws` and, when that is clear, the current device's word for moe_dispatch
+ * calls (which take no workspace): MOE_OK, MOE_ERR_TIMEOUT (a bounded wait
+ * gave up) or MOE_ERR_CUDA. If detail != NULL it receives the raw device code
+ * (0 = none). */
 MOE_API moe_status moe_read_error(void* ws, moe_stream_t stream, int* detail);
 
 #ifdef __cplusplus

@@ -288,6 +288,50 @@ def test_edge_cases(w):
     _gathered_vs_unfused(w)
 
 
+# rows longer than one 16 KB staging unit: the staged gather (K >= 4) copies
+# them in two segments
+LONG_ROWS = wl.TC_DROPLESS.replace(name="tc-top4of16-long-rows-d12352", n=300, d=12352, E=16,
+                                   K=4, h=64)
+
+
+@pytest.mark.parametrize("w", wl.SMALL + EDGE + [LONG_ROWS] + wl.FULL, ids=lambda w: w.name)
+def test_dispatch_exact_copy(w):
+    """The gather copies each token's row, byte for byte, to exactly the rows
+    row_token names, and leaves every other row of X_perm untouched."""
+    inp = wl.make_inputs(w, DEV, experts=False)
+    cfg = moe.config(w)
+    sz = moe.sizes(cfg)
+    rb = moe.RouteBuffers(cfg, DEV, logits=False)
+    ws = moe.workspace(cfg, DEV, layer=False)
+    moe.moe_route(cfg, inp["X"], inp["Wg"], inp["logit_bias"], inp["sel_bias"], rb, ws)
+    X_perm = torch.full((sz.rows, w.d), 12352.0, dtype=w.torch_dtype, device=DEV)
+    moe.moe_dispatch(cfg, inp["X"], rb, X_perm)
+    torch.cuda.synchronize()
+    used = int(rb.offsets[-1])
+    rt = rb.row_token[:used]
+    real = rt >= 0
+    assert torch.equal(X_perm[:used][real], inp["X"][rt[real].long()])
+    assert bool((X_perm[:used][~real] == 12352.0).all())
+    assert bool((X_perm[used:] == 12352.0).all())
+    _ws_ok(ws)
+
+
+def test_dispatch_rejects_misaligned_rows():
+    w = wl.SMALL[1]
+    inp = wl.make_inputs(w, DEV, experts=False)
+    cfg = moe.config(w)
+    sz = moe.sizes(cfg)
+    rb = moe.RouteBuffers(cfg, DEV, logits=False)
+    ws = moe.workspace(cfg, DEV, layer=False)
+    moe.moe_route(cfg, inp["X"], inp["Wg"], None, None, rb, ws)
+    buf = torch.empty(sz.rows * w.d + 8, dtype=w.torch_dtype, device=DEV)
+    X_perm = buf[1:1 + sz.rows * w.d].view(sz.rows, w.d)  # 2 bytes off a 16-byte boundary
+    with pytest.raises(moe.MoeError) as e:
+        moe.moe_dispatch(cfg, inp["X"], rb, X_perm)
+    assert e.value.status == moe.MOE_ERR_INVALID_ARG
+    _ws_ok(ws)
+
+
 def test_capacity_one_all_equal_scores():
     w = EDGE[3]
     cfg = moe.config(w)
