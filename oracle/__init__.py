@@ -27,7 +27,7 @@ import numpy as np
 
 from .build import build as _build
 
-SOFTMAX, SIGMOID = 0, 1
+SOFTMAX, SIGMOID, SQRTSOFTPLUS = 0, 1, 2
 RELU, GELU, SWIGLU = 0, 1, 2
 W_RAW, W_NORMALIZED = 0, 1
 STORE_F32, STORE_BF16 = 0, 1
@@ -118,7 +118,8 @@ def round_bf16(a) -> np.ndarray:
 
 
 def router(X, Wg, logit_bias=None, score=SOFTMAX):
-    """logits = X.W_g (+ logit bias), S = softmax/sigmoid(logits), lse per row."""
+    """logits = X.W_g (+ logit bias), S = softmax / sigmoid / sqrt(softplus) of
+    the logits, lse per row."""
     X = _f32(X)
     Wg = _f32(Wg)
     n, d = X.shape
@@ -245,7 +246,7 @@ def spec_of(w) -> dict:
     spec.update(act={"relu": RELU, "gelu": GELU, "swiglu": SWIGLU}[w.act],
                 store=STORE_F32 if w.dtype == "f32" else STORE_BF16,
                 n_shared=w.n_shared,
-                score=SIGMOID if w.score == "sigmoid" else SOFTMAX,
+                score={"sigmoid": SIGMOID, "sqrtsoftplus": SQRTSOFTPLUS}.get(w.score, SOFTMAX),
                 lb_coef=w.lb_coef, z_coef=w.z_coef)
     return spec
 

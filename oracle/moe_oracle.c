@@ -76,10 +76,19 @@ void orc_router(int n, int d, int E, const float* X, const float* Wg,
     lse[t] = m + log(z);
     for (int e = 0; e < E; ++e) {
       double s;
-      if (score == ORC_SIGMOID)
+      if (score == ORC_SIGMOID) {
         s = 1.0 / (1.0 + exp(-(double)L[e]));
-      else
+      } else if (score == ORC_SQRTSOFTPLUS) {
+        /* [Guide] "4. Sigmoid gating with aux-loss-free bias" names the
+         * score only; read as sqrt(softplus(l)), softplus(l) = ln(1 + e^l),
+         * evaluated as l + ln(1 + e^-l) for l > 0 so that e^l cannot
+         * overflow */
+        const double l = (double)L[e];
+        const double sp = l > 0.0 ? l + log1p(exp(-l)) : log1p(exp(l));
+        s = sqrt(sp);
+      } else {
         s = exp((double)L[e] - m) / z;
+      }
       S[(size_t)t * E + e] = (float)s;
     }
   }

@@ -30,7 +30,7 @@ extern "C" {
 #endif
 
 /* score functions, activations, weight modes and storage types */
-enum { ORC_SOFTMAX = 0, ORC_SIGMOID = 1 };
+enum { ORC_SOFTMAX = 0, ORC_SIGMOID = 1, ORC_SQRTSOFTPLUS = 2 };
 enum { ORC_RELU = 0, ORC_GELU = 1, ORC_SWIGLU = 2 };
 enum { ORC_W_RAW = 0, ORC_W_NORMALIZED = 1 };
 enum { ORC_STORE_F32 = 0, ORC_STORE_BF16 = 1 };

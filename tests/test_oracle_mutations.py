@@ -62,6 +62,10 @@ MUTATIONS = [
      "if (logit_bias) v += (double)logit_bias[e];",
      "if (logit_bias) v += 2.0 * (double)logit_bias[e];",
      ["test_router_against_library"]),
+    ("sqrt(softplus) score without the square root",
+     "        s = sqrt(sp);",
+     "        s = sp;",
+     ["test_sqrtsoftplus_closed_forms"]),
     ("expert choice gate read from the wrong expert",
      "G[(size_t)e * k + j] = S[(size_t)col[j].idx * E + e];",
      "G[(size_t)e * k + j] = S[(size_t)col[j].idx * E + (e + 1) % E];",

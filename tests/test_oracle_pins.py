@@ -292,6 +292,39 @@ def test_router_against_library():
     np.testing.assert_allclose(s, special.expit(L64), rtol=1e-6, atol=1e-9)
 
 
+def test_sqrtsoftplus_closed_forms():
+    """sqrt(softplus(l)) on logits fixed through the bias (X = 0): l = 0 gives
+    sqrt(ln 2); l = 100 gives 10 (ln(1 + e^-100) is below double precision at
+    100); l = -30 gives e^-15 to first order; l = 2 gives sqrt(2 + ln(1 +
+    e^-2)) = sqrt(ln(1 + e^2)); the score grows with l."""
+    b = np.array([0.0, 100.0, -30.0, 2.0, -1.0, 1.0], np.float32)
+    X = np.zeros((3, 4), np.float32)
+    Wg = np.ones((4, b.size), np.float32)
+    _, s, _ = oracle.router(X, Wg, b, score=oracle.SQRTSOFTPLUS)
+    assert np.allclose(s[:, 0], np.sqrt(np.log(2.0)), rtol=1e-7)
+    assert np.all(s[:, 1] == np.float32(10.0))
+    assert np.allclose(s[:, 2], np.exp(-15.0), rtol=1e-6)
+    assert np.allclose(s[:, 3], np.sqrt(np.log1p(np.exp(2.0))), rtol=1e-7)
+    order = np.argsort(b)
+    assert np.all(np.diff(s[0, order].astype(np.float64)) > 0)
+
+
+def test_monotone_scores_select_the_same_experts():
+    """Without a selection bias or groups, top-K of any score that grows with
+    the logit picks the same experts in the same order: softmax, sigmoid and
+    sqrt(softplus) agree on every token (distinct random logits)."""
+    rng = np.random.default_rng(11)
+    X = rng.standard_normal((64, 32)).astype(np.float32)
+    Wg = (rng.standard_normal((32, 16)) / np.sqrt(32)).astype(np.float32)
+    picks = []
+    for score in (oracle.SOFTMAX, oracle.SIGMOID, oracle.SQRTSOFTPLUS):
+        _, s, _ = oracle.router(X, Wg, score=score)
+        idx, _ = oracle.select_tc(s, 4)
+        picks.append(idx)
+    np.testing.assert_array_equal(picks[0], picks[1])
+    np.testing.assert_array_equal(picks[0], picks[2])
+
+
 # --------------------------------------------------------------------------
 # storage rounding
 # --------------------------------------------------------------------------
