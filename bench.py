@@ -382,9 +382,9 @@ def run_gpu(args, w: wl.Workload):
 
     value = whole_job_rate(w.n, world, args.steps, total_ms)
     e2e_value = whole_job_rate(w.n, world, args.steps, e2e_ms)
-    # route: router + select_ec + ec_finish (EC) or router + hist + scan + scatter (TC);
-    # dispatch: gather; expert FFN: up + down; combine
-    launches_per_step = (3 if w.mode == "ec" else 4) + 1 + 2 + 1
+    # route: router (+ split-k reduce) + select_ec + ec_finish (EC) or + hist +
+    # scan + scatter (TC); dispatch: gather; expert FFN: up + down; combine
+    launches_per_step = sum(moe.launch_counts(cfg).values())
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,

@@ -74,7 +74,10 @@ def _build_lib(sources, out_lib, force, ptxas_verbose) -> str:
     objs = [os.path.join(BUILD, s.replace(".cu", ".o")) for s in sources]
     if force or jobs or not os.path.exists(out_lib) or \
             os.path.getmtime(out_lib) < max(os.path.getmtime(o) for o in objs):
-        cmd = [nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", out_lib + ".tmp", *objs]
+        # --no-undefined: a symbol missing from the sources fails the build,
+        # not the first dlopen on a GPU machine
+        cmd = [nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", "-Xlinker", "--no-undefined",
+               "-o", out_lib + ".tmp", *objs]
         subprocess.check_call(cmd)
         os.replace(out_lib + ".tmp", out_lib)
     return out_lib

@@ -17,14 +17,15 @@ moe_status derive(const moe_config* c, Derived* d) {
   if (c->E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
   if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
   if (c->mode != MOE_EXPERT_CHOICE && c->mode != MOE_TOKEN_CHOICE) return MOE_ERR_INVALID_ARG;
-  if (c->score != MOE_SCORE_SOFTMAX && c->score != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (c->score != MOE_SCORE_SOFTMAX && c->score != MOE_SCORE_SIGMOID &&
+      c->score != MOE_SCORE_SQRTSOFTPLUS)
+    return MOE_ERR_INVALID_ARG;
   if (c->act != MOE_ACT_RELU && c->act != MOE_ACT_GELU && c->act != MOE_ACT_SWIGLU)
     return MOE_ERR_INVALID_ARG;
   if (c->weights != MOE_W_RAW && c->weights != MOE_W_NORMALIZED) return MOE_ERR_INVALID_ARG;
   if (c->n_shared < 0 || c->n_shared > MOE_MAX_SHARED) return MOE_ERR_INVALID_ARG;
   if (c->dtype == MOE_BF16) {
     if (c->d % 64 || c->h % 64) return MOE_ERR_UNSUPPORTED;
-    if (c->n_shared > 0 && c->n < 128) return MOE_ERR_UNSUPPORTED;
   } else {
     if (c->d % 8 || c->h % 8) return MOE_ERR_UNSUPPORTED;
   }
@@ -112,6 +113,11 @@ WsLayout ws_layout(const moe_config* c, const Derived& d) {
   if (c->mode == MOE_EXPERT_CHOICE) off = align_up(off + (size_t)c->n * c->E * 4, 256);
   w.ec_gate = off;
   if (c->mode == MOE_EXPERT_CHOICE) off = align_up(off + (size_t)c->n * c->E * 4, 256);
+  w.rpart = off;
+  {
+    const int ks = router_ksplit(c->E, c->n, c->d, c->dtype == MOE_BF16);
+    if (ks > 1) off = align_up(off + (size_t)ks * c->n * c->E * 4, 256);
+  }
   w.route_end = align_up(off, 1024);
   const size_t elt = c->dtype == MOE_BF16 ? 2 : 4;
   off = w.route_end;
@@ -247,9 +253,11 @@ static moe_status route_impl(const moe_config* c, const Derived& dv, const WsLay
   r.lse = o->lse;
   r.colsum = at<float>(ws, w.colsum);
   r.lse2 = at<double>(ws, w.lse2);
+  r.partial = at<float>(ws, w.rpart);
   MOE_CU(launch_router(r, s));
-  return finish_route(c, dv, w, o, ws, o->scores,
-                      ceil_div(c->n, router_block_rows(c->E, c->n)), true, s);
+  return finish_route(
+      c, dv, w, o, ws, o->scores,
+      ceil_div(c->n, router_block_rows(c->E, c->n, c->d, c->dtype == MOE_BF16)), true, s);
 }
 
 // X_perm == NULL: the routed rows are read from X through row_token (the
@@ -291,9 +299,17 @@ static moe_status ffn_impl(const moe_config* c, const Derived& dv, const void* X
   f.rows = dv.rows;
   f.err = err;
   // CTA pairs compute two 128-row blocks of one expert per tile: worth it when
-  // experts own several blocks (token choice, or expert choice with k > 128);
-  // with one block per expert half of a pair's MMA work would be padding
-  f.pair = c->mode == MOE_TOKEN_CHOICE || dv.kpad >= 2 * kRowAlign;
+  // experts own at least two blocks on average (expert choice with k > 128;
+  // token choice with min(nK/E, capacity) >= 256). With fewer rows per expert
+  // (small batches, decoding) half of a pair's MMA work would be padding, and
+  // the 128-row tiles of the single-CTA kernel waste half as much.
+  if (c->mode == MOE_TOKEN_CHOICE) {
+    long long avg = ((long long)c->n * dv.k + c->E - 1) / c->E;
+    if (dv.cap > 0 && avg > dv.cap) avg = dv.cap;
+    f.pair = avg >= 2 * kRowAlign;
+  } else {
+    f.pair = dv.kpad >= 2 * kRowAlign;
+  }
   return c->dtype == MOE_BF16 ? run_ffn_bf16(f, s) : run_ffn_f32(f, s);
 }
 
@@ -374,6 +390,19 @@ moe_status moe_sizes(const moe_config* cfg, int* k_eff, int* capacity_eff, int* 
   if (slots) *slots = d.slots;
   if (rows) *rows = (int)d.rows;
   if (shared_row_base) *shared_row_base = (int)d.shared_base;
+  return MOE_OK;
+}
+
+moe_status moe_launch_counts(const moe_config* cfg, int* route, int* dispatch, int* ffn,
+                             int* combine) {
+  Derived d;
+  moe_status st = derive(cfg, &d);
+  if (st != MOE_OK) return st;
+  const int split = router_ksplit(cfg->E, cfg->n, cfg->d, cfg->dtype == MOE_BF16) > 1;
+  if (route) *route = 1 + split + (cfg->mode == MOE_EXPERT_CHOICE ? 2 : 3);
+  if (dispatch) *dispatch = 1;
+  if (ffn) *ffn = 2;
+  if (combine) *combine = 1;
   return MOE_OK;
 }
 

@@ -59,7 +59,6 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* excl, int* warp_
 
 __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
   pdl_wait();
-  pdl_trigger();
   extern __shared__ __align__(16) unsigned char ec_smem[];
   const int n = a.n, E = a.E, k = a.k, e = blockIdx.x;
   const bool by_rank = k <= kEcRankMax;
@@ -71,7 +70,7 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
   __shared__ int hist[256];
   __shared__ int warp_tot[32];
   __shared__ uint32_t s_prefix, s_mask;
-  __shared__ int s_need;
+  __shared__ int s_need, s_done;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int32_t* my_rows = a.ec_row + (size_t)e * n;
 
@@ -89,6 +88,7 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
     s_prefix = 0u;
     s_mask = 0u;
     s_need = k;
+    s_done = 0;
   }
   __syncthreads();
 
@@ -98,11 +98,19 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
     for (int i = lane; i < 256; i += 32) myhist[i] = 0;
     const uint32_t prefix = s_prefix, mask = s_mask;
     __syncwarp();
+    // warp-aggregated counts: the lanes that share a digit add once, through
+    // their lowest lane, so a warp's private histogram needs no atomics
 #pragma unroll
     for (int i = 0; i < kEcMaxPerThread; ++i) {
+      if (i >= C) break;
       const int t = t0 + i;
-      if (i < C && t < n && (kreg[i] & mask) == prefix)
-        atomicAdd(&myhist[(kreg[i] >> shift) & 255u], 1);
+      const bool ok = t < n && (kreg[i] & mask) == prefix;
+      const unsigned act = __ballot_sync(0xffffffffu, ok);
+      if (ok) {
+        const unsigned dig = (kreg[i] >> shift) & 255u;
+        const unsigned peers = __match_any_sync(act, dig);
+        if (lane == __ffs(peers) - 1) myhist[dig] += __popc(peers);
+      }
     }
     __syncthreads();
     for (int b = tid; b < 256; b += kEcThreads) {
@@ -142,18 +150,23 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
         s_need = need - above;
         s_prefix = prefix | ((uint32_t)digit << shift);
         s_mask = mask | (255u << shift);
+        // every key in the chosen bucket is a pick: no later digit matters
+        if (above + hist[digit] == need) s_done = 1;
       }
     }
     __syncthreads();
+    if (s_done) break;
   }
-  const uint32_t T = s_prefix;
-  const int need_eq = s_need;  // ties at T to take, lowest token first
+  // picks: keys whose masked bits exceed T, plus the lowest-token need_eq of
+  // those equal to T (all of them when the passes stopped early)
+  const uint32_t T = s_prefix, M = s_mask;
+  const int need_eq = s_need;
 
   // the ties' ranks in token order, then every pick's slot in token order
   int my_eq = 0;
 #pragma unroll
   for (int i = 0; i < kEcMaxPerThread; ++i)
-    my_eq += (i < C && t0 + i < n && kreg[i] == T);
+    my_eq += (i < C && t0 + i < n && (kreg[i] & M) == T);
   int eq_base;
   block_exclusive_scan(my_eq, &eq_base, warp_tot);
   int my_sel = 0;
@@ -162,8 +175,9 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
 #pragma unroll
     for (int i = 0; i < kEcMaxPerThread; ++i) {
       if (!(i < C && t0 + i < n)) continue;
-      if (kreg[i] > T) ++my_sel;
-      else if (kreg[i] == T) my_sel += (rank++ < need_eq);
+      const uint32_t u = kreg[i] & M;
+      if (u > T) ++my_sel;
+      else if (u == T) my_sel += (rank++ < need_eq);
     }
   }
   int slot;
@@ -174,8 +188,8 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
     for (int i = 0; i < kEcMaxPerThread; ++i) {
       if (!(i < C && t0 + i < n)) continue;
       const uint32_t u = kreg[i];
-      bool sel = u > T;
-      if (u == T) sel = rank++ < need_eq;
+      bool sel = (u & M) > T;
+      if ((u & M) == T) sel = rank++ < need_eq;
       if (sel)
         sbuf[slot++] = ((uint64_t)u << 32) | (uint64_t)(0xffffffffu - (uint32_t)(t0 + i));
     }
@@ -269,7 +283,6 @@ cudaError_t launch_select_ec(const SelectEcArgs& a, cudaStream_t s) {
 // shared memory (coalesced reads), then one warp per token compacts it.
 __global__ void __launch_bounds__(256) ec_finish_kernel(EcFinishArgs a) {
   pdl_wait();
-  pdl_trigger();
   extern __shared__ __align__(16) unsigned char fin_smem[];
   int* rows_s = reinterpret_cast<int*>(fin_smem);              // [E][33]
   float* gates_s = reinterpret_cast<float*>(rows_s + a.E * 33);  // [E][33]
@@ -332,7 +345,6 @@ cudaError_t launch_ec_finish(const EcFinishArgs& a, cudaStream_t s) {
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kTokBlock) tc_hist_kernel(TcAssignArgs a) {
   pdl_wait();
-  pdl_trigger();
   __shared__ int hist[MOE_MAX_EXPERTS];
   for (int i = threadIdx.x; i < a.E; i += kTokBlock) hist[i] = 0;
   __syncthreads();
@@ -349,11 +361,12 @@ __global__ void __launch_bounds__(kTokBlock) tc_hist_kernel(TcAssignArgs a) {
 
 __global__ void __launch_bounds__(1024) tc_scan_kernel(TcAssignArgs a) {
   pdl_wait();
-  pdl_trigger();
   __shared__ int seg[MOE_MAX_EXPERTS];
   __shared__ int off[MOE_MAX_EXPERTS + 1];
+  __shared__ int load_s[MOE_MAX_EXPERTS], kept_s[MOE_MAX_EXPERTS];
   __shared__ double fp[MOE_MAX_EXPERTS];
   __shared__ double part[1024];  // [slice][expert] partial column sums of S
+  __shared__ double z_s;
   const int E = a.E, tid = threadIdx.x;
   // column sums of S for the balance loss: thread (slice, e) adds the router
   // blocks b = slice, slice + S, ... in order; the slices are then added in
@@ -366,19 +379,45 @@ __global__ void __launch_bounds__(1024) tc_scan_kernel(TcAssignArgs a) {
     part[tid] = col;
   }
   __syncthreads();
-  for (int e = tid; e < E; e += blockDim.x) {
+  // per expert: exclusive prefix of the token blocks' counts, one warp per
+  // expert, 32 blocks per step (a shuffle scan), so the block count adds
+  // steps of one load each, not a chain of dependent loads
+  const int lane = tid & 31, warp = tid >> 5;
+  for (int e = warp; e < E; e += (int)(blockDim.x >> 5)) {
     int run = 0;
-    for (int b = 0; b < a.tok_blocks; ++b) {
-      a.blk_base[(size_t)b * E + e] = run;
-      run += a.blk_hist[(size_t)b * E + e];
+    for (int b0 = 0; b0 < a.tok_blocks; b0 += 32) {
+      const int b = b0 + lane;
+      const int v = b < a.tok_blocks ? a.blk_hist[(size_t)b * E + e] : 0;
+      int incl = v;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (b < a.tok_blocks) a.blk_base[(size_t)b * E + e] = run + incl - v;
+      run += __shfl_sync(0xffffffffu, incl, 31);
     }
+    if (lane == 0) load_s[e] = run;
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) {
+    const int run = load_s[e];
     const int kept = a.cap < 0 ? run : min(run, a.cap);
     a.load[e] = run;
     a.counts[e] = kept;
+    kept_s[e] = kept;
     seg[e] = (kept + kRowAlign - 1) / kRowAlign * kRowAlign;
     double col = 0.0;
     for (int sl = 0; sl < S; ++sl) col += part[sl * E + e];
     fp[e] = ((double)run / ((double)a.n * a.K)) * (col / (double)a.n);
+  }
+  if (tid < 32) {
+    // sum of lse^2 over the router blocks: lane-strided, then a fixed
+    // shuffle tree, so the order never depends on scheduling
+    double z = 0.0;
+    if (a.lse2)
+      for (int b = tid; b < a.lse_blocks; b += 32) z += a.lse2[b];
+    for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    if (tid == 0) z_s = z;
   }
   __syncthreads();
   if (tid == 0) {
@@ -390,17 +429,12 @@ __global__ void __launch_bounds__(1024) tc_scan_kernel(TcAssignArgs a) {
       off[e] = run;
       run += seg[e];
       lbs += fp[e];
-      mx = max(mx, a.load[e]);
-      dropped += a.load[e] - a.counts[e];
+      mx = max(mx, load_s[e]);
+      dropped += load_s[e] - kept_s[e];
     }
     off[E] = run;
     a.aux[MOE_AUX_LB] = (float)((double)a.lb_coef * E * lbs);
-    double z = 0.0;
-    if (a.lse2) {
-      for (int b = 0; b < a.lse_blocks; ++b) z += a.lse2[b];
-      z = (double)a.z_coef * z / (double)a.n;
-    }
-    a.aux[MOE_AUX_Z] = (float)z;
+    a.aux[MOE_AUX_Z] = a.lse2 ? (float)((double)a.z_coef * z_s / (double)a.n) : 0.0f;
     a.aux[MOE_AUX_MAXVIO] = (float)((double)mx / ((double)a.n * a.K / E) - 1.0);
     a.aux[MOE_AUX_DROPPED] = (float)dropped;
     a.aux[MOE_AUX_TOKENS_SOME_DROPPED] = 0.0f;
@@ -410,23 +444,26 @@ __global__ void __launch_bounds__(1024) tc_scan_kernel(TcAssignArgs a) {
   }
   __syncthreads();
   for (int e = tid; e <= E; e += blockDim.x) a.offsets[e] = off[e];
-  // padding rows of each segment
-  for (int e = 0; e < E; ++e) {
-    const int lo = off[e] + a.counts[e], hi = off[e + 1];
-    for (int r = lo + tid; r < hi; r += blockDim.x) a.row_token[r] = -1;
+  // padding rows of each segment (fewer than kRowAlign per expert)
+  for (int i = tid; i < E * kRowAlign; i += blockDim.x) {
+    const int e = i / kRowAlign, r = off[e] + kept_s[e] + i % kRowAlign;
+    if (r < off[e + 1]) a.row_token[r] = -1;
   }
 }
 
 __global__ void __launch_bounds__(kTokBlock) tc_scatter_kernel(TcAssignArgs a) {
   pdl_wait();
-  pdl_trigger();
   extern __shared__ __align__(16) unsigned char sc_smem[];
+  constexpr int W = kTokBlock / 32;
   const int E = a.E, K = a.K;
-  uint32_t* mask = reinterpret_cast<uint32_t*>(sc_smem);      // [32][E]
-  int* wbase = reinterpret_cast<int*>(mask + 32 * E);         // [32][E]
+  uint32_t* mask = reinterpret_cast<uint32_t*>(sc_smem);      // [W][E]
+  int* wbase = reinterpret_cast<int*>(mask + W * E);          // [W][E]
+  int* base_s = wbase + W * E;                                // [E] block base + offset
   __shared__ int some_s, all_s;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int i = tid; i < 32 * E; i += kTokBlock) mask[i] = 0u;
+  for (int i = tid; i < W * E; i += kTokBlock) mask[i] = 0u;
+  for (int e = tid; e < E; e += kTokBlock)
+    base_s[e] = a.offsets[e] + a.blk_base[(size_t)blockIdx.x * E + e];
   if (tid == 0) {
     some_s = 0;
     all_s = 0;
@@ -442,7 +479,7 @@ __global__ void __launch_bounds__(kTokBlock) tc_scatter_kernel(TcAssignArgs a) {
   __syncthreads();
   for (int e = tid; e < E; e += kTokBlock) {
     int run = 0;
-    for (int w = 0; w < 32; ++w) {
+    for (int w = 0; w < W; ++w) {
       wbase[w * E + e] = run;
       run += __popc(mask[w * E + e]);
     }
@@ -456,11 +493,12 @@ __global__ void __launch_bounds__(kTokBlock) tc_scatter_kernel(TcAssignArgs a) {
       bool keep = false;
       int row = -1;
       if ((unsigned)e < (unsigned)E) {
-        const int pos = a.blk_base[(size_t)blockIdx.x * E + e] + wbase[warp * E + e] +
-                        __popc(mask[warp * E + e] & ((1u << lane) - 1u));
+        // arrival position: earlier blocks, earlier warps, earlier lanes
+        const int in_blk = wbase[warp * E + e] + __popc(mask[warp * E + e] & ((1u << lane) - 1u));
+        const int pos = base_s[e] - a.offsets[e] + in_blk;
         keep = a.cap < 0 || pos < a.cap;
         if (keep) {
-          row = a.offsets[e] + pos;
+          row = base_s[e] + in_blk;
           a.row_token[row] = t;
           a.tok_row[(size_t)t * K + kept] = row;
           a.tok_gate[(size_t)t * K + kept] = a.gate[aj];
@@ -488,7 +526,7 @@ cudaError_t launch_tc_assign(const TcAssignArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   e = launch_pdl(tc_scan_kernel, 1, 1024, 0, s, a);
   if (e != cudaSuccess) return e;
-  const size_t bytes = (size_t)64 * a.E * 4;
+  const size_t bytes = (size_t)(2 * (kTokBlock / 32) + 1) * a.E * 4;
   e = cudaFuncSetAttribute(tc_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)bytes);
   if (e != cudaSuccess) return e;

@@ -17,16 +17,14 @@ enum : int {
 };
 
 // Programmatic dependent launch. Every kernel of the library is launched
-// with programmatic stream serialisation (launch_pdl): it may start while the
-// previous kernel in the stream is finishing, so it calls pdl_wait() before
-// it touches anything that kernel wrote (the wait returns once the previous
-// grid has completed and its writes are visible; every kernel waits, so the
-// order is transitive). pdl_trigger() lets the next kernel's CTAs be
-// scheduled early, as this kernel's CTAs leave their SMs.
+// with programmatic stream serialisation (launch_pdl), so its launch is
+// processed while the previous kernel in the stream drains, and it calls
+// pdl_wait() before it touches anything that kernel wrote (the wait returns
+// once the previous grid has completed and its writes are visible; every
+// kernel waits, so the order is transitive). No kernel triggers its
+// dependents early: CTAs of the next kernel parked on SMs beside this one's
+// measured slower on B200 than letting them start as this one's CTAs exit.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_trigger() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
 
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,

@@ -38,7 +38,6 @@ __device__ int g_dispatch_error;  // timeouts of standalone dispatch calls
 
 __global__ void gather_kernel(GatherArgs a, int seg, int nseg, int ring, int slot_stride) {
   pdl_wait();
-  pdl_trigger();
   extern __shared__ __align__(128) unsigned char gsm[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int warps = blockDim.x >> 5;
@@ -133,7 +132,6 @@ __global__ void gather_kernel(GatherArgs a, int seg, int nseg, int ring, int slo
 // where the staged kernel would serialise a few round trips per warp.
 __global__ void __launch_bounds__(256) gather_rows_kernel(GatherArgs a) {
   pdl_wait();
-  pdl_trigger();
   const long long rows = min((long long)a.offsets[a.E], a.max_rows);
   const int lane = threadIdx.x & 31;
   const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -204,7 +202,6 @@ cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s) {
 template <bool BF16>
 __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
   pdl_wait();
-  pdl_trigger();
   __shared__ int rows_s[MOE_MAX_EXPERTS];
   __shared__ float gates_s[MOE_MAX_EXPERTS];
   __shared__ int cnt_s;
@@ -274,7 +271,6 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
 __global__ void bias_update_kernel(int n, int E, int K, const int32_t* load, float rate,
                                    float* bias) {
   pdl_wait();
-  pdl_trigger();
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= E) return;
   const long long diff = (long long)load[e] * E - (long long)n * K;

@@ -43,7 +43,6 @@ __device__ __forceinline__ int find_expert(const int32_t* offsets, int E, int ro
 template <bool SWIGLU>
 __global__ void __launch_bounds__(256) ffn_f32_kernel(F32GemmArgs a) {
   pdl_wait();
-  pdl_trigger();
   __shared__ float As[kFBK][kFBM + 4];
   __shared__ float Bs[kFBK][kFBN + 4];
   __shared__ float B3s[SWIGLU ? kFBK : 1][kFBN + 4];

@@ -187,10 +187,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     sm100::tmem_alloc(&st->tmem_base, kTmemCols);
     sm100::tmem_relinquish();
   }
-  // the set-up above overlaps the previous kernel's tail; from here on the
-  // routing offsets (and, for the second projection, H) are read
+  // the set-up above needs nothing from the previous kernel; from here on
+  // the routing offsets (and, for the second projection, H) are read
   pdl_wait();
-  pdl_trigger();
   for (int i = tid; i <= p.E; i += kGemmThreads) st->offs[i] = p.offsets[i];
   __syncthreads();
   if (tid == 0) {
@@ -534,10 +533,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     sm100::tmem_alloc_pair(&st->tmem_base, kTmemCols);
     sm100::tmem_relinquish_pair();
   }
-  // the set-up above overlaps the previous kernel's tail; from here on the
-  // routing offsets (and, for the second projection, H) are read
+  // the set-up above needs nothing from the previous kernel; from here on
+  // the routing offsets (and, for the second projection, H) are read
   pdl_wait();
-  pdl_trigger();
   for (int i = tid; i <= p.E; i += kGemmThreads) st->offs[i] = p.offsets[i];
   __syncthreads();
   if (tid == 0) {
@@ -758,8 +756,8 @@ static EncodeTiledFn encode_fn() {
 // 2-D bf16 row-major [rows, cols] map with a box of 64 columns x box_rows rows
 // and 128-byte swizzle. Out-of-range elements (including a box taller than
 // the whole tensor) load as zero.
-static bool make_map(CUtensorMap* m, const void* ptr, long long rows, long long cols,
-                     int box_rows) {
+bool make_bf16_sw128_map(CUtensorMap* m, const void* ptr, long long rows, long long cols,
+                         int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn || rows < 1 || cols < kBK) return false;
   if ((reinterpret_cast<uintptr_t>(ptr) & 15) || ((cols * 2) & 15)) return false;
@@ -844,29 +842,29 @@ moe_status run_ffn_bf16(const FfnArgs& f, cudaStream_t s) {
   const bool gather = f.X_perm == nullptr;  // A rows read from X through row_token
   if (gather) {
     // a box one row high: what a 4-row gather needs
-    if (!make_map(&m.xg, f.X, f.n, f.d, 1)) return MOE_ERR_UNSUPPORTED;
+    if (!make_bf16_sw128_map(&m.xg, f.X, f.n, f.d, 1)) return MOE_ERR_UNSUPPORTED;
     m.a0 = m.xg;  // unused for routed tiles when gathering
   } else {
-    if (!make_map(&m.a0, f.X_perm, rows, f.d, kBM)) return MOE_ERR_UNSUPPORTED;
+    if (!make_bf16_sw128_map(&m.a0, f.X_perm, rows, f.d, kBM)) return MOE_ERR_UNSUPPORTED;
     m.xg = m.a0;
   }
   if (f.n_shared > 0) {
-    if (!make_map(&m.a1, f.X, f.n, f.d, kBM)) return MOE_ERR_UNSUPPORTED;
+    if (!make_bf16_sw128_map(&m.a1, f.X, f.n, f.d, kBM)) return MOE_ERR_UNSUPPORTED;
   } else {
     m.a1 = m.a0;
   }
-  if (!make_map(&m.b0, f.W1, (long long)f.E * f.h, f.d, b_box_up)) return MOE_ERR_UNSUPPORTED;
+  if (!make_bf16_sw128_map(&m.b0, f.W1, (long long)f.E * f.h, f.d, b_box_up)) return MOE_ERR_UNSUPPORTED;
   if (swiglu) {
-    if (!make_map(&m.b0g, f.W3, (long long)f.E * f.h, f.d, b_box_up))
+    if (!make_bf16_sw128_map(&m.b0g, f.W3, (long long)f.E * f.h, f.d, b_box_up))
       return MOE_ERR_UNSUPPORTED;
   } else {
     m.b0g = m.b0;
   }
   if (f.n_shared > 0) {
-    if (!make_map(&m.b1, f.sW1, (long long)f.n_shared * f.h, f.d, b_box_up))
+    if (!make_bf16_sw128_map(&m.b1, f.sW1, (long long)f.n_shared * f.h, f.d, b_box_up))
       return MOE_ERR_UNSUPPORTED;
     if (swiglu) {
-      if (!make_map(&m.b1g, f.sW3, (long long)f.n_shared * f.h, f.d, b_box_up))
+      if (!make_bf16_sw128_map(&m.b1g, f.sW3, (long long)f.n_shared * f.h, f.d, b_box_up))
         return MOE_ERR_UNSUPPORTED;
     } else {
       m.b1g = m.b1;
@@ -903,12 +901,12 @@ moe_status run_ffn_bf16(const FfnArgs& f, cudaStream_t s) {
 
   // ---- down projection: Y = H W2^T
   Maps dm;
-  if (!make_map(&dm.a0, f.H, rows, f.h, kBM)) return MOE_ERR_UNSUPPORTED;
+  if (!make_bf16_sw128_map(&dm.a0, f.H, rows, f.h, kBM)) return MOE_ERR_UNSUPPORTED;
   dm.a1 = dm.a0;
-  if (!make_map(&dm.b0, f.W2, (long long)f.E * f.d, f.h, b_box_dn)) return MOE_ERR_UNSUPPORTED;
+  if (!make_bf16_sw128_map(&dm.b0, f.W2, (long long)f.E * f.d, f.h, b_box_dn)) return MOE_ERR_UNSUPPORTED;
   dm.b0g = dm.b0;
   if (f.n_shared > 0) {
-    if (!make_map(&dm.b1, f.sW2, (long long)f.n_shared * f.d, f.h, b_box_dn))
+    if (!make_bf16_sw128_map(&dm.b1, f.sW2, (long long)f.n_shared * f.d, f.h, b_box_dn))
       return MOE_ERR_UNSUPPORTED;
   } else {
     dm.b1 = dm.b0;

@@ -1,6 +1,7 @@
 // Internal host-side declarations shared by the libmoe translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -9,16 +10,19 @@
 
 namespace moe {
 
-constexpr int kTokBlock = 1024;   // tokens per block in the capacity scan
+constexpr int kTokBlock = 256;    // tokens per block in the capacity scan
 constexpr int kRowAlign = MOE_ROW_ALIGN;
 
 inline int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 inline long long round_up(long long a, long long b) { return (a + b - 1) / b * b; }
 
-// Router tile: padded expert count, and rows per CTA for (E, n) (>= 16).
+// Router tile: padded expert count; rows per CTA of the pass that writes the
+// per-CTA column sums (>= 16); k slices (1, or a split-k first pass plus a
+// reduce pass over [ksplit][n][E] partial logits).
 int router_tile_et(int E);
-int router_block_rows(int E, int n);
-constexpr int kRouterMinBlockRows = 16;
+int router_block_rows(int E, int n, int d, bool x_bf16);
+int router_ksplit(int E, int n, int d, bool x_bf16);
+constexpr int kRouterMinBlockRows = 4;  // also the rows per CTA of the split-k reduce
 
 struct Derived {
   int k;            // EC tokens per expert / TC experts per token
@@ -42,10 +46,17 @@ struct WsLayout {
   size_t blk_base;   // [tok_blocks, E] i32
   size_t ec_row;     // [n, E] i32 (expert choice, dense)
   size_t ec_gate;    // [n, E] f32 (expert choice, dense)
+  size_t rpart;      // [ksplit, n, E] f32 split-k router partials (small batches)
   size_t route_end;
   size_t xperm, hbuf, yperm;  // layer only
   size_t layer_end;
 };
+
+// 2-D bf16 row-major [rows, cols] TMA map, box 64 columns x box_rows rows,
+// 128-byte swizzle; out-of-range elements load as zero. False when the shape
+// or alignment cannot be encoded.
+bool make_bf16_sw128_map(CUtensorMap* m, const void* ptr, long long rows, long long cols,
+                         int box_rows);
 
 moe_status derive(const moe_config* c, Derived* d);
 WsLayout ws_layout(const moe_config* c, const Derived& d);
@@ -66,6 +77,8 @@ struct RouterArgs {
   float* lse;        // optional
   float* colsum;     // [blocks, E]
   double* lse2;      // [blocks]
+  float* partial;    // [ksplit, n, E] split-k partial logits (workspace)
+  int ksplit, chunks_per_split;  // set by launch_router
 };
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t s);
 

@@ -34,7 +34,7 @@ struct RCfg {
   static_assert(WY * LY * TN == ET, "columns");
   static_assert(WX * WY * WK == 8, "8 warps");
   static_assert(TN == 4 || TN == 8, "TN");
-  static_assert(TM == 1 || TM == 2 || TM % 4 == 0, "TM");
+  static_assert(TM >= 1 && TM <= 8, "TM");
   static_assert(BK % WK == 0 && ST >= 2, "pipeline");
 };
 // 4 x 8 (E = 64, 128) or 8 x 8 (E = 256) register tiles: the larger the tile
@@ -50,6 +50,15 @@ using R64s = RCfg<64, 4, 8, 4, 1, 1, 8, 64, 4>;
 using R128 = RCfg<128, 4, 8, 4, 2, 2, 2, 32, 4>;
 using R256 = RCfg<256, 8, 8, 4, 1, 4, 2, 32, 3>;
 using R256s = RCfg<256, 2, 8, 4, 2, 4, 1, 32, 3>;
+// bf16 X, E > 32: a family over TM (rows per thread), so that the batch
+// splits into about one CTA's worth of rows per SM (the contraction is bound
+// by the FFMA pipe, so an SM holding two CTAs' rows while another holds one
+// sets the time). "A" splits each chunk's k range over 8 warps (few rows per
+// CTA), "C" over 2 (many rows per CTA).
+template <int TM> using R64A = RCfg<64, TM, 8, 4, 1, 1, 8, 64, 4>;   // BM = 4 TM
+template <int TM> using R64C = RCfg<64, TM, 8, 4, 4, 1, 2, 32, 4>;   // BM = 16 TM
+template <int TM> using R128A = RCfg<128, TM, 8, 4, 2, 2, 2, 32, 4>; // BM = 8 TM
+template <int TM> using R256A = RCfg<256, TM, 8, 4, 1, 4, 2, 32, 3>; // BM = 4 TM
 
 constexpr int kSelectRowsPerWarp = 4;
 
@@ -68,26 +77,89 @@ static int num_sms_cached() {
   return sms;
 }
 
-// Which tile variant a (E, n) uses: the small-row variant when the big tile
-// would leave SMs without a CTA.
-static int router_variant(int E, int n) {
+// Which tile variant a (E, n, X dtype) uses. fp32 X: fixed tiles, the
+// small-row one when the big tile would leave SMs without a CTA. bf16 X with
+// E > 32: the (family, TM) whose rows per SM, BM * ceil(CTAs / SMs), is
+// smallest (ties to the larger BM). Codes: kFamilyCode + fam * 16 + TM with
+// fam 1 = R64A, 2 = R64C, 3 = R128A, 4 = R256A; otherwise the fixed tile's ET
+// (257: R256s, 65: R64s).
+constexpr int kFamilyCode = 1000;
+struct RouterFamily {
+  int code, unit, tm_lo;
+};
+static int router_variant(int E, int n, bool x_bf16) {
   const int et = router_tile_et(E);
   const int sms = num_sms_cached();
+  if (x_bf16 && et >= 64) {
+    static const RouterFamily fams64[] = {{1, 4, 4}, {2, 16, 4}};
+    static const RouterFamily fams128[] = {{3, 8, 2}};
+    static const RouterFamily fams256[] = {{4, 4, 4}};
+    const RouterFamily* fams = et == 64 ? fams64 : et == 128 ? fams128 : fams256;
+    const int nf = et == 64 ? 2 : 1;
+    long long best_cost = -1;
+    int best = 0, best_bm = 0;
+    for (int f = 0; f < nf; ++f)
+      for (int tm = fams[f].tm_lo; tm <= 8; ++tm) {
+        const int bm = fams[f].unit * tm;
+        const long long ctas = (n + bm - 1) / bm;
+        long long cost = (long long)bm * ((ctas + sms - 1) / sms);
+        // measured on B200: R64A (eight-way k split, few rows) pays off only
+        // in a single wave (c2: 28 rows per SM 26.9 us); with more CTAs than
+        // SMs its per-CTA reduction costs more than R64C's (n = 16384: 195 us
+        // vs 174). R64C splits each chunk over only two warp groups, so with
+        // one CTA per SM its eight warps hide too little latency (112 rows
+        // per SM took 203 us, 128 rows in two CTAs 174 us).
+        if (fams[f].code == 1 && ctas > sms) continue;
+        if (fams[f].code == 2 && ctas * 2 < 3LL * sms) cost = cost * 4 / 3;
+        if (best_cost < 0 || cost < best_cost || (cost == best_cost && bm > best_bm)) {
+          best_cost = cost;
+          best = kFamilyCode + fams[f].code * 16 + tm;
+          best_bm = bm;
+        }
+      }
+    return best;
+  }
   if (et == 64) return (n + R64::BM - 1) / R64::BM >= sms ? 64 : 65;
   if (et == 256) return (n + R256::BM - 1) / R256::BM >= sms ? 256 : 257;
   return et;
 }
 
-int router_block_rows(int E, int n) {
-  switch (router_variant(E, n)) {
-    case 8: return R8::BM;
-    case 32: return R32::BM;
-    case 64: return R64::BM;
-    case 65: return R64s::BM;
-    case 128: return R128::BM;
-    case 256: return R256::BM;
-    default: return R256s::BM;
+// rows (BM) and chunk length (BK) of a variant
+static void variant_tile(int v, int* bm, int* bk) {
+  switch (v) {
+    case 8: *bm = R8::BM; *bk = R8::BK; return;
+    case 32: *bm = R32::BM; *bk = R32::BK; return;
+    case 64: *bm = R64::BM; *bk = R64::BK; return;
+    case 65: *bm = R64s::BM; *bk = R64s::BK; return;
+    case 128: *bm = R128::BM; *bk = R128::BK; return;
+    case 256: *bm = R256::BM; *bk = R256::BK; return;
+    case 257: *bm = R256s::BM; *bk = R256s::BK; return;
+    default: {
+      const int code = v - kFamilyCode, fam = code / 16, tm = code % 16;
+      *bm = (fam == 2 ? 16 : fam == 3 ? 8 : 4) * tm;
+      *bk = fam == 1 ? 64 : 32;
+    }
   }
+}
+
+static int split_of(int ctas, int nchunks);
+
+// k slices the router uses for (E, n, d, X dtype): 1, or >= 2 with a reduce
+// pass whose CTAs own 16 rows each
+int router_ksplit(int E, int n, int d, bool x_bf16) {
+  int bm, bk;
+  variant_tile(router_variant(E, n, x_bf16), &bm, &bk);
+  const int nchunks = ceil_div(d, bk);
+  const int ks = split_of(ceil_div(n, bm), nchunks);
+  if (ks == 1) return 1;
+  return ceil_div(nchunks, ceil_div(nchunks, ks));
+}
+
+int router_block_rows(int E, int n, int d, bool x_bf16) {
+  if (router_ksplit(E, n, d, x_bf16) > 1) return kRouterMinBlockRows;
+  int bm, bk;
+  variant_tile(router_variant(E, n, x_bf16), &bm, &bk);
+  return bm;
 }
 
 int select_tc_block_rows() { return 8 * kSelectRowsPerWarp; }
@@ -244,10 +316,15 @@ __device__ __forceinline__ void router_rows_epilogue(const RouterArgs& a, const 
     const float lse = m + logf(z);
 #pragma unroll
     for (int v = 0; v < V; ++v) {
-      if (a.score == MOE_SCORE_SIGMOID)
+      if (a.score == MOE_SCORE_SIGMOID) {
         s[v] = ok[v] ? 1.0f / (1.0f + expf(-l[v])) : 0.0f;
-      else
+      } else if (a.score == MOE_SCORE_SQRTSOFTPLUS) {
+        // sqrt(ln(1 + e^l)), as l + ln(1 + e^-l) for l > 0 (no overflow)
+        const float sp = l[v] > 0.0f ? l[v] + log1pf(expf(-l[v])) : log1pf(expf(l[v]));
+        s[v] = ok[v] ? sqrtf(sp) : 0.0f;
+      } else {
         s[v] = ex[v] / z;
+      }
       csum[v] += ok[v] ? s[v] : 0.0f;
       const int cc = lane * V + v;
       if (ok[v]) {
@@ -302,7 +379,6 @@ struct RouterSmem {
 template <class C, bool XBF16>
 __global__ void __launch_bounds__(256) router_kernel(RouterArgs a) {
   pdl_wait();
-  pdl_trigger();
   using SM = RouterSmem<C, XBF16>;
   constexpr int ET = C::ET, BM = C::BM, BK = C::BK, TM = C::TM, TN = C::TN;
   constexpr int XB = SM::XB, AST = SM::AST;
@@ -364,14 +440,17 @@ __global__ void __launch_bounds__(256) router_kernel(RouterArgs a) {
     }
   };
 
+  // this CTA's k range: all of d, or one of a.ksplit slices of it
   const int nchunks = (d + BK - 1) / BK;
+  const int cb = (int)blockIdx.y * a.chunks_per_split;
+  const int ce = min(nchunks, cb + a.chunks_per_split);
 #pragma unroll 1
-  for (int c = 0; c < C::ST - 1; ++c) {
-    if (c < nchunks) issue(c);
+  for (int c = cb; c < cb + C::ST - 1; ++c) {
+    if (c < ce) issue(c);
     cp_async_commit();
   }
 #pragma unroll 1
-  for (int c = 0; c < nchunks; ++c) {
+  for (int c = cb; c < ce; ++c) {
     cp_async_wait<C::ST - 2>();
     __syncthreads();
     {  // convert the X chunk to fp32, transposed: As[kk][r]
@@ -396,7 +475,7 @@ __global__ void __launch_bounds__(256) router_kernel(RouterArgs a) {
       }
     }
     __syncthreads();
-    if (c + C::ST - 1 < nchunks) issue(c + C::ST - 1);
+    if (c + C::ST - 1 < ce) issue(c + C::ST - 1);
     cp_async_commit();
     const float* ws = Ws + (size_t)(c % C::ST) * BK * ET;
 #pragma unroll
@@ -412,11 +491,16 @@ __global__ void __launch_bounds__(256) router_kernel(RouterArgs a) {
           av[(4 * i4 + 2) % TM] = t.z;
           av[(4 * i4 + 3) % TM] = t.w;
         }
-      } else if (TM == 2) {
-        const float2 t = *reinterpret_cast<const float2*>(As + kk * AST + row0);
-        av[0] = t.x; av[1 % TM] = t.y;
+      } else if (TM % 2 == 0) {
+#pragma unroll
+        for (int i2 = 0; i2 < TM / 2; ++i2) {
+          const float2 t = *reinterpret_cast<const float2*>(As + kk * AST + row0 + 2 * i2);
+          av[(2 * i2) % TM] = t.x;
+          av[(2 * i2 + 1) % TM] = t.y;
+        }
       } else {
-        av[0] = As[kk * AST + row0];
+#pragma unroll
+        for (int i = 0; i < TM; ++i) av[i] = As[kk * AST + row0 + i];
       }
 #pragma unroll
       for (int g = 0; g < TN / 4; ++g) {
@@ -455,32 +539,140 @@ __global__ void __launch_bounds__(256) router_kernel(RouterArgs a) {
     __syncthreads();
   }
 
+  if (a.ksplit > 1) {
+    // a k slice: its partial logits go to a.partial[slice][n][E]; the
+    // reduce kernel sums the slices in order and runs the epilogue
+    float* part = a.partial + (size_t)blockIdx.y * n * E;
+    for (int q = tid; q < BM * E; q += 256) {
+      const int r = q / E, cc = q % E;
+      if (m0 + r < n) part[(size_t)(m0 + r) * E + cc] = Ls[r * LST + cc];
+    }
+    return;
+  }
   float* colsum_w = Ls + C::WK * BM * LST;                          // [8][ET]
   double* lse2_w = reinterpret_cast<double*>(colsum_w + 8 * ET);     // [8]
   router_rows_epilogue<ET>(a, Ls, colsum_w, lse2_w, BM, m0);
 }
 
+// Split-k router, second pass: kRouterMinBlockRows (4) rows per CTA, so that
+// the partials are read by many CTAs at once; each logit is the sum of the k
+// slices' partials in slice order (fixed, so results are reproducible), then
+// the common row epilogue.
+template <int ET>
+__global__ void __launch_bounds__(256) router_reduce_kernel(RouterArgs a) {
+  pdl_wait();
+  constexpr int LST = ET + 1, BMR = kRouterMinBlockRows;
+  __shared__ float Ls[BMR * LST];
+  __shared__ float colsum_w[8 * ET];
+  __shared__ double lse2_w[8];
+  const int n = a.n, E = a.E, m0 = blockIdx.x * BMR;
+  if (E % 4 == 0) {
+    const int E4 = E / 4;
+    for (int q = threadIdx.x; q < BMR * E4; q += 256) {
+      const int r = q / E4, c4 = (q % E4) * 4, t = m0 + r;
+      float4 sum = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      if (t < n) {
+#pragma unroll 8
+        for (int k = 0; k < a.ksplit; ++k) {
+          const float4 v = __ldcg(
+              reinterpret_cast<const float4*>(a.partial + ((size_t)k * n + t) * E + c4));
+          sum.x += v.x;
+          sum.y += v.y;
+          sum.z += v.z;
+          sum.w += v.w;
+        }
+      }
+      float* dst = Ls + r * LST + c4;
+      dst[0] = sum.x;
+      dst[1] = sum.y;
+      dst[2] = sum.z;
+      dst[3] = sum.w;
+    }
+  } else {
+    for (int q = threadIdx.x; q < BMR * E; q += 256) {
+      const int r = q / E, cc = q % E, t = m0 + r;
+      float sum = 0.0f;
+      if (t < n)
+#pragma unroll 8
+        for (int k = 0; k < a.ksplit; ++k) sum += __ldcg(a.partial + ((size_t)k * n + t) * E + cc);
+      Ls[r * LST + cc] = sum;
+    }
+  }
+  __syncthreads();
+  router_rows_epilogue<ET>(a, Ls, colsum_w, lse2_w, BMR, m0);
+}
+
+// k slices for a batch whose row tiles would fill fewer than half the SMs
+// (small batches, decoding): enough slices to give every SM a CTA, each at
+// least two chunks long, at most 32.
+static int split_of(int ctas, int nchunks) {
+  const int sms = num_sms_cached();
+  if (ctas * 2 > sms) return 1;
+  int ks = sms / ctas;
+  if (ks > nchunks / 2) ks = nchunks / 2;
+  if (ks > 32) ks = 32;
+  return ks < 2 ? 1 : ks;
+}
+
 template <class C, bool XBF16>
-static cudaError_t launch_router_t(const RouterArgs& a, cudaStream_t s) {
+static cudaError_t launch_router_t(const RouterArgs& a0, cudaStream_t s) {
   const size_t bytes = RouterSmem<C, XBF16>::bytes;
   auto kern = router_kernel<C, XBF16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)bytes);
   if (e != cudaSuccess) return e;
-  const int grid = ceil_div(a.n, C::BM);
-  return launch_pdl(kern, grid, 256, bytes, s, a);
+  const int grid = ceil_div(a0.n, C::BM);
+  const int nchunks = ceil_div(a0.d, C::BK);
+  RouterArgs a = a0;
+  a.ksplit = router_ksplit(a.E, a.n, a.d, XBF16);
+  a.chunks_per_split = ceil_div(nchunks, a.ksplit);
+  if (a.ksplit > 1 && !a.partial) return cudaErrorInvalidValue;
+  if (a.ksplit == 1) return launch_pdl(kern, grid, 256, bytes, s, a);
+  e = launch_pdl(kern, dim3(grid, a.ksplit), 256, bytes, s, a);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(router_reduce_kernel<C::ET>, ceil_div(a.n, kRouterMinBlockRows), 256, 0,
+                    s, a);
+}
+
+template <template <int> class F>
+static cudaError_t launch_family(int tm, const RouterArgs& a, cudaStream_t s) {
+  switch (tm) {
+    case 2: return launch_router_t<F<2>, true>(a, s);
+    case 3: return launch_router_t<F<3>, true>(a, s);
+    case 4: return launch_router_t<F<4>, true>(a, s);
+    case 5: return launch_router_t<F<5>, true>(a, s);
+    case 6: return launch_router_t<F<6>, true>(a, s);
+    case 7: return launch_router_t<F<7>, true>(a, s);
+    default: return launch_router_t<F<8>, true>(a, s);
+  }
+}
+
+static cudaError_t launch_router_bf16_family(int code, const RouterArgs& a, cudaStream_t s) {
+  const int fam = code / 16, tm = code % 16;
+  switch (fam) {
+    case 1: return launch_family<R64A>(tm, a, s);
+    case 2: return launch_family<R64C>(tm, a, s);
+    case 3: return launch_family<R128A>(tm, a, s);
+    default: return launch_family<R256A>(tm, a, s);
+  }
 }
 
 template <bool XBF16>
 static cudaError_t launch_router_dt(const RouterArgs& a, cudaStream_t s) {
-  switch (router_variant(a.E, a.n)) {
-    case 8: return launch_router_t<R8, XBF16>(a, s);
-    case 32: return launch_router_t<R32, XBF16>(a, s);
-    case 64: return launch_router_t<R64, XBF16>(a, s);
-    case 65: return launch_router_t<R64s, XBF16>(a, s);
-    case 128: return launch_router_t<R128, XBF16>(a, s);
-    case 256: return launch_router_t<R256, XBF16>(a, s);
-    default: return launch_router_t<R256s, XBF16>(a, s);
+  const int v = router_variant(a.E, a.n, XBF16);
+  if constexpr (XBF16) {
+    if (v >= kFamilyCode) return launch_router_bf16_family(v - kFamilyCode, a, s);
+    return v == 8 ? launch_router_t<R8, true>(a, s) : launch_router_t<R32, true>(a, s);
+  } else {
+    switch (v) {
+      case 8: return launch_router_t<R8, false>(a, s);
+      case 32: return launch_router_t<R32, false>(a, s);
+      case 64: return launch_router_t<R64, false>(a, s);
+      case 65: return launch_router_t<R64s, false>(a, s);
+      case 128: return launch_router_t<R128, false>(a, s);
+      case 256: return launch_router_t<R256, false>(a, s);
+      default: return launch_router_t<R256s, false>(a, s);
+    }
   }
 }
 
@@ -497,7 +689,6 @@ cudaError_t launch_router(const RouterArgs& a, cudaStream_t s) {
 template <int V>
 __global__ void __launch_bounds__(256) select_tc_kernel(SelectTcArgs a) {
   pdl_wait();
-  pdl_trigger();
   __shared__ float colsum_w[8][V * 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int rows_per_block = 8 * kSelectRowsPerWarp;

@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_PKG, "libmoe.so")
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, \
     MOE_ERR_TIMEOUT = range(6)
 MOE_EXPERT_CHOICE, MOE_TOKEN_CHOICE = 0, 1
-MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID = 0, 1
+MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID, MOE_SCORE_SQRTSOFTPLUS = 0, 1, 2
 MOE_W_RAW, MOE_W_NORMALIZED = 0, 1
 MOE_ACT_RELU, MOE_ACT_GELU, MOE_ACT_SWIGLU = 0, 1, 2
 MOE_F32, MOE_BF16 = 0, 1
@@ -35,7 +35,8 @@ AUX_NAMES = ["lb_loss", "z_loss", "maxvio", "dropped_assignments", "tokens_some_
 API_SYMBOLS = ["moe_status_string", "moe_validate", "moe_sizes", "moe_workspace_size",
                "moe_route", "moe_route_from_scores", "moe_dispatch", "moe_expert_ffn",
                "moe_combine", "moe_layer_forward", "moe_bias_update", "moe_workspace_init",
-               "moe_read_error", "moe_route_noalloc", "moe_expert_ffn_gathered"]
+               "moe_read_error", "moe_route_noalloc", "moe_expert_ffn_gathered",
+               "moe_launch_counts"]
 MOE_ROUTE_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -137,7 +138,8 @@ def config(w: Workload, **override) -> MoeConfig:
     c = MoeConfig(
         n=w.n, d=w.d, E=w.E, h=w.h,
         mode=MOE_EXPERT_CHOICE if ec else MOE_TOKEN_CHOICE,
-        score=MOE_SCORE_SIGMOID if w.score == "sigmoid" else MOE_SCORE_SOFTMAX,
+        score={"sigmoid": MOE_SCORE_SIGMOID,
+               "sqrtsoftplus": MOE_SCORE_SQRTSOFTPLUS}.get(w.score, MOE_SCORE_SOFTMAX),
         k=0 if ec else w.K,
         capacity_factor=w.c if ec else w.capacity_factor,
         capacity=0 if (not ec and w.capacity_factor > 0) else -1,
@@ -171,6 +173,14 @@ def sizes(cfg: MoeConfig) -> Sizes:
     _check(L.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(r), ctypes.byref(l)),
            "moe_workspace_size")
     return Sizes(k.value, cap.value, slots.value, rows.value, sb.value, r.value, l.value)
+
+
+def launch_counts(cfg: MoeConfig) -> dict:
+    """Kernels each call enqueues: route, dispatch, ffn, combine."""
+    vals = [ctypes.c_int() for _ in range(4)]
+    _check(lib().moe_launch_counts(ctypes.byref(cfg), *(ctypes.byref(v) for v in vals)),
+           "moe_launch_counts")
+    return dict(zip(("route", "dispatch", "ffn", "combine"), (v.value for v in vals)))
 
 
 def validate(cfg: MoeConfig) -> int:

@@ -38,7 +38,7 @@ class Workload:
     E: int
     h: int
     mode: str                 # "ec" (expert choice) or "tc" (token choice)
-    score: str = "softmax"    # "softmax" or "sigmoid"
+    score: str = "softmax"    # "softmax", "sigmoid" or "sqrtsoftplus"
     c: float = 0.0            # EC capacity factor (k = n c / E)
     K: int = 0                # TC experts per token
     capacity_factor: float = 0.0   # TC: > 0 enables a per-expert buffer
@@ -80,6 +80,12 @@ TC_SIGMOID_GROUPED = Workload(
     group_topn=2, weights="normalized", act="swiglu", n_shared=1, bias_steps=10)
 
 FULL = [EC_FP32, EC_BF16, TC_TOP2_CAP, TC_DROPLESS, TC_SIGMOID_GROUPED]
+# the decoding regime of the DeepSeek-V3-shaped layer: 64 tokens, so most of
+# the 256 experts see no token or one; the step streams the active experts'
+# weights (a bench workload, not one of the five configurations)
+DECODE = TC_SIGMOID_GROUPED.replace(
+    name="tc-sigmoid-grouped8keep4-top8of256-shared1-decode-n64-d7168-swiglu2048", n=64,
+    bias_steps=0)
 
 # Reduced sizes of the same five routings: the oracle finishes these in
 # seconds; they still span several GEMM tiles and leave ragged tails.
@@ -94,7 +100,7 @@ SMALL = [
                                "swiglu128", n=300, d=256, E=64, h=128, bias_steps=3),
 ]
 
-BY_NAME = {w.name: w for w in FULL + SMALL}
+BY_NAME = {w.name: w for w in FULL + SMALL + [DECODE]}
 
 
 def _gen(device, seed: int, stream: int) -> torch.Generator:
@@ -129,7 +135,7 @@ def make_inputs(w: Workload, device="cpu", experts: bool = True) -> dict:
     else:
         out["logit_bias"] = None
     out["sel_bias"] = (torch.zeros(w.E, dtype=torch.float32, device=device)
-                       if w.score == "sigmoid" else None)
+                       if w.score in ("sigmoid", "sqrtsoftplus") else None)
     if experts:
         big = w.E * w.h * w.d > (1 << 26)
         out["W1"] = _normal((w.E, w.h, w.d), (2.0 / w.d) ** 0.5, dt, device,

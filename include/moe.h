@@ -83,10 +83,16 @@ typedef enum {
  * choice). */
 typedef enum { MOE_EXPERT_CHOICE = 0, MOE_TOKEN_CHOICE = 1 } moe_mode;
 
-/* softmax over experts ([EC-math] "The transposed selection") or an
+/* softmax over experts ([EC-math] "The transposed selection"), an
  * element-wise sigmoid ([Guide] "4. Sigmoid gating with aux-loss-free
- * bias"). */
-typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score;
+ * bias"), or the element-wise sqrt(softplus(l)) = sqrt(ln(1 + e^l)) that the
+ * same section names for DeepSeek-V4 (the pages give only the name; this is
+ * the plain reading). Selection bias and weight modes apply to every score. */
+typedef enum {
+  MOE_SCORE_SOFTMAX = 0,
+  MOE_SCORE_SIGMOID = 1,
+  MOE_SCORE_SQRTSOFTPLUS = 2
+} moe_score;
 
 /* Token-choice mixing weights: RAW = the score of the selected expert;
  * NORMALIZED = the selected raw scores divided by their sum. For softmax
@@ -175,6 +181,14 @@ MOE_API const char* moe_status_string(moe_status s);
 
 /* Checks a config; MOE_OK if every entry point accepts it. */
 MOE_API moe_status moe_validate(const moe_config* cfg);
+
+/* Kernels each call enqueues for `cfg` on the current device (for graph
+ * capture and accounting): moe_route (router, one more for the split-k
+ * reduce that small batches use, then EC select + finish or TC histogram +
+ * scan + scatter), moe_dispatch, moe_expert_ffn, moe_combine. Any output
+ * pointer may be NULL. No counterpart on the pages. */
+MOE_API moe_status moe_launch_counts(const moe_config* cfg, int* route, int* dispatch,
+                                     int* ffn, int* combine);
 
 /* Derived sizes: k_eff (EC tokens per expert or TC experts per token),
  * capacity_eff (TC rows per expert, -1 dropless), slots (columns of

@@ -33,7 +33,7 @@ def declared_symbols():
 
 def test_every_declared_symbol_is_exported():
     syms = declared_symbols()
-    assert len(syms) == 15
+    assert len(syms) == 16
     assert sorted(moe.API_SYMBOLS) == syms
     L = ctypes.CDLL(moe.LIB_PATH)
     for s in syms:
@@ -177,3 +177,15 @@ def test_binding_refuses_to_run_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(moe, "_LIB", None)
     with pytest.raises(RuntimeError, match="missing"):
         moe.lib()
+
+
+def test_launch_counts():
+    """Kernels per call: the router (plus the split-k reduce that batches too
+    small to fill the SMs take), the selection kernels, one gather, two GEMMs,
+    one combine."""
+    ec = moe.launch_counts(moe.config(wl.EC_BF16))
+    assert ec == {"route": 3, "dispatch": 1, "ffn": 2, "combine": 1}
+    tc = moe.launch_counts(moe.config(wl.TC_DROPLESS))
+    assert tc == {"route": 4, "dispatch": 1, "ffn": 2, "combine": 1}
+    decode = moe.launch_counts(moe.config(wl.DECODE))
+    assert decode["route"] == 5

@@ -34,8 +34,21 @@ def _cleanup():
     torch.cuda.empty_cache()
 
 
+# "7 MoE routing strategies": 2. top-1 switch with a capacity factor, plus a
+# shared expert (Llama 4 Maverick); 5. grouping dropped (n_group = 1, Kimi
+# K2); 4. sqrt(softplus) scores with bias balancing (DeepSeek-V4)
+ROUTE_VARIANTS = [
+    wl.TC_TOP2_CAP.replace(name="tc-switch-top1-cap1.25-shared1", n=384, d=128, E=8, K=1, h=128,
+                           n_shared=1, logit_skew_var=0.0),
+    wl.TC_SIGMOID_GROUPED.replace(name="tc-sigmoid-ngroup1-top8of64", n=260, d=128, E=64, h=64,
+                                  n_groups=1, topk_groups=1, bias_steps=2),
+    wl.TC_SIGMOID_GROUPED.replace(name="tc-sqrtsoftplus-grouped8keep4-top8of64", n=300, d=192,
+                                  E=64, h=64, score="sqrtsoftplus", bias_steps=2),
+]
+
+
 def _sel_bias(w, seed, scale=0.05):
-    if w.score != "sigmoid":
+    if w.score not in ("sigmoid", "sqrtsoftplus"):
         return None
     g = torch.Generator().manual_seed(seed)
     return (torch.randn(w.E, generator=g) * scale).float()
@@ -51,7 +64,7 @@ def _ws_ok(ws):
 # --------------------------------------------------------------------------
 
 @pytest.mark.parametrize("kind", ["random", "ties"])
-@pytest.mark.parametrize("w", wl.SMALL + wl.FULL, ids=lambda w: w.name)
+@pytest.mark.parametrize("w", wl.SMALL + wl.FULL + ROUTE_VARIANTS, ids=lambda w: w.name)
 def test_route_from_scores_bit_exact(w, kind):
     S = (wl.tie_heavy_scores(w.n, w.E, 5, seed=11) if kind == "ties"
          else wl.random_scores(w.n, w.E, seed=12))
@@ -93,7 +106,7 @@ def _oracle_from_x(w, inp):
     return spec, logits, S, lse, r
 
 
-@pytest.mark.parametrize("w", wl.SMALL, ids=lambda w: w.name)
+@pytest.mark.parametrize("w", wl.SMALL + ROUTE_VARIANTS, ids=lambda w: w.name)
 def test_route_from_x(w):
     inp = wl.make_inputs(w, DEV, experts=False)
     cfg = moe.config(w)
@@ -266,7 +279,13 @@ def test_full_size_sampled(w):
 # edge cases
 # --------------------------------------------------------------------------
 
-EDGE = [
+EDGE = ROUTE_VARIANTS + [
+    # about 275 rows per expert, ragged: CTA pairs, with odd 128-row blocks
+    wl.TC_DROPLESS.replace(name="tc-pair-ragged-top2of8", n=1100, d=128, E=8, K=2, h=192),
+    # decoding: a handful of tokens, most experts idle, a shared expert over
+    # fewer rows than one 128-row tile
+    wl.TC_SIGMOID_GROUPED.replace(name="tc-decode-n16-top8of256-shared1", n=16, d=256, E=256,
+                                  h=128, bias_steps=0),
     wl.TC_DROPLESS.replace(name="tc-all-experts-k8of8", n=200, d=128, E=8, K=8, h=128),
     wl.TC_DROPLESS.replace(name="tc-single-expert", n=130, d=64, E=1, K=1, h=64),
     wl.TC_DROPLESS.replace(name="tc-one-token", n=1, d=128, E=16, K=2, h=192),
@@ -333,7 +352,7 @@ def test_dispatch_rejects_misaligned_rows():
 
 
 def test_capacity_one_all_equal_scores():
-    w = EDGE[3]
+    w = next(x for x in EDGE if x.name == "tc-capacity-1")
     cfg = moe.config(w)
     assert moe.sizes(cfg).capacity == 1
     S = torch.full((w.n, w.E), 0.125)
