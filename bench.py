@@ -199,6 +199,41 @@ def traffic_for(kernel_src: str, workload: str):
         return None
 
 
+def routing_stats(w, cfg, inp, rb, ws, moe, stream) -> dict:
+    """The per-workload routing figures: expert choice, the experts-per-token
+    histogram (the pages: most tokens on 1-2 experts, about 23% on 3-4, 3% on
+    more); a capacity, the dropped fractions; the balance and z losses; with a
+    selection bias, MaxVio over the simulated bias-update steps (moe_route
+    then moe_bias_update, the same X and W_g each step)."""
+    aux = rb.aux_dict()
+    out = {}
+    n, K = w.n, w.K
+    if w.mode == "ec":
+        h = rb.ec_hist.cpu().numpy().astype(np.int64)
+        out["experts_per_token"] = {"0": int(h[0]), "1-2": int(h[1:3].sum()),
+                                    "3-4": int(h[3:5].sum()), ">4": int(h[5:].sum())}
+        out["experts_per_token_frac"] = {k: round(v / n, 4)
+                                         for k, v in out["experts_per_token"].items()}
+        return out
+    if w.capacity_factor > 0:
+        out["dropped_assignment_frac"] = round(aux["dropped_assignments"] / (n * K), 4)
+        out["tokens_some_dropped_frac"] = round(aux["tokens_some_dropped"] / n, 4)
+        out["tokens_all_dropped_frac"] = round(aux["tokens_all_dropped"] / n, 4)
+    out["lb_loss"] = round(aux["lb_loss"], 6)
+    out["z_loss"] = round(aux["z_loss"], 6)
+    out["maxvio"] = round(aux["maxvio"], 4)
+    if inp.get("sel_bias") is not None and w.bias_steps > 0:
+        bias = torch.zeros_like(inp["sel_bias"])
+        rb2 = moe.RouteBuffers(cfg, inp["X"].device, logits=False)
+        per_step = []
+        for _ in range(w.bias_steps):
+            moe.moe_route(cfg, inp["X"], inp["Wg"], inp["logit_bias"], bias, rb2, ws, stream)
+            moe.moe_bias_update(cfg, rb2.load, w.bias_rate, bias, stream)
+            per_step.append(round(float(rb2.aux[moe.AUX_NAMES.index("maxvio")].item()), 4))
+        out["maxvio_per_bias_step"] = per_step
+    return out
+
+
 def run_gpu(args, w: wl.Workload):
     import torch.distributed as dist
 
@@ -328,6 +363,10 @@ def run_gpu(args, w: wl.Workload):
     e2e_ms = max_over_ranks(e2e_ms, dev)
 
 
+    # ---- routing statistics the workload statements ask for (from the last
+    # step's routing outputs; untimed)
+    routing = routing_stats(w, cfg, inp, rb, ws, moe, stream)
+
     # ---- algorithmic work and rooflines
     counts = rb.counts.cpu().numpy()
     rows_gathered = int(counts.sum())
@@ -399,6 +438,7 @@ def run_gpu(args, w: wl.Workload):
                    "l2": "flushed between timed steps (256 MB write, outside the events)"},
         "roofline": roof,
         "stages": stages,
+        "routing": routing,
         "stages_note": "medians of a second pass with an event between stages; value and "
                        "ms_per_step come from whole-step events",
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",

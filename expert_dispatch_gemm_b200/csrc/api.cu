@@ -262,6 +262,23 @@ static moe_status route_impl(const moe_config* c, const Derived& dv, const WsLay
 
 // X_perm == NULL: the routed rows are read from X through row_token (the
 // dispatch gather fused into the first projection's A loads)
+// rows per expert on average (token choice: min(nK/E, capacity); expert
+// choice: the padded quota)
+static long long avg_expert_rows(const moe_config* c, const Derived& dv) {
+  if (c->mode != MOE_TOKEN_CHOICE) return dv.kpad;
+  long long avg = ((long long)c->n * dv.k + c->E - 1) / c->E;
+  if (dv.cap > 0 && avg > dv.cap) avg = dv.cap;
+  return avg;
+}
+
+// CTA pairs compute two 128-row blocks of one expert per tile: worth it when
+// experts own at least two blocks on average. With fewer rows per expert
+// (small batches, decoding) half of a pair's MMA work would be padding, and
+// the 128-row tiles of the single-CTA kernel waste half as much.
+bool ffn_uses_pair(const moe_config* c, const Derived& dv) {
+  return c->dtype == MOE_BF16 && avg_expert_rows(c, dv) >= 2 * kRowAlign;
+}
+
 static moe_status ffn_impl(const moe_config* c, const Derived& dv, const void* X,
                            const void* X_perm, const int32_t* row_token, const int32_t* offsets,
                            const void* W1, const void* W3, const void* W2, const void* sW1,
@@ -298,18 +315,7 @@ static moe_status ffn_impl(const moe_config* c, const Derived& dv, const void* X
   f.shared_base = dv.shared_base;
   f.rows = dv.rows;
   f.err = err;
-  // CTA pairs compute two 128-row blocks of one expert per tile: worth it when
-  // experts own at least two blocks on average (expert choice with k > 128;
-  // token choice with min(nK/E, capacity) >= 256). With fewer rows per expert
-  // (small batches, decoding) half of a pair's MMA work would be padding, and
-  // the 128-row tiles of the single-CTA kernel waste half as much.
-  if (c->mode == MOE_TOKEN_CHOICE) {
-    long long avg = ((long long)c->n * dv.k + c->E - 1) / c->E;
-    if (dv.cap > 0 && avg > dv.cap) avg = dv.cap;
-    f.pair = avg >= 2 * kRowAlign;
-  } else {
-    f.pair = dv.kpad >= 2 * kRowAlign;
-  }
+  f.pair = ffn_uses_pair(c, dv);
   return c->dtype == MOE_BF16 ? run_ffn_bf16(f, s) : run_ffn_f32(f, s);
 }
 

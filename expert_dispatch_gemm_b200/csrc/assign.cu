@@ -28,9 +28,9 @@ __device__ __forceinline__ uint32_t ordered_key(float f) {
 // keys beyond that. The dense slot map is [E, n] so each CTA clears and
 // fills its own contiguous row.
 // ---------------------------------------------------------------------------
-constexpr int kEcThreads = 1024;
 constexpr int kEcRankMax = 1024;
-constexpr int kEcMaxPerThread = MOE_EC_MAX_TOKENS / kEcThreads;  // 16 keys in registers
+constexpr int kEcMaxPerThread = 16;  // keys per thread, in registers
+static_assert(MOE_EC_MAX_TOKENS <= 1024 * kEcMaxPerThread, "EC keys must fit in registers");
 
 // exclusive prefix sum over the CTA (threads in order); returns the total.
 // The 32 warp totals are scanned with shuffles by every warp.
@@ -57,7 +57,8 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* excl, int* warp_
   return total;
 }
 
-__global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
+template <int NT>
+__global__ void __launch_bounds__(NT) select_ec_kernel(SelectEcArgs a) {
   pdl_wait();
   extern __shared__ __align__(16) unsigned char ec_smem[];
   const int n = a.n, E = a.E, k = a.k, e = blockIdx.x;
@@ -75,7 +76,7 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
   int32_t* my_rows = a.ec_row + (size_t)e * n;
 
   // thread tid owns tokens [tid*C, tid*C + C), keys kept in registers
-  const int C = (n + kEcThreads - 1) / kEcThreads;
+  const int C = (n + NT - 1) / NT;
   const int t0 = tid * C;
   uint32_t kreg[kEcMaxPerThread];
 #pragma unroll
@@ -83,7 +84,7 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
     const int t = t0 + i;
     kreg[i] = (i < C && t < n) ? ordered_key(a.S[(size_t)t * E + e]) : 0u;
   }
-  for (int t = tid; t < n; t += kEcThreads) my_rows[t] = -1;
+  for (int t = tid; t < n; t += NT) my_rows[t] = -1;
   if (tid == 0) {
     s_prefix = 0u;
     s_mask = 0u;
@@ -113,9 +114,9 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
       }
     }
     __syncthreads();
-    for (int b = tid; b < 256; b += kEcThreads) {
+    for (int b = tid; b < 256; b += NT) {
       int c = 0;
-      for (int w = 0; w < kEcThreads / 32; ++w) c += whist[w * 256 + b];
+      for (int w = 0; w < NT / 32; ++w) c += whist[w * 256 + b];
       hist[b] = c;
     }
     __syncthreads();
@@ -198,7 +199,7 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
   __syncthreads();
   if (by_rank) {
     // composite keys are distinct: a pick's place is how many picks beat it
-    for (int j = tid; j < k; j += kEcThreads) {
+    for (int j = tid; j < k; j += NT) {
       const uint64_t c = sbuf[j];
       int r = 0;
 #pragma unroll 8
@@ -206,11 +207,11 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
       sorted[r] = c;
     }
   } else {
-    for (int i = k + tid; i < kp; i += kEcThreads) sbuf[i] = 0ull;
+    for (int i = k + tid; i < kp; i += NT) sbuf[i] = 0ull;
     __syncthreads();
     for (int size = 2; size <= kp; size <<= 1) {
       for (int stride = size >> 1; stride > 0; stride >>= 1) {
-        for (int i = tid; i < kp / 2; i += kEcThreads) {
+        for (int i = tid; i < kp / 2; i += NT) {
           const int lo = 2 * i - (i & (stride - 1));
           const int hi = lo + stride;
           const bool desc = ((lo & size) == 0);
@@ -225,7 +226,7 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
     }
   }
   __syncthreads();
-  for (int j = tid; j < a.kpad; j += kEcThreads) {
+  for (int j = tid; j < a.kpad; j += NT) {
     const size_t row = (size_t)e * a.kpad + j;
     if (j < k) {
       const int t = (int)(0xffffffffu - (uint32_t)(sorted[j] & 0xffffffffull));
@@ -248,7 +249,7 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
   if (e == 0) {
     // zero what the finish kernel accumulates into, and the fixed aux slots
     if (a.hist)
-      for (int i = tid; i <= E; i += kEcThreads) a.hist[i] = 0;
+      for (int i = tid; i <= E; i += NT) a.hist[i] = 0;
     if (tid < MOE_AUX_LEN && tid != MOE_AUX_Z) a.aux[tid] = 0.0f;
     if (warp == 1) {
       double s = 0.0;
@@ -260,21 +261,27 @@ __global__ void __launch_bounds__(kEcThreads) select_ec_kernel(SelectEcArgs a) {
   }
 }
 
-static size_t select_ec_smem(int n, int k) {
-  (void)n;
+static size_t select_ec_smem(int nt, int k) {
   int kp = 1;
   while (kp < k) kp <<= 1;
   const size_t buf = k <= kEcRankMax ? (size_t)2 * k * 8 : (size_t)kp * 8;
-  return buf + (size_t)(kEcThreads / 32) * 256 * 4;
+  return buf + (size_t)(nt / 32) * 256 * 4;
 }
 
-cudaError_t launch_select_ec(const SelectEcArgs& a, cudaStream_t s) {
-  const size_t bytes = select_ec_smem(a.n, a.k);
-  cudaError_t err = cudaFuncSetAttribute(select_ec_kernel,
+template <int NT>
+static cudaError_t launch_select_ec_t(const SelectEcArgs& a, cudaStream_t s) {
+  const size_t bytes = select_ec_smem(NT, a.k);
+  cudaError_t err = cudaFuncSetAttribute(select_ec_kernel<NT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)bytes);
   if (err != cudaSuccess) return err;
-  return launch_pdl(select_ec_kernel, a.E, kEcThreads, bytes, s, a);
+  return launch_pdl(select_ec_kernel<NT>, a.E, NT, bytes, s, a);
+}
+
+// One thread count for every batch: 256-thread CTAs (cheaper barriers, more
+// keys per thread) measured slower on B200 at n = 4096 (17.7 vs 16.6 us).
+cudaError_t launch_select_ec(const SelectEcArgs& a, cudaStream_t s) {
+  return launch_select_ec_t<1024>(a, s);
 }
 
 // Expert choice: each token's picks (expert order) compacted into its slot

@@ -126,10 +126,14 @@ __global__ void gather_kernel(GatherArgs a, int seg, int nseg, int ring, int slo
   sm100::bulk_wait_all();
 }
 
-// Low fan-out (a token feeds one or two rows on average): one warp per
-// dispatched row, 16-byte vectors, four in flight per lane. A token's row is
-// then read about once anyway, and every row gets its own warp at once,
-// where the staged kernel would serialise a few round trips per warp.
+// Low fan-out (a token feeds one or two rows on average): each warp copies
+// kRowsPerWarp consecutive dispatched rows with 16-byte vectors. The row
+// indices are loaded together, then every row's vectors, so a warp keeps
+// kRowsPerWarp rows' worth of loads in flight instead of one. A token's row
+// is read about once anyway, and the warps cover all rows at once, where the
+// staged kernel would serialise a few round trips per warp.
+constexpr int kRowsPerWarp = 4;
+
 __global__ void __launch_bounds__(256) gather_rows_kernel(GatherArgs a) {
   pdl_wait();
   const long long rows = min((long long)a.offsets[a.E], a.max_rows);
@@ -139,21 +143,31 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(GatherArgs a) {
   const int nvec = a.row_bytes / 16;
   const uint4* src = reinterpret_cast<const uint4*>(a.X);
   uint4* dst = reinterpret_cast<uint4*>(a.X_perm);
-  for (long long r = gw; r < rows; r += nw) {
-    const int t = a.row_token[r];
-    if (t < 0 || t >= a.n) continue;
-    const uint4* sp = src + (size_t)t * nvec;
-    uint4* o = dst + (size_t)r * nvec;
-    int v = lane;
-    for (; v + 96 < nvec; v += 128) {
-      const uint4 x0 = __ldg(sp + v), x1 = __ldg(sp + v + 32), x2 = __ldg(sp + v + 64),
-                  x3 = __ldg(sp + v + 96);
-      o[v] = x0;
-      o[v + 32] = x1;
-      o[v + 64] = x2;
-      o[v + 96] = x3;
+  for (long long r0 = gw * kRowsPerWarp; r0 < rows; r0 += nw * kRowsPerWarp) {
+    int tok[kRowsPerWarp];
+#pragma unroll
+    for (int i = 0; i < kRowsPerWarp; ++i) {
+      const long long r = r0 + i;
+      const int t = r < rows ? a.row_token[r] : -1;
+      tok[i] = (t >= 0 && t < a.n) ? t : -1;
     }
-    for (; v < nvec; v += 32) o[v] = __ldg(sp + v);
+    for (int v0 = 0; v0 < nvec; v0 += 128) {
+      uint4 x[kRowsPerWarp][4];
+#pragma unroll
+      for (int i = 0; i < kRowsPerWarp; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int v = v0 + j * 32 + lane;
+          if (tok[i] >= 0 && v < nvec) x[i][j] = __ldg(src + (size_t)tok[i] * nvec + v);
+        }
+#pragma unroll
+      for (int i = 0; i < kRowsPerWarp; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int v = v0 + j * 32 + lane;
+          if (tok[i] >= 0 && v < nvec) dst[(size_t)(r0 + i) * nvec + v] = x[i][j];
+        }
+    }
   }
 }
 
@@ -173,7 +187,11 @@ cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    return launch_pdl(gather_rows_kernel, sms * 8, 256, 0, s, a);
+    const long long warps = (a.max_rows + kRowsPerWarp - 1) / kRowsPerWarp;
+    long long ctas = (warps + 7) / 8;
+    if (ctas > (long long)sms * 8) ctas = (long long)sms * 8;
+    if (ctas < 1) ctas = 1;
+    return launch_pdl(gather_rows_kernel, (int)ctas, 256, 0, s, a);
   }
   const int nseg = (a.row_bytes + kGatherSeg - 1) / kGatherSeg;
   const int seg = ((a.row_bytes + nseg - 1) / nseg + 15) / 16 * 16;

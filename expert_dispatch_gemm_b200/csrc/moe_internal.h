@@ -191,6 +191,8 @@ struct FfnArgs {
   int* err;
   bool pair;  // bf16: CTA-pair (cta_group::2) kernel instead of the single-CTA one
 };
+// GEMM kernel choice for a config
+bool ffn_uses_pair(const moe_config* c, const Derived& d);
 moe_status run_ffn_bf16(const FfnArgs& a, cudaStream_t s);
 moe_status run_ffn_f32(const FfnArgs& a, cudaStream_t s);
 

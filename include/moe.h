@@ -23,9 +23,10 @@
  *   - Arguments are validated on the host before any launch; on a non-OK
  *     status nothing was enqueued. MOE_ERR_CUDA means a launch failed (the
  *     stream may hold the launches enqueued before it).
- *   - Device-side waits are bounded (about 4 s); a wait that gives up writes
- *     an error code into the first 256 bytes of the workspace, and the
- *     kernel returns. moe_read_error() reports it as MOE_ERR_TIMEOUT.
+ *   - Device-side waits are bounded (2 s each); a wait that gives up writes
+ *     an error code into the first 256 bytes of the workspace (moe_dispatch,
+ *     which takes no workspace: into a per-device word), and the kernel
+ *     returns. moe_read_error() reports it as MOE_ERR_TIMEOUT.
  *   - Indices are int32, gates fp32. Activations X, expert weights, the
  *     dispatched rows, the hidden activations and the expert outputs are
  *     all of the config's dtype (fp32 or bf16); the router weight W_g, the

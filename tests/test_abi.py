@@ -189,3 +189,4 @@ def test_launch_counts():
     assert tc == {"route": 4, "dispatch": 1, "ffn": 2, "combine": 1}
     decode = moe.launch_counts(moe.config(wl.DECODE))
     assert decode["route"] == 5
+    assert moe.launch_counts(moe.config(wl.TC_SIGMOID_GROUPED))["ffn"] == 2

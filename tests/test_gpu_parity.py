@@ -63,8 +63,13 @@ def _ws_ok(ws):
 # identical scores -> bit-exact routing
 # --------------------------------------------------------------------------
 
+# the largest expert-choice batch: 1024-thread selection CTAs, k > 1024 picks
+EC_MAX = wl.EC_BF16.replace(name="ec-max-tokens-n16384-k2048", n=16384, d=64, E=16, h=64, c=2.0)
+
+
 @pytest.mark.parametrize("kind", ["random", "ties"])
-@pytest.mark.parametrize("w", wl.SMALL + wl.FULL + ROUTE_VARIANTS, ids=lambda w: w.name)
+@pytest.mark.parametrize("w", wl.SMALL + wl.FULL + ROUTE_VARIANTS + [EC_MAX],
+                         ids=lambda w: w.name)
 def test_route_from_scores_bit_exact(w, kind):
     S = (wl.tie_heavy_scores(w.n, w.E, 5, seed=11) if kind == "ties"
          else wl.random_scores(w.n, w.E, seed=12))
@@ -280,6 +285,10 @@ def test_full_size_sampled(w):
 # --------------------------------------------------------------------------
 
 EDGE = ROUTE_VARIANTS + [
+    EC_MAX,
+    # a quota of three 128-row blocks per expert: CTA pairs, the second CTA of
+    # an expert's last pair repeats its block and stores nothing
+    wl.EC_BF16.replace(name="ec-k384-odd-blocks", n=768, d=128, E=8, h=128, c=4.0),
     # about 275 rows per expert, ragged: CTA pairs, with odd 128-row blocks
     wl.TC_DROPLESS.replace(name="tc-pair-ragged-top2of8", n=1100, d=128, E=8, K=2, h=192),
     # decoding: a handful of tokens, most experts idle, a shared expert over
