@@ -273,7 +273,8 @@ def run_gpu(args, w: wl.Workload):
         moe.moe_dispatch(cfg, X, rb, X_perm, stream)
         if ev: ev[2].record(stream)
         moe.moe_expert_ffn(cfg, X, X_perm, rb.offsets, inp["W1"], inp["W3"], inp["W2"],
-                           inp.get("sW1"), inp.get("sW3"), inp.get("sW2"), H, Y, ws, stream)
+                           inp.get("sW1"), inp.get("sW3"), inp.get("sW2"), H, Y, ws, stream,
+                           counts=rb.counts)
         if ev: ev[3].record(stream)
         moe.moe_combine(cfg, Y, rb, o, stream)
         if ev: ev[4].record(stream)
@@ -414,7 +415,7 @@ def run_gpu(args, w: wl.Workload):
         roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": tc_peak,
                 "unit": "TFLOP/s", "frac": round(ach / tc_peak, 3),
                 "peak_kind": tc_peak_kind}
-    roof.update({"traffic": traffic, "kernel": "tc_grouped_gemm_kernel (up + down, avg)",
+    roof.update({"traffic": traffic, "kernel": "grouped expert GEMM (up + down launches, avg)",
                  "peak_source": src,
                  "algorithmic_per_launch": bytes_["ffn"] / 2 if roof["bound"] == "hbm"
                  else flops / 2})

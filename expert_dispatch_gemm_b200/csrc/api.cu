@@ -279,9 +279,21 @@ bool ffn_uses_pair(const moe_config* c, const Derived& dv) {
   return c->dtype == MOE_BF16 && avg_expert_rows(c, dv) >= 2 * kRowAlign;
 }
 
+// Fine-grained token choice (128 to 512 rows per expert on average): the
+// weights-as-M down projection computes each expert's exact token count
+// (16-row granularity) where the 128-row tiles would round ~256 rows up to
+// 384 or 512. It needs the counts, which the caller passes. The up
+// projection stays on the token-side kernels, which measured faster there.
+static bool ffn_uses_swap(const moe_config* c, const Derived& dv) {
+  if (c->dtype != MOE_BF16 || c->mode != MOE_TOKEN_CHOICE) return false;
+  const long long avg = avg_expert_rows(c, dv);
+  return avg >= kRowAlign && avg <= 4 * kRowAlign;
+}
+
 static moe_status ffn_impl(const moe_config* c, const Derived& dv, const void* X,
                            const void* X_perm, const int32_t* row_token, const int32_t* offsets,
-                           const void* W1, const void* W3, const void* W2, const void* sW1,
+                           const int32_t* counts, const void* W1, const void* W3,
+                           const void* W2, const void* sW1,
                            const void* sW3, const void* sW2, void* H, void* Y, int* err,
                            cudaStream_t s) {
   if (!offsets || !W1 || !W2 || !H || !Y) return MOE_ERR_INVALID_ARG;
@@ -296,6 +308,7 @@ static moe_status ffn_impl(const moe_config* c, const Derived& dv, const void* X
   f.X_perm = X_perm;
   f.row_token = row_token;
   f.offsets = offsets;
+  f.counts = counts;
   f.W1 = W1;
   f.W3 = W3;
   f.W2 = W2;
@@ -316,7 +329,14 @@ static moe_status ffn_impl(const moe_config* c, const Derived& dv, const void* X
   f.rows = dv.rows;
   f.err = err;
   f.pair = ffn_uses_pair(c, dv);
-  return c->dtype == MOE_BF16 ? run_ffn_bf16(f, s) : run_ffn_f32(f, s);
+  if (c->dtype != MOE_BF16) return run_ffn_f32(f, s);
+  if (ffn_uses_swap(c, dv) && swap_down_supported(f)) {
+    f.skip_down = true;
+    const moe_status st = run_ffn_bf16(f, s);
+    if (st != MOE_OK) return st;
+    return run_ffn_down_swap(f, s);
+  }
+  return run_ffn_bf16(f, s);
 }
 
 // err: the workspace error word, or NULL (standalone moe_dispatch)
@@ -483,17 +503,17 @@ moe_status moe_dispatch(const moe_config* cfg, const void* X, const moe_route_ou
 }
 
 moe_status moe_expert_ffn(const moe_config* cfg, const void* X, const void* X_perm,
-                          const int32_t* offsets, const void* W1, const void* W3,
-                          const void* W2, const void* sW1, const void* sW3, const void* sW2,
-                          void* H, void* Y_perm, void* ws, size_t ws_bytes,
+                          const int32_t* offsets, const int32_t* counts, const void* W1,
+                          const void* W3, const void* W2, const void* sW1, const void* sW3,
+                          const void* sW2, void* H, void* Y_perm, void* ws, size_t ws_bytes,
                           moe_stream_t stream) {
   Derived d;
   moe_status st = derive(cfg, &d);
   if (st != MOE_OK) return st;
   if ((st = check_ws(ws, ws_bytes, MOE_WS_ERROR_BYTES)) != MOE_OK) return st;
   if (!X_perm) return MOE_ERR_INVALID_ARG;
-  return ffn_impl(cfg, d, X, X_perm, nullptr, offsets, W1, W3, W2, sW1, sW3, sW2, H, Y_perm,
-                  at<int>(ws, 0), (cudaStream_t)stream);
+  return ffn_impl(cfg, d, X, X_perm, nullptr, offsets, counts, W1, W3, W2, sW1, sW3, sW2, H,
+                  Y_perm, at<int>(ws, 0), (cudaStream_t)stream);
 }
 
 moe_status moe_combine(const moe_config* cfg, const void* Y_perm, const moe_route_out* route,
@@ -528,7 +548,8 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* X, const float* 
   // 32 four-row TMA gathers per 64-deep k-block, which the TMA unit issues
   // far slower than the two box loads the unfused GEMM needs
   if ((st = dispatch_impl(cfg, d, X, route, xp, at<int>(ws, w.err), s)) != MOE_OK) return st;
-  if ((st = ffn_impl(cfg, d, X, xp, nullptr, route->offsets, W1, W3, W2, sW1, sW3, sW2, hb, yp,
+  if ((st = ffn_impl(cfg, d, X, xp, nullptr, route->offsets, route->counts, W1, W3, W2, sW1,
+                     sW3, sW2, hb, yp,
                      at<int>(ws, w.err), s)) != MOE_OK)
     return st;
   return combine_impl(cfg, d, yp, route, out, s);
@@ -544,7 +565,8 @@ moe_status moe_expert_ffn_gathered(const moe_config* cfg, const void* X,
   if (st != MOE_OK) return st;
   if (!X || !route || !route->row_token || !route->offsets) return MOE_ERR_INVALID_ARG;
   if ((st = check_ws(ws, ws_bytes, MOE_WS_ERROR_BYTES)) != MOE_OK) return st;
-  return ffn_impl(cfg, d, X, nullptr, route->row_token, route->offsets, W1, W3, W2, sW1, sW3,
+  return ffn_impl(cfg, d, X, nullptr, route->row_token, route->offsets, nullptr, W1, W3, W2,
+                  sW1, sW3,
                   sW2, H, Y_perm, at<int>(ws, 0), (cudaStream_t)stream);
 }
 

@@ -890,7 +890,7 @@ moe_status run_ffn_bf16(const FfnArgs& f, cudaStream_t s) {
   p.out = static_cast<__nv_bfloat16*>(f.H);
   p.err = f.err;
   p.row_token = f.row_token;
-  cudaError_t e;
+  cudaError_t e = cudaSuccess;
   const int grid_up = persistent_grid(p, pair);
   switch (f.act) {
     case MOE_ACT_RELU: e = launch_gemm<ACT_RELU>(m, p, pair, gather, grid_up, s); break;
@@ -898,6 +898,7 @@ moe_status run_ffn_bf16(const FfnArgs& f, cudaStream_t s) {
     default: e = launch_gemm<ACT_SWIGLU>(m, p, pair, gather, grid_up, s); break;
   }
   if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if (f.skip_down) return MOE_OK;
 
   // ---- down projection: Y = H W2^T
   Maps dm;

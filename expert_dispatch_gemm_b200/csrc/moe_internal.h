@@ -183,6 +183,7 @@ struct FfnArgs {
   const void* X_perm;   // [rows, d], or NULL: routed rows are read from X via row_token
   const int32_t* row_token;  // [rows] (needed when X_perm is NULL)
   const int32_t* offsets;
+  const int32_t* counts;  // [E] real rows of each segment, or NULL (unknown)
   const void *W1, *W3, *W2, *sW1, *sW3, *sW2;
   void* H;              // [rows, h]
   void* Y;              // [rows, d]
@@ -190,10 +191,14 @@ struct FfnArgs {
   long long rows_routed, shared_base, rows;
   int* err;
   bool pair;  // bf16: CTA-pair (cta_group::2) kernel instead of the single-CTA one
+  bool skip_down;  // run the up projection only
 };
 // GEMM kernel choice for a config
 bool ffn_uses_pair(const moe_config* c, const Derived& d);
 moe_status run_ffn_bf16(const FfnArgs& a, cudaStream_t s);
+// the weights-as-M down projection for fine-grained experts (needs the counts)
+bool swap_down_supported(const FfnArgs& a);
+moe_status run_ffn_down_swap(const FfnArgs& a, cudaStream_t s);
 moe_status run_ffn_f32(const FfnArgs& a, cudaStream_t s);
 
 cudaError_t launch_bias_update(int n, int E, int K, const int32_t* load, float rate,

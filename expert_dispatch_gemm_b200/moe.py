@@ -86,7 +86,7 @@ def lib() -> ctypes.CDLL:
         L.moe_route.argtypes = [cfgp, P, P, P, P, outp, P, ctypes.c_size_t, P]
         L.moe_route_from_scores.argtypes = [cfgp, P, P, outp, P, ctypes.c_size_t, P]
         L.moe_dispatch.argtypes = [cfgp, P, outp, P, P]
-        L.moe_expert_ffn.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P,
+        L.moe_expert_ffn.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P,
                                      ctypes.c_size_t, P]
         L.moe_combine.argtypes = [cfgp, P, outp, P, P]
         L.moe_layer_forward.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, outp, P,
@@ -257,11 +257,11 @@ def moe_dispatch(cfg, X, route: RouteBuffers, X_perm, stream=None):
 
 
 def moe_expert_ffn(cfg, X, X_perm, offsets, W1, W3, W2, sW1, sW3, sW2, H, Y_perm, ws,
-                   stream=None):
+                   stream=None, counts=None):
     _check(lib().moe_expert_ffn(ctypes.byref(cfg), _ptr(X), _ptr(X_perm), _ptr(offsets),
-                                _ptr(W1), _ptr(W3), _ptr(W2), _ptr(sW1), _ptr(sW3), _ptr(sW2),
-                                _ptr(H), _ptr(Y_perm), _ptr(ws), ws.numel(), _stream(stream)),
-           "moe_expert_ffn")
+                                _ptr(counts), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(sW1),
+                                _ptr(sW3), _ptr(sW2), _ptr(H), _ptr(Y_perm), _ptr(ws),
+                                ws.numel(), _stream(stream)), "moe_expert_ffn")
 
 
 def moe_expert_ffn_gathered(cfg, X, route: RouteBuffers, W1, W3, W2, sW1, sW3, sW2, H, Y_perm,

@@ -244,11 +244,16 @@ MOE_API moe_status moe_dispatch(const moe_config* cfg, const void* X, const moe_
  * X. W1, W3 [E,h,d]; W2 [E,d,h]; sW1, sW3 [n_shared,h,d]; sW2
  * [n_shared,d,h]; W3 / sW3 only for SwiGLU (else NULL); shared pointers only
  * when n_shared > 0. H [rows,h] receives the hidden activations, Y_perm
- * [rows,d] the expert outputs (gate not applied). bf16 runs on the tcgen05
- * tensor cores with fp32 accumulation; fp32 runs on FFMA. */
+ * [rows,d] the expert outputs (gate not applied). counts [E] (moe_route's
+ * out->counts: the real rows at the start of each segment) may be NULL; with
+ * it, token choice with 128 to 512 rows per expert on average computes the
+ * down projection for those rows only (16-row granularity, weights as the
+ * MMA's M side) instead of whole 128-row blocks, and rows past counts[e] of
+ * Y_perm are then left unwritten. bf16 runs on the tcgen05 tensor cores with
+ * fp32 accumulation; fp32 runs on FFMA. */
 MOE_API moe_status moe_expert_ffn(const moe_config* cfg, const void* X, const void* X_perm,
-                          const int32_t* offsets, const void* W1, const void* W3,
-                          const void* W2, const void* sW1, const void* sW3,
+                          const int32_t* offsets, const int32_t* counts, const void* W1,
+                          const void* W3, const void* W2, const void* sW1, const void* sW3,
                           const void* sW2, void* H, void* Y_perm, void* ws,
                           size_t ws_bytes, moe_stream_t stream);
 

@@ -162,7 +162,7 @@ def test_null_pointers_and_short_workspace_fail_before_launch():
                              _fake(2), sz.route_ws, None)
     assert st == moe.MOE_ERR_WORKSPACE  # the layer needs the larger workspace
     # SwiGLU without W3
-    st = L.moe_expert_ffn(ctypes.byref(cfg), _fake(0), _fake(1), _fake(2), _fake(3), None,
+    st = L.moe_expert_ffn(ctypes.byref(cfg), _fake(0), _fake(1), _fake(2), None, _fake(3), None,
                           _fake(5), None, None, None, _fake(6), _fake(7), _fake(8), 4096, None)
     assert st == moe.MOE_ERR_INVALID_ARG
     # bias update is a token-choice operation

@@ -167,7 +167,7 @@ def test_stepwise_calls_equal_layer_forward():
     moe.moe_route(cfg, inp["X"], inp["Wg"], None, None, rb, ws)
     moe.moe_dispatch(cfg, inp["X"], rb, X_perm)
     moe.moe_expert_ffn(cfg, inp["X"], X_perm, rb.offsets, inp["W1"], inp["W3"], inp["W2"],
-                       None, None, None, H, Y, ws)
+                       None, None, None, H, Y, ws, counts=rb.counts)
     moe.moe_combine(cfg, Y, rb, out)
     torch.cuda.synchronize()
     assert torch.equal(out, ref)
@@ -286,6 +286,14 @@ def test_full_size_sampled(w):
 
 EDGE = ROUTE_VARIANTS + [
     EC_MAX,
+    # 128 to 512 rows per expert on average: the weights-as-M down projection
+    # (exact token counts, chunks of at most 256 tokens per tile)
+    wl.TC_DROPLESS.replace(name="tc-swap-swiglu-top4of16", n=1024, d=256, E=16, K=4, h=256),
+    wl.TC_DROPLESS.replace(name="tc-swap-gelu-shared-top2of8", n=600, d=256, E=8, K=2, h=256,
+                           act="gelu", n_shared=1),
+    wl.TC_DROPLESS.replace(name="tc-swap-chunks-top1of4", n=2048, d=256, E=4, K=1, h=128),
+    wl.TC_SIGMOID_GROUPED.replace(name="tc-swap-sigmoid-grouped-shared-top8of64", n=2048,
+                                  d=256, E=64, h=128, bias_steps=0),
     # a quota of three 128-row blocks per expert: CTA pairs, the second CTA of
     # an expert's last pair repeats its block and stores nothing
     wl.EC_BF16.replace(name="ec-k384-odd-blocks", n=768, d=128, E=8, h=128, c=4.0),
