@@ -89,9 +89,21 @@ def lib() -> ctypes.CDLL:
                               ctypes.POINTER(c_double)]
         L.orc_bias_update.argtypes = [c_int, c_int, c_int, _i32p, c_float, _f32p]
         L.orc_ec_histogram.argtypes = [c_int, c_int, c_int, _i32p, _i32p]
+        L.orc_combine_backward.argtypes = [c_int, c_int, c_int, _i32p, _f32p, _f32p, _f32p,
+                                           c_int, _f32p, _f32p]
+        L.orc_expert_ffn_backward.argtypes = [c_int, c_int, c_int, c_int, c_int, _f32p, _f32p,
+                                              _opt(_f32p), _f32p, _f32p, _f32p, _f32p,
+                                              _opt(_f32p), _f32p]
+        L.orc_gate_backward_tc.argtypes = [c_int, c_int, c_int, _f32p, _i32p, c_int, _f64p,
+                                           _f64p]
+        L.orc_score_backward.argtypes = [c_int, c_int, c_int, c_int, _f32p, _f32p, _f64p,
+                                         _opt(_i32p), c_double, c_double, _f64p, _f64p]
+        L.orc_router_backward.argtypes = [c_int, c_int, c_int, _f32p, _f32p, _f64p, _f32p,
+                                          _f64p]
         for name in ("orc_router", "orc_select_ec", "orc_select_tc", "orc_capacity",
                      "orc_expert_ffn", "orc_combine", "orc_aux", "orc_bias_update",
-                     "orc_ec_histogram"):
+                     "orc_ec_histogram", "orc_combine_backward", "orc_expert_ffn_backward",
+                     "orc_gate_backward_tc", "orc_score_backward", "orc_router_backward"):
             getattr(L, name).restype = None
         _LIB = L
     return _LIB
@@ -337,3 +349,166 @@ def layer_forward(spec: dict, X, routing: dict, expert_weights, shared_weights=N
     order = np.argsort(np.asarray(ptok, np.int64), kind="stable")
     return combine(len(rows), np.asarray(ptok, np.int32)[order],
                    np.asarray(pgate, np.float32)[order], Yall[order], store)
+
+
+# --------------------------------------------------------------------------
+# backward pass: the chain rule through the steps above
+# --------------------------------------------------------------------------
+
+def combine_backward(pair_token, pair_gate, Y, dout, store: int):
+    """dY[p] = gate[p] dout[token[p]] (stored), dgate[p] = <dout[token[p]], Y[p]>."""
+    Y = _f32(Y)
+    dout = _f32(dout)
+    P, d = Y.shape
+    dY = np.empty((P, d), np.float32)
+    dgate = np.empty((P,), np.float32)
+    if P:
+        lib().orc_combine_backward(dout.shape[0], d, P, _i32(pair_token), _f32(pair_gate), Y,
+                                   dout, store, dY, dgate)
+    return dY, dgate
+
+
+def expert_ffn_backward(X, W1, W3, W2, dY, act: int, store: int):
+    """One expert's backward over its rows: (dX [m,d], dW1 [h,d], dW3 [h,d] or
+    None, dW2 [d,h])."""
+    X = _f32(X)
+    m, d = X.shape
+    h = W1.shape[0]
+    dX = np.empty((m, d), np.float32)
+    dW1 = np.zeros((h, d), np.float32)
+    dW3 = np.zeros((h, d), np.float32) if act == SWIGLU else None
+    dW2 = np.zeros((d, h), np.float32)
+    if m:
+        lib().orc_expert_ffn_backward(m, d, h, act, store, X, _f32(W1),
+                                      None if W3 is None else _f32(W3), _f32(W2), _f32(dY),
+                                      dX, dW1, dW3, dW2)
+    return dX, dW1, dW3, dW2
+
+
+def gate_backward_tc(S, idx, weights: int, dw):
+    """dS [n,E] (double) from the gradients dw [n,K] of the mixing weights."""
+    S = _f32(S)
+    n, E = S.shape
+    K = idx.shape[1]
+    dS = np.zeros((n, E), np.float64)
+    lib().orc_gate_backward_tc(n, E, K, S, _i32(idx), weights,
+                               np.ascontiguousarray(dw, np.float64), dS)
+    return dS
+
+
+def score_backward(logits, S, lse, dS, score: int, load=None, K: int = 1,
+                   lb_coef: float = 0.0, z_coef: float = 0.0):
+    """dL [n,E] (double) from dS, with the balance- and z-loss terms."""
+    S = _f32(S)
+    n, E = S.shape
+    dL = np.empty((n, E), np.float64)
+    lib().orc_score_backward(n, E, K, score, _f32(logits), S,
+                             np.ascontiguousarray(lse, np.float64),
+                             None if load is None else _i32(load), lb_coef, z_coef,
+                             np.ascontiguousarray(dS, np.float64), dL)
+    return dL
+
+
+def router_backward(X, Wg, dL):
+    """(dWg [d,E] fp32, dXr [n,d] double)."""
+    X = _f32(X)
+    Wg = _f32(Wg)
+    n, d = X.shape
+    E = Wg.shape[1]
+    dWg = np.empty((d, E), np.float32)
+    dXr = np.empty((n, d), np.float64)
+    lib().orc_router_backward(n, d, E, X, Wg, np.ascontiguousarray(dL, np.float64), dWg, dXr)
+    return dWg, dXr
+
+
+def layer_backward(spec: dict, X, Wg, dout, expert_weights, shared_weights=None,
+                   logit_bias=None, sel_bias=None, tokens=None):
+    """Gradients of <dout, out> + lb_coef L_lb + z_coef L_z (token choice) for
+    the layer of ``layer_forward``, by the chain rule through the same steps:
+    combine -> expert FFN -> dispatch (a sum over each token's pairs), and
+    mixing weights -> scores -> router. Selections, drops and counts are
+    piecewise constant and carry no gradient.
+
+    Returns a dict: dX [n,d] (rounded to the layer's store), dL [n,E]
+    (double, the logits' gradient), dWg [d,E], dW1/dW3/dW2 {expert: array},
+    dsW1/dsW3/dsW2 {shared expert: array}, dgate {(t, e): value}.
+    With ``tokens`` only those rows of dX and dL are computed (each needs only
+    its own pairs), and no weight gradient is returned."""
+    X = _f32(X)
+    dout = _f32(dout)
+    n, d = X.shape
+    store, act = spec["store"], spec["act"]
+    score = spec.get("score", SOFTMAX)
+    logits, S, lse = router(X, Wg, logit_bias, score)
+    r = route(spec, S, lse, sel_bias)
+    E = S.shape[1]
+    rows = list(range(n)) if tokens is None else sorted(int(t) for t in tokens)
+    pairs = token_pairs(spec, r, n, rows if tokens is not None else None)
+    by_e = {}
+    for t, e, g in pairs:
+        by_e.setdefault(e, []).append((t, g))
+    dXacc = np.zeros((n, d), np.float64)
+    dgate = {}
+    grads = {"dW1": {}, "dW3": {}, "dW2": {}, "dsW1": {}, "dsW3": {}, "dsW2": {}}
+    for e in sorted(by_e):
+        W1, W3, W2 = expert_weights(e)
+        ts = [t for t, _ in by_e[e]]
+        gs = [g for _, g in by_e[e]]
+        Y = expert_ffn(X[ts], W1, W3, W2, act, store)
+        dY, dg = combine_backward(np.asarray(ts, np.int32), np.asarray(gs, np.float32), Y,
+                                  dout, store)
+        for t, v in zip(ts, dg):
+            dgate[(t, e)] = float(v)
+        dXp, dW1, dW3, dW2 = expert_ffn_backward(X[ts], W1, W3, W2, dY, act, store)
+        np.add.at(dXacc, np.asarray(ts), dXp.astype(np.float64))
+        if tokens is None:
+            grads["dW1"][e], grads["dW2"][e] = dW1, dW2
+            if dW3 is not None:
+                grads["dW3"][e] = dW3
+    for s_ in range(spec.get("n_shared", 0)):
+        W1, W3, W2 = shared_weights(s_)
+        dY, _ = combine_backward(np.asarray(rows, np.int32), np.ones(len(rows), np.float32),
+                                 np.zeros((len(rows), d), np.float32), dout, store)
+        dXp, dW1, dW3, dW2 = expert_ffn_backward(X[rows], W1, W3, W2, dY, act, store)
+        dXacc[rows] += dXp.astype(np.float64)
+        if tokens is None:
+            grads["dsW1"][s_], grads["dsW2"][s_] = dW1, dW2
+            if dW3 is not None:
+                grads["dsW3"][s_] = dW3
+    dS = np.zeros((n, E), np.float64)
+    if spec["mode"] == "ec":
+        I = r["I"]
+        for e in range(E):
+            for t in I[e]:
+                t = int(t)
+                if (t, e) in dgate:
+                    dS[t, e] += dgate[(t, e)]
+        lb_coef = z_coef = 0.0
+        K = 1
+    else:
+        idx, drop = r["idx"], r["drop"]
+        K = idx.shape[1]
+        dw = np.zeros(idx.shape, np.float64)
+        for t in rows:
+            for j in range(K):
+                if not drop[t, j]:
+                    dw[t, j] = dgate[(t, int(idx[t, j]))]
+        dS = gate_backward_tc(S, idx, spec.get("weights", W_RAW), dw)
+        lb_coef, z_coef = spec.get("lb_coef", 0.0), spec.get("z_coef", 0.0)
+    dL = score_backward(logits, S, lse, dS, score, r.get("load"), K, lb_coef, z_coef)
+    out = {"dgate": dgate, "routing": r, "logits": logits, "S": S, "lse": lse}
+    if tokens is None:
+        dWg, dXr = router_backward(X, Wg, dL)
+        out["dWg"] = dWg
+        dXacc += dXr
+        rws = slice(None)
+    else:
+        sub = np.asarray(rows)
+        _, dXr = router_backward(X[sub], Wg, dL[sub])
+        dXacc[sub] += dXr
+        rws = sub
+    dXs = dXacc[rws]
+    out["dX"] = round_bf16(dXs) if store == STORE_BF16 else dXs.astype(np.float32)
+    out["dL"] = dL[rws]
+    out.update(grads)
+    return out

@@ -316,3 +316,176 @@ void orc_ec_histogram(int n, int E, int k, const int32_t* I, int32_t* hist) {
   for (int t = 0; t < n; ++t) hist[cnt[t]] += 1;
   free(cnt);
 }
+
+/* ------------------------------------------------------------------ */
+/* backward pass: the gradient of the forward above by the chain rule.   */
+/* [TC-vs-EC] "What each direction guarantees" names the training-time  */
+/* losses (load balance 0.01, router z-loss 0.001) whose gradients join  */
+/* the task gradient here. Storage points mirror the forward: values the */
+/* GPU stores are rounded to `store` where it stores them.               */
+/* ------------------------------------------------------------------ */
+static double sigm(double u) { return 1.0 / (1.0 + exp(-u)); }
+
+/* d act / du; SwiGLU's gate part is handled by the caller */
+static double act_grad(int act, double u) {
+  if (act == ORC_RELU) return u > 0.0 ? 1.0 : 0.0;
+  /* d/du [u Phi(u)] = Phi(u) + u phi(u) */
+  const double pi = 3.14159265358979323846;
+  return 0.5 * (1.0 + erf(u / sqrt(2.0))) + u * exp(-0.5 * u * u) / sqrt(2.0 * pi);
+}
+
+void orc_combine_backward(int n, int d, int P, const int32_t* pair_token,
+                          const float* pair_gate, const float* Y,
+                          const float* dout, int store, float* dY,
+                          float* dgate) {
+  (void)n;
+  for (int p = 0; p < P; ++p) {
+    const int t = pair_token[p];
+    const double gate = pair_gate[p];
+    double s = 0.0;
+    for (int i = 0; i < d; ++i) {
+      const double go = dout[(size_t)t * d + i];
+      dY[(size_t)p * d + i] = round_store(gate * go, store);
+      s += go * (double)Y[(size_t)p * d + i];
+    }
+    dgate[p] = (float)s;
+  }
+}
+
+void orc_expert_ffn_backward(int m, int d, int h, int act, int store,
+                             const float* X, const float* W1, const float* W3,
+                             const float* W2, const float* dY, float* dX,
+                             float* dW1, float* dW3, float* dW2) {
+  const int swiglu = act == ORC_SWIGLU;
+  double* aW1 = (double*)calloc((size_t)h * d, sizeof(double));
+  double* aW3 = swiglu ? (double*)calloc((size_t)h * d, sizeof(double)) : NULL;
+  double* aW2 = (double*)calloc((size_t)d * h, sizeof(double));
+  float* Hs = (float*)malloc(sizeof(float) * (size_t)h);
+  float* dUs = (float*)malloc(sizeof(float) * (size_t)h);
+  float* dVs = (float*)malloc(sizeof(float) * (size_t)h);
+  for (int r = 0; r < m; ++r) {
+    const float* x = X + (size_t)r * d;
+    const float* dy = dY + (size_t)r * d;
+    for (int j = 0; j < h; ++j) {
+      /* pre-activations, as the forward computes them */
+      double u = 0.0, v = 0.0;
+      for (int i = 0; i < d; ++i) u += (double)x[i] * (double)W1[(size_t)j * d + i];
+      if (swiglu)
+        for (int i = 0; i < d; ++i) v += (double)x[i] * (double)W3[(size_t)j * d + i];
+      Hs[j] = round_store(swiglu ? (u / (1.0 + exp(-u))) * v : act_fn(act, u), store);
+      /* the stored pre-activations the backward works from */
+      const double us = round_store(u, store);
+      const double vs = swiglu ? (double)round_store(v, store) : 0.0;
+      /* dH = dY W2 (column j of W2), not stored */
+      double dh = 0.0;
+      for (int i = 0; i < d; ++i) dh += (double)dy[i] * (double)W2[(size_t)i * h + j];
+      if (swiglu) {
+        const double sg = sigm(us);
+        /* silu(u) = u sigma(u); silu'(u) = sigma(u) (1 + u (1 - sigma(u))) */
+        dUs[j] = round_store(dh * vs * sg * (1.0 + us * (1.0 - sg)), store);
+        dVs[j] = round_store(dh * us * sg, store);
+      } else {
+        dUs[j] = round_store(dh * act_grad(act, us), store);
+      }
+    }
+    /* dX = dU W1 (+ dV W3) */
+    for (int i = 0; i < d; ++i) {
+      double a = 0.0;
+      for (int j = 0; j < h; ++j) a += (double)dUs[j] * (double)W1[(size_t)j * d + i];
+      if (swiglu)
+        for (int j = 0; j < h; ++j) a += (double)dVs[j] * (double)W3[(size_t)j * d + i];
+      dX[(size_t)r * d + i] = round_store(a, store);
+    }
+    /* weight gradients: outer products summed over the rows */
+    for (int j = 0; j < h; ++j)
+      for (int i = 0; i < d; ++i) {
+        aW1[(size_t)j * d + i] += (double)dUs[j] * (double)x[i];
+        if (swiglu) aW3[(size_t)j * d + i] += (double)dVs[j] * (double)x[i];
+      }
+    for (int i = 0; i < d; ++i)
+      for (int j = 0; j < h; ++j) aW2[(size_t)i * h + j] += (double)dy[i] * (double)Hs[j];
+  }
+  for (size_t q = 0; q < (size_t)h * d; ++q) {
+    dW1[q] = round_store(aW1[q], store);
+    if (swiglu) dW3[q] = round_store(aW3[q], store);
+    dW2[q] = round_store(aW2[q], store);
+  }
+  free(aW1);
+  free(aW3);
+  free(aW2);
+  free(Hs);
+  free(dUs);
+  free(dVs);
+}
+
+void orc_gate_backward_tc(int n, int E, int K, const float* S,
+                          const int32_t* idx, int weights, const double* dw,
+                          double* dS) {
+  for (int t = 0; t < n; ++t) {
+    const int32_t* it = idx + (size_t)t * K;
+    const double* g = dw + (size_t)t * K;
+    double* ds = dS + (size_t)t * E;
+    if (weights == ORC_W_NORMALIZED) {
+      /* w_k = s_k / sum_j s_j over the K selected experts */
+      double sum = 0.0, dot = 0.0;
+      for (int j = 0; j < K; ++j) sum += (double)S[(size_t)t * E + it[j]];
+      for (int j = 0; j < K; ++j) dot += ((double)S[(size_t)t * E + it[j]] / sum) * g[j];
+      for (int j = 0; j < K; ++j) ds[it[j]] += (g[j] - dot) / sum;
+    } else {
+      for (int j = 0; j < K; ++j) ds[it[j]] += g[j];
+    }
+  }
+}
+
+void orc_score_backward(int n, int E, int K, int score, const float* logits,
+                        const float* S, const double* lse, const int32_t* load,
+                        double lb_coef, double z_coef, const double* dS,
+                        double* dL) {
+  double* g = (double*)malloc(sizeof(double) * (size_t)E);
+  for (int t = 0; t < n; ++t) {
+    const float* L = logits + (size_t)t * E;
+    const float* s = S + (size_t)t * E;
+    double* out = dL + (size_t)t * E;
+    /* dS plus the balance loss: d/dS[t,e] of lb E sum_e f_e mean_t S[t,e],
+     * with f_e = load_e / (n K) held fixed (it counts choices) */
+    for (int e = 0; e < E; ++e) {
+      g[e] = dS[(size_t)t * E + e];
+      if (lb_coef != 0.0)
+        g[e] += lb_coef * E * ((double)load[e] / ((double)n * K)) / n;
+    }
+    if (score == ORC_SIGMOID) {
+      for (int e = 0; e < E; ++e) out[e] = g[e] * (double)s[e] * (1.0 - (double)s[e]);
+    } else if (score == ORC_SQRTSOFTPLUS) {
+      /* s = sqrt(softplus(l)): ds/dl = sigma(l) / (2 s) */
+      for (int e = 0; e < E; ++e) out[e] = g[e] * sigm((double)L[e]) / (2.0 * (double)s[e]);
+    } else {
+      double dot = 0.0;
+      for (int e = 0; e < E; ++e) dot += (double)s[e] * g[e];
+      for (int e = 0; e < E; ++e) out[e] = (double)s[e] * (g[e] - dot);
+    }
+    /* z-loss: z mean_t lse_t^2; d lse_t / d l_e = softmax(l)_e */
+    if (z_coef != 0.0)
+      for (int e = 0; e < E; ++e)
+        out[e] += z_coef * 2.0 * lse[t] / n * exp((double)L[e] - lse[t]);
+  }
+  free(g);
+}
+
+void orc_router_backward(int n, int d, int E, const float* X, const float* Wg,
+                         const double* dL, float* dWg, double* dXr) {
+  double* acc = (double*)calloc((size_t)d * E, sizeof(double));
+  for (int t = 0; t < n; ++t) {
+    const double* g = dL + (size_t)t * E;
+    for (int i = 0; i < d; ++i) {
+      const double x = X[(size_t)t * d + i];
+      double a = 0.0;
+      for (int e = 0; e < E; ++e) {
+        acc[(size_t)i * E + e] += x * g[e];
+        a += g[e] * (double)Wg[(size_t)i * E + e];
+      }
+      dXr[(size_t)t * d + i] = a;
+    }
+  }
+  for (size_t q = 0; q < (size_t)d * E; ++q) dWg[q] = (float)acc[q];
+  free(acc);
+}

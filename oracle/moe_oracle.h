@@ -96,6 +96,54 @@ void orc_bias_update(int n, int E, int K, const int32_t* load, float rate,
  * picked by exactly j experts, j = 0..E. */
 void orc_ec_histogram(int n, int E, int k, const int32_t* I, int32_t* hist);
 
+/* ---- backward pass: the chain rule through the forward above ----------
+ * The loss is <dout, out> + lb_coef L_lb + z_coef L_z (token choice; expert
+ * choice has no aux loss). Counts, selections and drops are piecewise
+ * constant and pass no gradient. Values the GPU stores are rounded to
+ * `store` at the same points: dY, the pre-activations U (= X W1^T) and
+ * V (= X W3^T), dU, dV, the per-row dX of an expert and the weight
+ * gradients. */
+
+/* Combine backward, for each pair p = (token t, gate g): dY[p] = g dout[t]
+ * (rounded to store) and dgate[p] = <dout[t], Y[p]> (double sum, fp32). */
+void orc_combine_backward(int n, int d, int P, const int32_t* pair_token,
+                          const float* pair_gate, const float* Y,
+                          const float* dout, int store, float* dY,
+                          float* dgate);
+
+/* One expert's backward over its m rows X [m,d] with the stored output
+ * gradient dY [m,d]: dH = dY W2; dU = dH * act'(U) (SwiGLU: dU = dH V
+ * silu'(U), dV = dH silu(U), from the stored U, V); dX = dU W1 (+ dV W3)
+ * [m,d]; dW1 = dU^T X, dW3 = dV^T X [h,d]; dW2 = dY^T H [d,h], H as the
+ * forward stores it. dW3 only for SwiGLU (else may be NULL). */
+void orc_expert_ffn_backward(int m, int d, int h, int act, int store,
+                             const float* X, const float* W1, const float* W3,
+                             const float* W2, const float* dY, float* dX,
+                             float* dW1, float* dW3, float* dW2);
+
+/* Token-choice mixing weights backward: dS [n,E] (double, accumulated into)
+ * from the weight gradients dw [n,K] of the selected experts idx [n,K]:
+ * raw weights pass dw through; normalised weights w_k = s_k / sum_j s_j give
+ * dS_k = (dw_k - sum_j w_j dw_j) / sum_j s_j. */
+void orc_gate_backward_tc(int n, int E, int K, const float* S,
+                          const int32_t* idx, int weights, const double* dw,
+                          double* dS);
+
+/* Score backward: dL [n,E] from dS [n,E] plus the balance-loss term
+ * lb_coef E f_e / n (f_e = load_e / (n K)), through softmax (dL = S (dS -
+ * <S, dS>)), sigmoid (dS s (1 - s)) or sqrt(softplus) (dS sigma(l) / (2 s)),
+ * plus the z-loss term z_coef 2 lse_t / n softmax(l_t). lb_coef = 0 and
+ * z_coef = 0 switch the aux terms off (load may then be NULL). */
+void orc_score_backward(int n, int E, int K, int score, const float* logits,
+                        const float* S, const double* lse, const int32_t* load,
+                        double lb_coef, double z_coef, const double* dS,
+                        double* dL);
+
+/* Router backward: dWg = X^T dL [d,E] (fp32), dXr = dL Wg^T [n,d] (double,
+ * the router's share of dX). */
+void orc_router_backward(int n, int d, int E, const float* X, const float* Wg,
+                         const double* dL, float* dWg, double* dXr);
+
 #ifdef __cplusplus
 }
 #endif

@@ -12,6 +12,7 @@ import subprocess
 import pytest
 
 import oracle
+from tests import test_oracle_backward as bwd_pins
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "moe_oracle.c")
@@ -66,6 +67,52 @@ MUTATIONS = [
      "        s = sqrt(sp);",
      "        s = sp;",
      ["test_sqrtsoftplus_closed_forms"]),
+    # backward pass
+    ("SwiGLU backward drops the u (1 - sigma) part of silu'",
+     "dUs[j] = round_store(dh * vs * sg * (1.0 + us * (1.0 - sg)), store);",
+     "dUs[j] = round_store(dh * vs * sg, store);",
+     ["test_backward_matches_finite_differences", "test_expert_backward_against_autograd"]),
+    ("expert input gradient misses the W3 path",
+     "        for (int j = 0; j < h; ++j) a += (double)dVs[j] * (double)W3[(size_t)j * d + i];",
+     "        for (int j = 0; j < h; ++j) a += 0.0 * (double)dVs[j];",
+     ["test_backward_matches_finite_differences", "test_expert_backward_against_autograd"]),
+    ("GELU backward without the u phi(u) term",
+     "return 0.5 * (1.0 + erf(u / sqrt(2.0))) + u * exp(-0.5 * u * u) / sqrt(2.0 * pi);",
+     "return 0.5 * (1.0 + erf(u / sqrt(2.0))) + 0.0 * pi;",
+     ["test_backward_matches_finite_differences", "test_expert_backward_against_autograd"]),
+    ("combine backward forgets the gate in dY",
+     "dY[(size_t)p * d + i] = round_store(gate * go, store);",
+     "dY[(size_t)p * d + i] = round_store(go + 0.0 * gate, store);",
+     ["test_backward_matches_finite_differences"]),
+    ("softmax backward without the <S, dS> term",
+     "for (int e = 0; e < E; ++e) out[e] = (double)s[e] * (g[e] - dot);",
+     "for (int e = 0; e < E; ++e) out[e] = (double)s[e] * g[e] + 0.0 * dot;",
+     ["test_backward_matches_finite_differences",
+      "test_score_and_router_backward_against_autograd"]),
+    ("sigmoid backward as s instead of s (1 - s)",
+     "for (int e = 0; e < E; ++e) out[e] = g[e] * (double)s[e] * (1.0 - (double)s[e]);",
+     "for (int e = 0; e < E; ++e) out[e] = g[e] * (double)s[e];",
+     ["test_backward_matches_finite_differences",
+      "test_score_and_router_backward_against_autograd"]),
+    ("sqrt(softplus) backward without the 1/2",
+     "out[e] = g[e] * sigm((double)L[e]) / (2.0 * (double)s[e]);",
+     "out[e] = g[e] * sigm((double)L[e]) / (double)s[e];",
+     ["test_backward_matches_finite_differences",
+      "test_score_and_router_backward_against_autograd"]),
+    ("z-loss gradient without the factor 2",
+     "out[e] += z_coef * 2.0 * lse[t] / n * exp((double)L[e] - lse[t]);",
+     "out[e] += z_coef * lse[t] / n * exp((double)L[e] - lse[t]);",
+     ["test_backward_matches_finite_differences",
+      "test_score_and_router_backward_against_autograd"]),
+    ("balance-loss gradient not divided by n",
+     "g[e] += lb_coef * E * ((double)load[e] / ((double)n * K)) / n;",
+     "g[e] += lb_coef * E * ((double)load[e] / ((double)n * K));",
+     ["test_backward_matches_finite_differences",
+      "test_score_and_router_backward_against_autograd"]),
+    ("normalised weights backward without the sum w dw term",
+     "for (int j = 0; j < K; ++j) ds[it[j]] += (g[j] - dot) / sum;",
+     "for (int j = 0; j < K; ++j) ds[it[j]] += (g[j] + 0.0 * dot) / sum;",
+     ["test_backward_matches_finite_differences", "test_normalized_gate_backward_closed_form"]),
     ("expert choice gate read from the wrong expert",
      "G[(size_t)e * k + j] = S[(size_t)col[j].idx * E + e];",
      "G[(size_t)e * k + j] = S[(size_t)col[j].idx * E + (e + 1) % E];",
@@ -88,7 +135,7 @@ def _build_mutant(tmp_path, original, mutated):
 
 def _run_pin(name):
     """Run every parametrisation of a pin test; True if all of them pass."""
-    fn = getattr(pins, name)
+    fn = getattr(pins, name, None) or getattr(bwd_pins, name)
     params = getattr(fn, "pytestmark", [])
     cases = [{}]
     for m in params:
