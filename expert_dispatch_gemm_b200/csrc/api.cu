@@ -581,6 +581,293 @@ moe_status moe_bias_update(const moe_config* cfg, const int32_t* load, float rat
   return MOE_OK;
 }
 
+// ---------------------------------------------------------------------------
+// backward pass
+// ---------------------------------------------------------------------------
+struct BwdLayout {
+  size_t err, dy, u, v, hh, duv, dxp, dl, part, end;
+  int splits, launches;
+};
+
+static BwdLayout bwd_layout(const moe_config* c, const Derived& d) {
+  BwdLayout b{};
+  const bool swiglu = c->act == MOE_ACT_SWIGLU;
+  size_t off = 0;
+  b.err = off;
+  off += MOE_WS_ERROR_BYTES;
+  off = align_up(off, 1024);
+  b.dy = off;
+  off = align_up(off + (size_t)d.rows_routed * c->d * 2, 1024);
+  b.u = off;
+  off = align_up(off + (size_t)d.rows * c->h * 2, 1024);
+  b.v = off;
+  if (swiglu) off = align_up(off + (size_t)d.rows * c->h * 2, 1024);
+  b.hh = off;
+  off = align_up(off + (size_t)d.rows * c->h * 2, 1024);
+  b.duv = off;
+  off = align_up(off + (size_t)d.rows * c->h * (swiglu ? 4 : 2), 1024);
+  b.dxp = off;
+  off = align_up(off + (size_t)d.rows * c->d * 2, 1024);
+  b.dl = off;
+  off = align_up(off + (size_t)c->n * c->E * 4, 1024);
+  b.splits = router_bwd_splits(c->n, c->d, c->E);
+  b.part = off;
+  if (b.splits > 1) off = align_up(off + (size_t)b.splits * c->d * c->E * 4, 1024);
+  b.end = off;
+  // pad clear, combine backward, five grouped GEMMs, router dX, router dWg
+  // (+ its ordered reduce)
+  b.launches = 9 + (b.splits > 1 ? 1 : 0);
+  return b;
+}
+
+moe_status moe_backward_workspace_size(const moe_config* cfg, size_t* bytes, int* launches) {
+  Derived d;
+  moe_status st = derive(cfg, &d);
+  if (st != MOE_OK) return st;
+  if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  const BwdLayout b = bwd_layout(cfg, d);
+  if (bytes) *bytes = b.end;
+  if (launches) *launches = b.launches;
+  return MOE_OK;
+}
+
+moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float* Wg,
+                              const void* W1, const void* W3, const void* W2, const void* sW1,
+                              const void* sW3, const void* sW2, const moe_route_out* route,
+                              void* fwd_ws, size_t fwd_ws_bytes, const void* dout, void* dX,
+                              float* dWg, void* dW1, void* dW3, void* dW2, void* dsW1,
+                              void* dsW3, void* dsW2, float* dL, void* ws, size_t ws_bytes,
+                              moe_stream_t stream) {
+  Derived d;
+  moe_status st = derive(cfg, &d);
+  if (st != MOE_OK) return st;
+  if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  const bool swiglu = cfg->act == MOE_ACT_SWIGLU;
+  const bool tc = cfg->mode == MOE_TOKEN_CHOICE;
+  if (!X || !Wg || !W1 || !W2 || !dout || !dX || !dWg || !dW1 || !dW2) return MOE_ERR_INVALID_ARG;
+  if (swiglu && (!W3 || !dW3)) return MOE_ERR_INVALID_ARG;
+  if (cfg->n_shared > 0 && (!sW1 || !sW2 || !dsW1 || !dsW2 || (swiglu && (!sW3 || !dsW3))))
+    return MOE_ERR_INVALID_ARG;
+  if ((st = check_route_out(cfg, route)) != MOE_OK) return st;
+  const bool need_logits = (tc && cfg->z_coef != 0.0f) || cfg->score == MOE_SCORE_SQRTSOFTPLUS;
+  if (need_logits && (!route->logits || (tc && cfg->z_coef != 0.0f && !route->lse)))
+    return MOE_ERR_INVALID_ARG;
+  const WsLayout fw = ws_layout(cfg, d);
+  if ((st = check_ws(fwd_ws, fwd_ws_bytes, fw.layer_end)) != MOE_OK) return st;
+  const BwdLayout b = bwd_layout(cfg, d);
+  if ((st = check_ws(ws, ws_bytes, b.end)) != MOE_OK) return st;
+  const void* aligned[] = {X, dout, dX, fwd_ws, W1, W2, dW1, dW2, W3, dW3,
+                           sW1, sW2, sW3, dsW1, dsW2, dsW3};
+  for (const void* ptr : aligned)
+    if (reinterpret_cast<uintptr_t>(ptr) & 15) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  auto bf = [](const void* p) { return static_cast<__nv_bfloat16*>(const_cast<void*>(p)); };
+  __nv_bfloat16* xp = at<__nv_bfloat16>(fwd_ws, fw.xperm);
+  const __nv_bfloat16* yp = at<__nv_bfloat16>(fwd_ws, fw.yperm);
+  __nv_bfloat16* dy = at<__nv_bfloat16>(ws, b.dy);
+  __nv_bfloat16* U = at<__nv_bfloat16>(ws, b.u);
+  __nv_bfloat16* V = swiglu ? at<__nv_bfloat16>(ws, b.v) : nullptr;
+  __nv_bfloat16* H = at<__nv_bfloat16>(ws, b.hh);
+  __nv_bfloat16* duv = at<__nv_bfloat16>(ws, b.duv);
+  __nv_bfloat16* dxp = at<__nv_bfloat16>(ws, b.dxp);
+  float* dl = dL ? dL : at<float>(ws, b.dl);
+  int* err = at<int>(ws, b.err);
+  const int n = cfg->n, D = cfg->d, h = cfg->h, E = cfg->E, ns = cfg->n_shared;
+  const long long rows = d.rows;
+
+  // 1. padding rows of the dispatched inputs and output gradients read as
+  //    zeros by the weight-gradient reductions
+  MOE_CU(launch_pad_zero(route->offsets, route->counts, E, D, xp, dy, s));
+  // 2. output gradient per kept row, gate gradients, logit gradients
+  CombineBwdArgs cb{};
+  cb.Y_perm = yp;
+  cb.dout = static_cast<const __nv_bfloat16*>(dout);
+  cb.tok_row = route->tok_row;
+  cb.tok_gate = route->tok_gate;
+  cb.idx = route->idx;
+  cb.drop = route->drop;
+  cb.offsets = route->offsets;
+  cb.load = route->load;
+  cb.scores = route->scores;
+  cb.logits = route->logits;
+  cb.lse = route->lse;
+  cb.n = n;
+  cb.d = D;
+  cb.E = E;
+  cb.slots = d.slots;
+  cb.tc = tc;
+  cb.K = tc ? d.k : 0;
+  cb.score = cfg->score;
+  cb.weights = cfg->weights;
+  cb.lb_coef = tc ? cfg->lb_coef : 0.0f;
+  cb.z_coef = tc ? cfg->z_coef : 0.0f;
+  cb.dY_perm = dy;
+  cb.dL = dl;
+  MOE_CU(launch_combine_backward(cb, s));
+
+  BwdParams base{};
+  base.offsets = route->offsets;
+  base.counts = route->counts;
+  base.E = E;
+  base.n_shared = ns;
+  base.n = n;
+  base.swiglu = swiglu;
+  base.act = cfg->act;
+  base.shared_blocks = d.n_pad / kRowAlign;
+  base.max_routed_blocks = (int)(d.rows_routed / kRowAlign);
+  base.out_shared_base = d.shared_base;
+  base.n_pad = d.n_pad;
+  base.err = err;
+  const int rbox = kRowAlign;
+  auto map = [](CUtensorMap* m, const void* p, long long r, long long c, int box) {
+    return make_bf16_sw128_map(m, p, r, c, box);
+  };
+  // 3. SAVE: U (and V), H of every dispatched row again
+  {
+    BwdMaps m{};
+    BwdParams p = base;
+    if (!map(&m.a0, xp, rows, D, rbox)) return MOE_ERR_UNSUPPORTED;
+    m.a1 = m.a0;
+    if (ns > 0 && !map(&m.a1, X, n, D, rbox)) return MOE_ERR_UNSUPPORTED;
+    const int bbox = swiglu ? 128 : 256;
+    if (!map(&m.b0, W1, (long long)E * h, D, bbox)) return MOE_ERR_UNSUPPORTED;
+    m.b0g = m.b0;
+    if (swiglu && !map(&m.b0g, W3, (long long)E * h, D, bbox)) return MOE_ERR_UNSUPPORTED;
+    m.b1 = m.b0;
+    m.b1g = m.b0g;
+    if (ns > 0) {
+      if (!map(&m.b1, sW1, (long long)ns * h, D, bbox)) return MOE_ERR_UNSUPPORTED;
+      if (swiglu && !map(&m.b1g, sW3, (long long)ns * h, D, bbox)) return MOE_ERR_UNSUPPORTED;
+    }
+    p.K = D;
+    p.n_total = h;
+    p.n_block = swiglu ? 128 : 256;
+    p.nt_tiles = ceil_div(h, p.n_block);
+    p.b_rows_per_expert = h;
+    p.out0 = U;
+    p.out1 = V;
+    p.out2 = H;
+    p.ld_out = h;
+    MOE_CU(run_bwd_gemm(BW_SAVE, m, p, s));
+  }
+  // 4. DACT: dU (and dV) = (dY W2) * act'
+  {
+    BwdMaps m{};
+    BwdParams p = base;
+    if (!map(&m.a0, dy, d.rows_routed, D, rbox)) return MOE_ERR_UNSUPPORTED;
+    m.a1 = m.a0;
+    if (ns > 0 && !map(&m.a1, dout, n, D, rbox)) return MOE_ERR_UNSUPPORTED;
+    if (!map(&m.b0, W2, (long long)E * D, h, 64)) return MOE_ERR_UNSUPPORTED;
+    m.b0g = m.b1 = m.b1g = m.b0;
+    if (ns > 0 && !map(&m.b1, sW2, (long long)ns * D, h, 64)) return MOE_ERR_UNSUPPORTED;
+    p.K = D;
+    p.n_total = h;
+    p.n_block = 256;
+    p.nt_tiles = ceil_div(h, 256);
+    p.b_rows_per_expert = D;
+    p.in0 = U;
+    p.in1 = V;
+    p.ld_in = h;
+    p.out0 = duv;
+    p.ld_out = swiglu ? 2LL * h : h;
+    MOE_CU(run_bwd_gemm(BW_DACT, m, p, s));
+  }
+  // 5. DX: dX_perm = dU W1 (+ dV W3)
+  {
+    BwdMaps m{};
+    BwdParams p = base;
+    const long long kcols = swiglu ? 2LL * h : h;
+    if (!map(&m.a0, duv, rows, kcols, rbox)) return MOE_ERR_UNSUPPORTED;
+    m.a1 = m.a0;
+    p.a1_row_base = d.shared_base;
+    p.a1_row_stride = d.n_pad;
+    if (!map(&m.b0, W1, (long long)E * h, D, 64)) return MOE_ERR_UNSUPPORTED;
+    m.b0g = m.b0;
+    if (swiglu && !map(&m.b0g, W3, (long long)E * h, D, 64)) return MOE_ERR_UNSUPPORTED;
+    m.b1 = m.b0;
+    m.b1g = m.b0g;
+    if (ns > 0) {
+      if (!map(&m.b1, sW1, (long long)ns * h, D, 64)) return MOE_ERR_UNSUPPORTED;
+      if (swiglu && !map(&m.b1g, sW3, (long long)ns * h, D, 64)) return MOE_ERR_UNSUPPORTED;
+    }
+    p.K = (int)kcols;
+    p.k_split = h;
+    p.n_total = D;
+    p.n_block = 256;
+    p.nt_tiles = ceil_div(D, 256);
+    p.b_rows_per_expert = h;
+    p.out0 = dxp;
+    p.ld_out = D;
+    MOE_CU(run_bwd_gemm(BW_DX, m, p, s));
+  }
+  // 6. WG2: dW2_e = dY_e^T H_e
+  {
+    BwdMaps m{};
+    BwdParams p = base;
+    if (!map(&m.a0, dy, d.rows_routed, D, 64)) return MOE_ERR_UNSUPPORTED;
+    m.a1 = m.a0;
+    if (ns > 0 && !map(&m.a1, dout, n, D, 64)) return MOE_ERR_UNSUPPORTED;
+    if (!map(&m.b0, H, rows, h, 64)) return MOE_ERR_UNSUPPORTED;
+    m.b0g = m.b1 = m.b1g = m.b0;
+    p.b1_row_base = d.shared_base;
+    p.b1_row_stride = d.n_pad;
+    p.m_total = D;
+    p.m_split = D;
+    p.mt_tiles = ceil_div(D, 128);
+    p.ld_w = h;
+    p.nt_tiles = ceil_div(h, 256);
+    p.w_expert_stride = (long long)D * h;
+    p.w_out0 = bf(dW2);
+    p.w_out1 = bf(dW2);
+    p.sw_out0 = p.sw_out1 = ns > 0 ? bf(dsW2) : bf(dW2);
+    MOE_CU(run_bwd_gemm(BW_WG2, m, p, s));
+  }
+  // 7. WG13: [dW1_e; dW3_e] = [dU_e | dV_e]^T X_e
+  {
+    BwdMaps m{};
+    BwdParams p = base;
+    const long long mcols = swiglu ? 2LL * h : h;
+    if (!map(&m.a0, duv, rows, mcols, 64)) return MOE_ERR_UNSUPPORTED;
+    m.a1 = m.a0;
+    p.a1_row_base = d.shared_base;
+    p.a1_row_stride = d.n_pad;
+    if (!map(&m.b0, xp, rows, D, 64)) return MOE_ERR_UNSUPPORTED;
+    m.b0g = m.b1 = m.b1g = m.b0;
+    if (ns > 0 && !map(&m.b1, X, n, D, 64)) return MOE_ERR_UNSUPPORTED;
+    p.m_total = (int)mcols;
+    p.m_split = h;
+    p.mt_tiles = ceil_div(mcols, 128);
+    p.ld_w = D;
+    p.nt_tiles = ceil_div(D, 256);
+    p.w_expert_stride = (long long)h * D;
+    p.w_out0 = bf(dW1);
+    p.w_out1 = swiglu ? bf(dW3) : bf(dW1);
+    p.sw_out0 = ns > 0 ? bf(dsW1) : bf(dW1);
+    p.sw_out1 = ns > 0 && swiglu ? bf(dsW3) : p.sw_out0;
+    MOE_CU(run_bwd_gemm(BW_WG13, m, p, s));
+  }
+  // 8, 9. router: dX = dL Wg^T + the token's dispatched rows; dWg = X^T dL
+  RouterBwdArgs rb{};
+  rb.X = static_cast<const __nv_bfloat16*>(X);
+  rb.Wg = Wg;
+  rb.dL = dl;
+  rb.dX_perm = dxp;
+  rb.tok_row = route->tok_row;
+  rb.n = n;
+  rb.d = D;
+  rb.E = E;
+  rb.slots = d.slots;
+  rb.n_shared = ns;
+  rb.shared_base = d.shared_base;
+  rb.n_pad = d.n_pad;
+  rb.dX = static_cast<__nv_bfloat16*>(dX);
+  rb.dWg = dWg;
+  rb.partial = at<float>(ws, b.part);
+  rb.splits = b.splits;
+  MOE_CU(launch_router_backward(rb, s));
+  return MOE_OK;
+}
+
 moe_status moe_workspace_init(void* ws, moe_stream_t stream) {
   if (!ws) return MOE_ERR_WORKSPACE;
   MOE_CU(cudaMemsetAsync(ws, 0, MOE_WS_ERROR_BYTES, (cudaStream_t)stream));

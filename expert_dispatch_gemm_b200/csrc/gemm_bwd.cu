@@ -1,0 +1,583 @@
+// Grouped expert GEMMs of the layer's backward pass on the tcgen05 tensor
+// cores.
+//
+// The backward of "Expert choice routing" (aicassindra.com), "The math: a
+// gating matrix and top-k over tokens": the per-expert FFN Y = act(X W1^T
+// [, X W3^T]) W2^T is differentiated by the chain rule, one grouped GEMM per
+// step:
+//   SAVE   [U | V], H = X W1^T, X W3^T, act      (the forward's up projection
+//                                                 again, keeping U and V)
+//   DACT   dU, dV = (dY W2) * act'(U, V)          (W2 read MN-major)
+//   DX     dX_perm = dU W1 + dV W3                (W1, W3 read MN-major)
+//   WG2    dW2_e = dY_e^T H_e                     (both operands MN-major,
+//   WG13   [dW1_e; dW3_e] = [dU_e | dV_e]^T X_e    K = the expert's rows)
+// The first three tile the dispatched rows like the forward kernels (128-row
+// blocks of one expert x 256 output columns, shared experts after the routed
+// ones); the weight gradients tile each expert's output matrix (128 x 256)
+// and reduce over its rows.
+//
+// One persistent CTA per SM: warp 0 issues the TMA loads into a 4-stage ring
+// (A 128x64 and B 256x64 per stage), warp 1 issues tcgen05.mma (M128 N256
+// K16) into one of two TMEM accumulators, warps 2-5 run the epilogue. An
+// operand that is K-major in memory comes in as one 128-byte-swizzled box;
+// an MN-major one (a weight matrix read along its input dimension, or a row
+// block read across its columns) as boxes of 64 MN-elements x 64 K-rows,
+// described to the MMA as the canonical MN-major 128-byte-swizzle layout:
+// 64 contiguous MN-elements per 128-byte row, eight K-rows per 1024-byte
+// swizzle atom (the stride between atoms along K), and 8 KB between
+// consecutive 64-element MN chunks.
+// Every mbarrier wait is bounded (2 s): on a timeout the CTA records an
+// error, stops issuing, waits (bounded) for its own copies and MMAs, frees
+// TMEM and returns.
+#include <cuda.h>
+#include <math.h>
+
+#include "device_common.cuh"
+#include "moe_internal.h"
+#include "sm100.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kWBM = 128, kWBN = 256, kWBK = 64, kWStages = 4;
+constexpr int kWABytes = kWBM * kWBK * 2;     // 16 KB
+constexpr int kWBBytes = kWBN * kWBK * 2;     // 32 KB
+constexpr int kWStageBytes = kWABytes + kWBBytes;
+constexpr int kWThreads = 192;
+constexpr uint64_t kWWaitNs = 2000000000ull;  // 2 s
+constexpr uint32_t kMnChunkBytes = 64 * kWBK * 2;  // one 64 x 64 MN-major box: 8 KB
+
+struct BwdState {
+  uint64_t full[kWStages];
+  uint64_t empty[kWStages];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  volatile int abort_flag;
+  int offs[MOE_MAX_EXPERTS + 1];
+  int cnt[MOE_MAX_EXPERTS];
+  int tprefix[MOE_MAX_EXPERTS + 1];
+};
+
+__device__ __forceinline__ bool bwait(uint64_t* bar, uint32_t parity, BwdState* st, int* err,
+                                      int code) {
+  if (sm100::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (sm100::mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (st->abort_flag) return false;
+      if (global_timer_ns() - t0 > kWWaitNs) {
+        st->abort_flag = 1;
+        report_error(err, code);
+        return false;
+      }
+    }
+  }
+}
+
+// canonical MN-major layout with 128-byte swizzle: start address >> 4 in
+// [0,14), leading byte offset (between 64-element MN chunks) >> 4 in [16,30),
+// stride byte offset (between 8-row K groups, 1024 B) >> 4 in [32,46),
+// descriptor version 1 in [46,48), swizzle mode 2 (128 B) in [61,64)
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)(kMnChunkBytes >> 4) << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// kind::f16 instruction descriptor with the operands' majorness: bit 15 = A
+// MN-major, bit 16 = B MN-major
+__host__ __device__ constexpr uint32_t idesc_major(bool a_mn, bool b_mn) {
+  return sm100::idesc_bf16_f32(kWBM, kWBN) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16);
+}
+
+template <int MODE>
+struct ModeTraits {
+  static constexpr bool A_MN = MODE == BW_WG2 || MODE == BW_WG13;
+  static constexpr bool B_MN = MODE != BW_SAVE;
+  static constexpr bool WGRAD = A_MN;
+};
+
+struct BTile {
+  bool skip;           // a weight-gradient tile of an expert with no rows: write zeros
+  bool shared;
+  int expert;          // routed expert or shared index
+  int a_row;           // K-major A: first row; MN-major A: first K row
+  int b_row;           // K-major B: first row; MN-major B: first K row
+  int m0, n0;          // weight gradients: output block; row modes: n0 = first column
+  int kb;              // k-blocks of this tile
+  long long out_row;   // row modes: first output row
+};
+
+// Row modes: tiles expert by expert, 256-column block by block, the expert's
+// 128-row blocks innermost; shared experts after the routed ones.
+// Weight-gradient modes: expert by expert, 128-row output block, 256-column
+// output block innermost.
+template <int MODE>
+__device__ __forceinline__ BTile decode(int tile, const BwdParams& p, const BwdState* st,
+                                        int routed) {
+  BTile t{};
+  if (!ModeTraits<MODE>::WGRAD) {
+    int nt;
+    if (tile < routed) {
+      int lo = 0, hi = p.E - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (st->tprefix[mid] <= tile) lo = mid; else hi = mid - 1;
+      }
+      const int local = tile - st->tprefix[lo];
+      const int blocks = max((st->offs[lo + 1] - st->offs[lo]) / kWBM, 1);
+      nt = local / blocks;
+      t.a_row = st->offs[lo] + (local % blocks) * kWBM;
+      t.out_row = t.a_row;
+      t.expert = lo;
+      t.shared = false;
+    } else {
+      const int per = p.shared_blocks * p.nt_tiles;
+      const int q = tile - routed;
+      const int s = q / per, local = q % per;
+      nt = local / p.shared_blocks;
+      const int lm = local % p.shared_blocks;
+      t.a_row = (int)(p.a1_row_base + s * p.a1_row_stride + (long long)lm * kWBM);
+      t.out_row = p.out_shared_base + s * p.n_pad + (long long)lm * kWBM;
+      t.expert = s;
+      t.shared = true;
+    }
+    t.n0 = nt * p.n_block;
+    t.kb = p.K / kWBK;
+    // K-major B (SAVE): the expert's weight rows of this column block;
+    // MN-major B: the expert's first K row
+    t.b_row = MODE == BW_SAVE ? t.expert * p.b_rows_per_expert + t.n0
+                              : t.expert * p.b_rows_per_expert;
+  } else {
+    const int per = p.mt_tiles * p.nt_tiles;
+    const int q = tile / per, local = tile % per;
+    t.m0 = (local / p.nt_tiles) * kWBM;
+    t.n0 = (local % p.nt_tiles) * kWBN;
+    if (q < p.E) {
+      const int rows = st->cnt[q];
+      t.kb = (rows + kWBK - 1) / kWBK;
+      t.a_row = st->offs[q];
+      t.b_row = st->offs[q];
+      t.expert = q;
+      t.shared = false;
+    } else {
+      const int s = q - p.E;
+      t.kb = (p.n + kWBK - 1) / kWBK;
+      t.a_row = (int)(p.a1_row_base + s * p.a1_row_stride);
+      t.b_row = (int)(p.b1_row_base + s * p.b1_row_stride);
+      t.expert = s;
+      t.shared = true;
+    }
+    t.skip = t.kb == 0;
+  }
+  return t;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kWThreads, 1)
+    tc_bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,
+                       const __grid_constant__ CUtensorMap tmA1,
+                       const __grid_constant__ CUtensorMap tmB0,
+                       const __grid_constant__ CUtensorMap tmB0g,
+                       const __grid_constant__ CUtensorMap tmB1,
+                       const __grid_constant__ CUtensorMap tmB1g, const BwdParams p) {
+  using Tr = ModeTraits<MODE>;
+  extern __shared__ __align__(1024) unsigned char bsm[];
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(bsm) + 1023) & ~uintptr_t(1023));
+  unsigned char* sA = base;
+  unsigned char* sB = base + kWStages * kWABytes;
+  BwdState* st = reinterpret_cast<BwdState*>(base + kWStages * kWStageBytes);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < kWStages; ++s) {
+      sm100::mbar_init(&st->full[s], 1);
+      sm100::mbar_init(&st->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      sm100::mbar_init(&st->tfull[a], 1);
+      sm100::mbar_init(&st->tempty[a], 128);
+    }
+    sm100::mbar_init(&st->drain, 1);
+    st->abort_flag = 0;
+    sm100::fence_mbar_init();
+  }
+  if (warp == 1) {
+    sm100::tmem_alloc(&st->tmem_base, 512);
+    sm100::tmem_relinquish();
+  }
+  pdl_wait();
+  for (int i = tid; i <= p.E; i += kWThreads) st->offs[i] = p.offsets[i];
+  for (int i = tid; i < p.E; i += kWThreads) {
+    const int seg = p.offsets[i + 1] - p.offsets[i];
+    const int c = p.counts ? p.counts[i] : seg;
+    st->cnt[i] = max(0, min(c, seg));
+  }
+  __syncthreads();
+  if (tid == 0 && !Tr::WGRAD) {
+    int run = 0;
+    for (int e = 0; e < p.E; ++e) {
+      st->tprefix[e] = run;
+      run += max(st->offs[e + 1] - st->offs[e], 0) / kWBM * p.nt_tiles;
+    }
+    st->tprefix[p.E] = run;
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem = st->tmem_base;
+
+  int routed, total;
+  if (Tr::WGRAD) {
+    routed = p.E * p.mt_tiles * p.nt_tiles;
+    total = (p.E + p.n_shared) * p.mt_tiles * p.nt_tiles;
+  } else {
+    routed = min(st->tprefix[p.E], p.max_routed_blocks * p.nt_tiles);
+    total = routed + p.n_shared * p.shared_blocks * p.nt_tiles;
+  }
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0, issued = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        const BTile t = decode<MODE>(tile, p, st, routed);
+        if (t.skip) continue;
+        const CUtensorMap* ma = t.shared ? &tmA1 : &tmA0;
+        for (int kb = 0; kb < t.kb; ++kb) {
+          if (!bwait(&st->empty[stage], phase ^ 1u, st, p.err, kErrGemmTimeout | 0x51)) {
+            ok = false;
+            break;
+          }
+          uint64_t* fb = &st->full[stage];
+          unsigned char* a_dst = sA + stage * kWABytes;
+          unsigned char* b_dst = sB + stage * kWBBytes;
+          sm100::mbar_arrive_expect_tx(fb, kWStageBytes);
+          const int k0 = kb * kWBK;
+          if (Tr::A_MN) {
+#pragma unroll
+            for (int c = 0; c < kWBM / 64; ++c)
+              sm100::tma_load_2d(a_dst + c * kMnChunkBytes, ma, fb, t.m0 + 64 * c, t.a_row + k0);
+          } else {
+            sm100::tma_load_2d(a_dst, ma, fb, k0, t.a_row);
+          }
+          if (MODE == BW_SAVE) {
+            const CUtensorMap* mb = t.shared ? &tmB1 : &tmB0;
+            if (p.swiglu) {
+              const CUtensorMap* mbg = t.shared ? &tmB1g : &tmB0g;
+              sm100::tma_load_2d(b_dst, mb, fb, k0, t.b_row);
+              sm100::tma_load_2d(b_dst + kWBBytes / 2, mbg, fb, k0, t.b_row);
+            } else {
+              sm100::tma_load_2d(b_dst, mb, fb, k0, t.b_row);
+            }
+          } else {
+            // MN-major B: four 64-column chunks of K rows k0..k0+63
+            const CUtensorMap* mb;
+            int krow;
+            if (MODE == BW_DX && k0 >= p.k_split) {
+              mb = t.shared ? &tmB1g : &tmB0g;
+              krow = t.b_row + k0 - p.k_split;
+            } else {
+              mb = t.shared ? &tmB1 : &tmB0;
+              krow = t.b_row + k0;
+            }
+#pragma unroll
+            for (int c = 0; c < kWBN / 64; ++c)
+              sm100::tma_load_2d(b_dst + c * kMnChunkBytes, mb, fb, t.n0 + 64 * c, krow);
+          }
+          ++issued;
+          if (++stage == kWStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        int s = stage;
+        uint32_t ph = phase;
+        const int pending = issued < kWStages ? issued : kWStages;
+        for (int i = 0; i < pending; ++i) {
+          if (--s < 0) {
+            s = kWStages - 1;
+            ph ^= 1u;
+          }
+          const uint64_t t0 = global_timer_ns();
+          while (!sm100::mbar_try_wait(&st->full[s], ph) && global_timer_ns() - t0 < kWWaitNs) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_major(Tr::A_MN, Tr::B_MN);
+      int stage = 0, used = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        const BTile t = decode<MODE>(tile, p, st, routed);
+        if (t.skip) continue;
+        const int acc = used & 1;
+        const uint32_t acc_phase = (uint32_t)(used >> 1) & 1u;
+        ++used;
+        if (!bwait(&st->tempty[acc], acc_phase ^ 1u, st, p.err, kErrGemmTimeout | 0x52)) {
+          ok = false;
+          break;
+        }
+        sm100::tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(acc * kWBN);
+        for (int kb = 0; kb < t.kb; ++kb) {
+          if (!bwait(&st->full[stage], phase, st, p.err, kErrGemmTimeout | 0x53)) {
+            ok = false;
+            break;
+          }
+          sm100::tc_fence_after();
+          const uint32_t a_addr = sm100::smem_addr(sA + stage * kWABytes);
+          const uint32_t b_addr = sm100::smem_addr(sB + stage * kWBBytes);
+          const uint64_t adesc =
+              Tr::A_MN ? sw128_mnmajor_desc(a_addr) : sm100::sw128_kmajor_desc(a_addr);
+          const uint64_t bdesc =
+              Tr::B_MN ? sw128_mnmajor_desc(b_addr) : sm100::sw128_kmajor_desc(b_addr);
+          // one K16 step: +32 bytes inside a K-major row (+2 in the address
+          // field); +16 rows of 128 bytes in an MN-major tile (+128)
+          constexpr uint64_t a_step = Tr::A_MN ? 128 : 2;
+          constexpr uint64_t b_step = Tr::B_MN ? 128 : 2;
+#pragma unroll
+          for (int k = 0; k < kWBK / 16; ++k)
+            sm100::umma_f16(d_tmem, adesc + a_step * k, bdesc + b_step * k, idesc, (kb | k) != 0);
+          sm100::umma_commit(&st->empty[stage]);
+          if (++stage == kWStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        sm100::umma_commit(&st->tfull[acc]);
+      }
+      sm100::umma_commit(&st->drain);
+      const uint64_t t0 = global_timer_ns();
+      while (!sm100::mbar_try_wait(&st->drain, 0) && global_timer_ns() - t0 < kWWaitNs) {
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    const int row_in_tile = q * 32 + lane;
+    int used = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      const BTile t = decode<MODE>(tile, p, st, routed);
+      if (Tr::WGRAD) {
+        // this thread's output row of the weight gradient
+        const int m = t.m0 + row_in_tile;
+        __nv_bfloat16* orow = nullptr;
+        if (m < p.m_total) {
+          const bool hi = m >= p.m_split;
+          __nv_bfloat16* dst = t.shared ? (hi ? p.sw_out1 : p.sw_out0) : (hi ? p.w_out1 : p.w_out0);
+          orow = dst + (size_t)t.expert * p.w_expert_stride +
+                 (size_t)(hi ? m - p.m_split : m) * p.ld_w;
+        }
+        if (t.skip) {
+          if (orow) {
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            for (int cc = 0; cc < kWBN && t.n0 + cc < p.ld_w; cc += 8)
+              *reinterpret_cast<uint4*>(orow + t.n0 + cc) = z;
+          }
+          continue;
+        }
+      }
+      const int acc = used & 1;
+      const uint32_t acc_phase = (uint32_t)(used >> 1) & 1u;
+      ++used;
+      if (!bwait(&st->tfull[acc], acc_phase, st, p.err, kErrGemmTimeout | 0x54)) break;
+      sm100::tc_fence_after();
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kWBN);
+      if (Tr::WGRAD) {
+        const int m = t.m0 + row_in_tile;
+        const bool hi = m >= p.m_split;
+        __nv_bfloat16* dst = t.shared ? (hi ? p.sw_out1 : p.sw_out0) : (hi ? p.w_out1 : p.w_out0);
+        __nv_bfloat16* orow = dst + (size_t)t.expert * p.w_expert_stride +
+                              (size_t)(hi ? m - p.m_split : m) * p.ld_w;
+#pragma unroll 1
+        for (int cc = 0; cc < kWBN; cc += 32) {
+          if (t.n0 + cc >= p.ld_w) break;
+          uint32_t v[32];
+          sm100::tmem_ld_32x32b_x32(tbase + cc, v);
+          sm100::tmem_ld_wait();
+          if (m < p.m_total) {
+            uint4* o = reinterpret_cast<uint4*>(orow + t.n0 + cc);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              o[j] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1])),
+                                pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
+                                pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
+                                pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
+          }
+        }
+      } else {
+        const long long row = t.out_row + row_in_tile;
+        const int ncols = MODE == BW_SAVE && p.swiglu ? kWBN / 2 : kWBN;
+#pragma unroll 1
+        for (int cc = 0; cc < ncols; cc += 32) {
+          const int col = t.n0 + cc;
+          if (col >= p.n_total) break;
+          uint32_t v[32];
+          sm100::tmem_ld_32x32b_x32(tbase + cc, v);
+          float f[32], g[32];
+          if (MODE == BW_SAVE && p.swiglu) {
+            uint32_t w[32];
+            sm100::tmem_ld_32x32b_x32(tbase + kWBN / 2 + cc, w);
+            sm100::tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              f[i] = __uint_as_float(v[i]);
+              g[i] = __uint_as_float(w[i]);
+            }
+          } else {
+            sm100::tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
+          }
+          if (MODE == BW_SAVE) {
+            // U (and V) as stored pre-activations, H as the forward computes it
+            uint4* du = reinterpret_cast<uint4*>(p.out0 + row * p.ld_out + col);
+            uint4* dh = reinterpret_cast<uint4*>(p.out2 + row * p.ld_out + col);
+            float hv[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              if (p.swiglu) hv[i] = f[i] * __frcp_rn(1.0f + __expf(-f[i])) * g[i];
+              else if (p.act == MOE_ACT_RELU) hv[i] = fmaxf(f[i], 0.0f);
+              else hv[i] = 0.5f * f[i] * (1.0f + erff(f[i] * 0.70710678118654752f));
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              du[j] = make_uint4(pack_bf16x2(f[8 * j], f[8 * j + 1]), pack_bf16x2(f[8 * j + 2], f[8 * j + 3]),
+                                 pack_bf16x2(f[8 * j + 4], f[8 * j + 5]), pack_bf16x2(f[8 * j + 6], f[8 * j + 7]));
+              dh[j] = make_uint4(pack_bf16x2(hv[8 * j], hv[8 * j + 1]), pack_bf16x2(hv[8 * j + 2], hv[8 * j + 3]),
+                                 pack_bf16x2(hv[8 * j + 4], hv[8 * j + 5]), pack_bf16x2(hv[8 * j + 6], hv[8 * j + 7]));
+            }
+            if (p.swiglu) {
+              uint4* dv = reinterpret_cast<uint4*>(p.out1 + row * p.ld_out + col);
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                dv[j] = make_uint4(pack_bf16x2(g[8 * j], g[8 * j + 1]), pack_bf16x2(g[8 * j + 2], g[8 * j + 3]),
+                                   pack_bf16x2(g[8 * j + 4], g[8 * j + 5]), pack_bf16x2(g[8 * j + 6], g[8 * j + 7]));
+            }
+          } else if (MODE == BW_DACT) {
+            // f = dH; the stored U (and V) of the same row and columns
+            const uint4* pu = reinterpret_cast<const uint4*>(p.in0 + row * p.ld_in + col);
+            float u[32], vv[32];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint4 x = pu[j];
+              const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                u[8 * j + 2 * k] = __uint_as_float(w4[k] << 16);
+                u[8 * j + 2 * k + 1] = __uint_as_float(w4[k] & 0xFFFF0000u);
+              }
+            }
+            if (p.swiglu) {
+              const uint4* pv = reinterpret_cast<const uint4*>(p.in1 + row * p.ld_in + col);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const uint4 x = pv[j];
+                const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  vv[8 * j + 2 * k] = __uint_as_float(w4[k] << 16);
+                  vv[8 * j + 2 * k + 1] = __uint_as_float(w4[k] & 0xFFFF0000u);
+                }
+              }
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const float sg = __frcp_rn(1.0f + __expf(-u[i]));
+                g[i] = f[i] * u[i] * sg;                                   // dV = dH silu(U)
+                f[i] = f[i] * vv[i] * sg * (1.0f + u[i] * (1.0f - sg));    // dU = dH V silu'(U)
+              }
+            } else if (p.act == MOE_ACT_RELU) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) f[i] = u[i] > 0.0f ? f[i] : 0.0f;
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const float cdf = 0.5f * (1.0f + erff(u[i] * 0.70710678118654752f));
+                const float pdf = 0.3989422804014327f * __expf(-0.5f * u[i] * u[i]);
+                f[i] = f[i] * (cdf + u[i] * pdf);
+              }
+            }
+            uint4* du = reinterpret_cast<uint4*>(p.out0 + row * p.ld_out + col);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              du[j] = make_uint4(pack_bf16x2(f[8 * j], f[8 * j + 1]), pack_bf16x2(f[8 * j + 2], f[8 * j + 3]),
+                                 pack_bf16x2(f[8 * j + 4], f[8 * j + 5]), pack_bf16x2(f[8 * j + 6], f[8 * j + 7]));
+            if (p.swiglu) {
+              uint4* dv = reinterpret_cast<uint4*>(p.out0 + row * p.ld_out + p.n_total + col);
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                dv[j] = make_uint4(pack_bf16x2(g[8 * j], g[8 * j + 1]), pack_bf16x2(g[8 * j + 2], g[8 * j + 3]),
+                                   pack_bf16x2(g[8 * j + 4], g[8 * j + 5]), pack_bf16x2(g[8 * j + 6], g[8 * j + 7]));
+            }
+          } else {  // BW_DX
+            uint4* o = reinterpret_cast<uint4*>(p.out0 + row * p.ld_out + col);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              o[j] = make_uint4(pack_bf16x2(f[8 * j], f[8 * j + 1]), pack_bf16x2(f[8 * j + 2], f[8 * j + 3]),
+                                pack_bf16x2(f[8 * j + 4], f[8 * j + 5]), pack_bf16x2(f[8 * j + 6], f[8 * j + 7]));
+          }
+        }
+      }
+      sm100::tc_fence_before();
+      sm100::mbar_arrive(&st->tempty[acc]);
+    }
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    sm100::tc_fence_after();
+    sm100::tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+template <int MODE>
+static cudaError_t launch_bwd(const BwdMaps& m, const BwdParams& p, cudaStream_t s) {
+  const size_t bytes = (size_t)kWStages * kWStageBytes + sizeof(BwdState) + 1024;
+  auto kern = tc_bwd_gemm_kernel<MODE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  long long tiles;
+  if (ModeTraits<MODE>::WGRAD) {
+    tiles = (long long)(p.E + p.n_shared) * p.mt_tiles * p.nt_tiles;
+  } else {
+    tiles = (long long)(p.max_routed_blocks + p.E) * p.nt_tiles +
+            (long long)p.n_shared * p.shared_blocks * p.nt_tiles;
+  }
+  const int grid = (int)(tiles < sms ? (tiles < 1 ? 1 : tiles) : sms);
+  return launch_pdl(kern, grid, kWThreads, bytes, s, m.a0, m.a1, m.b0, m.b0g, m.b1, m.b1g, p);
+}
+
+cudaError_t run_bwd_gemm(int mode, const BwdMaps& m, const BwdParams& p, cudaStream_t s) {
+  switch (mode) {
+    case BW_SAVE: return launch_bwd<BW_SAVE>(m, p, s);
+    case BW_DACT: return launch_bwd<BW_DACT>(m, p, s);
+    case BW_DX: return launch_bwd<BW_DX>(m, p, s);
+    case BW_WG2: return launch_bwd<BW_WG2>(m, p, s);
+    default: return launch_bwd<BW_WG13>(m, p, s);
+  }
+}
+
+}  // namespace moe

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -200,6 +201,78 @@ moe_status run_ffn_bf16(const FfnArgs& a, cudaStream_t s);
 bool swap_down_supported(const FfnArgs& a);
 moe_status run_ffn_down_swap(const FfnArgs& a, cudaStream_t s);
 moe_status run_ffn_f32(const FfnArgs& a, cudaStream_t s);
+
+// ----- backward pass -----
+// grouped GEMMs of the expert FFN's backward (gemm_bwd.cu)
+enum { BW_SAVE = 0, BW_DACT = 1, BW_DX = 2, BW_WG2 = 3, BW_WG13 = 4 };
+struct BwdParams {
+  const int32_t* offsets;
+  const int32_t* counts;   // [E] rows kept per expert (weight gradients reduce over these)
+  int E, n_shared, n;
+  int swiglu, act;
+  // row modes (SAVE, DACT, DX): 128-row blocks of the dispatched rows
+  int K;                   // reduction length, multiple of 64
+  int k_split;             // DX: K rows below come from the W1 map, above from W3
+  int n_total;             // output columns
+  int n_block;             // output columns per tile (SAVE with SwiGLU: 128)
+  int nt_tiles;            // column blocks (weight gradients: 256-column blocks)
+  int b_rows_per_expert;   // weight rows per expert in the B map
+  int shared_blocks;       // 128-row blocks per shared expert
+  int max_routed_blocks;   // bound on offsets[E] / 128
+  long long a1_row_base, a1_row_stride;  // shared experts' A rows
+  long long out_shared_base, n_pad;
+  __nv_bfloat16 *out0, *out1, *out2;
+  long long ld_out;
+  const __nv_bfloat16 *in0, *in1;
+  long long ld_in;
+  // weight-gradient modes (WG2, WG13): the expert's [m_total, ld_w] output
+  int m_total, m_split, mt_tiles, ld_w;
+  long long b1_row_base, b1_row_stride;  // shared experts' B rows
+  long long w_expert_stride;             // elements between experts' outputs
+  __nv_bfloat16 *w_out0, *w_out1, *sw_out0, *sw_out1;  // rows < m_split / >= m_split
+  int* err;
+};
+struct BwdMaps {
+  CUtensorMap a0, a1, b0, b0g, b1, b1g;
+};
+cudaError_t run_bwd_gemm(int mode, const BwdMaps& m, const BwdParams& p, cudaStream_t s);
+
+// element-wise and FFMA kernels of the backward (bwd.cu)
+struct CombineBwdArgs {
+  const __nv_bfloat16* Y_perm;   // [rows, d] the forward's expert outputs
+  const __nv_bfloat16* dout;     // [n, d]
+  const int32_t* tok_row;        // [n, slots]
+  const float* tok_gate;         // [n, slots]
+  const int32_t* idx;            // TC [n, K]
+  const uint8_t* drop;           // TC [n, K]
+  const int32_t* offsets;        // [E+1]
+  const int32_t* load;           // [E]
+  const float* scores;           // [n, E]
+  const float* logits;           // [n, E] (z-loss, sqrt(softplus)) or NULL
+  const float* lse;              // [n] or NULL
+  int n, d, E, slots, tc, K, score, weights;
+  float lb_coef, z_coef;
+  __nv_bfloat16* dY_perm;        // [rows, d]: kept rows written
+  float* dL;                     // [n, E]
+};
+cudaError_t launch_combine_backward(const CombineBwdArgs& a, cudaStream_t s);
+cudaError_t launch_pad_zero(const int32_t* offsets, const int32_t* counts, int E, int d,
+                            __nv_bfloat16* a, __nv_bfloat16* b, cudaStream_t s);
+struct RouterBwdArgs {
+  const __nv_bfloat16* X;        // [n, d]
+  const float* Wg;               // [d, E]
+  const float* dL;               // [n, E]
+  const __nv_bfloat16* dX_perm;  // [rows, d]
+  const int32_t* tok_row;        // [n, slots]
+  int n, d, E, slots, n_shared;
+  long long shared_base, n_pad;
+  __nv_bfloat16* dX;             // [n, d]
+  float* dWg;                    // [d, E]
+  float* partial;                // [splits, d, E]
+  int splits;
+};
+int router_bwd_splits(int n, int d, int E);
+cudaError_t launch_router_backward(const RouterBwdArgs& a, cudaStream_t s);
 
 cudaError_t launch_bias_update(int n, int E, int K, const int32_t* load, float rate,
                                float* bias, cudaStream_t s);

@@ -36,7 +36,7 @@ API_SYMBOLS = ["moe_status_string", "moe_validate", "moe_sizes", "moe_workspace_
                "moe_route", "moe_route_from_scores", "moe_dispatch", "moe_expert_ffn",
                "moe_combine", "moe_layer_forward", "moe_bias_update", "moe_workspace_init",
                "moe_read_error", "moe_route_noalloc", "moe_expert_ffn_gathered",
-               "moe_launch_counts"]
+               "moe_launch_counts", "moe_backward_workspace_size", "moe_layer_backward"]
 MOE_ROUTE_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -97,6 +97,9 @@ def lib() -> ctypes.CDLL:
         L.moe_route_noalloc.argtypes = [cfgp, P, P, P, P, outp, P]
         L.moe_expert_ffn_gathered.argtypes = [cfgp, P, outp, P, P, P, P, P, P, P, P, P,
                                               ctypes.c_size_t, P]
+        L.moe_backward_workspace_size.argtypes = [cfgp, ctypes.POINTER(ctypes.c_size_t), ip]
+        L.moe_layer_backward.argtypes = [cfgp, P, P, P, P, P, P, P, P, outp, P, ctypes.c_size_t,
+                                         P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         for s in API_SYMBOLS[1:]:
             getattr(L, s).restype = ctypes.c_int
         _LIB = L
@@ -299,6 +302,31 @@ def moe_route_noalloc(cfg, X, Wg, logit_bias, sel_bias, route: RouteBuffers, str
            "moe_route_noalloc")
 
 
+def backward_workspace(cfg: MoeConfig, device, stream=None):
+    """(workspace tensor for moe_layer_backward, kernels it enqueues)."""
+    nbytes = ctypes.c_size_t()
+    launches = ctypes.c_int()
+    _check(lib().moe_backward_workspace_size(ctypes.byref(cfg), ctypes.byref(nbytes),
+                                             ctypes.byref(launches)),
+           "moe_backward_workspace_size")
+    ws = torch.empty(nbytes.value + 256, dtype=torch.uint8, device=device)
+    off = (-ws.data_ptr()) % 256
+    ws = ws[off:off + nbytes.value]
+    _check(lib().moe_workspace_init(_ptr(ws), _stream(stream)), "moe_workspace_init")
+    return ws, launches.value
+
+
+def moe_layer_backward(cfg, X, Wg, W1, W3, W2, sW1, sW3, sW2, route: RouteBuffers, fwd_ws,
+                       dout, dX, dWg, dW1, dW3, dW2, dsW1, dsW3, dsW2, dL, ws, stream=None):
+    _check(lib().moe_layer_backward(ctypes.byref(cfg), _ptr(X), _ptr(Wg), _ptr(W1), _ptr(W3),
+                                    _ptr(W2), _ptr(sW1), _ptr(sW3), _ptr(sW2),
+                                    ctypes.byref(route.c), _ptr(fwd_ws), fwd_ws.numel(),
+                                    _ptr(dout), _ptr(dX), _ptr(dWg), _ptr(dW1), _ptr(dW3),
+                                    _ptr(dW2), _ptr(dsW1), _ptr(dsW3), _ptr(dsW2), _ptr(dL),
+                                    _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_layer_backward")
+
+
 def moe_read_error(ws, stream=None):
     detail = ctypes.c_int()
     st = lib().moe_read_error(_ptr(ws), _stream(stream), ctypes.byref(detail))
@@ -328,3 +356,29 @@ class Layer:
                           i.get("sel_bias"), i["W1"], i.get("W3"), i["W2"], i.get("sW1"),
                           i.get("sW3"), i.get("sW2"), self.out, self.route, self.ws, stream)
         return self.out
+
+    def grads(self):
+        """Gradient buffers of the layer's inputs and weights (allocated once)."""
+        if not hasattr(self, "_grads"):
+            i, dev = self.inp, self.device
+            g = {"dX": torch.empty_like(i["X"]),
+                 "dWg": torch.empty_like(i["Wg"]),
+                 "dW1": torch.empty_like(i["W1"]), "dW2": torch.empty_like(i["W2"]),
+                 "dW3": torch.empty_like(i["W3"]) if i.get("W3") is not None else None,
+                 "dsW1": torch.empty_like(i["sW1"]) if i.get("sW1") is not None else None,
+                 "dsW2": torch.empty_like(i["sW2"]) if i.get("sW2") is not None else None,
+                 "dsW3": torch.empty_like(i["sW3"]) if i.get("sW3") is not None else None,
+                 "dL": torch.empty((self.w.n, self.w.E), dtype=torch.float32, device=dev)}
+            self._bws, self.bwd_launches = backward_workspace(self.cfg, dev)
+            self._grads = g
+        return self._grads
+
+    def backward(self, dout, X=None, stream=None):
+        """Gradients of <dout, out> + the aux losses after forward() on the same
+        inputs (the forward's workspace and routing are read)."""
+        i, g = self.inp, self.grads()
+        moe_layer_backward(self.cfg, i["X"] if X is None else X, i["Wg"], i["W1"], i.get("W3"),
+                           i["W2"], i.get("sW1"), i.get("sW3"), i.get("sW2"), self.route,
+                           self.ws, dout, g["dX"], g["dWg"], g["dW1"], g["dW3"], g["dW2"],
+                           g["dsW1"], g["dsW3"], g["dsW2"], g["dL"], self._bws, stream)
+        return g

@@ -317,6 +317,60 @@ MOE_API moe_status moe_route_noalloc(const moe_config* cfg, const void* X, const
                                      const float* logit_bias, const float* sel_bias,
                                      moe_route_out* out, moe_stream_t stream);
 
+/* ---- backward pass of moe_layer_forward -------------------------------
+ * The gradient, by the chain rule, of
+ *     loss = <dout, out> + L_lb + L_z
+ * where out is moe_layer_forward's output and L_lb, L_z are the aux losses
+ * of [TC-vs-EC] "What each direction guarantees" (token choice; coefficients
+ * lb_coef, z_coef as in aux[]). Selections, capacity drops and counts are
+ * piecewise constant and carry no gradient; the selection bias and the logit
+ * bias get none. Steps, in order ([EC-math] "The math": out =
+ * scatter_add(G * Expert(X_in))):
+ *   combine:  dY[r] = g dout[t] for each kept row r of token t with gate g
+ *             (stored bf16); dgate = <dout[t], Y_perm[r]> (fp32);
+ *   weights:  raw: dS = dgate; normalised w = s / sum s over the K selected:
+ *             dS_k = (dw_k - sum_j w_j dw_j) / sum_j s_j; expert choice:
+ *             dS[t, e] = dgate; plus lb_coef E f_e / n (f_e = load_e / (n K));
+ *   scores:   softmax dL = S (dS - <S, dS>); sigmoid dL = dS s (1 - s);
+ *             sqrt(softplus) dL = dS sigmoid(l) / (2 s); plus the z-loss
+ *             term z_coef 2 lse_t / n softmax(l_t);
+ *   experts:  U = X W1^T, V = X W3^T recomputed and stored bf16, H as the
+ *             forward computes it; dH = dY W2; dU = dH act'(U) (SwiGLU:
+ *             dU = dH V silu'(U), dV = dH silu(U)), stored bf16;
+ *             dX_perm = dU W1 + dV W3 (bf16); dW1 = dU^T X_perm,
+ *             dW3 = dV^T X_perm, dW2 = dY^T H over each expert's kept rows
+ *             (fp32 accumulation, stored bf16); shared experts take dout
+ *             itself as dY over all n tokens;
+ *   router:   dWg = X^T dL (fp32); dX = dL Wg^T + the sum of dX_perm over
+ *             the token's kept rows and shared rows (fp32, stored bf16).
+ * bf16 configs only (MOE_ERR_UNSUPPORTED otherwise). */
+
+/* Backward workspace bytes and the kernels moe_layer_backward enqueues. */
+MOE_API moe_status moe_backward_workspace_size(const moe_config* cfg, size_t* bytes,
+                                               int* launches);
+
+/* Arguments: the forward's inputs X, Wg, W1, W3, W2 (sW* for shared
+ * experts, else NULL); `route`, the routing moe_layer_forward wrote (with
+ * logits, and lse, filled when the score is sqrt(softplus) or token choice
+ * has z_coef != 0); fwd_ws, the workspace of that moe_layer_forward call,
+ * untouched since: its dispatched rows and expert outputs are read, and the
+ * padding rows of its dispatched rows are overwritten with zeros; dout [n,d]
+ * bf16. Outputs (device, caller-owned, every element written): dX [n,d]
+ * bf16, dWg [d,E] fp32, dW1, dW3 [E,h,d] and dW2 [E,d,h] bf16 (dW3 only for
+ * SwiGLU), dsW1, dsW3, dsW2 likewise for shared experts; dL [n,E] fp32, the
+ * logits' gradient, may be NULL. ws: moe_backward_workspace_size bytes,
+ * 256-byte aligned, error word zeroed once by moe_workspace_init; bounded
+ * waits report through it (moe_read_error). X, dout, dX, the weights and
+ * their gradients must be 16-byte aligned. */
+MOE_API moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float* Wg,
+                                      const void* W1, const void* W3, const void* W2,
+                                      const void* sW1, const void* sW3, const void* sW2,
+                                      const moe_route_out* route, void* fwd_ws,
+                                      size_t fwd_ws_bytes, const void* dout, void* dX,
+                                      float* dWg, void* dW1, void* dW3, void* dW2,
+                                      void* dsW1, void* dsW3, void* dsW2, float* dL,
+                                      void* ws, size_t ws_bytes, moe_stream_t stream);
+
 /* Zeroes the error word at the start of `ws` (enqueued on `stream`). */
 MOE_API moe_status moe_workspace_init(void* ws, moe_stream_t stream);
 

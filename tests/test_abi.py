@@ -33,7 +33,7 @@ def declared_symbols():
 
 def test_every_declared_symbol_is_exported():
     syms = declared_symbols()
-    assert len(syms) == 16
+    assert len(syms) == 18
     assert sorted(moe.API_SYMBOLS) == syms
     L = ctypes.CDLL(moe.LIB_PATH)
     for s in syms:
@@ -190,3 +190,43 @@ def test_launch_counts():
     decode = moe.launch_counts(moe.config(wl.DECODE))
     assert decode["route"] == 5
     assert moe.launch_counts(moe.config(wl.TC_SIGMOID_GROUPED))["ffn"] == 2
+
+
+def _bwd_size(cfg):
+    nbytes = ctypes.c_size_t()
+    launches = ctypes.c_int()
+    st = moe.lib().moe_backward_workspace_size(ctypes.byref(cfg), ctypes.byref(nbytes),
+                                               ctypes.byref(launches))
+    return st, nbytes.value, launches.value
+
+
+def test_backward_workspace_and_launches():
+    """The backward enqueues the padding clear, the combine backward, five
+    grouped GEMMs, the router's input gradient and its weight gradient (plus
+    the ordered reduce of the weight gradient's token slices when there is
+    more than one). fp32 layers have no backward."""
+    for w in (wl.EC_BF16, wl.TC_TOP2_CAP, wl.TC_DROPLESS, wl.TC_SIGMOID_GROUPED, wl.DECODE):
+        st, nbytes, launches = _bwd_size(moe.config(w))
+        assert st == moe.MOE_OK, w.name
+        sw = w.act == "swiglu"
+        sz = moe.sizes(moe.config(w))
+        # at least dY, U, (V), H, dU(,dV) and dX_perm over the dispatched rows
+        assert nbytes >= sz.rows * (w.d * 2 + w.h * (8 if sw else 4)), w.name
+        assert launches in (9, 10), w.name
+    st, _, _ = _bwd_size(moe.config(wl.EC_FP32))
+    assert st == moe.MOE_ERR_UNSUPPORTED
+
+
+def test_backward_rejects_bad_arguments_before_launching():
+    """Host-side validation: null required pointers and an fp32 config fail
+    without touching the (null) device pointers."""
+    cfg = moe.config(wl.TC_DROPLESS.replace(n=256, d=128, E=8, h=128))
+    L = moe.lib()
+    route = moe.MoeRouteOut()
+    st = L.moe_layer_backward(ctypes.byref(cfg), *([None] * 8), ctypes.byref(route), None, 0,
+                              *([None] * 10), None, 0, None)
+    assert st == moe.MOE_ERR_INVALID_ARG
+    cfg32 = moe.config(wl.EC_FP32)
+    st = L.moe_layer_backward(ctypes.byref(cfg32), *([None] * 8), ctypes.byref(route), None, 0,
+                              *([None] * 10), None, 0, None)
+    assert st == moe.MOE_ERR_UNSUPPORTED

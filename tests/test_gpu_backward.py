@@ -1,0 +1,145 @@
+"""GPU parity of the layer's backward pass (moe_layer_backward through the C
+ABI) against the oracle's chain-rule backward on the same seeded inputs.
+
+Every gradient the library writes is compared: the logits' gradient dL and
+the router weight gradient dWg (fp32) to a relative Frobenius error of 5e-3,
+the input gradient dX and every expert's and shared expert's weight
+gradients (bf16) to 2e-2, the same bar as the layer's bf16 outputs. Experts
+that received no rows must get exactly zero weight gradients.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from expert_dispatch_gemm_b200 import moe
+from expert_dispatch_gemm_b200 import workloads as wl
+from tests.gpu_common import expert_weights_from, explained_routing_diff, host
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+F32_GRAD_TOL = 5e-3
+BF16_GRAD_TOL = 2e-2
+
+BWD_SMALL = wl.SMALL[1:] + [
+    # ReLU experts, strong aux-loss coefficients (their gradient terms matter)
+    wl.TC_DROPLESS.replace(name="bwd-top4of16-relu-aux0.5-n1000-d192-h192", n=1000, d=192, E=16,
+                           K=4, h=192, act="relu", lb_coef=0.5, z_coef=0.5),
+    # sqrt(softplus) scores, shared expert, group-limited
+    wl.TC_SIGMOID_GROUPED.replace(name="bwd-sqrtsoftplus-grouped-shared-n300-d128-e64-h128",
+                                  n=300, d=128, E=64, h=128, score="sqrtsoftplus", bias_steps=0,
+                                  z_coef=0.2),
+    # 64 tokens over 64 experts, top-1: most experts get no rows (zero
+    # gradients) and the rest one or two
+    wl.TC_DROPLESS.replace(name="bwd-top1of64-sparse-n64-d128-h128", n=64, d=128, E=64, K=1,
+                           h=128),
+    # expert choice, GELU, the capacity of several 128-row blocks per expert
+    wl.EC_BF16.replace(name="bwd-ec-gelu-n768-d128-e8-c4-h256", n=768, d=128, E=8, h=256, c=4.0),
+]
+
+
+@pytest.fixture(autouse=True)
+def _cleanup():
+    yield
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def _dout(w, seed=17):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randn((w.n, w.d), generator=g).to(w.torch_dtype).to(DEV)
+
+
+def _rel(got, ref):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    den = np.linalg.norm(ref)
+    return np.linalg.norm(got - ref) / den if den > 0 else np.linalg.norm(got)
+
+
+def _ws_ok(ws):
+    st, detail = moe.moe_read_error(ws)
+    assert st == moe.MOE_OK, f"device error word {detail:#x}"
+
+
+def _oracle_route(w, inp):
+    spec = oracle.spec_of(w)
+    logits, S, lse = oracle.router(host(inp["X"]), host(inp["Wg"]), host(inp.get("logit_bias")),
+                                   spec["score"])
+    r = oracle.route(spec, S, lse, host(inp.get("sel_bias")))
+    return spec, S, r
+
+
+@pytest.mark.parametrize("w", BWD_SMALL, ids=lambda w: w.name)
+def test_backward_small(w):
+    inp = wl.make_inputs(w, DEV)
+    layer = moe.Layer(w, inp, DEV)
+    layer.forward()
+    dout = _dout(w)
+    g = layer.backward(dout)
+    torch.cuda.synchronize()
+    _ws_ok(layer.ws)
+    _ws_ok(layer._bws)
+    spec, S, r = _oracle_route(w, inp)
+    bad = explained_routing_diff(spec, r, layer.route, S, host(inp.get("sel_bias")))
+    assert not bad, f"routing differs from the oracle's on {len(bad)} tokens"
+    ref = oracle.layer_backward(spec, host(inp["X"]), host(inp["Wg"]), host(dout),
+                                expert_weights_from(inp),
+                                expert_weights_from(inp, "s") if w.n_shared else None,
+                                host(inp.get("logit_bias")), host(inp.get("sel_bias")))
+    assert _rel(host(g["dL"]), ref["dL"]) < F32_GRAD_TOL
+    assert _rel(host(g["dWg"]), ref["dWg"]) < F32_GRAD_TOL
+    assert _rel(host(g["dX"]), ref["dX"]) < BF16_GRAD_TOL
+    names = ["dW1", "dW2"] + (["dW3"] if w.act == "swiglu" else [])
+    for e in range(w.E):
+        for nm in names:
+            got = host(g[nm][e])
+            if e in ref[nm]:
+                assert _rel(got, ref[nm][e]) < BF16_GRAD_TOL, (nm, e)
+            else:
+                assert not got.any(), (nm, e, "expert without rows")
+    for s in range(w.n_shared):
+        for nm in names:
+            assert _rel(host(g["ds" + nm[1:]][s]), ref["ds" + nm[1:]][s]) < BF16_GRAD_TOL, (nm, s)
+
+
+def test_backward_repeatable_and_forward_unchanged():
+    """Two backward calls give bit-identical gradients (no atomics anywhere),
+    and the forward output is the same before and after (the backward only
+    clears padding rows of the forward's workspace)."""
+    w = wl.SMALL[3]
+    inp = wl.make_inputs(w, DEV)
+    layer = moe.Layer(w, inp, DEV)
+    out0 = layer.forward().clone()
+    dout = _dout(w, seed=3)
+    g1 = {k: v.clone() for k, v in layer.backward(dout).items() if v is not None}
+    g2 = layer.backward(dout)
+    torch.cuda.synchronize()
+    for k, v in g1.items():
+        assert torch.equal(v, g2[k]), k
+    out1 = layer.forward()
+    torch.cuda.synchronize()
+    assert torch.equal(out0, out1)
+    _ws_ok(layer._bws)
+
+
+def test_backward_zero_dout_gives_only_aux_gradients():
+    """dout = 0: every expert gradient and the experts' share of dX vanish;
+    what remains is the aux losses' gradient (token choice), so dL has the
+    closed form of the balance- and z-loss terms alone, which the oracle's
+    backward also gives."""
+    w = wl.SMALL[3].replace(lb_coef=0.3, z_coef=0.2)
+    inp = wl.make_inputs(w, DEV)
+    layer = moe.Layer(w, inp, DEV)
+    layer.forward()
+    dout = torch.zeros((w.n, w.d), dtype=w.torch_dtype, device=DEV)
+    g = layer.backward(dout)
+    torch.cuda.synchronize()
+    for nm in ("dW1", "dW2", "dW3"):
+        assert not g[nm].any(), nm
+    spec, S, r = _oracle_route(w, inp)
+    ref = oracle.layer_backward(spec, host(inp["X"]), host(inp["Wg"]), host(dout),
+                                expert_weights_from(inp), None, None, None)
+    assert _rel(host(g["dL"]), ref["dL"]) < F32_GRAD_TOL
+    assert _rel(host(g["dX"]), ref["dX"]) < BF16_GRAD_TOL
