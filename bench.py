@@ -1,7 +1,7 @@
 """Benchmark of the MoE routing-and-dispatch layer forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--impl reference]
+                    [--impl reference] [--pass forward|train]
 
 One step = one pass of the whole hot path over one batch, the calls
 moe_layer_forward makes: moe_route (router GEMM + scores + top-k + capacity
@@ -20,6 +20,10 @@ the timed region is the max over ranks.
 
 --impl reference times the CPU oracle as it stands (single thread) on the
 same workload, one bounded sample per step.
+
+--pass train times forward + backward (moe_layer_forward then
+moe_layer_backward: gradients of X, W_g and every expert weight) per step,
+with the backward's grouped-GEMM FLOPs against the tensor-core peak.
 """
 from __future__ import annotations
 
@@ -461,6 +465,195 @@ def run_gpu(args, w: wl.Workload):
 
 
 # ---------------------------------------------------------------------------
+# training step: forward + backward (--pass train)
+# ---------------------------------------------------------------------------
+
+METRIC_TRAIN = ("MoE-layer fwd+bwd tokens/s on 1 B200 (gradients of X, W_g and every expert "
+                "weight); backward grouped-GEMM TC util %")
+
+
+def backward_flops(w: wl.Workload, rows_gathered: int) -> dict:
+    """FLOPs of the backward's five grouped GEMMs and of the router's two
+    FFMA contractions, over the kept rows (and the shared experts' n rows)."""
+    g = 2 if w.act == "swiglu" else 1  # up projections per expert
+    rows = rows_gathered + w.n_shared * w.n
+    unit = 2.0 * rows * w.d * w.h
+    return {"recompute": unit * g, "dact": unit, "dx": unit * g, "dw2": unit, "dw13": unit * g,
+            "router": 4.0 * w.n * w.d * w.E}
+
+
+def run_gpu_train(args, w: wl.Workload):
+    import torch.distributed as dist
+
+    from expert_dispatch_gemm_b200 import moe
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    inp = wl.make_inputs(w, dev)
+    layer = moe.Layer(w, inp, dev)
+    gen = torch.Generator(device=dev).manual_seed(w.seed + 99)
+    dout = torch.randn((w.n, w.d), generator=gen, device=dev).to(w.torch_dtype)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    layer.grads()
+
+    def step(X=None, d=None, ev=None):
+        layer.forward(X=X, stream=stream)
+        if ev is not None:
+            ev.record(stream)
+        layer.backward(dout if d is None else d, X=X, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    for ws in (layer.ws, layer._bws):
+        st, detail = moe.moe_read_error(ws)
+        if st != moe.MOE_OK:
+            raise RuntimeError(f"device error after warm-up: {detail:#x}")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            evs[i][0].record(stream)
+            step(ev=evs[i][1])
+            evs[i][2].record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    step_ms = np.array([evs[i][0].elapsed_time(evs[i][2]) for i in range(args.steps)])
+    fwd_ms = np.array([evs[i][0].elapsed_time(evs[i][1]) for i in range(args.steps)])
+    bwd_ms = np.array([evs[i][1].elapsed_time(evs[i][2]) for i in range(args.steps)])
+    total_ms = max_over_ranks(float(step_ms.sum()), dev)
+    for ws in (layer.ws, layer._bws):
+        st, detail = moe.moe_read_error(ws)
+        if st != moe.MOE_OK:
+            raise RuntimeError(f"device error in the timed region: {detail:#x}")
+
+    # end to end: X and dout up from pinned host memory, dX back, every step
+    Xh = inp["X"].cpu().pin_memory()
+    dh = dout.cpu().pin_memory()
+    dXh = torch.empty(inp["X"].shape, dtype=inp["X"].dtype).pin_memory()
+    Xd, dd = torch.empty_like(inp["X"]), torch.empty_like(dout)
+
+    def e2e_step():
+        Xd.copy_(Xh, non_blocking=True)
+        dd.copy_(dh, non_blocking=True)
+        step(X=Xd, d=dd)
+        dXh.copy_(layer.grads()["dX"], non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+
+    rows_gathered = int(layer.route.counts.sum().item())
+    bf = backward_flops(w, rows_gathered)
+    gemm_flops = sum(v for k, v in bf.items() if k != "router")
+    hbm, tc_burst, tc_sust, src = peaks()
+    clocks = clk.summary()
+    capped = "sw_power_cap" in clocks.get("reasons", [])
+    tc_peak = tc_sust if (capped and tc_sust) else tc_burst
+    bwd_med = float(np.median(bwd_ms))
+    ach = gemm_flops / (bwd_med * 1e-3) / 1e12
+    roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": tc_peak, "unit": "TFLOP/s",
+            "frac": round(ach / tc_peak, 3),
+            "peak_kind": "sustained (sw_power_cap active)" if (capped and tc_sust) else "burst",
+            "traffic": None, "peak_source": src,
+            "kernel": "moe_layer_backward as a whole: the five grouped GEMMs' FLOPs over the "
+                      "whole call (its non-GEMM kernels included in the time)",
+            "algorithmic_per_launch": gemm_flops}
+    fwd_launches = sum(moe.launch_counts(layer.cfg).values())
+    res = {
+        "metric": METRIC_TRAIN,
+        "value": round(whole_job_rate(w.n, world, args.steps, total_ms), 1), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) activations and output gradient, random-init weights)",
+        "config": {"workload": w.name, "pass": "forward + backward", "tokens": w.n,
+                   "d_model": w.d, "experts": w.E, "hidden": w.h,
+                   "parallelism": f"replicas{world}" if world > 1 else "single-gpu",
+                   "l2": "flushed between timed steps (256 MB write, outside the events)"},
+        "roofline": roof,
+        "stages": {"forward": {"ms": round(float(np.median(fwd_ms)), 4)},
+                   "backward": {"ms": round(bwd_med, 4),
+                                "gemm_TFLOP": round(gemm_flops / 1e12, 3),
+                                "router_FFMA_GFLOP": round(bf["router"] / 1e9, 2)}},
+        "e2e": {"value": round(whole_job_rate(w.n, world, args.steps, e2e_ms), 1),
+                "unit": "tokens/s",
+                "h2d_bytes_per_step": int(Xh.numel() * Xh.element_size() +
+                                          dh.numel() * dh.element_size()),
+                "d2h_bytes_per_step": int(dXh.numel() * dXh.element_size()),
+                "note": "pinned host X and dout -> device -> forward + backward -> host dX "
+                        "every step, on the compute stream; no L2 flush"},
+        "gpu_launches": (fwd_launches + layer.bwd_launches) * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline_train(w, inp, dout, budget_s=args.cpu_budget)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+def cpu_baseline_train(w, inp, dout, budget_s=20.0):
+    """The oracle's forward routing plus its backward on sampled tokens (each
+    token's dX needs only its own pairs; their expert rows also carry the
+    weight-gradient work), extrapolated to the batch."""
+    import oracle
+    X, Wg, lb, sb, weights = _host_inputs(w, inp)
+    spec = oracle.spec_of(w)
+    dh = dout.float().cpu().numpy()
+    sw = None
+    if w.n_shared:
+        def sw(s):
+            return (inp["sW1"][s].float().cpu().numpy(),
+                    None if inp.get("sW3") is None else inp["sW3"][s].float().cpu().numpy(),
+                    inp["sW2"][s].float().cpu().numpy())
+    rng = np.random.default_rng(0)
+    t0 = time.perf_counter()
+    logits, S, lse = oracle.router(X, Wg, lb, spec["score"])
+    r = oracle.route(spec, S, lse, sb)
+    t_route = time.perf_counter() - t0
+
+    def run(toks):
+        t1 = time.perf_counter()
+        oracle.layer_backward(spec, X, Wg, dh, weights, sw, lb, sb, tokens=toks,
+                              pre=(logits, S, lse, r))
+        return time.perf_counter() - t1
+
+    probe = sorted(rng.choice(w.n, size=min(2, w.n), replace=False).tolist())
+    t_probe = run(probe)
+    sample = int(max(2, min(w.n, (budget_s - t_route) / max(t_probe / len(probe), 1e-6) * 0.5)))
+    toks = sorted(rng.choice(w.n, size=min(sample, w.n), replace=False).tolist())
+    t = run(toks)
+    est = t_route + t / len(toks) * w.n
+    return {"value": round(w.n / est, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": (f"oracle routing of all {w.n} tokens ({t_route:.2f} s) plus the "
+                       f"chain-rule backward of {len(toks)} seeded tokens (their expert rows, "
+                       f"weight-gradient work included; {t:.2f} s), extrapolated to {w.n} "
+                       "tokens; single-threaded C oracle, fp64")}
+
+
+# ---------------------------------------------------------------------------
 # CPU oracle (baseline leg and reference arm)
 # ---------------------------------------------------------------------------
 
@@ -552,12 +745,18 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--ref-sample", type=int, default=48)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "train"],
+                    help="forward: the layer's forward (default); train: forward + backward")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = wl.BY_NAME[args.workload]
     if args.impl == "reference":
         run_reference(args, w)
+    elif args.pass_ == "train":
+        if w.dtype != "bf16":
+            ap.error("--pass train needs a bf16 workload")
+        run_gpu_train(args, w)
     else:
         run_gpu(args, w)
 

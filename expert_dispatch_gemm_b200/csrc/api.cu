@@ -585,7 +585,7 @@ moe_status moe_bias_update(const moe_config* cfg, const int32_t* load, float rat
 // backward pass
 // ---------------------------------------------------------------------------
 struct BwdLayout {
-  size_t err, dy, u, v, hh, duv, dxp, dl, part, end;
+  size_t err, dy, u, v, hh, duv, dxp, dl, wgt, part, end;
   int splits, launches;
 };
 
@@ -610,13 +610,15 @@ static BwdLayout bwd_layout(const moe_config* c, const Derived& d) {
   off = align_up(off + (size_t)d.rows * c->d * 2, 1024);
   b.dl = off;
   off = align_up(off + (size_t)c->n * c->E * 4, 1024);
+  b.wgt = off;
+  off = align_up(off + (size_t)c->d * c->E * 4, 1024);
   b.splits = router_bwd_splits(c->n, c->d, c->E);
   b.part = off;
   if (b.splits > 1) off = align_up(off + (size_t)b.splits * c->d * c->E * 4, 1024);
   b.end = off;
-  // pad clear, combine backward, five grouped GEMMs, router dX, router dWg
-  // (+ its ordered reduce)
-  b.launches = 9 + (b.splits > 1 ? 1 : 0);
+  // pad clear, combine backward, five grouped GEMMs, W_g transpose, router
+  // dX, router dWg (+ its ordered reduce)
+  b.launches = 10 + (b.splits > 1 ? 1 : 0);
   return b;
 }
 
@@ -722,6 +724,12 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float*
   auto map = [](CUtensorMap* m, const void* p, long long r, long long c, int box) {
     return make_bf16_sw128_map(m, p, r, c, box);
   };
+  // row GEMMs on CTA pairs when experts average two 128-row blocks, as the
+  // forward does. The weight gradients stay on single CTAs: their few
+  // k-blocks per tile leave the epilogue in charge, and pairs measured ~10%
+  // slower there (c5: 6.07 / 3.13 ms against 5.56 / 2.77 ms)
+  const bool rpair = ffn_uses_pair(cfg, d);
+  const bool wpair = false;
   // 3. SAVE: U (and V), H of every dispatched row again
   {
     BwdMaps m{};
@@ -729,7 +737,7 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float*
     if (!map(&m.a0, xp, rows, D, rbox)) return MOE_ERR_UNSUPPORTED;
     m.a1 = m.a0;
     if (ns > 0 && !map(&m.a1, X, n, D, rbox)) return MOE_ERR_UNSUPPORTED;
-    const int bbox = swiglu ? 128 : 256;
+    const int bbox = swiglu || rpair ? 128 : 256;
     if (!map(&m.b0, W1, (long long)E * h, D, bbox)) return MOE_ERR_UNSUPPORTED;
     m.b0g = m.b0;
     if (swiglu && !map(&m.b0g, W3, (long long)E * h, D, bbox)) return MOE_ERR_UNSUPPORTED;
@@ -748,7 +756,7 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float*
     p.out1 = V;
     p.out2 = H;
     p.ld_out = h;
-    MOE_CU(run_bwd_gemm(BW_SAVE, m, p, s));
+    MOE_CU(run_bwd_gemm(BW_SAVE, rpair, m, p, s));
   }
   // 4. DACT: dU (and dV) = (dY W2) * act'
   {
@@ -770,7 +778,7 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float*
     p.ld_in = h;
     p.out0 = duv;
     p.ld_out = swiglu ? 2LL * h : h;
-    MOE_CU(run_bwd_gemm(BW_DACT, m, p, s));
+    MOE_CU(run_bwd_gemm(BW_DACT, rpair, m, p, s));
   }
   // 5. DX: dX_perm = dU W1 (+ dV W3)
   {
@@ -798,7 +806,7 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float*
     p.b_rows_per_expert = h;
     p.out0 = dxp;
     p.ld_out = D;
-    MOE_CU(run_bwd_gemm(BW_DX, m, p, s));
+    MOE_CU(run_bwd_gemm(BW_DX, rpair, m, p, s));
   }
   // 6. WG2: dW2_e = dY_e^T H_e
   {
@@ -813,14 +821,14 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float*
     p.b1_row_stride = d.n_pad;
     p.m_total = D;
     p.m_split = D;
-    p.mt_tiles = ceil_div(D, 128);
+    p.mt_tiles = ceil_div(D, wpair ? 256 : 128);
     p.ld_w = h;
     p.nt_tiles = ceil_div(h, 256);
     p.w_expert_stride = (long long)D * h;
     p.w_out0 = bf(dW2);
     p.w_out1 = bf(dW2);
     p.sw_out0 = p.sw_out1 = ns > 0 ? bf(dsW2) : bf(dW2);
-    MOE_CU(run_bwd_gemm(BW_WG2, m, p, s));
+    MOE_CU(run_bwd_gemm(BW_WG2, wpair, m, p, s));
   }
   // 7. WG13: [dW1_e; dW3_e] = [dU_e | dV_e]^T X_e
   {
@@ -836,7 +844,7 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float*
     if (ns > 0 && !map(&m.b1, X, n, D, 64)) return MOE_ERR_UNSUPPORTED;
     p.m_total = (int)mcols;
     p.m_split = h;
-    p.mt_tiles = ceil_div(mcols, 128);
+    p.mt_tiles = ceil_div(mcols, wpair ? 256 : 128);
     p.ld_w = D;
     p.nt_tiles = ceil_div(D, 256);
     p.w_expert_stride = (long long)h * D;
@@ -844,12 +852,13 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float*
     p.w_out1 = swiglu ? bf(dW3) : bf(dW1);
     p.sw_out0 = ns > 0 ? bf(dsW1) : bf(dW1);
     p.sw_out1 = ns > 0 && swiglu ? bf(dsW3) : p.sw_out0;
-    MOE_CU(run_bwd_gemm(BW_WG13, m, p, s));
+    MOE_CU(run_bwd_gemm(BW_WG13, wpair, m, p, s));
   }
   // 8, 9. router: dX = dL Wg^T + the token's dispatched rows; dWg = X^T dL
   RouterBwdArgs rb{};
   rb.X = static_cast<const __nv_bfloat16*>(X);
   rb.Wg = Wg;
+  rb.WgT = at<float>(ws, b.wgt);
   rb.dL = dl;
   rb.dX_perm = dxp;
   rb.tok_row = route->tok_row;

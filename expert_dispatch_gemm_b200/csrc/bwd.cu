@@ -168,53 +168,76 @@ __global__ void __launch_bounds__(256) pad_zero_kernel(const int32_t* offsets,
   }
 }
 
+// WgT[e, i] = Wg[i, e], through 32 x 32 shared-memory tiles, so that the
+// input-gradient tiles below read rows of W_g^T with consecutive threads on
+// consecutive addresses
+__global__ void __launch_bounds__(256) transpose_wg_kernel(const float* Wg, int d, int E,
+                                                           float* WgT) {
+  pdl_wait();
+  __shared__ float tile[32][33];
+  const int i0 = blockIdx.x * 32, e0 = blockIdx.y * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int r = ty; r < 32; r += 8) {
+    const int i = i0 + r, e = e0 + tx;
+    tile[r][tx] = (i < d && e < E) ? Wg[(size_t)i * E + e] : 0.0f;
+  }
+  __syncthreads();
+  for (int r = ty; r < 32; r += 8) {
+    const int e = e0 + r, i = i0 + tx;
+    if (e < E && i < d) WgT[(size_t)e * d + i] = tile[tx][r];
+  }
+}
+
 // dX[t, i] = sum_e dL[t, e] Wg[i, e] + sum over the token's dispatched rows
 // of dX_perm[row, i] (+ the shared experts' rows), fp32, stored bf16.
-// Tile: 32 tokens x 128 columns, experts in chunks of 64; thread (ty, tx)
-// holds tokens ty + 8k (k < 4) and columns 4tx..4tx+3.
-constexpr int kRxBM = 32, kRxBN = 128, kRxEC = 64;
+// Tile: 64 tokens x 128 columns, experts in chunks of 32; thread (ty, tx)
+// holds tokens 8ty..8ty+7 and columns 4tx..4tx+3, so each expert step takes
+// three 16-byte shared-memory loads for 32 FMAs.
+constexpr int kRxBM = 64, kRxBN = 128, kRxEC = 32;
 __global__ void __launch_bounds__(256) router_dx_kernel(RouterBwdArgs a) {
   pdl_wait();
-  __shared__ float dls[kRxBM][kRxEC];
-  __shared__ __align__(16) float wts[kRxEC][kRxBN];
+  __shared__ __align__(16) float dls[kRxEC][kRxBM + 4];  // transposed: [expert][token]
+  __shared__ __align__(16) float wts[kRxEC][kRxBN];      // [expert][column]
   const int tid = threadIdx.x, tx = tid & 31, ty = tid >> 5;
   const int t0 = blockIdx.x * kRxBM, i0 = blockIdx.y * kRxBN;
-  float acc[4][4];
+  float acc[8][4];
 #pragma unroll
-  for (int k = 0; k < 4; ++k)
+  for (int k = 0; k < 8; ++k)
 #pragma unroll
     for (int c = 0; c < 4; ++c) acc[k][c] = 0.0f;
   for (int e0 = 0; e0 < a.E; e0 += kRxEC) {
     __syncthreads();
     for (int q = tid; q < kRxBM * kRxEC; q += 256) {
-      const int r = q / kRxEC, c = q % kRxEC;
+      const int r = q / kRxEC, c = q % kRxEC;  // consecutive threads: consecutive experts
       const int t = t0 + r, e = e0 + c;
-      dls[r][c] = (t < a.n && e < a.E) ? a.dL[(size_t)t * a.E + e] : 0.0f;
+      dls[c][r] = (t < a.n && e < a.E) ? a.dL[(size_t)t * a.E + e] : 0.0f;
     }
     for (int q = tid; q < kRxBN * kRxEC; q += 256) {
-      const int i = q % kRxBN, c = q / kRxBN;  // consecutive threads: consecutive i
+      const int i = q % kRxBN, c = q / kRxBN;  // consecutive threads: consecutive columns
       const int gi = i0 + i, e = e0 + c;
-      wts[c][i] = (gi < a.d && e < a.E) ? a.Wg[(size_t)gi * a.E + e] : 0.0f;
+      wts[c][i] = (gi < a.d && e < a.E) ? a.WgT[(size_t)e * a.d + gi] : 0.0f;
     }
     __syncthreads();
 #pragma unroll 8
     for (int c = 0; c < kRxEC; ++c) {
       const float4 w = *reinterpret_cast<const float4*>(&wts[c][4 * tx]);
+      const float4 g0 = *reinterpret_cast<const float4*>(&dls[c][8 * ty]);
+      const float4 g1 = *reinterpret_cast<const float4*>(&dls[c][8 * ty + 4]);
+      const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float g = dls[ty + 8 * k][c];
-        acc[k][0] = fmaf(g, w.x, acc[k][0]);
-        acc[k][1] = fmaf(g, w.y, acc[k][1]);
-        acc[k][2] = fmaf(g, w.z, acc[k][2]);
-        acc[k][3] = fmaf(g, w.w, acc[k][3]);
+      for (int k = 0; k < 8; ++k) {
+        acc[k][0] = fmaf(g[k], w.x, acc[k][0]);
+        acc[k][1] = fmaf(g[k], w.y, acc[k][1]);
+        acc[k][2] = fmaf(g[k], w.z, acc[k][2]);
+        acc[k][3] = fmaf(g[k], w.w, acc[k][3]);
       }
     }
   }
   const int col = i0 + 4 * tx;
   if (col >= a.d) return;
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int t = t0 + ty + 8 * k;
+  for (int k = 0; k < 8; ++k) {
+    const int t = t0 + 8 * ty + k;
     if (t >= a.n) continue;
     float v[4] = {acc[k][0], acc[k][1], acc[k][2], acc[k][3]};
     auto add_row = [&](long long row) {
@@ -333,8 +356,11 @@ int router_bwd_splits(int n, int d, int E) {
 }
 
 cudaError_t launch_router_backward(const RouterBwdArgs& a, cudaStream_t s) {
+  const dim3 gt(ceil_div(a.d, 32), ceil_div(a.E, 32));
+  cudaError_t e = launch_pdl(transpose_wg_kernel, gt, 256, 0, s, a.Wg, a.d, a.E, a.WgT);
+  if (e != cudaSuccess) return e;
   const dim3 gx(ceil_div(a.n, kRxBM), ceil_div(a.d, kRxBN));
-  cudaError_t e = launch_pdl(router_dx_kernel, gx, 256, 0, s, a);
+  e = launch_pdl(router_dx_kernel, gx, 256, 0, s, a);
   if (e != cudaSuccess) return e;
   const int per = ceil_div(ceil_div(a.n, a.splits), kRwBT) * kRwBT;
   const dim3 gw(ceil_div(a.d, kRwBM), ceil_div(a.E, kRwBN), a.splits);

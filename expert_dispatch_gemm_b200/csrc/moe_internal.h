@@ -235,7 +235,10 @@ struct BwdParams {
 struct BwdMaps {
   CUtensorMap a0, a1, b0, b0g, b1, b1g;
 };
-cudaError_t run_bwd_gemm(int mode, const BwdMaps& m, const BwdParams& p, cudaStream_t s);
+// pair: CTA pairs (cta_group::2, 256-row tiles); weight modes then take
+// mt_tiles in 256-row blocks
+cudaError_t run_bwd_gemm(int mode, bool pair, const BwdMaps& m, const BwdParams& p,
+                         cudaStream_t s);
 
 // element-wise and FFMA kernels of the backward (bwd.cu)
 struct CombineBwdArgs {
@@ -261,6 +264,7 @@ cudaError_t launch_pad_zero(const int32_t* offsets, const int32_t* counts, int E
 struct RouterBwdArgs {
   const __nv_bfloat16* X;        // [n, d]
   const float* Wg;               // [d, E]
+  float* WgT;                    // [E, d] workspace: W_g transposed
   const float* dL;               // [n, E]
   const __nv_bfloat16* dX_perm;  // [rows, d]
   const int32_t* tok_row;        // [n, slots]

@@ -422,7 +422,7 @@ def router_backward(X, Wg, dL):
 
 
 def layer_backward(spec: dict, X, Wg, dout, expert_weights, shared_weights=None,
-                   logit_bias=None, sel_bias=None, tokens=None):
+                   logit_bias=None, sel_bias=None, tokens=None, pre=None):
     """Gradients of <dout, out> + lb_coef L_lb + z_coef L_z (token choice) for
     the layer of ``layer_forward``, by the chain rule through the same steps:
     combine -> expert FFN -> dispatch (a sum over each token's pairs), and
@@ -433,14 +433,19 @@ def layer_backward(spec: dict, X, Wg, dout, expert_weights, shared_weights=None,
     (double, the logits' gradient), dWg [d,E], dW1/dW3/dW2 {expert: array},
     dsW1/dsW3/dsW2 {shared expert: array}, dgate {(t, e): value}.
     With ``tokens`` only those rows of dX and dL are computed (each needs only
-    its own pairs), and no weight gradient is returned."""
+    its own pairs), and no weight gradient is returned. ``pre`` = (logits, S,
+    lse, routing) from an earlier ``router`` + ``route`` of the same inputs
+    skips recomputing them."""
     X = _f32(X)
     dout = _f32(dout)
     n, d = X.shape
     store, act = spec["store"], spec["act"]
     score = spec.get("score", SOFTMAX)
-    logits, S, lse = router(X, Wg, logit_bias, score)
-    r = route(spec, S, lse, sel_bias)
+    if pre is None:
+        logits, S, lse = router(X, Wg, logit_bias, score)
+        r = route(spec, S, lse, sel_bias)
+    else:
+        logits, S, lse, r = pre
     E = S.shape[1]
     rows = list(range(n)) if tokens is None else sorted(int(t) for t in tokens)
     pairs = token_pairs(spec, r, n, rows if tokens is not None else None)

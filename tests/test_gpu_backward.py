@@ -143,3 +143,86 @@ def test_backward_zero_dout_gives_only_aux_gradients():
                                 expert_weights_from(inp), None, None, None)
     assert _rel(host(g["dL"]), ref["dL"]) < F32_GRAD_TOL
     assert _rel(host(g["dX"]), ref["dX"]) < BF16_GRAD_TOL
+
+
+def _flip_free_experts(spec, r, rb, bad):
+    """Experts whose rows are the same on both sides (no selection flip
+    touches them)."""
+    if not bad:
+        return None
+    if spec["mode"] == "ec":
+        I_g = rb.idx.cpu().numpy()
+        return {e for e in range(I_g.shape[0]) if set(I_g[e].tolist()) == set(r["I"][e].tolist())}
+    idx_g = rb.idx.cpu().numpy()
+    touched = set()
+    for t in bad:
+        touched |= set(idx_g[t].tolist()) | set(r["idx"][t].tolist())
+    return {e for e in range(rb.counts.numel()) if e not in touched}
+
+
+@pytest.mark.parametrize("w", [wl.EC_BF16, wl.TC_TOP2_CAP, wl.TC_DROPLESS, wl.TC_SIGMOID_GROUPED],
+                         ids=lambda w: w.name)
+def test_backward_full_size_sampled(w):
+    """The benchmark's workloads at full size: dX and dL on sampled tokens
+    (each needs only its own pairs), sampled hidden units of the weight
+    gradients of two experts and of the shared expert (a hidden unit's
+    weight gradients depend on that unit alone, so the oracle runs the
+    expert's backward restricted to the sampled units), and dWg = X^T dL as
+    a property of the library's own dL."""
+    inp = wl.make_inputs(w, DEV)
+    layer = moe.Layer(w, inp, DEV)
+    layer.forward()
+    dout = _dout(w, seed=5)
+    g = layer.backward(dout)
+    torch.cuda.synchronize()
+    _ws_ok(layer.ws)
+    _ws_ok(layer._bws)
+    spec = oracle.spec_of(w)
+    X = host(inp["X"])
+    logits, S, lse = oracle.router(X, host(inp["Wg"]), host(inp.get("logit_bias")),
+                                   spec["score"])
+    r = oracle.route(spec, S, lse, host(inp.get("sel_bias")))
+    bad = explained_routing_diff(spec, r, layer.route, S, host(inp.get("sel_bias")))
+    rng = np.random.default_rng(3)
+    toks = sorted([int(t) for t in rng.choice(w.n, size=16, replace=False)
+                   if int(t) not in bad][:4])
+    ref = oracle.layer_backward(spec, X, host(inp["Wg"]), host(dout), expert_weights_from(inp),
+                                expert_weights_from(inp, "s") if w.n_shared else None,
+                                host(inp.get("logit_bias")), host(inp.get("sel_bias")),
+                                tokens=toks, pre=(logits, S, lse, r))
+    assert _rel(host(g["dX"][torch.as_tensor(toks, device=DEV)]), ref["dX"]) < BF16_GRAD_TOL
+    assert _rel(host(g["dL"][torch.as_tensor(toks, device=DEV)]), ref["dL"]) < F32_GRAD_TOL
+    # the router weight gradient against X^T dL of the library's own dL
+    want = inp["X"].double().T @ g["dL"].double()
+    assert _rel(host(g["dWg"]), want.cpu().numpy()) < 1e-5
+    # weight gradients: sampled hidden units of two experts (and the shared one)
+    pairs = oracle.token_pairs(spec, r, w.n)
+    by_e = {}
+    for t, e, gate in pairs:
+        by_e.setdefault(e, []).append((t, gate))
+    ok = _flip_free_experts(spec, r, layer.route, bad)
+    cands = [e for e in sorted(by_e) if ok is None or e in ok]
+    experts = [cands[0], cands[len(cands) // 2]]
+    J = np.sort(rng.choice(w.h, size=3, replace=False))
+    W1, W3, W2 = inp["W1"], inp.get("W3"), inp["W2"]
+    swiglu = W3 is not None
+    checks = [(e, False) for e in experts] + [(s, True) for s in range(w.n_shared)]
+    for e, shared in checks:
+        p = "s" if shared else ""
+        if shared:
+            ts, gs = list(range(w.n)), [1.0] * w.n
+        else:
+            ts, gs = [t for t, _ in by_e[e]], [gt for _, gt in by_e[e]]
+        dY, _ = oracle.combine_backward(np.asarray(ts, np.int32), np.asarray(gs, np.float32),
+                                        np.zeros((len(ts), w.d), np.float32), host(dout),
+                                        spec["store"])
+        w1 = host(inp[p + "W1"][e])[J]
+        w3 = host(inp[p + "W3"][e])[J] if swiglu else None
+        w2 = host(inp[p + "W2"][e])[:, J]
+        _, r1, r3, r2 = oracle.expert_ffn_backward(X[ts], w1, w3, w2, dY, spec["act"],
+                                                   spec["store"])
+        jt = torch.as_tensor(J, device=DEV)
+        assert _rel(host(g["d" + p + "W1"][e][jt]), r1) < BF16_GRAD_TOL, (e, shared, "W1")
+        assert _rel(host(g["d" + p + "W2"][e][:, jt]), r2) < BF16_GRAD_TOL, (e, shared, "W2")
+        if swiglu:
+            assert _rel(host(g["d" + p + "W3"][e][jt]), r3) < BF16_GRAD_TOL, (e, shared, "W3")
