@@ -644,6 +644,9 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float*
   moe_status st = derive(cfg, &d);
   if (st != MOE_OK) return st;
   if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  // the weight-gradient epilogue writes 32-row groups that never straddle
+  // the W1 / W3 boundary (h) or the end of the output (d, h or 2h)
+  if (cfg->d % 64 != 0 || cfg->h % 64 != 0) return MOE_ERR_UNSUPPORTED;
   const bool swiglu = cfg->act == MOE_ACT_SWIGLU;
   const bool tc = cfg->mode == MOE_TOKEN_CHOICE;
   if (!X || !Wg || !W1 || !W2 || !dout || !dX || !dWg || !dW1 || !dW2) return MOE_ERR_INVALID_ARG;

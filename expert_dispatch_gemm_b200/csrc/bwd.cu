@@ -240,19 +240,31 @@ __global__ void __launch_bounds__(256) router_dx_kernel(RouterBwdArgs a) {
     const int t = t0 + 8 * ty + k;
     if (t >= a.n) continue;
     float v[4] = {acc[k][0], acc[k][1], acc[k][2], acc[k][3]};
-    auto add_row = [&](long long row) {
-      const uint2 x = *reinterpret_cast<const uint2*>(a.dX_perm + (size_t)row * a.d + col);
+    auto add = [&](const uint2 x) {
       v[0] += bf_lo(x.x);
       v[1] += bf_hi(x.x);
       v[2] += bf_lo(x.y);
       v[3] += bf_hi(x.y);
     };
-    for (int j = 0; j < a.slots; ++j) {
-      const int r = a.tok_row[(size_t)t * a.slots + j];
-      if (r < 0) break;
-      add_row(r);
+    auto at_row = [&](long long row) {
+      return *reinterpret_cast<const uint2*>(a.dX_perm + (size_t)row * a.d + col);
+    };
+    // the token's rows four at a time, so that four independent loads are in
+    // flight (sums stay in slot order)
+    const int32_t* tr = a.tok_row + (size_t)t * a.slots;
+    for (int j = 0; j < a.slots; j += 4) {
+      int r[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) r[u] = j + u < a.slots ? tr[j + u] : -1;
+      uint2 x[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) x[u] = r[u] >= 0 ? at_row(r[u]) : make_uint2(0, 0);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (r[u] >= 0) add(x[u]);
+      if (r[3] < 0) break;
     }
-    for (int sidx = 0; sidx < a.n_shared; ++sidx) add_row(a.shared_base + sidx * a.n_pad + t);
+    for (int sidx = 0; sidx < a.n_shared; ++sidx) add(at_row(a.shared_base + sidx * a.n_pad + t));
     uint2 o;
     o.x = pack_bf16x2(v[0], v[1]);
     o.y = pack_bf16x2(v[2], v[3]);

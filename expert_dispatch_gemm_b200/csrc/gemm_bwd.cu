@@ -629,14 +629,18 @@ __device__ __forceinline__ void bwd_body(const CUtensorMap* tmA0, const CUtensor
             *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) * 16)) = pk;
           }
           __syncwarp();
+          // the warp's 32 rows lie on one side of m_split and of m_total
+          // (both multiples of 64), so one base pointer serves them all
+          __nv_bfloat16* gbase = wgrad_row(p, t, t.m0 + q * 32);
+          if (gbase) {
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int idx = lane + 32 * k, r = idx >> 3, pc = idx & 7;
-            const int col = t.n0 + cc + 8 * pc;
-            __nv_bfloat16* orow = wgrad_row(p, t, t.m0 + q * 32 + r);
-            if (orow && col < p.ld_w)
-              *reinterpret_cast<uint4*>(orow + col) =
-                  *reinterpret_cast<const uint4*>(stg + r * 128 + ((pc ^ (r & 7)) * 16));
+            for (int k = 0; k < 8; ++k) {
+              const int idx = lane + 32 * k, r = idx >> 3, pc = idx & 7;
+              const int col = t.n0 + cc + 8 * pc;
+              if (col < p.ld_w)
+                *reinterpret_cast<uint4*>(gbase + (size_t)r * p.ld_w + col) =
+                    *reinterpret_cast<const uint4*>(stg + r * 128 + ((pc ^ (r & 7)) * 16));
+            }
           }
           __syncwarp();
         }
