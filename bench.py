@@ -265,10 +265,16 @@ def run_gpu(args, w: wl.Workload):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     sb = inp["sel_bias"]
+    fused = args.fused_combine
+    if fused:
+        acc = torch.empty((w.n, w.d), dtype=torch.float32, device=dev)
+        row_gate = torch.empty(max(sz.rows, 1), dtype=torch.float32, device=dev)
 
     def step(ev=None, X=None, out_buf=None):
         """One pass of the layer, the calls moe_layer_forward makes:
-        route -> dispatch gather -> grouped expert FFN -> combine."""
+        route -> dispatch gather -> grouped expert FFN -> combine (with
+        --fused-combine: the combine inside the down projection's epilogue,
+        moe_expert_ffn_combined)."""
         X = inp["X"] if X is None else X
         o = out if out_buf is None else out_buf
         if ev: ev[0].record(stream)
@@ -276,11 +282,17 @@ def run_gpu(args, w: wl.Workload):
         if ev: ev[1].record(stream)
         moe.moe_dispatch(cfg, X, rb, X_perm, stream)
         if ev: ev[2].record(stream)
-        moe.moe_expert_ffn(cfg, X, X_perm, rb.offsets, inp["W1"], inp["W3"], inp["W2"],
-                           inp.get("sW1"), inp.get("sW3"), inp.get("sW2"), H, Y, ws, stream,
-                           counts=rb.counts)
-        if ev: ev[3].record(stream)
-        moe.moe_combine(cfg, Y, rb, o, stream)
+        if fused:
+            moe.moe_expert_ffn_combined(cfg, X, X_perm, rb, inp["W1"], inp["W3"], inp["W2"],
+                                        inp.get("sW1"), inp.get("sW3"), inp.get("sW2"), H, acc,
+                                        row_gate, o, ws, stream)
+            if ev: ev[3].record(stream)
+        else:
+            moe.moe_expert_ffn(cfg, X, X_perm, rb.offsets, inp["W1"], inp["W3"], inp["W2"],
+                               inp.get("sW1"), inp.get("sW3"), inp.get("sW2"), H, Y, ws, stream,
+                               counts=rb.counts)
+            if ev: ev[3].record(stream)
+            moe.moe_combine(cfg, Y, rb, o, stream)
         if ev: ev[4].record(stream)
 
     for _ in range(args.warmup):
@@ -429,6 +441,8 @@ def run_gpu(args, w: wl.Workload):
     # route: router (+ split-k reduce) + select_ec + ec_finish (EC) or + hist +
     # scan + scatter (TC); dispatch: gather; expert FFN: up + down; combine
     launches_per_step = sum(moe.launch_counts(cfg).values())
+    if fused:
+        launches_per_step += 1  # prep + up + down + finish replace up + down + combine
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
@@ -440,7 +454,9 @@ def run_gpu(args, w: wl.Workload):
                    "hidden": w.h, "routing": ("expert-choice c=%g" % w.c if w.mode == "ec"
                                               else "token-choice top-%d" % w.K),
                    "parallelism": f"replicas{world}" if world > 1 else "single-gpu",
-                   "l2": "flushed between timed steps (256 MB write, outside the events)"},
+                   "l2": "flushed between timed steps (256 MB write, outside the events)",
+                   **({"combine": "fused into the down projection (moe_expert_ffn_combined); "
+                                  "the ffn stage includes it"} if fused else {})},
         "roofline": roof,
         "stages": stages,
         "routing": routing,
@@ -745,6 +761,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--ref-sample", type=int, default=48)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fused-combine", action="store_true",
+                    help="forward: the combine inside the down projection's epilogue")
     ap.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "train"],
                     help="forward: the layer's forward (default); train: forward + backward")
     args = ap.parse_args()

@@ -290,13 +290,16 @@ static bool ffn_uses_swap(const moe_config* c, const Derived& dv) {
   return avg >= kRowAlign && avg <= 4 * kRowAlign;
 }
 
+// row_gate / out32: the combine fused into the down projection (then Y is
+// not written and may be NULL)
 static moe_status ffn_impl(const moe_config* c, const Derived& dv, const void* X,
                            const void* X_perm, const int32_t* row_token, const int32_t* offsets,
                            const int32_t* counts, const void* W1, const void* W3,
                            const void* W2, const void* sW1,
                            const void* sW3, const void* sW2, void* H, void* Y, int* err,
-                           cudaStream_t s) {
-  if (!offsets || !W1 || !W2 || !H || !Y) return MOE_ERR_INVALID_ARG;
+                           cudaStream_t s, const float* row_gate = nullptr,
+                           float* out32 = nullptr) {
+  if (!offsets || !W1 || !W2 || !H || (!Y && !out32)) return MOE_ERR_INVALID_ARG;
   if (!X_perm && (!X || !row_token)) return MOE_ERR_INVALID_ARG;
   if (c->act == MOE_ACT_SWIGLU && !W3) return MOE_ERR_INVALID_ARG;
   if (c->n_shared > 0) {
@@ -329,8 +332,10 @@ static moe_status ffn_impl(const moe_config* c, const Derived& dv, const void* X
   f.rows = dv.rows;
   f.err = err;
   f.pair = ffn_uses_pair(c, dv);
-  if (c->dtype != MOE_BF16) return run_ffn_f32(f, s);
-  if (ffn_uses_swap(c, dv) && swap_down_supported(f)) {
+  f.row_gate = row_gate;
+  f.out32 = out32;
+  if (c->dtype != MOE_BF16) return out32 ? MOE_ERR_UNSUPPORTED : run_ffn_f32(f, s);
+  if (!out32 && ffn_uses_swap(c, dv) && swap_down_supported(f)) {
     f.skip_down = true;
     const moe_status st = run_ffn_bf16(f, s);
     if (st != MOE_OK) return st;
@@ -568,6 +573,31 @@ moe_status moe_expert_ffn_gathered(const moe_config* cfg, const void* X,
   return ffn_impl(cfg, d, X, nullptr, route->row_token, route->offsets, nullptr, W1, W3, W2,
                   sW1, sW3,
                   sW2, H, Y_perm, at<int>(ws, 0), (cudaStream_t)stream);
+}
+
+moe_status moe_expert_ffn_combined(const moe_config* cfg, const void* X, const void* X_perm,
+                                   const moe_route_out* route, const void* W1, const void* W3,
+                                   const void* W2, const void* sW1, const void* sW3,
+                                   const void* sW2, void* H, float* acc, float* row_gate,
+                                   void* out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  Derived d;
+  moe_status st = derive(cfg, &d);
+  if (st != MOE_OK) return st;
+  if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (!X || !route || !route->row_token || !route->offsets || !route->tok_row ||
+      !route->tok_gate || !acc || !row_gate || !out)
+    return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(acc) | reinterpret_cast<uintptr_t>(out)) & 15)
+    return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(ws, ws_bytes, MOE_WS_ERROR_BYTES)) != MOE_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  MOE_CU(launch_combine_prep(route->tok_row, route->tok_gate, cfg->n, d.slots, cfg->d, row_gate,
+                             acc, s));
+  if ((st = ffn_impl(cfg, d, X, X_perm, route->row_token, route->offsets, nullptr, W1, W3, W2,
+                     sW1, sW3, sW2, H, nullptr, at<int>(ws, 0), s, row_gate, acc)) != MOE_OK)
+    return st;
+  MOE_CU(launch_combine_finish(acc, cfg->n, cfg->d, out, s));
+  return MOE_OK;
 }
 
 moe_status moe_bias_update(const moe_config* cfg, const int32_t* load, float rate, float* bias,

@@ -283,6 +283,58 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
   return launch_pdl(combine_kernel<false>, a.n, 128, 0, s, a);
 }
 
+// The combine fused into the down projection ("Expert choice routing",
+// "The math": out = scatter_add(G * Y)): the epilogue adds gate * Y rows into
+// an fp32 [n, d] buffer with vector reductions. Before it, this kernel zeroes
+// the buffer and writes each dispatched row's gate; after it, the buffer is
+// rounded into the output.
+__global__ void __launch_bounds__(256) combine_prep_kernel(const int32_t* tok_row,
+                                                           const float* tok_gate, int n,
+                                                           int slots, int d, float* row_gate,
+                                                           float* out32) {
+  pdl_wait();
+  const long long tid = (long long)blockIdx.x * 256 + threadIdx.x;
+  const long long nthreads = (long long)gridDim.x * 256;
+  for (long long q = tid; q < (long long)n * slots; q += nthreads) {
+    const int r = tok_row[q];
+    if (r >= 0) row_gate[r] = tok_gate[q];
+  }
+  const long long nvec = (long long)n * d / 4;
+  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (long long q = tid; q < nvec; q += nthreads) reinterpret_cast<float4*>(out32)[q] = z;
+}
+
+__global__ void __launch_bounds__(256) combine_finish_kernel(const float* out32, long long count,
+                                                             __nv_bfloat16* out) {
+  pdl_wait();
+  const long long nvec = count / 8;
+  for (long long q = (long long)blockIdx.x * 256 + threadIdx.x; q < nvec;
+       q += (long long)gridDim.x * 256) {
+    const float4 a = reinterpret_cast<const float4*>(out32)[2 * q];
+    const float4 b = reinterpret_cast<const float4*>(out32)[2 * q + 1];
+    reinterpret_cast<uint4*>(out)[q] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w),
+                                                  pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+  }
+}
+
+static int fill_grid() {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return 4 * sms;
+}
+
+cudaError_t launch_combine_prep(const int32_t* tok_row, const float* tok_gate, int n, int slots,
+                                int d, float* row_gate, float* out32, cudaStream_t s) {
+  return launch_pdl(combine_prep_kernel, fill_grid(), 256, 0, s, tok_row, tok_gate, n, slots, d,
+                    row_gate, out32);
+}
+
+cudaError_t launch_combine_finish(const float* out32, int n, int d, void* out, cudaStream_t s) {
+  return launch_pdl(combine_finish_kernel, fill_grid(), 256, 0, s, out32, (long long)n * d,
+                    static_cast<__nv_bfloat16*>(out));
+}
+
 // "MoE routing strategies explained", "4. Sigmoid gating with aux-loss-free
 // bias": after each step the bias drops for overloaded experts and rises for
 // idle ones. The sign is taken exactly in integers: load*E vs n*K.

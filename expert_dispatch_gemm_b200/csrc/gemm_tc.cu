@@ -42,6 +42,10 @@ constexpr int kGemmThreads = 192;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 enum { ACT_NONE = 0, ACT_RELU = 1, ACT_GELU = 2, ACT_SWIGLU = 3 };
+// what a projection fuses: nothing; the dispatch gather into its A loads (up
+// projection); the gate-scaled scatter-add of the combine into its epilogue
+// (down projection)
+enum { FUSE_NONE = 0, FUSE_GATHER = 1, FUSE_SCATTER = 2 };
 
 struct TcGemmParams {
   const int32_t* offsets;
@@ -59,7 +63,10 @@ struct TcGemmParams {
   long long n_pad;
   __nv_bfloat16* out;       // [rows, n_out]
   int* err;
-  const int32_t* row_token;  // source token of each dispatched row (gathered A)
+  const int32_t* row_token;  // source token of each dispatched row (gathered A, scatter)
+  const float* row_gate;     // scatter: gate of each dispatched row
+  float* out32;              // scatter: [n_tok, n_out] fp32 sums
+  int n_tok;
 };
 
 struct SharedState {
@@ -140,6 +147,13 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, const TcGemmParams& p
   return c;
 }
 
+// fp32 vector reduction into global memory (sm_90+), 16-byte aligned
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
 template <int ACT>
 __device__ __forceinline__ float act_fn(float v) {
   if (ACT == ACT_RELU) return fmaxf(v, 0.0f);
@@ -147,7 +161,7 @@ __device__ __forceinline__ float act_fn(float v) {
   return v;
 }
 
-template <int ACT, bool GATHER>
+template <int ACT, int FUSE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,
                            const __grid_constant__ CUtensorMap tmA1,
@@ -211,7 +225,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0) {
     // the whole warp walks the schedule; lane 0 waits and issues the 2-D
-    // loads, and with GATHER every lane issues one 4-row gather of A
+    // loads, and with FUSE_GATHER every lane issues one 4-row gather of A
     int stage = 0;
     uint32_t phase = 0;
     int issued = 0;
@@ -223,7 +237,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const CUtensorMap* mbg = c.b_sel ? &tmB1g : &tmB0g;
       // routed rows straight from X: lane l brings rows 4l..4l+3 of the block;
       // padding rows read token 0 and their outputs are never used
-      const bool gather = GATHER && c.a_sel == 0;
+      const bool gather = FUSE == FUSE_GATHER && c.a_sel == 0;
       int tok[4] = {0, 0, 0, 0};
       if (gather) {
 #pragma unroll
@@ -336,6 +350,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const TileCoord c = decode_tile<ACT>(tile, p, st->offs, st->tprefix, routed);
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN);
       __nv_bfloat16* orow = p.out + (size_t)(c.out_row + row_in_tile) * p.n_out;
+      // scatter: the row's token and gate (shared experts: weight 1, the
+      // token is the row within the expert's block of n_pad rows)
+      int tok = -1;
+      float gate = 0.0f;
+      if (FUSE == FUSE_SCATTER) {
+        const long long r = c.out_row + row_in_tile;
+        if (c.a_sel == 0) {
+          tok = p.row_token[r];
+          gate = tok >= 0 ? p.row_gate[r] : 0.0f;
+        } else {
+          const long long q2 = (r - p.out_shared_base) % p.n_pad;
+          tok = q2 < p.n_tok ? (int)q2 : -1;
+          gate = 1.0f;
+        }
+      }
 #pragma unroll 1
       for (int cc = 0; cc < BNO; cc += 32) {
         if (c.col0 + cc >= p.n_out) break;
@@ -357,15 +386,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) f[i] = act_fn<ACT>(__uint_as_float(v[i]));
         }
-        uint4* dst = reinterpret_cast<uint4*>(orow + c.col0 + cc);
+        if (FUSE == FUSE_SCATTER) {
+          if (tok >= 0) {
+            float* dst = p.out32 + (size_t)tok * p.n_out + c.col0 + cc;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint4 o;
-          o.x = pack_bf16x2(f[8 * j + 0], f[8 * j + 1]);
-          o.y = pack_bf16x2(f[8 * j + 2], f[8 * j + 3]);
-          o.z = pack_bf16x2(f[8 * j + 4], f[8 * j + 5]);
-          o.w = pack_bf16x2(f[8 * j + 6], f[8 * j + 7]);
-          dst[j] = o;
+            for (int j = 0; j < 8; ++j)
+              red_add_v4(dst + 4 * j, gate * f[4 * j], gate * f[4 * j + 1], gate * f[4 * j + 2],
+                         gate * f[4 * j + 3]);
+          }
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c.col0 + cc);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint4 o;
+            o.x = pack_bf16x2(f[8 * j + 0], f[8 * j + 1]);
+            o.y = pack_bf16x2(f[8 * j + 2], f[8 * j + 3]);
+            o.z = pack_bf16x2(f[8 * j + 4], f[8 * j + 5]);
+            o.w = pack_bf16x2(f[8 * j + 6], f[8 * j + 7]);
+            dst[j] = o;
+          }
         }
       }
       sm100::tc_fence_before();
@@ -490,7 +529,7 @@ __device__ __forceinline__ PairCoord decode_pair(int tile, const TcGemmParams& p
   return c;
 }
 
-template <int ACT, bool GATHER>
+template <int ACT, int FUSE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     tc_grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0,
                                 const __grid_constant__ CUtensorMap tmA1,
@@ -561,7 +600,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0) {
     // the whole warp walks the schedule; lane 0 waits and issues the 2-D
-    // loads, and with GATHER every lane issues one 4-row gather of A
+    // loads, and with FUSE_GATHER every lane issues one 4-row gather of A
     int stage = 0;
     uint32_t phase = 0;
     int issued = 0;
@@ -576,7 +615,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         mb = c.b_sel ? &tmB1 : &tmB0;
       // routed rows straight from X: lane l brings rows 4l..4l+3 of the block;
       // padding rows read token 0 and their outputs are never used
-      const bool gather = GATHER && c.a_sel == 0;
+      const bool gather = FUSE == FUSE_GATHER && c.a_sel == 0;
       int tok[4] = {0, 0, 0, 0};
       if (gather) {
 #pragma unroll
@@ -683,6 +722,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const PairCoord c = decode_pair<ACT>(tile, p, st->offs, st->tprefix, routed, rank);
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kBN);
       __nv_bfloat16* orow = p.out + (size_t)(c.out_row + row_in_tile) * p.n_out;
+      // scatter: the row's token and gate (shared experts: weight 1, the
+      // token is the row within the expert's block of n_pad rows)
+      int tok = -1;
+      float gate = 0.0f;
+      if (FUSE == FUSE_SCATTER) {
+        const long long r = c.out_row + row_in_tile;
+        if (c.a_sel == 0) {
+          tok = p.row_token[r];
+          gate = tok >= 0 ? p.row_gate[r] : 0.0f;
+        } else {
+          const long long q2 = (r - p.out_shared_base) % p.n_pad;
+          tok = q2 < p.n_tok ? (int)q2 : -1;
+          gate = 1.0f;
+        }
+      }
       if (c.valid) {
 #pragma unroll 1
         for (int cc = 0; cc < BNO; cc += 32) {
@@ -705,15 +759,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) f[i] = act_fn<ACT>(__uint_as_float(v[i]));
           }
-          uint4* dst = reinterpret_cast<uint4*>(orow + c.col0 + cc);
+          if (FUSE == FUSE_SCATTER) {
+            if (tok >= 0) {
+              float* dst = p.out32 + (size_t)tok * p.n_out + c.col0 + cc;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint4 o;
-            o.x = pack_bf16x2(f[8 * j + 0], f[8 * j + 1]);
-            o.y = pack_bf16x2(f[8 * j + 2], f[8 * j + 3]);
-            o.z = pack_bf16x2(f[8 * j + 4], f[8 * j + 5]);
-            o.w = pack_bf16x2(f[8 * j + 6], f[8 * j + 7]);
-            dst[j] = o;
+              for (int j = 0; j < 8; ++j)
+                red_add_v4(dst + 4 * j, gate * f[4 * j], gate * f[4 * j + 1], gate * f[4 * j + 2],
+                           gate * f[4 * j + 3]);
+            }
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c.col0 + cc);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint4 o;
+              o.x = pack_bf16x2(f[8 * j + 0], f[8 * j + 1]);
+              o.y = pack_bf16x2(f[8 * j + 2], f[8 * j + 3]);
+              o.z = pack_bf16x2(f[8 * j + 4], f[8 * j + 5]);
+              o.w = pack_bf16x2(f[8 * j + 6], f[8 * j + 7]);
+              dst[j] = o;
+            }
           }
         }
       }
@@ -790,15 +854,20 @@ static cudaError_t launch_one(K kern, const Maps& m, const TcGemmParams& p, int 
 }
 
 // grid: CTAs for the single-CTA kernel, CTA pairs for the pair kernel
+template <int ACT, int FUSE>
+static cudaError_t launch_gemm_t(const Maps& m, const TcGemmParams& p, bool pair, int grid,
+                                 cudaStream_t s) {
+  const size_t bytes = gemm_smem_bytes(pair);
+  if (pair) return launch_one(tc_grouped_gemm_pair_kernel<ACT, FUSE>, m, p, 2 * grid, bytes, s);
+  return launch_one(tc_grouped_gemm_kernel<ACT, FUSE>, m, p, grid, bytes, s);
+}
+
+// up projections fuse nothing or the gather
 template <int ACT>
 static cudaError_t launch_gemm(const Maps& m, const TcGemmParams& p, bool pair, bool gather,
                                int grid, cudaStream_t s) {
-  const size_t bytes = gemm_smem_bytes(pair);
-  if (pair)
-    return gather ? launch_one(tc_grouped_gemm_pair_kernel<ACT, true>, m, p, 2 * grid, bytes, s)
-                  : launch_one(tc_grouped_gemm_pair_kernel<ACT, false>, m, p, 2 * grid, bytes, s);
-  return gather ? launch_one(tc_grouped_gemm_kernel<ACT, true>, m, p, grid, bytes, s)
-                : launch_one(tc_grouped_gemm_kernel<ACT, false>, m, p, grid, bytes, s);
+  return gather ? launch_gemm_t<ACT, FUSE_GATHER>(m, p, pair, grid, s)
+                : launch_gemm_t<ACT, FUSE_NONE>(m, p, pair, grid, s);
 }
 
 static int num_sms() {
@@ -922,7 +991,15 @@ moe_status run_ffn_bf16(const FfnArgs& f, cudaStream_t s) {
   q.a1_row_base = f.shared_base;
   q.a1_row_stride = f.n_pad;
   q.out = static_cast<__nv_bfloat16*>(f.Y);
-  e = launch_gemm<ACT_NONE>(dm, q, pair, false, persistent_grid(q, pair), s);
+  if (f.out32) {
+    // the combine fused into the epilogue: out32[token] += gate * Y row
+    q.row_gate = f.row_gate;
+    q.out32 = f.out32;
+    q.n_tok = f.n;
+    e = launch_gemm_t<ACT_NONE, FUSE_SCATTER>(dm, q, pair, persistent_grid(q, pair), s);
+  } else {
+    e = launch_gemm_t<ACT_NONE, FUSE_NONE>(dm, q, pair, persistent_grid(q, pair), s);
+  }
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }

@@ -193,6 +193,10 @@ struct FfnArgs {
   int* err;
   bool pair;  // bf16: CTA-pair (cta_group::2) kernel instead of the single-CTA one
   bool skip_down;  // run the up projection only
+  // combine fused into the down projection: out32[token] += gate * row
+  // (fp32 reductions), row_gate [rows]; Y is then not written
+  const float* row_gate;
+  float* out32;
 };
 // GEMM kernel choice for a config
 bool ffn_uses_pair(const moe_config* c, const Derived& d);
@@ -277,6 +281,12 @@ struct RouterBwdArgs {
 };
 int router_bwd_splits(int n, int d, int E);
 cudaError_t launch_router_backward(const RouterBwdArgs& a, cudaStream_t s);
+
+// the fused combine's bookkeeping: zero out32 [n, d] and write each
+// dispatched row's gate; then round out32 into the output
+cudaError_t launch_combine_prep(const int32_t* tok_row, const float* tok_gate, int n, int slots,
+                                int d, float* row_gate, float* out32, cudaStream_t s);
+cudaError_t launch_combine_finish(const float* out32, int n, int d, void* out, cudaStream_t s);
 
 cudaError_t launch_bias_update(int n, int E, int K, const int32_t* load, float rate,
                                float* bias, cudaStream_t s);

@@ -36,7 +36,8 @@ API_SYMBOLS = ["moe_status_string", "moe_validate", "moe_sizes", "moe_workspace_
                "moe_route", "moe_route_from_scores", "moe_dispatch", "moe_expert_ffn",
                "moe_combine", "moe_layer_forward", "moe_bias_update", "moe_workspace_init",
                "moe_read_error", "moe_route_noalloc", "moe_expert_ffn_gathered",
-               "moe_launch_counts", "moe_backward_workspace_size", "moe_layer_backward"]
+               "moe_launch_counts", "moe_backward_workspace_size", "moe_layer_backward",
+               "moe_expert_ffn_combined"]
 MOE_ROUTE_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -97,6 +98,8 @@ def lib() -> ctypes.CDLL:
         L.moe_route_noalloc.argtypes = [cfgp, P, P, P, P, outp, P]
         L.moe_expert_ffn_gathered.argtypes = [cfgp, P, outp, P, P, P, P, P, P, P, P, P,
                                               ctypes.c_size_t, P]
+        L.moe_expert_ffn_combined.argtypes = [cfgp, P, P, outp, P, P, P, P, P, P, P, P, P, P,
+                                              P, ctypes.c_size_t, P]
         L.moe_backward_workspace_size.argtypes = [cfgp, ctypes.POINTER(ctypes.c_size_t), ip]
         L.moe_layer_backward.argtypes = [cfgp, P, P, P, P, P, P, P, P, outp, P, ctypes.c_size_t,
                                          P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
@@ -273,6 +276,15 @@ def moe_expert_ffn_gathered(cfg, X, route: RouteBuffers, W1, W3, W2, sW1, sW3, s
                                          _ptr(W1), _ptr(W3), _ptr(W2), _ptr(sW1), _ptr(sW3),
                                          _ptr(sW2), _ptr(H), _ptr(Y_perm), _ptr(ws), ws.numel(),
                                          _stream(stream)), "moe_expert_ffn_gathered")
+
+
+def moe_expert_ffn_combined(cfg, X, X_perm, route: RouteBuffers, W1, W3, W2, sW1, sW3, sW2, H,
+                            acc, row_gate, out, ws, stream=None):
+    _check(lib().moe_expert_ffn_combined(ctypes.byref(cfg), _ptr(X), _ptr(X_perm),
+                                         ctypes.byref(route.c), _ptr(W1), _ptr(W3), _ptr(W2),
+                                         _ptr(sW1), _ptr(sW3), _ptr(sW2), _ptr(H), _ptr(acc),
+                                         _ptr(row_gate), _ptr(out), _ptr(ws), ws.numel(),
+                                         _stream(stream)), "moe_expert_ffn_combined")
 
 
 def moe_combine(cfg, Y_perm, route: RouteBuffers, out, stream=None):

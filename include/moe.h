@@ -317,6 +317,23 @@ MOE_API moe_status moe_route_noalloc(const moe_config* cfg, const void* X, const
                                      const float* logit_bias, const float* sel_bias,
                                      moe_route_out* out, moe_stream_t stream);
 
+/* moe_expert_ffn + moe_combine with the combine fused into the down
+ * projection's epilogue ([EC-math] "The math": out = scatter_add(G * Y)):
+ * each row's output is scaled by its gate and added, in fp32, into acc
+ * [n,d] at its token (vector reductions, so the summation order is not
+ * fixed), and acc is then rounded into out [n,d]. Y_perm is never written,
+ * and Y rows are not rounded to bf16 before the gate multiplies them. X_perm
+ * may be NULL: the first projection then gathers its rows from X as in
+ * moe_expert_ffn_gathered. acc (16-byte aligned) and row_gate [rows] are
+ * caller-owned scratch. bf16 configs only. Measured slower than the separate
+ * combine on every workload; the layer does not use it. */
+MOE_API moe_status moe_expert_ffn_combined(const moe_config* cfg, const void* X,
+                                           const void* X_perm, const moe_route_out* route,
+                                           const void* W1, const void* W3, const void* W2,
+                                           const void* sW1, const void* sW3, const void* sW2,
+                                           void* H, float* acc, float* row_gate, void* out,
+                                           void* ws, size_t ws_bytes, moe_stream_t stream);
+
 /* ---- backward pass of moe_layer_forward -------------------------------
  * The gradient, by the chain rule, of
  *     loss = <dout, out> + L_lb + L_z

@@ -384,3 +384,45 @@ def test_capacity_one_all_equal_scores():
     assert drop[0].sum() == 0 and (drop[1:] == 1).all()
     spec = oracle.spec_of(w)
     check_routing_exact(spec, oracle.route(spec, S.numpy()), rb, w.n, w.E, weights_rtol(spec))
+
+
+# --------------------------------------------------------------------------
+# the combine fused into the down projection (moe_expert_ffn_combined)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("w", wl.SMALL[1:] + [wl.TC_DROPLESS], ids=lambda w: w.name)
+@pytest.mark.parametrize("gathered", [False, True], ids=["x_perm", "gathered"])
+def test_fused_combine(w, gathered):
+    """out from the gate-scaled scatter-add in the down projection's epilogue
+    against the oracle (bf16 bar on the tokens whose routing agrees) and
+    against the unfused layer: the only differences are the fp32 reduction
+    order and Y not being rounded to bf16 first."""
+    inp = wl.make_inputs(w, DEV)
+    layer = moe.Layer(w, inp, DEV)
+    ref_out = layer.forward().clone()
+    cfg, rb = layer.cfg, layer.route
+    sz = moe.sizes(cfg)
+    X_perm = None
+    if not gathered:
+        X_perm = torch.empty((sz.rows, w.d), dtype=w.torch_dtype, device=DEV)
+        moe.moe_dispatch(cfg, inp["X"], rb, X_perm)
+    H = torch.empty((sz.rows, w.h), dtype=w.torch_dtype, device=DEV)
+    acc = torch.empty((w.n, w.d), dtype=torch.float32, device=DEV)
+    row_gate = torch.empty(max(sz.rows, 1), dtype=torch.float32, device=DEV)
+    out = torch.empty((w.n, w.d), dtype=w.torch_dtype, device=DEV)
+    moe.moe_expert_ffn_combined(cfg, inp["X"], X_perm, rb, inp["W1"], inp.get("W3"), inp["W2"],
+                                inp.get("sW1"), inp.get("sW3"), inp.get("sW2"), H, acc, row_gate,
+                                out, layer.ws)
+    torch.cuda.synchronize()
+    _ws_ok(layer.ws)
+    got = host(out).astype(np.float64)
+    unfused = host(ref_out).astype(np.float64)
+    rel = np.linalg.norm(got - unfused) / np.linalg.norm(unfused)
+    assert rel < 5e-3, rel
+    if w.n <= 2048:
+        spec, logits, S, lse, r = _oracle_from_x(w, inp)
+        bad = explained_routing_diff(spec, r, layer.route, S, host(inp.get("sel_bias")))
+        ref = oracle.layer_forward(spec, host(inp["X"]), r, expert_weights_from(inp),
+                                   expert_weights_from(inp, "s") if w.n_shared else None)
+        keep = np.array([t not in bad for t in range(w.n)])
+        compare_out(spec["store"], got[keep], ref[keep], w.name)
