@@ -587,20 +587,28 @@ def run_gpu_train(args, w: wl.Workload):
     tc_peak = tc_sust if (capped and tc_sust) else tc_burst
     bwd_med = float(np.median(bwd_ms))
     ach = gemm_flops / (bwd_med * 1e-3) / 1e12
-    roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": tc_peak, "unit": "TFLOP/s",
-            "frac": round(ach / tc_peak, 3),
-            "peak_kind": "sustained (sw_power_cap active)" if (capped and tc_sust) else "burst",
-            "traffic": None, "peak_source": src,
-            "kernel": "moe_layer_backward as a whole: the five grouped GEMMs' FLOPs over the "
-                      "whole call (its non-GEMM kernels included in the time)",
-            "algorithmic_per_launch": gemm_flops}
+    if w.dtype == "f32":
+        # the fp32 layer's GEMMs run on FFMA: their roof is that pipe
+        fpk = ffma_peak_tflops(dev)
+        roof = {"bound": "alu", "achieved": round(ach, 2), "peak": round(fpk, 1),
+                "unit": "TFLOP/s", "frac": round(ach / fpk, 3),
+                "peak_kind": "FP32 FFMA, measured by the probe kernel"}
+    else:
+        roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": tc_peak,
+                "unit": "TFLOP/s", "frac": round(ach / tc_peak, 3),
+                "peak_kind": "sustained (sw_power_cap active)" if (capped and tc_sust)
+                else "burst"}
+    roof.update({"traffic": None, "peak_source": src,
+                 "kernel": "moe_layer_backward as a whole: the five grouped GEMMs' FLOPs over "
+                           "the whole call (its non-GEMM kernels included in the time)",
+                 "algorithmic_per_launch": gemm_flops})
     fwd_launches = sum(moe.launch_counts(layer.cfg).values())
     res = {
         "metric": METRIC_TRAIN,
         "value": round(whole_job_rate(w.n, world, args.steps, total_ms), 1), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic (seeded N(0,1) activations and output gradient, random-init weights)",
         "config": {"workload": w.name, "pass": "forward + backward", "tokens": w.n,
                    "d_model": w.d, "experts": w.E, "hidden": w.h,
@@ -772,8 +780,6 @@ def main():
     if args.impl == "reference":
         run_reference(args, w)
     elif args.pass_ == "train":
-        if w.dtype != "bf16":
-            ap.error("--pass train needs a bf16 workload")
         run_gpu_train(args, w)
     else:
         run_gpu(args, w)

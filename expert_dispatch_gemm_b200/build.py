@@ -22,7 +22,8 @@ LIB = os.path.join(PKG, "libmoe.so")
 INCLUDE = os.path.join(ROOT, "include")
 
 SOURCES = ["api.cu", "router.cu", "assign.cu", "dispatch_combine.cu", "ffn_f32.cu",
-           "gemm_tc.cu", "gemm_swap.cu", "route_noalloc.cu", "gemm_bwd.cu", "bwd.cu"]
+           "gemm_tc.cu", "gemm_swap.cu", "route_noalloc.cu", "gemm_bwd.cu", "bwd.cu",
+           "bwd_f32.cu"]
 PROBE_SOURCES = ["probe.cu"]
 PROBE_LIB = os.path.join(PKG, "libmoe_probe.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -622,22 +622,23 @@ struct BwdLayout {
 static BwdLayout bwd_layout(const moe_config* c, const Derived& d) {
   BwdLayout b{};
   const bool swiglu = c->act == MOE_ACT_SWIGLU;
+  const size_t elt = c->dtype == MOE_BF16 ? 2 : 4;
   size_t off = 0;
   b.err = off;
   off += MOE_WS_ERROR_BYTES;
   off = align_up(off, 1024);
   b.dy = off;
-  off = align_up(off + (size_t)d.rows_routed * c->d * 2, 1024);
+  off = align_up(off + (size_t)d.rows_routed * c->d * elt, 1024);
   b.u = off;
-  off = align_up(off + (size_t)d.rows * c->h * 2, 1024);
+  off = align_up(off + (size_t)d.rows * c->h * elt, 1024);
   b.v = off;
-  if (swiglu) off = align_up(off + (size_t)d.rows * c->h * 2, 1024);
+  if (swiglu) off = align_up(off + (size_t)d.rows * c->h * elt, 1024);
   b.hh = off;
-  off = align_up(off + (size_t)d.rows * c->h * 2, 1024);
+  off = align_up(off + (size_t)d.rows * c->h * elt, 1024);
   b.duv = off;
-  off = align_up(off + (size_t)d.rows * c->h * (swiglu ? 4 : 2), 1024);
+  off = align_up(off + (size_t)d.rows * c->h * elt * (swiglu ? 2 : 1), 1024);
   b.dxp = off;
-  off = align_up(off + (size_t)d.rows * c->d * 2, 1024);
+  off = align_up(off + (size_t)d.rows * c->d * elt, 1024);
   b.dl = off;
   off = align_up(off + (size_t)c->n * c->E * 4, 1024);
   b.wgt = off;
@@ -656,7 +657,6 @@ moe_status moe_backward_workspace_size(const moe_config* cfg, size_t* bytes, int
   Derived d;
   moe_status st = derive(cfg, &d);
   if (st != MOE_OK) return st;
-  if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   const BwdLayout b = bwd_layout(cfg, d);
   if (bytes) *bytes = b.end;
   if (launches) *launches = b.launches;
@@ -673,10 +673,10 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float*
   Derived d;
   moe_status st = derive(cfg, &d);
   if (st != MOE_OK) return st;
-  if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
-  // the weight-gradient epilogue writes 32-row groups that never straddle
-  // the W1 / W3 boundary (h) or the end of the output (d, h or 2h)
-  if (cfg->d % 64 != 0 || cfg->h % 64 != 0) return MOE_ERR_UNSUPPORTED;
+  const bool bf16 = cfg->dtype == MOE_BF16;
+  // the bf16 weight-gradient epilogue writes 32-row groups that never
+  // straddle the W1 / W3 boundary (h) or the end of the output (d, h or 2h)
+  if (bf16 && (cfg->d % 64 != 0 || cfg->h % 64 != 0)) return MOE_ERR_UNSUPPORTED;
   const bool swiglu = cfg->act == MOE_ACT_SWIGLU;
   const bool tc = cfg->mode == MOE_TOKEN_CHOICE;
   if (!X || !Wg || !W1 || !W2 || !dout || !dX || !dWg || !dW1 || !dW2) return MOE_ERR_INVALID_ARG;
@@ -712,11 +712,13 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float*
 
   // 1. padding rows of the dispatched inputs and output gradients read as
   //    zeros by the weight-gradient reductions
-  MOE_CU(launch_pad_zero(route->offsets, route->counts, E, D, xp, dy, s));
+  const int elt = bf16 ? 2 : 4;
+  MOE_CU(launch_pad_zero(route->offsets, route->counts, E, D * elt, xp, dy, s));
   // 2. output gradient per kept row, gate gradients, logit gradients
   CombineBwdArgs cb{};
+  cb.bf16 = bf16;
   cb.Y_perm = yp;
-  cb.dout = static_cast<const __nv_bfloat16*>(dout);
+  cb.dout = dout;
   cb.tok_row = route->tok_row;
   cb.tok_gate = route->tok_gate;
   cb.idx = route->idx;
@@ -740,6 +742,117 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float*
   cb.dL = dl;
   MOE_CU(launch_combine_backward(cb, s));
 
+  if (!bf16) {
+    // fp32: the five grouped GEMMs on FFMA
+    auto fp = [](const void* p) { return static_cast<const float*>(p); };
+    auto fm = [](void* p) { return static_cast<float*>(p); };
+    BwdF32Args f{};
+    f.offsets = route->offsets;
+    f.counts = route->counts;
+    f.E = E;
+    f.n_shared = ns;
+    f.n = n;
+    f.n_pad = d.n_pad;
+    f.rows_routed = d.rows_routed;
+    f.shared_base = d.shared_base;
+    f.act = cfg->act;
+    f.swiglu = swiglu;
+    const long long hcols = swiglu ? 2LL * h : h;
+    float* Uf = reinterpret_cast<float*>(U);
+    float* Vf = reinterpret_cast<float*>(V);
+    float* Hf = reinterpret_cast<float*>(H);
+    float* duvf = reinterpret_cast<float*>(duv);
+    float* dyf = reinterpret_cast<float*>(dy);
+    float* dxpf = reinterpret_cast<float*>(dxp);
+    float* xpf = reinterpret_cast<float*>(xp);
+    // SAVE: U (V), H
+    BwdF32Args q = f;
+    q.N = h;
+    q.K = D;
+    q.A = xpf;
+    q.lda = D;
+    q.A_sh = fp(X);
+    q.B = fp(W1);
+    q.B3 = fp(W3);
+    q.sB = fp(sW1);
+    q.sB3 = fp(sW3);
+    q.b_expert_stride = (long long)h * D;
+    q.out0 = Uf;
+    q.out1 = Vf;
+    q.out2 = Hf;
+    q.ld_out = h;
+    MOE_CU(run_bwd_f32(BW_SAVE, q, s));
+    // DACT: dU (dV) = (dY W2) * act'
+    q = f;
+    q.N = h;
+    q.K = D;
+    q.A = dyf;
+    q.lda = D;
+    q.A_sh = fp(dout);
+    q.B = fp(W2);
+    q.sB = fp(sW2);
+    q.b_expert_stride = (long long)D * h;
+    q.in0 = Uf;
+    q.in1 = Vf;
+    q.ld_in = h;
+    q.out0 = duvf;
+    q.ld_out = hcols;
+    MOE_CU(run_bwd_f32(BW_DACT, q, s));
+    // DX: dX_perm = dU W1 (+ dV W3)
+    q = f;
+    q.N = D;
+    q.K = (int)hcols;
+    q.k_split = h;
+    q.A = duvf;
+    q.lda = hcols;
+    q.A_sh = duvf;
+    q.a_sh_base = d.shared_base;
+    q.a_sh_stride = d.n_pad;
+    q.B = fp(W1);
+    q.B3 = fp(W3);
+    q.sB = fp(sW1);
+    q.sB3 = fp(sW3);
+    q.b_expert_stride = (long long)h * D;
+    q.out0 = dxpf;
+    q.ld_out = D;
+    MOE_CU(run_bwd_f32(BW_DX, q, s));
+    // WG2: dW2_e = dY_e^T H_e
+    q = f;
+    q.M = D;
+    q.m_split = D;
+    q.N = h;
+    q.WA = dyf;
+    q.ld_wa = D;
+    q.WA_sh = fp(dout);
+    q.WB = Hf;
+    q.ld_wb = h;
+    q.WB_sh = Hf;
+    q.wb_sh_base = d.shared_base;
+    q.wb_sh_stride = d.n_pad;
+    q.w_out0 = q.w_out1 = fm(dW2);
+    q.sw_out0 = q.sw_out1 = ns > 0 ? fm(dsW2) : fm(dW2);
+    q.w_expert_stride = (long long)D * h;
+    MOE_CU(run_bwd_f32(BW_WG2, q, s));
+    // WG13: [dW1_e; dW3_e] = [dU_e | dV_e]^T X_e
+    q = f;
+    q.M = (int)hcols;
+    q.m_split = h;
+    q.N = D;
+    q.WA = duvf;
+    q.ld_wa = hcols;
+    q.WA_sh = duvf;
+    q.wa_sh_base = d.shared_base;
+    q.wa_sh_stride = d.n_pad;
+    q.WB = xpf;
+    q.ld_wb = D;
+    q.WB_sh = fp(X);
+    q.w_out0 = fm(dW1);
+    q.w_out1 = swiglu ? fm(dW3) : fm(dW1);
+    q.sw_out0 = ns > 0 ? fm(dsW1) : fm(dW1);
+    q.sw_out1 = ns > 0 && swiglu ? fm(dsW3) : q.sw_out0;
+    q.w_expert_stride = (long long)h * D;
+    MOE_CU(run_bwd_f32(BW_WG13, q, s));
+  } else {
   BwdParams base{};
   base.offsets = route->offsets;
   base.counts = route->counts;
@@ -887,9 +1000,11 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float*
     p.sw_out1 = ns > 0 && swiglu ? bf(dsW3) : p.sw_out0;
     MOE_CU(run_bwd_gemm(BW_WG13, wpair, m, p, s));
   }
+  }
   // 8, 9. router: dX = dL Wg^T + the token's dispatched rows; dWg = X^T dL
   RouterBwdArgs rb{};
-  rb.X = static_cast<const __nv_bfloat16*>(X);
+  rb.bf16 = bf16;
+  rb.X = X;
   rb.Wg = Wg;
   rb.WgT = at<float>(ws, b.wgt);
   rb.dL = dl;
@@ -902,7 +1017,7 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float*
   rb.n_shared = ns;
   rb.shared_base = d.shared_base;
   rb.n_pad = d.n_pad;
-  rb.dX = static_cast<__nv_bfloat16*>(dX);
+  rb.dX = dX;
   rb.dWg = dWg;
   rb.partial = at<float>(ws, b.part);
   rb.splits = b.splits;

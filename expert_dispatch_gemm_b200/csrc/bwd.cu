@@ -22,6 +22,72 @@ namespace {
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// 16 bytes of T as floats (bf16: 8, fp32: 4)
+template <typename T>
+struct V16;
+template <>
+struct V16<__nv_bfloat16> {
+  static constexpr int W = 8;
+  __device__ static void unpack(const uint4 x, float* f) {
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = bf_lo(w[i]);
+      f[2 * i + 1] = bf_hi(w[i]);
+    }
+  }
+  __device__ static uint4 pack(const float* f) {
+    return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                      pack_bf16x2(f[6], f[7]));
+  }
+};
+template <>
+struct V16<float> {
+  static constexpr int W = 4;
+  __device__ static void unpack(const uint4 x, float* f) {
+    f[0] = __uint_as_float(x.x);
+    f[1] = __uint_as_float(x.y);
+    f[2] = __uint_as_float(x.z);
+    f[3] = __uint_as_float(x.w);
+  }
+  __device__ static uint4 pack(const float* f) {
+    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                      __float_as_uint(f[3]));
+  }
+};
+
+// four consecutive elements (8 bytes of bf16, 16 of fp32)
+__device__ __forceinline__ void load4(const __nv_bfloat16* p, float* f) {
+  const uint2 x = *reinterpret_cast<const uint2*>(p);
+  f[0] = bf_lo(x.x);
+  f[1] = bf_hi(x.x);
+  f[2] = bf_lo(x.y);
+  f[3] = bf_hi(x.y);
+}
+__device__ __forceinline__ void load4(const float* p, float* f) {
+  const float4 x = *reinterpret_cast<const float4*>(p);
+  f[0] = x.x;
+  f[1] = x.y;
+  f[2] = x.z;
+  f[3] = x.w;
+}
+__device__ __forceinline__ void store4(__nv_bfloat16* p, const float* f) {
+  *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]));
+}
+__device__ __forceinline__ void store4(float* p, const float* f) {
+  *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
+}
+__device__ __forceinline__ void load2(const __nv_bfloat16* p, float& lo, float& hi) {
+  const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
+  lo = bf_lo(w);
+  hi = bf_hi(w);
+}
+__device__ __forceinline__ void load2(const float* p, float& lo, float& hi) {
+  const float2 w = *reinterpret_cast<const float2*>(p);
+  lo = w.x;
+  hi = w.y;
+}
+
 // sum over the block (256 threads); every thread gets the total
 __device__ __forceinline__ float block_sum256(float v, float* red) {
 #pragma unroll
@@ -43,6 +109,7 @@ __device__ __forceinline__ float block_sum256(float v, float* red) {
 // choice: dS[t, e] = dgate), the balance-loss term lb E f_e / n
 // (f_e = load_e / (n K)), the score's backward and the z-loss term
 // 2 z lse_t / n softmax(l_t).
+template <typename T>
 __global__ void __launch_bounds__(256) combine_backward_kernel(CombineBwdArgs a) {
   pdl_wait();
   __shared__ int rows_s[MOE_MAX_EXPERTS];
@@ -64,7 +131,8 @@ __global__ void __launch_bounds__(256) combine_backward_kernel(CombineBwdArgs a)
   }
   __syncthreads();
   const int cnt = cnt_s;
-  const int nvec = a.d / 8;
+  constexpr int W = V16<T>::W;
+  const int nvec = a.d / W;
   const uint4* go = reinterpret_cast<const uint4*>(a.dout) + (size_t)t * nvec;
   for (int j = 0; j < cnt; ++j) {
     const long long r = rows_s[j];
@@ -73,19 +141,15 @@ __global__ void __launch_bounds__(256) combine_backward_kernel(CombineBwdArgs a)
     uint4* dy = reinterpret_cast<uint4*>(a.dY_perm) + (size_t)r * nvec;
     float part = 0.0f;
     for (int v = tid; v < nvec; v += 256) {
-      const uint4 o = __ldg(go + v);
-      const uint4 yy = __ldg(y + v);
-      const uint32_t ow[4] = {o.x, o.y, o.z, o.w};
-      const uint32_t yw[4] = {yy.x, yy.y, yy.z, yy.w};
-      uint32_t res[4];
+      float o[W], yy[W], res[W];
+      V16<T>::unpack(__ldg(go + v), o);
+      V16<T>::unpack(__ldg(y + v), yy);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float o0 = bf_lo(ow[i]), o1 = bf_hi(ow[i]);
-        part = fmaf(o0, bf_lo(yw[i]), part);
-        part = fmaf(o1, bf_hi(yw[i]), part);
-        res[i] = pack_bf16x2(g * o0, g * o1);
+      for (int i = 0; i < W; ++i) {
+        part = fmaf(o[i], yy[i], part);
+        res[i] = g * o[i];
       }
-      dy[v] = make_uint4(res[0], res[1], res[2], res[3]);
+      dy[v] = V16<T>::pack(res);
     }
     const float dot = block_sum256(part, red);
     if (tid == 0) dots_s[j] = dot;
@@ -150,15 +214,15 @@ __global__ void __launch_bounds__(256) combine_backward_kernel(CombineBwdArgs a)
   }
 }
 
-// zero rows [offsets[e] + counts[e], offsets[e+1]) of two [rows, d] buffers
+// zero rows [offsets[e] + counts[e], offsets[e+1]) of two [rows, row_bytes] buffers
 __global__ void __launch_bounds__(256) pad_zero_kernel(const int32_t* offsets,
-                                                       const int32_t* counts, int d,
-                                                       __nv_bfloat16* a, __nv_bfloat16* b) {
+                                                       const int32_t* counts, int row_bytes,
+                                                       void* a, void* b) {
   pdl_wait();
   const int e = blockIdx.x;
   const int beg = offsets[e], end = offsets[e + 1];
   const int first = beg + max(0, min(counts[e], end - beg));
-  const int nvec = d / 8;
+  const int nvec = row_bytes / 16;
   const long long total = (long long)(end - first) * nvec;
   const uint4 z = make_uint4(0, 0, 0, 0);
   for (long long q = threadIdx.x; q < total; q += 256) {
@@ -194,6 +258,7 @@ __global__ void __launch_bounds__(256) transpose_wg_kernel(const float* Wg, int 
 // holds tokens 8ty..8ty+7 and columns 4tx..4tx+3, so each expert step takes
 // three 16-byte shared-memory loads for 32 FMAs.
 constexpr int kRxBM = 64, kRxBN = 128, kRxEC = 32;
+template <typename T>
 __global__ void __launch_bounds__(256) router_dx_kernel(RouterBwdArgs a) {
   pdl_wait();
   __shared__ __align__(16) float dls[kRxEC][kRxBM + 4];  // transposed: [expert][token]
@@ -240,14 +305,12 @@ __global__ void __launch_bounds__(256) router_dx_kernel(RouterBwdArgs a) {
     const int t = t0 + 8 * ty + k;
     if (t >= a.n) continue;
     float v[4] = {acc[k][0], acc[k][1], acc[k][2], acc[k][3]};
-    auto add = [&](const uint2 x) {
-      v[0] += bf_lo(x.x);
-      v[1] += bf_hi(x.x);
-      v[2] += bf_lo(x.y);
-      v[3] += bf_hi(x.y);
-    };
-    auto at_row = [&](long long row) {
-      return *reinterpret_cast<const uint2*>(a.dX_perm + (size_t)row * a.d + col);
+    const T* xp = static_cast<const T*>(a.dX_perm);
+    auto add = [&](const float* x) {
+      v[0] += x[0];
+      v[1] += x[1];
+      v[2] += x[2];
+      v[3] += x[3];
     };
     // the token's rows four at a time, so that four independent loads are in
     // flight (sums stay in slot order)
@@ -256,19 +319,22 @@ __global__ void __launch_bounds__(256) router_dx_kernel(RouterBwdArgs a) {
       int r[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) r[u] = j + u < a.slots ? tr[j + u] : -1;
-      uint2 x[4];
+      float x[4][4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) x[u] = r[u] >= 0 ? at_row(r[u]) : make_uint2(0, 0);
+      for (int u = 0; u < 4; ++u) {
+        if (r[u] >= 0) load4(xp + (size_t)r[u] * a.d + col, x[u]);
+      }
 #pragma unroll
       for (int u = 0; u < 4; ++u)
         if (r[u] >= 0) add(x[u]);
       if (r[3] < 0) break;
     }
-    for (int sidx = 0; sidx < a.n_shared; ++sidx) add(at_row(a.shared_base + sidx * a.n_pad + t));
-    uint2 o;
-    o.x = pack_bf16x2(v[0], v[1]);
-    o.y = pack_bf16x2(v[2], v[3]);
-    *reinterpret_cast<uint2*>(a.dX + (size_t)t * a.d + col) = o;
+    for (int sidx = 0; sidx < a.n_shared; ++sidx) {
+      float x[4];
+      load4(xp + (size_t)(a.shared_base + sidx * a.n_pad + t) * a.d + col, x);
+      add(x);
+    }
+    store4(static_cast<T*>(a.dX) + (size_t)t * a.d + col, v);
   }
 }
 
@@ -277,6 +343,7 @@ __global__ void __launch_bounds__(256) router_dx_kernel(RouterBwdArgs a) {
 // 4te..4te+3. blockIdx.z = a contiguous slice of the tokens; slices are
 // added in slice order by router_dwg_reduce_kernel.
 constexpr int kRwBM = 128, kRwBN = 64, kRwBT = 32;
+template <typename T>
 __global__ void __launch_bounds__(256) router_dwg_kernel(RouterBwdArgs a, int per_split) {
   pdl_wait();
   __shared__ __align__(16) float xs[kRwBT][kRwBM];
@@ -296,11 +363,7 @@ __global__ void __launch_bounds__(256) router_dwg_kernel(RouterBwdArgs a, int pe
       const int r = q / (kRwBM / 2), c = 2 * (q % (kRwBM / 2));
       const int t = c0 + r, i = i0 + c;
       float lo = 0.0f, hi = 0.0f;
-      if (t < tend && i < a.d) {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(a.X + (size_t)t * a.d + i);
-        lo = bf_lo(w);
-        hi = bf_hi(w);
-      }
+      if (t < tend && i < a.d) load2(static_cast<const T*>(a.X) + (size_t)t * a.d + i, lo, hi);
       xs[r][c] = lo;
       xs[r][c + 1] = hi;
     }
@@ -349,12 +412,13 @@ __global__ void __launch_bounds__(256) router_dwg_reduce_kernel(const float* par
 }  // namespace
 
 cudaError_t launch_combine_backward(const CombineBwdArgs& a, cudaStream_t s) {
-  return launch_pdl(combine_backward_kernel, a.n, 256, 0, s, a);
+  if (a.bf16) return launch_pdl(combine_backward_kernel<__nv_bfloat16>, a.n, 256, 0, s, a);
+  return launch_pdl(combine_backward_kernel<float>, a.n, 256, 0, s, a);
 }
 
-cudaError_t launch_pad_zero(const int32_t* offsets, const int32_t* counts, int E, int d,
-                            __nv_bfloat16* a, __nv_bfloat16* b, cudaStream_t s) {
-  return launch_pdl(pad_zero_kernel, E, 256, 0, s, offsets, counts, d, a, b);
+cudaError_t launch_pad_zero(const int32_t* offsets, const int32_t* counts, int E, int row_bytes,
+                            void* a, void* b, cudaStream_t s) {
+  return launch_pdl(pad_zero_kernel, E, 256, 0, s, offsets, counts, row_bytes, a, b);
 }
 
 // token slices of the router-weight gradient: enough CTAs for two waves,
@@ -372,11 +436,13 @@ cudaError_t launch_router_backward(const RouterBwdArgs& a, cudaStream_t s) {
   cudaError_t e = launch_pdl(transpose_wg_kernel, gt, 256, 0, s, a.Wg, a.d, a.E, a.WgT);
   if (e != cudaSuccess) return e;
   const dim3 gx(ceil_div(a.n, kRxBM), ceil_div(a.d, kRxBN));
-  e = launch_pdl(router_dx_kernel, gx, 256, 0, s, a);
+  e = a.bf16 ? launch_pdl(router_dx_kernel<__nv_bfloat16>, gx, 256, 0, s, a)
+             : launch_pdl(router_dx_kernel<float>, gx, 256, 0, s, a);
   if (e != cudaSuccess) return e;
   const int per = ceil_div(ceil_div(a.n, a.splits), kRwBT) * kRwBT;
   const dim3 gw(ceil_div(a.d, kRwBM), ceil_div(a.E, kRwBN), a.splits);
-  e = launch_pdl(router_dwg_kernel, gw, 256, 0, s, a, per);
+  e = a.bf16 ? launch_pdl(router_dwg_kernel<__nv_bfloat16>, gw, 256, 0, s, a, per)
+             : launch_pdl(router_dwg_kernel<float>, gw, 256, 0, s, a, per);
   if (e != cudaSuccess || a.splits <= 1) return e;
   const long long count = (long long)a.d * a.E;
   return launch_pdl(router_dwg_reduce_kernel, ceil_div(count, 256), 256, 0, s,

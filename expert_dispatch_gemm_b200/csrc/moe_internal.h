@@ -244,10 +244,41 @@ struct BwdMaps {
 cudaError_t run_bwd_gemm(int mode, bool pair, const BwdMaps& m, const BwdParams& p,
                          cudaStream_t s);
 
-// element-wise and FFMA kernels of the backward (bwd.cu)
+// fp32 grouped GEMMs of the backward on FFMA (bwd_f32.cu), same modes
+struct BwdF32Args {
+  const int32_t* offsets;
+  const int32_t* counts;
+  int E, n_shared, n, n_pad;
+  long long rows_routed, shared_base;
+  int act, swiglu;
+  // row modes: C[rows, N] over K
+  int N, K, k_split;
+  const float* A;                     // routed A rows, row pitch lda
+  long long lda;
+  const float* A_sh;                  // shared A rows: A_sh + (a_sh_base + s * a_sh_stride + i) * lda
+  long long a_sh_base, a_sh_stride;
+  const float *B, *B3, *sB, *sB3;     // weights; SAVE: [.., N, K]; DACT/DX: [.., K, N]
+  long long b_expert_stride;
+  float *out0, *out1, *out2;
+  long long ld_out;
+  const float *in0, *in1;
+  long long ld_in;
+  // weight modes: per expert C[M, N] = sum over its rows k of A(m, k) B(n, k),
+  // A(m, k) = WA[(row0 + k) * ld_wa + m], B(n, k) = WB[(row0 + k) * ld_wb + n]
+  int M, m_split;
+  const float *WA, *WA_sh, *WB, *WB_sh;
+  long long ld_wa, ld_wb, wa_sh_base, wa_sh_stride, wb_sh_base, wb_sh_stride;
+  float *w_out0, *w_out1, *sw_out0, *sw_out1;
+  long long w_expert_stride;
+};
+cudaError_t run_bwd_f32(int mode, const BwdF32Args& a, cudaStream_t s);
+
+// element-wise and FFMA kernels of the backward (bwd.cu); activations,
+// expert outputs and their gradients are bf16 or fp32 (bf16 = 1)
 struct CombineBwdArgs {
-  const __nv_bfloat16* Y_perm;   // [rows, d] the forward's expert outputs
-  const __nv_bfloat16* dout;     // [n, d]
+  int bf16;
+  const void* Y_perm;            // [rows, d] the forward's expert outputs
+  const void* dout;              // [n, d]
   const int32_t* tok_row;        // [n, slots]
   const float* tok_gate;         // [n, slots]
   const int32_t* idx;            // TC [n, K]
@@ -259,22 +290,24 @@ struct CombineBwdArgs {
   const float* lse;              // [n] or NULL
   int n, d, E, slots, tc, K, score, weights;
   float lb_coef, z_coef;
-  __nv_bfloat16* dY_perm;        // [rows, d]: kept rows written
+  void* dY_perm;                 // [rows, d]: kept rows written
   float* dL;                     // [n, E]
 };
 cudaError_t launch_combine_backward(const CombineBwdArgs& a, cudaStream_t s);
-cudaError_t launch_pad_zero(const int32_t* offsets, const int32_t* counts, int E, int d,
-                            __nv_bfloat16* a, __nv_bfloat16* b, cudaStream_t s);
+// zero rows [offsets[e] + counts[e], offsets[e+1]) of two [rows, row_bytes] buffers
+cudaError_t launch_pad_zero(const int32_t* offsets, const int32_t* counts, int E, int row_bytes,
+                            void* a, void* b, cudaStream_t s);
 struct RouterBwdArgs {
-  const __nv_bfloat16* X;        // [n, d]
+  int bf16;
+  const void* X;                 // [n, d]
   const float* Wg;               // [d, E]
   float* WgT;                    // [E, d] workspace: W_g transposed
   const float* dL;               // [n, E]
-  const __nv_bfloat16* dX_perm;  // [rows, d]
+  const void* dX_perm;           // [rows, d]
   const int32_t* tok_row;        // [n, slots]
   int n, d, E, slots, n_shared;
   long long shared_base, n_pad;
-  __nv_bfloat16* dX;             // [n, d]
+  void* dX;                      // [n, d]
   float* dWg;                    // [d, E]
   float* partial;                // [splits, d, E]
   int splits;

@@ -360,7 +360,9 @@ MOE_API moe_status moe_expert_ffn_combined(const moe_config* cfg, const void* X,
  *             itself as dY over all n tokens;
  *   router:   dWg = X^T dL (fp32); dX = dL Wg^T + the sum of dX_perm over
  *             the token's kept rows and shared rows (fp32, stored bf16).
- * bf16 configs only (MOE_ERR_UNSUPPORTED otherwise). */
+ * bf16 configs run the grouped GEMMs on the tcgen05 tensor cores (d and h
+ * multiples of 64); fp32 configs run them on FFMA and store every value in
+ * fp32 (no rounding to bf16 anywhere). */
 
 /* Backward workspace bytes and the kernels moe_layer_backward enqueues. */
 MOE_API moe_status moe_backward_workspace_size(const moe_config* cfg, size_t* bytes,
@@ -372,9 +374,10 @@ MOE_API moe_status moe_backward_workspace_size(const moe_config* cfg, size_t* by
  * has z_coef != 0); fwd_ws, the workspace of that moe_layer_forward call,
  * untouched since: its dispatched rows and expert outputs are read, and the
  * padding rows of its dispatched rows are overwritten with zeros; dout [n,d]
- * bf16. Outputs (device, caller-owned, every element written): dX [n,d]
- * bf16, dWg [d,E] fp32, dW1, dW3 [E,h,d] and dW2 [E,d,h] bf16 (dW3 only for
- * SwiGLU), dsW1, dsW3, dsW2 likewise for shared experts; dL [n,E] fp32, the
+ * (the config's dtype). Outputs (device, caller-owned, every element
+ * written): dX [n,d] of the config's dtype, dWg [d,E] fp32, dW1, dW3 [E,h,d]
+ * and dW2 [E,d,h] of the config's dtype (dW3 only for SwiGLU), dsW1, dsW3,
+ * dsW2 likewise for shared experts; dL [n,E] fp32, the
  * logits' gradient, may be NULL. ws: moe_backward_workspace_size bytes,
  * 256-byte aligned, error word zeroed once by moe_workspace_init; bounded
  * waits report through it (moe_read_error). X, dout, dX, the weights and

@@ -204,22 +204,22 @@ def test_backward_workspace_and_launches():
     """The backward enqueues the padding clear, the combine backward, five
     grouped GEMMs, the W_g transpose, the router's input gradient and its
     weight gradient (plus the ordered reduce of the weight gradient's token
-    slices when there is more than one). fp32 layers have no backward."""
-    for w in (wl.EC_BF16, wl.TC_TOP2_CAP, wl.TC_DROPLESS, wl.TC_SIGMOID_GROUPED, wl.DECODE):
+    slices when there is more than one), for bf16 and fp32 layers alike."""
+    for w in (wl.EC_FP32, wl.EC_BF16, wl.TC_TOP2_CAP, wl.TC_DROPLESS, wl.TC_SIGMOID_GROUPED,
+              wl.DECODE):
         st, nbytes, launches = _bwd_size(moe.config(w))
         assert st == moe.MOE_OK, w.name
         sw = w.act == "swiglu"
         sz = moe.sizes(moe.config(w))
+        elt = 4 if w.dtype == "f32" else 2
         # at least dY, U, (V), H, dU(,dV) and dX_perm over the dispatched rows
-        assert nbytes >= sz.rows * (w.d * 2 + w.h * (8 if sw else 4)), w.name
+        assert nbytes >= sz.rows * elt * (w.d + w.h * (4 if sw else 2)), w.name
         assert launches in (10, 11), w.name
-    st, _, _ = _bwd_size(moe.config(wl.EC_FP32))
-    assert st == moe.MOE_ERR_UNSUPPORTED
 
 
 def test_backward_rejects_bad_arguments_before_launching():
-    """Host-side validation: null required pointers and an fp32 config fail
-    without touching the (null) device pointers."""
+    """Host-side validation: null required pointers fail without touching
+    the (null) device pointers, for bf16 and fp32 configs."""
     cfg = moe.config(wl.TC_DROPLESS.replace(n=256, d=128, E=8, h=128))
     L = moe.lib()
     route = moe.MoeRouteOut()
@@ -229,4 +229,4 @@ def test_backward_rejects_bad_arguments_before_launching():
     cfg32 = moe.config(wl.EC_FP32)
     st = L.moe_layer_backward(ctypes.byref(cfg32), *([None] * 8), ctypes.byref(route), None, 0,
                               *([None] * 10), None, 0, None)
-    assert st == moe.MOE_ERR_UNSUPPORTED
+    assert st == moe.MOE_ERR_INVALID_ARG
