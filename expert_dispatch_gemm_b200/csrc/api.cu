@@ -974,6 +974,10 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float*
     p.w_out0 = bf(dW2);
     p.w_out1 = bf(dW2);
     p.sw_out0 = p.sw_out1 = ns > 0 ? bf(dsW2) : bf(dW2);
+    if (!map(&m.o0, dW2, (long long)E * D, h, 32)) return MOE_ERR_UNSUPPORTED;
+    m.o1 = m.o2 = m.o3 = m.o0;
+    if (ns > 0 && !map(&m.o2, dsW2, (long long)ns * D, h, 32)) return MOE_ERR_UNSUPPORTED;
+    m.o3 = m.o2;
     MOE_CU(run_bwd_gemm(BW_WG2, wpair, m, p, s));
   }
   // 7. WG13: [dW1_e; dW3_e] = [dU_e | dV_e]^T X_e
@@ -998,6 +1002,14 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float*
     p.w_out1 = swiglu ? bf(dW3) : bf(dW1);
     p.sw_out0 = ns > 0 ? bf(dsW1) : bf(dW1);
     p.sw_out1 = ns > 0 && swiglu ? bf(dsW3) : p.sw_out0;
+    if (!map(&m.o0, dW1, (long long)E * h, D, 32)) return MOE_ERR_UNSUPPORTED;
+    m.o1 = m.o2 = m.o3 = m.o0;
+    if (swiglu && !map(&m.o1, dW3, (long long)E * h, D, 32)) return MOE_ERR_UNSUPPORTED;
+    if (ns > 0) {
+      if (!map(&m.o2, dsW1, (long long)ns * h, D, 32)) return MOE_ERR_UNSUPPORTED;
+      m.o3 = m.o2;
+      if (swiglu && !map(&m.o3, dsW3, (long long)ns * h, D, 32)) return MOE_ERR_UNSUPPORTED;
+    }
     MOE_CU(run_bwd_gemm(BW_WG13, wpair, m, p, s));
   }
   }

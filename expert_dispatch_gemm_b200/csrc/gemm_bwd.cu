@@ -64,7 +64,7 @@ constexpr int kWStagesMax = 6;
 // staging blocks.
 template <bool PAIR, bool WG>
 struct Ring {
-  static constexpr int stages = PAIR ? (WG ? 5 : 6) : (WG ? 3 : 4);
+  static constexpr int stages = PAIR ? (WG ? 4 : 6) : (WG ? 3 : 4);
   static constexpr int b_bytes = (PAIR ? kWBN / 2 : kWBN) * kWBK * 2;
   static constexpr int stage_bytes = kWABytes + b_bytes;
 };
@@ -83,7 +83,8 @@ struct BwdState {
 };
 
 constexpr int kStateBytes = (sizeof(BwdState) + 127) / 128 * 128;
-constexpr int kWStageOut = 8 * 32 * 128;  // weight-gradient epilogue staging, per warp 32 x 128 B
+// weight-gradient epilogue staging: per warp two 32 x 128-byte blocks
+constexpr int kWStageOut = 8 * 2 * 32 * 128;
 
 template <bool CLUSTER_ACQUIRE>
 __device__ __forceinline__ bool bwait(uint64_t* bar, uint32_t parity, BwdState* st, int* err,
@@ -361,17 +362,22 @@ __device__ __forceinline__ __nv_bfloat16* wgrad_row(const BwdParams& p, const BT
 }
 
 template <int MODE, bool PAIR>
+// tmO0..tmO3: weight-gradient outputs for TMA stores (routed rows below /
+// above m_split, shared rows below / above), boxes of 64 columns x 32 rows
 __device__ __forceinline__ void bwd_body(const CUtensorMap* tmA0, const CUtensorMap* tmA1,
                                          const CUtensorMap* tmB0, const CUtensorMap* tmB0g,
                                          const CUtensorMap* tmB1, const CUtensorMap* tmB1g,
+                                         const CUtensorMap* tmO0, const CUtensorMap* tmO1,
+                                         const CUtensorMap* tmO2, const CUtensorMap* tmO3,
                                          const BwdParams& p, unsigned char* base) {
   using Tr = ModeTraits<MODE>;
   using R = Ring<PAIR, Tr::WGRAD>;
   unsigned char* sA = base;
   unsigned char* sB = base + R::stages * kWABytes;
   BwdState* st = reinterpret_cast<BwdState*>(base + R::stages * R::stage_bytes);
-  // weight-gradient epilogue staging: [8 warps][32 rows][128 bytes]
-  unsigned char* wstage = base + R::stages * R::stage_bytes + kStateBytes;
+  // weight-gradient epilogue staging: [8 warps][2][32 rows][128 bytes],
+  // 1024-byte aligned like a 128-byte-swizzled TMA box
+  unsigned char* wstage = base + R::stages * R::stage_bytes + (kStateBytes + 1023) / 1024 * 1024;
   const uint32_t rank = PAIR ? sm100::cluster_ctarank() : 0u;
   const bool leader = rank == 0;
 
@@ -587,6 +593,7 @@ __device__ __forceinline__ void bwd_body(const CUtensorMap* tmA0, const CUtensor
     const int half = (warp - 2) >> 2;
     const int row_in_tile = q * 32 + lane;
     int used = 0;
+    int sbuf = 0;  // weight gradients: the staging block to fill next
     for (int tile = first; tile < total; tile += stride) {
       const BTile t = decode<MODE, PAIR>(tile, p, st, routed, rank);
       if (Tr::WGRAD && t.skip) {
@@ -607,17 +614,29 @@ __device__ __forceinline__ void bwd_body(const CUtensorMap* tmA0, const CUtensor
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kWBN);
       if (Tr::WGRAD) {
         // 64 columns at a time: each thread packs its row's 128 bytes into
-        // the warp's staging block (16-byte pieces XOR-swizzled by row, so
-        // eight consecutive lanes hit eight different bank groups), then the
-        // warp writes the block out four whole 128-byte rows per store
-        unsigned char* stg = wstage + (warp - 2) * (32 * 128);
+        // one of the warp's two staging blocks in the 128-byte-swizzled
+        // layout (16-byte piece j of row r at piece j ^ (r % 8)), and lane 0
+        // stores the block with one TMA copy; the block is rewritten only
+        // once that copy has finished reading it
+        const int grp = t.m0 + q * 32;  // the warp's 32 rows never straddle m_split or m_total
+        const bool hi = grp >= p.m_split;
+        const CUtensorMap* om = t.shared ? (hi ? tmO3 : tmO2) : (hi ? tmO1 : tmO0);
+        const int orow = t.expert * (hi ? p.m_total - p.m_split : p.m_split) +
+                         (hi ? grp - p.m_split : grp);
+        // rows past the end (an output of fewer rows than the tile) store
+        // nothing, so every staging block that is written is also stored
+        // and the two blocks strictly alternate between committed copies
 #pragma unroll 1
-        for (int cc = half * (kWBN / 2); cc < (half + 1) * (kWBN / 2); cc += 64) {
+        for (int cc = half * (kWBN / 2); cc < (half + 1) * (kWBN / 2) && grp < p.m_total;
+             cc += 64) {
           if (t.n0 + cc >= p.ld_w) break;
           uint32_t v[32], w[32];
           sm100::tmem_ld_32x32b_x32(tbase + cc, v);
           sm100::tmem_ld_32x32b_x32(tbase + cc + 32, w);
           sm100::tmem_ld_wait();
+          unsigned char* stg = wstage + ((warp - 2) * 2 + sbuf) * (32 * 128);
+          if (lane == 0) sm100::bulk_wait_read_1();
+          __syncwarp();
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const uint32_t* src = j < 4 ? v + 8 * j : w + 8 * (j - 4);
@@ -628,21 +647,13 @@ __device__ __forceinline__ void bwd_body(const CUtensorMap* tmA0, const CUtensor
                 pack_bf16x2(__uint_as_float(src[6]), __uint_as_float(src[7])));
             *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) * 16)) = pk;
           }
+          sm100::fence_proxy_async_smem();
           __syncwarp();
-          // the warp's 32 rows lie on one side of m_split and of m_total
-          // (both multiples of 64), so one base pointer serves them all
-          __nv_bfloat16* gbase = wgrad_row(p, t, t.m0 + q * 32);
-          if (gbase) {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const int idx = lane + 32 * k, r = idx >> 3, pc = idx & 7;
-              const int col = t.n0 + cc + 8 * pc;
-              if (col < p.ld_w)
-                *reinterpret_cast<uint4*>(gbase + (size_t)r * p.ld_w + col) =
-                    *reinterpret_cast<const uint4*>(stg + r * 128 + ((pc ^ (r & 7)) * 16));
-            }
+          if (lane == 0) {
+            sm100::tma_store_2d(om, t.n0 + cc, orow, stg);
+            sm100::bulk_commit_group();
           }
-          __syncwarp();
+          sbuf ^= 1;
         }
       } else if (t.valid) {
         row_epilogue<MODE>(p, t, tbase, row_in_tile, half);
@@ -651,6 +662,8 @@ __device__ __forceinline__ void bwd_body(const CUtensorMap* tmA0, const CUtensor
       if (PAIR) sm100::mbar_arrive_cluster(sm100::mapa_shared(sm100::smem_addr(&st->tempty[acc]), 0));
       else sm100::mbar_arrive(&st->tempty[acc]);
     }
+    // the weight gradients' TMA stores complete before the CTA exits
+    if (Tr::WGRAD && lane == 0) sm100::bulk_wait_all();
   }
   sm100::tc_fence_before();
   __syncthreads();
@@ -674,9 +687,14 @@ __global__ void __launch_bounds__(kWThreads, 1)
                        const __grid_constant__ CUtensorMap tmB0,
                        const __grid_constant__ CUtensorMap tmB0g,
                        const __grid_constant__ CUtensorMap tmB1,
-                       const __grid_constant__ CUtensorMap tmB1g, const BwdParams p) {
+                       const __grid_constant__ CUtensorMap tmB1g,
+                       const __grid_constant__ CUtensorMap tmO0,
+                       const __grid_constant__ CUtensorMap tmO1,
+                       const __grid_constant__ CUtensorMap tmO2,
+                       const __grid_constant__ CUtensorMap tmO3, const BwdParams p) {
   extern __shared__ __align__(1024) unsigned char bsm[];
-  bwd_body<MODE, false>(&tmA0, &tmA1, &tmB0, &tmB0g, &tmB1, &tmB1g, p, aligned_smem(bsm));
+  bwd_body<MODE, false>(&tmA0, &tmA1, &tmB0, &tmB0g, &tmB1, &tmB1g, &tmO0, &tmO1, &tmO2, &tmO3,
+                        p, aligned_smem(bsm));
 }
 
 // CTA pairs (cta_group::2): each CTA loads its 128 rows of A and one half
@@ -690,9 +708,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kWThreads, 1)
                             const __grid_constant__ CUtensorMap tmB0,
                             const __grid_constant__ CUtensorMap tmB0g,
                             const __grid_constant__ CUtensorMap tmB1,
-                            const __grid_constant__ CUtensorMap tmB1g, const BwdParams p) {
+                            const __grid_constant__ CUtensorMap tmB1g,
+                            const __grid_constant__ CUtensorMap tmO0,
+                            const __grid_constant__ CUtensorMap tmO1,
+                            const __grid_constant__ CUtensorMap tmO2,
+                            const __grid_constant__ CUtensorMap tmO3, const BwdParams p) {
   extern __shared__ __align__(1024) unsigned char bsm[];
-  bwd_body<MODE, true>(&tmA0, &tmA1, &tmB0, &tmB0g, &tmB1, &tmB1g, p, aligned_smem(bsm));
+  bwd_body<MODE, true>(&tmA0, &tmA1, &tmB0, &tmB0g, &tmB1, &tmB1g, &tmO0, &tmO1, &tmO2, &tmO3,
+                       p, aligned_smem(bsm));
 }
 
 }  // namespace
@@ -703,7 +726,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kWThreads, 1)
 template <int MODE, bool PAIR>
 static cudaError_t launch_bwd(const BwdMaps& m, const BwdParams& p, cudaStream_t s) {
   using R = Ring<PAIR, ModeTraits<MODE>::WGRAD>;
-  const size_t bytes = (size_t)R::stages * R::stage_bytes + kStateBytes +
+  const size_t bytes = (size_t)R::stages * R::stage_bytes + (kStateBytes + 1023) / 1024 * 1024 +
                        (ModeTraits<MODE>::WGRAD ? kWStageOut : 0) + 1024;
   auto kern = PAIR ? tc_bwd_gemm_pair_kernel<MODE> : tc_bwd_gemm_kernel<MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
@@ -722,7 +745,8 @@ static cudaError_t launch_bwd(const BwdMaps& m, const BwdParams& p, cudaStream_t
   const long long slots = PAIR ? sms / 2 : sms;
   const long long units = tiles < slots ? (tiles < 1 ? 1 : tiles) : slots;
   const int grid = (int)(PAIR ? 2 * units : units);
-  return launch_pdl(kern, grid, kWThreads, bytes, s, m.a0, m.a1, m.b0, m.b0g, m.b1, m.b1g, p);
+  return launch_pdl(kern, grid, kWThreads, bytes, s, m.a0, m.a1, m.b0, m.b0g, m.b1, m.b1g, m.o0,
+                    m.o1, m.o2, m.o3, p);
 }
 
 template <bool PAIR>

@@ -238,6 +238,7 @@ struct BwdParams {
 };
 struct BwdMaps {
   CUtensorMap a0, a1, b0, b0g, b1, b1g;
+  CUtensorMap o0, o1, o2, o3;  // weight-gradient outputs (TMA stores), boxes 64 x 32
 };
 // pair: CTA pairs (cta_group::2, 256-row tiles); weight modes then take
 // mt_tiles in 256-row blocks
