@@ -246,6 +246,19 @@ __device__ __forceinline__ void row_epilogue(const BwdParams& p, const BTile& t,
   for (int cc = half * (ncols / 2); cc < (half + 1) * (ncols / 2); cc += 32) {
     const int col = t.n0 + cc;
     if (col >= p.n_total) break;
+    // DACT: the stored U (and V) of this row's 32 columns, loaded before the
+    // accumulator so the two latencies overlap
+    uint4 ur[4], vr[4];
+    if (MODE == BW_DACT) {
+      const uint4* pu = reinterpret_cast<const uint4*>(p.in0 + row * p.ld_in + col);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) ur[j] = pu[j];
+      if (p.swiglu) {
+        const uint4* pv = reinterpret_cast<const uint4*>(p.in1 + row * p.ld_in + col);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) vr[j] = pv[j];
+      }
+    }
     uint32_t v[32];
     sm100::tmem_ld_32x32b_x32(tbase + cc, v);
     float f[32], g[32];
@@ -290,11 +303,10 @@ __device__ __forceinline__ void row_epilogue(const BwdParams& p, const BTile& t,
       }
     } else if (MODE == BW_DACT) {
       // f = dH; the stored U (and V) of the same row and columns
-      const uint4* pu = reinterpret_cast<const uint4*>(p.in0 + row * p.ld_in + col);
       float u[32], vv[32];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const uint4 x = pu[j];
+        const uint4 x = ur[j];
         const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -303,10 +315,9 @@ __device__ __forceinline__ void row_epilogue(const BwdParams& p, const BTile& t,
         }
       }
       if (p.swiglu) {
-        const uint4* pv = reinterpret_cast<const uint4*>(p.in1 + row * p.ld_in + col);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const uint4 x = pv[j];
+          const uint4 x = vr[j];
           const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
           for (int k = 0; k < 4; ++k) {

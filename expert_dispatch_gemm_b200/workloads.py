@@ -100,7 +100,17 @@ SMALL = [
                                "swiglu128", n=300, d=256, E=64, h=128, bias_steps=3),
 ]
 
-BY_NAME = {w.name: w for w in FULL + SMALL + [DECODE]}
+# Reduced versions of two token-choice layers (same d and h; a quarter of the
+# batch, or an eighth of the batch and of the experts) for ncu captures that
+# replay every launch: a few GB on the device at most
+PROFILE = [
+    TC_DROPLESS.replace(name="tc-softmax-top8of64-dropless-n4096-d2048-swiglu1024", n=4096),
+    TC_SIGMOID_GROUPED.replace(
+        name="tc-sigmoid-grouped8keep4-top8of32-shared1-n1024-d7168-swiglu2048", n=1024, E=32,
+        bias_steps=0),
+]
+
+BY_NAME = {w.name: w for w in FULL + SMALL + [DECODE] + PROFILE}
 
 
 def _gen(device, seed: int, stream: int) -> torch.Generator:
