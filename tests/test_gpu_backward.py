@@ -40,6 +40,10 @@ BWD_SMALL = wl.SMALL + [
                            h=128),
     # expert choice, GELU, the capacity of several 128-row blocks per expert
     wl.EC_BF16.replace(name="bwd-ec-gelu-n768-d128-e8-c4-h256", n=768, d=128, E=8, h=256, c=4.0),
+    # the decoding regime: 16 tokens over 64 grouped sigmoid experts plus a
+    # shared expert of fewer than 128 rows
+    wl.TC_SIGMOID_GROUPED.replace(name="bwd-decode-n16-top8of64-shared1-d256-h128", n=16, d=256,
+                                  E=64, h=128, bias_steps=0),
 ]
 
 
