@@ -653,206 +653,157 @@ static BwdLayout bwd_layout(const moe_config* c, const Derived& d) {
   return b;
 }
 
-moe_status moe_backward_workspace_size(const moe_config* cfg, size_t* bytes, int* launches) {
-  Derived d;
-  moe_status st = derive(cfg, &d);
-  if (st != MOE_OK) return st;
-  const BwdLayout b = bwd_layout(cfg, d);
-  if (bytes) *bytes = b.end;
-  if (launches) *launches = b.launches;
+// The buffers of one backward call (device, the config's dtype).
+struct BwdBufs {
+  void *xp, *dy, *U, *V, *H, *duv, *dxp;
+};
+
+// The five grouped GEMMs of an fp32 layer, on FFMA.
+// (err: the FFMA kernels wait on nothing, so they report no error)
+static moe_status bwd_gemms_f32(const moe_config* cfg, const Derived& d, const BwdBufs& B,
+                                const void* X, const void* W1, const void* W3, const void* W2,
+                                const void* sW1, const void* sW3, const void* sW2,
+                                const moe_route_out* route, const void* dout, void* dW1,
+                                void* dW3, void* dW2, void* dsW1, void* dsW3, void* dsW2,
+                                int* /*err*/, cudaStream_t s) {
+  const bool swiglu = cfg->act == MOE_ACT_SWIGLU;
+  const int n = cfg->n, D = cfg->d, h = cfg->h, E = cfg->E, ns = cfg->n_shared;
+  void* xp = B.xp;
+  void* dy = B.dy;
+  void* U = B.U;
+  void* V = B.V;
+  void* H = B.H;
+  void* duv = B.duv;
+  void* dxp = B.dxp;
+  auto fp = [](const void* p) { return static_cast<const float*>(p); };
+  auto fm = [](void* p) { return static_cast<float*>(p); };
+  BwdF32Args f{};
+  f.offsets = route->offsets;
+  f.counts = route->counts;
+  f.E = E;
+  f.n_shared = ns;
+  f.n = n;
+  f.n_pad = d.n_pad;
+  f.rows_routed = d.rows_routed;
+  f.shared_base = d.shared_base;
+  f.act = cfg->act;
+  f.swiglu = swiglu;
+  const long long hcols = swiglu ? 2LL * h : h;
+  float* Uf = static_cast<float*>(U);
+  float* Vf = static_cast<float*>(V);
+  float* Hf = static_cast<float*>(H);
+  float* duvf = static_cast<float*>(duv);
+  float* dyf = static_cast<float*>(dy);
+  float* dxpf = static_cast<float*>(dxp);
+  float* xpf = static_cast<float*>(xp);
+  // SAVE: U (V), H
+  BwdF32Args q = f;
+  q.N = h;
+  q.K = D;
+  q.A = xpf;
+  q.lda = D;
+  q.A_sh = fp(X);
+  q.B = fp(W1);
+  q.B3 = fp(W3);
+  q.sB = fp(sW1);
+  q.sB3 = fp(sW3);
+  q.b_expert_stride = (long long)h * D;
+  q.out0 = Uf;
+  q.out1 = Vf;
+  q.out2 = Hf;
+  q.ld_out = h;
+  MOE_CU(run_bwd_f32(BW_SAVE, q, s));
+  // DACT: dU (dV) = (dY W2) * act'
+  q = f;
+  q.N = h;
+  q.K = D;
+  q.A = dyf;
+  q.lda = D;
+  q.A_sh = fp(dout);
+  q.B = fp(W2);
+  q.sB = fp(sW2);
+  q.b_expert_stride = (long long)D * h;
+  q.in0 = Uf;
+  q.in1 = Vf;
+  q.ld_in = h;
+  q.out0 = duvf;
+  q.ld_out = hcols;
+  MOE_CU(run_bwd_f32(BW_DACT, q, s));
+  // DX: dX_perm = dU W1 (+ dV W3)
+  q = f;
+  q.N = D;
+  q.K = (int)hcols;
+  q.k_split = h;
+  q.A = duvf;
+  q.lda = hcols;
+  q.A_sh = duvf;
+  q.a_sh_base = d.shared_base;
+  q.a_sh_stride = d.n_pad;
+  q.B = fp(W1);
+  q.B3 = fp(W3);
+  q.sB = fp(sW1);
+  q.sB3 = fp(sW3);
+  q.b_expert_stride = (long long)h * D;
+  q.out0 = dxpf;
+  q.ld_out = D;
+  MOE_CU(run_bwd_f32(BW_DX, q, s));
+  // WG2: dW2_e = dY_e^T H_e
+  q = f;
+  q.M = D;
+  q.m_split = D;
+  q.N = h;
+  q.WA = dyf;
+  q.ld_wa = D;
+  q.WA_sh = fp(dout);
+  q.WB = Hf;
+  q.ld_wb = h;
+  q.WB_sh = Hf;
+  q.wb_sh_base = d.shared_base;
+  q.wb_sh_stride = d.n_pad;
+  q.w_out0 = q.w_out1 = fm(dW2);
+  q.sw_out0 = q.sw_out1 = ns > 0 ? fm(dsW2) : fm(dW2);
+  q.w_expert_stride = (long long)D * h;
+  MOE_CU(run_bwd_f32(BW_WG2, q, s));
+  // WG13: [dW1_e; dW3_e] = [dU_e | dV_e]^T X_e
+  q = f;
+  q.M = (int)hcols;
+  q.m_split = h;
+  q.N = D;
+  q.WA = duvf;
+  q.ld_wa = hcols;
+  q.WA_sh = duvf;
+  q.wa_sh_base = d.shared_base;
+  q.wa_sh_stride = d.n_pad;
+  q.WB = xpf;
+  q.ld_wb = D;
+  q.WB_sh = fp(X);
+  q.w_out0 = fm(dW1);
+  q.w_out1 = swiglu ? fm(dW3) : fm(dW1);
+  q.sw_out0 = ns > 0 ? fm(dsW1) : fm(dW1);
+  q.sw_out1 = ns > 0 && swiglu ? fm(dsW3) : q.sw_out0;
+  q.w_expert_stride = (long long)h * D;
+  MOE_CU(run_bwd_f32(BW_WG13, q, s));
   return MOE_OK;
 }
 
-moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float* Wg,
-                              const void* W1, const void* W3, const void* W2, const void* sW1,
-                              const void* sW3, const void* sW2, const moe_route_out* route,
-                              void* fwd_ws, size_t fwd_ws_bytes, const void* dout, void* dX,
-                              float* dWg, void* dW1, void* dW3, void* dW2, void* dsW1,
-                              void* dsW3, void* dsW2, float* dL, void* ws, size_t ws_bytes,
-                              moe_stream_t stream) {
-  Derived d;
-  moe_status st = derive(cfg, &d);
-  if (st != MOE_OK) return st;
-  const bool bf16 = cfg->dtype == MOE_BF16;
-  // the bf16 weight-gradient epilogue writes 32-row groups that never
-  // straddle the W1 / W3 boundary (h) or the end of the output (d, h or 2h)
-  if (bf16 && (cfg->d % 64 != 0 || cfg->h % 64 != 0)) return MOE_ERR_UNSUPPORTED;
+// The five grouped GEMMs of a bf16 layer, on the tcgen05 tensor cores.
+static moe_status bwd_gemms_bf16(const moe_config* cfg, const Derived& d, const BwdBufs& B,
+                                 const void* X, const void* W1, const void* W3, const void* W2,
+                                 const void* sW1, const void* sW3, const void* sW2,
+                                 const moe_route_out* route, const void* dout, void* dW1,
+                                 void* dW3, void* dW2, void* dsW1, void* dsW3, void* dsW2,
+                                 int* err, cudaStream_t s) {
   const bool swiglu = cfg->act == MOE_ACT_SWIGLU;
-  const bool tc = cfg->mode == MOE_TOKEN_CHOICE;
-  if (!X || !Wg || !W1 || !W2 || !dout || !dX || !dWg || !dW1 || !dW2) return MOE_ERR_INVALID_ARG;
-  if (swiglu && (!W3 || !dW3)) return MOE_ERR_INVALID_ARG;
-  if (cfg->n_shared > 0 && (!sW1 || !sW2 || !dsW1 || !dsW2 || (swiglu && (!sW3 || !dsW3))))
-    return MOE_ERR_INVALID_ARG;
-  if ((st = check_route_out(cfg, route)) != MOE_OK) return st;
-  const bool need_logits = (tc && cfg->z_coef != 0.0f) || cfg->score == MOE_SCORE_SQRTSOFTPLUS;
-  if (need_logits && (!route->logits || (tc && cfg->z_coef != 0.0f && !route->lse)))
-    return MOE_ERR_INVALID_ARG;
-  const WsLayout fw = ws_layout(cfg, d);
-  if ((st = check_ws(fwd_ws, fwd_ws_bytes, fw.layer_end)) != MOE_OK) return st;
-  const BwdLayout b = bwd_layout(cfg, d);
-  if ((st = check_ws(ws, ws_bytes, b.end)) != MOE_OK) return st;
-  const void* aligned[] = {X, dout, dX, fwd_ws, W1, W2, dW1, dW2, W3, dW3,
-                           sW1, sW2, sW3, dsW1, dsW2, dsW3};
-  for (const void* ptr : aligned)
-    if (reinterpret_cast<uintptr_t>(ptr) & 15) return MOE_ERR_INVALID_ARG;
-  cudaStream_t s = (cudaStream_t)stream;
-  auto bf = [](const void* p) { return static_cast<__nv_bfloat16*>(const_cast<void*>(p)); };
-  __nv_bfloat16* xp = at<__nv_bfloat16>(fwd_ws, fw.xperm);
-  const __nv_bfloat16* yp = at<__nv_bfloat16>(fwd_ws, fw.yperm);
-  __nv_bfloat16* dy = at<__nv_bfloat16>(ws, b.dy);
-  __nv_bfloat16* U = at<__nv_bfloat16>(ws, b.u);
-  __nv_bfloat16* V = swiglu ? at<__nv_bfloat16>(ws, b.v) : nullptr;
-  __nv_bfloat16* H = at<__nv_bfloat16>(ws, b.hh);
-  __nv_bfloat16* duv = at<__nv_bfloat16>(ws, b.duv);
-  __nv_bfloat16* dxp = at<__nv_bfloat16>(ws, b.dxp);
-  float* dl = dL ? dL : at<float>(ws, b.dl);
-  int* err = at<int>(ws, b.err);
   const int n = cfg->n, D = cfg->d, h = cfg->h, E = cfg->E, ns = cfg->n_shared;
   const long long rows = d.rows;
-
-  // 1. padding rows of the dispatched inputs and output gradients read as
-  //    zeros by the weight-gradient reductions
-  const int elt = bf16 ? 2 : 4;
-  MOE_CU(launch_pad_zero(route->offsets, route->counts, E, D * elt, xp, dy, s));
-  // 2. output gradient per kept row, gate gradients, logit gradients
-  CombineBwdArgs cb{};
-  cb.bf16 = bf16;
-  cb.Y_perm = yp;
-  cb.dout = dout;
-  cb.tok_row = route->tok_row;
-  cb.tok_gate = route->tok_gate;
-  cb.idx = route->idx;
-  cb.drop = route->drop;
-  cb.offsets = route->offsets;
-  cb.load = route->load;
-  cb.scores = route->scores;
-  cb.logits = route->logits;
-  cb.lse = route->lse;
-  cb.n = n;
-  cb.d = D;
-  cb.E = E;
-  cb.slots = d.slots;
-  cb.tc = tc;
-  cb.K = tc ? d.k : 0;
-  cb.score = cfg->score;
-  cb.weights = cfg->weights;
-  cb.lb_coef = tc ? cfg->lb_coef : 0.0f;
-  cb.z_coef = tc ? cfg->z_coef : 0.0f;
-  cb.dY_perm = dy;
-  cb.dL = dl;
-  MOE_CU(launch_combine_backward(cb, s));
-
-  if (!bf16) {
-    // fp32: the five grouped GEMMs on FFMA
-    auto fp = [](const void* p) { return static_cast<const float*>(p); };
-    auto fm = [](void* p) { return static_cast<float*>(p); };
-    BwdF32Args f{};
-    f.offsets = route->offsets;
-    f.counts = route->counts;
-    f.E = E;
-    f.n_shared = ns;
-    f.n = n;
-    f.n_pad = d.n_pad;
-    f.rows_routed = d.rows_routed;
-    f.shared_base = d.shared_base;
-    f.act = cfg->act;
-    f.swiglu = swiglu;
-    const long long hcols = swiglu ? 2LL * h : h;
-    float* Uf = reinterpret_cast<float*>(U);
-    float* Vf = reinterpret_cast<float*>(V);
-    float* Hf = reinterpret_cast<float*>(H);
-    float* duvf = reinterpret_cast<float*>(duv);
-    float* dyf = reinterpret_cast<float*>(dy);
-    float* dxpf = reinterpret_cast<float*>(dxp);
-    float* xpf = reinterpret_cast<float*>(xp);
-    // SAVE: U (V), H
-    BwdF32Args q = f;
-    q.N = h;
-    q.K = D;
-    q.A = xpf;
-    q.lda = D;
-    q.A_sh = fp(X);
-    q.B = fp(W1);
-    q.B3 = fp(W3);
-    q.sB = fp(sW1);
-    q.sB3 = fp(sW3);
-    q.b_expert_stride = (long long)h * D;
-    q.out0 = Uf;
-    q.out1 = Vf;
-    q.out2 = Hf;
-    q.ld_out = h;
-    MOE_CU(run_bwd_f32(BW_SAVE, q, s));
-    // DACT: dU (dV) = (dY W2) * act'
-    q = f;
-    q.N = h;
-    q.K = D;
-    q.A = dyf;
-    q.lda = D;
-    q.A_sh = fp(dout);
-    q.B = fp(W2);
-    q.sB = fp(sW2);
-    q.b_expert_stride = (long long)D * h;
-    q.in0 = Uf;
-    q.in1 = Vf;
-    q.ld_in = h;
-    q.out0 = duvf;
-    q.ld_out = hcols;
-    MOE_CU(run_bwd_f32(BW_DACT, q, s));
-    // DX: dX_perm = dU W1 (+ dV W3)
-    q = f;
-    q.N = D;
-    q.K = (int)hcols;
-    q.k_split = h;
-    q.A = duvf;
-    q.lda = hcols;
-    q.A_sh = duvf;
-    q.a_sh_base = d.shared_base;
-    q.a_sh_stride = d.n_pad;
-    q.B = fp(W1);
-    q.B3 = fp(W3);
-    q.sB = fp(sW1);
-    q.sB3 = fp(sW3);
-    q.b_expert_stride = (long long)h * D;
-    q.out0 = dxpf;
-    q.ld_out = D;
-    MOE_CU(run_bwd_f32(BW_DX, q, s));
-    // WG2: dW2_e = dY_e^T H_e
-    q = f;
-    q.M = D;
-    q.m_split = D;
-    q.N = h;
-    q.WA = dyf;
-    q.ld_wa = D;
-    q.WA_sh = fp(dout);
-    q.WB = Hf;
-    q.ld_wb = h;
-    q.WB_sh = Hf;
-    q.wb_sh_base = d.shared_base;
-    q.wb_sh_stride = d.n_pad;
-    q.w_out0 = q.w_out1 = fm(dW2);
-    q.sw_out0 = q.sw_out1 = ns > 0 ? fm(dsW2) : fm(dW2);
-    q.w_expert_stride = (long long)D * h;
-    MOE_CU(run_bwd_f32(BW_WG2, q, s));
-    // WG13: [dW1_e; dW3_e] = [dU_e | dV_e]^T X_e
-    q = f;
-    q.M = (int)hcols;
-    q.m_split = h;
-    q.N = D;
-    q.WA = duvf;
-    q.ld_wa = hcols;
-    q.WA_sh = duvf;
-    q.wa_sh_base = d.shared_base;
-    q.wa_sh_stride = d.n_pad;
-    q.WB = xpf;
-    q.ld_wb = D;
-    q.WB_sh = fp(X);
-    q.w_out0 = fm(dW1);
-    q.w_out1 = swiglu ? fm(dW3) : fm(dW1);
-    q.sw_out0 = ns > 0 ? fm(dsW1) : fm(dW1);
-    q.sw_out1 = ns > 0 && swiglu ? fm(dsW3) : q.sw_out0;
-    q.w_expert_stride = (long long)h * D;
-    MOE_CU(run_bwd_f32(BW_WG13, q, s));
-  } else {
+  __nv_bfloat16* xp = static_cast<__nv_bfloat16*>(B.xp);
+  __nv_bfloat16* dy = static_cast<__nv_bfloat16*>(B.dy);
+  __nv_bfloat16* U = static_cast<__nv_bfloat16*>(B.U);
+  __nv_bfloat16* V = static_cast<__nv_bfloat16*>(B.V);
+  __nv_bfloat16* H = static_cast<__nv_bfloat16*>(B.H);
+  __nv_bfloat16* duv = static_cast<__nv_bfloat16*>(B.duv);
+  __nv_bfloat16* dxp = static_cast<__nv_bfloat16*>(B.dxp);
+  auto bf = [](const void* p) { return static_cast<__nv_bfloat16*>(const_cast<void*>(p)); };
   BwdParams base{};
   base.offsets = route->offsets;
   base.counts = route->counts;
@@ -1012,7 +963,101 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float*
     }
     MOE_CU(run_bwd_gemm(BW_WG13, wpair, m, p, s));
   }
-  }
+  return MOE_OK;
+}
+
+moe_status moe_backward_workspace_size(const moe_config* cfg, size_t* bytes, int* launches) {
+  Derived d;
+  moe_status st = derive(cfg, &d);
+  if (st != MOE_OK) return st;
+  const BwdLayout b = bwd_layout(cfg, d);
+  if (bytes) *bytes = b.end;
+  if (launches) *launches = b.launches;
+  return MOE_OK;
+}
+
+moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float* Wg,
+                              const void* W1, const void* W3, const void* W2, const void* sW1,
+                              const void* sW3, const void* sW2, const moe_route_out* route,
+                              void* fwd_ws, size_t fwd_ws_bytes, const void* dout, void* dX,
+                              float* dWg, void* dW1, void* dW3, void* dW2, void* dsW1,
+                              void* dsW3, void* dsW2, float* dL, void* ws, size_t ws_bytes,
+                              moe_stream_t stream) {
+  Derived d;
+  moe_status st = derive(cfg, &d);
+  if (st != MOE_OK) return st;
+  const bool bf16 = cfg->dtype == MOE_BF16;
+  // the bf16 weight-gradient epilogue writes 32-row groups that never
+  // straddle the W1 / W3 boundary (h) or the end of the output (d, h or 2h)
+  if (bf16 && (cfg->d % 64 != 0 || cfg->h % 64 != 0)) return MOE_ERR_UNSUPPORTED;
+  const bool swiglu = cfg->act == MOE_ACT_SWIGLU;
+  const bool tc = cfg->mode == MOE_TOKEN_CHOICE;
+  if (!X || !Wg || !W1 || !W2 || !dout || !dX || !dWg || !dW1 || !dW2) return MOE_ERR_INVALID_ARG;
+  if (swiglu && (!W3 || !dW3)) return MOE_ERR_INVALID_ARG;
+  if (cfg->n_shared > 0 && (!sW1 || !sW2 || !dsW1 || !dsW2 || (swiglu && (!sW3 || !dsW3))))
+    return MOE_ERR_INVALID_ARG;
+  if ((st = check_route_out(cfg, route)) != MOE_OK) return st;
+  const bool need_logits = (tc && cfg->z_coef != 0.0f) || cfg->score == MOE_SCORE_SQRTSOFTPLUS;
+  if (need_logits && (!route->logits || (tc && cfg->z_coef != 0.0f && !route->lse)))
+    return MOE_ERR_INVALID_ARG;
+  const WsLayout fw = ws_layout(cfg, d);
+  if ((st = check_ws(fwd_ws, fwd_ws_bytes, fw.layer_end)) != MOE_OK) return st;
+  const BwdLayout b = bwd_layout(cfg, d);
+  if ((st = check_ws(ws, ws_bytes, b.end)) != MOE_OK) return st;
+  const void* aligned[] = {X, dout, dX, fwd_ws, W1, W2, dW1, dW2, W3, dW3,
+                           sW1, sW2, sW3, dsW1, dsW2, dsW3};
+  for (const void* ptr : aligned)
+    if (reinterpret_cast<uintptr_t>(ptr) & 15) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  __nv_bfloat16* xp = at<__nv_bfloat16>(fwd_ws, fw.xperm);
+  const __nv_bfloat16* yp = at<__nv_bfloat16>(fwd_ws, fw.yperm);
+  __nv_bfloat16* dy = at<__nv_bfloat16>(ws, b.dy);
+  __nv_bfloat16* U = at<__nv_bfloat16>(ws, b.u);
+  __nv_bfloat16* V = swiglu ? at<__nv_bfloat16>(ws, b.v) : nullptr;
+  __nv_bfloat16* H = at<__nv_bfloat16>(ws, b.hh);
+  __nv_bfloat16* duv = at<__nv_bfloat16>(ws, b.duv);
+  __nv_bfloat16* dxp = at<__nv_bfloat16>(ws, b.dxp);
+  float* dl = dL ? dL : at<float>(ws, b.dl);
+  int* err = at<int>(ws, b.err);
+  const int n = cfg->n, D = cfg->d, E = cfg->E, ns = cfg->n_shared;
+
+  // 1. padding rows of the dispatched inputs and output gradients read as
+  //    zeros by the weight-gradient reductions
+  const int elt = bf16 ? 2 : 4;
+  MOE_CU(launch_pad_zero(route->offsets, route->counts, E, D * elt, xp, dy, s));
+  // 2. output gradient per kept row, gate gradients, logit gradients
+  CombineBwdArgs cb{};
+  cb.bf16 = bf16;
+  cb.Y_perm = yp;
+  cb.dout = dout;
+  cb.tok_row = route->tok_row;
+  cb.tok_gate = route->tok_gate;
+  cb.idx = route->idx;
+  cb.drop = route->drop;
+  cb.offsets = route->offsets;
+  cb.load = route->load;
+  cb.scores = route->scores;
+  cb.logits = route->logits;
+  cb.lse = route->lse;
+  cb.n = n;
+  cb.d = D;
+  cb.E = E;
+  cb.slots = d.slots;
+  cb.tc = tc;
+  cb.K = tc ? d.k : 0;
+  cb.score = cfg->score;
+  cb.weights = cfg->weights;
+  cb.lb_coef = tc ? cfg->lb_coef : 0.0f;
+  cb.z_coef = tc ? cfg->z_coef : 0.0f;
+  cb.dY_perm = dy;
+  cb.dL = dl;
+  MOE_CU(launch_combine_backward(cb, s));
+
+  const BwdBufs bufs{xp, dy, U, V, H, duv, dxp};
+  if ((st = (bf16 ? bwd_gemms_bf16 : bwd_gemms_f32)(cfg, d, bufs, X, W1, W3, W2, sW1, sW3, sW2,
+                                                     route, dout, dW1, dW3, dW2, dsW1, dsW3,
+                                                     dsW2, err, s)) != MOE_OK)
+    return st;
   // 8, 9. router: dX = dL Wg^T + the token's dispatched rows; dWg = X^T dL
   RouterBwdArgs rb{};
   rb.bf16 = bf16;
