@@ -14,7 +14,7 @@ timed with CUDA events on the launching stream.
 Default workload: the expert-choice layer of the pages' worked example
 (4,096 tokens, d 1024, 64 experts, c = 2, GELU FFN 1024 -> 4096 -> 1024, bf16).
 
-Multi-GPU: the layer does not shard in this build ("replicas only"): each
+Multi-GPU: the layer does not shard ("replicas only"): each
 rank runs an independent replica, no collective touches the data path, and
 the timed region is the max over ranks.
 

@@ -73,7 +73,7 @@ typedef struct CUstream_st* moe_stream_t;
 typedef enum {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = 1, /* a null required pointer, a bad size or mode */
-  MOE_ERR_UNSUPPORTED = 2, /* a valid shape this build has no kernel for */
+  MOE_ERR_UNSUPPORTED = 2, /* a valid shape the library has no kernel for */
   MOE_ERR_WORKSPACE = 3,   /* workspace null or smaller than required */
   MOE_ERR_CUDA = 4,        /* a CUDA call or launch failed */
   MOE_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up */

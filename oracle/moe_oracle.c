@@ -321,8 +321,8 @@ void orc_ec_histogram(int n, int E, int k, const int32_t* I, int32_t* hist) {
 /* backward pass: the gradient of the forward above by the chain rule.   */
 /* [TC-vs-EC] "What each direction guarantees" names the training-time  */
 /* losses (load balance 0.01, router z-loss 0.001) whose gradients join  */
-/* the task gradient here. Storage points mirror the forward: values the */
-/* GPU stores are rounded to `store` where it stores them.               */
+/* the gradient of <dout, out> here. Storage points mirror the forward:  */
+/* values the GPU stores are rounded to `store` where it stores them.    */
 /* ------------------------------------------------------------------ */
 static double sigm(double u) { return 1.0 / (1.0 + exp(-u)); }
 
