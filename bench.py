@@ -21,9 +21,9 @@ the timed region is the max over ranks.
 --impl reference times the CPU oracle as it stands (single thread) on the
 same workload, one bounded sample per step.
 
---pass train times forward + backward (moe_layer_forward then
-moe_layer_backward: gradients of X, W_g and every expert weight) per step,
-with the backward's grouped-GEMM FLOPs against the tensor-core peak.
+--pass train times forward + backward (moe_layer_forward_train then
+moe_layer_backward_train: gradients of X, W_g and every expert weight) per
+step, with the backward's grouped-GEMM FLOPs against the tensor-core peak.
 """
 from __future__ import annotations
 
@@ -489,13 +489,18 @@ METRIC_TRAIN = ("MoE-layer fwd+bwd tokens/s on 1 B200 (gradients of X, W_g and e
 
 
 def backward_flops(w: wl.Workload, rows_gathered: int) -> dict:
-    """FLOPs of the backward's five grouped GEMMs and of the router's two
-    FFMA contractions, over the kept rows (and the shared experts' n rows)."""
+    """FLOPs of the backward's grouped GEMMs and of the router's two FFMA
+    contractions, over the kept rows (and the shared experts' n rows). bf16
+    layers keep U, V and H from the training forward, so their backward runs
+    four GEMMs; fp32 layers recompute the up projection."""
     g = 2 if w.act == "swiglu" else 1  # up projections per expert
     rows = rows_gathered + w.n_shared * w.n
     unit = 2.0 * rows * w.d * w.h
-    return {"recompute": unit * g, "dact": unit, "dx": unit * g, "dw2": unit, "dw13": unit * g,
-            "router": 4.0 * w.n * w.d * w.E}
+    out = {"dact": unit, "dx": unit * g, "dw2": unit, "dw13": unit * g,
+           "router": 4.0 * w.n * w.d * w.E}
+    if w.dtype == "f32":
+        out["recompute"] = unit * g
+    return out
 
 
 def run_gpu_train(args, w: wl.Workload):
@@ -520,10 +525,12 @@ def run_gpu_train(args, w: wl.Workload):
     layer.grads()
 
     def step(X=None, d=None, ev=None):
-        layer.forward(X=X, stream=stream)
+        """The training pair: the forward keeps U, V and H for the backward
+        (bf16 layers; fp32 layers recompute them)."""
+        layer.forward_train(X=X, stream=stream)
         if ev is not None:
             ev.record(stream)
-        layer.backward(dout if d is None else d, X=X, stream=stream)
+        layer.backward_train(dout if d is None else d, X=X, stream=stream)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -599,7 +606,7 @@ def run_gpu_train(args, w: wl.Workload):
                 "peak_kind": "sustained (sw_power_cap active)" if (capped and tc_sust)
                 else "burst"}
     roof.update({"traffic": None, "peak_source": src,
-                 "kernel": "moe_layer_backward as a whole: the five grouped GEMMs' FLOPs over "
+                 "kernel": "moe_layer_backward_train as a whole: its grouped GEMMs' FLOPs over "
                            "the whole call (its non-GEMM kernels included in the time)",
                  "algorithmic_per_launch": gemm_flops})
     fwd_launches = sum(moe.launch_counts(layer.cfg).values())

@@ -298,7 +298,8 @@ static moe_status ffn_impl(const moe_config* c, const Derived& dv, const void* X
                            const void* W2, const void* sW1,
                            const void* sW3, const void* sW2, void* H, void* Y, int* err,
                            cudaStream_t s, const float* row_gate = nullptr,
-                           float* out32 = nullptr) {
+                           float* out32 = nullptr, void* save_u = nullptr,
+                           void* save_v = nullptr) {
   if (!offsets || !W1 || !W2 || !H || (!Y && !out32)) return MOE_ERR_INVALID_ARG;
   if (!X_perm && (!X || !row_token)) return MOE_ERR_INVALID_ARG;
   if (c->act == MOE_ACT_SWIGLU && !W3) return MOE_ERR_INVALID_ARG;
@@ -334,6 +335,8 @@ static moe_status ffn_impl(const moe_config* c, const Derived& dv, const void* X
   f.pair = ffn_uses_pair(c, dv);
   f.row_gate = row_gate;
   f.out32 = out32;
+  f.save_u = save_u;
+  f.save_v = save_v;
   if (c->dtype != MOE_BF16) return out32 ? MOE_ERR_UNSUPPORTED : run_ffn_f32(f, s);
   if (!out32 && ffn_uses_swap(c, dv) && swap_down_supported(f)) {
     f.skip_down = true;
@@ -656,6 +659,7 @@ static BwdLayout bwd_layout(const moe_config* c, const Derived& d) {
 // The buffers of one backward call (device, the config's dtype).
 struct BwdBufs {
   void *xp, *dy, *U, *V, *H, *duv, *dxp;
+  bool saved;  // U, V and H were kept by moe_layer_forward_train (bf16)
 };
 
 // The five grouped GEMMs of an fp32 layer, on FFMA.
@@ -827,8 +831,9 @@ static moe_status bwd_gemms_bf16(const moe_config* cfg, const Derived& d, const 
   // slower there (c5: 6.07 / 3.13 ms against 5.56 / 2.77 ms)
   const bool rpair = ffn_uses_pair(cfg, d);
   const bool wpair = false;
-  // 3. SAVE: U (and V), H of every dispatched row again
-  {
+  // 3. SAVE: U (and V), H of every dispatched row again (unless the
+  //    training forward kept them)
+  if (!B.saved) {
     BwdMaps m{};
     BwdParams p = base;
     if (!map(&m.a0, xp, rows, D, rbox)) return MOE_ERR_UNSUPPORTED;
@@ -976,13 +981,14 @@ moe_status moe_backward_workspace_size(const moe_config* cfg, size_t* bytes, int
   return MOE_OK;
 }
 
-moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float* Wg,
-                              const void* W1, const void* W3, const void* W2, const void* sW1,
-                              const void* sW3, const void* sW2, const moe_route_out* route,
-                              void* fwd_ws, size_t fwd_ws_bytes, const void* dout, void* dX,
-                              float* dWg, void* dW1, void* dW3, void* dW2, void* dsW1,
-                              void* dsW3, void* dsW2, float* dL, void* ws, size_t ws_bytes,
-                              moe_stream_t stream) {
+static moe_status layer_backward_impl(const moe_config* cfg, const void* X, const float* Wg,
+                                      const void* W1, const void* W3, const void* W2,
+                                      const void* sW1, const void* sW3, const void* sW2,
+                                      const moe_route_out* route, void* fwd_ws,
+                                      size_t fwd_ws_bytes, const void* dout, void* dX,
+                                      float* dWg, void* dW1, void* dW3, void* dW2, void* dsW1,
+                                      void* dsW3, void* dsW2, float* dL, void* ws,
+                                      size_t ws_bytes, moe_stream_t stream, bool saved) {
   Derived d;
   moe_status st = derive(cfg, &d);
   if (st != MOE_OK) return st;
@@ -1053,7 +1059,7 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float*
   cb.dL = dl;
   MOE_CU(launch_combine_backward(cb, s));
 
-  const BwdBufs bufs{xp, dy, U, V, H, duv, dxp};
+  const BwdBufs bufs{xp, dy, U, V, H, duv, dxp, saved && bf16};
   if ((st = (bf16 ? bwd_gemms_bf16 : bwd_gemms_f32)(cfg, d, bufs, X, W1, W3, W2, sW1, sW3, sW2,
                                                      route, dout, dW1, dW3, dW2, dsW1, dsW3,
                                                      dsW2, err, s)) != MOE_OK)
@@ -1080,6 +1086,67 @@ moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float*
   rb.splits = b.splits;
   MOE_CU(launch_router_backward(rb, s));
   return MOE_OK;
+}
+
+moe_status moe_layer_backward(const moe_config* cfg, const void* X, const float* Wg,
+                              const void* W1, const void* W3, const void* W2, const void* sW1,
+                              const void* sW3, const void* sW2, const moe_route_out* route,
+                              void* fwd_ws, size_t fwd_ws_bytes, const void* dout, void* dX,
+                              float* dWg, void* dW1, void* dW3, void* dW2, void* dsW1,
+                              void* dsW3, void* dsW2, float* dL, void* ws, size_t ws_bytes,
+                              moe_stream_t stream) {
+  return layer_backward_impl(cfg, X, Wg, W1, W3, W2, sW1, sW3, sW2, route, fwd_ws, fwd_ws_bytes,
+                             dout, dX, dWg, dW1, dW3, dW2, dsW1, dsW3, dsW2, dL, ws, ws_bytes,
+                             stream, false);
+}
+
+moe_status moe_layer_backward_train(const moe_config* cfg, const void* X, const float* Wg,
+                                    const void* W1, const void* W3, const void* W2,
+                                    const void* sW1, const void* sW3, const void* sW2,
+                                    const moe_route_out* route, void* fwd_ws,
+                                    size_t fwd_ws_bytes, const void* dout, void* dX,
+                                    float* dWg, void* dW1, void* dW3, void* dW2, void* dsW1,
+                                    void* dsW3, void* dsW2, float* dL, void* ws, size_t ws_bytes,
+                                    moe_stream_t stream) {
+  return layer_backward_impl(cfg, X, Wg, W1, W3, W2, sW1, sW3, sW2, route, fwd_ws, fwd_ws_bytes,
+                             dout, dX, dWg, dW1, dW3, dW2, dsW1, dsW3, dsW2, dL, ws, ws_bytes,
+                             stream, true);
+}
+
+moe_status moe_layer_forward_train(const moe_config* cfg, const void* X, const float* Wg,
+                                   const float* logit_bias, const float* sel_bias,
+                                   const void* W1, const void* W3, const void* W2,
+                                   const void* sW1, const void* sW3, const void* sW2, void* out,
+                                   moe_route_out* route, void* ws, size_t ws_bytes,
+                                   void* bwd_ws, size_t bwd_ws_bytes, moe_stream_t stream) {
+  if (!cfg || cfg->dtype != MOE_BF16)  // fp32 layers keep nothing: their backward recomputes
+    return moe_layer_forward(cfg, X, Wg, logit_bias, sel_bias, W1, W3, W2, sW1, sW3, sW2, out,
+                             route, ws, ws_bytes, stream);
+  Derived d;
+  moe_status st = derive(cfg, &d);
+  if (st != MOE_OK) return st;
+  if (!X || !Wg || !out || !W1 || !W2) return MOE_ERR_INVALID_ARG;
+  if ((st = check_route_out(cfg, route)) != MOE_OK) return st;
+  const WsLayout w = ws_layout(cfg, d);
+  if ((st = check_ws(ws, ws_bytes, w.layer_end)) != MOE_OK) return st;
+  const BwdLayout b = bwd_layout(cfg, d);
+  if ((st = check_ws(bwd_ws, bwd_ws_bytes, b.end)) != MOE_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  void* xp = at<void>(ws, w.xperm);
+  void* yp = at<void>(ws, w.yperm);
+  void* U = at<void>(bwd_ws, b.u);
+  void* V = cfg->act == MOE_ACT_SWIGLU ? at<void>(bwd_ws, b.v) : nullptr;
+  void* H = at<void>(bwd_ws, b.hh);
+  if ((st = route_impl(cfg, d, w, X, Wg, logit_bias, sel_bias, route, ws, s)) != MOE_OK)
+    return st;
+  if ((st = dispatch_impl(cfg, d, X, route, xp, at<int>(ws, w.err), s)) != MOE_OK) return st;
+  // padding rows of X_perm as zeros, so that the kept U, V and H are zero
+  // there and the weight-gradient reductions may read them
+  MOE_CU(launch_pad_zero(route->offsets, route->counts, cfg->E, cfg->d * 2, xp, nullptr, s));
+  if ((st = ffn_impl(cfg, d, X, xp, nullptr, route->offsets, route->counts, W1, W3, W2, sW1,
+                     sW3, sW2, H, yp, at<int>(ws, w.err), s, nullptr, nullptr, U, V)) != MOE_OK)
+    return st;
+  return combine_impl(cfg, d, yp, route, out, s);
 }
 
 moe_status moe_workspace_init(void* ws, moe_stream_t stream) {

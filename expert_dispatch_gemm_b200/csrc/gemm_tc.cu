@@ -44,8 +44,9 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 enum { ACT_NONE = 0, ACT_RELU = 1, ACT_GELU = 2, ACT_SWIGLU = 3 };
 // what a projection fuses: nothing; the dispatch gather into its A loads (up
 // projection); the gate-scaled scatter-add of the combine into its epilogue
-// (down projection)
-enum { FUSE_NONE = 0, FUSE_GATHER = 1, FUSE_SCATTER = 2 };
+// (down projection); or, for training, the up projection also stores its
+// pre-activations U (and V) beside H for the backward pass
+enum { FUSE_NONE = 0, FUSE_GATHER = 1, FUSE_SCATTER = 2, FUSE_SAVE = 3 };
 
 struct TcGemmParams {
   const int32_t* offsets;
@@ -67,6 +68,8 @@ struct TcGemmParams {
   const float* row_gate;     // scatter: gate of each dispatched row
   float* out32;              // scatter: [n_tok, n_out] fp32 sums
   int n_tok;
+  __nv_bfloat16* save_u;     // save: [rows, n_out] pre-activations U = X W1^T
+  __nv_bfloat16* save_v;     // save (SwiGLU): [rows, n_out] V = X W3^T
 };
 
 struct SharedState {
@@ -145,6 +148,17 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, const TcGemmParams& p
   c.col0 = nt * BNO;
   c.b_row += c.col0;
   return c;
+}
+
+// 32 fp32 accumulator values (as bits) rounded to bf16 into 64 bytes
+__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t* v) {
+  uint4* o = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    o[j] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
+                      pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
+                      pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
+                      pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
 }
 
 // fp32 vector reduction into global memory (sm_90+), 16-byte aligned
@@ -381,11 +395,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const float b = __uint_as_float(g[i]);
             f[i] = a * __frcp_rn(1.0f + __expf(-a)) * b;
           }
+          if (FUSE == FUSE_SAVE) store_row32(p.save_v + (orow - p.out) + c.col0 + cc, g);
         } else {
           sm100::tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; ++i) f[i] = act_fn<ACT>(__uint_as_float(v[i]));
         }
+        if (FUSE == FUSE_SAVE) store_row32(p.save_u + (orow - p.out) + c.col0 + cc, v);
         if (FUSE == FUSE_SCATTER) {
           if (tok >= 0) {
             float* dst = p.out32 + (size_t)tok * p.n_out + c.col0 + cc;
@@ -754,11 +770,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
               const float b = __uint_as_float(g[i]);
               f[i] = a * __frcp_rn(1.0f + __expf(-a)) * b;
             }
+            if (FUSE == FUSE_SAVE) store_row32(p.save_v + (orow - p.out) + c.col0 + cc, g);
           } else {
             sm100::tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i) f[i] = act_fn<ACT>(__uint_as_float(v[i]));
           }
+          if (FUSE == FUSE_SAVE) store_row32(p.save_u + (orow - p.out) + c.col0 + cc, v);
           if (FUSE == FUSE_SCATTER) {
             if (tok >= 0) {
               float* dst = p.out32 + (size_t)tok * p.n_out + c.col0 + cc;
@@ -862,10 +880,11 @@ static cudaError_t launch_gemm_t(const Maps& m, const TcGemmParams& p, bool pair
   return launch_one(tc_grouped_gemm_kernel<ACT, FUSE>, m, p, grid, bytes, s);
 }
 
-// up projections fuse nothing or the gather
+// up projections fuse nothing, the gather, or the saving of U (and V)
 template <int ACT>
 static cudaError_t launch_gemm(const Maps& m, const TcGemmParams& p, bool pair, bool gather,
                                int grid, cudaStream_t s) {
+  if (p.save_u) return launch_gemm_t<ACT, FUSE_SAVE>(m, p, pair, grid, s);
   return gather ? launch_gemm_t<ACT, FUSE_GATHER>(m, p, pair, grid, s)
                 : launch_gemm_t<ACT, FUSE_NONE>(m, p, pair, grid, s);
 }
@@ -959,6 +978,8 @@ moe_status run_ffn_bf16(const FfnArgs& f, cudaStream_t s) {
   p.out = static_cast<__nv_bfloat16*>(f.H);
   p.err = f.err;
   p.row_token = f.row_token;
+  p.save_u = static_cast<__nv_bfloat16*>(f.save_u);
+  p.save_v = static_cast<__nv_bfloat16*>(f.save_v);
   cudaError_t e = cudaSuccess;
   const int grid_up = persistent_grid(p, pair);
   switch (f.act) {
@@ -984,6 +1005,7 @@ moe_status run_ffn_bf16(const FfnArgs& f, cudaStream_t s) {
   dm.b1g = dm.b1;
   dm.xg = dm.a0;
   TcGemmParams q = p;
+  q.save_u = q.save_v = nullptr;
   q.K = f.h;
   q.n_out = f.d;
   q.nt_tiles = ceil_div(f.d, kBN);

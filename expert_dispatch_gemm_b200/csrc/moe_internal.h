@@ -197,6 +197,9 @@ struct FfnArgs {
   // (fp32 reductions), row_gate [rows]; Y is then not written
   const float* row_gate;
   float* out32;
+  // training: the up projection also stores U (and V) [rows, h] (bf16)
+  void* save_u;
+  void* save_v;
 };
 // GEMM kernel choice for a config
 bool ffn_uses_pair(const moe_config* c, const Derived& d);

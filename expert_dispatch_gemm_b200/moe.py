@@ -37,7 +37,7 @@ API_SYMBOLS = ["moe_status_string", "moe_validate", "moe_sizes", "moe_workspace_
                "moe_combine", "moe_layer_forward", "moe_bias_update", "moe_workspace_init",
                "moe_read_error", "moe_route_noalloc", "moe_expert_ffn_gathered",
                "moe_launch_counts", "moe_backward_workspace_size", "moe_layer_backward",
-               "moe_expert_ffn_combined"]
+               "moe_expert_ffn_combined", "moe_layer_forward_train", "moe_layer_backward_train"]
 MOE_ROUTE_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -100,6 +100,11 @@ def lib() -> ctypes.CDLL:
                                               ctypes.c_size_t, P]
         L.moe_expert_ffn_combined.argtypes = [cfgp, P, P, outp, P, P, P, P, P, P, P, P, P, P,
                                               P, ctypes.c_size_t, P]
+        L.moe_layer_forward_train.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, outp, P,
+                                              ctypes.c_size_t, P, ctypes.c_size_t, P]
+        L.moe_layer_backward_train.argtypes = [cfgp, P, P, P, P, P, P, P, P, outp, P,
+                                               ctypes.c_size_t, P, P, P, P, P, P, P, P, P, P, P,
+                                               ctypes.c_size_t, P]
         L.moe_backward_workspace_size.argtypes = [cfgp, ctypes.POINTER(ctypes.c_size_t), ip]
         L.moe_layer_backward.argtypes = [cfgp, P, P, P, P, P, P, P, P, outp, P, ctypes.c_size_t,
                                          P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
@@ -339,6 +344,27 @@ def moe_layer_backward(cfg, X, Wg, W1, W3, W2, sW1, sW3, sW2, route: RouteBuffer
            "moe_layer_backward")
 
 
+def moe_layer_forward_train(cfg, X, Wg, logit_bias, sel_bias, W1, W3, W2, sW1, sW3, sW2, out,
+                            route: RouteBuffers, ws, bwd_ws, stream=None):
+    _check(lib().moe_layer_forward_train(ctypes.byref(cfg), _ptr(X), _ptr(Wg), _ptr(logit_bias),
+                                         _ptr(sel_bias), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(sW1),
+                                         _ptr(sW3), _ptr(sW2), _ptr(out), ctypes.byref(route.c),
+                                         _ptr(ws), ws.numel(), _ptr(bwd_ws), bwd_ws.numel(),
+                                         _stream(stream)), "moe_layer_forward_train")
+
+
+def moe_layer_backward_train(cfg, X, Wg, W1, W3, W2, sW1, sW3, sW2, route: RouteBuffers, fwd_ws,
+                             dout, dX, dWg, dW1, dW3, dW2, dsW1, dsW3, dsW2, dL, ws,
+                             stream=None):
+    _check(lib().moe_layer_backward_train(ctypes.byref(cfg), _ptr(X), _ptr(Wg), _ptr(W1),
+                                          _ptr(W3), _ptr(W2), _ptr(sW1), _ptr(sW3), _ptr(sW2),
+                                          ctypes.byref(route.c), _ptr(fwd_ws), fwd_ws.numel(),
+                                          _ptr(dout), _ptr(dX), _ptr(dWg), _ptr(dW1), _ptr(dW3),
+                                          _ptr(dW2), _ptr(dsW1), _ptr(dsW3), _ptr(dsW2),
+                                          _ptr(dL), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_layer_backward_train")
+
+
 def moe_read_error(ws, stream=None):
     detail = ctypes.c_int()
     st = lib().moe_read_error(_ptr(ws), _stream(stream), ctypes.byref(detail))
@@ -384,6 +410,27 @@ class Layer:
             self._bws, self.bwd_launches = backward_workspace(self.cfg, dev)
             self._grads = g
         return self._grads
+
+    def forward_train(self, X=None, stream=None):
+        """forward() that also keeps the up projection's U, V and H for
+        backward_train() (moe_layer_forward_train)."""
+        i = self.inp
+        self.grads()
+        moe_layer_forward_train(self.cfg, i["X"] if X is None else X, i["Wg"],
+                                i.get("logit_bias"), i.get("sel_bias"), i["W1"], i.get("W3"),
+                                i["W2"], i.get("sW1"), i.get("sW3"), i.get("sW2"), self.out,
+                                self.route, self.ws, self._bws, stream)
+        return self.out
+
+    def backward_train(self, dout, X=None, stream=None):
+        """backward() after forward_train(): no recompute of the up projection."""
+        i, g = self.inp, self.grads()
+        moe_layer_backward_train(self.cfg, i["X"] if X is None else X, i["Wg"], i["W1"],
+                                 i.get("W3"), i["W2"], i.get("sW1"), i.get("sW3"), i.get("sW2"),
+                                 self.route, self.ws, dout, g["dX"], g["dWg"], g["dW1"],
+                                 g["dW3"], g["dW2"], g["dsW1"], g["dsW3"], g["dsW2"], g["dL"],
+                                 self._bws, stream)
+        return g
 
     def backward(self, dout, X=None, stream=None):
         """Gradients of <dout, out> + the aux losses after forward() on the same

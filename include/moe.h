@@ -391,6 +391,33 @@ MOE_API moe_status moe_layer_backward(const moe_config* cfg, const void* X, cons
                                       void* dsW1, void* dsW3, void* dsW2, float* dL,
                                       void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* The training pair. moe_layer_forward_train is moe_layer_forward that also
+ * keeps, in `bwd_ws` (moe_backward_workspace_size bytes), what the backward
+ * would otherwise recompute: the up projection's pre-activations U = X W1^T
+ * (and V = X W3^T for SwiGLU) and H, all bf16, with the dispatched rows'
+ * padding rows cleared first so that they are zero there. out, route and
+ * ws are as for moe_layer_forward (H is kept in bwd_ws instead of ws).
+ * moe_layer_backward_train takes moe_layer_backward's arguments, with ws the
+ * same bwd_ws, and skips the recompute. fp32 configs keep nothing: the pair
+ * then behaves as moe_layer_forward / moe_layer_backward. */
+MOE_API moe_status moe_layer_forward_train(const moe_config* cfg, const void* X,
+                                           const float* Wg, const float* logit_bias,
+                                           const float* sel_bias, const void* W1,
+                                           const void* W3, const void* W2, const void* sW1,
+                                           const void* sW3, const void* sW2, void* out,
+                                           moe_route_out* route, void* ws, size_t ws_bytes,
+                                           void* bwd_ws, size_t bwd_ws_bytes,
+                                           moe_stream_t stream);
+MOE_API moe_status moe_layer_backward_train(const moe_config* cfg, const void* X,
+                                            const float* Wg, const void* W1, const void* W3,
+                                            const void* W2, const void* sW1, const void* sW3,
+                                            const void* sW2, const moe_route_out* route,
+                                            void* fwd_ws, size_t fwd_ws_bytes, const void* dout,
+                                            void* dX, float* dWg, void* dW1, void* dW3,
+                                            void* dW2, void* dsW1, void* dsW3, void* dsW2,
+                                            float* dL, void* ws, size_t ws_bytes,
+                                            moe_stream_t stream);
+
 /* Zeroes the error word at the start of `ws` (enqueued on `stream`). */
 MOE_API moe_status moe_workspace_init(void* ws, moe_stream_t stream);
 

@@ -33,7 +33,7 @@ def declared_symbols():
 
 def test_every_declared_symbol_is_exported():
     syms = declared_symbols()
-    assert len(syms) == 19
+    assert len(syms) == 21
     assert sorted(moe.API_SYMBOLS) == syms
     L = ctypes.CDLL(moe.LIB_PATH)
     for s in syms:

@@ -237,3 +237,26 @@ def test_backward_full_size_sampled(w):
         assert _rel(host(g["d" + p + "W2"][e][:, jt]), r2) < BF16_GRAD_TOL, (e, shared, "W2")
         if swiglu:
             assert _rel(host(g["d" + p + "W3"][e][jt]), r3) < BF16_GRAD_TOL, (e, shared, "W3")
+
+
+@pytest.mark.parametrize("w", wl.SMALL + [wl.TC_SIGMOID_GROUPED.replace(
+    name="bwd-train-pair-swap-top8of64-shared1-n2048-d256-h128", n=2048, d=256, E=64, h=128,
+    bias_steps=0)], ids=lambda w: w.name)
+def test_training_pair_matches_recompute(w):
+    """moe_layer_forward_train + moe_layer_backward_train (U, V and H kept by
+    the forward) against moe_layer_forward + moe_layer_backward (recomputed):
+    the same kernels compute U, V and H from the same fp32 accumulators, so
+    every output and gradient agrees to rounding."""
+    inp = wl.make_inputs(w, DEV)
+    layer = moe.Layer(w, inp, DEV)
+    out0 = layer.forward().clone()
+    dout = _dout(w, seed=23)
+    g0 = {k: v.clone() for k, v in layer.backward(dout).items() if v is not None}
+    out1 = layer.forward_train()
+    g1 = layer.backward_train(dout)
+    torch.cuda.synchronize()
+    _ws_ok(layer.ws)
+    _ws_ok(layer._bws)
+    assert _rel(host(out1), host(out0)) < 1e-6
+    for k, v in g0.items():
+        assert _rel(host(g1[k]), host(v)) < (1e-6 if w.dtype == "f32" else 2e-3), k
