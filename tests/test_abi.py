@@ -11,6 +11,7 @@ import subprocess
 import tempfile
 
 import pytest
+import torch
 
 from expert_dispatch_gemm_b200 import build as build_mod
 from expert_dispatch_gemm_b200 import moe
@@ -230,3 +231,37 @@ def test_backward_rejects_bad_arguments_before_launching():
     st = L.moe_layer_backward(ctypes.byref(cfg32), *([None] * 8), ctypes.byref(route), None, 0,
                               *([None] * 10), None, 0, None)
     assert st == moe.MOE_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(),
+                    reason="hands fake device pointers to the library: host-only check")
+def test_backward_host_validation_without_device_memory():
+    """The backward entry points check workspaces and alignment on the host
+    before any launch: fake (never dereferenced) 256-byte-aligned pointers
+    with too-small workspaces, and a misaligned gradient pointer, are
+    refused with the documented status."""
+    cfg = moe.config(wl.TC_DROPLESS.replace(n=256, d=128, E=8, h=128))
+    L = moe.lib()
+    route = moe.MoeRouteOut(*[0x10000 + 0x1000 * i for i in range(14)])
+    fake = [ctypes.c_void_p(0x100000 + 0x10000 * i) for i in range(24)]
+    st, need, _ = _bwd_size(cfg)
+    assert st == moe.MOE_OK and need > 0
+    args = lambda fwd_bytes, ws_bytes, dX: (
+        ctypes.byref(cfg), *fake[:8], ctypes.byref(route), fake[8], fwd_bytes, fake[9], dX,
+        *fake[11:19], fake[19], ws_bytes, None)
+    # forward workspace too small
+    st = L.moe_layer_backward(*args(16, need, fake[10]))
+    assert st == moe.MOE_ERR_WORKSPACE
+    fwd_need = moe.sizes(cfg).layer_ws
+    # backward workspace too small
+    st = L.moe_layer_backward(*args(fwd_need, need - 1, fake[10]))
+    assert st == moe.MOE_ERR_WORKSPACE
+    st = L.moe_layer_backward_train(*args(fwd_need, need - 1, fake[10]))
+    assert st == moe.MOE_ERR_WORKSPACE
+    # dX not 16-byte aligned
+    st = L.moe_layer_backward(*args(fwd_need, need, ctypes.c_void_p(0x200008)))
+    assert st == moe.MOE_ERR_INVALID_ARG
+    # the training forward checks its backward workspace too
+    st = L.moe_layer_forward_train(ctypes.byref(cfg), *fake[:11], ctypes.byref(route), fake[11],
+                                   fwd_need, fake[12], need - 1, None)
+    assert st == moe.MOE_ERR_WORKSPACE
