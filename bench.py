@@ -650,15 +650,9 @@ def cpu_baseline_train(w, inp, dout, budget_s=20.0):
     token's dX needs only its own pairs; their expert rows also carry the
     weight-gradient work), extrapolated to the batch."""
     import oracle
-    X, Wg, lb, sb, weights = _host_inputs(w, inp)
+    X, Wg, lb, sb, weights, sw = _host_inputs(w, inp)
     spec = oracle.spec_of(w)
     dh = dout.float().cpu().numpy()
-    sw = None
-    if w.n_shared:
-        def sw(s):
-            return (inp["sW1"][s].float().cpu().numpy(),
-                    None if inp.get("sW3") is None else inp["sW3"][s].float().cpu().numpy(),
-                    inp["sW2"][s].float().cpu().numpy())
     rng = np.random.default_rng(0)
     t0 = time.perf_counter()
     logits, S, lse = oracle.router(X, Wg, lb, spec["score"])
@@ -688,8 +682,9 @@ def cpu_baseline_train(w, inp, dout, budget_s=20.0):
 # CPU oracle (baseline leg and reference arm)
 # ---------------------------------------------------------------------------
 
-def _oracle_layer_sample(w, X, Wg, lb, sb, weights, sample_tokens):
-    """Routing of the whole batch, FFN + combine for `sample_tokens`."""
+def _oracle_layer_sample(w, X, Wg, lb, sb, weights, shared, sample_tokens):
+    """Routing of the whole batch, FFN + combine for `sample_tokens` (the
+    shared experts included)."""
     import oracle
     spec = oracle.spec_of(w)
     t0 = time.perf_counter()
@@ -697,7 +692,7 @@ def _oracle_layer_sample(w, X, Wg, lb, sb, weights, sample_tokens):
     r = oracle.route(spec, S, lse, sb)
     t_route = time.perf_counter() - t0
     t0 = time.perf_counter()
-    oracle.layer_forward(spec, X, r, weights, None, tokens=sample_tokens)
+    oracle.layer_forward(spec, X, r, weights, shared, tokens=sample_tokens)
     t_ffn = time.perf_counter() - t0
     return t_route, t_ffn
 
@@ -713,20 +708,26 @@ def _host_inputs(w, inp=None):
 
     def weights(e):
         return h(W1[e]), None if W3 is None else h(W3[e]), h(W2[e])
-    return X, Wg, lb, sb, weights
+
+    shared = None
+    if w.n_shared:
+        def shared(s):
+            return (h(inp["sW1"][s]), None if inp.get("sW3") is None else h(inp["sW3"][s]),
+                    h(inp["sW2"][s]))
+    return X, Wg, lb, sb, weights, shared
 
 
 def cpu_baseline(w, inp=None, budget_s=20.0, sample=None):
-    X, Wg, lb, sb, weights = _host_inputs(w, inp)
+    X, Wg, lb, sb, weights, shared = _host_inputs(w, inp)
     rng = np.random.default_rng(0)
     if sample is None:
         # size the FFN sample from a short probe so the whole leg takes ~budget_s
         probe = sorted(rng.choice(w.n, size=min(8, w.n), replace=False).tolist())
-        t_route, t_ffn = _oracle_layer_sample(w, X, Wg, lb, sb, weights, probe)
+        t_route, t_ffn = _oracle_layer_sample(w, X, Wg, lb, sb, weights, shared, probe)
         per_tok = t_ffn / len(probe)
         sample = int(max(8, min(w.n, (budget_s - t_route) / max(per_tok, 1e-6))))
     toks = sorted(rng.choice(w.n, size=min(sample, w.n), replace=False).tolist())
-    t_route, t_ffn = _oracle_layer_sample(w, X, Wg, lb, sb, weights, toks)
+    t_route, t_ffn = _oracle_layer_sample(w, X, Wg, lb, sb, weights, shared, toks)
     est = t_route + t_ffn / len(toks) * w.n
     return {"value": round(w.n / est, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": (f"routing of all {w.n} tokens ({t_route:.2f} s) + expert FFN and "
@@ -739,13 +740,13 @@ def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    X, Wg, lb, sb, weights = _host_inputs(w)
+    X, Wg, lb, sb, weights, shared = _host_inputs(w)
     rng = np.random.default_rng(1)
     sample = args.ref_sample
     times = []
     for i in range(args.warmup + args.steps):
         toks = sorted(rng.choice(w.n, size=min(sample, w.n), replace=False).tolist())
-        t_route, t_ffn = _oracle_layer_sample(w, X, Wg, lb, sb, weights, toks)
+        t_route, t_ffn = _oracle_layer_sample(w, X, Wg, lb, sb, weights, shared, toks)
         if i >= args.warmup:
             times.append(t_route + t_ffn / len(toks) * w.n)
     est = float(np.mean(times))
