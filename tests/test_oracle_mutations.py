@@ -67,6 +67,22 @@ MUTATIONS = [
      "        s = sqrt(sp);",
      "        s = sp;",
      ["test_sqrtsoftplus_closed_forms"]),
+    ("SwiGLU up value from W1 instead of W3",
+     "        for (int i = 0; i < d; ++i) b += (double)x[i] * (double)W3[(size_t)j * d + i];",
+     "        for (int i = 0; i < d; ++i) b += (double)x[i] * (double)W1[(size_t)j * d + i];",
+     ["test_expert_ffn_against_torch"]),
+    ("down projection reads W2 transposed",
+     "      for (int j = 0; j < h; ++j) y += (double)W2[(size_t)i * h + j] * (double)H[j];",
+     "      for (int j = 0; j < h; ++j) y += (double)W2[(size_t)j * d + i] * (double)H[j];",
+     ["test_expert_ffn_against_torch"]),
+    ("router reads W_g transposed",
+     "      for (int e = 0; e < E; ++e) acc[e] += x * (double)w[e];",
+     "      for (int e = 0; e < E; ++e) acc[e] += x * (double)Wg[(size_t)e * d + i] + 0.0 * w[e];",
+     ["test_router_against_library"]),
+    ("top-k keeps the smallest keys",
+     "  if (a->key > b->key) return -1;\n  if (a->key < b->key) return 1;",
+     "  if (a->key < b->key) return -1;\n  if (a->key > b->key) return 1;",
+     ["test_tc_topk_matches_brute_force", "test_ec_topk_matches_brute_force"]),
     # backward pass
     ("SwiGLU backward drops the u (1 - sigma) part of silu'",
      "dUs[j] = round_store(dh * vs * sg * (1.0 + us * (1.0 - sg)), store);",
