@@ -609,7 +609,9 @@ def run_gpu_train(args, w: wl.Workload):
                  "kernel": "moe_layer_backward_train as a whole: its grouped GEMMs' FLOPs over "
                            "the whole call (its non-GEMM kernels included in the time)",
                  "algorithmic_per_launch": gemm_flops})
-    fwd_launches = sum(moe.launch_counts(layer.cfg).values())
+    # the training forward launches the layer's kernels plus, for bf16, the
+    # clearing of the dispatched rows' padding before the up projection
+    fwd_launches = sum(moe.launch_counts(layer.cfg).values()) + (1 if w.dtype == "bf16" else 0)
     res = {
         "metric": METRIC_TRAIN,
         "value": round(whole_job_rate(w.n, world, args.steps, total_ms), 1), "unit": "tokens/s",
