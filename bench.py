@@ -635,7 +635,9 @@ def run_gpu_train(args, w: wl.Workload):
                 "d2h_bytes_per_step": int(dXh.numel() * dXh.element_size()),
                 "note": "pinned host X and dout -> device -> forward + backward -> host dX "
                         "every step, on the compute stream; no L2 flush"},
-        "gpu_launches": (fwd_launches + layer.bwd_launches) * args.steps,
+        # the training backward skips the recompute GEMM on bf16 layers
+        "gpu_launches": (fwd_launches + layer.bwd_launches - (1 if w.dtype == "bf16" else 0))
+        * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

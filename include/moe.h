@@ -364,7 +364,9 @@ MOE_API moe_status moe_expert_ffn_combined(const moe_config* cfg, const void* X,
  * multiples of 64); fp32 configs run them on FFMA and store every value in
  * fp32 (no rounding to bf16 anywhere). */
 
-/* Backward workspace bytes and the kernels moe_layer_backward enqueues. */
+/* Backward workspace bytes and the kernels moe_layer_backward enqueues
+ * (moe_layer_backward_train enqueues one fewer for bf16 configs: it skips
+ * the recompute of the up projection). */
 MOE_API moe_status moe_backward_workspace_size(const moe_config* cfg, size_t* bytes,
                                                int* launches);
 
