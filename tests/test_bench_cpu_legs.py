@@ -32,3 +32,21 @@ def test_reference_arm_prints_one_json_line():
     assert j["impl"] == "reference" and j["config"]["workload"] == w.name
     assert j["value"] > 0 and j["cpu_baseline"]["kind"] == "oracle"
     assert j["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_training_cpu_baseline_and_flop_count():
+    """The training line's CPU baseline (the oracle's backward on sampled
+    tokens) runs for a layer with a shared expert, and the backward's GEMM
+    FLOPs count the recompute only for fp32 layers (bf16 layers keep U, V, H
+    from the training forward)."""
+    import torch
+    w = wl.SMALL[4]
+    inp = wl.make_inputs(w, "cpu")
+    dout = torch.randn((w.n, w.d)).to(w.torch_dtype)
+    res = bench.cpu_baseline_train(w, inp, dout, budget_s=2.0)
+    assert res["kind"] == "oracle" and res["value"] > 0
+    bf = bench.backward_flops(w, 2400)
+    assert "recompute" not in bf
+    rows = 2400 + w.n
+    assert bf["dw13"] == 2 * (2.0 * rows * w.d * w.h)  # SwiGLU: W1 and W3
+    assert "recompute" in bench.backward_flops(wl.EC_FP32, 1024)
