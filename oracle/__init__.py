@@ -174,7 +174,7 @@ def select_tc(S, K: int, sel_bias=None, n_groups: int = 1, topk_groups: int = 1,
     n, E = S.shape
     if n_groups > 1:
         assert E % n_groups == 0 and 1 <= topk_groups <= n_groups
-        assert 1 <= group_topn <= E // n_groups <= 1024
+        assert 1 <= group_topn <= E // n_groups
         assert K <= topk_groups * (E // n_groups)
     assert 1 <= K <= E
     idx = np.empty((n, K), np.int32)

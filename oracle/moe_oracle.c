@@ -143,6 +143,7 @@ void orc_select_tc(int n, int E, int K, const float* S, const float* sel_bias,
   keyed* cand = (keyed*)malloc(sizeof(keyed) * (size_t)E);
   keyed* grp = (keyed*)malloc(sizeof(keyed) * (size_t)(n_groups > 0 ? n_groups : 1));
   char* allowed = (char*)malloc((size_t)E);
+  keyed* tmp = (keyed*)malloc(sizeof(keyed) * (size_t)E); /* one group's keys */
   for (int t = 0; t < n; ++t) {
     const float* s = S + (size_t)t * E;
     for (int e = 0; e < E; ++e) {
@@ -153,7 +154,6 @@ void orc_select_tc(int n, int E, int K, const float* S, const float* sel_bias,
     if (n_groups > 1) {
       int gsize = E / n_groups;
       for (int g = 0; g < n_groups; ++g) {
-        keyed tmp[1024];
         for (int j = 0; j < gsize; ++j) tmp[j] = all[g * gsize + j];
         qsort(tmp, (size_t)gsize, sizeof(keyed), cmp_keyed);
         float sum = 0.0f; /* fp32, largest key first */
@@ -185,6 +185,7 @@ void orc_select_tc(int n, int E, int K, const float* S, const float* sel_bias,
   free(cand);
   free(grp);
   free(allowed);
+  free(tmp);
 }
 
 /* [TC-vs-EC] "Dropped tokens flow in opposite directions": tokens that arrive

@@ -173,6 +173,23 @@ def test_one_group_or_all_groups_reduce_to_plain_topk():
     np.testing.assert_array_equal(plain, allg)
 
 
+def test_groups_larger_than_1024_experts():
+    """Groups of 1,280 experts (no fixed-size buffer in the C entry): keeping
+    both groups reduces to plain top-K, and keeping one group takes every
+    pick from the group whose two largest keys sum highest."""
+    E, G, K = 2560, 2, 8
+    S = wl.random_scores(4, E, seed=9).numpy()
+    plain, _ = oracle.select_tc(S, K)
+    both, _ = oracle.select_tc(S, K, n_groups=G, topk_groups=2, group_topn=2)
+    np.testing.assert_array_equal(plain, both)
+    S[:, 1280 + 7] = 2.0       # group 1: the two largest keys sum above 2
+    S[:, 1280 + 1000] = 1.5
+    S[:, 3] = 2.5              # group 0 holds the largest key, but its two sum below 3.5
+    one, _ = oracle.select_tc(S, K, n_groups=G, topk_groups=1, group_topn=2)
+    assert (one >= 1280).all()
+    assert (one[:, 0] == 1280 + 7).all() and (one[:, 1] == 1280 + 1000).all()
+
+
 # --------------------------------------------------------------------------
 # capacity and overflow ("Dropped tokens flow in opposite directions";
 # "2. Top-1 switch routing with a capacity factor")
