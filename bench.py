@@ -3,23 +3,31 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl reference] [--pass forward|train]
 
-One step = one pass of the whole hot path over one batch, the calls
-moe_layer_forward makes: moe_route (router GEMM + scores + top-k + capacity
-scan) -> moe_dispatch (gather) -> moe_expert_ffn (tcgen05 grouped GEMM, up +
-down) -> moe_combine. Inputs and
-weights are resident in HBM before timing; L2 (126 MB) is flushed by writing
-a 256 MB buffer between timed steps, outside the timed events. Each stage is
-timed with CUDA events on the launching stream.
+One step = one moe_layer_forward call over one batch: moe_route (router GEMM
++ scores + top-k + capacity scan) -> moe_dispatch (gather) -> moe_expert_ffn
+(tcgen05 grouped GEMM, up + down) -> moe_combine. Inputs and weights are
+resident in HBM before timing; L2 (126 MB) is flushed by writing a 256 MB
+buffer between timed steps, outside the timed events. Steps are timed with
+CUDA events on the launching stream; a second pass calls the four stages one
+by one with an event between them for the per-stage figures.
 
-Default workload: the expert-choice layer of the pages' worked example
-(4,096 tokens, d 1024, 64 experts, c = 2, GELU FFN 1024 -> 4096 -> 1024, bf16).
+Default workload: the largest configuration, the DeepSeek-V3-shaped layer
+("MoE routing strategies explained", sections 3-5: 256 routed experts plus
+one shared, sigmoid scores with a selection-only bias, 8 groups keep 4,
+top-8, normalised weights; 8,192 tokens, d 7168, SwiGLU h 2048, bf16).
 
-Multi-GPU: the layer does not shard ("replicas only"): each
-rank runs an independent replica, no collective touches the data path, and
-the timed region is the max over ranks.
+e2e: the same layer through moe_layer_forward_host, the C call that takes
+host X and host out (page-locked) and copies them itself on the caller's
+stream; two such calls alternate on two streams so that one call's copies
+overlap the other's kernels.
+
+Multi-GPU: the layer does not shard ("replicas only"): each rank runs an
+independent replica, no collective touches the data path, and the timed
+region is the max over ranks.
 
 --impl reference times the CPU oracle as it stands (single thread) on the
-same workload, one bounded sample per step.
+same workload, a bounded sample of tokens per step (the rule of
+oracle_sample_tokens, shared with the cpu_baseline leg).
 
 --pass train times forward + backward (moe_layer_forward_train then
 moe_layer_backward_train: gradients of X, W_g and every expert weight) per
@@ -44,7 +52,7 @@ import torch  # noqa: E402
 from expert_dispatch_gemm_b200 import workloads as wl  # noqa: E402
 
 METRIC = "MoE-layer fwd tokens/s on 1 B200; route/dispatch HBM GB/s; expert-GEMM TC util %"
-DEFAULT = wl.EC_BF16
+DEFAULT = wl.TC_SIGMOID_GROUPED
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -187,18 +195,26 @@ def ffma_peak_tflops(dev) -> float:
     return flops / (float(np.median(times)) * 1e-3) / 1e12
 
 
-def traffic_for(kernel_src: str, workload: str):
-    """DRAM bytes per launch of the grouped GEMM from the committed ncu summary,
-    or None when the device code changed since that capture (the hash covers
-    the source up to its host-side section) or the workload was not captured."""
+def source_sha(name: str) -> str:
+    """Hash of a CUDA source's device code (the file up to its '// host side'
+    marker, or all of it), to tell whether a committed capture still holds."""
+    code = open(os.path.join(ROOT, "expert_dispatch_gemm_b200", "csrc", name), "rb").read()
+    return hashlib.sha256(code.split(b"// host side")[0]).hexdigest()[:16]
+
+
+def traffic_for(workload: str):
+    """DRAM bytes per launch of the grouped GEMM from the committed ncu summary
+    (profiles/gemm_traffic.json), or None when the device code of a source it
+    was captured from changed since, or the workload was not captured."""
     path = os.path.join(ROOT, "profiles", "gemm_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
-        dev_code = open(kernel_src, "rb").read().split(b"// host side")[0]
-        if rec.get("kernel_sha") != hashlib.sha256(dev_code).hexdigest()[:16]:
-            return None
-        return rec.get("bytes_per_launch", {}).get(workload)
+        entry = rec["bytes_per_launch"][workload]
+        for src, sha in entry["sources"].items():
+            if source_sha(src) != sha:
+                return None
+        return entry["bytes"]
     except Exception:
         return None
 
@@ -238,6 +254,16 @@ def routing_stats(w, cfg, inp, rb, ws, moe, stream) -> dict:
     return out
 
 
+def config_dict(w: wl.Workload, world: int, **extra) -> dict:
+    """The `config` object of both arms' JSON lines."""
+    return {"workload": w.name, "tokens": w.n, "d_model": w.d, "experts": w.E, "hidden": w.h,
+            "shared_experts": w.n_shared,
+            "routing": ("expert-choice c=%g" % w.c if w.mode == "ec"
+                        else "token-choice top-%d" % w.K),
+            "parallelism": f"replicas{world}" if world > 1 else "single-gpu",
+            "l2": "flushed between timed steps (256 MB write, outside the events)", **extra}
+
+
 def run_gpu(args, w: wl.Workload):
     import torch.distributed as dist
 
@@ -255,7 +281,8 @@ def run_gpu(args, w: wl.Workload):
     inp = wl.make_inputs(w, dev)
     cfg = moe.config(w)
     sz = moe.sizes(cfg)
-    rb = moe.RouteBuffers(cfg, dev)
+    layer = moe.Layer(w, inp, dev)           # the timed calls: moe_layer_forward
+    rb = moe.RouteBuffers(cfg, dev)          # the stage pass: the four calls one by one
     ws = moe.workspace(cfg, dev, layer=False)
     dt = w.torch_dtype
     X_perm = torch.empty((sz.rows, w.d), dtype=dt, device=dev)
@@ -270,13 +297,19 @@ def run_gpu(args, w: wl.Workload):
         acc = torch.empty((w.n, w.d), dtype=torch.float32, device=dev)
         row_gate = torch.empty(max(sz.rows, 1), dtype=torch.float32, device=dev)
 
-    def step(ev=None, X=None, out_buf=None):
-        """One pass of the layer, the calls moe_layer_forward makes:
-        route -> dispatch gather -> grouped expert FFN -> combine (with
-        --fused-combine: the combine inside the down projection's epilogue,
-        moe_expert_ffn_combined)."""
-        X = inp["X"] if X is None else X
-        o = out if out_buf is None else out_buf
+    def step():
+        """One pass of the layer: one moe_layer_forward call (with
+        --fused-combine: the four calls, the combine inside the down
+        projection's epilogue by moe_expert_ffn_combined)."""
+        if fused:
+            staged()
+        else:
+            layer.forward(stream=stream)
+
+    def staged(ev=None):
+        """The calls moe_layer_forward makes, one by one: route -> dispatch
+        gather -> grouped expert FFN -> combine, with an event between them."""
+        X = inp["X"]
         if ev: ev[0].record(stream)
         moe.moe_route(cfg, X, inp["Wg"], inp["logit_bias"], sb, rb, ws, stream)
         if ev: ev[1].record(stream)
@@ -285,23 +318,27 @@ def run_gpu(args, w: wl.Workload):
         if fused:
             moe.moe_expert_ffn_combined(cfg, X, X_perm, rb, inp["W1"], inp["W3"], inp["W2"],
                                         inp.get("sW1"), inp.get("sW3"), inp.get("sW2"), H, acc,
-                                        row_gate, o, ws, stream)
+                                        row_gate, out, ws, stream)
             if ev: ev[3].record(stream)
         else:
             moe.moe_expert_ffn(cfg, X, X_perm, rb.offsets, inp["W1"], inp["W3"], inp["W2"],
                                inp.get("sW1"), inp.get("sW3"), inp.get("sW2"), H, Y, ws, stream,
                                counts=rb.counts)
             if ev: ev[3].record(stream)
-            moe.moe_combine(cfg, Y, rb, o, stream)
+            moe.moe_combine(cfg, Y, rb, out, stream)
         if ev: ev[4].record(stream)
+
+    def check_errors(when):
+        for wsp in (layer.ws, ws):
+            st, detail = moe.moe_read_error(wsp)
+            if st != moe.MOE_OK:
+                raise RuntimeError(f"device error {when}: {detail:#x}")
 
     for _ in range(args.warmup):
         flush.zero_()
         step()
     torch.cuda.synchronize(dev)
-    st, detail = moe.moe_read_error(ws)
-    if st != moe.MOE_OK:
-        raise RuntimeError(f"device error after warm-up: {detail:#x}")
+    check_errors("after warm-up")
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     if world > 1:
@@ -327,58 +364,57 @@ def run_gpu(args, w: wl.Workload):
     sevs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     for i in range(args.steps):
         flush.zero_()
-        step(sevs[i])
+        staged(sevs[i])
     torch.cuda.synchronize(dev)
     stage_ms = np.array([[sevs[i][j].elapsed_time(sevs[i][j + 1]) for j in range(4)]
                          for i in range(args.steps)])
-    st, detail = moe.moe_read_error(ws)
-    if st != moe.MOE_OK:
-        raise RuntimeError(f"device error in the timed region: {detail:#x}")
+    check_errors("in the timed region")
 
-    # ---- end to end: every step copies its input X from pinned host memory
-    # and its output back to pinned host memory, through the same public
-    # calls. The copies run on their own streams, double-buffered, so step
-    # i+1's input upload and step i-1's download overlap step i's compute.
+    # ---- end to end through the C call that takes host buffers
+    # (moe_layer_forward_host): every step uploads X from page-locked host
+    # memory and downloads out into page-locked host memory, the library
+    # issuing both copies on the call's stream. Two lanes (stream, device
+    # buffers, routing, workspace, host output) alternate, so one call's
+    # copies overlap the other lane's kernels.
     Xh = inp["X"].cpu().pin_memory()
-    outh = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
-    Xd = [torch.empty_like(inp["X"]) for _ in range(2)]
-    outd = [torch.empty_like(out) for _ in range(2)]
-    up_s, down_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ev_in = [torch.cuda.Event() for _ in range(2)]     # upload of buffer b done
-    ev_used = [torch.cuda.Event() for _ in range(2)]   # compute done with buffer b
-    ev_out = [torch.cuda.Event() for _ in range(2)]    # download of buffer b done
+    lanes = []
+    for _ in range(2):
+        lanes.append(dict(s=torch.cuda.Stream(dev), Xd=torch.empty_like(inp["X"]),
+                          od=torch.empty_like(out), rb=moe.RouteBuffers(cfg, dev, logits=False),
+                          ws=moe.workspace(cfg, dev, layer=True),
+                          oh=torch.empty(out.shape, dtype=out.dtype).pin_memory(),
+                          done=torch.cuda.Event()))
 
     def e2e_run(nsteps):
         for i in range(nsteps):
-            b = i & 1
-            if i >= 2:
-                up_s.wait_event(ev_used[b])
-            with torch.cuda.stream(up_s):
-                Xd[b].copy_(Xh, non_blocking=True)
-            ev_in[b].record(up_s)
-            stream.wait_event(ev_in[b])
-            if i >= 2:
-                stream.wait_event(ev_out[b])
-            step(X=Xd[b], out_buf=outd[b])
-            ev_used[b].record(stream)
-            down_s.wait_event(ev_used[b])
-            with torch.cuda.stream(down_s):
-                outh[b].copy_(outd[b], non_blocking=True)
-            ev_out[b].record(down_s)
+            ln = lanes[i & 1]
+            moe.moe_layer_forward_host(cfg, Xh, inp["Wg"], inp["logit_bias"], sb, inp["W1"],
+                                       inp.get("W3"), inp["W2"], inp.get("sW1"), inp.get("sW3"),
+                                       inp.get("sW2"), ln["oh"], ln["Xd"], ln["od"], ln["rb"],
+                                       ln["ws"], ln["s"])
+            ln["done"].record(ln["s"])
 
+    torch.cuda.synchronize(dev)
     e2e_run(max(2, args.warmup))
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    up_s.wait_event(e0)
+    for ln in lanes:
+        ln["s"].wait_event(e0)
     e2e_run(args.steps)
-    stream.wait_event(ev_out[0])
-    stream.wait_event(ev_out[1])
+    for ln in lanes:
+        stream.wait_event(ln["done"])
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1)
     e2e_ms = max_over_ranks(e2e_ms, dev)
-
+    for ln in lanes:
+        st, detail = moe.moe_read_error(ln["ws"], ln["s"])
+        if st != moe.MOE_OK:
+            raise RuntimeError(f"device error in the end-to-end run: {detail:#x}")
+    # the host copy of the last step's output is the layer's output
+    if not torch.equal(lanes[(args.steps - 1) & 1]["oh"], layer.out.cpu()):
+        raise RuntimeError("moe_layer_forward_host returned a different output")
 
     # ---- routing statistics the workload statements ask for (from the last
     # step's routing outputs; untimed)
@@ -420,8 +456,7 @@ def run_gpu(args, w: wl.Workload):
     t_hbm = bytes_["ffn"] / (hbm * 1e9)
     t_tc = flops / (tc_peak * 1e12)
     per_launch_ms = float(med[2]) / 2.0
-    kernel_src = os.path.join(ROOT, "expert_dispatch_gemm_b200", "csrc", "gemm_tc.cu")
-    traffic = traffic_for(kernel_src, w.name) if w.dtype == "bf16" else None
+    traffic = traffic_for(w.name) if w.dtype == "bf16" else None
     if t_hbm >= t_tc:
         ach = bytes_["ffn"] / 2 / (per_launch_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
@@ -443,6 +478,7 @@ def run_gpu(args, w: wl.Workload):
     launches_per_step = sum(moe.launch_counts(cfg).values())
     if fused:
         launches_per_step += 1  # prep + up + down + finish replace up + down + combine
+    xbytes = int(Xh.numel() * Xh.element_size())
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
@@ -450,29 +486,26 @@ def run_gpu(args, w: wl.Workload):
         "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic (seeded N(0,1) activations, random-init weights)",
-        "config": {"workload": w.name, "tokens": w.n, "d_model": w.d, "experts": w.E,
-                   "hidden": w.h, "routing": ("expert-choice c=%g" % w.c if w.mode == "ec"
-                                              else "token-choice top-%d" % w.K),
-                   "parallelism": f"replicas{world}" if world > 1 else "single-gpu",
-                   "l2": "flushed between timed steps (256 MB write, outside the events)",
-                   **({"combine": "fused into the down projection (moe_expert_ffn_combined); "
-                                  "the ffn stage includes it"} if fused else {})},
+        "config": config_dict(w, world, **(
+            {"combine": "fused into the down projection (moe_expert_ffn_combined); "
+                        "the ffn stage includes it"} if fused else {})),
         "roofline": roof,
         "stages": stages,
         "routing": routing,
         "stages_note": "medians of a second pass with an event between stages; value and "
-                       "ms_per_step come from whole-step events",
+                       "ms_per_step come from whole-step events around moe_layer_forward",
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
-                "h2d_bytes_per_step": int(Xh.numel() * Xh.element_size()),
-                "d2h_bytes_per_step": int(outh[0].numel() * outh[0].element_size()),
-                "note": "pinned host X -> device -> layer -> host out every step; copies "
-                        "double-buffered on their own streams; no L2 flush"},
+                "h2d_bytes_per_step": xbytes, "d2h_bytes_per_step": xbytes,
+                "note": "moe_layer_forward_host (C ABI): page-locked host X -> device -> "
+                        "layer -> page-locked host out every step, the copies issued by the "
+                        "library on the call's stream; two calls alternate on two streams; "
+                        "no L2 flush"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
         "wall_s_timed": round(t_wall, 4),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(w, inp, budget_s=args.cpu_budget)
+        res["cpu_baseline"] = cpu_baseline(w, inp)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -609,9 +642,7 @@ def run_gpu_train(args, w: wl.Workload):
                  "kernel": "moe_layer_backward_train as a whole: its grouped GEMMs' FLOPs over "
                            "the whole call (its non-GEMM kernels included in the time)",
                  "algorithmic_per_launch": gemm_flops})
-    # the training forward launches the layer's kernels plus, for bf16, the
-    # clearing of the dispatched rows' padding before the up projection
-    fwd_launches = sum(moe.launch_counts(layer.cfg).values()) + (1 if w.dtype == "bf16" else 0)
+    fwd_launches, bwd_launches = moe.train_launch_counts(layer.cfg)
     res = {
         "metric": METRIC_TRAIN,
         "value": round(whole_job_rate(w.n, world, args.steps, total_ms), 1), "unit": "tokens/s",
@@ -619,10 +650,7 @@ def run_gpu_train(args, w: wl.Workload):
         "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic (seeded N(0,1) activations and output gradient, random-init weights)",
-        "config": {"workload": w.name, "pass": "forward + backward", "tokens": w.n,
-                   "d_model": w.d, "experts": w.E, "hidden": w.h,
-                   "parallelism": f"replicas{world}" if world > 1 else "single-gpu",
-                   "l2": "flushed between timed steps (256 MB write, outside the events)"},
+        "config": config_dict(w, world, **{"pass": "forward + backward"}),
         "roofline": roof,
         "stages": {"forward": {"ms": round(float(np.median(fwd_ms)), 4)},
                    "backward": {"ms": round(bwd_med, 4),
@@ -635,9 +663,7 @@ def run_gpu_train(args, w: wl.Workload):
                 "d2h_bytes_per_step": int(dXh.numel() * dXh.element_size()),
                 "note": "pinned host X and dout -> device -> forward + backward -> host dX "
                         "every step, on the compute stream; no L2 flush"},
-        # the training backward skips the recompute GEMM on bf16 layers
-        "gpu_launches": (fwd_launches + layer.bwd_launches - (1 if w.dtype == "bf16" else 0))
-        * args.steps,
+        "gpu_launches": (fwd_launches + bwd_launches) * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -686,19 +712,80 @@ def cpu_baseline_train(w, inp, dout, budget_s=20.0):
 # CPU oracle (baseline leg and reference arm)
 # ---------------------------------------------------------------------------
 
-def _oracle_layer_sample(w, X, Wg, lb, sb, weights, shared, sample_tokens):
-    """Routing of the whole batch, FFN + combine for `sample_tokens` (the
-    shared experts included)."""
+ORACLE_STEP_FLOP = 8e9  # expert-FFN FLOPs of one oracle step (seconds of one core)
+
+
+def oracle_sample_tokens(w: wl.Workload) -> int:
+    """Tokens whose expert FFN and combine one oracle step computes: about
+    ORACLE_STEP_FLOP of expert FFN, the whole batch when that is smaller.
+    A fixed rule, shared by the reference arm and the cpu_baseline leg, so
+    that both time the same work."""
+    nproj = 3 if w.act == "swiglu" else 2
+    per_token = w.c if w.mode == "ec" else w.K
+    flop = 2.0 * nproj * w.d * w.h * (per_token + w.n_shared)
+    return int(max(4, min(w.n, ORACLE_STEP_FLOP // flop)))
+
+
+def routes_per_token(w: wl.Workload) -> bool:
+    """Token choice without a capacity routes each token from its own row
+    alone ("MoE token-choice routing": no batch coordination), so a sample
+    of tokens is a complete layer call on those tokens. Expert choice and a
+    capacity buffer need the whole batch's scores."""
+    return w.mode == "tc" and w.capacity_factor <= 0
+
+
+def _oracle_step(w, X, Wg, lb, sb, weights, shared, toks):
+    """One oracle step over the tokens `toks`: (seconds routing, seconds of
+    expert FFN + combine). Token choice without a capacity routes only the
+    sampled tokens; otherwise the whole batch is routed and the FFN and
+    combine run for the sample. The expert weights the sample needs are
+    converted to the oracle's fp32 arrays before the clock starts (input
+    marshalling, not the oracle's work)."""
     import oracle
     spec = oracle.spec_of(w)
+    Xs = X[toks] if routes_per_token(w) else X
     t0 = time.perf_counter()
-    _, S, lse = oracle.router(X, Wg, lb, spec["score"])
+    _, S, lse = oracle.router(Xs, Wg, lb, spec["score"])
     r = oracle.route(spec, S, lse, sb)
     t_route = time.perf_counter() - t0
+    local = list(range(len(toks))) if routes_per_token(w) else toks
+    need = sorted({e for _, e, _ in oracle.token_pairs(spec, r, Xs.shape[0], local)})
+    cache = {e: weights(e) for e in need}
     t0 = time.perf_counter()
-    oracle.layer_forward(spec, X, r, weights, shared, tokens=sample_tokens)
+    oracle.layer_forward(spec, Xs, r, cache.__getitem__, shared, tokens=local)
     t_ffn = time.perf_counter() - t0
     return t_route, t_ffn
+
+
+def oracle_steps(w, host, steps: int, warmup: int = 0, seed: int = 0):
+    """`warmup` untimed then `steps` timed oracle steps on the sample rule's
+    token count, a fresh seeded sample each step. Returns (value tokens/s,
+    measured seconds per step, tokens per step, extrapolated, description)."""
+    X, Wg, lb, sb, weights, shared = host
+    rng = np.random.default_rng(seed)
+    m = oracle_sample_tokens(w)
+    per_tok = routes_per_token(w)
+    times, full = [], []
+    for i in range(warmup + steps):
+        toks = sorted(rng.choice(w.n, size=m, replace=False).tolist())
+        t_route, t_ffn = _oracle_step(w, X, Wg, lb, sb, weights, shared, toks)
+        if i >= warmup:
+            times.append(t_route + t_ffn)
+            full.append(t_route + t_ffn / m * w.n)
+    sec = float(np.mean(times))
+    if per_tok or m == w.n:
+        value, extrap = m / sec, False
+        what = (f"per step: the whole layer (router, grouped top-k, expert FFN incl. shared, "
+                f"combine) for {m} seeded tokens of the {w.n}-token batch (each token routes "
+                "from its own row alone), timed as it runs")
+        if m == w.n:
+            what = f"per step: the whole {w.n}-token batch, timed as it runs"
+    else:
+        value, extrap = w.n / float(np.mean(full)), True
+        what = (f"per step: routing of all {w.n} tokens (it needs the whole batch) plus the "
+                f"expert FFN and combine of {m} seeded tokens; value extrapolates the FFN and "
+                f"combine to {w.n} tokens")
+    return value, sec, m, extrap, what + "; single-threaded C oracle, fp64 accumulation"
 
 
 def _host_inputs(w, inp=None):
@@ -721,52 +808,38 @@ def _host_inputs(w, inp=None):
     return X, Wg, lb, sb, weights, shared
 
 
-def cpu_baseline(w, inp=None, budget_s=20.0, sample=None):
-    X, Wg, lb, sb, weights, shared = _host_inputs(w, inp)
-    rng = np.random.default_rng(0)
-    if sample is None:
-        # size the FFN sample from a short probe so the whole leg takes ~budget_s
-        probe = sorted(rng.choice(w.n, size=min(8, w.n), replace=False).tolist())
-        t_route, t_ffn = _oracle_layer_sample(w, X, Wg, lb, sb, weights, shared, probe)
-        per_tok = t_ffn / len(probe)
-        sample = int(max(8, min(w.n, (budget_s - t_route) / max(per_tok, 1e-6))))
-    toks = sorted(rng.choice(w.n, size=min(sample, w.n), replace=False).tolist())
-    t_route, t_ffn = _oracle_layer_sample(w, X, Wg, lb, sb, weights, shared, toks)
-    est = t_route + t_ffn / len(toks) * w.n
-    return {"value": round(w.n / est, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": (f"routing of all {w.n} tokens ({t_route:.2f} s) + expert FFN and "
-                       f"combine of {len(toks)} seeded tokens ({t_ffn:.2f} s), extrapolated "
-                       f"to {w.n} tokens; single-threaded C oracle, fp64")}
+def cpu_baseline(w, inp=None, steps: int = 2):
+    """The GPU arm's cpu_baseline leg: the reference arm's oracle step (same
+    sample rule), `steps` times."""
+    value, sec, m, extrap, what = oracle_steps(w, _host_inputs(w, inp), steps)
+    return {"value": round(value, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{what}; mean of {steps} steps of {sec:.2f} s",
+            "tokens_per_step": m, "extrapolated": extrap}
 
 
 def run_reference(args, w):
+    """The reference arm: the oracle as it stands, on the host's cores."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    X, Wg, lb, sb, weights, shared = _host_inputs(w)
-    rng = np.random.default_rng(1)
-    sample = args.ref_sample
-    times = []
-    for i in range(args.warmup + args.steps):
-        toks = sorted(rng.choice(w.n, size=min(sample, w.n), replace=False).tolist())
-        t_route, t_ffn = _oracle_layer_sample(w, X, Wg, lb, sb, weights, shared, toks)
-        if i >= args.warmup:
-            times.append(t_route + t_ffn / len(toks) * w.n)
-    est = float(np.mean(times))
-    value = w.n / est
-    res = {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
+    host = _host_inputs(w)
+    t0 = time.perf_counter()
+    value, sec, m, extrap, what = oracle_steps(w, host, args.steps, args.warmup, seed=1)
+    wall = time.perf_counter() - t0
+    cb = {"value": round(value, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+          "sample": what, "tokens_per_step": m, "extrapolated": extrap}
+    res = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-           "ms_per_step": round(est * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+           "ms_per_step": round(sec * 1e3, 3), "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
-           "config": {"workload": w.name, "tokens": w.n, "d_model": w.d, "experts": w.E,
-                      "hidden": w.h},
-           "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": 1,
-                            "kind": "oracle",
-                            "sample": (f"per step: routing of all {w.n} tokens + expert FFN "
-                                       f"and combine of {sample} seeded tokens, extrapolated "
-                                       f"to {w.n}; single-threaded C oracle")},
-           "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+           "config": config_dict(w, world),
+           "tokens_per_step": m,
+           "ms_per_step_note": ("measured oracle time per step (its routing, FFN and combine; "
+                                "the conversion of the weights it reads is excluded)"),
+           "wall_s": round(wall, 2),
+           "cpu_baseline": cb,
+           "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0}}
     print(json.dumps(res), flush=True)
 
@@ -778,8 +851,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT.name, choices=sorted(wl.BY_NAME))
     ap.add_argument("--impl", default="libmoe", choices=["libmoe", "reference"])
-    ap.add_argument("--cpu-budget", type=float, default=20.0)
-    ap.add_argument("--ref-sample", type=int, default=48)
+    ap.add_argument("--cpu-budget", type=float, default=20.0,
+                    help="--pass train: seconds of the oracle's backward baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fused-combine", action="store_true",
                     help="forward: the combine inside the down projection's epilogue")

@@ -140,6 +140,15 @@ static moe_status check_route_out(const moe_config* c, const moe_route_out* o) {
   return MOE_OK;
 }
 
+moe_status route_call_check(const moe_config* c, const void* X, const float* Wg,
+                            const moe_route_out* o) {
+  Derived d;
+  moe_status st = derive(c, &d);
+  if (st != MOE_OK) return st;
+  if (!X || !Wg) return MOE_ERR_INVALID_ARG;
+  return check_route_out(c, o);
+}
+
 static moe_status check_ws(void* ws, size_t have, size_t need) {
   if (!ws) return MOE_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(ws) & 255) return MOE_ERR_WORKSPACE;
@@ -534,19 +543,26 @@ moe_status moe_combine(const moe_config* cfg, const void* Y_perm, const moe_rout
   return combine_impl(cfg, d, Y_perm, route, out, (cudaStream_t)stream);
 }
 
-moe_status moe_layer_forward(const moe_config* cfg, const void* X, const float* Wg,
-                             const float* logit_bias, const float* sel_bias, const void* W1,
-                             const void* W3, const void* W2, const void* sW1, const void* sW3,
-                             const void* sW2, void* out, moe_route_out* route, void* ws,
-                             size_t ws_bytes, moe_stream_t stream) {
-  Derived d;
-  moe_status st = derive(cfg, &d);
+// the layer's host-side checks: on a non-OK status nothing may be enqueued
+static moe_status layer_forward_check(const moe_config* cfg, Derived* d, WsLayout* w,
+                                      const void* X, const float* Wg, const void* out,
+                                      const void* W1, const void* W2,
+                                      const moe_route_out* route, void* ws, size_t ws_bytes) {
+  moe_status st = derive(cfg, d);
   if (st != MOE_OK) return st;
   if (!X || !Wg || !out || !W1 || !W2) return MOE_ERR_INVALID_ARG;
   if ((st = check_route_out(cfg, route)) != MOE_OK) return st;
-  const WsLayout w = ws_layout(cfg, d);
-  if ((st = check_ws(ws, ws_bytes, w.layer_end)) != MOE_OK) return st;
-  cudaStream_t s = (cudaStream_t)stream;
+  *w = ws_layout(cfg, *d);
+  return check_ws(ws, ws_bytes, w->layer_end);
+}
+
+static moe_status layer_forward_impl(const moe_config* cfg, const Derived& d, const WsLayout& w,
+                                     const void* X, const float* Wg, const float* logit_bias,
+                                     const float* sel_bias, const void* W1, const void* W3,
+                                     const void* W2, const void* sW1, const void* sW3,
+                                     const void* sW2, void* out, moe_route_out* route, void* ws,
+                                     cudaStream_t s) {
+  moe_status st;
   void* xp = at<void>(ws, w.xperm);
   void* hb = at<void>(ws, w.hbuf);
   void* yp = at<void>(ws, w.yperm);
@@ -561,6 +577,42 @@ moe_status moe_layer_forward(const moe_config* cfg, const void* X, const float* 
                      at<int>(ws, w.err), s)) != MOE_OK)
     return st;
   return combine_impl(cfg, d, yp, route, out, s);
+}
+
+moe_status moe_layer_forward(const moe_config* cfg, const void* X, const float* Wg,
+                             const float* logit_bias, const float* sel_bias, const void* W1,
+                             const void* W3, const void* W2, const void* sW1, const void* sW3,
+                             const void* sW2, void* out, moe_route_out* route, void* ws,
+                             size_t ws_bytes, moe_stream_t stream) {
+  Derived d;
+  WsLayout w;
+  moe_status st = layer_forward_check(cfg, &d, &w, X, Wg, out, W1, W2, route, ws, ws_bytes);
+  if (st != MOE_OK) return st;
+  return layer_forward_impl(cfg, d, w, X, Wg, logit_bias, sel_bias, W1, W3, W2, sW1, sW3, sW2,
+                            out, route, ws, (cudaStream_t)stream);
+}
+
+moe_status moe_layer_forward_host(const moe_config* cfg, const void* X_host, const float* Wg,
+                                  const float* logit_bias, const float* sel_bias,
+                                  const void* W1, const void* W3, const void* W2,
+                                  const void* sW1, const void* sW3, const void* sW2,
+                                  void* out_host, void* X_dev, void* out_dev,
+                                  moe_route_out* route, void* ws, size_t ws_bytes,
+                                  moe_stream_t stream) {
+  Derived d;
+  WsLayout w;
+  if (!X_host || !out_host) return MOE_ERR_INVALID_ARG;
+  moe_status st = layer_forward_check(cfg, &d, &w, X_dev, Wg, out_dev, W1, W2, route, ws,
+                                      ws_bytes);
+  if (st != MOE_OK) return st;
+  const size_t bytes = (size_t)cfg->n * cfg->d * (cfg->dtype == MOE_BF16 ? 2 : 4);
+  cudaStream_t s = (cudaStream_t)stream;
+  MOE_CU(cudaMemcpyAsync(X_dev, X_host, bytes, cudaMemcpyHostToDevice, s));
+  if ((st = layer_forward_impl(cfg, d, w, X_dev, Wg, logit_bias, sel_bias, W1, W3, W2, sW1, sW3,
+                               sW2, out_dev, route, ws, s)) != MOE_OK)
+    return st;
+  MOE_CU(cudaMemcpyAsync(out_host, out_dev, bytes, cudaMemcpyDeviceToHost, s));
+  return MOE_OK;
 }
 
 moe_status moe_expert_ffn_gathered(const moe_config* cfg, const void* X,
@@ -981,6 +1033,19 @@ moe_status moe_backward_workspace_size(const moe_config* cfg, size_t* bytes, int
   return MOE_OK;
 }
 
+moe_status moe_train_launch_counts(const moe_config* cfg, int* forward, int* backward) {
+  int r = 0, g = 0, f = 0, c = 0, b = 0;
+  moe_status st = moe_launch_counts(cfg, &r, &g, &f, &c);
+  if (st != MOE_OK) return st;
+  if ((st = moe_backward_workspace_size(cfg, nullptr, &b)) != MOE_OK) return st;
+  // bf16: the training forward also clears the dispatched rows' padding
+  // before its up projection, and the training backward skips the recompute
+  const int bf16 = cfg->dtype == MOE_BF16;
+  if (forward) *forward = r + g + f + c + bf16;
+  if (backward) *backward = b - bf16;
+  return MOE_OK;
+}
+
 static moe_status layer_backward_impl(const moe_config* cfg, const void* X, const float* Wg,
                                       const void* W1, const void* W3, const void* W2,
                                       const void* sW1, const void* sW3, const void* sW2,
@@ -1156,15 +1221,19 @@ moe_status moe_workspace_init(void* ws, moe_stream_t stream) {
 }
 
 moe_status moe_read_error(void* ws, moe_stream_t stream, int* detail) {
-  if (!ws) return MOE_ERR_WORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
   int code = 0;
   if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
-  if (cudaMemcpy(&code, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  const int zero = 0;
-  if (cudaMemcpy(ws, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  if (ws == nullptr) {
+    // no workspace: the word of moe_route_noalloc's static scratch
+    code = take_noalloc_error();
+  } else {
+    if (cudaMemcpy(&code, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpy(ws, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
   if (code == 0) code = take_dispatch_error();
   if (detail) *detail = code;
   if (code == 0) return MOE_OK;

@@ -167,6 +167,13 @@ struct GatherArgs {
 cudaError_t launch_gather(const GatherArgs& a, cudaStream_t s);
 // Reads and clears the error word of dispatch calls made without a workspace.
 int take_dispatch_error();
+// Reads and clears the error word of moe_route_noalloc's static scratch on the
+// current device (0 when that device has made no such call).
+int take_noalloc_error();
+// moe_route's host-side checks of the config, X, W_g and the route outputs
+// (those that need no workspace).
+moe_status route_call_check(const moe_config* c, const void* X, const float* Wg,
+                            const moe_route_out* o);
 
 struct CombineArgs {
   const void* Y;

@@ -37,7 +37,8 @@ API_SYMBOLS = ["moe_status_string", "moe_validate", "moe_sizes", "moe_workspace_
                "moe_combine", "moe_layer_forward", "moe_bias_update", "moe_workspace_init",
                "moe_read_error", "moe_route_noalloc", "moe_expert_ffn_gathered",
                "moe_launch_counts", "moe_backward_workspace_size", "moe_layer_backward",
-               "moe_expert_ffn_combined", "moe_layer_forward_train", "moe_layer_backward_train"]
+               "moe_expert_ffn_combined", "moe_layer_forward_train", "moe_layer_backward_train",
+               "moe_layer_forward_host", "moe_train_launch_counts"]
 MOE_ROUTE_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -92,6 +93,9 @@ def lib() -> ctypes.CDLL:
         L.moe_combine.argtypes = [cfgp, P, outp, P, P]
         L.moe_layer_forward.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, outp, P,
                                         ctypes.c_size_t, P]
+        L.moe_layer_forward_host.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P, outp,
+                                             P, ctypes.c_size_t, P]
+        L.moe_train_launch_counts.argtypes = [cfgp, ip, ip]
         L.moe_bias_update.argtypes = [cfgp, P, ctypes.c_float, P, P]
         L.moe_workspace_init.argtypes = [P, P]
         L.moe_read_error.argtypes = [P, P, ip]
@@ -192,6 +196,14 @@ def launch_counts(cfg: MoeConfig) -> dict:
     _check(lib().moe_launch_counts(ctypes.byref(cfg), *(ctypes.byref(v) for v in vals)),
            "moe_launch_counts")
     return dict(zip(("route", "dispatch", "ffn", "combine"), (v.value for v in vals)))
+
+
+def train_launch_counts(cfg: MoeConfig) -> tuple:
+    """Kernels of the training pair: (moe_layer_forward_train, moe_layer_backward_train)."""
+    f, b = ctypes.c_int(), ctypes.c_int()
+    _check(lib().moe_train_launch_counts(ctypes.byref(cfg), ctypes.byref(f), ctypes.byref(b)),
+           "moe_train_launch_counts")
+    return f.value, b.value
 
 
 def validate(cfg: MoeConfig) -> int:
@@ -306,6 +318,22 @@ def moe_layer_forward(cfg, X, Wg, logit_bias, sel_bias, W1, W3, W2, sW1, sW3, sW
            "moe_layer_forward")
 
 
+def moe_layer_forward_host(cfg, X_host, Wg, logit_bias, sel_bias, W1, W3, W2, sW1, sW3, sW2,
+                           out_host, X_dev, out_dev, route: RouteBuffers, ws, stream=None):
+    """moe_layer_forward on host X / out (CPU tensors, ideally pinned): the
+    library copies X_host into X_dev, runs the layer and copies out_dev back
+    into out_host, all on `stream`, without synchronising."""
+    for t in (X_host, out_host):
+        if t.is_cuda:
+            raise ValueError("X_host and out_host must be host tensors")
+    _check(lib().moe_layer_forward_host(ctypes.byref(cfg), _ptr(X_host), _ptr(Wg),
+                                        _ptr(logit_bias), _ptr(sel_bias), _ptr(W1), _ptr(W3),
+                                        _ptr(W2), _ptr(sW1), _ptr(sW3), _ptr(sW2),
+                                        _ptr(out_host), _ptr(X_dev), _ptr(out_dev),
+                                        ctypes.byref(route.c), _ptr(ws), ws.numel(),
+                                        _stream(stream)), "moe_layer_forward_host")
+
+
 def moe_bias_update(cfg, load, rate: float, bias, stream=None):
     _check(lib().moe_bias_update(ctypes.byref(cfg), _ptr(load), ctypes.c_float(rate),
                                  _ptr(bias), _stream(stream)), "moe_bias_update")
@@ -366,6 +394,8 @@ def moe_layer_backward_train(cfg, X, Wg, W1, W3, W2, sW1, sW3, sW2, route: Route
 
 
 def moe_read_error(ws, stream=None):
+    """(status, raw code) of the error word of `ws`; ws=None reads the word
+    of moe_route_noalloc's built-in scratch on the current device."""
     detail = ctypes.c_int()
     st = lib().moe_read_error(_ptr(ws), _stream(stream), ctypes.byref(detail))
     return st, detail.value

@@ -292,6 +292,28 @@ MOE_API moe_status moe_layer_forward(const moe_config* cfg, const void* X, const
                              moe_route_out* route, void* ws, size_t ws_bytes,
                              moe_stream_t stream);
 
+/* moe_layer_forward for a caller whose activations live in host memory:
+ * enqueues on `stream` one cudaMemcpyAsync of X_host [n,d] into X_dev, the
+ * whole layer on X_dev (as moe_layer_forward, writing out_dev), and one
+ * cudaMemcpyAsync of out_dev [n,d] back into out_host, all of the config's
+ * dtype. X_host and out_host should be page-locked (cudaHostAlloc or
+ * cudaHostRegister) so that the copies run asynchronously; pageable memory
+ * still gives correct results, with the copies synchronous to the host.
+ * X_dev and out_dev are caller-owned device buffers of n*d elements (16-byte
+ * aligned); nothing is allocated. out_host holds the result once the stream
+ * reaches the end of the call (the call itself does not synchronise). Every
+ * check of moe_layer_forward runs before the first copy is enqueued; a
+ * failed copy returns MOE_ERR_CUDA. The pages' problem statement ([EC-math]
+ * "The math") starts and ends on the device; the copies are the only
+ * addition. */
+MOE_API moe_status moe_layer_forward_host(const moe_config* cfg, const void* X_host,
+                                          const float* Wg, const float* logit_bias,
+                                          const float* sel_bias, const void* W1,
+                                          const void* W3, const void* W2, const void* sW1,
+                                          const void* sW3, const void* sW2, void* out_host,
+                                          void* X_dev, void* out_dev, moe_route_out* route,
+                                          void* ws, size_t ws_bytes, moe_stream_t stream);
+
 /* Selection-bias update after a step ([Guide] "4. Sigmoid gating with
  * aux-loss-free bias"): bias[e] -= rate * sign(load[e] - n K / E), in fp32;
  * load [E] int32 (from moe_route_out.load), bias [E] fp32 updated in place. */
@@ -309,9 +331,12 @@ MOE_API moe_status moe_bias_update(const moe_config* cfg, const int32_t* load, f
  * (moe_workspace_size's route_bytes) return MOE_ERR_WORKSPACE before
  * anything is enqueued. It calls no cudaMalloc, cudaFree or other allocating
  * routine. The first call on a device looks up the array's device address
- * and zeroes its error word (a synchronous cudaMemset); make that first call
- * before any stream capture. Every call shares the one array, so calls that
- * overlap on the GPU (on different streams or threads) race. */
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * Every call first zeroes the array's error word with a cudaMemsetAsync on
+ * `stream`, so the word reports that call's routing only; read it with
+ * moe_read_error(NULL, stream, &detail) after the call and before the next
+ * one. Every call shares the one array, so calls that overlap on the GPU (on
+ * different streams or threads) race. */
 #define MOE_ROUTE_NOALLOC_SCRATCH_BYTES (4u << 20)
 MOE_API moe_status moe_route_noalloc(const moe_config* cfg, const void* X, const float* Wg,
                                      const float* logit_bias, const float* sel_bias,
@@ -370,6 +395,12 @@ MOE_API moe_status moe_expert_ffn_combined(const moe_config* cfg, const void* X,
 MOE_API moe_status moe_backward_workspace_size(const moe_config* cfg, size_t* bytes,
                                                int* launches);
 
+/* Kernels the training pair enqueues for `cfg`: forward =
+ * moe_layer_forward_train's (moe_layer_forward's plus, for bf16, the clear of
+ * the dispatched rows' padding), backward = moe_layer_backward_train's.
+ * Either output may be NULL. No counterpart on the pages. */
+MOE_API moe_status moe_train_launch_counts(const moe_config* cfg, int* forward, int* backward);
+
 /* Arguments: the forward's inputs X, Wg, W1, W3, W2 (sW* for shared
  * experts, else NULL); `route`, the routing moe_layer_forward wrote (with
  * logits, and lse, filled when the score is sqrt(softplus) or token choice
@@ -426,8 +457,10 @@ MOE_API moe_status moe_workspace_init(void* ws, moe_stream_t stream);
 /* Synchronises `stream`, then reads and clears the error word at the start
  * of `ws` and, when that is clear, the current device's word for moe_dispatch
  * calls (which take no workspace): MOE_OK, MOE_ERR_TIMEOUT (a bounded wait
- * gave up) or MOE_ERR_CUDA. If detail != NULL it receives the raw device code
- * (0 = none). */
+ * gave up) or MOE_ERR_CUDA. With ws == NULL it reads and clears instead the
+ * error word of moe_route_noalloc's scratch array on the current device (a
+ * clear word if that device has made no such call), then the moe_dispatch
+ * word. If detail != NULL it receives the raw device code (0 = none). */
 MOE_API moe_status moe_read_error(void* ws, moe_stream_t stream, int* detail);
 
 #ifdef __cplusplus

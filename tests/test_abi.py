@@ -34,7 +34,7 @@ def declared_symbols():
 
 def test_every_declared_symbol_is_exported():
     syms = declared_symbols()
-    assert len(syms) == 21
+    assert len(syms) == 23
     assert sorted(moe.API_SYMBOLS) == syms
     L = ctypes.CDLL(moe.LIB_PATH)
     for s in syms:
@@ -170,7 +170,24 @@ def test_null_pointers_and_short_workspace_fail_before_launch():
     ec = moe.config(wl.EC_FP32)
     st = L.moe_bias_update(ctypes.byref(ec), _fake(0), ctypes.c_float(0.001), _fake(1), None)
     assert st == moe.MOE_ERR_INVALID_ARG
-    assert L.moe_read_error(None, None, None) == moe.MOE_ERR_WORKSPACE
+    # host buffers: the host pointers are checked, then everything moe_layer_forward checks
+    lw = sz.layer_ws
+    st = L.moe_layer_forward_host(ctypes.byref(cfg), None, _fake(1), None, None, _fake(3),
+                                  _fake(4), _fake(5), None, None, None, _fake(6), _fake(7),
+                                  _fake(8), ctypes.byref(out), _fake(2), lw, None)
+    assert st == moe.MOE_ERR_INVALID_ARG
+    st = L.moe_layer_forward_host(ctypes.byref(cfg), _fake(0), _fake(1), None, None, _fake(3),
+                                  _fake(4), _fake(5), None, None, None, _fake(6), None,
+                                  _fake(8), ctypes.byref(out), _fake(2), lw, None)
+    assert st == moe.MOE_ERR_INVALID_ARG  # no device copy of X
+    st = L.moe_layer_forward_host(ctypes.byref(cfg), _fake(0), _fake(1), None, None, _fake(3),
+                                  _fake(4), _fake(5), None, None, None, _fake(6), _fake(7),
+                                  _fake(8), ctypes.byref(out), _fake(2), lw - 1, None)
+    assert st == moe.MOE_ERR_WORKSPACE
+    if not torch.cuda.is_available():
+        # no workspace: the no-alloc routing scratch's word, after a stream
+        # synchronise that cannot succeed without a device
+        assert L.moe_read_error(None, None, None) == moe.MOE_ERR_CUDA
 
 
 def test_binding_refuses_to_run_without_library(monkeypatch, tmp_path):
@@ -191,6 +208,18 @@ def test_launch_counts():
     decode = moe.launch_counts(moe.config(wl.DECODE))
     assert decode["route"] == 5
     assert moe.launch_counts(moe.config(wl.TC_SIGMOID_GROUPED))["ffn"] == 2
+
+
+def test_train_launch_counts():
+    """The training forward enqueues the layer's kernels plus, for bf16, the
+    clear of the dispatched rows' padding; the training backward one fewer
+    than moe_layer_backward for bf16 (no recompute of the up projection)."""
+    for w in (wl.EC_FP32, wl.EC_BF16, wl.TC_DROPLESS, wl.TC_SIGMOID_GROUPED):
+        cfg = moe.config(w)
+        f, b = moe.train_launch_counts(cfg)
+        bf16 = int(w.dtype == "bf16")
+        assert f == sum(moe.launch_counts(cfg).values()) + bf16, w.name
+        assert b == _bwd_size(cfg)[2] - bf16, w.name
 
 
 def _bwd_size(cfg):

@@ -16,22 +16,57 @@ def test_cpu_baseline_covers_shared_experts():
     w = wl.SMALL[4]  # grouped sigmoid routing with a shared expert
     assert w.n_shared == 1
     inp = wl.make_inputs(w, "cpu")
-    res = bench.cpu_baseline(w, inp, budget_s=2.0)
+    res = bench.cpu_baseline(w, inp, steps=1)
     assert res["kind"] == "oracle" and res["cores"] == 1 and res["value"] > 0
+    assert res["tokens_per_step"] == bench.oracle_sample_tokens(w)
+
+
+def test_oracle_sample_rule():
+    """One rule sizes both CPU legs: about 8 GFLOP of expert FFN per step,
+    the whole batch when that is less; token choice without a capacity
+    routes each token alone, so its steps need no extrapolation."""
+    assert bench.oracle_sample_tokens(wl.EC_FP32) == wl.EC_FP32.n
+    for w in wl.FULL[1:]:
+        m = bench.oracle_sample_tokens(w)
+        assert 4 <= m < w.n
+    assert bench.routes_per_token(wl.TC_SIGMOID_GROUPED)
+    assert bench.routes_per_token(wl.TC_DROPLESS)
+    assert not bench.routes_per_token(wl.TC_TOP2_CAP)  # capacity: needs the whole batch
+    assert not bench.routes_per_token(wl.EC_BF16)
+
+
+def test_sampled_oracle_step_equals_full_batch_rows():
+    """Routing a sample of tokens alone gives those tokens the same layer
+    output as routing the whole batch (token choice without a capacity), so
+    the reference arm's sampled step is the layer on those tokens."""
+    import numpy as np
+    import oracle
+    w = wl.SMALL[4]
+    X, Wg, lb, sb, weights, shared = bench._host_inputs(w, wl.make_inputs(w, "cpu"))
+    spec = oracle.spec_of(w)
+    toks = [3, 17, 150, 299]
+    _, S, lse = oracle.router(X, Wg, lb, spec["score"])
+    full = oracle.layer_forward(spec, X, oracle.route(spec, S, lse, sb), weights, shared,
+                                tokens=toks)
+    _, S2, lse2 = oracle.router(X[toks], Wg, lb, spec["score"])
+    part = oracle.layer_forward(spec, X[toks], oracle.route(spec, S2, lse2, sb), weights, shared)
+    np.testing.assert_array_equal(full, part)
 
 
 def test_reference_arm_prints_one_json_line():
     w = wl.SMALL[4]
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                          "--workload", w.name, "--steps", "1", "--warmup", "3",
-                          "--ref-sample", "4"],
+                          "--workload", w.name, "--steps", "2", "--warmup", "3"],
                          capture_output=True, text=True, timeout=600, cwd=ROOT, check=True)
     lines = [l for l in out.stdout.splitlines() if l.strip()]
     assert len(lines) == 1
     j = json.loads(lines[0])
-    assert j["impl"] == "reference" and j["config"]["workload"] == w.name
+    assert j["impl"] == "reference" and j["config"] == bench.config_dict(w, 1)
     assert j["value"] > 0 and j["cpu_baseline"]["kind"] == "oracle"
     assert j["e2e"]["h2d_bytes_per_step"] == 0
+    # ms_per_step is time that elapsed: the timed steps fit in the run
+    assert j["ms_per_step"] * j["steps"] / 1e3 <= j["wall_s"]
+    assert j["tokens_per_step"] == bench.oracle_sample_tokens(w)
 
 
 def test_training_cpu_baseline_and_flop_count():

@@ -63,6 +63,10 @@ def test_noalloc_route_matches_workspace_route(w):
         assert st == moe.MOE_OK, moe.status_string(st)
         torch.cuda.synchronize()
         _compare(ref, got)
+        # the routing left the scratch array's error word clear; a NULL
+        # workspace reads (and clears) that word
+        st, detail = moe.moe_read_error(None)
+        assert st == moe.MOE_OK and detail == 0
 
 
 def test_noalloc_refuses_configs_beyond_its_scratch():
