@@ -232,6 +232,7 @@ static moe_status finish_route(const moe_config* c, const Derived& dv, const WsL
   a.lse_blocks = colsum_blocks;
   a.lb_coef = c->lb_coef;
   a.z_coef = c->z_coef;
+  a.err = err;
   MOE_CU(launch_tc_assign(a, s));
   return MOE_OK;
 }
@@ -289,10 +290,12 @@ bool ffn_uses_pair(const moe_config* c, const Derived& dv) {
 }
 
 // Fine-grained token choice (128 to 512 rows per expert on average): the
-// weights-as-M down projection computes each expert's exact token count
-// (16-row granularity) where the 128-row tiles would round ~256 rows up to
-// 384 or 512. It needs the counts, which the caller passes. The up
-// projection stays on the token-side kernels, which measured faster there.
+// weights-as-M projections compute each expert's exact token count (16-row
+// granularity) where the 128-row tiles would round ~256 rows up to 384 or
+// 512. They need the counts, which the caller passes. The SwiGLU up
+// projection takes W1 and W3 as two A operands into two accumulators; other
+// activations, the fused gather and the training forward's kept U and V
+// keep the up projection on the token-side kernels.
 static bool ffn_uses_swap(const moe_config* c, const Derived& dv) {
   if (c->dtype != MOE_BF16 || c->mode != MOE_TOKEN_CHOICE) return false;
   const long long avg = avg_expert_rows(c, dv);
@@ -348,8 +351,13 @@ static moe_status ffn_impl(const moe_config* c, const Derived& dv, const void* X
   f.save_v = save_v;
   if (c->dtype != MOE_BF16) return out32 ? MOE_ERR_UNSUPPORTED : run_ffn_f32(f, s);
   if (!out32 && ffn_uses_swap(c, dv) && swap_down_supported(f)) {
-    f.skip_down = true;
-    const moe_status st = run_ffn_bf16(f, s);
+    moe_status st;
+    if (swap_up_supported(f)) {
+      st = run_ffn_up_swap(f, s);
+    } else {
+      f.skip_down = true;
+      st = run_ffn_bf16(f, s);
+    }
     if (st != MOE_OK) return st;
     return run_ffn_down_swap(f, s);
   }
@@ -381,8 +389,10 @@ static moe_status dispatch_impl(const moe_config* c, const Derived& dv, const vo
   return MOE_OK;
 }
 
+// err: the workspace error word, or NULL (standalone moe_combine)
 static moe_status combine_impl(const moe_config* c, const Derived& dv, const void* Y,
-                               const moe_route_out* o, void* out, cudaStream_t s) {
+                               const moe_route_out* o, void* out, cudaStream_t s,
+                               int* err = nullptr) {
   CombineArgs a{};
   a.Y = Y;
   a.tok_row = o->tok_row;
@@ -396,6 +406,7 @@ static moe_status combine_impl(const moe_config* c, const Derived& dv, const voi
   a.shared_base = dv.shared_base;
   a.max_rows = dv.rows_routed;
   a.out = out;
+  a.err = err;
   MOE_CU(launch_combine(a, s));
   return MOE_OK;
 }
@@ -576,7 +587,7 @@ static moe_status layer_forward_impl(const moe_config* cfg, const Derived& d, co
                      sW3, sW2, hb, yp,
                      at<int>(ws, w.err), s)) != MOE_OK)
     return st;
-  return combine_impl(cfg, d, yp, route, out, s);
+  return combine_impl(cfg, d, yp, route, out, s, at<int>(ws, w.err));
 }
 
 moe_status moe_layer_forward(const moe_config* cfg, const void* X, const float* Wg,
@@ -646,8 +657,8 @@ moe_status moe_expert_ffn_combined(const moe_config* cfg, const void* X, const v
     return MOE_ERR_INVALID_ARG;
   if ((st = check_ws(ws, ws_bytes, MOE_WS_ERROR_BYTES)) != MOE_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
-  MOE_CU(launch_combine_prep(route->tok_row, route->tok_gate, cfg->n, d.slots, cfg->d, row_gate,
-                             acc, s));
+  MOE_CU(launch_combine_prep(route->tok_row, route->tok_gate, cfg->n, d.slots, cfg->d,
+                             d.rows_routed, row_gate, acc, at<int>(ws, 0), s));
   if ((st = ffn_impl(cfg, d, X, X_perm, route->row_token, route->offsets, nullptr, W1, W3, W2,
                      sW1, sW3, sW2, H, nullptr, at<int>(ws, 0), s, row_gate, acc)) != MOE_OK)
     return st;
@@ -1122,6 +1133,8 @@ static moe_status layer_backward_impl(const moe_config* cfg, const void* X, cons
   cb.z_coef = tc ? cfg->z_coef : 0.0f;
   cb.dY_perm = dy;
   cb.dL = dl;
+  cb.max_rows = d.rows_routed;
+  cb.err = err;
   MOE_CU(launch_combine_backward(cb, s));
 
   const BwdBufs bufs{xp, dy, U, V, H, duv, dxp, saved && bf16};
@@ -1147,6 +1160,8 @@ static moe_status layer_backward_impl(const moe_config* cfg, const void* X, cons
   rb.n_pad = d.n_pad;
   rb.dX = dX;
   rb.dWg = dWg;
+  rb.max_rows = d.rows_routed;
+  rb.err = err;
   rb.partial = at<float>(ws, b.part);
   rb.splits = b.splits;
   MOE_CU(launch_router_backward(rb, s));
@@ -1211,8 +1226,10 @@ moe_status moe_layer_forward_train(const moe_config* cfg, const void* X, const f
   if ((st = ffn_impl(cfg, d, X, xp, nullptr, route->offsets, route->counts, W1, W3, W2, sW1,
                      sW3, sW2, H, yp, at<int>(ws, w.err), s, nullptr, nullptr, U, V)) != MOE_OK)
     return st;
-  return combine_impl(cfg, d, yp, route, out, s);
+  return combine_impl(cfg, d, yp, route, out, s, at<int>(ws, w.err));
 }
+
+moe_status moe_debug_inject_fault(moe_fault fault) { return set_fault((int)fault); }
 
 moe_status moe_workspace_init(void* ws, moe_stream_t stream) {
   if (!ws) return MOE_ERR_WORKSPACE;

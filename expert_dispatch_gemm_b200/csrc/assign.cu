@@ -359,7 +359,10 @@ __global__ void __launch_bounds__(kTokBlock) tc_hist_kernel(TcAssignArgs a) {
   if (t < a.n)
     for (int j = 0; j < a.K; ++j) {
       const int e = a.idx[(size_t)t * a.K + j];
-      if ((unsigned)e < (unsigned)a.E) atomicAdd(&hist[e], 1);
+      if ((unsigned)e < (unsigned)a.E)
+        atomicAdd(&hist[e], 1);
+      else
+        bad_index(a.err, kSiteScatterIdx);
     }
   __syncthreads();
   for (int i = threadIdx.x; i < a.E; i += kTokBlock)

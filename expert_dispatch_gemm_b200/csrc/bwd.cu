@@ -124,7 +124,11 @@ __global__ void __launch_bounds__(256) combine_backward_kernel(CombineBwdArgs a)
   for (int e = tid; e < a.E; e += 256) dS_s[e] = 0.0f;
   __syncthreads();
   for (int j = tid; j < slots; j += 256) {
-    const int r = a.tok_row[(size_t)t * slots + j];
+    int r = a.tok_row[(size_t)t * slots + j];
+    if (r < -1 || r >= a.max_rows) {
+      bad_index(a.err, kSiteBwdTokRow);
+      r = -1;
+    }
     rows_s[j] = r;
     gates_s[j] = a.tok_gate[(size_t)t * slots + j];
     if (r < 0) atomicMin(&cnt_s, j);
@@ -318,7 +322,13 @@ __global__ void __launch_bounds__(256) router_dx_kernel(RouterBwdArgs a) {
     for (int j = 0; j < a.slots; j += 4) {
       int r[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) r[u] = j + u < a.slots ? tr[j + u] : -1;
+      for (int u = 0; u < 4; ++u) {
+        r[u] = j + u < a.slots ? tr[j + u] : -1;
+        if (r[u] < -1 || r[u] >= a.max_rows) {
+          bad_index(a.err, kSiteBwdTokRow);
+          r[u] = -1;
+        }
+      }
       float x[4][4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {

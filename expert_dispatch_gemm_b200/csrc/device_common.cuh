@@ -46,6 +46,39 @@ __device__ __forceinline__ void report_error(int* err, int code) {
   if (err) atomicCAS(err, 0, code);
 }
 
+// Index checks. Every build skips an index read from the routing outputs
+// (row_token, tok_row, offsets, counts, idx) that lies outside its range
+// instead of reading or writing through it. The checked build
+// (-DMOE_DEBUG_CHECKS, libmoe_checked.so) also reports each such index as
+// kErrBadIndex | site in the error word, where moe_read_error finds it; the
+// default build compiles the report away.
+#ifdef MOE_DEBUG_CHECKS
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+
+enum : int {
+  kSiteGatherTokRow = 0x01,
+  kSiteGatherRowToken = 0x02,
+  kSiteGatherOffsets = 0x03,
+  kSiteCombineTokRow = 0x04,
+  kSiteCombinePrepTokRow = 0x05,
+  kSiteGemmOffsets = 0x10,
+  kSiteGemmPairOffsets = 0x11,
+  kSiteGemmGatherToken = 0x12,
+  kSiteGemmScatterToken = 0x13,
+  kSiteSwapOffsets = 0x20,
+  kSiteScatterIdx = 0x30,
+  kSiteEcFinishIdx = 0x31,
+  kSiteBwdTokRow = 0x40,
+  kSiteBwdOffsets = 0x41,
+};
+
+__device__ __forceinline__ void bad_index(int* err, int site) {
+  if (kDebugChecks) report_error(err, kErrBadIndex | site);
+}
+
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

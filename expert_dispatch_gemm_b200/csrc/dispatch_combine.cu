@@ -109,6 +109,8 @@ __global__ void gather_kernel(GatherArgs a, int seg, int nseg, int ring, int slo
       const int r = rr[c];
       if (r >= 0 && r < a.max_rows)
         sm100::bulk_store_global(XP + (size_t)r * row_bytes + (size_t)sg * seg, src, b);
+      else if (r < -1 || r >= a.max_rows)
+        bad_index(err, kSiteGatherTokRow);
     }
     sm100::bulk_commit_group();
     sm100::bulk_wait_read_all();
@@ -136,7 +138,11 @@ constexpr int kRowsPerWarp = 4;
 
 __global__ void __launch_bounds__(256) gather_rows_kernel(GatherArgs a) {
   pdl_wait();
-  const long long rows = min((long long)a.offsets[a.E], a.max_rows);
+  int* err = a.err ? a.err : &g_dispatch_error;
+  const long long used = a.offsets[a.E];
+  const long long rows = min(used, a.max_rows);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && (used < 0 || used > a.max_rows))
+    bad_index(err, kSiteGatherOffsets);
   const int lane = threadIdx.x & 31;
   const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
@@ -150,6 +156,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(GatherArgs a) {
       const long long r = r0 + i;
       const int t = r < rows ? a.row_token[r] : -1;
       tok[i] = (t >= 0 && t < a.n) ? t : -1;
+      if (t < -1 || t >= a.n) bad_index(err, kSiteGatherRowToken);
     }
     for (int v0 = 0; v0 < nvec; v0 += 128) {
       uint4 x[kRowsPerWarp][4];
@@ -229,7 +236,10 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
   __syncthreads();
   for (int j = threadIdx.x; j < slots; j += blockDim.x) {
     int r = a.tok_row[(size_t)t * slots + j];
-    if (r >= a.max_rows) r = -1;
+    if (r < -1 || r >= a.max_rows) {
+      bad_index(a.err ? a.err : &g_dispatch_error, kSiteCombineTokRow);
+      r = -1;
+    }
     rows_s[j] = r;
     gates_s[j] = a.tok_gate[(size_t)t * slots + j];
     if (r < 0) atomicMin(&cnt_s, j);
@@ -290,14 +300,18 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
 // rounded into the output.
 __global__ void __launch_bounds__(256) combine_prep_kernel(const int32_t* tok_row,
                                                            const float* tok_gate, int n,
-                                                           int slots, int d, float* row_gate,
-                                                           float* out32) {
+                                                           int slots, int d, long long max_rows,
+                                                           float* row_gate, float* out32,
+                                                           int* err) {
   pdl_wait();
   const long long tid = (long long)blockIdx.x * 256 + threadIdx.x;
   const long long nthreads = (long long)gridDim.x * 256;
   for (long long q = tid; q < (long long)n * slots; q += nthreads) {
     const int r = tok_row[q];
-    if (r >= 0) row_gate[r] = tok_gate[q];
+    if (r >= 0 && r < max_rows)
+      row_gate[r] = tok_gate[q];
+    else if (r < -1 || r >= max_rows)
+      bad_index(err ? err : &g_dispatch_error, kSiteCombinePrepTokRow);
   }
   const long long nvec = (long long)n * d / 4;
   const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -325,9 +339,10 @@ static int fill_grid() {
 }
 
 cudaError_t launch_combine_prep(const int32_t* tok_row, const float* tok_gate, int n, int slots,
-                                int d, float* row_gate, float* out32, cudaStream_t s) {
+                                int d, long long max_rows, float* row_gate, float* out32,
+                                int* err, cudaStream_t s) {
   return launch_pdl(combine_prep_kernel, fill_grid(), 256, 0, s, tok_row, tok_gate, n, slots, d,
-                    row_gate, out32);
+                    max_rows, row_gate, out32, err);
 }
 
 cudaError_t launch_combine_finish(const float* out32, int n, int d, void* out, cudaStream_t s) {

@@ -25,6 +25,7 @@
 #include <cuda.h>
 #include <math.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "device_common.cuh"
@@ -67,9 +68,10 @@ struct TcGemmParams {
   const int32_t* row_token;  // source token of each dispatched row (gathered A, scatter)
   const float* row_gate;     // scatter: gate of each dispatched row
   float* out32;              // scatter: [n_tok, n_out] fp32 sums
-  int n_tok;
+  int n_tok;                 // tokens (rows of X and out32)
   __nv_bfloat16* save_u;     // save: [rows, n_out] pre-activations U = X W1^T
   __nv_bfloat16* save_v;     // save (SwiGLU): [rows, n_out] V = X W3^T
+  int inject_no_loads;       // failure-path test: the producer issues no loads
 };
 
 struct SharedState {
@@ -224,9 +226,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int run = 0;
     for (int e = 0; e < p.E; ++e) {
       st->tprefix[e] = run;
-      run += max(st->offs[e + 1] - st->offs[e], 0) / kBM * p.nt_tiles;
+      const int seg = st->offs[e + 1] - st->offs[e];
+      if (seg < 0 || (st->offs[e] % kBM) != 0) bad_index(p.err, kSiteGemmOffsets);
+      run += max(seg, 0) / kBM * p.nt_tiles;
     }
     st->tprefix[p.E] = run;
+    if (st->offs[p.E] > p.max_routed_tiles * kBM) bad_index(p.err, kSiteGemmOffsets);
   }
   sm100::tc_fence_before();
   __syncthreads();
@@ -255,7 +260,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int tok[4] = {0, 0, 0, 0};
       if (gather) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) tok[j] = max(p.row_token[c.a_row + 4 * lane + j], 0);
+        for (int j = 0; j < 4; ++j) {
+          const int t = p.row_token[c.a_row + 4 * lane + j];
+          if (t < -1 || t >= p.n_tok) bad_index(p.err, kSiteGemmGatherToken);
+          tok[j] = (t >= 0 && t < p.n_tok) ? t : 0;
+        }
       }
       for (int kb = 0; kb < KB; ++kb) {
         int okw = 1;
@@ -267,20 +276,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         unsigned char* a_dst = sA + stage * kABytes;
         unsigned char* b_dst = sB + stage * kBBytes;
-        if (lane == 0) {
-          sm100::mbar_arrive_expect_tx(&st->full[stage], kStageBytes);
-          if (!gather) sm100::tma_load_2d(a_dst, ma, &st->full[stage], kb * kBK, c.a_row);
-          if (SWIGLU) {
-            sm100::tma_load_2d(b_dst, mb, &st->full[stage], kb * kBK, c.b_row);
-            sm100::tma_load_2d(b_dst + kBBytes / 2, mbg, &st->full[stage], kb * kBK, c.b_row);
-          } else {
-            sm100::tma_load_2d(b_dst, mb, &st->full[stage], kb * kBK, c.b_row);
+        // (a failure-path test withholds every load: the MMA warp's bounded
+        // wait on this stage then runs out)
+        if (!p.inject_no_loads) {
+          if (lane == 0) {
+            sm100::mbar_arrive_expect_tx(&st->full[stage], kStageBytes);
+            if (!gather) sm100::tma_load_2d(a_dst, ma, &st->full[stage], kb * kBK, c.a_row);
+            if (SWIGLU) {
+              sm100::tma_load_2d(b_dst, mb, &st->full[stage], kb * kBK, c.b_row);
+              sm100::tma_load_2d(b_dst + kBBytes / 2, mbg, &st->full[stage], kb * kBK, c.b_row);
+            } else {
+              sm100::tma_load_2d(b_dst, mb, &st->full[stage], kb * kBK, c.b_row);
+            }
           }
+          if (gather)
+            sm100::tma_gather4(a_dst + lane * 4 * (kBK * 2), &tmXg, &st->full[stage], kb * kBK,
+                               tok[0], tok[1], tok[2], tok[3]);
+          ++issued;
         }
-        if (gather)
-          sm100::tma_gather4(a_dst + lane * 4 * (kBK * 2), &tmXg, &st->full[stage], kb * kBK,
-                             tok[0], tok[1], tok[2], tok[3]);
-        ++issued;
         if (++stage == kStages) {
           stage = 0;
           phase ^= 1u;
@@ -372,6 +385,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const long long r = c.out_row + row_in_tile;
         if (c.a_sel == 0) {
           tok = p.row_token[r];
+          if (tok < -1 || tok >= p.n_tok) {
+            bad_index(p.err, kSiteGemmScatterToken);
+            tok = -1;
+          }
           gate = tok >= 0 ? p.row_gate[r] : 0.0f;
         } else {
           const long long q2 = (r - p.out_shared_base) % p.n_pad;
@@ -597,10 +614,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     int run = 0;
     for (int e = 0; e < p.E; ++e) {
       st->tprefix[e] = run;
-      const int cnt = max(st->offs[e + 1] - st->offs[e], 0) / kBM;
+      const int seg = st->offs[e + 1] - st->offs[e];
+      if (seg < 0 || (st->offs[e] % kBM) != 0) bad_index(p.err, kSiteGemmPairOffsets);
+      const int cnt = max(seg, 0) / kBM;
       run += (cnt + 1) / 2 * p.nt_tiles;
     }
     st->tprefix[p.E] = run;
+    if (st->offs[p.E] > p.max_routed_tiles * kBM) bad_index(p.err, kSiteGemmPairOffsets);
   }
   sm100::tc_fence_before();
   __syncthreads();
@@ -635,7 +655,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int tok[4] = {0, 0, 0, 0};
       if (gather) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) tok[j] = max(p.row_token[c.a_row + 4 * lane + j], 0);
+        for (int j = 0; j < 4; ++j) {
+          const int t = p.row_token[c.a_row + 4 * lane + j];
+          if (t < -1 || t >= p.n_tok) bad_index(p.err, kSiteGemmGatherToken);
+          tok[j] = (t >= 0 && t < p.n_tok) ? t : 0;
+        }
       }
       for (int kb = 0; kb < KB; ++kb) {
         int okw = 1;
@@ -746,6 +770,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const long long r = c.out_row + row_in_tile;
         if (c.a_sel == 0) {
           tok = p.row_token[r];
+          if (tok < -1 || tok >= p.n_tok) {
+            bad_index(p.err, kSiteGemmScatterToken);
+            tok = -1;
+          }
           gate = tok >= 0 ? p.row_gate[r] : 0.0f;
         } else {
           const long long q2 = (r - p.out_shared_base) % p.n_pad;
@@ -915,6 +943,22 @@ static int persistent_grid(const TcGemmParams& p, bool pair) {
   return g < 1 ? 1 : (int)g;
 }
 
+// One-shot failure-path test hooks (moe_debug_inject_fault): armed on the
+// host, taken by the next up projection that can honour them.
+static std::atomic<int> g_fault{0};
+
+moe_status set_fault(int fault) {
+  if (fault < MOE_FAULT_NONE || fault > MOE_FAULT_LAUNCH) return MOE_ERR_INVALID_ARG;
+  g_fault.store(fault);
+  return MOE_OK;
+}
+
+// the armed fault if it is `kind` (then disarmed), else MOE_FAULT_NONE
+static int take_fault(int kind) {
+  int want = kind;
+  return g_fault.compare_exchange_strong(want, MOE_FAULT_NONE) ? kind : MOE_FAULT_NONE;
+}
+
 moe_status run_ffn_bf16(const FfnArgs& f, cudaStream_t s) {
   const bool swiglu = f.act == MOE_ACT_SWIGLU;
   const bool pair = f.pair;
@@ -978,8 +1022,13 @@ moe_status run_ffn_bf16(const FfnArgs& f, cudaStream_t s) {
   p.out = static_cast<__nv_bfloat16*>(f.H);
   p.err = f.err;
   p.row_token = f.row_token;
+  p.n_tok = f.n;
   p.save_u = static_cast<__nv_bfloat16*>(f.save_u);
   p.save_v = static_cast<__nv_bfloat16*>(f.save_v);
+  // failure-path tests: a launch that fails on the host, or (single-CTA
+  // kernel) a producer that issues no loads
+  if (take_fault(MOE_FAULT_LAUNCH) == MOE_FAULT_LAUNCH) return MOE_ERR_CUDA;
+  if (!pair) p.inject_no_loads = take_fault(MOE_FAULT_GEMM_NO_LOADS) == MOE_FAULT_GEMM_NO_LOADS;
   cudaError_t e = cudaSuccess;
   const int grid_up = persistent_grid(p, pair);
   switch (f.act) {
@@ -1006,6 +1055,7 @@ moe_status run_ffn_bf16(const FfnArgs& f, cudaStream_t s) {
   dm.xg = dm.a0;
   TcGemmParams q = p;
   q.save_u = q.save_v = nullptr;
+  q.inject_no_loads = 0;
   q.K = f.h;
   q.n_out = f.d;
   q.nt_tiles = ceil_div(f.d, kBN);

@@ -149,6 +149,7 @@ struct TcAssignArgs {
   const double* lse2;   // or NULL
   int lse_blocks;
   float lb_coef, z_coef;
+  int* err;             // device error word
 };
 cudaError_t launch_tc_assign(const TcAssignArgs& a, cudaStream_t s);
 
@@ -170,6 +171,8 @@ int take_dispatch_error();
 // Reads and clears the error word of moe_route_noalloc's static scratch on the
 // current device (0 when that device has made no such call).
 int take_noalloc_error();
+// Arms a one-shot failure-path test fault (moe_debug_inject_fault).
+moe_status set_fault(int fault);
 // moe_route's host-side checks of the config, X, W_g and the route outputs
 // (those that need no workspace).
 moe_status route_call_check(const moe_config* c, const void* X, const float* Wg,
@@ -183,6 +186,7 @@ struct CombineArgs {
   long long shared_base;
   long long max_rows;   // routed rows bound; larger slot entries are ignored
   void* out;
+  int* err;             // device error word, or NULL for the module's own
 };
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 
@@ -214,6 +218,9 @@ moe_status run_ffn_bf16(const FfnArgs& a, cudaStream_t s);
 // the weights-as-M down projection for fine-grained experts (needs the counts)
 bool swap_down_supported(const FfnArgs& a);
 moe_status run_ffn_down_swap(const FfnArgs& a, cudaStream_t s);
+// the weights-as-M SwiGLU up projection (W1 and W3 as two A operands)
+bool swap_up_supported(const FfnArgs& a);
+moe_status run_ffn_up_swap(const FfnArgs& a, cudaStream_t s);
 moe_status run_ffn_f32(const FfnArgs& a, cudaStream_t s);
 
 // ----- backward pass -----
@@ -303,6 +310,8 @@ struct CombineBwdArgs {
   float lb_coef, z_coef;
   void* dY_perm;                 // [rows, d]: kept rows written
   float* dL;                     // [n, E]
+  long long max_rows;            // routed rows bound; larger tok_row entries are skipped
+  int* err;                      // device error word
 };
 cudaError_t launch_combine_backward(const CombineBwdArgs& a, cudaStream_t s);
 // zero rows [offsets[e] + counts[e], offsets[e+1]) of two [rows, row_bytes] buffers
@@ -322,6 +331,8 @@ struct RouterBwdArgs {
   float* dWg;                    // [d, E]
   float* partial;                // [splits, d, E]
   int splits;
+  long long max_rows;            // routed rows bound; larger tok_row entries are skipped
+  int* err;                      // device error word
 };
 int router_bwd_splits(int n, int d, int E);
 cudaError_t launch_router_backward(const RouterBwdArgs& a, cudaStream_t s);
@@ -329,7 +340,8 @@ cudaError_t launch_router_backward(const RouterBwdArgs& a, cudaStream_t s);
 // the fused combine's bookkeeping: zero out32 [n, d] and write each
 // dispatched row's gate; then round out32 into the output
 cudaError_t launch_combine_prep(const int32_t* tok_row, const float* tok_gate, int n, int slots,
-                                int d, float* row_gate, float* out32, cudaStream_t s);
+                                int d, long long max_rows, float* row_gate, float* out32,
+                                int* err, cudaStream_t s);
 cudaError_t launch_combine_finish(const float* out32, int n, int d, void* out, cudaStream_t s);
 
 cudaError_t launch_bias_update(int n, int E, int K, const int32_t* load, float rate,

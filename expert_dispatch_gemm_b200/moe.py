@@ -17,6 +17,11 @@ from .workloads import Workload
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmoe.so")
+# the checked build (every out-of-range routing index reported in the error
+# word); MOE_LIBRARY=checked in the environment loads it instead
+CHECKED_LIB_PATH = os.path.join(_PKG, "libmoe_checked.so")
+if os.environ.get("MOE_LIBRARY") == "checked":
+    LIB_PATH = CHECKED_LIB_PATH
 
 # enums and limits of include/moe.h
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, \
@@ -38,7 +43,8 @@ API_SYMBOLS = ["moe_status_string", "moe_validate", "moe_sizes", "moe_workspace_
                "moe_read_error", "moe_route_noalloc", "moe_expert_ffn_gathered",
                "moe_launch_counts", "moe_backward_workspace_size", "moe_layer_backward",
                "moe_expert_ffn_combined", "moe_layer_forward_train", "moe_layer_backward_train",
-               "moe_layer_forward_host", "moe_train_launch_counts"]
+               "moe_layer_forward_host", "moe_train_launch_counts", "moe_debug_inject_fault"]
+MOE_FAULT_NONE, MOE_FAULT_GEMM_NO_LOADS, MOE_FAULT_LAUNCH = 0, 1, 2
 MOE_ROUTE_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -96,6 +102,7 @@ def lib() -> ctypes.CDLL:
         L.moe_layer_forward_host.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P, outp,
                                              P, ctypes.c_size_t, P]
         L.moe_train_launch_counts.argtypes = [cfgp, ip, ip]
+        L.moe_debug_inject_fault.argtypes = [ctypes.c_int]
         L.moe_bias_update.argtypes = [cfgp, P, ctypes.c_float, P, P]
         L.moe_workspace_init.argtypes = [P, P]
         L.moe_read_error.argtypes = [P, P, ip]
@@ -391,6 +398,11 @@ def moe_layer_backward_train(cfg, X, Wg, W1, W3, W2, sW1, sW3, sW2, route: Route
                                           _ptr(dW2), _ptr(dsW1), _ptr(dsW3), _ptr(dsW2),
                                           _ptr(dL), _ptr(ws), ws.numel(), _stream(stream)),
            "moe_layer_backward_train")
+
+
+def debug_inject_fault(fault: int):
+    """Arms a one-shot failure-path test fault (moe_debug_inject_fault)."""
+    _check(lib().moe_debug_inject_fault(fault), "moe_debug_inject_fault")
 
 
 def moe_read_error(ws, stream=None):

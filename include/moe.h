@@ -451,6 +451,27 @@ MOE_API moe_status moe_layer_backward_train(const moe_config* cfg, const void* X
                                             float* dL, void* ws, size_t ws_bytes,
                                             moe_stream_t stream);
 
+/* Failure-path test hooks (no counterpart on the pages). Arms one fault,
+ * taken by the next grouped-FFN up projection that can honour it, in any
+ * thread of the process; MOE_FAULT_NONE disarms.
+ *   MOE_FAULT_GEMM_NO_LOADS: the next up projection that runs on the
+ *     single-CTA kernel (bf16, fewer than 256 rows per expert on average)
+ *     issues no operand loads; its MMA warp's bounded wait runs out after
+ *     the 2 s limit, every warp of the kernel returns, and the workspace's
+ *     error word then reads MOE_ERR_TIMEOUT. That call's outputs are
+ *     undefined; the GPU context stays usable.
+ *   MOE_FAULT_LAUNCH: the next up projection is not launched and the call
+ *     returns MOE_ERR_CUDA, as for a failed launch (the kernels enqueued
+ *     before it stay enqueued).
+ * Nothing here faults the device. Returns MOE_ERR_INVALID_ARG for an
+ * unknown fault. */
+typedef enum {
+  MOE_FAULT_NONE = 0,
+  MOE_FAULT_GEMM_NO_LOADS = 1,
+  MOE_FAULT_LAUNCH = 2
+} moe_fault;
+MOE_API moe_status moe_debug_inject_fault(moe_fault fault);
+
 /* Zeroes the error word at the start of `ws` (enqueued on `stream`). */
 MOE_API moe_status moe_workspace_init(void* ws, moe_stream_t stream);
 

@@ -79,6 +79,7 @@ def lib() -> ctypes.CDLL:
         L.orc_select_ec.argtypes = [c_int, c_int, c_int, _f32p, _i32p, _f32p]
         L.orc_select_tc.argtypes = [c_int, c_int, c_int, _f32p, _opt(_f32p), c_int, c_int,
                                     c_int, c_int, _i32p, _f32p]
+        L.orc_weights_tc.argtypes = [c_int, c_int, c_int, _f32p, _i32p, c_int, _f32p]
         L.orc_capacity.argtypes = [c_int, c_int, c_int, _i32p, c_int, _u8p, _i32p, _i32p,
                                    _i32p]
         L.orc_expert_ffn.argtypes = [c_int, c_int, c_int, c_int, c_int, _f32p, _f32p,
@@ -100,7 +101,8 @@ def lib() -> ctypes.CDLL:
                                          _opt(_i32p), c_double, c_double, _f64p, _f64p]
         L.orc_router_backward.argtypes = [c_int, c_int, c_int, _f32p, _f32p, _f64p, _f32p,
                                           _f64p]
-        for name in ("orc_router", "orc_select_ec", "orc_select_tc", "orc_capacity",
+        for name in ("orc_router", "orc_select_ec", "orc_select_tc", "orc_weights_tc",
+                     "orc_capacity",
                      "orc_expert_ffn", "orc_combine", "orc_aux", "orc_bias_update",
                      "orc_ec_histogram", "orc_combine_backward", "orc_expert_ffn_backward",
                      "orc_gate_backward_tc", "orc_score_backward", "orc_router_backward"):
@@ -182,6 +184,19 @@ def select_tc(S, K: int, sel_bias=None, n_groups: int = 1, topk_groups: int = 1,
     lib().orc_select_tc(n, E, K, S, None if sel_bias is None else _f32(sel_bias),
                         n_groups, topk_groups, group_topn, weights, idx, w)
     return idx, w
+
+
+def weights_tc(S, idx, weights: int = W_RAW):
+    """Mixing weights [n,K] of the given selection idx [n,K] from the scores S
+    (the weights select_tc returns along with its own selection)."""
+    S = _f32(S)
+    idx = _i32(idx)
+    n, E = S.shape
+    K = idx.shape[1]
+    assert idx.shape[0] == n and ((idx >= 0) & (idx < E)).all()
+    w = np.empty((n, K), np.float32)
+    lib().orc_weights_tc(n, E, K, S, idx, weights, w)
+    return w
 
 
 def apply_capacity(idx, E: int, cap: int):

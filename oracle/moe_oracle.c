@@ -188,6 +188,24 @@ void orc_select_tc(int n, int E, int K, const float* S, const float* sel_bias,
   free(tmp);
 }
 
+/* Mixing weights of a given token-choice selection idx [n,K]: the raw score
+ * of each selected expert, or ([Guide] "1." softmax over the kept scores,
+ * "4." weights from the raw sigmoid scores) each selected raw score divided
+ * by their sum, taken in the order idx lists them. For the selection
+ * orc_select_tc makes, this is the weight it returns. */
+void orc_weights_tc(int n, int E, int K, const float* S, const int32_t* idx, int weights,
+                    float* w) {
+  for (int t = 0; t < n; ++t) {
+    const float* s = S + (size_t)t * E;
+    const int32_t* sel = idx + (size_t)t * K;
+    double denom = 0.0;
+    for (int j = 0; j < K; ++j) denom += (double)s[sel[j]];
+    for (int j = 0; j < K; ++j)
+      w[(size_t)t * K + j] =
+          (weights == ORC_W_NORMALIZED) ? (float)((double)s[sel[j]] / denom) : s[sel[j]];
+  }
+}
+
 /* [TC-vs-EC] "Dropped tokens flow in opposite directions": tokens that arrive
  * after an expert's buffer fills skip it and pass on the residual.
  * [Guide] "2. Top-1 switch routing with a capacity factor": buffer = tokens

@@ -60,6 +60,12 @@ void orc_select_tc(int n, int E, int K, const float* S, const float* sel_bias,
                    int n_groups, int topk_groups, int group_topn, int weights,
                    int32_t* idx, float* w);
 
+/* The mixing weights of a given selection idx [n,K] (raw, or normalised over
+ * the K selected raw scores in idx order): orc_select_tc's weights for its
+ * own selection. */
+void orc_weights_tc(int n, int E, int K, const float* S, const int32_t* idx, int weights,
+                    float* w);
+
 /* Capacity in arrival (token) order. cap < 0 means dropless.
  * load[E] = selections per expert, kept[E] = rows kept per expert,
  * drop[n,K] = 1 where the assignment overflowed, pos[n,K] = queue position

@@ -192,14 +192,127 @@ def expert_weights_from(inputs, prefix=""):
     return get
 
 
-def compare_out(store, got, ref, what=""):
+def bf16_ulp(x):
+    """Spacing of bf16 values at |x| (8 significant bits): 2^(e - 7) for
+    |x| in [2^e, 2^(e+1)); the smallest normal spacing below that range."""
+    a = np.maximum(np.abs(np.asarray(x, np.float64)), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(a)) - 7)
+
+
+# element-wise bound of bf16 results: each side rounds its expert outputs and
+# its result to bf16 (R22), and where the two sides' unrounded values straddle
+# a rounding boundary the stored values differ by one spacing, once for each
+# of the two roundings; on top of that, 1% of the row's rms covers the
+# different fp32 / fp64 accumulation orders
+BF16_ULPS = 2.0
+BF16_ROW_RMS_TOL = 1e-2
+
+
+def compare_out(store, got, ref, what="", ulps=BF16_ULPS, rms_tol=BF16_ROW_RMS_TOL,
+                row_tol=BF16_REL_TOL):
+    """Layer outputs (rows = tokens) against the oracle's, element by element.
+
+    fp32: max-abs error <= 1e-4. bf16, three checks that must all hold:
+      * every row: ||got_t - ref_t|| / ||ref_t|| <= 2e-2 (a row the oracle
+        leaves at zero, a token with no kept expert, must be exactly zero);
+      * every element: |got - ref| <= ulps bf16 spacings of ref + rms_tol *
+        rms(ref_t);
+      * the whole block: ||got - ref||_F / ||ref||_F <= 2e-2.
+    Returns the worst per-row relative error."""
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
     if store == oracle.STORE_F32:
         err = np.abs(got - ref).max() if got.size else 0.0
         assert err <= F32_ABS_TOL, f"{what} max-abs error {err}"
         return err
-    den = np.linalg.norm(ref)
-    err = np.linalg.norm(got - ref) / (den if den > 0 else 1.0)
+    if got.size == 0:
+        return 0.0
+    g2 = got.reshape(got.shape[0], -1)
+    r2 = ref.reshape(ref.shape[0], -1)
+    diff = np.abs(g2 - r2)
+    norms = np.linalg.norm(r2, axis=1)
+    zero = norms == 0
+    assert not diff[zero].any(), f"{what}: rows the oracle leaves at zero are not zero"
+    rel_rows = np.linalg.norm(g2 - r2, axis=1)[~zero] / norms[~zero]
+    worst = float(rel_rows.max()) if rel_rows.size else 0.0
+    assert worst <= row_tol, (f"{what}: row {int(np.nonzero(~zero)[0][rel_rows.argmax()])} "
+                              f"relative error {worst:.4g}")
+    rms = norms / np.sqrt(r2.shape[1])
+    bound = ulps * bf16_ulp(r2) + rms_tol * rms[:, None]
+    over = diff > bound
+    if over.any():
+        i, j = np.argwhere(over)[0]
+        raise AssertionError(
+            f"{what}: {int(over.sum())} elements beyond the element-wise bound; first at "
+            f"[{i}, {j}]: got {g2[i, j]:.6g} ref {r2[i, j]:.6g} (row rms {rms[i]:.4g}, "
+            f"bound {bound[i, j]:.4g})")
+    den = np.linalg.norm(r2)
+    err = np.linalg.norm(g2 - r2) / (den if den > 0 else 1.0)
     assert err <= BF16_REL_TOL, f"{what} relative error {err}"
-    return err
+    return worst
+
+
+# --------------------------------------------------------------------------
+# sampling at full size, and the oracle on the GPU's selection
+# --------------------------------------------------------------------------
+
+def covering_tokens(spec, r, n, E, seed, extra=8):
+    """Tokens whose outputs, together, exercise every expert's GEMM tiles:
+      * for every expert, the token in its last kept row (the expert's last
+        128-row block, which a CTA pair repeats when the block count is odd,
+        and the tail of its last weights-as-M token chunk);
+      * greedily, tokens until every expert with a kept row is covered;
+      * `extra` seeded random tokens; under a capacity, tokens with a drop
+        and with every choice dropped; under expert choice, tokens with no
+        expert and the token with the most.
+    Returns a sorted list of token ids."""
+    rng = np.random.default_rng(seed)
+    rows = {e: [] for e in range(E)}        # kept tokens of each expert, row order
+    if spec["mode"] == "ec":
+        for e in range(E):
+            rows[e] = [int(t) for t in r["I"][e]]
+    else:
+        idx, drop = r["idx"], r["drop"]
+        for t in range(n):
+            for j in range(idx.shape[1]):
+                if not drop[t, j]:
+                    rows[int(idx[t, j])].append(t)
+    picks = {l[-1] for l in rows.values() if l}
+    experts_of = {}
+    for e, l in rows.items():
+        for t in l:
+            experts_of.setdefault(t, set()).add(e)
+    covered = set()
+    for t in picks:
+        covered |= experts_of.get(t, set())
+    need = {e for e, l in rows.items() if l} - covered
+    while need:
+        t = max(experts_of, key=lambda u: (len(experts_of[u] & need), -u))
+        picks.add(t)
+        need -= experts_of[t]
+    picks |= set(rng.choice(n, size=min(extra, n), replace=False).tolist())
+    if spec["mode"] == "tc" and spec.get("capacity", -1) >= 0:
+        picks |= set(np.nonzero(r["drop"].any(1))[0][:2].tolist())
+        picks |= set(np.nonzero(r["drop"].all(1))[0][:1].tolist())
+    if spec["mode"] == "ec":
+        per_token = np.bincount(r["I"].ravel(), minlength=n)
+        picks |= set(np.nonzero(per_token == 0)[0][:2].tolist())
+        picks |= set(np.argsort(-per_token, kind="stable")[:1].tolist())
+    return sorted(int(t) for t in picks)
+
+
+def routing_on_gpu_selection(spec, S_or, rb: moe.RouteBuffers):
+    """The oracle's routing dict with the GPU's selection (and, under a
+    capacity, its drops) in place of the oracle's own, the weights computed
+    by the oracle from its own scores (R24: where a boundary gap below
+    GAP_TOL lets the two sides select differently, the outputs are compared
+    on the GPU's selection)."""
+    if spec["mode"] == "ec":
+        I = rb.idx.cpu().numpy().astype(np.int32)
+        E = I.shape[0]
+        G = np.stack([S_or[I[e], e] for e in range(E)]).astype(np.float32)
+        return {"I": I, "G": G}
+    idx = rb.idx.cpu().numpy().astype(np.int32)
+    w = oracle.weights_tc(S_or, idx, spec.get("weights", oracle.W_RAW))
+    return {"idx": idx, "w": w, "drop": rb.drop.cpu().numpy()}

@@ -34,7 +34,7 @@ def declared_symbols():
 
 def test_every_declared_symbol_is_exported():
     syms = declared_symbols()
-    assert len(syms) == 23
+    assert len(syms) == 24
     assert sorted(moe.API_SYMBOLS) == syms
     L = ctypes.CDLL(moe.LIB_PATH)
     for s in syms:
@@ -208,6 +208,16 @@ def test_launch_counts():
     decode = moe.launch_counts(moe.config(wl.DECODE))
     assert decode["route"] == 5
     assert moe.launch_counts(moe.config(wl.TC_SIGMOID_GROUPED))["ffn"] == 2
+
+
+def test_fault_hook_arguments():
+    """The failure-path hook takes the documented faults only, and
+    MOE_FAULT_NONE disarms it (nothing is launched here)."""
+    L = moe.lib()
+    assert L.moe_debug_inject_fault(7) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_debug_inject_fault(-1) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_debug_inject_fault(moe.MOE_FAULT_LAUNCH) == moe.MOE_OK
+    assert L.moe_debug_inject_fault(moe.MOE_FAULT_NONE) == moe.MOE_OK
 
 
 def test_train_launch_counts():

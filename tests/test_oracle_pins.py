@@ -259,6 +259,30 @@ def test_softmax_over_kept_logits_identity():
     np.testing.assert_allclose(w, ref, rtol=2e-6, atol=0)
 
 
+def test_weights_of_a_given_selection():
+    """weights_tc on select_tc's own selection returns select_tc's weights
+    bit for bit (raw and normalised, with a selection bias and groups), and
+    on any other selection the softmax-over-kept identity holds: normalised
+    weights of softmax scores equal a softmax over the chosen logits."""
+    rng = np.random.default_rng(5)
+    X = rng.standard_normal((50, 24)).astype(np.float32)
+    Wg = (rng.standard_normal((24, 32)) / 5).astype(np.float32)
+    logits, S, _ = oracle.router(X, Wg)
+    _, s, _ = oracle.router(X, Wg, score=oracle.SIGMOID)
+    bias = (rng.standard_normal(32) * 0.1).astype(np.float32)
+    for scores, b, G in ((S, None, 1), (s, bias, 4), (s, None, 8)):
+        for mode in (oracle.W_RAW, oracle.W_NORMALIZED):
+            idx, w = oracle.select_tc(scores, 4, b, n_groups=G, topk_groups=min(2, G),
+                                      group_topn=2 if G > 1 else 1, weights=mode)
+            np.testing.assert_array_equal(oracle.weights_tc(scores, idx, mode), w)
+    other = np.stack([rng.permutation(32)[:3] for _ in range(50)]).astype(np.int32)
+    w = oracle.weights_tc(S, other, oracle.W_NORMALIZED)
+    ref = special.softmax(np.take_along_axis(logits.astype(np.float64), other, 1), axis=1)
+    np.testing.assert_allclose(w, ref, rtol=2e-6, atol=0)
+    raw = oracle.weights_tc(S, other, oracle.W_RAW)
+    np.testing.assert_array_equal(raw, np.take_along_axis(S, other, 1))
+
+
 def test_selection_only_bias():
     rng = np.random.default_rng(1)
     X = rng.standard_normal((64, 32)).astype(np.float32)
