@@ -33,7 +33,7 @@ struct RCfg {
                        WY = WY_, WK = WK_, BK = BK_, ST = ST_, BM = WX_ * LX_ * TM_;
   static_assert(WY * LY * TN == ET, "columns");
   static_assert(WX * WY * WK == 8, "8 warps");
-  static_assert(TN == 4 || TN == 8, "TN");
+  static_assert(TN == 4 || TN == 8 || TN == 16, "TN");
   static_assert(TM >= 1 && TM <= 8, "TM");
   static_assert(BK % WK == 0 && ST >= 2, "pipeline");
 };
@@ -59,6 +59,11 @@ template <int TM> using R64A = RCfg<64, TM, 8, 4, 1, 1, 8, 64, 4>;   // BM = 4 T
 template <int TM> using R64C = RCfg<64, TM, 8, 4, 4, 1, 2, 32, 4>;   // BM = 16 TM
 template <int TM> using R128A = RCfg<128, TM, 8, 4, 2, 2, 2, 32, 4>; // BM = 8 TM
 template <int TM> using R256A = RCfg<256, TM, 8, 4, 1, 4, 2, 32, 3>; // BM = 4 TM
+// E = 256 with 16 columns per thread: per 16-deep step a warp issues TM*16
+// FFMAs for TM + 16 shared-memory wavefronts (TM x 8 tiles: TM*8 for TM + 8),
+// so the FMA pipe, not shared-memory bandwidth, sets the pace; one CTA per
+// SM (about 160 registers a thread)
+template <int TM> using R256B = RCfg<256, TM, 16, 4, 2, 2, 2, 32, 3>; // BM = 8 TM
 
 constexpr int kSelectRowsPerWarp = 4;
 
@@ -81,8 +86,8 @@ static int num_sms_cached() {
 // small-row one when the big tile would leave SMs without a CTA. bf16 X with
 // E > 32: the (family, TM) whose rows per SM, BM * ceil(CTAs / SMs), is
 // smallest (ties to the larger BM). Codes: kFamilyCode + fam * 16 + TM with
-// fam 1 = R64A, 2 = R64C, 3 = R128A, 4 = R256A; otherwise the fixed tile's ET
-// (257: R256s, 65: R64s).
+// fam 1 = R64A, 2 = R64C, 3 = R128A, 4 = R256A, 5 = R256B; otherwise the
+// fixed tile's ET (257: R256s, 65: R64s).
 constexpr int kFamilyCode = 1000;
 struct RouterFamily {
   int code, unit, tm_lo;
@@ -93,9 +98,9 @@ static int router_variant(int E, int n, bool x_bf16) {
   if (x_bf16 && et >= 64) {
     static const RouterFamily fams64[] = {{1, 4, 4}, {2, 16, 4}};
     static const RouterFamily fams128[] = {{3, 8, 2}};
-    static const RouterFamily fams256[] = {{4, 4, 4}};
+    static const RouterFamily fams256[] = {{4, 4, 4}, {5, 8, 4}};
     const RouterFamily* fams = et == 64 ? fams64 : et == 128 ? fams128 : fams256;
-    const int nf = et == 64 ? 2 : 1;
+    const int nf = et == 128 ? 1 : 2;
     long long best_cost = -1;
     int best = 0, best_bm = 0;
     for (int f = 0; f < nf; ++f)
@@ -111,6 +116,10 @@ static int router_variant(int E, int n, bool x_bf16) {
         // per SM took 203 us, 128 rows in two CTAs 174 us).
         if (fams[f].code == 1 && ctas > sms) continue;
         if (fams[f].code == 2 && ctas * 2 < 3LL * sms) cost = cost * 4 / 3;
+        // TM x 8 tiles at E = 256 are bound by shared-memory wavefronts
+        // (TM + 8 per TM*8 FFMAs per step), the 16-column tiles by the FMA
+        // pipe: charge the narrower tile a quarter more per row
+        if (fams[f].code == 4) cost = cost * 5 / 4;
         if (best_cost < 0 || cost < best_cost || (cost == best_cost && bm > best_bm)) {
           best_cost = cost;
           best = kFamilyCode + fams[f].code * 16 + tm;
@@ -136,7 +145,7 @@ static void variant_tile(int v, int* bm, int* bk) {
     case 257: *bm = R256s::BM; *bk = R256s::BK; return;
     default: {
       const int code = v - kFamilyCode, fam = code / 16, tm = code % 16;
-      *bm = (fam == 2 ? 16 : fam == 3 ? 8 : 4) * tm;
+      *bm = (fam == 2 ? 16 : fam == 3 || fam == 5 ? 8 : 4) * tm;
       *bk = fam == 1 ? 64 : 32;
     }
   }
@@ -653,7 +662,8 @@ static cudaError_t launch_router_bf16_family(int code, const RouterArgs& a, cuda
     case 1: return launch_family<R64A>(tm, a, s);
     case 2: return launch_family<R64C>(tm, a, s);
     case 3: return launch_family<R128A>(tm, a, s);
-    default: return launch_family<R256A>(tm, a, s);
+    case 4: return launch_family<R256A>(tm, a, s);
+    default: return launch_family<R256B>(tm, a, s);
   }
 }
 

@@ -45,6 +45,10 @@ ROUTE_VARIANTS = [
                                   n_groups=1, topk_groups=1, bias_steps=2),
     wl.TC_SIGMOID_GROUPED.replace(name="tc-sqrtsoftplus-grouped8keep4-top8of64", n=300, d=192,
                                   E=64, h=64, score="sqrtsoftplus", bias_steps=2),
+    # 256 experts over 4,096 tokens: the router's 16-column register tiles
+    # (32 rows per CTA), as the full DeepSeek-V3-shaped layer uses (56 rows)
+    wl.TC_SIGMOID_GROUPED.replace(name="tc-router16-grouped8keep4-top8of256-n4096-d512", n=4096,
+                                  d=512, E=256, h=64, bias_steps=2),
 ]
 
 
@@ -112,7 +116,14 @@ def _oracle_from_x(w, inp):
     return spec, logits, S, lse, r
 
 
-@pytest.mark.parametrize("w", wl.SMALL + ROUTE_VARIANTS, ids=lambda w: w.name)
+# the DeepSeek-V3-shaped layer's routing at full size (8,192 tokens, d 7168,
+# 256 experts): the router launch the benchmark times, without the experts'
+# weights (routing only)
+ROUTE_FULL = [wl.TC_SIGMOID_GROUPED.replace(
+    name="route-only-sigmoid-grouped8keep4-top8of256-n8192-d7168", bias_steps=0)]
+
+
+@pytest.mark.parametrize("w", wl.SMALL + ROUTE_VARIANTS + ROUTE_FULL, ids=lambda w: w.name)
 def test_route_from_x(w):
     inp = wl.make_inputs(w, DEV, experts=False)
     cfg = moe.config(w)
