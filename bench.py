@@ -370,6 +370,27 @@ def run_gpu(args, w: wl.Workload):
                          for i in range(args.steps)])
     check_errors("in the timed region")
 
+    # ---- a floor for the two copy-like stages: a plain device-to-device copy
+    # (torch, the copy engine's kernel) moving the same bytes as the stage
+    # (half read, half written), timed the same way (L2 flushed before each,
+    # events around it); a stage at the copy's time is at what this size allows
+    def copy_floor_ms(nbytes):
+        half = max(16, int(nbytes // 2) // 16 * 16)
+        src = torch.empty(half, dtype=torch.uint8, device=dev)
+        dst = torch.empty_like(src)
+        ts = []
+        for i in range(args.warmup + args.steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            dst.copy_(src)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if i >= args.warmup:
+                ts.append(e0.elapsed_time(e1))
+        del src, dst
+        return float(np.median(ts))
+
     # ---- end to end through the C call that takes host buffers
     # (moe_layer_forward_host): every step uploads X from page-locked host
     # memory and downloads out into page-locked host memory, the library
@@ -449,6 +470,10 @@ def run_gpu(args, w: wl.Workload):
     stages["route"].update({"router_FLOP": router_flops, "FFMA_TFLOP/s": round(route_tflops, 2),
                             "ffma_peak_TFLOP/s": round(ffma_peak, 1),
                             "ffma_frac": round(route_tflops / ffma_peak, 3)})
+    for nm in ("dispatch", "combine"):
+        fl = copy_floor_ms(bytes_[nm])
+        stages[nm].update({"copy_floor_ms": round(fl, 4),
+                           "frac_of_copy": round(fl / stages[nm]["ms"], 3)})
     ffn_tflops = flops / (med[2] * 1e-3) / 1e12
     stages["ffn"]["TFLOP/s"] = round(ffn_tflops, 1)
     stages["ffn"]["tc_frac"] = round(ffn_tflops / tc_peak, 3)
@@ -493,7 +518,10 @@ def run_gpu(args, w: wl.Workload):
         "stages": stages,
         "routing": routing,
         "stages_note": "medians of a second pass with an event between stages; value and "
-                       "ms_per_step come from whole-step events around moe_layer_forward",
+                       "ms_per_step come from whole-step events around moe_layer_forward; "
+                       "copy_floor_ms: a plain device-to-device copy moving the stage's bytes "
+                       "(half read, half written) from a cold L2, frac_of_copy = its time / "
+                       "the stage's",
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": xbytes, "d2h_bytes_per_step": xbytes,
                 "note": "moe_layer_forward_host (C ABI): page-locked host X -> device -> "

@@ -375,10 +375,17 @@ __device__ __forceinline__ void router_rows_epilogue(const RouterArgs& a, const 
 template <class C, bool XBF16>
 struct RouterSmem {
   static constexpr int XB = XBF16 ? 2 : 4;
-  static constexpr int AST = C::BM + 4;  // transposed fp32 A tile row stride
+  // The transposed A tile As[kk][row] keeps X's own type: bf16 X stays bf16
+  // (each value widens exactly to fp32 when loaded), so a thread's rows come
+  // in one vector load of half the bytes. A thread's TM rows sit together;
+  // with bf16 an odd TM gets one padding slot (TMP = TM + 1) so the group
+  // starts on an even element.
+  static constexpr int TMP = (XBF16 && (C::TM % 2)) ? C::TM + 1 : C::TM;
+  static constexpr int BMP = C::BM / C::TM * TMP;          // padded rows
+  static constexpr int AST = BMP + (XBF16 ? 8 : 4);        // row stride, elements
   static constexpr size_t xs_bytes = (size_t)C::ST * C::BM * C::BK * XB;
   static constexpr size_t ws_bytes = (size_t)C::ST * C::BK * C::ET * 4;
-  static constexpr size_t as_bytes = (size_t)C::BK * AST * 4;
+  static constexpr size_t as_bytes = (size_t)C::BK * AST * XB;
   static constexpr size_t main_bytes = xs_bytes + ws_bytes + as_bytes;
   static constexpr size_t epi_bytes =
       ((size_t)C::WK * C::BM * (C::ET + 1) + 8 * C::ET) * 4 + 8 * 8;
@@ -390,12 +397,12 @@ __global__ void __launch_bounds__(256) router_kernel(RouterArgs a) {
   pdl_wait();
   using SM = RouterSmem<C, XBF16>;
   constexpr int ET = C::ET, BM = C::BM, BK = C::BK, TM = C::TM, TN = C::TN;
-  constexpr int XB = SM::XB, AST = SM::AST;
-  constexpr int V = ET >= 32 ? ET / 32 : 1;
+  constexpr int XB = SM::XB, AST = SM::AST, TMP = SM::TMP;
   extern __shared__ __align__(16) unsigned char rsm[];
   unsigned char* Xs = rsm;                                        // [S][BM][BK] raw
   float* Ws = reinterpret_cast<float*>(rsm + SM::xs_bytes);       // [S][BK][ET]
-  float* As = reinterpret_cast<float*>(rsm + SM::xs_bytes + SM::ws_bytes);  // [BK][AST]
+  float* As = reinterpret_cast<float*>(rsm + SM::xs_bytes + SM::ws_bytes);  // [BK][AST] fp32
+  uint16_t* As16 = reinterpret_cast<uint16_t*>(As);                         // [BK][AST] bf16
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int lx = lane / C::LY, ly = lane % C::LY;
@@ -403,6 +410,7 @@ __global__ void __launch_bounds__(256) router_kernel(RouterArgs a) {
   const int wrem = warp % (C::WX * C::WY);
   const int wx = wrem / C::WY, wy = wrem % C::WY;
   const int row0 = (wx * C::LX + lx) * TM;
+  const int arow0 = (wx * C::LX + lx) * TMP;  // the same rows in the (padded) A tile
   const int colb = wy * C::LY * TN + ly * 4;  // first column of group 0; group g adds g*4*LY
   const int m0 = blockIdx.x * BM;
   const int n = a.n, d = a.d, E = a.E;
@@ -472,10 +480,11 @@ __global__ void __launch_bounds__(256) router_kernel(RouterArgs a) {
         const uint4 v = *reinterpret_cast<const uint4*>(xs + (size_t)r * BK * XB + p * 16);
         const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
         if (XBF16) {
+          const int rr = r / TM * TMP + r % TM;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            As[(p * 8 + 2 * j) * AST + r] = __uint_as_float(w4[j] << 16);
-            As[(p * 8 + 2 * j + 1) * AST + r] = __uint_as_float(w4[j] & 0xffff0000u);
+            As16[(p * 8 + 2 * j) * AST + rr] = (uint16_t)(w4[j] & 0xffffu);
+            As16[(p * 8 + 2 * j + 1) * AST + rr] = (uint16_t)(w4[j] >> 16);
           }
         } else {
 #pragma unroll
@@ -491,7 +500,28 @@ __global__ void __launch_bounds__(256) router_kernel(RouterArgs a) {
     for (int q = 0; q < BK / C::WK; ++q) {
       const int kk = wk * (BK / C::WK) + q;
       float av[TM], bv[TN];
-      if (TM % 4 == 0) {
+      if constexpr (XBF16) {
+        // the thread's TMP bf16 values: one 16- or 8-byte load, else 4-byte loads
+        const uint16_t* ap = As16 + kk * AST + arow0;
+        uint32_t w[TMP / 2];
+        if constexpr (TMP == 8) {
+          const uint4 t = *reinterpret_cast<const uint4*>(ap);
+          w[0] = t.x;
+          w[1] = t.y;
+          w[2] = t.z;
+          w[3] = t.w;
+        } else if constexpr (TMP == 4) {
+          const uint2 t = *reinterpret_cast<const uint2*>(ap);
+          w[0] = t.x;
+          w[1] = t.y;
+        } else {
+#pragma unroll
+          for (int i = 0; i < TMP / 2; ++i) w[i] = reinterpret_cast<const uint32_t*>(ap)[i];
+        }
+#pragma unroll
+        for (int i = 0; i < TM; ++i)
+          av[i] = __uint_as_float(i % 2 ? (w[i / 2] & 0xffff0000u) : (w[i / 2] << 16));
+      } else if (TM % 4 == 0) {
 #pragma unroll
         for (int i4 = 0; i4 < TM / 4; ++i4) {
           const float4 t = *reinterpret_cast<const float4*>(As + kk * AST + row0 + 4 * i4);
