@@ -369,7 +369,9 @@ __global__ void __launch_bounds__(kTokBlock) tc_hist_kernel(TcAssignArgs a) {
     a.blk_hist[(size_t)blockIdx.x * a.E + i] = hist[i];
 }
 
-__global__ void __launch_bounds__(1024) tc_scan_kernel(TcAssignArgs a) {
+constexpr int kScanThreads = 1024;
+
+__global__ void __launch_bounds__(kScanThreads) tc_scan_kernel(TcAssignArgs a) {
   pdl_wait();
   __shared__ int seg[MOE_MAX_EXPERTS];
   __shared__ int off[MOE_MAX_EXPERTS + 1];
@@ -385,19 +387,41 @@ __global__ void __launch_bounds__(1024) tc_scan_kernel(TcAssignArgs a) {
   if (tid < S * E) {
     const int e = tid % E, slice = tid / E;
     double col = 0.0;
-    for (int b = slice; b < a.colsum_blocks; b += S) col += (double)a.colsum[(size_t)b * E + e];
+    // eight loads in flight, added in the same block order as one at a time
+    constexpr int U = 8;
+    int b = slice;
+    for (; b + (U - 1) * S < a.colsum_blocks; b += U * S) {
+      float v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) v[u] = a.colsum[(size_t)(b + u * S) * E + e];
+#pragma unroll
+      for (int u = 0; u < U; ++u) col += (double)v[u];
+    }
+    for (; b < a.colsum_blocks; b += S) col += (double)a.colsum[(size_t)b * E + e];
     part[tid] = col;
   }
   __syncthreads();
   // per expert: exclusive prefix of the token blocks' counts, one warp per
   // expert, 32 blocks per step (a shuffle scan), so the block count adds
-  // steps of one load each, not a chain of dependent loads
+  // steps of one load each, not a chain of dependent loads; a warp loads the
+  // first 32 blocks of all its experts before scanning any of them
   const int lane = tid & 31, warp = tid >> 5;
-  for (int e = warp; e < E; e += (int)(blockDim.x >> 5)) {
+  constexpr int nwarps = kScanThreads / 32;
+  constexpr int kExpertsPerWarp = (MOE_MAX_EXPERTS + nwarps - 1) / nwarps;
+  int first[kExpertsPerWarp];
+#pragma unroll
+  for (int j = 0; j < kExpertsPerWarp; ++j) {
+    const int e = warp + j * nwarps;
+    first[j] = (e < E && lane < a.tok_blocks) ? a.blk_hist[(size_t)lane * E + e] : 0;
+  }
+#pragma unroll
+  for (int j = 0; j < kExpertsPerWarp; ++j) {
+    const int e = warp + j * nwarps;
+    if (e >= E) break;
     int run = 0;
     for (int b0 = 0; b0 < a.tok_blocks; b0 += 32) {
       const int b = b0 + lane;
-      const int v = b < a.tok_blocks ? a.blk_hist[(size_t)b * E + e] : 0;
+      const int v = b0 == 0 ? first[j] : (b < a.tok_blocks ? a.blk_hist[(size_t)b * E + e] : 0);
       int incl = v;
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, incl, o);
@@ -534,7 +558,7 @@ __global__ void __launch_bounds__(kTokBlock) tc_scatter_kernel(TcAssignArgs a) {
 cudaError_t launch_tc_assign(const TcAssignArgs& a, cudaStream_t s) {
   cudaError_t e = launch_pdl(tc_hist_kernel, a.tok_blocks, kTokBlock, 0, s, a);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(tc_scan_kernel, 1, 1024, 0, s, a);
+  e = launch_pdl(tc_scan_kernel, 1, kScanThreads, 0, s, a);
   if (e != cudaSuccess) return e;
   const size_t bytes = (size_t)(2 * (kTokBlock / 32) + 1) * a.E * 4;
   e = cudaFuncSetAttribute(tc_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
