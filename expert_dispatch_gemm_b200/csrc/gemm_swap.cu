@@ -41,6 +41,11 @@ constexpr int kSStageBytes = kSABytes + kSBBytes;
 constexpr int kSTmemCols = 512;                  // two 256-column accumulators
 constexpr int kSMaxTokens = 256;                 // tokens per tile (MMA N <= 256)
 constexpr uint64_t kSWaitNs = 2000000000ull;     // 2 s
+// The weight tiles (the A side) come from HBM once each, at the MMA's pace,
+// with a latency under load that a ring of shared-memory stages alone does not
+// cover: the producer also brings the weight rows of the k-block this many
+// steps ahead of its loads into L2, so the loads themselves hit L2.
+constexpr int kSPrefetch = 8;
 
 struct SwapParams {
   const int32_t* offsets;   // [E+1] segment starts
@@ -231,6 +236,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSThreads, 1)
       int stage = 0, issued = 0;
       uint32_t phase = 0;
       bool ok = true;
+      // L2 prefetch cursor over the same (tile, k-block) sequence, ahead
+      int pf_tile = pair_id, pf_kb = 0, pf_decoded = -1, pf_wrow = 0;
+      bool pf_shared = false;
+      auto prefetch_next = [&]() {
+        if (pf_tile >= total) return;
+        if (pf_decoded != pf_tile) {
+          const SwapTile u = decode_swap(pf_tile, p, st, routed);
+          pf_wrow = u.expert * p.m_per_expert + u.m0 + (int)rank * 128;
+          pf_shared = u.shared;
+          pf_decoded = pf_tile;
+        }
+        sm100::tma_prefetch_l2_2d(pf_shared ? &tmWs : &tmW, pf_kb * kSBK, pf_wrow);
+        if (++pf_kb == KB) {
+          pf_kb = 0;
+          pf_tile += num_pairs;
+        }
+      };
+      for (int i = 0; i < kSPrefetch; ++i) prefetch_next();
       for (int tile = pair_id; ok && tile < total; tile += num_pairs) {
         const SwapTile t = decode_swap(tile, p, st, routed);
         const CUtensorMap* tm[3];
@@ -247,6 +270,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSThreads, 1)
         // this CTA's half of the tile's tokens
         const long long trow1 = t.tok_row + (long long)rank * (t.n / 2);
         for (int kb = 0; kb < KB; ++kb) {
+          prefetch_next();
           if (!swap_wait<false>(&st->empty[stage], phase ^ 1u, st, p.err, kErrGemmTimeout | 0xA1)) {
             ok = false;
             break;
@@ -468,6 +492,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSThreads, 1)
       int stage = 0, issued = 0;
       uint32_t phase = 0;
       bool ok = true;
+      // L2 prefetch cursor over the same (tile, k-block) sequence, ahead
+      int pf_tile = pair_id, pf_kb = 0, pf_decoded = -1, pf_wrow = 0;
+      bool pf_shared = false;
+      auto prefetch_next = [&]() {
+        if (pf_tile >= total) return;
+        if (pf_decoded != pf_tile) {
+          const SwapTile u = decode_swap(pf_tile, p, st, routed);
+          pf_wrow = u.expert * p.m_per_expert + u.m0 + (int)rank * 128;
+          pf_shared = u.shared;
+          pf_decoded = pf_tile;
+        }
+        sm100::tma_prefetch_l2_2d(pf_shared ? &tmW1s : &tmW1, pf_kb * kSBK, pf_wrow);
+        sm100::tma_prefetch_l2_2d(pf_shared ? &tmW3s : &tmW3, pf_kb * kSBK, pf_wrow);
+        if (++pf_kb == KB) {
+          pf_kb = 0;
+          pf_tile += num_pairs;
+        }
+      };
+      for (int i = 0; i < kSPrefetch; ++i) prefetch_next();
       for (int tile = pair_id; ok && tile < total; tile += num_pairs) {
         const SwapTile t = decode_swap(tile, p, st, routed);
         const CUtensorMap* tm[3];
@@ -485,6 +528,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSThreads, 1)
         // this CTA's half of the tile's tokens
         const long long trow1 = t.tok_row + (long long)rank * (t.n / 2);
         for (int kb = 0; kb < KB; ++kb) {
+          prefetch_next();
           if (!swap_wait<false>(&st->empty[stage], phase ^ 1u, st, p.err, kErrGemmTimeout | 0xD1)) {
             ok = false;
             break;

@@ -330,14 +330,16 @@ def token_pairs(spec: dict, routing: dict, n: int, tokens=None):
 
 
 def layer_forward(spec: dict, X, routing: dict, expert_weights, shared_weights=None,
-                  tokens=None):
+                  tokens=None, absum: bool = False):
     """out rows for `tokens` (all when None) of the MoE layer given a routing.
 
     expert_weights(e) -> (W1 [h,d], W3 [h,d] or None, W2 [d,h]) as float32;
     shared_weights(s) -> same for always-on shared expert s (weight 1,
     "MoE routing strategies explained", section "3. Shared plus routed
     experts"). The residual is not added: the layer returns scatter_add only.
-    """
+    With absum=True, returns (out, A) where A is the same combine taken over
+    |gate| * |Y| (fp32, unrounded): the scale of each output element's terms,
+    which the tests use to bound rounding differences."""
     X = _f32(X)
     n, d = X.shape
     store, act = spec["store"], spec["act"]
@@ -362,8 +364,12 @@ def layer_forward(spec: dict, X, routing: dict, expert_weights, shared_weights=N
         pgate += [1.0] * len(rows)
     Yall = np.concatenate(Ys, 0) if Ys else np.zeros((0, d), np.float32)
     order = np.argsort(np.asarray(ptok, np.int64), kind="stable")
-    return combine(len(rows), np.asarray(ptok, np.int32)[order],
-                   np.asarray(pgate, np.float32)[order], Yall[order], store)
+    tok_o = np.asarray(ptok, np.int32)[order]
+    gate_o = np.asarray(pgate, np.float32)[order]
+    out = combine(len(rows), tok_o, gate_o, Yall[order], store)
+    if not absum:
+        return out
+    return out, combine(len(rows), tok_o, np.abs(gate_o), np.abs(Yall[order]), STORE_F32)
 
 
 # --------------------------------------------------------------------------

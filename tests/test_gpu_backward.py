@@ -71,9 +71,10 @@ def _close(got, ref, tol, bf16, what=""):
     units of a weight gradient): the whole block and every row within `tol`
     relative Frobenius error (a row the oracle leaves at zero must be zero),
     and, for values stored in bf16, every element within two bf16 spacings of
-    the oracle's value plus 1% of its row's rms (the two sides' roundings of
-    the stored rows may land one spacing apart; the rest is accumulation
-    order)."""
+    the oracle's value plus 2% of its row's rms (the two sides' roundings of
+    a stored value may land one spacing apart, and a weight gradient sums an
+    expert's few rows of bf16 products, where one flipped input moves an
+    element by up to a few percent of the row's rms)."""
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
     g2 = got.reshape(got.shape[0], -1)
@@ -87,10 +88,29 @@ def _close(got, ref, tol, bf16, what=""):
     assert rows.size == 0 or rows.max() < tol, f"{what}: worst row error {rows.max():.4g}"
     if bf16:
         rms = norms / np.sqrt(r2.shape[1])
-        bound = 2.0 * bf16_ulp(r2) + 1e-2 * rms[:, None]
+        bound = 2.0 * bf16_ulp(r2) + 2e-2 * rms[:, None]
         over = np.abs(g2 - r2) > bound
         assert not over.any(), (f"{what}: {int(over.sum())} elements beyond two bf16 "
-                                f"spacings + 1% of the row rms")
+                                f"spacings + 2% of the row rms; worst excess "
+                                f"{float((np.abs(g2 - r2) - bound).max()):.4g}")
+    return rel
+
+
+def _close_dwg(got, ref, X, dL_ref, tol=F32_GRAD_TOL, what="dWg"):
+    """dW_g = X^T dL against the oracle's: the block within `tol` relative
+    Frobenius error, and every element within tol * sum_t |X[t, i]| *
+    ||dL_ref[t]||: what the per-token bound ||dL_t - dL_ref_t|| <= tol
+    ||dL_ref_t|| allows for a sum over tokens (a per-expert bound would not
+    hold where the tokens' terms cancel)."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    rel = _rel(got, ref)
+    assert rel < tol, f"{what}: relative error {rel:.4g}"
+    scale = np.abs(np.asarray(X, np.float64)).T @ np.linalg.norm(
+        np.asarray(dL_ref, np.float64), axis=1)
+    bound = tol * scale[:, None] + 1e-7
+    over = np.abs(got - ref) > bound
+    assert not over.any(), f"{what}: {int(over.sum())} elements beyond the token-sum bound"
     return rel
 
 
@@ -129,7 +149,7 @@ def test_backward_small(w):
     tol = FP32_LAYER_TOL if f32 else BF16_GRAD_TOL
     bf16 = not f32
     _close(host(g["dL"]), ref["dL"], tol_f32, False, "dL")
-    _close(host(g["dWg"]).T, ref["dWg"].T, tol_f32, False, "dWg")
+    _close_dwg(host(g["dWg"]), ref["dWg"], host(inp["X"]), ref["dL"], tol_f32)
     _close(host(g["dX"]), ref["dX"], tol, bf16, "dX")
     names = ["dW1", "dW2"] + (["dW3"] if w.act == "swiglu" else [])
     for e in range(w.E):
@@ -234,30 +254,6 @@ def test_backward_full_size_sampled(w):
     tt = torch.as_tensor(toks, device=DEV)
     _close(host(g["dX"][tt]), ref["dX"], BF16_GRAD_TOL, True, "dX")
     _close(host(g["dL"][tt]), ref["dL"], F32_GRAD_TOL, False, "dL")
-    # the router weight gradient dWg = X^T dL sums over every token: a second
-    # backward with dout zero outside `toks` leaves the other tokens' dL at
-    # the aux losses' terms alone, which the oracle's score backward gives
-    # for every row at once (dS = 0); the oracle's router backward then
-    # gives the whole dWg
-    mask = torch.zeros((w.n, 1), dtype=dout.dtype, device=DEV)
-    mask[tt] = 1
-    dout_t = dout * mask
-    layer.forward()
-    g_t = layer.backward(dout_t)
-    torch.cuda.synchronize()
-    ref_t = oracle.layer_backward(spec, X, host(inp["Wg"]), host(dout_t),
-                                  expert_weights_from(inp),
-                                  expert_weights_from(inp, "s") if w.n_shared else None,
-                                  host(inp.get("logit_bias")), host(inp.get("sel_bias")),
-                                  tokens=toks, pre=(logits, S, lse, r))
-    tc = spec["mode"] == "tc"
-    dL_all = oracle.score_backward(logits, S, lse, np.zeros(S.shape), spec["score"],
-                                   r.get("load"), spec.get("K", 1),
-                                   w.lb_coef if tc else 0.0, w.z_coef if tc else 0.0)
-    dL_all[toks] = ref_t["dL"]
-    dWg_ref, _ = oracle.router_backward(X, host(inp["Wg"]), dL_all)
-    _close(host(g_t["dL"][tt]), ref_t["dL"], F32_GRAD_TOL, False, "dL (masked dout)")
-    _close(host(g_t["dWg"]).T, dWg_ref.T, F32_GRAD_TOL, False, "dWg (masked dout)")
     # weight gradients: sampled hidden units of two experts (and the shared one)
     pairs = oracle.token_pairs(spec, r, w.n)
     by_e = {}
@@ -289,6 +285,30 @@ def test_backward_full_size_sampled(w):
         _close(host(g["d" + p + "W2"][e][:, jt]).T, r2.T, BF16_GRAD_TOL, True, f"d{p}W2[{e}]")
         if swiglu:
             _close(host(g["d" + p + "W3"][e][jt]), r3, BF16_GRAD_TOL, True, f"d{p}W3[{e}]")
+    # the router weight gradient dWg = X^T dL sums over every token. A second
+    # backward, with dout zero outside `toks`, leaves the other tokens' dL at
+    # the aux losses' terms alone, which the oracle's score backward gives for
+    # every row at once (dS = 0); the oracle's router backward then gives the
+    # whole dWg. (Last: this backward reuses the gradient buffers.)
+    mask = torch.zeros((w.n, 1), dtype=dout.dtype, device=DEV)
+    mask[tt] = 1
+    dout_t = dout * mask
+    layer.forward()
+    g_t = layer.backward(dout_t)
+    torch.cuda.synchronize()
+    ref_t = oracle.layer_backward(spec, X, host(inp["Wg"]), host(dout_t),
+                                  expert_weights_from(inp),
+                                  expert_weights_from(inp, "s") if w.n_shared else None,
+                                  host(inp.get("logit_bias")), host(inp.get("sel_bias")),
+                                  tokens=toks, pre=(logits, S, lse, r))
+    tc = spec["mode"] == "tc"
+    dL_all = oracle.score_backward(logits, S, lse, np.zeros(S.shape), spec["score"],
+                                   r.get("load"), spec.get("K", 1),
+                                   w.lb_coef if tc else 0.0, w.z_coef if tc else 0.0)
+    dL_all[toks] = ref_t["dL"]
+    dWg_ref, _ = oracle.router_backward(X, host(inp["Wg"]), dL_all)
+    _close(host(g_t["dL"][tt]), ref_t["dL"], F32_GRAD_TOL, False, "dL (masked dout)")
+    _close_dwg(host(g_t["dWg"]), dWg_ref, X, dL_all, what="dWg (masked dout)")
 
 
 @pytest.mark.parametrize("w", wl.SMALL + [wl.TC_SIGMOID_GROUPED.replace(

@@ -164,13 +164,14 @@ def check_layer_rows(w, inp, out, rb, spec, S, r, tokens=None):
     got = host(out)
     worst = 0.0
     if good:
-        ref = oracle.layer_forward(spec, X, r, ew, sw, tokens=good)
-        worst = compare_out(spec["store"], got[good], ref, w.name)
+        ref, terms = oracle.layer_forward(spec, X, r, ew, sw, tokens=good, absum=True)
+        worst = compare_out(spec["store"], got[good], ref, w.name, absum=terms)
     if flipped:
         rg = routing_on_gpu_selection(spec, S, rb)
-        ref = oracle.layer_forward(spec, X, rg, ew, sw, tokens=flipped)
+        ref, terms = oracle.layer_forward(spec, X, rg, ew, sw, tokens=flipped, absum=True)
         worst = max(worst, compare_out(spec["store"], got[flipped], ref,
-                                       w.name + " (flipped tokens, GPU selection)"))
+                                       w.name + " (flipped tokens, GPU selection)",
+                                       absum=terms))
     return good, flipped, worst
 
 
@@ -481,9 +482,10 @@ def test_fused_combine(w, gathered):
     if w.n <= 2048:
         spec, logits, S, lse, r = _oracle_from_x(w, inp)
         bad = explained_routing_diff(spec, r, layer.route, S, host(inp.get("sel_bias")))
-        ref = oracle.layer_forward(spec, host(inp["X"]), r, expert_weights_from(inp),
-                                   expert_weights_from(inp, "s") if w.n_shared else None)
+        ref, terms = oracle.layer_forward(spec, host(inp["X"]), r, expert_weights_from(inp),
+                                          expert_weights_from(inp, "s") if w.n_shared else None,
+                                          absum=True)
         keep = np.array([t not in bad for t in range(w.n)])
         # the fused epilogue adds each gate-scaled row unrounded (no bf16 Y)
         # in a varying order: one bf16 rounding fewer than the oracle's
-        compare_out(spec["store"], got[keep], ref[keep], w.name)
+        compare_out(spec["store"], got[keep], ref[keep], w.name, absum=terms[keep])
