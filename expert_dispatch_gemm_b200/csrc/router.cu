@@ -31,8 +31,9 @@ template <int ET_, int TM_, int TN_, int LX_, int WX_, int WY_, int WK_, int BK_
 struct RCfg {
   static constexpr int ET = ET_, TM = TM_, TN = TN_, LX = LX_, LY = 32 / LX_, WX = WX_,
                        WY = WY_, WK = WK_, BK = BK_, ST = ST_, BM = WX_ * LX_ * TM_;
+  static constexpr int NW = WX * WY * WK, NT = 32 * NW;  // warps, threads
   static_assert(WY * LY * TN == ET, "columns");
-  static_assert(WX * WY * WK == 8, "8 warps");
+  static_assert(NW == 8 || NW == 12, "8 or 12 warps");
   static_assert(TN == 4 || TN == 8 || TN == 16, "TN");
   static_assert(TM >= 1 && TM <= 8, "TM");
   static_assert(BK % WK == 0 && ST >= 2, "pipeline");
@@ -64,6 +65,11 @@ template <int TM> using R256A = RCfg<256, TM, 8, 4, 1, 4, 2, 32, 3>; // BM = 4 T
 // so the FMA pipe, not shared-memory bandwidth, sets the pace; one CTA per
 // SM (about 160 registers a thread)
 template <int TM> using R256B = RCfg<256, TM, 16, 4, 2, 2, 2, 32, 3>; // BM = 8 TM
+// the same tiles with a three-way k split over 12 warps (three per SM
+// sub-partition instead of two, so one warp's shared-memory and dependency
+// waits hide behind two others'), 48-deep chunks; one CTA per SM, at most
+// 168 registers a thread
+template <int TM> using R256C = RCfg<256, TM, 16, 4, 2, 2, 3, 48, 3>; // BM = 8 TM
 
 constexpr int kSelectRowsPerWarp = 4;
 
@@ -86,8 +92,8 @@ static int num_sms_cached() {
 // small-row one when the big tile would leave SMs without a CTA. bf16 X with
 // E > 32: the (family, TM) whose rows per SM, BM * ceil(CTAs / SMs), is
 // smallest (ties to the larger BM). Codes: kFamilyCode + fam * 16 + TM with
-// fam 1 = R64A, 2 = R64C, 3 = R128A, 4 = R256A, 5 = R256B; otherwise the
-// fixed tile's ET (257: R256s, 65: R64s).
+// fam 1 = R64A, 2 = R64C, 3 = R128A, 4 = R256A, 5 = R256B, 6 = R256C; otherwise
+// the fixed tile's ET (257: R256s, 65: R64s).
 constexpr int kFamilyCode = 1000;
 struct RouterFamily {
   int code, unit, tm_lo;
@@ -98,9 +104,9 @@ static int router_variant(int E, int n, bool x_bf16) {
   if (x_bf16 && et >= 64) {
     static const RouterFamily fams64[] = {{1, 4, 4}, {2, 16, 4}};
     static const RouterFamily fams128[] = {{3, 8, 2}};
-    static const RouterFamily fams256[] = {{4, 4, 4}, {5, 8, 4}};
+    static const RouterFamily fams256[] = {{6, 8, 4}, {5, 8, 4}, {4, 4, 4}};
     const RouterFamily* fams = et == 64 ? fams64 : et == 128 ? fams128 : fams256;
-    const int nf = et == 128 ? 1 : 2;
+    const int nf = et == 128 ? 1 : et == 64 ? 2 : 3;
     long long best_cost = -1;
     int best = 0, best_bm = 0;
     for (int f = 0; f < nf; ++f)
@@ -120,6 +126,9 @@ static int router_variant(int E, int n, bool x_bf16) {
         // (TM + 8 per TM*8 FFMAs per step), the 16-column tiles by the FMA
         // pipe: charge the narrower tile a quarter more per row
         if (fams[f].code == 4) cost = cost * 5 / 4;
+        // 12 warps where their registers fit (TM <= 7); listed first, so an
+        // equal cost keeps them
+        if (fams[f].code == 6 && tm > 7) continue;
         if (best_cost < 0 || cost < best_cost || (cost == best_cost && bm > best_bm)) {
           best_cost = cost;
           best = kFamilyCode + fams[f].code * 16 + tm;
@@ -145,8 +154,8 @@ static void variant_tile(int v, int* bm, int* bk) {
     case 257: *bm = R256s::BM; *bk = R256s::BK; return;
     default: {
       const int code = v - kFamilyCode, fam = code / 16, tm = code % 16;
-      *bm = (fam == 2 ? 16 : fam == 3 || fam == 5 ? 8 : 4) * tm;
-      *bk = fam == 1 ? 64 : 32;
+      *bm = (fam == 2 ? 16 : fam == 3 || fam == 5 || fam == 6 ? 8 : 4) * tm;
+      *bk = fam == 1 ? 64 : fam == 6 ? 48 : 32;
     }
   }
 }
@@ -285,9 +294,10 @@ __device__ __forceinline__ void tc_select_row(const float (&key)[V], const float
 // Adds the bias, applies the score function, writes logits / scores / lse,
 // selects the token-choice experts, and leaves this CTA's partial column sums
 // of S and its sum of lse^2 in colsum / lse2 at index blockIdx.x.
-// colsum_w [8][ET] floats and lse2_w [8] doubles are shared-memory scratch.
+// colsum_w [NW][ET] floats and lse2_w [NW] doubles are shared-memory scratch
+// (NW warps).
 // ---------------------------------------------------------------------------
-template <int ET>
+template <int ET, int NW>
 __device__ __forceinline__ void router_rows_epilogue(const RouterArgs& a, const float* Ls,
                                                      float* colsum_w, double* lse2_w, int BM,
                                                      int m0) {
@@ -300,7 +310,7 @@ __device__ __forceinline__ void router_rows_epilogue(const RouterArgs& a, const 
   for (int v = 0; v < V; ++v) csum[v] = 0.0f;
   double my_lse2 = 0.0;
 
-  for (int r = warp; r < BM; r += 8) {
+  for (int r = warp; r < BM; r += NW) {
     const int t = m0 + r;
     if (t >= n) break;
     float l[V], s[V], key[V];
@@ -357,14 +367,14 @@ __device__ __forceinline__ void router_rows_epilogue(const RouterArgs& a, const 
   }
   if (lane == 0) lse2_w[warp] = my_lse2;
   __syncthreads();
-  for (int cc = tid; cc < E; cc += 256) {
+  for (int cc = tid; cc < E; cc += 32 * NW) {
     float sum = 0.0f;
-    for (int w = 0; w < 8; ++w) sum += colsum_w[w * ET + cc];
+    for (int w = 0; w < NW; ++w) sum += colsum_w[w * ET + cc];
     a.colsum[(size_t)blockIdx.x * E + cc] = sum;
   }
   if (tid == 0) {
     double sum = 0.0;
-    for (int w = 0; w < 8; ++w) sum += lse2_w[w];
+    for (int w = 0; w < NW; ++w) sum += lse2_w[w];
     a.lse2[blockIdx.x] = sum;
   }
 }
@@ -388,12 +398,12 @@ struct RouterSmem {
   static constexpr size_t as_bytes = (size_t)C::BK * AST * XB;
   static constexpr size_t main_bytes = xs_bytes + ws_bytes + as_bytes;
   static constexpr size_t epi_bytes =
-      ((size_t)C::WK * C::BM * (C::ET + 1) + 8 * C::ET) * 4 + 8 * 8;
+      ((size_t)C::WK * C::BM * (C::ET + 1) + C::NW * C::ET) * 4 + C::NW * 8;
   static constexpr size_t bytes = (main_bytes > epi_bytes ? main_bytes : epi_bytes) + 128;
 };
 
 template <class C, bool XBF16>
-__global__ void __launch_bounds__(256) router_kernel(RouterArgs a) {
+__global__ void __launch_bounds__(C::NT) router_kernel(RouterArgs a) {
   pdl_wait();
   using SM = RouterSmem<C, XBF16>;
   constexpr int ET = C::ET, BM = C::BM, BK = C::BK, TM = C::TM, TN = C::TN;
@@ -429,7 +439,7 @@ __global__ void __launch_bounds__(256) router_kernel(RouterArgs a) {
     constexpr int XCH = BM * BK * XB / 16;          // 16-byte pieces of the X chunk
     constexpr int XPR = BK * XB / 16;               // pieces per row
     unsigned char* xs = Xs + (size_t)st * BM * BK * XB;
-    for (int q = tid; q < XCH; q += 256) {
+    for (int q = tid; q < XCH; q += C::NT) {
       const int r = q / XPR, p = q % XPR;
       const int row = m0 + r, k = k0 + p * (16 / XB);
       const bool ok = row < n && k < d;
@@ -440,7 +450,7 @@ __global__ void __launch_bounds__(256) router_kernel(RouterArgs a) {
     float* ws = Ws + (size_t)st * BK * ET;
     if (w_vec) {
       constexpr int WCH = BK * ET / 4;
-      for (int q = tid; q < WCH; q += 256) {
+      for (int q = tid; q < WCH; q += C::NT) {
         const int kk = q / (ET / 4), c4 = (q % (ET / 4)) * 4;
         const int k = k0 + kk;
         const bool ok = k < d && c4 < E;
@@ -448,7 +458,7 @@ __global__ void __launch_bounds__(256) router_kernel(RouterArgs a) {
       }
     } else {
       constexpr int WCH = BK * ET;
-      for (int q = tid; q < WCH; q += 256) {
+      for (int q = tid; q < WCH; q += C::NT) {
         const int kk = q / ET, cc = q % ET;
         const int k = k0 + kk;
         const bool ok = k < d && cc < E;
@@ -475,7 +485,7 @@ __global__ void __launch_bounds__(256) router_kernel(RouterArgs a) {
       const unsigned char* xs = Xs + (size_t)st * BM * BK * XB;
       constexpr int EPP = 16 / XB;                 // elements per 16-byte piece
       constexpr int PCS = BM * BK / EPP;
-      for (int q = tid; q < PCS; q += 256) {
+      for (int q = tid; q < PCS; q += C::NT) {
         const int r = q % BM, p = q / BM;
         const uint4 v = *reinterpret_cast<const uint4*>(xs + (size_t)r * BK * XB + p * 16);
         const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
@@ -568,7 +578,7 @@ __global__ void __launch_bounds__(256) router_kernel(RouterArgs a) {
       Ls[(wk * BM + row0 + i) * LST + colb + (j / 4) * 4 * C::LY + (j % 4)] = acc[i][j];
   __syncthreads();
   if (C::WK > 1) {
-    for (int q = tid; q < BM * ET; q += 256) {
+    for (int q = tid; q < BM * ET; q += C::NT) {
       const int r = q / ET, cc = q % ET;
       float s = Ls[r * LST + cc];
 #pragma unroll
@@ -582,15 +592,15 @@ __global__ void __launch_bounds__(256) router_kernel(RouterArgs a) {
     // a k slice: its partial logits go to a.partial[slice][n][E]; the
     // reduce kernel sums the slices in order and runs the epilogue
     float* part = a.partial + (size_t)blockIdx.y * n * E;
-    for (int q = tid; q < BM * E; q += 256) {
+    for (int q = tid; q < BM * E; q += C::NT) {
       const int r = q / E, cc = q % E;
       if (m0 + r < n) part[(size_t)(m0 + r) * E + cc] = Ls[r * LST + cc];
     }
     return;
   }
-  float* colsum_w = Ls + C::WK * BM * LST;                          // [8][ET]
-  double* lse2_w = reinterpret_cast<double*>(colsum_w + 8 * ET);     // [8]
-  router_rows_epilogue<ET>(a, Ls, colsum_w, lse2_w, BM, m0);
+  float* colsum_w = Ls + C::WK * BM * LST;                          // [NW][ET]
+  double* lse2_w = reinterpret_cast<double*>(colsum_w + C::NW * ET);  // [NW]
+  router_rows_epilogue<ET, C::NW>(a, Ls, colsum_w, lse2_w, BM, m0);
 }
 
 // Split-k router, second pass: kRouterMinBlockRows (4) rows per CTA, so that
@@ -638,7 +648,7 @@ __global__ void __launch_bounds__(256) router_reduce_kernel(RouterArgs a) {
     }
   }
   __syncthreads();
-  router_rows_epilogue<ET>(a, Ls, colsum_w, lse2_w, BMR, m0);
+  router_rows_epilogue<ET, 8>(a, Ls, colsum_w, lse2_w, BMR, m0);
 }
 
 // k slices for a batch whose row tiles would fill fewer than half the SMs
@@ -666,8 +676,8 @@ static cudaError_t launch_router_t(const RouterArgs& a0, cudaStream_t s) {
   a.ksplit = router_ksplit(a.E, a.n, a.d, XBF16);
   a.chunks_per_split = ceil_div(nchunks, a.ksplit);
   if (a.ksplit > 1 && !a.partial) return cudaErrorInvalidValue;
-  if (a.ksplit == 1) return launch_pdl(kern, grid, 256, bytes, s, a);
-  e = launch_pdl(kern, dim3(grid, a.ksplit), 256, bytes, s, a);
+  if (a.ksplit == 1) return launch_pdl(kern, grid, C::NT, bytes, s, a);
+  e = launch_pdl(kern, dim3(grid, a.ksplit), C::NT, bytes, s, a);
   if (e != cudaSuccess) return e;
   return launch_pdl(router_reduce_kernel<C::ET>, ceil_div(a.n, kRouterMinBlockRows), 256, 0,
                     s, a);
@@ -686,6 +696,17 @@ static cudaError_t launch_family(int tm, const RouterArgs& a, cudaStream_t s) {
   }
 }
 
+// families whose register budget stops at TM = 7 (12 warps)
+template <template <int> class F>
+static cudaError_t launch_family_upto7(int tm, const RouterArgs& a, cudaStream_t s) {
+  switch (tm) {
+    case 4: return launch_router_t<F<4>, true>(a, s);
+    case 5: return launch_router_t<F<5>, true>(a, s);
+    case 6: return launch_router_t<F<6>, true>(a, s);
+    default: return launch_router_t<F<7>, true>(a, s);
+  }
+}
+
 static cudaError_t launch_router_bf16_family(int code, const RouterArgs& a, cudaStream_t s) {
   const int fam = code / 16, tm = code % 16;
   switch (fam) {
@@ -693,7 +714,8 @@ static cudaError_t launch_router_bf16_family(int code, const RouterArgs& a, cuda
     case 2: return launch_family<R64C>(tm, a, s);
     case 3: return launch_family<R128A>(tm, a, s);
     case 4: return launch_family<R256A>(tm, a, s);
-    default: return launch_family<R256B>(tm, a, s);
+    case 5: return launch_family<R256B>(tm, a, s);
+    default: return launch_family_upto7<R256C>(tm, a, s);
   }
 }
 
