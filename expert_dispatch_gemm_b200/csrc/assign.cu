@@ -22,7 +22,8 @@ __device__ __forceinline__ uint32_t ordered_key(float f) {
 
 // ---------------------------------------------------------------------------
 // Expert choice: one CTA per expert. Radix-select the k-th largest key of the
-// column, take every key above it plus the lowest-index ties (ordered block
+// column (one block histogram per 8-bit pass, warp-aggregated shared-memory
+// atomics), take every key above it plus the lowest-index ties (ordered block
 // scans, no atomics), then order the k picks by (score desc, token asc): by
 // counting ranks for k <= kEcRankMax, by a bitonic sort of 64-bit composite
 // keys beyond that. The dense slot map is [E, n] so each CTA clears and
@@ -67,7 +68,6 @@ __global__ void __launch_bounds__(NT) select_ec_kernel(SelectEcArgs a) {
   while (kp < k) kp <<= 1;
   uint64_t* sbuf = reinterpret_cast<uint64_t*>(ec_smem);    // [k] picks, or [kp] to sort
   uint64_t* sorted = by_rank ? sbuf + k : sbuf;              // [k]
-  int* whist = reinterpret_cast<int*>(sbuf + (by_rank ? 2 * k : kp));  // [32 warps][256]
   __shared__ int hist[256];
   __shared__ int warp_tot[32];
   __shared__ uint32_t s_prefix, s_mask;
@@ -93,14 +93,13 @@ __global__ void __launch_bounds__(NT) select_ec_kernel(SelectEcArgs a) {
   }
   __syncthreads();
 
-  int* myhist = whist + warp * 256;
+  for (int b = tid; b < 256; b += NT) hist[b] = 0;
+  __syncthreads();
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
-    for (int i = lane; i < 256; i += 32) myhist[i] = 0;
     const uint32_t prefix = s_prefix, mask = s_mask;
-    __syncwarp();
-    // warp-aggregated counts: the lanes that share a digit add once, through
-    // their lowest lane, so a warp's private histogram needs no atomics
+    // one block histogram; warp-aggregated: the lanes that share a digit add
+    // once, through their lowest lane (integer counts: exact in any order)
 #pragma unroll
     for (int i = 0; i < kEcMaxPerThread; ++i) {
       if (i >= C) break;
@@ -110,22 +109,18 @@ __global__ void __launch_bounds__(NT) select_ec_kernel(SelectEcArgs a) {
       if (ok) {
         const unsigned dig = (kreg[i] >> shift) & 255u;
         const unsigned peers = __match_any_sync(act, dig);
-        if (lane == __ffs(peers) - 1) myhist[dig] += __popc(peers);
+        if (lane == __ffs(peers) - 1) atomicAdd(&hist[dig], (int)__popc(peers));
       }
     }
     __syncthreads();
-    for (int b = tid; b < 256; b += NT) {
-      int c = 0;
-      for (int w = 0; w < NT / 32; ++w) c += whist[w * 256 + b];
-      hist[b] = c;
-    }
-    __syncthreads();
     if (warp == 0) {
-      // lane l holds digits 255-8l down to 248-8l (descending)
+      // lane l holds digits 255-8l down to 248-8l (descending); it clears
+      // them for the next pass as it reads them
       int cnt[8], local = 0;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         cnt[i] = hist[255 - 8 * lane - i];
+        hist[255 - 8 * lane - i] = 0;
         local += cnt[i];
       }
       int incl = local;
@@ -139,11 +134,12 @@ __global__ void __launch_bounds__(NT) select_ec_kernel(SelectEcArgs a) {
       const unsigned who = __ballot_sync(0xffffffffu, here);
       if (here && lane == __ffs(who) - 1) {
         int above = excl;
-        int digit = 0;
+        int digit = 0, dcount = 0;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           if (above + cnt[i] >= need) {
             digit = 255 - 8 * lane - i;
+            dcount = cnt[i];
             break;
           }
           above += cnt[i];
@@ -152,7 +148,7 @@ __global__ void __launch_bounds__(NT) select_ec_kernel(SelectEcArgs a) {
         s_prefix = prefix | ((uint32_t)digit << shift);
         s_mask = mask | (255u << shift);
         // every key in the chosen bucket is a pick: no later digit matters
-        if (above + hist[digit] == need) s_done = 1;
+        if (above + dcount == need) s_done = 1;
       }
     }
     __syncthreads();
@@ -261,11 +257,10 @@ __global__ void __launch_bounds__(NT) select_ec_kernel(SelectEcArgs a) {
   }
 }
 
-static size_t select_ec_smem(int nt, int k) {
+static size_t select_ec_smem(int /*nt*/, int k) {
   int kp = 1;
   while (kp < k) kp <<= 1;
-  const size_t buf = k <= kEcRankMax ? (size_t)2 * k * 8 : (size_t)kp * 8;
-  return buf + (size_t)(nt / 32) * 256 * 4;
+  return k <= kEcRankMax ? (size_t)2 * k * 8 : (size_t)kp * 8;
 }
 
 template <int NT>
