@@ -85,3 +85,15 @@ def test_training_cpu_baseline_and_flop_count():
     rows = 2400 + w.n
     assert bf["dw13"] == 2 * (2.0 * rows * w.d * w.h)  # SwiGLU: W1 and W3
     assert "recompute" in bench.backward_flops(wl.EC_FP32, 1024)
+
+
+def test_reference_arm_other_ranks_exit_without_output():
+    """Under torchrun the reference arm runs on rank 0 alone; the other ranks
+    exit 0 without work or output."""
+    w = wl.SMALL[4]
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", w.name, "--steps", "2", "--warmup", "3"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT, env=env)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert out.stdout.strip() == ""
