@@ -18,10 +18,13 @@ from .workloads import Workload
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmoe.so")
 # the checked build (every out-of-range routing index reported in the error
-# word); MOE_LIBRARY=checked in the environment loads it instead
+# word); MOE_LIBRARY=checked in the environment loads it instead, and
+# MOE_LIBRARY=<path of a .so> loads another build of the same sources
 CHECKED_LIB_PATH = os.path.join(_PKG, "libmoe_checked.so")
 if os.environ.get("MOE_LIBRARY") == "checked":
     LIB_PATH = CHECKED_LIB_PATH
+elif os.environ.get("MOE_LIBRARY"):
+    LIB_PATH = os.path.abspath(os.environ["MOE_LIBRARY"])
 
 # enums and limits of include/moe.h
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, \
