@@ -41,11 +41,6 @@ constexpr int kSStageBytes = kSABytes + kSBBytes;
 constexpr int kSTmemCols = 512;                  // two 256-column accumulators
 constexpr int kSMaxTokens = 256;                 // tokens per tile (MMA N <= 256)
 constexpr uint64_t kSWaitNs = 2000000000ull;     // 2 s
-// The weight tiles (the A side) come from HBM once each, at the MMA's pace,
-// with a latency under load that a ring of shared-memory stages alone does not
-// cover: the producer also brings the weight rows of the k-block this many
-// steps ahead of its loads into L2, so the loads themselves hit L2.
-constexpr int kSPrefetch = 8;
 
 struct SwapParams {
   const int32_t* offsets;   // [E+1] segment starts
@@ -236,24 +231,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSThreads, 1)
       int stage = 0, issued = 0;
       uint32_t phase = 0;
       bool ok = true;
-      // L2 prefetch cursor over the same (tile, k-block) sequence, ahead
-      int pf_tile = pair_id, pf_kb = 0, pf_decoded = -1, pf_wrow = 0;
-      bool pf_shared = false;
-      auto prefetch_next = [&]() {
-        if (pf_tile >= total) return;
-        if (pf_decoded != pf_tile) {
-          const SwapTile u = decode_swap(pf_tile, p, st, routed);
-          pf_wrow = u.expert * p.m_per_expert + u.m0 + (int)rank * 128;
-          pf_shared = u.shared;
-          pf_decoded = pf_tile;
-        }
-        sm100::tma_prefetch_l2_2d(pf_shared ? &tmWs : &tmW, pf_kb * kSBK, pf_wrow);
-        if (++pf_kb == KB) {
-          pf_kb = 0;
-          pf_tile += num_pairs;
-        }
-      };
-      for (int i = 0; i < kSPrefetch; ++i) prefetch_next();
       for (int tile = pair_id; ok && tile < total; tile += num_pairs) {
         const SwapTile t = decode_swap(tile, p, st, routed);
         const CUtensorMap* tm[3];
@@ -270,7 +247,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSThreads, 1)
         // this CTA's half of the tile's tokens
         const long long trow1 = t.tok_row + (long long)rank * (t.n / 2);
         for (int kb = 0; kb < KB; ++kb) {
-          prefetch_next();
           if (!swap_wait<false>(&st->empty[stage], phase ^ 1u, st, p.err, kErrGemmTimeout | 0xA1)) {
             ok = false;
             break;
@@ -397,267 +373,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// SwiGLU up projection with the weights as the M side: H_e^T = silu(W1_e
-// X_e^T) * (W3_e X_e^T). A tile is (expert, 256 hidden units, up to 256 of
-// the expert's tokens). Each CTA loads its 128 rows of W1 and the same 128
-// rows of W3 as two A operands and half of the tile's tokens as B; the leader
-// issues two M=256 MMAs per 16-deep step with the same B, one into TMEM
-// columns [0, 256) (W1: the gate pre-activation U) and one into [256, 512)
-// (W3: V), so a hidden unit's U and V sit in the same TMEM lane and meet in
-// one epilogue thread. The 512 columns hold one tile; the producer runs ahead
-// into the next tile's stages while the epilogue drains.
-//   warp 0     TMA producer (4-stage ring: W1 16 KB + W3 16 KB + tokens <= 16 KB);
-//   warp 1     TMEM allocation; the leader's lane 0 issues the MMAs;
-//   warps 2-5  epilogue: U and V 32 tokens at a time, silu(U) V in fp32,
-//              bf16, a transpose through shared memory, and 16-byte stores
-//              of each token's 32 consecutive hidden units.
-// ---------------------------------------------------------------------------
-constexpr int kUStages = 4;
-constexpr int kUWBytes = 128 * kSBK * 2;                       // 128 rows of W1 or W3
-constexpr int kUStageBytes = 2 * kUWBytes + kSBBytes;          // 48 KB
-
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSThreads, 1)
-    tc_swap_up_pair_kernel(const __grid_constant__ CUtensorMap tmT0,
-                           const __grid_constant__ CUtensorMap tmT1,
-                           const __grid_constant__ CUtensorMap tmT2,
-                           const __grid_constant__ CUtensorMap tmTs0,
-                           const __grid_constant__ CUtensorMap tmTs1,
-                           const __grid_constant__ CUtensorMap tmTs2,
-                           const __grid_constant__ CUtensorMap tmW1,
-                           const __grid_constant__ CUtensorMap tmW3,
-                           const __grid_constant__ CUtensorMap tmW1s,
-                           const __grid_constant__ CUtensorMap tmW3s, const SwapParams p) {
-  extern __shared__ __align__(1024) unsigned char usm[];
-  unsigned char* base = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(usm) + 1023) & ~uintptr_t(1023));
-  SwapState* st = reinterpret_cast<SwapState*>(base + kUStages * kUStageBytes);
-  // epilogue staging, [4 warps][32 tokens][32 hidden units] bf16
-  __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(
-      base + kUStages * kUStageBytes + ((sizeof(SwapState) + 127) & ~size_t(127)));
-  auto sW1 = [&](int s) { return base + s * kUStageBytes; };
-  auto sW3 = [&](int s) { return base + s * kUStageBytes + kUWBytes; };
-  auto sB = [&](int s) { return base + s * kUStageBytes + 2 * kUWBytes; };
-
-  const uint32_t rank = sm100::cluster_ctarank();
-  const bool leader = rank == 0;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (tid == 0) {
-    for (int s = 0; s < kUStages; ++s) {
-      sm100::mbar_init(&st->full[s], 1);
-      sm100::mbar_init(&st->empty[s], 1);
-    }
-    sm100::mbar_init(&st->tfull[0], 1);
-    sm100::mbar_init(&st->tempty[0], 256);
-    sm100::mbar_init(&st->drain, 1);
-    st->abort_flag = 0;
-    sm100::fence_mbar_init();
-  }
-  if (warp == 1) {
-    sm100::tmem_alloc_pair(&st->tmem_base, kSTmemCols);
-    sm100::tmem_relinquish_pair();
-  }
-  // the set-up above needs nothing from the previous kernel; the segment
-  // starts, the counts and the dispatched rows are read from here on
-  pdl_wait();
-  for (int i = tid; i <= p.E; i += kSThreads) st->offs[i] = p.offsets[i];
-  for (int i = tid; i < p.E; i += kSThreads) {
-    const int seg = p.offsets[i + 1] - p.offsets[i];
-    const int c = p.counts ? p.counts[i] : seg;
-    if (seg < 0 || c < 0 || c > seg) bad_index(p.err, kSiteSwapOffsets);
-    st->cnt[i] = max(0, min(c, seg));  // never past the expert's own segment
-  }
-  __syncthreads();
-  if (tid == 0) {
-    int run = 0;
-    for (int e = 0; e < p.E; ++e) {
-      st->tprefix[e] = run;
-      run += (st->cnt[e] + kSMaxTokens - 1) / kSMaxTokens * p.mt_tiles;
-    }
-    st->tprefix[p.E] = run;
-  }
-  sm100::tc_fence_before();
-  __syncthreads();
-  sm100::cluster_sync();  // both CTAs' barriers exist before any remote arrive
-  sm100::tc_fence_after();
-  const uint32_t tmem = st->tmem_base;
-
-  const int routed = st->tprefix[p.E];
-  const int shared_chunks = (p.n + kSMaxTokens - 1) / kSMaxTokens;
-  const int total = routed + p.n_shared * p.mt_tiles * shared_chunks;
-  const int KB = p.K / kSBK;
-  const int pair_id = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      int stage = 0, issued = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      // L2 prefetch cursor over the same (tile, k-block) sequence, ahead
-      int pf_tile = pair_id, pf_kb = 0, pf_decoded = -1, pf_wrow = 0;
-      bool pf_shared = false;
-      auto prefetch_next = [&]() {
-        if (pf_tile >= total) return;
-        if (pf_decoded != pf_tile) {
-          const SwapTile u = decode_swap(pf_tile, p, st, routed);
-          pf_wrow = u.expert * p.m_per_expert + u.m0 + (int)rank * 128;
-          pf_shared = u.shared;
-          pf_decoded = pf_tile;
-        }
-        sm100::tma_prefetch_l2_2d(pf_shared ? &tmW1s : &tmW1, pf_kb * kSBK, pf_wrow);
-        sm100::tma_prefetch_l2_2d(pf_shared ? &tmW3s : &tmW3, pf_kb * kSBK, pf_wrow);
-        if (++pf_kb == KB) {
-          pf_kb = 0;
-          pf_tile += num_pairs;
-        }
-      };
-      for (int i = 0; i < kSPrefetch; ++i) prefetch_next();
-      for (int tile = pair_id; ok && tile < total; tile += num_pairs) {
-        const SwapTile t = decode_swap(tile, p, st, routed);
-        const CUtensorMap* tm[3];
-        if (t.shared) {
-          tm[0] = &tmTs0; tm[1] = &tmTs1; tm[2] = &tmTs2;
-        } else {
-          tm[0] = &tmT0; tm[1] = &tmT1; tm[2] = &tmT2;
-        }
-        const int b1 = box_rows(t.n);
-        const CUtensorMap* m1 = tm[b1 == 32 ? 0 : b1 == 64 ? 1 : 2];
-        const uint32_t bytes = 2 * kUWBytes + (uint32_t)b1 * kSBK * 2;
-        const CUtensorMap* mw1 = t.shared ? &tmW1s : &tmW1;
-        const CUtensorMap* mw3 = t.shared ? &tmW3s : &tmW3;
-        const int wrow = t.expert * p.m_per_expert + t.m0 + (int)rank * 128;  // this CTA's 128
-        // this CTA's half of the tile's tokens
-        const long long trow1 = t.tok_row + (long long)rank * (t.n / 2);
-        for (int kb = 0; kb < KB; ++kb) {
-          prefetch_next();
-          if (!swap_wait<false>(&st->empty[stage], phase ^ 1u, st, p.err, kErrGemmTimeout | 0xD1)) {
-            ok = false;
-            break;
-          }
-          const uint32_t fl = sm100::mapa_shared(sm100::smem_addr(&st->full[stage]), 0);
-          if (leader) sm100::mbar_arrive_expect_tx(&st->full[stage], 2 * bytes);
-          sm100::tma_load_2d_pair(sW1(stage), mw1, fl, kb * kSBK, wrow);
-          sm100::tma_load_2d_pair(sW3(stage), mw3, fl, kb * kSBK, wrow);
-          sm100::tma_load_2d_pair(sB(stage), m1, fl, kb * kSBK, (int)trow1);
-          ++issued;
-          if (++stage == kUStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      }
-      if (!ok && leader) {
-        // wait (bounded) until the copies of the outstanding stages have landed
-        int s = stage;
-        uint32_t ph = phase;
-        const int pending = issued < kUStages ? issued : kUStages;
-        for (int i = 0; i < pending; ++i) {
-          if (--s < 0) {
-            s = kUStages - 1;
-            ph ^= 1u;
-          }
-          const uint64_t t0 = global_timer_ns();
-          while (!sm100::mbar_try_wait(&st->full[s], ph) && global_timer_ns() - t0 < kSWaitNs) {
-          }
-        }
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0 && leader) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int local = 0;
-      bool ok = true;
-      for (int tile = pair_id; ok && tile < total; tile += num_pairs, ++local) {
-        const SwapTile t = decode_swap(tile, p, st, routed);
-        const uint32_t acc_phase = (uint32_t)local & 1u;
-        if (!swap_wait<true>(&st->tempty[0], acc_phase ^ 1u, st, p.err, kErrGemmTimeout | 0xE2)) {
-          ok = false;
-          break;
-        }
-        sm100::tc_fence_after();
-        const uint32_t idesc = sm100::idesc_bf16_f32(256, t.n);
-        for (int kb = 0; kb < KB; ++kb) {
-          if (!swap_wait<false>(&st->full[stage], phase, st, p.err, kErrGemmTimeout | 0xE3)) {
-            ok = false;
-            break;
-          }
-          sm100::tc_fence_after();
-          const uint64_t d1 = sm100::sw128_kmajor_desc(sm100::smem_addr(sW1(stage)));
-          const uint64_t d3 = sm100::sw128_kmajor_desc(sm100::smem_addr(sW3(stage)));
-          const uint64_t db = sm100::sw128_kmajor_desc(sm100::smem_addr(sB(stage)));
-#pragma unroll
-          for (int k = 0; k < kSBK / 16; ++k) {
-            sm100::umma_f16_pair(tmem, d1 + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
-            sm100::umma_f16_pair(tmem + 256u, d3 + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
-          }
-          sm100::umma_commit_pair_mc(&st->empty[stage], 0x3);
-          if (++stage == kUStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-        if (!ok) break;
-        sm100::umma_commit_pair_mc(&st->tfull[0], 0x3);
-      }
-      sm100::umma_commit_pair_mc(&st->drain, 0x1);
-      const uint64_t t0 = global_timer_ns();
-      while (!sm100::mbar_try_wait(&st->drain, 0) && global_timer_ns() - t0 < kSWaitNs) {
-      }
-    }
-  } else {
-    // epilogue: TMEM lanes = this CTA's 128 hidden units, columns = tokens
-    // (U in [0, 256), V in [256, 512)); warp q owns lanes 32q..32q+31
-    const int q = warp & 3;
-    constexpr int CW = 32;            // hidden units per warp
-    constexpr int VPR = CW * 2 / 16;  // 16-byte pieces of a token's CW units
-    __nv_bfloat16* stg = stage + q * (32 * CW);  // [32 tokens][CW] bf16
-    int local = 0;
-    for (int tile = pair_id; tile < total; tile += num_pairs, ++local) {
-      const SwapTile t = decode_swap(tile, p, st, routed);
-      const uint32_t acc_phase = (uint32_t)local & 1u;
-      const int col0 = t.m0 + (int)rank * 128 + 32 * q;
-      __nv_bfloat16* outt = p.out + (size_t)t.out_row * p.n_out + col0;
-      if (!swap_wait<true>(&st->tfull[0], acc_phase, st, p.err, kErrGemmTimeout | 0xF4)) break;
-      sm100::tc_fence_after();
-      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16);
-#pragma unroll 1
-      for (int cc = 0; cc < t.n; cc += 32) {
-        uint32_t u[32], v[32];
-        sm100::tmem_ld_32x32b_x32(tbase + cc, u);
-        sm100::tmem_ld_32x32b_x32(tbase + 256u + cc, v);
-        sm100::tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float a = __uint_as_float(u[i]);
-          const float b = __uint_as_float(v[i]);
-          stg[i * CW + lane] = __float2bfloat16_rn(a * __frcp_rn(1.0f + __expf(-a)) * b);
-        }
-        __syncwarp();
-        // each token's CW hidden units leave as 16-byte stores
-#pragma unroll
-        for (int idx = lane; idx < 32 * VPR; idx += 32) {
-          const int i = idx / VPR, vv = idx % VPR;
-          const int j = cc + i;  // token within the tile
-          if (j < t.valid)
-            *reinterpret_cast<uint4*>(outt + (size_t)j * p.n_out + vv * 8) =
-                *reinterpret_cast<const uint4*>(stg + i * CW + vv * 8);
-        }
-        __syncwarp();
-      }
-      sm100::tc_fence_before();
-      sm100::mbar_arrive_cluster(sm100::mapa_shared(sm100::smem_addr(&st->tempty[0]), 0));
-    }
-  }
-  sm100::tc_fence_before();
-  __syncthreads();
-  sm100::cluster_sync();  // no CTA leaves while its peer may still signal it
-  if (warp == 1) {
-    sm100::tc_fence_after();
-    sm100::tmem_dealloc_pair(tmem, kSTmemCols);
-  }
-}
-
-// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 struct SwapMaps {
@@ -693,67 +408,7 @@ static int swap_pairs(const SwapParams& p, long long max_routed_rows) {
   return g < 1 ? 1 : (int)g;
 }
 
-static cudaError_t launch_swap_up(const SwapMaps& m, const CUtensorMap& w3,
-                                  const CUtensorMap& w3s, const SwapParams& p, int pairs,
-                                  cudaStream_t s) {
-  const size_t bytes = (size_t)kUStages * kUStageBytes +
-                       ((sizeof(SwapState) + 127) & ~size_t(127)) +
-                       4 * 32 * 32 * sizeof(__nv_bfloat16) + 1024;
-  auto kern = tc_swap_up_pair_kernel;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(kern, 2 * pairs, kSThreads, bytes, s, m.t[0], m.t[1], m.t[2], m.ts[0],
-                    m.ts[1], m.ts[2], m.w, w3, m.ws, w3s, p);
-}
-
 }  // namespace
-
-bool swap_up_supported(const FfnArgs& f) {
-  return f.act == MOE_ACT_SWIGLU && f.X_perm != nullptr && f.save_u == nullptr &&
-         f.counts != nullptr && f.E <= MOE_MAX_EXPERTS && f.h % 256 == 0 && f.d % kSBK == 0;
-}
-
-// H = silu(X_perm W1^T) * (X_perm W3^T) per expert over each expert's real
-// tokens (and per shared expert over the n rows of X), weights as the M side;
-// padding rows of H are not written
-moe_status run_ffn_up_swap(const FfnArgs& f, cudaStream_t s) {
-  SwapMaps m;
-  if (!token_maps(m.t, f.X_perm, f.rows, f.d)) return MOE_ERR_UNSUPPORTED;
-  CUtensorMap w3, w3s;
-  if (!make_bf16_sw128_map(&m.w, f.W1, (long long)f.E * f.h, f.d, 128)) return MOE_ERR_UNSUPPORTED;
-  if (!make_bf16_sw128_map(&w3, f.W3, (long long)f.E * f.h, f.d, 128)) return MOE_ERR_UNSUPPORTED;
-  if (f.n_shared > 0) {
-    // shared experts read the tokens of X itself
-    if (!token_maps(m.ts, f.X, f.n, f.d)) return MOE_ERR_UNSUPPORTED;
-    if (!make_bf16_sw128_map(&m.ws, f.sW1, (long long)f.n_shared * f.h, f.d, 128) ||
-        !make_bf16_sw128_map(&w3s, f.sW3, (long long)f.n_shared * f.h, f.d, 128))
-      return MOE_ERR_UNSUPPORTED;
-  } else {
-    for (int b = 0; b < 3; ++b) m.ts[b] = m.t[b];
-    m.ws = m.w;
-    w3s = w3;
-  }
-  SwapParams q{};
-  q.offsets = f.offsets;
-  q.counts = f.counts;
-  q.E = f.E;
-  q.K = f.d;
-  q.m_per_expert = f.h;
-  q.mt_tiles = f.h / 256;
-  q.n_shared = f.n_shared;
-  q.n = f.n;
-  q.shared_in_row = 0;
-  q.shared_in_stride = 0;
-  q.shared_out_row = f.shared_base;
-  q.n_pad = f.n_pad;
-  q.n_out = f.h;
-  q.out = static_cast<__nv_bfloat16*>(f.H);
-  q.err = f.err;
-  if (launch_swap_up(m, w3, w3s, q, swap_pairs(q, f.rows_routed), s) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  return MOE_OK;
-}
 
 bool swap_down_supported(const FfnArgs& f) {
   return f.counts != nullptr && f.E <= MOE_MAX_EXPERTS && f.d % 256 == 0 && f.h % kSBK == 0;

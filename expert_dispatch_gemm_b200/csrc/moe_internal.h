@@ -218,9 +218,6 @@ moe_status run_ffn_bf16(const FfnArgs& a, cudaStream_t s);
 // the weights-as-M down projection for fine-grained experts (needs the counts)
 bool swap_down_supported(const FfnArgs& a);
 moe_status run_ffn_down_swap(const FfnArgs& a, cudaStream_t s);
-// the weights-as-M SwiGLU up projection (W1 and W3 as two A operands)
-bool swap_up_supported(const FfnArgs& a);
-moe_status run_ffn_up_swap(const FfnArgs& a, cudaStream_t s);
 moe_status run_ffn_f32(const FfnArgs& a, cudaStream_t s);
 
 // ----- backward pass -----

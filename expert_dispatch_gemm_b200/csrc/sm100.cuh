@@ -56,15 +56,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uin
       : "memory");
 }
 
-// Brings a 2-D tile of the map into L2 only (no shared memory, no barrier),
-// so that a later tma_load of the same tile hits L2.
-__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int x, int y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(m)),
-               "r"(x), "r"(y)
-               : "memory");
-}
-
 // ---- untiled bulk copies (addresses 16-byte aligned, sizes multiples of 16) ----
 // global -> this CTA's shared memory, completion counted in bytes on `bar`
 __device__ __forceinline__ void bulk_load_smem(void* dst, const void* src, uint32_t bytes,
