@@ -169,30 +169,38 @@ class ClockSampler:
 # GPU arm
 # ---------------------------------------------------------------------------
 
-def ffma_peak_tflops(dev) -> float:
-    """FP32 FFMA throughput of this device, measured with the probe kernel in
+def ffma_peak_tflops(dev, detail: dict = None) -> float:
+    """FP32 FMA throughput of this device, measured with the probe kernels in
     libmoe_probe.so (the router's roof; not among the measured HBM / tensor
-    peaks). Median of 5 timed launches after 2 warm-ups."""
+    peaks): single FFMAs and packed fp32x2 FMAs, the faster of the two. Median
+    of 5 timed launches after 2 warm-ups each."""
     import ctypes
     lib = ctypes.CDLL(os.path.join(ROOT, "expert_dispatch_gemm_b200", "libmoe_probe.so"))
-    lib.moe_probe_ffma.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     blocks, iters = sms * 8, 2048
     out = torch.empty(blocks, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    times = []
-    for i in range(7):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        rc = lib.moe_probe_ffma(blocks, iters, out.data_ptr(), ctypes.c_void_p(stream.cuda_stream))
-        e1.record(stream)
-        if rc != 0:
-            raise RuntimeError(f"FFMA probe launch failed: {rc}")
-        torch.cuda.synchronize(dev)
-        if i >= 2:
-            times.append(e0.elapsed_time(e1))
     flops = 2.0 * blocks * 256 * iters * 16
-    return flops / (float(np.median(times)) * 1e-3) / 1e12
+    rates = {}
+    for name in ("moe_probe_ffma", "moe_probe_ffma2"):
+        fn = getattr(lib, name)
+        fn.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+        times = []
+        for i in range(7):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            rc = fn(blocks, iters, out.data_ptr(), ctypes.c_void_p(stream.cuda_stream))
+            e1.record(stream)
+            if rc != 0:
+                raise RuntimeError(f"{name} launch failed: {rc}")
+            torch.cuda.synchronize(dev)
+            if i >= 2:
+                times.append(e0.elapsed_time(e1))
+        rates[name] = flops / (float(np.median(times)) * 1e-3) / 1e12
+    if detail is not None:
+        detail.update({"ffma_TFLOP/s": round(rates["moe_probe_ffma"], 1),
+                       "ffma2_TFLOP/s": round(rates["moe_probe_ffma2"], 1)})
+    return max(rates.values())
 
 
 def source_sha(name: str) -> str:
@@ -464,11 +472,13 @@ def run_gpu(args, w: wl.Workload):
     tc_peak_kind = "sustained (sw_power_cap active)" if use_sust else "burst"
     # the router contraction runs on FP32 FFMA: its roof is that pipe, taken
     # here over the whole route stage (router + selection kernels)
-    ffma_peak = ffma_peak_tflops(dev)
+    probes = {}
+    ffma_peak = ffma_peak_tflops(dev, probes)
     router_flops = 2.0 * w.n * w.d * w.E
     route_tflops = router_flops / (med[0] * 1e-3) / 1e12
     stages["route"].update({"router_FLOP": router_flops, "FFMA_TFLOP/s": round(route_tflops, 2),
                             "ffma_peak_TFLOP/s": round(ffma_peak, 1),
+                            "ffma_probes": probes,
                             "ffma_frac": round(route_tflops / ffma_peak, 3)})
     for nm in ("dispatch", "combine"):
         fl = copy_floor_ms(bytes_[nm])

@@ -426,11 +426,14 @@ __global__ void __launch_bounds__(C::NT) router_kernel(RouterArgs a) {
   const int n = a.n, d = a.d, E = a.E;
   const bool w_vec = (E % 4 == 0);
 
-  float acc[TM][TN];
+  // accumulators in column pairs: one packed fp32x2 FMA (__ffma2_rn: a
+  // single-rounding fma per element, so each logit is the same chain of
+  // fmaf as one at a time) updates two of them per issue slot
+  float2 acc[TM][TN / 2];
 #pragma unroll
   for (int i = 0; i < TM; ++i)
 #pragma unroll
-    for (int j = 0; j < TN; ++j) acc[i][j] = 0.0f;
+    for (int j = 0; j < TN / 2; ++j) acc[i][j] = make_float2(0.0f, 0.0f);
 
   // stage loader: X chunk [BM][BK] and W_g chunk [BK][ET] of chunk `c`
   auto issue = [&](int c) {
@@ -560,9 +563,12 @@ __global__ void __launch_bounds__(C::NT) router_kernel(RouterArgs a) {
         bv[4 * g + 3] = t.w;
       }
 #pragma unroll
-      for (int i = 0; i < TM; ++i)
+      for (int i = 0; i < TM; ++i) {
+        const float2 a2 = make_float2(av[i], av[i]);
 #pragma unroll
-        for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        for (int j = 0; j < TN / 2; ++j)
+          acc[i][j] = __ffma2_rn(a2, make_float2(bv[2 * j], bv[2 * j + 1]), acc[i][j]);
+      }
     }
   }
   cp_async_wait<0>();
@@ -575,7 +581,8 @@ __global__ void __launch_bounds__(C::NT) router_kernel(RouterArgs a) {
   for (int i = 0; i < TM; ++i)
 #pragma unroll
     for (int j = 0; j < TN; ++j)
-      Ls[(wk * BM + row0 + i) * LST + colb + (j / 4) * 4 * C::LY + (j % 4)] = acc[i][j];
+      Ls[(wk * BM + row0 + i) * LST + colb + (j / 4) * 4 * C::LY + (j % 4)] =
+          (j % 2) ? acc[i][j / 2].y : acc[i][j / 2].x;
   __syncthreads();
   if (C::WK > 1) {
     for (int q = tid; q < BM * ET; q += C::NT) {
