@@ -15,7 +15,8 @@
 // epilogue overlaps the next tile's main loop.
 //   warp 0     TMA producer (6-stage ring: A 16 KB + B up to 16 KB);
 //   warp 1     TMEM allocation; the leader's lane 0 issues the MMAs;
-//   warps 2-5  epilogue: tcgen05.ld 32 tokens at a time, a transpose through
+//   warps 2-9  epilogue, two per TMEM lane quadrant on alternate 32-token
+//              groups: tcgen05.ld 32 tokens at a time, a transpose through
 //              shared memory, and 16-byte stores of each token's 32
 //              consecutive output columns.
 // Every mbarrier wait is bounded, as in the other GEMM kernels.
@@ -34,7 +35,8 @@ namespace moe {
 
 namespace {
 
-constexpr int kSBK = 64, kSStages = 6, kSThreads = 192;
+// warps: 0 producer, 1 MMA, 2-9 epilogue (two per TMEM lane quadrant)
+constexpr int kSBK = 64, kSStages = 6, kSEpiWarps = 8, kSThreads = 32 * (2 + kSEpiWarps);
 constexpr int kSABytes = 128 * kSBK * 2;         // this CTA's 128 weight rows
 constexpr int kSBBytes = 128 * kSBK * 2;         // up to 128 token rows
 constexpr int kSStageBytes = kSABytes + kSBBytes;
@@ -169,7 +171,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSThreads, 1)
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(ssm) + 1023) & ~uintptr_t(1023));
   SwapState* st = reinterpret_cast<SwapState*>(base + kSStages * kSStageBytes);
-  // epilogue staging, [4 warps][32 tokens][32 columns] bf16
+  // epilogue staging, [8 warps][32 tokens][32 columns] bf16
   __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(
       base + kSStages * kSStageBytes + ((sizeof(SwapState) + 127) & ~size_t(127)));
   auto sA = [&](int s) { return base + s * kSStageBytes; };
@@ -185,7 +187,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       sm100::mbar_init(&st->tfull[a], 1);
-      sm100::mbar_init(&st->tempty[a], 256);
+      sm100::mbar_init(&st->tempty[a], 2 * 32 * kSEpiWarps);  // both CTAs' epilogues
     }
     sm100::mbar_init(&st->drain, 1);
     st->abort_flag = 0;
@@ -322,11 +324,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSThreads, 1)
     }
   } else {
     // epilogue: TMEM lanes = this CTA's 128 weight rows (output columns),
-    // TMEM columns = tokens; warp q owns lanes 32q..32q+31
+    // TMEM columns = tokens; warps q and q + 4 own lanes 32q..32q+31 (q =
+    // warp % 4) and take alternate 32-token column groups
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     constexpr int CW = 32;  // output columns per warp
     constexpr int VPR = CW * 2 / 16;  // 16-byte pieces of a token's CW columns
-    __nv_bfloat16* stg = stage + q * (32 * CW);  // [32 tokens][CW] bf16
+    __nv_bfloat16* stg = stage + (warp - 2) * (32 * CW);  // [32 tokens][CW] bf16
     int local = 0;
     for (int tile = pair_id; tile < total; tile += num_pairs, ++local) {
       const SwapTile t = decode_swap(tile, p, st, routed);
@@ -340,7 +344,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSThreads, 1)
         sm100::tc_fence_after();
         const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256);
 #pragma unroll 1
-        for (int cc = 0; cc < t.n; cc += 32) {
+        for (int cc = 32 * half; cc < t.n; cc += 64) {
           uint32_t v[32];
           sm100::tmem_ld_32x32b_x32(tbase + cc, v);
           sm100::tmem_ld_wait();
@@ -381,7 +385,7 @@ struct SwapMaps {
 
 static cudaError_t launch_swap(const SwapMaps& m, const SwapParams& p, int pairs, cudaStream_t s) {
   const size_t bytes = (size_t)kSStages * kSStageBytes + ((sizeof(SwapState) + 127) & ~size_t(127)) +
-                       4 * 32 * 32 * sizeof(__nv_bfloat16) + 1024;
+                       kSEpiWarps * 32 * 32 * sizeof(__nv_bfloat16) + 1024;
   auto kern = tc_swap_pair_kernel;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
