@@ -294,11 +294,29 @@ __global__ void __launch_bounds__(256) ec_finish_kernel(EcFinishArgs a) {
   const int t0 = blockIdx.x * 32;
   for (int i = threadIdx.x; i <= E; i += blockDim.x) hist_s[i] = 0;
   if (threadIdx.x == 0) none_s = 0;
-  for (int e = warp; e < E; e += 8) {
+  // a warp's experts e = warp, warp + 8, ...: all their loads are issued
+  // before any is used (the gate is read whether or not the expert picked
+  // the token, and kept only when it did), so one round trip covers them
+  {
+    constexpr int U = MOE_MAX_EXPERTS / 8;
     const bool in = t0 + lane < n;
-    const int r = in ? a.ec_row[(size_t)e * n + t0 + lane] : -1;
-    rows_s[e * 33 + lane] = r;
-    gates_s[e * 33 + lane] = r >= 0 ? a.ec_gate[(size_t)e * n + t0 + lane] : 0.0f;
+    int r[U];
+    float g[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int e = warp + 8 * u;
+      const bool ok = in && e < E;
+      r[u] = ok ? a.ec_row[(size_t)e * n + t0 + lane] : -1;
+      g[u] = ok ? a.ec_gate[(size_t)e * n + t0 + lane] : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int e = warp + 8 * u;
+      if (e < E) {
+        rows_s[e * 33 + lane] = r[u];
+        gates_s[e * 33 + lane] = r[u] >= 0 ? g[u] : 0.0f;
+      }
+    }
   }
   __syncthreads();
   for (int tt = warp; tt < 32; tt += 8) {
