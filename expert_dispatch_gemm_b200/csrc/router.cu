@@ -58,6 +58,9 @@ using R256s = RCfg<256, 2, 8, 4, 2, 4, 1, 32, 3>;
 // CTA), "C" over 2 (many rows per CTA).
 template <int TM> using R64A = RCfg<64, TM, 8, 4, 1, 1, 8, 64, 4>;   // BM = 4 TM
 template <int TM> using R64C = RCfg<64, TM, 8, 4, 4, 1, 2, 32, 4>;   // BM = 16 TM
+// R64A's tiles on 12 warps (a twelve-way k split of 48-deep chunks): in a
+// single wave of one CTA per SM, 50% more warps to hide the chunks' loads
+template <int TM> using R64D = RCfg<64, TM, 8, 4, 1, 1, 12, 48, 4>;  // BM = 4 TM
 template <int TM> using R128A = RCfg<128, TM, 8, 4, 2, 2, 2, 32, 4>; // BM = 8 TM
 template <int TM> using R256A = RCfg<256, TM, 8, 4, 1, 4, 2, 32, 3>; // BM = 4 TM
 // E = 256 with 16 columns per thread: per 16-deep step a warp issues TM*16
@@ -92,8 +95,8 @@ static int num_sms_cached() {
 // small-row one when the big tile would leave SMs without a CTA. bf16 X with
 // E > 32: the (family, TM) whose rows per SM, BM * ceil(CTAs / SMs), is
 // smallest (ties to the larger BM). Codes: kFamilyCode + fam * 16 + TM with
-// fam 1 = R64A, 2 = R64C, 3 = R128A, 4 = R256A, 5 = R256B, 6 = R256C; otherwise
-// the fixed tile's ET (257: R256s, 65: R64s).
+// fam 1 = R64A, 2 = R64C, 3 = R128A, 4 = R256A, 5 = R256B, 6 = R256C,
+// 7 = R64D; otherwise the fixed tile's ET (257: R256s, 65: R64s).
 constexpr int kFamilyCode = 1000;
 struct RouterFamily {
   int code, unit, tm_lo;
@@ -102,11 +105,11 @@ static int router_variant(int E, int n, bool x_bf16) {
   const int et = router_tile_et(E);
   const int sms = num_sms_cached();
   if (x_bf16 && et >= 64) {
-    static const RouterFamily fams64[] = {{1, 4, 4}, {2, 16, 4}};
+    static const RouterFamily fams64[] = {{7, 4, 4}, {1, 4, 4}, {2, 16, 4}};
     static const RouterFamily fams128[] = {{3, 8, 2}};
     static const RouterFamily fams256[] = {{6, 8, 4}, {5, 8, 4}, {4, 4, 4}};
     const RouterFamily* fams = et == 64 ? fams64 : et == 128 ? fams128 : fams256;
-    const int nf = et == 128 ? 1 : et == 64 ? 2 : 3;
+    const int nf = et == 128 ? 1 : 3;
     long long best_cost = -1;
     int best = 0, best_bm = 0;
     for (int f = 0; f < nf; ++f)
@@ -120,7 +123,7 @@ static int router_variant(int E, int n, bool x_bf16) {
         // vs 174). R64C splits each chunk over only two warp groups, so with
         // one CTA per SM its eight warps hide too little latency (112 rows
         // per SM took 203 us, 128 rows in two CTAs 174 us).
-        if (fams[f].code == 1 && ctas > sms) continue;
+        if ((fams[f].code == 1 || fams[f].code == 7) && ctas > sms) continue;
         if (fams[f].code == 2 && ctas * 2 < 3LL * sms) cost = cost * 4 / 3;
         // TM x 8 tiles at E = 256 are bound by shared-memory wavefronts
         // (TM + 8 per TM*8 FFMAs per step), the 16-column tiles by the FMA
@@ -155,7 +158,7 @@ static void variant_tile(int v, int* bm, int* bk) {
     default: {
       const int code = v - kFamilyCode, fam = code / 16, tm = code % 16;
       *bm = (fam == 2 ? 16 : fam == 3 || fam == 5 || fam == 6 ? 8 : 4) * tm;
-      *bk = fam == 1 ? 64 : fam == 6 ? 48 : 32;
+      *bk = fam == 1 ? 64 : fam == 6 || fam == 7 ? 48 : 32;
     }
   }
 }
@@ -722,7 +725,8 @@ static cudaError_t launch_router_bf16_family(int code, const RouterArgs& a, cuda
     case 3: return launch_family<R128A>(tm, a, s);
     case 4: return launch_family<R256A>(tm, a, s);
     case 5: return launch_family<R256B>(tm, a, s);
-    default: return launch_family_upto7<R256C>(tm, a, s);
+    case 6: return launch_family_upto7<R256C>(tm, a, s);
+    default: return launch_family<R64D>(tm, a, s);
   }
 }
 
