@@ -290,10 +290,12 @@ bool ffn_uses_pair(const moe_config* c, const Derived& dv) {
 }
 
 // Fine-grained token choice (128 to 512 rows per expert on average): the
-// weights-as-M down projection computes each expert's exact token count
-// (16-row granularity) where the 128-row tiles would round ~256 rows up to
-// 384 or 512. It needs the counts, which the caller passes. The up
-// projection stays on the token-side kernels, which measured faster there.
+// weights-as-M projections compute each expert's exact token count (16-row
+// granularity) where the 128-row tiles would round ~256 rows up to 384 or
+// 512. They need the counts, which the caller passes. The SwiGLU up
+// projection takes W1 and W3 as two A operands into two accumulators; other
+// activations, the fused gather and the training forward's kept U and V
+// keep the up projection on the token-side kernels.
 static bool ffn_uses_swap(const moe_config* c, const Derived& dv) {
   if (c->dtype != MOE_BF16 || c->mode != MOE_TOKEN_CHOICE) return false;
   const long long avg = avg_expert_rows(c, dv);
@@ -349,8 +351,13 @@ static moe_status ffn_impl(const moe_config* c, const Derived& dv, const void* X
   f.save_v = save_v;
   if (c->dtype != MOE_BF16) return out32 ? MOE_ERR_UNSUPPORTED : run_ffn_f32(f, s);
   if (!out32 && ffn_uses_swap(c, dv) && swap_down_supported(f)) {
-    f.skip_down = true;
-    const moe_status st = run_ffn_bf16(f, s);
+    moe_status st;
+    if (swap_up_supported(f)) {
+      st = run_ffn_up_swap(f, s);
+    } else {
+      f.skip_down = true;
+      st = run_ffn_bf16(f, s);
+    }
     if (st != MOE_OK) return st;
     return run_ffn_down_swap(f, s);
   }

@@ -10,15 +10,26 @@
 //
 // CTA pairs (cta_group::2). A tile is (expert, 256 rows of W2, up to 256 of
 // the expert's tokens): each CTA loads its 128 weight rows as A and half of
-// the tile's tokens as B, and the leader issues M=256 MMAs with N = tokens (a
-// multiple of 16) into one of two 256-column TMEM accumulators, so one tile's
-// epilogue overlaps the next tile's main loop.
-//   warp 0     TMA producer (6-stage ring: A 16 KB + B up to 16 KB);
-//   warp 1     TMEM allocation; the leader's lane 0 issues the MMAs;
-//   warps 2-9  epilogue, two per TMEM lane quadrant on alternate 32-token
-//              groups: tcgen05.ld 32 tokens at a time, a transpose through
-//              shared memory, and 16-byte stores of each token's 32
-//              consecutive output columns.
+// the tile's tokens as B, and the MMA is M=256 with N = tokens (a multiple
+// of 16).
+//
+// On B200 one thread issues at most one tcgen05.mma about every 95 cycles,
+// whatever N is, while an M=256 pair MMA needs N/2 cycles of the tensor
+// pipe: below N = 192 a single issuer leaves the pipe idle, and the token
+// chunks of experts with more than 256 rows are 128-160 wide. Two issuers
+// on independent accumulators keep it busy down to N = 128. So the pair runs
+// two tile streams, each with its own producer, shared-memory ring and
+// 256-column TMEM accumulator; stream s takes every other tile of the pair.
+//   warps 0 / 2   TMA producers of streams 0 / 1 (3-stage rings of 32 KB:
+//                 A 16 KB + B up to 16 KB);
+//   warps 1 / 3   the leader's lane 0 issues the MMAs of stream 0 / 1
+//                 (warp 1 also holds the TMEM allocation);
+//   warps 4-11    epilogue, four per stream (one per TMEM lane quadrant):
+//                 tcgen05.ld 32 tokens at a time, a transpose through shared
+//                 memory, and 16-byte stores of each token's 32 consecutive
+//                 output columns.
+// While one stream's epilogue drains its accumulator the other stream keeps
+// the tensor pipe busy.
 // Every mbarrier wait is bounded, as in the other GEMM kernels.
 //
 // Only the down projection runs here. The same scheme for the SwiGLU up
@@ -35,12 +46,13 @@ namespace moe {
 
 namespace {
 
-// warps: 0 producer, 1 MMA, 2-9 epilogue (two per TMEM lane quadrant)
-constexpr int kSBK = 64, kSStages = 6, kSEpiWarps = 8, kSThreads = 32 * (2 + kSEpiWarps);
+// warps: 0/2 producers, 1/3 MMA issuers, 4-11 epilogue (streams 0 and 1)
+constexpr int kSBK = 64, kSStages = 3, kSStreams = 2, kSEpiWarps = 8;
+constexpr int kSThreads = 32 * (4 + kSEpiWarps);
 constexpr int kSABytes = 128 * kSBK * 2;         // this CTA's 128 weight rows
 constexpr int kSBBytes = 128 * kSBK * 2;         // up to 128 token rows
 constexpr int kSStageBytes = kSABytes + kSBBytes;
-constexpr int kSTmemCols = 512;                  // two 256-column accumulators
+constexpr int kSTmemCols = 512;                  // one 256-column accumulator per stream
 constexpr int kSMaxTokens = 256;                 // tokens per tile (MMA N <= 256)
 constexpr uint64_t kSWaitNs = 2000000000ull;     // 2 s
 
@@ -61,11 +73,11 @@ struct SwapParams {
 };
 
 struct SwapState {
-  uint64_t full[kSStages];
-  uint64_t empty[kSStages];
-  uint64_t tfull[2];
-  uint64_t tempty[2];
-  uint64_t drain;
+  uint64_t full[kSStreams][kSStages];
+  uint64_t empty[kSStreams][kSStages];
+  uint64_t tfull[kSStreams];
+  uint64_t tempty[kSStreams];
+  uint64_t drain[kSStreams];
   uint32_t tmem_base;
   volatile int abort_flag;
   int offs[MOE_MAX_EXPERTS + 1];
@@ -73,8 +85,8 @@ struct SwapState {
   int tprefix[MOE_MAX_EXPERTS + 1];  // tiles of the experts before e
 };
 
-template <bool CLUSTER_ACQUIRE>
-__device__ __forceinline__ bool swap_wait(uint64_t* bar, uint32_t parity, SwapState* st, int* err,
+template <bool CLUSTER_ACQUIRE, class State>
+__device__ __forceinline__ bool swap_wait(uint64_t* bar, uint32_t parity, State* st, int* err,
                                           int code) {
   auto probe = [&]() {
     return CLUSTER_ACQUIRE ? sm100::mbar_try_wait_cluster(bar, parity)
@@ -109,7 +121,8 @@ struct SwapTile {
 // innermost; shared experts last. An expert's tokens split into
 // ceil(count / 256) chunks of equal size (rounded up to 16), so that 272
 // tokens become 144 + 128 rather than 256 + 16.
-__device__ __forceinline__ SwapTile decode_swap(int tile, const SwapParams& p, const SwapState* st,
+template <class State>
+__device__ __forceinline__ SwapTile decode_swap(int tile, const SwapParams& p, const State* st,
                                                int routed) {
   SwapTile t;
   int chunk, chunks, count;
@@ -170,26 +183,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSThreads, 1)
   extern __shared__ __align__(1024) unsigned char ssm[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(ssm) + 1023) & ~uintptr_t(1023));
-  SwapState* st = reinterpret_cast<SwapState*>(base + kSStages * kSStageBytes);
+  constexpr int kRingBytes = kSStreams * kSStages * kSStageBytes;
+  SwapState* st = reinterpret_cast<SwapState*>(base + kRingBytes);
   // epilogue staging, [8 warps][32 tokens][32 columns] bf16
   __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(
-      base + kSStages * kSStageBytes + ((sizeof(SwapState) + 127) & ~size_t(127)));
-  auto sA = [&](int s) { return base + s * kSStageBytes; };
-  auto sB = [&](int s) { return base + s * kSStageBytes + kSABytes; };
+      base + kRingBytes + ((sizeof(SwapState) + 127) & ~size_t(127)));
+  auto sA = [&](int sx, int j) { return base + (sx * kSStages + j) * kSStageBytes; };
+  auto sB = [&](int sx, int j) { return sA(sx, j) + kSABytes; };
 
   const uint32_t rank = sm100::cluster_ctarank();
   const bool leader = rank == 0;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
-    for (int s = 0; s < kSStages; ++s) {
-      sm100::mbar_init(&st->full[s], 1);
-      sm100::mbar_init(&st->empty[s], 1);
+    for (int sx = 0; sx < kSStreams; ++sx) {
+      for (int j = 0; j < kSStages; ++j) {
+        sm100::mbar_init(&st->full[sx][j], 1);
+        sm100::mbar_init(&st->empty[sx][j], 1);
+      }
+      sm100::mbar_init(&st->tfull[sx], 1);
+      // every thread of the stream's epilogue warps, in both CTAs
+      sm100::mbar_init(&st->tempty[sx], 2 * 32 * (kSEpiWarps / kSStreams));
+      sm100::mbar_init(&st->drain[sx], 1);
     }
-    for (int a = 0; a < 2; ++a) {
-      sm100::mbar_init(&st->tfull[a], 1);
-      sm100::mbar_init(&st->tempty[a], 2 * 32 * kSEpiWarps);  // both CTAs' epilogues
-    }
-    sm100::mbar_init(&st->drain, 1);
     st->abort_flag = 0;
     sm100::fence_mbar_init();
   }
@@ -202,6 +217,264 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSThreads, 1)
   pdl_wait();
   for (int i = tid; i <= p.E; i += kSThreads) st->offs[i] = p.offsets[i];
   for (int i = tid; i < p.E; i += kSThreads) {
+    const int seg = p.offsets[i + 1] - p.offsets[i];
+    const int c = p.counts ? p.counts[i] : seg;
+    if (seg < 0 || c < 0 || c > seg) bad_index(p.err, kSiteSwapOffsets);
+    st->cnt[i] = max(0, min(c, seg));  // never past the expert's own segment
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int e = 0; e < p.E; ++e) {
+      st->tprefix[e] = run;
+      run += (st->cnt[e] + kSMaxTokens - 1) / kSMaxTokens * p.mt_tiles;
+    }
+    st->tprefix[p.E] = run;
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::cluster_sync();  // both CTAs' barriers exist before any remote arrive
+  sm100::tc_fence_after();
+  const uint32_t tmem = st->tmem_base;
+
+  const int routed = st->tprefix[p.E];
+  const int shared_chunks = (p.n + kSMaxTokens - 1) / kSMaxTokens;
+  const int total = routed + p.n_shared * p.mt_tiles * shared_chunks;
+  const int KB = p.K / kSBK;
+  const int pair_id = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+  // the pair's tiles are pair_id + i * num_pairs; stream sx takes i = sx, sx + 2, ...
+  const int sx = warp < 4 ? (warp >> 1) : (warp - 4) / (kSEpiWarps / kSStreams);
+  const int first = pair_id + sx * num_pairs, step = kSStreams * num_pairs;
+
+  if (warp < 4 && (warp & 1) == 0) {
+    // producer of stream sx
+    if (lane == 0) {
+      int stage = 0, issued = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = first; ok && tile < total; tile += step) {
+        const SwapTile t = decode_swap(tile, p, st, routed);
+        const CUtensorMap* tm[3];
+        if (t.shared) {
+          tm[0] = &tmTs0; tm[1] = &tmTs1; tm[2] = &tmTs2;
+        } else {
+          tm[0] = &tmT0; tm[1] = &tmT1; tm[2] = &tmT2;
+        }
+        const int b1 = box_rows(t.n);
+        const CUtensorMap* m1 = tm[b1 == 32 ? 0 : b1 == 64 ? 1 : 2];
+        const uint32_t bytes = kSABytes + (uint32_t)b1 * kSBK * 2;
+        const CUtensorMap* mw = t.shared ? &tmWs : &tmW;
+        const int wrow = t.expert * p.m_per_expert + t.m0 + (int)rank * 128;  // this CTA's 128
+        // this CTA's half of the tile's tokens
+        const long long trow1 = t.tok_row + (long long)rank * (t.n / 2);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!swap_wait<false>(&st->empty[sx][stage], phase ^ 1u, st, p.err,
+                                kErrGemmTimeout | 0xA1)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fl = sm100::mapa_shared(sm100::smem_addr(&st->full[sx][stage]), 0);
+          if (leader) sm100::mbar_arrive_expect_tx(&st->full[sx][stage], 2 * bytes);
+          sm100::tma_load_2d_pair(sA(sx, stage), mw, fl, kb * kSBK, wrow);
+          sm100::tma_load_2d_pair(sB(sx, stage), m1, fl, kb * kSBK, (int)trow1);
+          ++issued;
+          if (++stage == kSStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok && leader) {
+        // wait (bounded) until the copies of the outstanding stages have landed
+        int j = stage;
+        uint32_t ph = phase;
+        const int pending = issued < kSStages ? issued : kSStages;
+        for (int i = 0; i < pending; ++i) {
+          if (--j < 0) {
+            j = kSStages - 1;
+            ph ^= 1u;
+          }
+          const uint64_t t0 = global_timer_ns();
+          while (!sm100::mbar_try_wait(&st->full[sx][j], ph) && global_timer_ns() - t0 < kSWaitNs) {
+          }
+        }
+      }
+    }
+  } else if (warp < 4) {
+    // MMA issuer of stream sx: the leader's lane 0
+    if (lane == 0 && leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      const uint32_t d_tmem = tmem + (uint32_t)(sx * 256);
+      for (int tile = first; ok && tile < total; tile += step, ++local) {
+        const SwapTile t = decode_swap(tile, p, st, routed);
+        // the accumulator is free once both CTAs' epilogues drained the last tile
+        if (!swap_wait<true>(&st->tempty[sx], ((uint32_t)local & 1u) ^ 1u, st, p.err,
+                             kErrGemmTimeout | 0xB2)) {
+          ok = false;
+          break;
+        }
+        sm100::tc_fence_after();
+        const uint32_t idesc = sm100::idesc_bf16_f32(256, t.n);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!swap_wait<false>(&st->full[sx][stage], phase, st, p.err, kErrGemmTimeout | 0xB3)) {
+            ok = false;
+            break;
+          }
+          sm100::tc_fence_after();
+          const uint64_t adesc = sm100::sw128_kmajor_desc(sm100::smem_addr(sA(sx, stage)));
+          const uint64_t bdesc = sm100::sw128_kmajor_desc(sm100::smem_addr(sB(sx, stage)));
+#pragma unroll
+          for (int k = 0; k < kSBK / 16; ++k)
+            sm100::umma_f16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0);
+          sm100::umma_commit_pair_mc(&st->empty[sx][stage], 0x3);
+          if (++stage == kSStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        sm100::umma_commit_pair_mc(&st->tfull[sx], 0x3);
+      }
+      sm100::umma_commit_pair_mc(&st->drain[sx], 0x1);
+      const uint64_t t0 = global_timer_ns();
+      while (!sm100::mbar_try_wait(&st->drain[sx], 0) && global_timer_ns() - t0 < kSWaitNs) {
+      }
+    }
+  } else {
+    // epilogue of stream sx: TMEM lanes = this CTA's 128 weight rows (output
+    // columns), TMEM columns = tokens; warp q = warp % 4 owns lanes
+    // 32q..32q+31 and walks all the tile's tokens, 32 at a time
+    const int q = warp & 3;
+    constexpr int CW = 32;  // output columns per warp
+    constexpr int VPR = CW * 2 / 16;  // 16-byte pieces of a token's CW columns
+    __nv_bfloat16* stg = stage + (warp - 4) * (32 * CW);  // [32 tokens][CW] bf16
+    int local = 0;
+    for (int tile = first; tile < total; tile += step, ++local) {
+      const SwapTile t = decode_swap(tile, p, st, routed);
+      const int col0 = t.m0 + (int)rank * 128 + 32 * q;
+      __nv_bfloat16* outt = p.out + (size_t)t.out_row * p.n_out + col0;
+      if (!swap_wait<true>(&st->tfull[sx], (uint32_t)local & 1u, st, p.err, kErrGemmTimeout | 0xC4))
+        break;
+      sm100::tc_fence_after();
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(sx * 256);
+#pragma unroll 1
+      for (int cc = 0; cc < t.n; cc += 32) {
+        uint32_t v[32];
+        sm100::tmem_ld_32x32b_x32(tbase + cc, v);
+        sm100::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) stg[i * CW + lane] = __float2bfloat16_rn(__uint_as_float(v[i]));
+        __syncwarp();
+        // each token's CW columns leave as 16-byte stores
+#pragma unroll
+        for (int idx = lane; idx < 32 * VPR; idx += 32) {
+          const int i = idx / VPR, vv = idx % VPR;
+          const int j = cc + i;  // token within the tile
+          if (j < t.valid)
+            *reinterpret_cast<uint4*>(outt + (size_t)j * p.n_out + vv * 8) =
+                *reinterpret_cast<const uint4*>(stg + i * CW + vv * 8);
+        }
+        __syncwarp();
+      }
+      sm100::tc_fence_before();
+      sm100::mbar_arrive_cluster(sm100::mapa_shared(sm100::smem_addr(&st->tempty[sx]), 0));
+    }
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::cluster_sync();  // no CTA leaves while its peer may still signal it
+  if (warp == 1) {
+    sm100::tc_fence_after();
+    sm100::tmem_dealloc_pair(tmem, kSTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// SwiGLU up projection with the weights as the M side: H_e^T = silu(W1_e
+// X_e^T) * (W3_e X_e^T). A tile is (expert, 256 hidden units, up to 256 of
+// the expert's tokens). Each CTA loads its 128 rows of W1 and the same 128
+// rows of W3 as two A operands and half of the tile's tokens as B. Two
+// threads of the leader issue the MMAs: one the W1 products into TMEM
+// columns [0, 256) (the gate pre-activation U), the other the W3 products
+// into [256, 512) (V), both from the same stage, so a hidden unit's U and V
+// sit in one TMEM lane and meet in one epilogue thread, and the tensor pipe
+// sees two issuers (a single one cannot feed it below N = 192). The 512
+// columns hold one tile; the producer runs ahead into the next tile's stages
+// while the epilogue drains.
+//   warp 0     TMA producer (4-stage ring: W1 16 KB + W3 16 KB + tokens <= 16 KB);
+//   warp 1     TMEM allocation; the leader's lane 0 issues the W1 MMAs;
+//   warp 2     the leader's lane 0 issues the W3 MMAs;
+//   warp 3     idle;
+//   warps 4-11 epilogue, two per TMEM lane quadrant on alternate 32-token
+//              groups: U and V 32 tokens at a time, silu(U) V in fp32, bf16,
+//              a transpose through shared memory, and 16-byte stores of each
+//              token's 32 consecutive hidden units.
+// ---------------------------------------------------------------------------
+constexpr int kUStages = 4, kUEpiWarps = 8, kUThreads = 32 * (4 + kUEpiWarps);
+constexpr int kUWBytes = 128 * kSBK * 2;                       // 128 rows of W1 or W3
+constexpr int kUStageBytes = 2 * kUWBytes + kSBBytes;          // 48 KB
+
+struct UpState {
+  uint64_t full[kUStages];
+  uint64_t empty[kUStages];   // released by both issuers' commits
+  uint64_t tfull;             // both issuers' last commits of a tile
+  uint64_t tempty;            // both CTAs' epilogues
+  uint64_t drain[2];
+  uint32_t tmem_base;
+  volatile int abort_flag;
+  int offs[MOE_MAX_EXPERTS + 1];
+  int cnt[MOE_MAX_EXPERTS];
+  int tprefix[MOE_MAX_EXPERTS + 1];
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kUThreads, 1)
+    tc_swap_up_pair_kernel(const __grid_constant__ CUtensorMap tmT0,
+                           const __grid_constant__ CUtensorMap tmT1,
+                           const __grid_constant__ CUtensorMap tmT2,
+                           const __grid_constant__ CUtensorMap tmTs0,
+                           const __grid_constant__ CUtensorMap tmTs1,
+                           const __grid_constant__ CUtensorMap tmTs2,
+                           const __grid_constant__ CUtensorMap tmW1,
+                           const __grid_constant__ CUtensorMap tmW3,
+                           const __grid_constant__ CUtensorMap tmW1s,
+                           const __grid_constant__ CUtensorMap tmW3s, const SwapParams p) {
+  extern __shared__ __align__(1024) unsigned char usm[];
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(usm) + 1023) & ~uintptr_t(1023));
+  UpState* st = reinterpret_cast<UpState*>(base + kUStages * kUStageBytes);
+  // epilogue staging, [8 warps][32 tokens][32 hidden units] bf16
+  __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(
+      base + kUStages * kUStageBytes + ((sizeof(UpState) + 127) & ~size_t(127)));
+  auto sW = [&](int j, int which) { return base + j * kUStageBytes + which * kUWBytes; };
+  auto sB = [&](int j) { return base + j * kUStageBytes + 2 * kUWBytes; };
+
+  const uint32_t rank = sm100::cluster_ctarank();
+  const bool leader = rank == 0;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int j = 0; j < kUStages; ++j) {
+      sm100::mbar_init(&st->full[j], 1);
+      sm100::mbar_init(&st->empty[j], 2);
+    }
+    sm100::mbar_init(&st->tfull, 2);
+    sm100::mbar_init(&st->tempty, 2 * 32 * kUEpiWarps);  // both CTAs' epilogues
+    sm100::mbar_init(&st->drain[0], 1);
+    sm100::mbar_init(&st->drain[1], 1);
+    st->abort_flag = 0;
+    sm100::fence_mbar_init();
+  }
+  if (warp == 1) {
+    sm100::tmem_alloc_pair(&st->tmem_base, kSTmemCols);
+    sm100::tmem_relinquish_pair();
+  }
+  // the set-up above needs nothing from the previous kernel; the segment
+  // starts, the counts and the dispatched rows are read from here on
+  pdl_wait();
+  for (int i = tid; i <= p.E; i += kUThreads) st->offs[i] = p.offsets[i];
+  for (int i = tid; i < p.E; i += kUThreads) {
     const int seg = p.offsets[i + 1] - p.offsets[i];
     const int c = p.counts ? p.counts[i] : seg;
     if (seg < 0 || c < 0 || c > seg) bad_index(p.err, kSiteSwapOffsets);
@@ -243,22 +516,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSThreads, 1)
         }
         const int b1 = box_rows(t.n);
         const CUtensorMap* m1 = tm[b1 == 32 ? 0 : b1 == 64 ? 1 : 2];
-        const uint32_t bytes = kSABytes + (uint32_t)b1 * kSBK * 2;
-        const CUtensorMap* mw = t.shared ? &tmWs : &tmW;
+        const uint32_t bytes = 2 * kUWBytes + (uint32_t)b1 * kSBK * 2;
+        const CUtensorMap* mw1 = t.shared ? &tmW1s : &tmW1;
+        const CUtensorMap* mw3 = t.shared ? &tmW3s : &tmW3;
         const int wrow = t.expert * p.m_per_expert + t.m0 + (int)rank * 128;  // this CTA's 128
         // this CTA's half of the tile's tokens
         const long long trow1 = t.tok_row + (long long)rank * (t.n / 2);
         for (int kb = 0; kb < KB; ++kb) {
-          if (!swap_wait<false>(&st->empty[stage], phase ^ 1u, st, p.err, kErrGemmTimeout | 0xA1)) {
+          if (!swap_wait<false>(&st->empty[stage], phase ^ 1u, st, p.err, kErrGemmTimeout | 0xD1)) {
             ok = false;
             break;
           }
           const uint32_t fl = sm100::mapa_shared(sm100::smem_addr(&st->full[stage]), 0);
           if (leader) sm100::mbar_arrive_expect_tx(&st->full[stage], 2 * bytes);
-          sm100::tma_load_2d_pair(sA(stage), mw, fl, kb * kSBK, wrow);
+          sm100::tma_load_2d_pair(sW(stage, 0), mw1, fl, kb * kSBK, wrow);
+          sm100::tma_load_2d_pair(sW(stage, 1), mw3, fl, kb * kSBK, wrow);
           sm100::tma_load_2d_pair(sB(stage), m1, fl, kb * kSBK, (int)trow1);
           ++issued;
-          if (++stage == kSStages) {
+          if (++stage == kUStages) {
             stage = 0;
             phase ^= 1u;
           }
@@ -266,105 +541,107 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSThreads, 1)
       }
       if (!ok && leader) {
         // wait (bounded) until the copies of the outstanding stages have landed
-        int s = stage;
+        int j = stage;
         uint32_t ph = phase;
-        const int pending = issued < kSStages ? issued : kSStages;
+        const int pending = issued < kUStages ? issued : kUStages;
         for (int i = 0; i < pending; ++i) {
-          if (--s < 0) {
-            s = kSStages - 1;
+          if (--j < 0) {
+            j = kUStages - 1;
             ph ^= 1u;
           }
           const uint64_t t0 = global_timer_ns();
-          while (!sm100::mbar_try_wait(&st->full[s], ph) && global_timer_ns() - t0 < kSWaitNs) {
+          while (!sm100::mbar_try_wait(&st->full[j], ph) && global_timer_ns() - t0 < kSWaitNs) {
           }
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 2) {
+    // issuer `which`: W1 products into columns [0, 256), W3 into [256, 512)
     if (lane == 0 && leader) {
+      const int which = warp - 1;
+      const uint32_t d_tmem = tmem + (uint32_t)(which * 256);
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
       for (int tile = pair_id; ok && tile < total; tile += num_pairs, ++local) {
         const SwapTile t = decode_swap(tile, p, st, routed);
-        const int acc = local & 1;
-        const uint32_t acc_phase = (uint32_t)(local >> 1) & 1u;
-        if (!swap_wait<true>(&st->tempty[acc], acc_phase ^ 1u, st, p.err, kErrGemmTimeout | 0xB2)) {
+        if (!swap_wait<true>(&st->tempty, ((uint32_t)local & 1u) ^ 1u, st, p.err,
+                             kErrGemmTimeout | 0xE2)) {
           ok = false;
           break;
         }
         sm100::tc_fence_after();
         const uint32_t idesc = sm100::idesc_bf16_f32(256, t.n);
-        const uint32_t d_tmem = tmem + (uint32_t)(acc * 256);
         for (int kb = 0; kb < KB; ++kb) {
-          if (!swap_wait<false>(&st->full[stage], phase, st, p.err, kErrGemmTimeout | 0xB3)) {
+          if (!swap_wait<false>(&st->full[stage], phase, st, p.err, kErrGemmTimeout | 0xE3)) {
             ok = false;
             break;
           }
           sm100::tc_fence_after();
-          const uint64_t adesc = sm100::sw128_kmajor_desc(sm100::smem_addr(sA(stage)));
-          const uint64_t bdesc = sm100::sw128_kmajor_desc(sm100::smem_addr(sB(stage)));
+          const uint64_t da = sm100::sw128_kmajor_desc(sm100::smem_addr(sW(stage, which)));
+          const uint64_t db = sm100::sw128_kmajor_desc(sm100::smem_addr(sB(stage)));
 #pragma unroll
           for (int k = 0; k < kSBK / 16; ++k)
-            sm100::umma_f16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0);
+            sm100::umma_f16_pair(d_tmem, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
           sm100::umma_commit_pair_mc(&st->empty[stage], 0x3);
-          if (++stage == kSStages) {
+          if (++stage == kUStages) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        sm100::umma_commit_pair_mc(&st->tfull[acc], 0x3);
+        sm100::umma_commit_pair_mc(&st->tfull, 0x3);
       }
-      sm100::umma_commit_pair_mc(&st->drain, 0x1);
+      sm100::umma_commit_pair_mc(&st->drain[which], 0x1);
       const uint64_t t0 = global_timer_ns();
-      while (!sm100::mbar_try_wait(&st->drain, 0) && global_timer_ns() - t0 < kSWaitNs) {
+      while (!sm100::mbar_try_wait(&st->drain[which], 0) && global_timer_ns() - t0 < kSWaitNs) {
       }
     }
-  } else {
-    // epilogue: TMEM lanes = this CTA's 128 weight rows (output columns),
-    // TMEM columns = tokens; warps q and q + 4 own lanes 32q..32q+31 (q =
-    // warp % 4) and take alternate 32-token column groups
+  } else if (warp >= 4) {
+    // epilogue: TMEM lanes = this CTA's 128 hidden units, columns = tokens
+    // (U in [0, 256), V in [256, 512)); warps q and q + 4 own lanes
+    // 32q..32q+31 (q = warp % 4) and take alternate 32-token groups
     const int q = warp & 3;
-    const int half = (warp - 2) >> 2;
-    constexpr int CW = 32;  // output columns per warp
-    constexpr int VPR = CW * 2 / 16;  // 16-byte pieces of a token's CW columns
-    __nv_bfloat16* stg = stage + (warp - 2) * (32 * CW);  // [32 tokens][CW] bf16
+    const int half = (warp - 4) >> 2;
+    constexpr int CW = 32;            // hidden units per warp
+    constexpr int VPR = CW * 2 / 16;  // 16-byte pieces of a token's CW units
+    __nv_bfloat16* stg = stage + (warp - 4) * (32 * CW);  // [32 tokens][CW] bf16
     int local = 0;
     for (int tile = pair_id; tile < total; tile += num_pairs, ++local) {
       const SwapTile t = decode_swap(tile, p, st, routed);
-      const int acc = local & 1;
-      const uint32_t acc_phase = (uint32_t)(local >> 1) & 1u;
       const int col0 = t.m0 + (int)rank * 128 + 32 * q;
       __nv_bfloat16* outt = p.out + (size_t)t.out_row * p.n_out + col0;
-      {
-        if (!swap_wait<true>(&st->tfull[acc], acc_phase, st, p.err, kErrGemmTimeout | 0xC4))
-          break;
-        sm100::tc_fence_after();
-        const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256);
+      if (!swap_wait<true>(&st->tfull, (uint32_t)local & 1u, st, p.err, kErrGemmTimeout | 0xF4))
+        break;
+      sm100::tc_fence_after();
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
-        for (int cc = 32 * half; cc < t.n; cc += 64) {
-          uint32_t v[32];
-          sm100::tmem_ld_32x32b_x32(tbase + cc, v);
-          sm100::tmem_ld_wait();
+      for (int cc = 32 * half; cc < t.n; cc += 64) {
+        uint32_t u[32], v[32];
+        sm100::tmem_ld_32x32b_x32(tbase + cc, u);
+        sm100::tmem_ld_32x32b_x32(tbase + 256u + cc, v);
+        sm100::tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) stg[i * CW + lane] = __float2bfloat16_rn(__uint_as_float(v[i]));
-          __syncwarp();
-          // each token's CW columns leave as 16-byte stores
-#pragma unroll
-          for (int idx = lane; idx < 32 * VPR; idx += 32) {
-            const int i = idx / VPR, vv = idx % VPR;
-            const int j = cc + i;  // token within the tile
-            if (j < t.valid)
-              *reinterpret_cast<uint4*>(outt + (size_t)j * p.n_out + vv * 8) =
-                  *reinterpret_cast<const uint4*>(stg + i * CW + vv * 8);
-          }
-          __syncwarp();
+        for (int i = 0; i < 32; ++i) {
+          const float a = __uint_as_float(u[i]);
+          const float b = __uint_as_float(v[i]);
+          stg[i * CW + lane] = __float2bfloat16_rn(a * __frcp_rn(1.0f + __expf(-a)) * b);
         }
-        sm100::tc_fence_before();
-        sm100::mbar_arrive_cluster(sm100::mapa_shared(sm100::smem_addr(&st->tempty[acc]), 0));
+        __syncwarp();
+        // each token's CW hidden units leave as 16-byte stores
+#pragma unroll
+        for (int idx = lane; idx < 32 * VPR; idx += 32) {
+          const int i = idx / VPR, vv = idx % VPR;
+          const int j = cc + i;  // token within the tile
+          if (j < t.valid)
+            *reinterpret_cast<uint4*>(outt + (size_t)j * p.n_out + vv * 8) =
+                *reinterpret_cast<const uint4*>(stg + i * CW + vv * 8);
+        }
+        __syncwarp();
       }
+      sm100::tc_fence_before();
+      sm100::mbar_arrive_cluster(sm100::mapa_shared(sm100::smem_addr(&st->tempty), 0));
     }
   }
   sm100::tc_fence_before();
@@ -384,7 +661,8 @@ struct SwapMaps {
 };
 
 static cudaError_t launch_swap(const SwapMaps& m, const SwapParams& p, int pairs, cudaStream_t s) {
-  const size_t bytes = (size_t)kSStages * kSStageBytes + ((sizeof(SwapState) + 127) & ~size_t(127)) +
+  const size_t bytes = (size_t)kSStreams * kSStages * kSStageBytes +
+                       ((sizeof(SwapState) + 127) & ~size_t(127)) +
                        kSEpiWarps * 32 * 32 * sizeof(__nv_bfloat16) + 1024;
   auto kern = tc_swap_pair_kernel;
   cudaError_t e =
@@ -412,7 +690,68 @@ static int swap_pairs(const SwapParams& p, long long max_routed_rows) {
   return g < 1 ? 1 : (int)g;
 }
 
+
+static cudaError_t launch_swap_up(const SwapMaps& m, const CUtensorMap& w3,
+                                  const CUtensorMap& w3s, const SwapParams& p, int pairs,
+                                  cudaStream_t s) {
+  const size_t bytes = (size_t)kUStages * kUStageBytes +
+                       ((sizeof(UpState) + 127) & ~size_t(127)) +
+                       kUEpiWarps * 32 * 32 * sizeof(__nv_bfloat16) + 1024;
+  auto kern = tc_swap_up_pair_kernel;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, 2 * pairs, kUThreads, bytes, s, m.t[0], m.t[1], m.t[2], m.ts[0],
+                    m.ts[1], m.ts[2], m.w, w3, m.ws, w3s, p);
+}
+
 }  // namespace
+
+bool swap_up_supported(const FfnArgs& f) {
+  return f.act == MOE_ACT_SWIGLU && f.X_perm != nullptr && f.save_u == nullptr &&
+         f.counts != nullptr && f.E <= MOE_MAX_EXPERTS && f.h % 256 == 0 && f.d % kSBK == 0;
+}
+
+// H = silu(X_perm W1^T) * (X_perm W3^T) per expert over each expert's real
+// tokens (and per shared expert over the n rows of X), weights as the M side;
+// padding rows of H are not written
+moe_status run_ffn_up_swap(const FfnArgs& f, cudaStream_t s) {
+  SwapMaps m;
+  if (!token_maps(m.t, f.X_perm, f.rows, f.d)) return MOE_ERR_UNSUPPORTED;
+  CUtensorMap w3, w3s;
+  if (!make_bf16_sw128_map(&m.w, f.W1, (long long)f.E * f.h, f.d, 128)) return MOE_ERR_UNSUPPORTED;
+  if (!make_bf16_sw128_map(&w3, f.W3, (long long)f.E * f.h, f.d, 128)) return MOE_ERR_UNSUPPORTED;
+  if (f.n_shared > 0) {
+    // shared experts read the tokens of X itself
+    if (!token_maps(m.ts, f.X, f.n, f.d)) return MOE_ERR_UNSUPPORTED;
+    if (!make_bf16_sw128_map(&m.ws, f.sW1, (long long)f.n_shared * f.h, f.d, 128) ||
+        !make_bf16_sw128_map(&w3s, f.sW3, (long long)f.n_shared * f.h, f.d, 128))
+      return MOE_ERR_UNSUPPORTED;
+  } else {
+    for (int b = 0; b < 3; ++b) m.ts[b] = m.t[b];
+    m.ws = m.w;
+    w3s = w3;
+  }
+  SwapParams q{};
+  q.offsets = f.offsets;
+  q.counts = f.counts;
+  q.E = f.E;
+  q.K = f.d;
+  q.m_per_expert = f.h;
+  q.mt_tiles = f.h / 256;
+  q.n_shared = f.n_shared;
+  q.n = f.n;
+  q.shared_in_row = 0;
+  q.shared_in_stride = 0;
+  q.shared_out_row = f.shared_base;
+  q.n_pad = f.n_pad;
+  q.n_out = f.h;
+  q.out = static_cast<__nv_bfloat16*>(f.H);
+  q.err = f.err;
+  if (launch_swap_up(m, w3, w3s, q, swap_pairs(q, f.rows_routed), s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
 
 bool swap_down_supported(const FfnArgs& f) {
   return f.counts != nullptr && f.E <= MOE_MAX_EXPERTS && f.d % 256 == 0 && f.h % kSBK == 0;

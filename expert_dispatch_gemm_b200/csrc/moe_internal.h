@@ -216,6 +216,8 @@ struct FfnArgs {
 bool ffn_uses_pair(const moe_config* c, const Derived& d);
 moe_status run_ffn_bf16(const FfnArgs& a, cudaStream_t s);
 // the weights-as-M down projection for fine-grained experts (needs the counts)
+bool swap_up_supported(const FfnArgs& a);
+moe_status run_ffn_up_swap(const FfnArgs& a, cudaStream_t s);
 bool swap_down_supported(const FfnArgs& a);
 moe_status run_ffn_down_swap(const FfnArgs& a, cudaStream_t s);
 moe_status run_ffn_f32(const FfnArgs& a, cudaStream_t s);

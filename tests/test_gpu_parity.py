@@ -319,8 +319,10 @@ def test_full_size_sampled(w):
 
 EDGE = ROUTE_VARIANTS + [
     EC_MAX,
-    # 128 to 512 rows per expert on average: the weights-as-M down projection
-    # (exact token counts, chunks of at most 256 tokens per tile)
+    # 128 to 512 rows per expert on average: the weights-as-M projections
+    # (exact token counts, chunks of at most 256 tokens per tile; the SwiGLU
+    # up projection with two MMA issuers when h is a multiple of 256, the
+    # down projection on two tile streams)
     wl.TC_DROPLESS.replace(name="tc-swap-swiglu-top4of16", n=1024, d=256, E=16, K=4, h=256),
     wl.TC_DROPLESS.replace(name="tc-swap-gelu-shared-top2of8", n=600, d=256, E=8, K=2, h=256,
                            act="gelu", n_shared=1),
