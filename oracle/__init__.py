@@ -94,7 +94,8 @@ def lib() -> ctypes.CDLL:
                                            c_int, _f32p, _f32p]
         L.orc_expert_ffn_backward.argtypes = [c_int, c_int, c_int, c_int, c_int, _f32p, _f32p,
                                               _opt(_f32p), _f32p, _f32p, _f32p, _f32p,
-                                              _opt(_f32p), _f32p]
+                                              _opt(_f32p), _f32p, _opt(_f32p), _opt(_f32p),
+                                              _opt(_f32p)]
         L.orc_gate_backward_tc.argtypes = [c_int, c_int, c_int, _f32p, _i32p, c_int, _f64p,
                                            _f64p]
         L.orc_score_backward.argtypes = [c_int, c_int, c_int, c_int, _f32p, _f32p, _f64p,
@@ -389,9 +390,12 @@ def combine_backward(pair_token, pair_gate, Y, dout, store: int):
     return dY, dgate
 
 
-def expert_ffn_backward(X, W1, W3, W2, dY, act: int, store: int):
+def expert_ffn_backward(X, W1, W3, W2, dY, act: int, store: int, absum: bool = False):
     """One expert's backward over its rows: (dX [m,d], dW1 [h,d], dW3 [h,d] or
-    None, dW2 [d,h])."""
+    None, dW2 [d,h]). With absum=True, also (aW1, aW3, aW2): the weight
+    gradients' sums taken over the absolute values of their terms
+    (sum_r |dU_rj| |x_ri|, ...), a bound helper for comparing gradients whose
+    factors were stored in bf16."""
     X = _f32(X)
     m, d = X.shape
     h = W1.shape[0]
@@ -399,10 +403,15 @@ def expert_ffn_backward(X, W1, W3, W2, dY, act: int, store: int):
     dW1 = np.zeros((h, d), np.float32)
     dW3 = np.zeros((h, d), np.float32) if act == SWIGLU else None
     dW2 = np.zeros((d, h), np.float32)
+    aW1 = np.zeros((h, d), np.float32) if absum else None
+    aW3 = np.zeros((h, d), np.float32) if absum and act == SWIGLU else None
+    aW2 = np.zeros((d, h), np.float32) if absum else None
     if m:
         lib().orc_expert_ffn_backward(m, d, h, act, store, X, _f32(W1),
                                       None if W3 is None else _f32(W3), _f32(W2), _f32(dY),
-                                      dX, dW1, dW3, dW2)
+                                      dX, dW1, dW3, dW2, aW1, aW3, aW2)
+    if absum:
+        return dX, dW1, dW3, dW2, aW1, aW3, aW2
     return dX, dW1, dW3, dW2
 
 
@@ -443,7 +452,8 @@ def router_backward(X, Wg, dL):
 
 
 def layer_backward(spec: dict, X, Wg, dout, expert_weights, shared_weights=None,
-                   logit_bias=None, sel_bias=None, tokens=None, pre=None):
+                   logit_bias=None, sel_bias=None, tokens=None, pre=None,
+                   absum: bool = False):
     """Gradients of <dout, out> + lb_coef L_lb + z_coef L_z (token choice) for
     the layer of ``layer_forward``, by the chain rule through the same steps:
     combine -> expert FFN -> dispatch (a sum over each token's pairs), and
@@ -456,7 +466,9 @@ def layer_backward(spec: dict, X, Wg, dout, expert_weights, shared_weights=None,
     With ``tokens`` only those rows of dX and dL are computed (each needs only
     its own pairs), and no weight gradient is returned. ``pre`` = (logits, S,
     lse, routing) from an earlier ``router`` + ``route`` of the same inputs
-    skips recomputing them."""
+    skips recomputing them. With ``absum`` (and no ``tokens``) the dict also
+    holds aW1/aW3/aW2 and asW1/asW3/asW2: each weight gradient's sum over the
+    absolute values of its terms (see ``expert_ffn_backward``)."""
     X = _f32(X)
     dout = _f32(dout)
     n, d = X.shape
@@ -476,6 +488,9 @@ def layer_backward(spec: dict, X, Wg, dout, expert_weights, shared_weights=None,
     dXacc = np.zeros((n, d), np.float64)
     dgate = {}
     grads = {"dW1": {}, "dW3": {}, "dW2": {}, "dsW1": {}, "dsW3": {}, "dsW2": {}}
+    want_abs = absum and tokens is None
+    if want_abs:
+        grads.update({"aW1": {}, "aW3": {}, "aW2": {}, "asW1": {}, "asW3": {}, "asW2": {}})
     for e in sorted(by_e):
         W1, W3, W2 = expert_weights(e)
         ts = [t for t, _ in by_e[e]]
@@ -485,7 +500,12 @@ def layer_backward(spec: dict, X, Wg, dout, expert_weights, shared_weights=None,
                                   dout, store)
         for t, v in zip(ts, dg):
             dgate[(t, e)] = float(v)
-        dXp, dW1, dW3, dW2 = expert_ffn_backward(X[ts], W1, W3, W2, dY, act, store)
+        res = expert_ffn_backward(X[ts], W1, W3, W2, dY, act, store, absum=want_abs)
+        dXp, dW1, dW3, dW2 = res[:4]
+        if want_abs:
+            grads["aW1"][e], grads["aW2"][e] = res[4], res[6]
+            if res[5] is not None:
+                grads["aW3"][e] = res[5]
         np.add.at(dXacc, np.asarray(ts), dXp.astype(np.float64))
         if tokens is None:
             grads["dW1"][e], grads["dW2"][e] = dW1, dW2
@@ -495,7 +515,12 @@ def layer_backward(spec: dict, X, Wg, dout, expert_weights, shared_weights=None,
         W1, W3, W2 = shared_weights(s_)
         dY, _ = combine_backward(np.asarray(rows, np.int32), np.ones(len(rows), np.float32),
                                  np.zeros((len(rows), d), np.float32), dout, store)
-        dXp, dW1, dW3, dW2 = expert_ffn_backward(X[rows], W1, W3, W2, dY, act, store)
+        res = expert_ffn_backward(X[rows], W1, W3, W2, dY, act, store, absum=want_abs)
+        dXp, dW1, dW3, dW2 = res[:4]
+        if want_abs:
+            grads["asW1"][s_], grads["asW2"][s_] = res[4], res[6]
+            if res[5] is not None:
+                grads["asW3"][s_] = res[5]
         dXacc[rows] += dXp.astype(np.float64)
         if tokens is None:
             grads["dsW1"][s_], grads["dsW2"][s_] = dW1, dW2

@@ -374,11 +374,17 @@ void orc_combine_backward(int n, int d, int P, const int32_t* pair_token,
 void orc_expert_ffn_backward(int m, int d, int h, int act, int store,
                              const float* X, const float* W1, const float* W3,
                              const float* W2, const float* dY, float* dX,
-                             float* dW1, float* dW3, float* dW2) {
+                             float* dW1, float* dW3, float* dW2, float* absW1,
+                             float* absW3, float* absW2) {
   const int swiglu = act == ORC_SWIGLU;
+  const int want_abs = absW1 != NULL;
   double* aW1 = (double*)calloc((size_t)h * d, sizeof(double));
   double* aW3 = swiglu ? (double*)calloc((size_t)h * d, sizeof(double)) : NULL;
   double* aW2 = (double*)calloc((size_t)d * h, sizeof(double));
+  /* the same sums over |terms| (a bound helper for comparing stored values) */
+  double* bW1 = want_abs ? (double*)calloc((size_t)h * d, sizeof(double)) : NULL;
+  double* bW3 = want_abs && swiglu ? (double*)calloc((size_t)h * d, sizeof(double)) : NULL;
+  double* bW2 = want_abs ? (double*)calloc((size_t)d * h, sizeof(double)) : NULL;
   float* Hs = (float*)malloc(sizeof(float) * (size_t)h);
   float* dUs = (float*)malloc(sizeof(float) * (size_t)h);
   float* dVs = (float*)malloc(sizeof(float) * (size_t)h);
@@ -423,15 +429,34 @@ void orc_expert_ffn_backward(int m, int d, int h, int act, int store,
       }
     for (int i = 0; i < d; ++i)
       for (int j = 0; j < h; ++j) aW2[(size_t)i * h + j] += (double)dy[i] * (double)Hs[j];
+    if (want_abs) {
+      for (int j = 0; j < h; ++j)
+        for (int i = 0; i < d; ++i) {
+          bW1[(size_t)j * d + i] += fabs((double)dUs[j]) * fabs((double)x[i]);
+          if (swiglu) bW3[(size_t)j * d + i] += fabs((double)dVs[j]) * fabs((double)x[i]);
+        }
+      for (int i = 0; i < d; ++i)
+        for (int j = 0; j < h; ++j)
+          bW2[(size_t)i * h + j] += fabs((double)dy[i]) * fabs((double)Hs[j]);
+    }
   }
   for (size_t q = 0; q < (size_t)h * d; ++q) {
     dW1[q] = round_store(aW1[q], store);
     if (swiglu) dW3[q] = round_store(aW3[q], store);
     dW2[q] = round_store(aW2[q], store);
   }
+  if (want_abs)
+    for (size_t q = 0; q < (size_t)h * d; ++q) {
+      absW1[q] = (float)bW1[q];
+      if (swiglu && absW3) absW3[q] = (float)bW3[q];
+      if (absW2) absW2[q] = (float)bW2[q];
+    }
   free(aW1);
   free(aW3);
   free(aW2);
+  free(bW1);
+  free(bW3);
+  free(bW2);
   free(Hs);
   free(dUs);
   free(dVs);

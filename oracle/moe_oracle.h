@@ -121,11 +121,17 @@ void orc_combine_backward(int n, int d, int P, const int32_t* pair_token,
  * gradient dY [m,d]: dH = dY W2; dU = dH * act'(U) (SwiGLU: dU = dH V
  * silu'(U), dV = dH silu(U), from the stored U, V); dX = dU W1 (+ dV W3)
  * [m,d]; dW1 = dU^T X, dW3 = dV^T X [h,d]; dW2 = dY^T H [d,h], H as the
- * forward stores it. dW3 only for SwiGLU (else may be NULL). */
+ * forward stores it. dW3 only for SwiGLU (else may be NULL). absW1 / absW3
+ * / absW2, when absW1 is not NULL, receive the same sums taken over the
+ * absolute values of their terms (sum_r |dU_rj| |x_ri| and so on): not part
+ * of the method, a bound for comparing a computed gradient whose factors
+ * were stored at lower precision (a factor's rounding moves an element by at
+ * most its relative spacing times that term). */
 void orc_expert_ffn_backward(int m, int d, int h, int act, int store,
                              const float* X, const float* W1, const float* W3,
                              const float* W2, const float* dY, float* dX,
-                             float* dW1, float* dW3, float* dW2);
+                             float* dW1, float* dW3, float* dW2, float* absW1,
+                             float* absW3, float* absW2);
 
 /* Token-choice mixing weights backward: dS [n,E] (double, accumulated into)
  * from the weight gradients dw [n,K] of the selected experts idx [n,K]:

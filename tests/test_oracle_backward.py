@@ -203,6 +203,45 @@ def test_expert_backward_against_autograd(act):
         np.testing.assert_allclose(dW3, t3.grad.numpy(), rtol=1e-5, atol=1e-5)
 
 
+@pytest.mark.parametrize("act", [oracle.SWIGLU, oracle.GELU])
+def test_expert_backward_term_magnitudes(act):
+    """The weight gradients' sums over |terms| (the comparison bound's input):
+    sum_r |dU_rj| |x_ri| (and dV, and sum_r |dY_ri| |H_rj|) against the same
+    sums of autograd's pre-activation gradients and hidden rows; each sum is
+    at least |gradient|, and with one row it is |gradient| itself."""
+    rng = np.random.default_rng(11)
+    m, d, h = 9, 12, 10
+    X = rng.standard_normal((m, d)).astype(np.float32)
+    W1 = (rng.standard_normal((h, d)) / 3).astype(np.float32)
+    W3 = (rng.standard_normal((h, d)) / 3).astype(np.float32)
+    W2 = (rng.standard_normal((d, h)) / 3).astype(np.float32)
+    dY = rng.standard_normal((m, d)).astype(np.float32)
+    sw = act == oracle.SWIGLU
+    _, dW1, dW3, dW2, a1, a3, a2 = oracle.expert_ffn_backward(
+        X, W1, W3 if sw else None, W2, dY, act, F32, absum=True)
+    tX = torch.tensor(X, dtype=torch.float64)
+    u = (tX @ torch.tensor(W1, dtype=torch.float64).T).requires_grad_(True)
+    v = (tX @ torch.tensor(W3, dtype=torch.float64).T).requires_grad_(True)
+    hdn = torch.nn.functional.silu(u) * v if sw else torch.nn.functional.gelu(u)
+    y = hdn @ torch.tensor(W2, dtype=torch.float64).T
+    y.backward(torch.tensor(dY, dtype=torch.float64))
+    ax = tX.abs()
+    np.testing.assert_allclose(a1, (u.grad.abs().T @ ax).numpy(), rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(a2, (torch.tensor(dY, dtype=torch.float64).abs().T
+                                    @ hdn.detach().abs()).numpy(), rtol=1e-5, atol=1e-6)
+    if sw:
+        np.testing.assert_allclose(a3, (v.grad.abs().T @ ax).numpy(), rtol=1e-5, atol=1e-6)
+    else:
+        assert a3 is None
+    for g, a in ((dW1, a1), (dW2, a2)) + (((dW3, a3),) if sw else ()):
+        assert (a >= np.abs(g) * (1 - 1e-6)).all()
+    # one row: every sum has a single term
+    _, g1, g3, g2, b1, b3, b2 = oracle.expert_ffn_backward(
+        X[:1], W1, W3 if sw else None, W2, dY[:1], act, F32, absum=True)
+    for g, a in ((g1, b1), (g2, b2)) + (((g3, b3),) if sw else ()):
+        np.testing.assert_allclose(a, np.abs(g), rtol=1e-6, atol=0)
+
+
 @pytest.mark.parametrize("score", [oracle.SOFTMAX, oracle.SIGMOID, oracle.SQRTSOFTPLUS])
 def test_score_and_router_backward_against_autograd(score):
     """With every expert selected and raw weights, the router's gradient is
