@@ -97,3 +97,21 @@ def test_reference_arm_other_ranks_exit_without_output():
                          capture_output=True, text=True, timeout=600, cwd=ROOT, env=env)
     assert out.returncode == 0, out.stderr[-2000:]
     assert out.stdout.strip() == ""
+
+
+def test_clock_summary_reads_nvml_masks_and_smi_lines():
+    """The clock record: median SM clock under load, the maximum, and every
+    clock-event reason seen in any sample, from NVML bitmasks (hw slowdown
+    0x8, sw power cap 0x4, ...) or from nvidia-smi's csv fields."""
+    c = bench.ClockSampler(0)
+    c.samples = [(1700, 1965, 0x4), (1650, 1965, 0x4 | 0x8), (1750, 1965, 0x0)]
+    c.lines = []
+    s = c.summary()
+    assert s["sm_mhz"] == 1700.0 and s["sm_max_mhz"] == 1965.0 and s["samples"] == 3
+    assert s["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    c = bench.ClockSampler(0)
+    c.lines = ["0, 1800, 1965, 950.1, 0x4, Not Active, Not Active, Not Active, Active",
+               "0, 1900, 1965, 900.0, 0x0, Not Active, Not Active, Not Active, Not Active"]
+    s = c.summary()
+    assert s["sm_mhz"] == 1850.0 and s["reasons"] == ["sw_power_cap"]
+    assert bench.ClockSampler(0).summary()["reasons"] == ["unsampled"]
