@@ -163,21 +163,34 @@ __device__ __forceinline__ SwapTile decode_swap(int tile, const SwapParams& p, c
   return t;
 }
 
-// token rows one CTA loads for an N-column slot: N/2, as a TMA box of 32, 64 or 128
-__device__ __forceinline__ int box_rows(int n) {
-  const int half = n / 2;
-  return half <= 32 ? 32 : half <= 64 ? 64 : 128;
+// The token operand: a CTA loads exactly its N/2 rows (a multiple of 8, at
+// most 128) as boxes of 128, 64, 32, 16 and 8 rows, each at a 1 KB-aligned
+// shared-memory offset (whole 8-row atoms of the 128-byte swizzle, so the
+// tile is laid out as one box would lay it out), all completing on the
+// leader's barrier `fl`.
+constexpr int kTokBoxes = 5;
+struct TokenMaps {
+  CUtensorMap m[kTokBoxes];  // box of 8 << b rows
+};
+
+__device__ __forceinline__ void load_token_rows(unsigned char* dst, const TokenMaps& tk,
+                                                uint32_t fl, int x, long long row0, int rows) {
+  int off = 0;
+#pragma unroll
+  for (int b = kTokBoxes - 1; b >= 0; --b) {
+    const int r = 8 << b;
+    if (rows & r) {
+      sm100::tma_load_2d_pair(dst + off * 128, &tk.m[b], fl, x, (int)(row0 + off));
+      off += r;
+    }
+  }
 }
 
-// token maps: tmT[b] / tmTs[b] = routed / shared token rows of H with a box
-// of 32 << b rows; weights: tmW (routed) / tmWs (shared), boxes of 128 rows
+// token maps: tk / tks = routed / shared token rows of H; weights: tmW
+// (routed) / tmWs (shared), boxes of 128 rows
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSThreads, 1)
-    tc_swap_pair_kernel(const __grid_constant__ CUtensorMap tmT0,
-                        const __grid_constant__ CUtensorMap tmT1,
-                        const __grid_constant__ CUtensorMap tmT2,
-                        const __grid_constant__ CUtensorMap tmTs0,
-                        const __grid_constant__ CUtensorMap tmTs1,
-                        const __grid_constant__ CUtensorMap tmTs2,
+    tc_swap_pair_kernel(const __grid_constant__ TokenMaps tk,
+                        const __grid_constant__ TokenMaps tks,
                         const __grid_constant__ CUtensorMap tmW,
                         const __grid_constant__ CUtensorMap tmWs, const SwapParams p) {
   extern __shared__ __align__(1024) unsigned char ssm[];
@@ -254,15 +267,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSThreads, 1)
       bool ok = true;
       for (int tile = first; ok && tile < total; tile += step) {
         const SwapTile t = decode_swap(tile, p, st, routed);
-        const CUtensorMap* tm[3];
-        if (t.shared) {
-          tm[0] = &tmTs0; tm[1] = &tmTs1; tm[2] = &tmTs2;
-        } else {
-          tm[0] = &tmT0; tm[1] = &tmT1; tm[2] = &tmT2;
-        }
-        const int b1 = box_rows(t.n);
-        const CUtensorMap* m1 = tm[b1 == 32 ? 0 : b1 == 64 ? 1 : 2];
-        const uint32_t bytes = kSABytes + (uint32_t)b1 * kSBK * 2;
+        const TokenMaps& tmk = t.shared ? tks : tk;
+        const int half_rows = t.n / 2;  // this CTA's token rows
+        const uint32_t bytes = kSABytes + (uint32_t)half_rows * kSBK * 2;
         const CUtensorMap* mw = t.shared ? &tmWs : &tmW;
         const int wrow = t.expert * p.m_per_expert + t.m0 + (int)rank * 128;  // this CTA's 128
         // this CTA's half of the tile's tokens
@@ -276,7 +283,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSThreads, 1)
           const uint32_t fl = sm100::mapa_shared(sm100::smem_addr(&st->full[sx][stage]), 0);
           if (leader) sm100::mbar_arrive_expect_tx(&st->full[sx][stage], 2 * bytes);
           sm100::tma_load_2d_pair(sA(sx, stage), mw, fl, kb * kSBK, wrow);
-          sm100::tma_load_2d_pair(sB(sx, stage), m1, fl, kb * kSBK, (int)trow1);
+          load_token_rows(sB(sx, stage), tmk, fl, kb * kSBK, trow1, half_rows);
           ++issued;
           if (++stage == kSStages) {
             stage = 0;
@@ -431,12 +438,8 @@ struct UpState {
 };
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kUThreads, 1)
-    tc_swap_up_pair_kernel(const __grid_constant__ CUtensorMap tmT0,
-                           const __grid_constant__ CUtensorMap tmT1,
-                           const __grid_constant__ CUtensorMap tmT2,
-                           const __grid_constant__ CUtensorMap tmTs0,
-                           const __grid_constant__ CUtensorMap tmTs1,
-                           const __grid_constant__ CUtensorMap tmTs2,
+    tc_swap_up_pair_kernel(const __grid_constant__ TokenMaps tk,
+                           const __grid_constant__ TokenMaps tks,
                            const __grid_constant__ CUtensorMap tmW1,
                            const __grid_constant__ CUtensorMap tmW3,
                            const __grid_constant__ CUtensorMap tmW1s,
@@ -508,15 +511,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kUThreads, 1)
       bool ok = true;
       for (int tile = pair_id; ok && tile < total; tile += num_pairs) {
         const SwapTile t = decode_swap(tile, p, st, routed);
-        const CUtensorMap* tm[3];
-        if (t.shared) {
-          tm[0] = &tmTs0; tm[1] = &tmTs1; tm[2] = &tmTs2;
-        } else {
-          tm[0] = &tmT0; tm[1] = &tmT1; tm[2] = &tmT2;
-        }
-        const int b1 = box_rows(t.n);
-        const CUtensorMap* m1 = tm[b1 == 32 ? 0 : b1 == 64 ? 1 : 2];
-        const uint32_t bytes = 2 * kUWBytes + (uint32_t)b1 * kSBK * 2;
+        const TokenMaps& tmk = t.shared ? tks : tk;
+        const int half_rows = t.n / 2;  // this CTA's token rows
+        const uint32_t bytes = 2 * kUWBytes + (uint32_t)half_rows * kSBK * 2;
         const CUtensorMap* mw1 = t.shared ? &tmW1s : &tmW1;
         const CUtensorMap* mw3 = t.shared ? &tmW3s : &tmW3;
         const int wrow = t.expert * p.m_per_expert + t.m0 + (int)rank * 128;  // this CTA's 128
@@ -531,7 +528,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kUThreads, 1)
           if (leader) sm100::mbar_arrive_expect_tx(&st->full[stage], 2 * bytes);
           sm100::tma_load_2d_pair(sW(stage, 0), mw1, fl, kb * kSBK, wrow);
           sm100::tma_load_2d_pair(sW(stage, 1), mw3, fl, kb * kSBK, wrow);
-          sm100::tma_load_2d_pair(sB(stage), m1, fl, kb * kSBK, (int)trow1);
+          load_token_rows(sB(stage), tmk, fl, kb * kSBK, trow1, half_rows);
           ++issued;
           if (++stage == kUStages) {
             stage = 0;
@@ -657,7 +654,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kUThreads, 1)
 // host side
 // ---------------------------------------------------------------------------
 struct SwapMaps {
-  CUtensorMap t[3], ts[3], w, ws;
+  TokenMaps t, ts;
+  CUtensorMap w, ws;
 };
 
 static cudaError_t launch_swap(const SwapMaps& m, const SwapParams& p, int pairs, cudaStream_t s) {
@@ -668,13 +666,12 @@ static cudaError_t launch_swap(const SwapMaps& m, const SwapParams& p, int pairs
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, 2 * pairs, kSThreads, bytes, s, m.t[0], m.t[1], m.t[2], m.ts[0],
-                    m.ts[1], m.ts[2], m.w, m.ws, p);
+  return launch_pdl(kern, 2 * pairs, kSThreads, bytes, s, m.t, m.ts, m.w, m.ws, p);
 }
 
-static bool token_maps(CUtensorMap (&t)[3], const void* ptr, long long rows, long long cols) {
-  for (int b = 0; b < 3; ++b)
-    if (!make_bf16_sw128_map(&t[b], ptr, rows, cols, 32 << b)) return false;
+static bool token_maps(TokenMaps& t, const void* ptr, long long rows, long long cols) {
+  for (int b = 0; b < kTokBoxes; ++b)
+    if (!make_bf16_sw128_map(&t.m[b], ptr, rows, cols, 8 << b)) return false;
   return true;
 }
 
@@ -701,8 +698,7 @@ static cudaError_t launch_swap_up(const SwapMaps& m, const CUtensorMap& w3,
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, 2 * pairs, kUThreads, bytes, s, m.t[0], m.t[1], m.t[2], m.ts[0],
-                    m.ts[1], m.ts[2], m.w, w3, m.ws, w3s, p);
+  return launch_pdl(kern, 2 * pairs, kUThreads, bytes, s, m.t, m.ts, m.w, w3, m.ws, w3s, p);
 }
 
 }  // namespace
@@ -728,7 +724,7 @@ moe_status run_ffn_up_swap(const FfnArgs& f, cudaStream_t s) {
         !make_bf16_sw128_map(&w3s, f.sW3, (long long)f.n_shared * f.h, f.d, 128))
       return MOE_ERR_UNSUPPORTED;
   } else {
-    for (int b = 0; b < 3; ++b) m.ts[b] = m.t[b];
+    m.ts = m.t;
     m.ws = m.w;
     w3s = w3;
   }
@@ -762,7 +758,7 @@ bool swap_down_supported(const FfnArgs& f) {
 moe_status run_ffn_down_swap(const FfnArgs& f, cudaStream_t s) {
   SwapMaps m;
   if (!token_maps(m.t, f.H, f.rows, f.h)) return MOE_ERR_UNSUPPORTED;
-  for (int b = 0; b < 3; ++b) m.ts[b] = m.t[b];  // shared rows are rows of H too
+  m.ts = m.t;  // shared rows are rows of H too
   if (!make_bf16_sw128_map(&m.w, f.W2, (long long)f.E * f.d, f.h, 128)) return MOE_ERR_UNSUPPORTED;
   if (f.n_shared > 0) {
     if (!make_bf16_sw128_map(&m.ws, f.sW2, (long long)f.n_shared * f.d, f.h, 128))
