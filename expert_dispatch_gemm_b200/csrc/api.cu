@@ -889,11 +889,13 @@ static moe_status bwd_gemms_bf16(const moe_config* cfg, const Derived& d, const 
     return make_bf16_sw128_map(m, p, r, c, box);
   };
   // row GEMMs on CTA pairs when experts average two 128-row blocks, as the
-  // forward does. The weight gradients stay on single CTAs: their few
-  // k-blocks per tile leave the epilogue in charge, and pairs measured ~10%
-  // slower there (c5: 6.07 / 3.13 ms against 5.56 / 2.77 ms)
+  // forward does; the weight gradients too. A single CTA's 128 x 256 tile
+  // over an expert's few k-blocks waits on its operands (c5: the MMA thread
+  // idles 46% of the time for loads); a pair's 256 x 256 tile loads half of
+  // B per CTA (16% waiting for loads, 27% for the epilogue), 8-9% fewer
+  // cycles per launch
   const bool rpair = ffn_uses_pair(cfg, d);
-  const bool wpair = false;
+  const bool wpair = rpair;
   // 3. SAVE: U (and V), H of every dispatched row again (unless the
   //    training forward kept them)
   if (!B.saved) {
