@@ -947,8 +947,34 @@ static moe_status bwd_gemms_bf16(const moe_config* cfg, const Derived& d, const 
     p.ld_out = swiglu ? 2LL * h : h;
     MOE_CU(run_bwd_gemm(BW_DACT, rpair, m, p, s));
   }
-  // 5. DX: dX_perm = dU W1 (+ dV W3)
-  {
+  // 5. DX: dX_perm = dU W1 (+ dV W3). Fine-grained token choice (128 to 512
+  //    rows per expert on average) puts the weights on the M side, as the
+  //    forward's down projection does: each expert's exact token count instead
+  //    of whole 256-row pair tiles
+  SwapDxArgs sx{};
+  sx.duv = duv;
+  sx.rows = rows;
+  sx.rows_routed = d.rows_routed;
+  sx.kcols = swiglu ? 2 * h : h;
+  sx.E = E;
+  sx.h = h;
+  sx.d = D;
+  sx.n_shared = ns;
+  sx.n = n;
+  sx.shared_base = d.shared_base;
+  sx.n_pad = d.n_pad;
+  sx.W1 = W1;
+  sx.W3 = swiglu ? W3 : nullptr;
+  sx.sW1 = sW1;
+  sx.sW3 = swiglu ? sW3 : nullptr;
+  sx.offsets = route->offsets;
+  sx.counts = route->counts;
+  sx.dxp = dxp;
+  sx.err = err;
+  if (ffn_uses_swap(cfg, d) && swap_dx_supported(sx)) {
+    const moe_status st = run_bwd_dx_swap(sx, s);
+    if (st != MOE_OK) return st;
+  } else {
     BwdMaps m{};
     BwdParams p = base;
     const long long kcols = swiglu ? 2LL * h : h;

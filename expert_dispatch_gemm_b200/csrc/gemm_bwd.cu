@@ -55,7 +55,7 @@ constexpr int kWABytes = kWBM * kWBK * 2;          // 16 KB: this CTA's 128 rows
 constexpr int kWThreads = 320;  // producer, MMA, eight epilogue warps
 constexpr int kEpiThreads = 256;
 constexpr uint64_t kWWaitNs = 2000000000ull;       // 2 s
-constexpr uint32_t kMnChunkBytes = 64 * kWBK * 2;  // one 64 x 64 MN-major box: 8 KB
+constexpr uint32_t kMnChunkBytes = sm100::kMnChunkBytes;  // one 64 x 64 MN-major box: 8 KB
 constexpr int kWStagesMax = 6;
 
 // shared-memory ring: a single CTA holds all 256 rows of B (48 KB stages);
@@ -106,19 +106,6 @@ __device__ __forceinline__ bool bwait(uint64_t* bar, uint32_t parity, BwdState* 
       }
     }
   }
-}
-
-// canonical MN-major layout with 128-byte swizzle: start address >> 4 in
-// [0,14), leading byte offset (between 64-element MN chunks) >> 4 in [16,30),
-// stride byte offset (between 8-row K groups, 1024 B) >> 4 in [32,46),
-// descriptor version 1 in [46,48), swizzle mode 2 (128 B) in [61,64)
-__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t saddr) {
-  uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
-  d |= (uint64_t)(kMnChunkBytes >> 4) << 16;
-  d |= (uint64_t)(1024 >> 4) << 32;
-  d |= (uint64_t)1 << 46;
-  d |= (uint64_t)2 << 61;
-  return d;
 }
 
 // kind::f16 instruction descriptor with the operands' majorness: bit 15 = A
@@ -564,9 +551,9 @@ __device__ __forceinline__ void bwd_body(const CUtensorMap* tmA0, const CUtensor
           const uint32_t a_addr = sm100::smem_addr(sA + stage * kWABytes);
           const uint32_t b_addr = sm100::smem_addr(sB + stage * R::b_bytes);
           const uint64_t adesc =
-              Tr::A_MN ? sw128_mnmajor_desc(a_addr) : sm100::sw128_kmajor_desc(a_addr);
+              Tr::A_MN ? sm100::sw128_mnmajor_desc(a_addr) : sm100::sw128_kmajor_desc(a_addr);
           const uint64_t bdesc =
-              Tr::B_MN ? sw128_mnmajor_desc(b_addr) : sm100::sw128_kmajor_desc(b_addr);
+              Tr::B_MN ? sm100::sw128_mnmajor_desc(b_addr) : sm100::sw128_kmajor_desc(b_addr);
           // one K16 step: +32 bytes inside a K-major row (+2 in the address
           // field); +16 rows of 128 bytes in an MN-major tile (+128)
           constexpr uint64_t a_step = Tr::A_MN ? 128 : 2;

@@ -70,6 +70,10 @@ struct SwapParams {
   int n_out;                // output row pitch (d)
   __nv_bfloat16* out;
   int* err;
+  // MN-major weights (the backward's dX = dU W1 + dV W3): K index where the
+  // second weight matrix takes over, and K rows per expert in the maps
+  int k_split;
+  int w_k_rows;
 };
 
 struct SwapState {
@@ -186,13 +190,19 @@ __device__ __forceinline__ void load_token_rows(unsigned char* dst, const TokenM
   }
 }
 
-// token maps: tk / tks = routed / shared token rows of H; weights: tmW
-// (routed) / tmWs (shared), boxes of 128 rows
+// token maps: tk / tks = routed / shared token rows of the B source; weights:
+// tmW (routed) / tmWs (shared), K-major boxes of 128 rows. A_MN: the weights
+// are read MN-major (the backward's dX^T = W1^T dU^T + W3^T dV^T: W1 and W3
+// stored [h, d], the output index d contiguous) as two 64 x 64 boxes per
+// stage, from tmW / tmWs below K = k_split and tmW3 / tmW3s above it.
+template <bool A_MN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSThreads, 1)
     tc_swap_pair_kernel(const __grid_constant__ TokenMaps tk,
                         const __grid_constant__ TokenMaps tks,
                         const __grid_constant__ CUtensorMap tmW,
-                        const __grid_constant__ CUtensorMap tmWs, const SwapParams p) {
+                        const __grid_constant__ CUtensorMap tmW3,
+                        const __grid_constant__ CUtensorMap tmWs,
+                        const __grid_constant__ CUtensorMap tmW3s, const SwapParams p) {
   extern __shared__ __align__(1024) unsigned char ssm[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(ssm) + 1023) & ~uintptr_t(1023));
@@ -282,7 +292,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSThreads, 1)
           }
           const uint32_t fl = sm100::mapa_shared(sm100::smem_addr(&st->full[sx][stage]), 0);
           if (leader) sm100::mbar_arrive_expect_tx(&st->full[sx][stage], 2 * bytes);
-          sm100::tma_load_2d_pair(sA(sx, stage), mw, fl, kb * kSBK, wrow);
+          if (A_MN) {
+            const int k0 = kb * kSBK;
+            const bool second = k0 >= p.k_split;
+            const CUtensorMap* mk = t.shared ? (second ? &tmW3s : &tmWs) : (second ? &tmW3 : &tmW);
+            const int ky = t.expert * p.w_k_rows + (second ? k0 - p.k_split : k0);
+            const int mx = t.m0 + (int)rank * 128;  // this CTA's 128 outputs, two 64-wide boxes
+            sm100::tma_load_2d_pair(sA(sx, stage), mk, fl, mx, ky);
+            sm100::tma_load_2d_pair(sA(sx, stage) + sm100::kMnChunkBytes, mk, fl, mx + 64, ky);
+          } else {
+            sm100::tma_load_2d_pair(sA(sx, stage), mw, fl, kb * kSBK, wrow);
+          }
           load_token_rows(sB(sx, stage), tmk, fl, kb * kSBK, trow1, half_rows);
           ++issued;
           if (++stage == kSStages) {
@@ -324,18 +344,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSThreads, 1)
           break;
         }
         sm100::tc_fence_after();
-        const uint32_t idesc = sm100::idesc_bf16_f32(256, t.n);
+        // bit 15: A MN-major
+        const uint32_t idesc = sm100::idesc_bf16_f32(256, t.n) | (A_MN ? (1u << 15) : 0u);
         for (int kb = 0; kb < KB; ++kb) {
           if (!swap_wait<false>(&st->full[sx][stage], phase, st, p.err, kErrGemmTimeout | 0xB3)) {
             ok = false;
             break;
           }
           sm100::tc_fence_after();
-          const uint64_t adesc = sm100::sw128_kmajor_desc(sm100::smem_addr(sA(sx, stage)));
+          const uint32_t a_addr = sm100::smem_addr(sA(sx, stage));
+          const uint64_t adesc =
+              A_MN ? sm100::sw128_mnmajor_desc(a_addr) : sm100::sw128_kmajor_desc(a_addr);
           const uint64_t bdesc = sm100::sw128_kmajor_desc(sm100::smem_addr(sB(sx, stage)));
+          // one K16 step: +32 bytes in a K-major row, +16 rows in an MN-major tile
+          constexpr uint64_t a_step = A_MN ? 128 : 2;
 #pragma unroll
           for (int k = 0; k < kSBK / 16; ++k)
-            sm100::umma_f16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0);
+            sm100::umma_f16_pair(d_tmem, adesc + a_step * k, bdesc + 2 * k, idesc, (kb | k) != 0);
           sm100::umma_commit_pair_mc(&st->empty[sx][stage], 0x3);
           if (++stage == kSStages) {
             stage = 0;
@@ -658,15 +683,17 @@ struct SwapMaps {
   CUtensorMap w, ws;
 };
 
-static cudaError_t launch_swap(const SwapMaps& m, const SwapParams& p, int pairs, cudaStream_t s) {
+template <bool A_MN>
+static cudaError_t launch_swap(const SwapMaps& m, const CUtensorMap& w3, const CUtensorMap& w3s,
+                               const SwapParams& p, int pairs, cudaStream_t s) {
   const size_t bytes = (size_t)kSStreams * kSStages * kSStageBytes +
                        ((sizeof(SwapState) + 127) & ~size_t(127)) +
                        kSEpiWarps * 32 * 32 * sizeof(__nv_bfloat16) + 1024;
-  auto kern = tc_swap_pair_kernel;
+  auto kern = tc_swap_pair_kernel<A_MN>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, 2 * pairs, kSThreads, bytes, s, m.t, m.ts, m.w, m.ws, p);
+  return launch_pdl(kern, 2 * pairs, kSThreads, bytes, s, m.t, m.ts, m.w, w3, m.ws, w3s, p);
 }
 
 static bool token_maps(TokenMaps& t, const void* ptr, long long rows, long long cols) {
@@ -782,7 +809,59 @@ moe_status run_ffn_down_swap(const FfnArgs& f, cudaStream_t s) {
   q.n_out = f.d;
   q.out = static_cast<__nv_bfloat16*>(f.Y);
   q.err = f.err;
-  if (launch_swap(m, q, swap_pairs(q, f.rows_routed), s) != cudaSuccess) return MOE_ERR_CUDA;
+  q.k_split = q.K;
+  q.w_k_rows = 0;
+  if (launch_swap<false>(m, m.w, m.ws, q, swap_pairs(q, f.rows_routed), s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+bool swap_dx_supported(const SwapDxArgs& a) {
+  return a.counts != nullptr && a.E <= MOE_MAX_EXPERTS && a.d % 256 == 0 && a.h % kSBK == 0 &&
+         a.kcols % kSBK == 0;
+}
+
+// dX_perm^T = W1^T dU^T (+ W3^T dV^T) per expert (and per shared expert), over
+// each expert's real tokens only; padding rows of dX_perm are not written
+moe_status run_bwd_dx_swap(const SwapDxArgs& a, cudaStream_t s) {
+  SwapMaps m;
+  if (!token_maps(m.t, a.duv, a.rows, a.kcols)) return MOE_ERR_UNSUPPORTED;
+  m.ts = m.t;  // shared rows are rows of dU (dV) too
+  CUtensorMap w3, w3s;
+  // MN-major weights: [experts * h, d] with 64 x 64 boxes
+  if (!make_bf16_sw128_map(&m.w, a.W1, (long long)a.E * a.h, a.d, 64)) return MOE_ERR_UNSUPPORTED;
+  w3 = m.w;
+  if (a.W3 && !make_bf16_sw128_map(&w3, a.W3, (long long)a.E * a.h, a.d, 64))
+    return MOE_ERR_UNSUPPORTED;
+  m.ws = m.w;
+  w3s = w3;
+  if (a.n_shared > 0) {
+    if (!make_bf16_sw128_map(&m.ws, a.sW1, (long long)a.n_shared * a.h, a.d, 64))
+      return MOE_ERR_UNSUPPORTED;
+    w3s = m.ws;
+    if (a.sW3 && !make_bf16_sw128_map(&w3s, a.sW3, (long long)a.n_shared * a.h, a.d, 64))
+      return MOE_ERR_UNSUPPORTED;
+  }
+  SwapParams q{};
+  q.offsets = a.offsets;
+  q.counts = a.counts;
+  q.E = a.E;
+  q.K = a.kcols;
+  q.m_per_expert = a.d;
+  q.mt_tiles = a.d / 256;
+  q.n_shared = a.n_shared;
+  q.n = a.n;
+  q.shared_in_row = a.shared_base;
+  q.shared_in_stride = a.n_pad;
+  q.shared_out_row = a.shared_base;
+  q.n_pad = a.n_pad;
+  q.n_out = a.d;
+  q.out = static_cast<__nv_bfloat16*>(a.dxp);
+  q.err = a.err;
+  q.k_split = a.W3 ? a.h : a.kcols;
+  q.w_k_rows = a.h;
+  if (launch_swap<true>(m, w3, w3s, q, swap_pairs(q, a.rows_routed), s) != cudaSuccess)
+    return MOE_ERR_CUDA;
   return MOE_OK;
 }
 

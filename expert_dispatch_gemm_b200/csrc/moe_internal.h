@@ -219,6 +219,21 @@ moe_status run_ffn_bf16(const FfnArgs& a, cudaStream_t s);
 bool swap_up_supported(const FfnArgs& a);
 moe_status run_ffn_up_swap(const FfnArgs& a, cudaStream_t s);
 bool swap_down_supported(const FfnArgs& a);
+// the backward's dX_perm = dU W1 (+ dV W3) with the weights as the M side
+struct SwapDxArgs {
+  const void* duv;          // [rows, kcols]: dU, then dV (SwiGLU) in columns h..2h
+  long long rows;           // rows of duv and dxp (routed, padding, shared)
+  long long rows_routed;
+  int kcols, E, h, d, n_shared, n;
+  long long shared_base, n_pad;
+  const void *W1, *W3, *sW1, *sW3;  // W3 / sW3 NULL without SwiGLU
+  const int32_t* offsets;
+  const int32_t* counts;
+  void* dxp;                // [rows, d]
+  int* err;
+};
+bool swap_dx_supported(const SwapDxArgs& a);
+moe_status run_bwd_dx_swap(const SwapDxArgs& a, cudaStream_t s);
 moe_status run_ffn_down_swap(const FfnArgs& a, cudaStream_t s);
 moe_status run_ffn_f32(const FfnArgs& a, cudaStream_t s);
 

@@ -272,6 +272,23 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory matrix descriptor for an MN-major operand tile of 64 x 64
+// boxes (64 MN-elements per 128-byte row, 64 K-rows) laid out by TMA with
+// 128-byte swizzling, the canonical MN-major layout: start address >> 4 in
+// [0,14), leading byte offset (8 KB between 64-element MN chunks) >> 4 in
+// [16,30), stride byte offset (1 KB between 8-row K groups) >> 4 in [32,46),
+// descriptor version 1 in [46,48), layout type 2 (128-byte swizzle) in
+// [61,64). One K16 step advances the start address by 16 rows of 128 bytes.
+constexpr uint32_t kMnChunkBytes = 64 * 64 * 2;
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)(kMnChunkBytes >> 4) << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
 // Instruction descriptor, kind::f16: fp32 accumulator (bits [4,6) = 1), A and
 // B bf16 (bits [7,10) = 1, [10,13) = 1), both K-major (bits 15, 16 = 0),
 // N >> 3 in [17,23), M >> 4 in [24,29).

@@ -44,6 +44,13 @@ BWD_SMALL = wl.SMALL + [
     # shared expert of fewer than 128 rows
     wl.TC_SIGMOID_GROUPED.replace(name="bwd-decode-n16-top8of64-shared1-d256-h128", n=16, d=256,
                                   E=64, h=128, bias_steps=0),
+    # about 256 rows per expert: dX with the weights as the M side (W1 read
+    # MN-major), with a shared expert; GELU (one weight matrix) and SwiGLU
+    # (W3 from K = h on, the forward's weights-as-M up projection too)
+    wl.TC_DROPLESS.replace(name="bwd-swap-top4of16-shared1-gelu-n1024-d256-h256", n=1024, d=256,
+                           E=16, K=4, h=256, act="gelu", n_shared=1),
+    wl.TC_SIGMOID_GROUPED.replace(name="bwd-swap-grouped-top8of32-shared1-n1024-d256-h256",
+                                  n=1024, d=256, E=32, h=256, bias_steps=0),
 ]
 
 
