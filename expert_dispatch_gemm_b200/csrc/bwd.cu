@@ -260,7 +260,8 @@ __global__ void __launch_bounds__(256) transpose_wg_kernel(const float* Wg, int 
 // of dX_perm[row, i] (+ the shared experts' rows), fp32, stored bf16.
 // Tile: 64 tokens x 128 columns, experts in chunks of 32; thread (ty, tx)
 // holds tokens 8ty..8ty+7 and columns 4tx..4tx+3, so each expert step takes
-// three 16-byte shared-memory loads for 32 FMAs.
+// three 16-byte shared-memory loads for 32 FMAs, issued as 16 packed fp32x2
+// FMAs (__ffma2_rn: each element rounds once, as fmaf would).
 constexpr int kRxBM = 64, kRxBN = 128, kRxEC = 32;
 template <typename T>
 __global__ void __launch_bounds__(256) router_dx_kernel(RouterBwdArgs a) {
@@ -269,11 +270,11 @@ __global__ void __launch_bounds__(256) router_dx_kernel(RouterBwdArgs a) {
   __shared__ __align__(16) float wts[kRxEC][kRxBN];      // [expert][column]
   const int tid = threadIdx.x, tx = tid & 31, ty = tid >> 5;
   const int t0 = blockIdx.x * kRxBM, i0 = blockIdx.y * kRxBN;
-  float acc[8][4];
+  float2 acc[8][2];
 #pragma unroll
   for (int k = 0; k < 8; ++k)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) acc[k][c] = 0.0f;
+    for (int c = 0; c < 2; ++c) acc[k][c] = make_float2(0.0f, 0.0f);
   for (int e0 = 0; e0 < a.E; e0 += kRxEC) {
     __syncthreads();
     for (int q = tid; q < kRxBM * kRxEC; q += 256) {
@@ -293,12 +294,12 @@ __global__ void __launch_bounds__(256) router_dx_kernel(RouterBwdArgs a) {
       const float4 g0 = *reinterpret_cast<const float4*>(&dls[c][8 * ty]);
       const float4 g1 = *reinterpret_cast<const float4*>(&dls[c][8 * ty + 4]);
       const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+      const float2 w01 = make_float2(w.x, w.y), w23 = make_float2(w.z, w.w);
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        acc[k][0] = fmaf(g[k], w.x, acc[k][0]);
-        acc[k][1] = fmaf(g[k], w.y, acc[k][1]);
-        acc[k][2] = fmaf(g[k], w.z, acc[k][2]);
-        acc[k][3] = fmaf(g[k], w.w, acc[k][3]);
+        const float2 gg = make_float2(g[k], g[k]);
+        acc[k][0] = __ffma2_rn(gg, w01, acc[k][0]);
+        acc[k][1] = __ffma2_rn(gg, w23, acc[k][1]);
       }
     }
   }
@@ -308,7 +309,7 @@ __global__ void __launch_bounds__(256) router_dx_kernel(RouterBwdArgs a) {
   for (int k = 0; k < 8; ++k) {
     const int t = t0 + 8 * ty + k;
     if (t >= a.n) continue;
-    float v[4] = {acc[k][0], acc[k][1], acc[k][2], acc[k][3]};
+    float v[4] = {acc[k][0].x, acc[k][0].y, acc[k][1].x, acc[k][1].y};
     const T* xp = static_cast<const T*>(a.dX_perm);
     auto add = [&](const float* x) {
       v[0] += x[0];
@@ -350,8 +351,9 @@ __global__ void __launch_bounds__(256) router_dx_kernel(RouterBwdArgs a) {
 
 // dWg[i, e] = sum_t X[t, i] dL[t, e]. Tile 128 (i) x 64 (e), tokens in
 // chunks of 32; thread (ti, te) holds rows 8ti..8ti+7 and experts
-// 4te..4te+3. blockIdx.z = a contiguous slice of the tokens; slices are
-// added in slice order by router_dwg_reduce_kernel.
+// 4te..4te+3 (packed fp32x2 FMAs over expert pairs). blockIdx.z = a
+// contiguous slice of the tokens; slices are added in slice order by
+// router_dwg_reduce_kernel.
 constexpr int kRwBM = 128, kRwBN = 64, kRwBT = 32;
 template <typename T>
 __global__ void __launch_bounds__(256) router_dwg_kernel(RouterBwdArgs a, int per_split) {
@@ -361,11 +363,11 @@ __global__ void __launch_bounds__(256) router_dwg_kernel(RouterBwdArgs a, int pe
   const int tid = threadIdx.x, te = tid & 15, ti = tid >> 4;
   const int i0 = blockIdx.x * kRwBM, e0 = blockIdx.y * kRwBN;
   const int tb = blockIdx.z * per_split, tend = min(a.n, tb + per_split);
-  float acc[8][4];
+  float2 acc[8][2];
 #pragma unroll
   for (int r = 0; r < 8; ++r)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) acc[r][c] = 0.0f;
+    for (int c = 0; c < 2; ++c) acc[r][c] = make_float2(0.0f, 0.0f);
   for (int c0 = tb; c0 < tend; c0 += kRwBT) {
     __syncthreads();
     // X chunk: 32 tokens x 128 columns as pairs of bf16
@@ -389,11 +391,13 @@ __global__ void __launch_bounds__(256) router_dwg_kernel(RouterBwdArgs a, int pe
       const float4 x1 = *reinterpret_cast<const float4*>(&xs[r][8 * ti + 4]);
       const float4 l = *reinterpret_cast<const float4*>(&ls[r][4 * te]);
       const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-      const float lv[4] = {l.x, l.y, l.z, l.w};
+      const float2 l01 = make_float2(l.x, l.y), l23 = make_float2(l.z, l.w);
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc[u][c] = fmaf(xv[u], lv[c], acc[u][c]);
+      for (int u = 0; u < 8; ++u) {
+        const float2 xx = make_float2(xv[u], xv[u]);
+        acc[u][0] = __ffma2_rn(xx, l01, acc[u][0]);
+        acc[u][1] = __ffma2_rn(xx, l23, acc[u][1]);
+      }
     }
   }
   float* dst = a.splits > 1 ? a.partial + (size_t)blockIdx.z * a.d * a.E : a.dWg;
@@ -404,7 +408,7 @@ __global__ void __launch_bounds__(256) router_dwg_kernel(RouterBwdArgs a, int pe
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       const int e = e0 + 4 * te + c;
-      if (e < a.E) dst[(size_t)i * a.E + e] = acc[u][c];
+      if (e < a.E) dst[(size_t)i * a.E + e] = c & 1 ? acc[u][c >> 1].y : acc[u][c >> 1].x;
     }
   }
 }
