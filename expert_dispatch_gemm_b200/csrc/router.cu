@@ -58,9 +58,12 @@ using R256s = RCfg<256, 2, 8, 4, 2, 4, 1, 32, 3>;
 // CTA), "C" over 2 (many rows per CTA).
 template <int TM> using R64A = RCfg<64, TM, 8, 4, 1, 1, 8, 64, 4>;   // BM = 4 TM
 template <int TM> using R64C = RCfg<64, TM, 8, 4, 4, 1, 2, 32, 4>;   // BM = 16 TM
-// R64A's tiles on 12 warps (a twelve-way k split of 48-deep chunks): in a
-// single wave of one CTA per SM, 50% more warps to hide the chunks' loads
-template <int TM> using R64D = RCfg<64, TM, 8, 4, 1, 1, 12, 48, 4>;  // BM = 4 TM
+// R64A's tiles on 12 warps (a twelve-way k split of 96-deep chunks): in a
+// single wave of one CTA per SM, 50% more warps to hide the chunks' loads.
+// 96-deep chunks (eight steps per warp between barriers) measured 46.0 us
+// for the expert-choice route stage at n 4096, d 1024 against 48.1 with 48
+// (longer chunks or deeper rings gave no more)
+template <int TM> using R64D = RCfg<64, TM, 8, 4, 1, 1, 12, 96, 4>;  // BM = 4 TM
 template <int TM> using R128A = RCfg<128, TM, 8, 4, 2, 2, 2, 32, 4>; // BM = 8 TM
 template <int TM> using R256A = RCfg<256, TM, 8, 4, 1, 4, 2, 32, 3>; // BM = 4 TM
 // E = 256 with 16 columns per thread: per 16-deep step a warp issues TM*16
@@ -158,7 +161,7 @@ static void variant_tile(int v, int* bm, int* bk) {
     default: {
       const int code = v - kFamilyCode, fam = code / 16, tm = code % 16;
       *bm = (fam == 2 ? 16 : fam == 3 || fam == 5 || fam == 6 ? 8 : 4) * tm;
-      *bk = fam == 1 ? 64 : fam == 6 || fam == 7 ? 48 : 32;
+      *bk = fam == 1 ? 64 : fam == 7 ? 96 : fam == 6 ? 48 : 32;
     }
   }
 }
