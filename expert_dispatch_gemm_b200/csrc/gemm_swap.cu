@@ -1,40 +1,43 @@
-// Down projection of the grouped expert FFN for fine-grained experts, with
-// the weights as the M side.
+// Grouped expert GEMMs for fine-grained experts with the weights as the M
+// side: the SwiGLU up projection, the down projection, and the backward's
+// dX_perm.
 //
 // "Expert choice routing" (aicassindra.com), "The math: a gating matrix and
-// top-k over tokens": each expert's gathered rows form a dense batch; here the
-// product Y_e = H_e W2_e^T is taken transposed, Y_e^T = W2_e H_e^T, so that an
+// top-k over tokens": each expert's gathered rows form a dense batch; here
+// each product is taken transposed (Y_e^T = W2_e H_e^T, H_e^T = silu(W1_e
+// X_e^T) * (W3_e X_e^T), dX_e^T = W1_e^T dU_e^T + W3_e^T dV_e^T), so that an
 // expert's tokens are the N side of the MMA and need only 16-row granularity,
-// where the 128-row M tiles of the other kernels round an expert of ~256 rows
-// up to 384 or 512.
+// where the 128-row M tiles of the token-side kernels round an expert of ~256
+// rows up to 384 or 512.
 //
-// CTA pairs (cta_group::2). A tile is (expert, 256 rows of W2, up to 256 of
+// CTA pairs (cta_group::2). A tile is (expert, 256 weight rows, up to 256 of
 // the expert's tokens): each CTA loads its 128 weight rows as A and half of
-// the tile's tokens as B, and the MMA is M=256 with N = tokens (a multiple
-// of 16).
+// the tile's tokens as B (exactly its N/2 rows), and the MMA is M=256 with
+// N = tokens (a multiple of 16).
 //
 // On B200 one thread issues at most one tcgen05.mma about every 95 cycles,
 // whatever N is, while an M=256 pair MMA needs N/2 cycles of the tensor
 // pipe: below N = 192 a single issuer leaves the pipe idle, and the token
 // chunks of experts with more than 256 rows are 128-160 wide. Two issuers
-// on independent accumulators keep it busy down to N = 128. So the pair runs
-// two tile streams, each with its own producer, shared-memory ring and
-// 256-column TMEM accumulator; stream s takes every other tile of the pair.
-//   warps 0 / 2   TMA producers of streams 0 / 1 (3-stage rings of 32 KB:
-//                 A 16 KB + B up to 16 KB);
-//   warps 1 / 3   the leader's lane 0 issues the MMAs of stream 0 / 1
-//                 (warp 1 also holds the TMEM allocation);
-//   warps 4-11    epilogue, four per stream (one per TMEM lane quadrant):
-//                 tcgen05.ld 32 tokens at a time, a transpose through shared
-//                 memory, and 16-byte stores of each token's 32 consecutive
-//                 output columns.
-// While one stream's epilogue drains its accumulator the other stream keeps
-// the tensor pipe busy.
+// on independent accumulators keep it busy down to N = 128. So:
+// - tc_swap_pair_kernel (down projection; backward dX with the weights read
+//   MN-major) runs two tile streams, each with its own producer,
+//   shared-memory ring and 256-column TMEM accumulator; stream s takes every
+//   other tile of the pair.
+//     warps 0 / 2   TMA producers of streams 0 / 1 (3-stage rings of 32 KB:
+//                   A 16 KB + B up to 16 KB);
+//     warps 1 / 3   the leader's lane 0 issues the MMAs of stream 0 / 1
+//                   (warp 1 also holds the TMEM allocation);
+//     warps 4-11    epilogue, four per stream (one per TMEM lane quadrant):
+//                   tcgen05.ld 32 tokens at a time, a transpose through
+//                   shared memory, and 16-byte stores of each token's 32
+//                   consecutive output columns.
+//   While one stream's epilogue drains its accumulator the other stream
+//   keeps the tensor pipe busy.
+// - tc_swap_up_pair_kernel (SwiGLU up projection) loads W1 and W3 rows as
+//   two A operands of one stage and issues their MMAs from two threads into
+//   two accumulators (U, V), which meet in one epilogue thread.
 // Every mbarrier wait is bounded, as in the other GEMM kernels.
-//
-// Only the down projection runs here. The same scheme for the SwiGLU up
-// projection (64 W1 and 64 W3 rows per CTA, gate and up values meeting
-// through shared memory) was slower on B200 than the token-side CTA pairs.
 #include <cuda.h>
 #include <math.h>
 
