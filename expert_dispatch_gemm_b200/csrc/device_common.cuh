@@ -85,39 +85,6 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
-// Strict total order used by every top-k: larger key first, then lower
-// index. IEEE comparison, so -0 == +0. `valid` marks a real candidate.
-struct Cand {
-  float key;
-  int idx;
-  bool valid;
-};
-
-__device__ __forceinline__ bool cand_better(const Cand& a, const Cand& b) {
-  if (!a.valid) return false;
-  if (!b.valid) return true;
-  if (a.key > b.key) return true;
-  if (a.key < b.key) return false;
-  return a.idx < b.idx;
-}
-
-__device__ __forceinline__ Cand shfl_xor_cand(const Cand& c, int m) {
-  Cand o;
-  o.key = __shfl_xor_sync(0xffffffffu, c.key, m);
-  o.idx = __shfl_xor_sync(0xffffffffu, c.idx, m);
-  o.valid = __shfl_xor_sync(0xffffffffu, (int)c.valid, m) != 0;
-  return o;
-}
-
-// Reduce over aligned groups of `width` lanes (power of two).
-__device__ __forceinline__ Cand group_best(Cand c, int width) {
-  for (int m = 1; m < width; m <<= 1) {
-    Cand o = shfl_xor_cand(c, m);
-    if (cand_better(o, c)) c = o;
-  }
-  return c;
-}
-
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) {
   return __uint_as_float(((uint32_t)b) << 16);
 }

@@ -215,71 +215,103 @@ __device__ __forceinline__ void cp_async_wait() {
 // Order: key desc, expert asc. Group score: fp32 sum of the group_topn
 // largest keys, largest first; groups ranked by (score desc, group asc).
 // Weights always come from the raw scores.
+//
+// Each key becomes a 32-bit code that orders like the IEEE comparison
+// (-0 folded into +0; code 0 means "no candidate"), so one round of a
+// top-k is a lane-local max, one warp max-reduction (redux.sync) and a
+// ballot: the winner is the lowest lane holding the maximum code, and
+// within it the lowest slot, i.e. the lowest expert index among equal keys.
+// NaN keys are outside the contract.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t select_code(float k) {
+  const uint32_t u = __float_as_uint(k + 0.0f);  // -0 + 0 = +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float select_key(uint32_t c) {
+  return __uint_as_float((c & 0x80000000u) ? (c & 0x7fffffffu) : ~c);
+}
+template <int V>
+__device__ __forceinline__ uint32_t lane_max_code(const uint32_t (&c)[V]) {
+  uint32_t m[V];
+#pragma unroll
+  for (int v = 0; v < V; ++v) m[v] = c[v];
+#pragma unroll
+  for (int w = 1; w < V; w <<= 1)
+#pragma unroll
+    for (int v = 0; v + w < V; v += 2 * w) m[v] = max(m[v], m[v + w]);
+  return m[0];
+}
+// Clears the lowest slot holding code M (the caller knows there is one) and
+// returns that slot.
+template <int V>
+__device__ __forceinline__ int take_code(uint32_t (&c)[V], uint32_t M) {
+  int pos = 0;
+#pragma unroll
+  for (int v = V - 1; v >= 0; --v)
+    if (c[v] == M) pos = v;
+#pragma unroll
+  for (int v = 0; v < V; ++v)
+    if (v == pos) c[v] = 0u;
+  return pos;
+}
+
 template <int V>
 __device__ __forceinline__ void tc_select_row(const float (&key)[V], const float (&raw)[V],
                                               const bool (&ok)[V], int lane, int E, int K,
                                               int n_groups, int topk_groups, int group_topn,
                                               int weights, int32_t* idx_out,
                                               float* gate_out) {
-  bool allowed[V];
+  uint32_t code[V];
 #pragma unroll
-  for (int v = 0; v < V; ++v) allowed[v] = ok[v];
+  for (int v = 0; v < V; ++v) code[v] = ok[v] ? select_code(key[v]) : 0u;
   if (n_groups > 1) {
     const int gs = E / n_groups;
-    const int lpg = gs / V;
-    const int g = (lane * V) / gs;
-    bool taken[V];
+    const int lpg = gs / V;             // lanes per group, a power of two <= 16
+    const int g = lane / lpg;           // this lane's group
+    const unsigned gmask = lpg >= 32 ? 0xffffffffu : ((1u << lpg) - 1u) << (g * lpg);
+    uint32_t gc[V];
 #pragma unroll
-    for (int v = 0; v < V; ++v) taken[v] = false;
+    for (int v = 0; v < V; ++v) gc[v] = code[v];
     float gsum = 0.0f;
     for (int r = 0; r < group_topn; ++r) {
-      Cand c{0.0f, 0, false};
-#pragma unroll
-      for (int v = 0; v < V; ++v) {
-        Cand x{key[v], lane * V + v, allowed[v] && !taken[v]};
-        if (cand_better(x, c)) c = x;
-      }
-      c = group_best(c, lpg);
-      if (c.valid) gsum = gsum + c.key;
-#pragma unroll
-      for (int v = 0; v < V; ++v)
-        if (c.valid && c.idx == lane * V + v) taken[v] = true;
+      const uint32_t best = lane_max_code<V>(gc);
+      uint32_t M = best;
+      for (int m = 1; m < lpg; m <<= 1) M = max(M, __shfl_xor_sync(0xffffffffu, M, m));
+      const unsigned hold = __ballot_sync(0xffffffffu, M != 0u && best == M) & gmask;
+      if (M == 0u) continue;            // the group has no candidate left
+      gsum = gsum + select_key(M);
+      if (lane == __ffs(hold) - 1) take_code<V>(gc, M);
     }
-    bool gsel = false;
-    const bool gvalid = g < n_groups;
-    for (int r = 0; r < topk_groups; ++r) {
-      Cand c{gsum, g, gvalid && !gsel};
-      c = group_best(c, 32);
-      if (c.valid && c.idx == g) gsel = true;
+    // rank of this lane's group: groups ahead of it by (score desc, group asc)
+    int rank = 0;
+    for (int h = 0; h < n_groups; ++h) {
+      const float o = __shfl_sync(0xffffffffu, gsum, h * lpg);
+      rank += (o > gsum || (o == gsum && h < g)) ? 1 : 0;
     }
+    const bool gsel = g < n_groups && rank < topk_groups;
 #pragma unroll
-    for (int v = 0; v < V; ++v) allowed[v] = allowed[v] && gsel;
+    for (int v = 0; v < V; ++v) code[v] = gsel ? code[v] : 0u;
   }
-  bool picked[V];
-#pragma unroll
-  for (int v = 0; v < V; ++v) picked[v] = false;
   int my_e = -1;
   float my_raw = 0.0f;
   for (int j = 0; j < K; ++j) {
-    Cand c{0.0f, 0, false};
-#pragma unroll
-    for (int v = 0; v < V; ++v) {
-      Cand x{key[v], lane * V + v, allowed[v] && !picked[v]};
-      if (cand_better(x, c)) c = x;
-    }
-    c = group_best(c, 32);
+    const uint32_t best = lane_max_code<V>(code);
+    const uint32_t M = __reduce_max_sync(0xffffffffu, best);
+    const unsigned hold = __ballot_sync(0xffffffffu, M != 0u && best == M);
+    const int win = hold ? __ffs(hold) - 1 : 0;
+    int e = -1;
     float rv = 0.0f;
+    if (hold && lane == win) {
+      const int pos = take_code<V>(code, M);
+      e = lane * V + pos;
 #pragma unroll
-    for (int v = 0; v < V; ++v)
-      if (c.valid && c.idx == lane * V + v) {
-        picked[v] = true;
-        rv = raw[v];
-      }
-    const int owner = c.valid ? c.idx / V : 0;
-    rv = __shfl_sync(0xffffffffu, rv, owner);
+      for (int v = 0; v < V; ++v)
+        if (v == pos) rv = raw[v];
+    }
+    e = __shfl_sync(0xffffffffu, e, win);
+    rv = __shfl_sync(0xffffffffu, rv, win);
     if (lane == j) {
-      my_e = c.valid ? c.idx : -1;
+      my_e = e;
       my_raw = rv;
     }
   }
