@@ -36,7 +36,7 @@ struct RCfg {
   static_assert(NW == 8 || NW == 12, "8 or 12 warps");
   static_assert(TN == 4 || TN == 8 || TN == 16, "TN");
   static_assert(TM >= 1 && TM <= 8, "TM");
-  static_assert(BK % WK == 0 && ST >= 2, "pipeline");
+  static_assert(BK % WK == 0 && ST >= 3, "pipeline");
 };
 // 4 x 8 (E = 64, 128) or 8 x 8 (E = 256) register tiles: the larger the tile
 // the fewer shared-memory fragment loads per FMA. The "s" variants trade rows
@@ -435,7 +435,7 @@ struct RouterSmem {
   static constexpr size_t xs_bytes = (size_t)C::ST * C::BM * C::BK * XB;
   static constexpr size_t ws_bytes = (size_t)C::ST * C::BK * C::ET * 4;
   static constexpr size_t as_bytes = (size_t)C::BK * AST * XB;
-  static constexpr size_t main_bytes = xs_bytes + ws_bytes + as_bytes;
+  static constexpr size_t main_bytes = xs_bytes + ws_bytes + 2 * as_bytes;  // two A tiles
   static constexpr size_t epi_bytes =
       ((size_t)C::WK * C::BM * (C::ET + 1) + C::NW * C::ET) * 4 + C::NW * 8;
   static constexpr size_t bytes = (main_bytes > epi_bytes ? main_bytes : epi_bytes) + 128;
@@ -450,8 +450,8 @@ __global__ void __launch_bounds__(C::NT) router_kernel(RouterArgs a) {
   extern __shared__ __align__(16) unsigned char rsm[];
   unsigned char* Xs = rsm;                                        // [S][BM][BK] raw
   float* Ws = reinterpret_cast<float*>(rsm + SM::xs_bytes);       // [S][BK][ET]
-  float* As = reinterpret_cast<float*>(rsm + SM::xs_bytes + SM::ws_bytes);  // [BK][AST] fp32
-  uint16_t* As16 = reinterpret_cast<uint16_t*>(As);                         // [BK][AST] bf16
+  float* As = reinterpret_cast<float*>(rsm + SM::xs_bytes + SM::ws_bytes);  // [2][BK][AST] fp32
+  uint16_t* As16 = reinterpret_cast<uint16_t*>(As);                         // [2][BK][AST] bf16
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int lx = lane / C::LY, ly = lane % C::LY;
@@ -474,38 +474,74 @@ __global__ void __launch_bounds__(C::NT) router_kernel(RouterArgs a) {
 #pragma unroll
     for (int j = 0; j < TN / 2; ++j) acc[i][j] = make_float2(0.0f, 0.0f);
 
-  // stage loader: X chunk [BM][BK] and W_g chunk [BK][ET] of chunk `c`
-  auto issue = [&](int c) {
+  // Chunk c's loads, as parts that can be spread over the previous chunk's
+  // FMA steps: part i < XIT copies 16-byte piece tid + i*NT of the X chunk
+  // [BM][BK], the rest pieces of the W_g chunk [BK][ET] (4-float pieces when
+  // E % 4 == 0, else single floats, all in part XIT).
+  constexpr int XCH = BM * BK * XB / 16;          // 16-byte pieces of the X chunk
+  constexpr int XPR = BK * XB / 16;               // pieces per row
+  constexpr int XIT = (XCH + C::NT - 1) / C::NT;
+  constexpr int WCH = BK * ET / 4;
+  constexpr int WIT = (WCH + C::NT - 1) / C::NT;
+  auto issue_part = [&](int c, int i) {
     const int st = c % C::ST;
     const int k0 = c * BK;
-    constexpr int XCH = BM * BK * XB / 16;          // 16-byte pieces of the X chunk
-    constexpr int XPR = BK * XB / 16;               // pieces per row
-    unsigned char* xs = Xs + (size_t)st * BM * BK * XB;
-    for (int q = tid; q < XCH; q += C::NT) {
-      const int r = q / XPR, p = q % XPR;
-      const int row = m0 + r, k = k0 + p * (16 / XB);
-      const bool ok = row < n && k < d;
-      const char* src = static_cast<const char*>(a.X) +
-                        ((size_t)(ok ? row : 0) * d + (ok ? k : 0)) * XB;
-      cp_async16(xs + (size_t)r * BK * XB + p * 16, src, ok);
+    if (i < XIT) {
+      const int q = tid + i * C::NT;
+      if (XCH % C::NT == 0 || q < XCH) {
+        unsigned char* xs = Xs + (size_t)st * BM * BK * XB;
+        const int r = q / XPR, p = q % XPR;
+        const int row = m0 + r, k = k0 + p * (16 / XB);
+        const bool ok = row < n && k < d;
+        const char* src = static_cast<const char*>(a.X) +
+                          ((size_t)(ok ? row : 0) * d + (ok ? k : 0)) * XB;
+        cp_async16(xs + (size_t)r * BK * XB + p * 16, src, ok);
+      }
+      return;
     }
     float* ws = Ws + (size_t)st * BK * ET;
     if (w_vec) {
-      constexpr int WCH = BK * ET / 4;
-      for (int q = tid; q < WCH; q += C::NT) {
+      const int q = tid + (i - XIT) * C::NT;
+      if (WCH % C::NT == 0 || q < WCH) {
         const int kk = q / (ET / 4), c4 = (q % (ET / 4)) * 4;
         const int k = k0 + kk;
         const bool ok = k < d && c4 < E;
         cp_async16(ws + kk * ET + c4, a.Wg + (ok ? (size_t)k * E + c4 : 0), ok);
       }
-    } else {
-      constexpr int WCH = BK * ET;
-      for (int q = tid; q < WCH; q += C::NT) {
+    } else if (i == XIT) {
+      for (int q = tid; q < BK * ET; q += C::NT) {
         const int kk = q / ET, cc = q % ET;
         const int k = k0 + kk;
         const bool ok = k < d && cc < E;
         cp_async4(ws + kk * ET + cc, a.Wg + (ok ? (size_t)k * E + cc : 0), ok);
       }
+    }
+  };
+  // Part i of chunk c's transposition into its A tile (As buffer c % 2):
+  // 16-byte piece tid + i*NT of the X chunk, written column-wise, As[kk][r]
+  // (bf16 X stays bf16; fp32 X stays fp32).
+  constexpr int EPP = 16 / XB;                     // elements per 16-byte piece
+  constexpr int PCS = BM * BK / EPP;
+  constexpr int TIT = (PCS + C::NT - 1) / C::NT;
+  auto transpose_part = [&](int c, int i) {
+    const int q = tid + i * C::NT;
+    if (PCS % C::NT != 0 && q >= PCS) return;
+    const unsigned char* xs = Xs + (size_t)(c % C::ST) * BM * BK * XB;
+    const int r = q % BM, p = q / BM;
+    const uint4 v = *reinterpret_cast<const uint4*>(xs + (size_t)r * BK * XB + p * 16);
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+    if (XBF16) {
+      uint16_t* as16 = As16 + (size_t)(c & 1) * BK * AST;
+      const int rr = r / TM * TMP + r % TM;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        as16[(p * 8 + 2 * j) * AST + rr] = (uint16_t)(w4[j] & 0xffffu);
+        as16[(p * 8 + 2 * j + 1) * AST + rr] = (uint16_t)(w4[j] >> 16);
+      }
+    } else {
+      float* as = As + (size_t)(c & 1) * BK * AST;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) as[(p * 4 + j) * AST + r] = __uint_as_float(w4[j]);
     }
   };
 
@@ -515,46 +551,45 @@ __global__ void __launch_bounds__(C::NT) router_kernel(RouterArgs a) {
   const int ce = min(nchunks, cb + a.chunks_per_split);
 #pragma unroll 1
   for (int c = cb; c < cb + C::ST - 1; ++c) {
-    if (c < ce) issue(c);
+    if (c < ce)
+      for (int i = 0; i < XIT + WIT; ++i) issue_part(c, i);
     cp_async_commit();
   }
+  cp_async_wait<C::ST - 2>();
+  __syncthreads();
+  if (cb < ce)
+    for (int i = 0; i < TIT; ++i) transpose_part(cb, i);
+  // One barrier per chunk. At the top of chunk c: chunk c + 1 has landed,
+  // chunk c's A tile is written, and every warp is done with chunk c - 1, so
+  // its ring stage and A buffer are free. During chunk c's FMA steps each
+  // thread transposes its pieces of chunk c + 1 and issues its copies of
+  // chunk c + ST - 1 (into chunk c - 1's stage), a few per step, so that no
+  // phase of the loop leaves the FMA pipe to itself.
+  constexpr int QS = BK / C::WK;                  // FMA steps per warp per chunk
+  constexpr int NPART = TIT + XIT + WIT;
 #pragma unroll 1
   for (int c = cb; c < ce; ++c) {
-    cp_async_wait<C::ST - 2>();
+    cp_async_wait<C::ST - 3>();
     __syncthreads();
-    {  // convert the X chunk to fp32, transposed: As[kk][r]
-      const int st = c % C::ST;
-      const unsigned char* xs = Xs + (size_t)st * BM * BK * XB;
-      constexpr int EPP = 16 / XB;                 // elements per 16-byte piece
-      constexpr int PCS = BM * BK / EPP;
-      for (int q = tid; q < PCS; q += C::NT) {
-        const int r = q % BM, p = q / BM;
-        const uint4 v = *reinterpret_cast<const uint4*>(xs + (size_t)r * BK * XB + p * 16);
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-        if (XBF16) {
-          const int rr = r / TM * TMP + r % TM;
+    const bool do_t = c + 1 < ce, do_i = c + C::ST - 1 < ce;
+    const float* ws = Ws + (size_t)(c % C::ST) * BK * ET;
+    const uint16_t* as16 = As16 + (size_t)(c & 1) * BK * AST;
+    const float* as = As + (size_t)(c & 1) * BK * AST;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            As16[(p * 8 + 2 * j) * AST + rr] = (uint16_t)(w4[j] & 0xffffu);
-            As16[(p * 8 + 2 * j + 1) * AST + rr] = (uint16_t)(w4[j] >> 16);
-          }
-        } else {
+    for (int q = 0; q < QS; ++q) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j) As[(p * 4 + j) * AST + r] = __uint_as_float(w4[j]);
+      for (int i = (q * NPART + QS - 1) / QS; i < ((q + 1) * NPART + QS - 1) / QS; ++i) {
+        if (i < TIT) {
+          if (do_t) transpose_part(c + 1, i);
+        } else if (do_i) {
+          issue_part(c + C::ST - 1, i - TIT);
         }
       }
-    }
-    __syncthreads();
-    if (c + C::ST - 1 < ce) issue(c + C::ST - 1);
-    cp_async_commit();
-    const float* ws = Ws + (size_t)(c % C::ST) * BK * ET;
-#pragma unroll
-    for (int q = 0; q < BK / C::WK; ++q) {
-      const int kk = wk * (BK / C::WK) + q;
+      const int kk = wk * QS + q;
       float av[TM], bv[TN];
       if constexpr (XBF16) {
         // the thread's TMP bf16 values: one 16- or 8-byte load, else 4-byte loads
-        const uint16_t* ap = As16 + kk * AST + arow0;
+        const uint16_t* ap = as16 + kk * AST + arow0;
         uint32_t w[TMP / 2];
         if constexpr (TMP == 8) {
           const uint4 t = *reinterpret_cast<const uint4*>(ap);
@@ -576,7 +611,7 @@ __global__ void __launch_bounds__(C::NT) router_kernel(RouterArgs a) {
       } else if (TM % 4 == 0) {
 #pragma unroll
         for (int i4 = 0; i4 < TM / 4; ++i4) {
-          const float4 t = *reinterpret_cast<const float4*>(As + kk * AST + row0 + 4 * i4);
+          const float4 t = *reinterpret_cast<const float4*>(as + kk * AST + row0 + 4 * i4);
           av[(4 * i4 + 0) % TM] = t.x;
           av[(4 * i4 + 1) % TM] = t.y;
           av[(4 * i4 + 2) % TM] = t.z;
@@ -585,13 +620,13 @@ __global__ void __launch_bounds__(C::NT) router_kernel(RouterArgs a) {
       } else if (TM % 2 == 0) {
 #pragma unroll
         for (int i2 = 0; i2 < TM / 2; ++i2) {
-          const float2 t = *reinterpret_cast<const float2*>(As + kk * AST + row0 + 2 * i2);
+          const float2 t = *reinterpret_cast<const float2*>(as + kk * AST + row0 + 2 * i2);
           av[(2 * i2) % TM] = t.x;
           av[(2 * i2 + 1) % TM] = t.y;
         }
       } else {
 #pragma unroll
-        for (int i = 0; i < TM; ++i) av[i] = As[kk * AST + row0 + i];
+        for (int i = 0; i < TM; ++i) av[i] = as[kk * AST + row0 + i];
       }
 #pragma unroll
       for (int g = 0; g < TN / 4; ++g) {
@@ -609,6 +644,7 @@ __global__ void __launch_bounds__(C::NT) router_kernel(RouterArgs a) {
           acc[i][j] = __ffma2_rn(a2, make_float2(bv[2 * j], bv[2 * j + 1]), acc[i][j]);
       }
     }
+    cp_async_commit();
   }
   cp_async_wait<0>();
   __syncthreads();
