@@ -56,9 +56,11 @@ using R256s = RCfg<256, 2, 8, 4, 2, 4, 1, 32, 3>;
 // splits into about one CTA's worth of rows per SM (the contraction is bound
 // by the FFMA pipe, so an SM holding two CTAs' rows while another holds one
 // sets the time). "A" splits each chunk's k range over 8 warps (few rows per
-// CTA), "C" over 2 (many rows per CTA).
+// CTA), "C" over 3 warp groups of 4 (many rows per CTA): 12 warps, 48-deep
+// chunks, so that one CTA per SM of 112 rows hides its loads (n 16384, d 2048:
+// route stage 147.4 us, against 174.1 with 8 warps and two CTAs of 64 rows)
 template <int TM> using R64A = RCfg<64, TM, 8, 4, 1, 1, 8, 64, 4>;   // BM = 4 TM
-template <int TM> using R64C = RCfg<64, TM, 8, 4, 4, 1, 2, 32, 4>;   // BM = 16 TM
+template <int TM> using R64C = RCfg<64, TM, 8, 4, 4, 1, 3, 48, 3>;   // BM = 16 TM
 // R64A's tiles on 12 warps (a twelve-way k split of 96-deep chunks): in a
 // single wave of one CTA per SM, 50% more warps to hide the chunks' loads.
 // 96-deep chunks (eight steps per warp between barriers) measured 46.0 us
@@ -124,11 +126,8 @@ static int router_variant(int E, int n, bool x_bf16) {
         // measured on B200: R64A (eight-way k split, few rows) pays off only
         // in a single wave (c2: 28 rows per SM 26.9 us); with more CTAs than
         // SMs its per-CTA reduction costs more than R64C's (n = 16384: 195 us
-        // vs 174). R64C splits each chunk over only two warp groups, so with
-        // one CTA per SM its eight warps hide too little latency (112 rows
-        // per SM took 203 us, 128 rows in two CTAs 174 us).
+        // vs 174, when R64C had 8 warps).
         if ((fams[f].code == 1 || fams[f].code == 7) && ctas > sms) continue;
-        if (fams[f].code == 2 && ctas * 2 < 3LL * sms) cost = cost * 4 / 3;
         // TM x 8 tiles at E = 256 are bound by shared-memory wavefronts
         // (TM + 8 per TM*8 FFMAs per step), the 16-column tiles by the FMA
         // pipe: charge the narrower tile a quarter more per row
@@ -162,7 +161,7 @@ static void variant_tile(int v, int* bm, int* bk) {
     default: {
       const int code = v - kFamilyCode, fam = code / 16, tm = code % 16;
       *bm = (fam == 2 ? 16 : fam == 3 || fam == 5 || fam == 6 ? 8 : 4) * tm;
-      *bk = fam == 1 ? 64 : fam == 7 ? 96 : fam == 6 ? 48 : 32;
+      *bk = fam == 1 ? 64 : fam == 7 ? 96 : fam == 6 || fam == 2 ? 48 : 32;
     }
   }
 }
