@@ -14,12 +14,15 @@
 // tensor cores.
 //
 // Main loop: one CTA owns BM rows and all E columns (so the epilogue sees
-// whole rows). X and W_g chunks of BK along d stream through a 4-deep
-// cp.async ring; each X chunk is converted once to fp32 into a transposed
-// tile. Each thread holds TM x TN accumulators; a lane's TN columns are two
-// groups of 4 that sit 4*LY columns apart, so every 8-lane phase of a 128-bit
-// shared load reads one contiguous 128 bytes (no bank conflicts). WK > 1
-// splits each chunk's k range across warp groups, summed in a fixed order.
+// whole rows). X and W_g chunks of BK along d stream through a 3- or 4-deep
+// cp.async ring; each X chunk is transposed once into one of two A tiles
+// (bf16 X stays bf16 there and is widened per fragment). One barrier per
+// chunk: the next chunk's transposition and copies are spread over the
+// current chunk's FMA steps. Each thread holds TM x TN accumulators, updated
+// with packed fp32x2 FMAs; a lane's TN columns are groups of 4 that sit 4*LY
+// columns apart, so every 8-lane phase of a 128-bit shared load reads one
+// contiguous 128 bytes (no bank conflicts). WK > 1 splits each chunk's k
+// range across warp groups, summed in a fixed order.
 #include <math.h>
 
 #include "device_common.cuh"
